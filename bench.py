@@ -1,0 +1,475 @@
+#!/usr/bin/env python
+"""Benchmark of the selective-scan (S6) forward pass on B200.
+
+One step = one forward scan (ssm_scan_fwd through the C ABI) over one batch of the workload
+the metric is quoted on: the Mamba-370m-shaped layer, batch 8 x dim 2048 x L 2048, N 16, bf16
+io, f32 state.  Inputs are seeded synthetic tensors resident in HBM when timing starts
+(270 MB of compulsory traffic per step, more than the 126 MB L2, so no flush is needed
+between steps).  Prints ONE JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same workload on this
+machine's host cores (the reference arm; there is no upstream implementation to install).
+Multi-GPU (torchrun, one process per GPU): every rank scans its own batch (weak scaling; the
+path has no exchange step, so no collective touches the data); time is the max over ranks.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from selective_state_space_23_b200.inputs import make_inputs, workload  # noqa: E402
+
+METRIC = "selective-scan fwd tokens/s and achieved HBM GB/s (% of B200 peak) at 1 GPU"
+UNIT = "tokens/s"
+WORKLOAD = "mamba370m_fwd"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "source": "fallback"}
+
+# Unit counts of a B200 SM used for the ALU roofline (per clock): 128 FP32 FMA lanes, 16 MUFU
+# (ex2) lanes.  One (channel, step, state) element needs 4 FP32 ops (Δ*A, Δ*x*B, state FMA,
+# C readout) plus one 2^x, which costs 1 MUFU op or 7 FP32 ops on the FMA pipe (range
+# reduction 3 + polynomial 4).  With a fraction f of the exponentials on MUFU the two pipes
+# balance at (4 + 7(1-f))/128 = f/16, i.e. f = 11/15, giving 16*15/11 = 21.8 elements/clk/SM.
+FP32_PER_CLK, MUFU_PER_CLK, BASE_FP32, EXP_FP32 = 128, 16, 4, 7
+
+
+def alu_peak_elems_per_s(sms: int, mhz: float) -> float:
+    f = (BASE_FP32 + EXP_FP32) / (EXP_FP32 + FP32_PER_CLK / MUFU_PER_CLK)
+    per_clk = MUFU_PER_CLK / f
+    return sms * mhz * 1e6 * per_clk
+
+
+def compulsory_bytes(w) -> int:
+    es = 2 if w.io_dtype == torch.bfloat16 else 4
+    x = w.batch * w.dim * w.seqlen * es
+    bc = w.batch * w.dstate * w.seqlen * es
+    return 4 * x + 2 * bc + w.dim * w.dstate * 4 + 2 * w.dim * 4
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "sm_max_mhz": float(d.get("sm_max_mhz", 1965.0)),
+                "source": "measured"}
+    return dict(FALLBACK_PEAKS)
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("ssm_fwd.cu", "ssm_device.cuh", "ssm_kernels.h"):
+        with open(os.path.join(ROOT, "selective_state_space_23_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per launch of the forward kernel from the committed ncu summary, or None when
+    the kernel source changed since that capture."""
+    p = os.path.join(ROOT, "profiles", "fwd_kernel_mamba370m_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    kv = {}
+    with open(p) as fh:
+        for line in fh:
+            if "=" in line and not line.startswith("#"):
+                k, v = line.split("=", 1)
+                kv[k.strip()] = v.strip()
+    if kv.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    try:
+        return int(kv["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons, power = [], None, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        busy = [s for s in sm if mx and s > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power) if power else None}
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+def oracle_sample_time(w, seed: int, target_s: float = 3.0):
+    """Time the fp64 oracle (as it stands) on a channel sample of the workload; return
+    (tokens_per_s_extrapolated, cores, description).  The sample grows until it takes about
+    target_s seconds or covers the whole workload."""
+    import oracle
+    x = make_inputs(w, seed=seed)
+    f = {k: v.to(torch.float64).numpy() for k, v in x.items()}
+    cores = oracle.max_threads()
+    nd = min(w.dim, 64)
+    while True:
+        sel = np.arange(nd)
+        t0 = time.perf_counter()
+        oracle.scan_fwd(f["u"][:, sel], f["delta"][:, sel], f["A"][sel], f["B"], f["C"],
+                        D=f["D"][sel], z=f["z"][:, sel], dt_bias=f["dt_bias"][sel])
+        dt = time.perf_counter() - t0
+        if dt >= target_s or nd >= w.dim:
+            break
+        nd = min(w.dim, max(nd * 2, int(nd * target_s / max(dt, 1e-3))))
+    full_s = dt * w.dim / nd
+    desc = (f"oracle fp64 on {w.batch}x{nd} of {w.batch}x{w.dim} channels x L {w.seqlen} x N "
+            f"{w.dstate} ({dt:.2f} s), extrapolated by channel count")
+    return w.tokens / full_s, cores, desc, dt
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    w = workload(WORKLOAD)
+    # warm-up steps (untimed), then K timed steps; each step a bounded channel sample
+    import oracle
+    x = make_inputs(w, seed=0)
+    f = {k: v.to(torch.float64).numpy() for k, v in x.items()}
+    cores = oracle.max_threads()
+    nd = int(os.environ.get("SSM_REF_CHANNELS", "128"))
+    sel = np.arange(nd)
+    sub = dict(u=f["u"][:, sel], delta=f["delta"][:, sel], A=f["A"][sel], B=f["B"], C=f["C"],
+               D=f["D"][sel], z=f["z"][:, sel], dt_bias=f["dt_bias"][sel])
+    run = lambda: oracle.scan_fwd(sub["u"], sub["delta"], sub["A"], sub["B"], sub["C"], D=sub["D"],
+                                  z=sub["z"], dt_bias=sub["dt_bias"])
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    el = time.perf_counter() - t0
+    per_step_full = el / args.steps * w.dim / nd
+    value = w.tokens / per_step_full
+    sample = (f"each step: oracle fp64 on {w.batch}x{nd} of {w.batch}x{w.dim} channels "
+              f"(L {w.seqlen}, N {w.dstate}); throughput extrapolated by channel count")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step_full * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "config": {"workload": f"{WORKLOAD}: batch 8 x dim 2048 x L 2048, N 16, bf16 io rounded then f64",
+                   "global_batch": w.batch, "seq_len": w.seqlen, "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+def bench_extras(dev):
+    """Timing of the other hot-path calls on their workloads (inputs drawn on the GPU)."""
+    import selective_state_space_23_b200 as ssm
+    g = torch.Generator(device=dev).manual_seed(1)
+    out = {}
+
+    def rnd(shape, std=1.0):
+        return (torch.randn(shape, device=dev, generator=g) * std).to(torch.bfloat16)
+
+    def prm(dim, N, lo, hi):
+        dt = torch.exp(torch.rand(dim, device=dev, generator=g) * (np.log(hi) - np.log(lo)) + np.log(lo))
+        bias = dt + torch.log(-torch.expm1(-dt))
+        A = -torch.arange(1, N + 1, device=dev, dtype=torch.float32).repeat(dim, 1)
+        return A.contiguous(), torch.randn(dim, device=dev, generator=g), bias.float()
+
+    def timeit(fn, reps):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    # training step (forward with checkpoints + backward) on the Mamba-2.8B-shaped layer
+    b, d, L, N = 4, 5120, 2048, 16
+    u, de, z, dout = rnd((b, d, L)), rnd((b, d, L), 0.5), rnd((b, d, L)), rnd((b, d, L))
+    B, C = rnd((b, N, L)), rnd((b, N, L))
+    A, D, bias = prm(d, N, 1e-3, 1e-1)
+    ws = torch.empty(ssm.bwd_workspace_bytes(b, d, L, N, torch.bfloat16, True), dtype=torch.uint8, device=dev)
+
+    def train():
+        _, ck = ssm.ssm_scan_fwd(u, de, A, B, C, D=D, z=z, dt_bias=bias, return_ckpt=True)
+        ssm.ssm_scan_bwd(u, de, A, B, C, dout, D=D, z=z, dt_bias=bias, ckpt=ck, workspace=ws)
+
+    def fwd_only():
+        ssm.ssm_scan_fwd(u, de, A, B, C, D=D, z=z, dt_bias=bias)
+
+    ms_tr = timeit(train, 5)
+    ms_f = timeit(fwd_only, 10)
+    out["mamba2p8b_train"] = {"shape": "4x5120x2048 N16 bf16", "fwd_ms": ms_f,
+                              "fwd_bwd_ms": ms_tr, "tokens_per_s": b * L / (ms_tr * 1e-3)}
+    del u, de, z, dout, ws
+    torch.cuda.empty_cache()
+
+    # long sequence
+    b, d, L = 1, 256, 1 << 20
+    u, de, z = rnd((b, d, L)), rnd((b, d, L), 0.5), rnd((b, d, L))
+    B, C = rnd((b, N, L)), rnd((b, N, L))
+    A, D, bias = prm(d, N, 1e-4, 1e-2)
+    ws = torch.empty(max(1, ssm.fwd_workspace_bytes(b, d, L, N, torch.bfloat16)), dtype=torch.uint8, device=dev)
+    ms = timeit(lambda: ssm.ssm_scan_fwd(u, de, A, B, C, D=D, z=z, dt_bias=bias, workspace=ws), 5)
+    byt = 4 * b * d * L * 2 + 2 * b * N * L * 2
+    out["long_seq_1m"] = {"shape": "1x256x1048576 N16 bf16", "fwd_ms": ms,
+                          "tokens_per_s": b * L / (ms * 1e-3), "hbm_gbs": byt / (ms * 1e-3) / 1e9}
+    del u, de, z, B, C, ws
+    torch.cuda.empty_cache()
+
+    # decode: 256 x 5120 x 16 state; L2 (126 MB) is flushed before every step so the 84 MB
+    # state comes from HBM, the flush itself is timed separately and subtracted
+    b, d = 256, 5120
+    state = torch.zeros((b, d, N), device=dev)
+    x, dtr, zz = rnd((b, d)), rnd((b, d), 0.5), rnd((b, d))
+    Bd, Cd = rnd((b, N)), rnd((b, N))
+    A, D, bias = prm(d, N, 1e-3, 1e-1)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    t_flush = timeit(lambda: flush.fill_(1), 20)
+    t_all = timeit(lambda: (flush.fill_(1), ssm.ssm_state_update(state, x, dtr, A, Bd, Cd, D=D, z=zz,
+                                                                  dt_bias=bias)), 50)
+    us = (t_all - t_flush) * 1e3
+    byt = 2 * b * d * N * 4 + 4 * b * d * 2 + 2 * b * N * 2
+    out["decode_b256"] = {"shape": "256x5120x16 f32 state, bf16 io", "us_per_step": us,
+                          "hbm_gbs": byt / (us * 1e-6) / 1e9, "l2": "flushed before each step"}
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-baseline", action="store_true", help="skip the CPU oracle timing")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank, world, local = dist_env()
+
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import selective_state_space_23_b200 as ssm
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU (the library has no CPU path)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    ssm.library_path()
+
+    w = workload(WORKLOAD)
+    x = make_inputs(w, seed=rank)  # each rank scans its own batch
+    xd = {k: v.to(dev) for k, v in x.items()}
+    out = torch.empty_like(xd["u"])
+    nws = ssm.fwd_workspace_bytes(w.batch, w.dim, w.seqlen, w.dstate, w.io_dtype)
+    ws = torch.empty(nws, dtype=torch.uint8, device=dev) if nws else None
+    launches_per_step = 3 if nws else 1  # time split: summary, carry, output passes
+
+    def step():
+        ssm.ssm_scan_fwd(xd["u"], xd["delta"], xd["A"], xd["B"], xd["C"], D=xd["D"], z=xd["z"],
+                         dt_bias=xd["dt_bias"], out=out, workspace=ws)
+
+    K, W = args.steps, args.warmup
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize()
+        barrier(world)
+        e0.record()
+        for i in range(K):
+            ev_s[i].record()
+            step()
+            ev_e[i].record()
+        e1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+    total_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    kern_ms = statistics.fmean(ev_s[i].elapsed_time(ev_e[i]) for i in range(K))
+    kern_ms = max_over_ranks(kern_ms, world, dev)
+    ms_step = total_ms / K
+    value = world * w.tokens / (ms_step * 1e-3)
+
+    # end to end through the public call with host buffers: pinned H2D of the step's inputs,
+    # the scan, D2H of the output, every step
+    hx = {k: v.pin_memory() for k, v in x.items()}
+    hout = torch.empty_like(x["u"]).pin_memory()
+    names_in = ("u", "delta", "z", "B", "C")
+    h2d = sum(hx[k].numel() * hx[k].element_size() for k in names_in)
+    d2h = hout.numel() * hout.element_size()
+
+    def e2e_step():
+        for k in names_in:
+            xd[k].copy_(hx[k], non_blocking=True)
+        step()
+        hout.copy_(out, non_blocking=True)
+
+    e2e_ms = e2e_value = None
+    if args.e2e_steps > 0:
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record()
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        f1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_ms = max_over_ranks(f0.elapsed_time(f1), world, dev) / args.e2e_steps
+        e2e_value = world * w.tokens / (e2e_ms * 1e-3)
+
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+        return 0
+
+    peaks = load_peaks()
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    byts = compulsory_bytes(w)
+    elems = w.batch * w.dim * w.seqlen * w.dstate
+    hbm_gbs = byts / (kern_ms * 1e-3) / 1e9
+    alu_peak = alu_peak_elems_per_s(sms, peaks["sm_max_mhz"])
+    alu_ach = elems / (kern_ms * 1e-3)
+    traffic = recorded_traffic()
+    if args.no_baseline:
+        cb_value = cb_cores = None
+        cb_desc = "skipped (--no-baseline)"
+    else:
+        cb_value, cb_cores, cb_desc, _ = oracle_sample_time(w, seed=0)
+    extras = {} if args.no_extras else bench_extras(dev)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 io / f32 state", "data": "synthetic (seeded)",
+        "config": {"workload": "mamba370m_fwd: batch 8 x dim 2048 x L 2048, N 16 (Mamba-370m layer shape)",
+                   "global_batch": w.batch * world, "seq_len": w.seqlen, "dstate": w.dstate,
+                   "parallelism": f"dp{world} (independent batches, no collective)",
+                   "l2": "inputs (270 MB/step) larger than L2 (126 MB); no flush",
+                   "hbm_gbs": hbm_gbs, "hbm_frac_of_measured": hbm_gbs / peaks["hbm_gbs"]},
+        "roofline": {"bound": "alu", "achieved": alu_ach / 1e9, "peak": alu_peak / 1e9,
+                     "unit": "Gelem/s", "frac": alu_ach / alu_peak, "traffic": traffic,
+                     "element": "one (channel, step, state) update: 4 fp32 ops + one 2^x",
+                     "peak_basis": f"{sms} SMs x {peaks['sm_max_mhz']:.0f} MHz x 21.8 elem/clk/SM "
+                                   "(128 FMA + 16 MUFU lanes, best exp split)",
+                     "hbm": {"achieved": hbm_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": hbm_gbs / peaks["hbm_gbs"], "peak_source": peaks["source"],
+                             "bytes_per_launch": byts},
+                     "kernel_ms": kern_ms},
+        "cpu_baseline": {"value": cb_value, "unit": UNIT, "cores": cb_cores, "kind": "oracle",
+                         "sample": cb_desc},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms},
+        "gpu_launches": K * launches_per_step,
+        "clocks": clk.summary(),
+        "extras": extras,
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,162 @@
+/*
+ * ssm_scan.h -- C ABI of the B200 selective state-space (S6) scan library (libssm_b200.so).
+ *
+ * The operation (all three entry points compute parts of it):
+ *   "Mamba: Linear-Time Sequence Modeling with Selective State Spaces" (Gu & Dao, arXiv
+ *   2312.00752; Turkish summary page):
+ *     section "Yöntem"                 -- diagonal SSM discretised with step Δ: Ā = exp(ΔA),
+ *                                         recurrence h_t = Ā h_{t-1} + B̄ x_t, readout y_t = C h_t;
+ *     section "Seçim Mekanizması (S6)" -- B_t, C_t are per-token N-vectors shared by all D
+ *                                         channels; Δ_t = softplus(Parameter + s_Δ(x_t));
+ *     section "Donanım Duyarlı Durum Genişletme" -- the expanded (batch, L, D, N) state is kept
+ *                                         on chip and never written to HBM; the backward pass
+ *                                         recomputes the states;
+ *     section "Sorular"                -- generation keeps only a fixed D x N state per layer.
+ *   Per channel (b, d), time t and state n < N this library computes
+ *     Δ_t      = softplus(delta[b,d,t] + dt_bias[d])   (delta_softplus != 0)
+ *              = delta[b,d,t] + dt_bias[d]              (delta_softplus == 0)
+ *     h[n]     = exp(Δ_t A[d,n]) h[n] + Δ_t B[b,n,t] u[b,d,t]
+ *     y        = Σ_n C[b,n,t] h[n] + D[d] u[b,d,t]
+ *     out      = y * silu(z[b,d,t])        (out = y when z is NULL)
+ *   The input term Δ_t B_t x_t is the first-order form of the zero-order-hold B̄; the state is
+ *   updated before it is read out (y_t uses h_t).
+ *
+ * Conventions for every entry point:
+ *   - Pointers are DEVICE pointers (or host memory registered/mapped for device access) on the
+ *     CURRENT CUDA device, owned by the caller.  The library allocates no memory; scratch space
+ *     comes from the caller through `workspace`.  Outputs must not alias inputs, except
+ *     `state` in ssm_state_update, which is updated in place by design.
+ *   - io_dtype (ssm_dtype) is the element type of every "io" tensor (u, delta, z, B, C, out,
+ *     dout, du, ddelta, dz, dB, dC, x, dt): SSM_F32 or SSM_BF16.  A, D, dt_bias, h0, hL, ckpt,
+ *     dhL, dh0, dA, dD, ddt_bias and state are always float32.
+ *   - All tensors are dense and row-major (last index contiguous), with the layouts given per
+ *     argument.  1 <= dstate <= 16 (SSM_EUNSUPPORTED above).
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream) and the call
+ *     returns without synchronising.  A launch failure is reported by the return value; an
+ *     error raised later by the device is reported by CUDA on the stream as usual.
+ *   - Errors are returned, never raised by abort/exit.  Arguments are validated on the host
+ *     before anything is enqueued: NULL required pointers, non-positive sizes, bad dtype codes,
+ *     misaligned pointers, pointers the current device cannot access, and device allocations
+ *     smaller than the tensor they must hold all return SSM_EINVAL with nothing launched;
+ *     ssm_last_error() gives a one-line description (per thread).
+ *   - Not thread-safe with respect to concurrent use of the SAME workspace.
+ */
+#ifndef SSM_SCAN_H_
+#define SSM_SCAN_H_
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define SSM_API __attribute__((visibility("default")))
+#else
+#define SSM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Number of time steps between two stored states in the checkpoint tensor `ckpt`. */
+#define SSM_CKPT_STEPS 16
+/* Largest supported dstate (N). */
+#define SSM_MAX_DSTATE 16
+
+typedef enum { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype;
+
+typedef enum {
+  SSM_OK = 0,
+  SSM_EINVAL = 1,        /* invalid argument; nothing was launched */
+  SSM_EUNSUPPORTED = 2,  /* valid request this build does not implement (e.g. dstate > 16) */
+  SSM_ECUDA = 3,         /* a CUDA runtime call or kernel launch failed */
+  SSM_EWORKSPACE = 4     /* workspace NULL or smaller than the size function returned */
+} ssm_status;
+
+/* Static description of a status code. */
+SSM_API const char* ssm_status_string(int status);
+/* Description of the last failure on the calling thread ("" if none). */
+SSM_API const char* ssm_last_error(void);
+/* Library version string. */
+SSM_API const char* ssm_version(void);
+
+/*
+ * Bytes of workspace ssm_scan_fwd may use for this shape on the current device (0 when the
+ * launch plan needs none).  With less (or NULL) workspace ssm_scan_fwd still computes the same
+ * result, without splitting the time axis (slower when batch*dim is small).
+ */
+SSM_API size_t ssm_scan_fwd_workspace_size(int batch, int dim, int seqlen, int dstate, int io_dtype);
+
+/*
+ * Forward selective scan ("Yöntem", "Seçim Mekanizması (S6)", "Donanım Duyarlı Durum Genişletme").
+ *   u, delta, z [batch][dim][seqlen] io    inputs x_t, raw step s_Δ(x_t), gate input (z may be NULL)
+ *   A         [dim][dstate] f32           diagonal state matrix (any real values)
+ *   B, C      [batch][dstate][seqlen] io  input-dependent B_t, C_t, shared across dim
+ *   D         [dim] f32 or NULL           skip term D x_t (added before the gate)
+ *   dt_bias   [dim] f32 or NULL           the per-channel "Parameter" added to delta
+ *   h0        [batch][dim][dstate] f32 or NULL   initial state (NULL = zero)
+ *   hL        [batch][dim][dstate] f32 or NULL   OUT: final state h_{L-1}
+ *   out       [batch][dim][seqlen] io     OUT: gated output
+ *   ckpt      [batch][dim][ceil(seqlen/SSM_CKPT_STEPS)][dstate] f32 or NULL
+ *             OUT: state entering every SSM_CKPT_STEPS-step block (block k holds h_{16k-1},
+ *             block 0 holds h0); pass it to ssm_scan_bwd to skip its state replay pass.
+ *   workspace, workspace_bytes            scratch (may be NULL/0), see the size function.
+ * Returns SSM_OK or an error code (nothing launched on error).
+ */
+SSM_API int ssm_scan_fwd(const void* u, const void* delta, const float* A, const void* B, const void* C,
+                 const float* D, const void* z, const float* dt_bias, int delta_softplus,
+                 const float* h0, float* hL, void* out, float* ckpt, void* workspace,
+                 size_t workspace_bytes, int batch, int dim, int seqlen, int dstate,
+                 int io_dtype, void* stream);
+
+/*
+ * Bytes of workspace ssm_scan_bwd needs.  have_ckpt != 0: the caller will pass the `ckpt`
+ * written by ssm_scan_fwd with the same inputs (smaller workspace, one pass fewer).
+ */
+SSM_API size_t ssm_scan_bwd_workspace_size(int batch, int dim, int seqlen, int dstate, int io_dtype,
+                                   int have_ckpt);
+
+/*
+ * Backward pass of ssm_scan_fwd with state recomputation ("Donanım Duyarlı Durum Genişletme":
+ * intermediate states are recomputed, not stored).  Gradients by the chain rule through the
+ * forward recurrence:
+ *   λ_t  = g_t C_t + exp(Δ_{t+1} A) λ_{t+1},  g_t = dout_t silu(z_t),  λ_{L-1} += dhL
+ *   du_t = g_t D + Δ_t Σ_n λ_t B_t;   ddelta_t = (Σ_n λ_t (A Ā_t h_{t-1} + B_t u_t)) softplus'
+ *   dB_t = Σ_d λ_t Δ_t u_t;   dC_t = Σ_d g_t h_t;   dA = Σ_{b,t} λ_t Δ_t Ā_t h_{t-1}
+ *   dD = Σ_{b,t} g_t u_t;   ddt_bias = Σ_{b,t} ddelta_t;   dz_t = dout_t y_t silu'(z_t);
+ *   dh0 = Ā_0 λ_0.
+ * Inputs: as ssm_scan_fwd, plus
+ *   dout      [batch][dim][seqlen] io     upstream gradient of `out`
+ *   dhL       [batch][dim][dstate] f32 or NULL   upstream gradient of hL
+ *   ckpt      as written by ssm_scan_fwd, or NULL (then recomputed into the workspace)
+ * Outputs (each may be NULL to skip it, except that at least one must be given):
+ *   du, ddelta, dz [batch][dim][seqlen] io (dz only when z != NULL)
+ *   dB, dC    [batch][dstate][seqlen] io
+ *   dA [dim][dstate] f32;  dD, ddt_bias [dim] f32;  dh0 [batch][dim][dstate] f32
+ * All outputs are OVERWRITTEN (not accumulated).  Summed gradients are reduced in a fixed
+ * order, so results are bitwise reproducible run to run.
+ * workspace: at least ssm_scan_bwd_workspace_size(..., ckpt != NULL) bytes, 256-byte aligned.
+ */
+SSM_API int ssm_scan_bwd(const void* u, const void* delta, const float* A, const void* B, const void* C,
+                 const float* D, const void* z, const float* dt_bias, int delta_softplus,
+                 const float* h0, const void* dout, const float* dhL, const float* ckpt,
+                 void* du, void* ddelta, float* dA, void* dB, void* dC, float* dD, void* dz,
+                 float* ddt_bias, float* dh0, void* workspace, size_t workspace_bytes,
+                 int batch, int dim, int seqlen, int dstate, int io_dtype, void* stream);
+
+/*
+ * One-token recurrent step ("Sorular": fixed D x N state per layer, O(1) per token).
+ *   state     [batch][dim][dstate] f32    IN/OUT, updated in place: h <- exp(ΔA) h + Δ B x
+ *   x, dt, z  [batch][dim] io            token input, raw step, gate input (z may be NULL)
+ *   A [dim][dstate] f32;  B, C [batch][dstate] io;  D, dt_bias [dim] f32 or NULL
+ *   out       [batch][dim] io             OUT: (C.h + D x) * silu(z)
+ * Calling it L times reproduces ssm_scan_fwd over L steps (same arithmetic per step).
+ */
+SSM_API int ssm_state_update(float* state, const void* x, const void* dt, const float* A, const void* B,
+                     const void* C, const float* D, const void* z, const float* dt_bias,
+                     int delta_softplus, void* out, int batch, int dim, int dstate,
+                     int io_dtype, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSM_SCAN_H_ */

@@ -1,0 +1,196 @@
+"""B200-native selective state-space (S6) scan: Python binding of libssm_b200.so.
+
+The three entry points mirror the C ABI (include/ssm_scan.h) and do argument marshalling only:
+every step of the computation runs in the library's sm_100a kernels.  Tensors are torch CUDA
+tensors (PyTorch provides device memory and streams); outputs not supplied by the caller are
+allocated here with torch.  Work is enqueued on the current torch CUDA stream.
+
+  ssm_scan_fwd      forward selective scan (gated output, optional final state / checkpoints)
+  ssm_scan_bwd      gradients of ssm_scan_fwd, recomputing the states
+  ssm_state_update  one-token recurrent step, state updated in place
+"""
+import ctypes
+
+import torch
+
+from . import _abi
+from ._abi import CKPT_STEPS, MAX_DSTATE
+
+__all__ = ["ssm_scan_fwd", "ssm_scan_bwd", "ssm_state_update", "fwd_workspace_bytes",
+           "bwd_workspace_bytes", "CKPT_STEPS", "MAX_DSTATE", "library_path"]
+
+_IO = {torch.float32: _abi.SSM_F32, torch.bfloat16: _abi.SSM_BF16}
+
+
+def library_path() -> str:
+    _abi.lib()
+    return _abi.LIB_PATH
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need(t, name, shape, dtype, device):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    _opt(t, name, shape, dtype, device)
+
+
+def _opt(t, name, shape, dtype, device):
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _io_code(dtype):
+    if dtype not in _IO:
+        raise TypeError(f"io dtype must be float32 or bfloat16, got {dtype}")
+    return _IO[dtype]
+
+
+def fwd_workspace_bytes(batch, dim, seqlen, dstate, dtype) -> int:
+    return int(_abi.lib().ssm_scan_fwd_workspace_size(batch, dim, seqlen, dstate, _io_code(dtype)))
+
+
+def bwd_workspace_bytes(batch, dim, seqlen, dstate, dtype, have_ckpt) -> int:
+    return int(_abi.lib().ssm_scan_bwd_workspace_size(batch, dim, seqlen, dstate, _io_code(dtype),
+                                                       int(bool(have_ckpt))))
+
+
+def _workspace(nbytes, device, given):
+    if nbytes == 0:
+        return None
+    if given is not None:
+        if given.device != device or given.numel() * given.element_size() < nbytes:
+            raise ValueError(f"workspace must hold {nbytes} bytes on {device}")
+        return given
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def ssm_scan_fwd(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=True, h0=None,
+                 return_final_state=False, return_ckpt=False, out=None, workspace=None):
+    """Forward scan.  u, delta, z: [batch, dim, L]; B, C: [batch, N, L] (io dtype f32 or bf16);
+    A: [dim, N] f32; D, dt_bias: [dim] f32; h0: [batch, dim, N] f32.
+    Returns out, or a tuple (out, hL?, ckpt?) when those are requested."""
+    dev = u.device
+    batch, dim, L = u.shape
+    N = A.shape[-1]
+    io = u.dtype
+    code = _io_code(io)
+    _need(u, "u", (batch, dim, L), io, dev)
+    _need(delta, "delta", (batch, dim, L), io, dev)
+    _need(A, "A", (dim, N), torch.float32, dev)
+    _need(B, "B", (batch, N, L), io, dev)
+    _need(C, "C", (batch, N, L), io, dev)
+    _opt(D, "D", (dim,), torch.float32, dev)
+    _opt(z, "z", (batch, dim, L), io, dev)
+    _opt(dt_bias, "dt_bias", (dim,), torch.float32, dev)
+    _opt(h0, "h0", (batch, dim, N), torch.float32, dev)
+    if out is None:
+        out = torch.empty((batch, dim, L), dtype=io, device=dev)
+    _need(out, "out", (batch, dim, L), io, dev)
+    hL = torch.empty((batch, dim, N), dtype=torch.float32, device=dev) if return_final_state else None
+    nblk = (L + CKPT_STEPS - 1) // CKPT_STEPS
+    ckpt = torch.empty((batch, dim, nblk, N), dtype=torch.float32, device=dev) if return_ckpt else None
+    ws = _workspace(fwd_workspace_bytes(batch, dim, L, N, io), dev, workspace)
+    rc = _abi.lib().ssm_scan_fwd(
+        _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias),
+        int(bool(delta_softplus)), _ptr(h0), _ptr(hL), _ptr(out), _ptr(ckpt), _ptr(ws),
+        0 if ws is None else ws.numel(), batch, dim, L, N, code, _stream(dev))
+    _abi.check(rc, "ssm_scan_fwd")
+    if not return_final_state and not return_ckpt:
+        return out
+    res = (out,)
+    if return_final_state:
+        res += (hL,)
+    if return_ckpt:
+        res += (ckpt,)
+    return res
+
+
+def ssm_scan_bwd(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None, delta_softplus=True,
+                 h0=None, dhL=None, ckpt=None, workspace=None, need=None):
+    """Gradients of :func:`ssm_scan_fwd`.  Returns a dict with du, ddelta, dA, dB, dC, dD, dz,
+    ddt_bias, dh0 (entries are None when the matching input is absent or not in ``need``)."""
+    dev = u.device
+    batch, dim, L = u.shape
+    N = A.shape[-1]
+    io = u.dtype
+    code = _io_code(io)
+    _need(u, "u", (batch, dim, L), io, dev)
+    _need(delta, "delta", (batch, dim, L), io, dev)
+    _need(A, "A", (dim, N), torch.float32, dev)
+    _need(B, "B", (batch, N, L), io, dev)
+    _need(C, "C", (batch, N, L), io, dev)
+    _need(dout, "dout", (batch, dim, L), io, dev)
+    _opt(D, "D", (dim,), torch.float32, dev)
+    _opt(z, "z", (batch, dim, L), io, dev)
+    _opt(dt_bias, "dt_bias", (dim,), torch.float32, dev)
+    _opt(h0, "h0", (batch, dim, N), torch.float32, dev)
+    _opt(dhL, "dhL", (batch, dim, N), torch.float32, dev)
+    nblk = (L + CKPT_STEPS - 1) // CKPT_STEPS
+    _opt(ckpt, "ckpt", (batch, dim, nblk, N), torch.float32, dev)
+    want = set(need) if need is not None else {"du", "ddelta", "dA", "dB", "dC", "dD", "dz",
+                                                "ddt_bias", "dh0"}
+    e = lambda shape, dt: torch.empty(shape, dtype=dt, device=dev)
+    g = {
+        "du": e((batch, dim, L), io) if "du" in want else None,
+        "ddelta": e((batch, dim, L), io) if "ddelta" in want else None,
+        "dz": e((batch, dim, L), io) if ("dz" in want and z is not None) else None,
+        "dB": e((batch, N, L), io) if "dB" in want else None,
+        "dC": e((batch, N, L), io) if "dC" in want else None,
+        "dA": e((dim, N), torch.float32) if "dA" in want else None,
+        "dD": e((dim,), torch.float32) if "dD" in want else None,
+        "ddt_bias": e((dim,), torch.float32) if "ddt_bias" in want else None,
+        "dh0": e((batch, dim, N), torch.float32) if "dh0" in want else None,
+    }
+    ws = _workspace(bwd_workspace_bytes(batch, dim, L, N, io, ckpt is not None), dev, workspace)
+    rc = _abi.lib().ssm_scan_bwd(
+        _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias),
+        int(bool(delta_softplus)), _ptr(h0), _ptr(dout), _ptr(dhL), _ptr(ckpt),
+        _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]),
+        _ptr(g["dD"]), _ptr(g["dz"]), _ptr(g["ddt_bias"]), _ptr(g["dh0"]),
+        _ptr(ws), 0 if ws is None else ws.numel(), batch, dim, L, N, code, _stream(dev))
+    _abi.check(rc, "ssm_scan_bwd")
+    return g
+
+
+def ssm_state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=True,
+                     out=None):
+    """One decode step; ``state`` [batch, dim, N] f32 is updated in place.  x, dt, z:
+    [batch, dim]; B, C: [batch, N] (io dtype).  Returns out [batch, dim]."""
+    dev = state.device
+    batch, dim, N = state.shape
+    io = x.dtype
+    code = _io_code(io)
+    _need(state, "state", (batch, dim, N), torch.float32, dev)
+    _need(x, "x", (batch, dim), io, dev)
+    _need(dt, "dt", (batch, dim), io, dev)
+    _need(A, "A", (dim, N), torch.float32, dev)
+    _need(B, "B", (batch, N), io, dev)
+    _need(C, "C", (batch, N), io, dev)
+    _opt(D, "D", (dim,), torch.float32, dev)
+    _opt(z, "z", (batch, dim), io, dev)
+    _opt(dt_bias, "dt_bias", (dim,), torch.float32, dev)
+    if out is None:
+        out = torch.empty((batch, dim), dtype=io, device=dev)
+    _need(out, "out", (batch, dim), io, dev)
+    rc = _abi.lib().ssm_state_update(
+        _ptr(state), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+        _ptr(dt_bias), int(bool(delta_softplus)), _ptr(out), batch, dim, N, code, _stream(dev))
+    _abi.check(rc, "ssm_state_update")
+    return out

@@ -1,0 +1,63 @@
+"""ctypes loader for libssm_b200.so (the C ABI in include/ssm_scan.h).
+
+Loading fails loudly: there is no fallback implementation of any entry point.
+"""
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libssm_b200.so")
+
+SSM_F32, SSM_BF16 = 0, 1
+SSM_OK, SSM_EINVAL, SSM_EUNSUPPORTED, SSM_ECUDA, SSM_EWORKSPACE = 0, 1, 2, 3, 4
+CKPT_STEPS = 16
+MAX_DSTATE = 16
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_sz = ctypes.c_size_t
+
+# name -> (restype, argtypes)
+SIGNATURES = {
+    "ssm_status_string": (ctypes.c_char_p, [_i]),
+    "ssm_last_error": (ctypes.c_char_p, []),
+    "ssm_version": (ctypes.c_char_p, []),
+    "ssm_scan_fwd_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
+    "ssm_scan_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _sz,
+                          _i, _i, _i, _i, _i, _vp]),
+    "ssm_scan_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "ssm_scan_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp,
+                          _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                          _i, _i, _i, _i, _i, _vp]),
+    "ssm_state_update": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp,
+                              _i, _i, _i, _i, _vp]),
+}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (raises RuntimeError if it is missing or incomplete)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m selective_state_space_23_b200.build` "
+                "(nvcc, sm_100a). There is no CPU or fallback implementation.")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(l, name)  # AttributeError if the symbol is not exported
+            f.restype = res
+            f.argtypes = args
+        _lib = l
+    return _lib
+
+
+def last_error() -> str:
+    return lib().ssm_last_error().decode()
+
+
+def check(rc: int, what: str) -> None:
+    if rc != SSM_OK:
+        msg = lib().ssm_status_string(rc).decode()
+        raise RuntimeError(f"{what} failed: {msg} ({rc}): {last_error()}")

@@ -1,0 +1,423 @@
+// C-ABI layer: argument validation, launch planning and workspace carving for the selective
+// scan kernels.  Declarations and the full contract are in include/ssm_scan.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/ssm_scan.h"
+#include "ssm_kernels.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(SSM_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// ------------------------------------------------------------------ device properties
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 148;
+  }
+  static std::mutex mu;
+  static int cached[64] = {0};
+  std::lock_guard<std::mutex> lk(mu);
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = 148;
+  }
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  return n;
+}
+
+int env_int(const char* name, int dflt) {
+  const char* v = getenv(name);
+  if (!v || !*v) return dflt;
+  return atoi(v);
+}
+
+// ------------------------------------------------------------------ pointer validation
+typedef int (*PFN_getAddressRange)(unsigned long long*, size_t*, unsigned long long);
+
+PFN_getAddressRange address_range_fn() {
+  static PFN_getAddressRange fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_getAddressRange>(p);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
+// The pointer must be usable by kernels on the current device and hold `bytes` bytes.
+int check_ptr(const void* p, size_t bytes, size_t align, const char* name) {
+  if (!p) return fail(SSM_EINVAL, "%s is NULL", name);
+  if (reinterpret_cast<uintptr_t>(p) % align)
+    return fail(SSM_EINVAL, "%s is not %zu-byte aligned", name, align);
+  cudaPointerAttributes at;
+  cudaError_t e = cudaPointerGetAttributes(&at, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(SSM_EINVAL, "%s: cannot query pointer (%s)", name, cudaGetErrorString(e));
+  }
+  int dev = -1;
+  cudaGetDevice(&dev);
+  switch (at.type) {
+    case cudaMemoryTypeDevice:
+    case cudaMemoryTypeManaged: {
+      if (at.type == cudaMemoryTypeDevice && at.device != dev)
+        return fail(SSM_EINVAL, "%s lives on device %d, current device is %d", name, at.device, dev);
+      PFN_getAddressRange fn = address_range_fn();
+      if (fn) {
+        unsigned long long base = 0;
+        size_t size = 0;
+        if (fn(&base, &size, (unsigned long long)(uintptr_t)p) == 0) {
+          const unsigned long long q = (unsigned long long)(uintptr_t)p;
+          if (q < base || q - base + bytes > size)
+            return fail(SSM_EINVAL, "%s: allocation holds %llu bytes from this pointer, %zu needed",
+                        name, (unsigned long long)(base + size - q), bytes);
+        }
+      }
+      return SSM_OK;
+    }
+    case cudaMemoryTypeHost:
+      if (at.devicePointer != p)
+        return fail(SSM_EINVAL, "%s is page-locked host memory not mapped at the same address", name);
+      return SSM_OK;
+    default:
+      return fail(SSM_EINVAL, "%s is not device-accessible memory (pageable host pointer?)", name);
+  }
+}
+
+int check_opt(const void* p, size_t bytes, size_t align, const char* name) {
+  return p ? check_ptr(p, bytes, align, name) : SSM_OK;
+}
+
+#define TRY(x)                 \
+  do {                         \
+    int _rc = (x);             \
+    if (_rc != SSM_OK) return _rc; \
+  } while (0)
+
+int check_dims(int batch, int dim, int seqlen, int dstate, int io) {
+  if (batch <= 0 || dim <= 0 || seqlen <= 0 || dstate <= 0)
+    return fail(SSM_EINVAL, "sizes must be positive (batch=%d dim=%d seqlen=%d dstate=%d)", batch,
+                dim, seqlen, dstate);
+  if (io != SSM_F32 && io != SSM_BF16) return fail(SSM_EINVAL, "io_dtype %d is not SSM_F32/SSM_BF16", io);
+  if (dstate > SSM_MAX_DSTATE)
+    return fail(SSM_EUNSUPPORTED, "dstate %d > %d is not implemented", dstate, SSM_MAX_DSTATE);
+  if ((long long)batch * ((dim + 31) / 32) > (1LL << 30))
+    return fail(SSM_EUNSUPPORTED, "batch*dim too large for one launch");
+  return SSM_OK;
+}
+
+size_t esize(int io) { return io == SSM_BF16 ? 2 : 4; }
+size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
+
+bool aligned16(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// ------------------------------------------------------------------ forward launch plan
+struct FwdPlan {
+  int nchunk;
+  int chunk_len;
+  size_t ws_bytes;
+};
+
+FwdPlan plan_fwd(int batch, int dim, int seqlen) {
+  const int smsp = 4 * sm_count();
+  const long long warps = (long long)batch * ((dim + 31) / 32);
+  const int nblk = (seqlen + ssm::kBlk - 1) / ssm::kBlk;
+  int S = 1;
+  const int forced = env_int("SSM_FWD_SPLIT", 0);
+  if (forced > 0) {
+    S = forced;
+  } else if (warps * 2 < smsp) {
+    // fewer than half a warp per scheduler: split time so every scheduler gets ~2 warps
+    S = (int)((2LL * smsp + warps - 1) / warps);
+  }
+  S = S < 1 ? 1 : (S > nblk ? nblk : S);
+  FwdPlan p;
+  if (S <= 1) {
+    p.nchunk = 1;
+    p.chunk_len = nblk * ssm::kBlk;
+    p.ws_bytes = 0;
+    return p;
+  }
+  const int blk_per_chunk = (nblk + S - 1) / S;
+  p.chunk_len = blk_per_chunk * ssm::kBlk;
+  p.nchunk = (seqlen + p.chunk_len - 1) / p.chunk_len;
+  if (p.nchunk <= 1) {
+    p.nchunk = 1;
+    p.ws_bytes = 0;
+    return p;
+  }
+  const size_t nch = (size_t)batch * dim;
+  p.ws_bytes = align_up(p.nchunk * nch * ssm::kNS * 4) * 2 + align_up(p.nchunk * nch * 4);
+  return p;
+}
+
+int fwd_wpb() {
+  const int w = env_int("SSM_FWD_WPB", 4);
+  return (w == 1 || w == 2 || w == 4) ? w : 4;
+}
+int fwd_kmufu() { return env_int("SSM_FWD_KMUFU", 10); }
+
+struct BwdLayout {
+  size_t ckpt, part_bc, part_adt, total;
+  int wpb, ngroups;
+};
+
+BwdLayout layout_bwd(int batch, int dim, int seqlen, int dstate, bool have_ckpt) {
+  BwdLayout l;
+  l.wpb = env_int("SSM_BWD_WPB", 1);
+  if (l.wpb < 1 || l.wpb > 4) l.wpb = 1;
+  const int warps_per_b = (dim + 31) / 32;
+  l.ngroups = (warps_per_b + l.wpb - 1) / l.wpb;
+  const size_t nch = (size_t)batch * dim;
+  const size_t nblk = (seqlen + ssm::kBlk - 1) / ssm::kBlk;
+  l.ckpt = have_ckpt ? 0 : align_up(nch * nblk * dstate * 4);
+  l.part_bc = align_up((size_t)l.ngroups * batch * 2 * ssm::kNS * seqlen * 4);
+  l.part_adt = align_up(nch * (ssm::kNS + 2) * 4);
+  l.total = l.ckpt + l.part_bc + l.part_adt;
+  return l;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ssm_status_string(int status) {
+  switch (status) {
+    case SSM_OK: return "ok";
+    case SSM_EINVAL: return "invalid argument";
+    case SSM_EUNSUPPORTED: return "unsupported";
+    case SSM_ECUDA: return "CUDA error";
+    case SSM_EWORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+const char* ssm_last_error(void) { return g_err; }
+
+const char* ssm_version(void) { return "ssm_b200 0.1 (sm_100a)"; }
+
+size_t ssm_scan_fwd_workspace_size(int batch, int dim, int seqlen, int dstate, int io_dtype) {
+  if (check_dims(batch, dim, seqlen, dstate, io_dtype) != SSM_OK) return 0;
+  return plan_fwd(batch, dim, seqlen).ws_bytes;
+}
+
+int ssm_scan_fwd(const void* u, const void* delta, const float* A, const void* B, const void* C,
+                 const float* D, const void* z, const float* dt_bias, int delta_softplus,
+                 const float* h0, float* hL, void* out, float* ckpt, void* workspace,
+                 size_t workspace_bytes, int batch, int dim, int seqlen, int dstate,
+                 int io_dtype, void* stream) {
+  g_err[0] = 0;
+  TRY(check_dims(batch, dim, seqlen, dstate, io_dtype));
+  const size_t es = esize(io_dtype);
+  const size_t nx = (size_t)batch * dim * seqlen * es;
+  const size_t nbc = (size_t)batch * dstate * seqlen * es;
+  const size_t nst = (size_t)batch * dim * dstate * 4;
+  const size_t nblk = (seqlen + ssm::kBlk - 1) / ssm::kBlk;
+  TRY(check_ptr(u, nx, es, "u"));
+  TRY(check_ptr(delta, nx, es, "delta"));
+  TRY(check_ptr(A, (size_t)dim * dstate * 4, 4, "A"));
+  TRY(check_ptr(B, nbc, es, "B"));
+  TRY(check_ptr(C, nbc, es, "C"));
+  TRY(check_ptr(out, nx, es, "out"));
+  TRY(check_opt(D, (size_t)dim * 4, 4, "D"));
+  TRY(check_opt(z, nx, es, "z"));
+  TRY(check_opt(dt_bias, (size_t)dim * 4, 4, "dt_bias"));
+  TRY(check_opt(h0, nst, 4, "h0"));
+  TRY(check_opt(hL, nst, 4, "hL"));
+  TRY(check_opt(ckpt, (size_t)batch * dim * nblk * dstate * 4, 4, "ckpt"));
+  if (out == u || out == delta || out == z) return fail(SSM_EINVAL, "out aliases an input");
+
+  FwdPlan plan = plan_fwd(batch, dim, seqlen);
+  if (plan.nchunk > 1 && (!workspace || workspace_bytes < plan.ws_bytes ||
+                          (reinterpret_cast<uintptr_t>(workspace) & 255))) {
+    plan.nchunk = 1;  // not enough scratch: same result without the time split
+    plan.chunk_len = (int)nblk * ssm::kBlk;
+  }
+  if (plan.nchunk > 1) TRY(check_ptr(workspace, plan.ws_bytes, 256, "workspace"));
+
+  ssm::FwdArgs a;
+  memset(&a, 0, sizeof(a));
+  a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
+  a.A = A; a.D = D; a.dt_bias = dt_bias; a.h0 = h0;
+  a.out = out; a.hL = hL; a.ckpt = ckpt;
+  a.batch = batch; a.dim = dim; a.L = seqlen; a.N = dstate;
+  a.chunk_len = plan.chunk_len; a.nchunk = plan.nchunk;
+  a.softplus = delta_softplus ? 1 : 0;
+  a.warps_per_b = (dim + 31) / 32;
+  a.nwarps = (long long)batch * a.warps_per_b;
+  const bool vec = (seqlen * es) % 16 == 0 && aligned16(u) && aligned16(delta) && aligned16(z) &&
+                   aligned16(out) && aligned16(B) && aligned16(C);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int wpb = fwd_wpb(), km = fwd_kmufu();
+  cudaError_t e;
+  if (plan.nchunk > 1) {
+    const size_t nch = (size_t)batch * dim;
+    char* w = reinterpret_cast<char*>(workspace);
+    float* summ = reinterpret_cast<float*>(w);
+    float* hin = reinterpret_cast<float*>(w + align_up(plan.nchunk * nch * ssm::kNS * 4));
+    float* dsum = reinterpret_cast<float*>(w + 2 * align_up(plan.nchunk * nch * ssm::kNS * 4));
+    ssm::FwdArgs as = a;
+    as.summ = summ; as.dsum = dsum;
+    as.out = nullptr; as.hL = nullptr; as.ckpt = nullptr; as.h0 = nullptr;
+    if ((e = ssm::launch_fwd(as, io_dtype, vec, ssm::kFwdSummary, wpb, km, s)) != cudaSuccess)
+      return cuda_fail(e, "forward summary pass");
+    if ((e = ssm::launch_fwd_carry(a, summ, dsum, hin, s)) != cudaSuccess)
+      return cuda_fail(e, "forward carry pass");
+    a.hin = hin;
+  }
+  if ((e = ssm::launch_fwd(a, io_dtype, vec, ssm::kFwdOut, wpb, km, s)) != cudaSuccess)
+    return cuda_fail(e, "forward pass");
+  return SSM_OK;
+}
+
+size_t ssm_scan_bwd_workspace_size(int batch, int dim, int seqlen, int dstate, int io_dtype,
+                                   int have_ckpt) {
+  if (check_dims(batch, dim, seqlen, dstate, io_dtype) != SSM_OK) return 0;
+  return layout_bwd(batch, dim, seqlen, dstate, have_ckpt != 0).total;
+}
+
+int ssm_scan_bwd(const void* u, const void* delta, const float* A, const void* B, const void* C,
+                 const float* D, const void* z, const float* dt_bias, int delta_softplus,
+                 const float* h0, const void* dout, const float* dhL, const float* ckpt,
+                 void* du, void* ddelta, float* dA, void* dB, void* dC, float* dD, void* dz,
+                 float* ddt_bias, float* dh0, void* workspace, size_t workspace_bytes,
+                 int batch, int dim, int seqlen, int dstate, int io_dtype, void* stream) {
+  g_err[0] = 0;
+  TRY(check_dims(batch, dim, seqlen, dstate, io_dtype));
+  const size_t es = esize(io_dtype);
+  const size_t nx = (size_t)batch * dim * seqlen * es;
+  const size_t nbc = (size_t)batch * dstate * seqlen * es;
+  const size_t nst = (size_t)batch * dim * dstate * 4;
+  const size_t nblk = (seqlen + ssm::kBlk - 1) / ssm::kBlk;
+  TRY(check_ptr(u, nx, es, "u"));
+  TRY(check_ptr(delta, nx, es, "delta"));
+  TRY(check_ptr(A, (size_t)dim * dstate * 4, 4, "A"));
+  TRY(check_ptr(B, nbc, es, "B"));
+  TRY(check_ptr(C, nbc, es, "C"));
+  TRY(check_ptr(dout, nx, es, "dout"));
+  TRY(check_opt(D, (size_t)dim * 4, 4, "D"));
+  TRY(check_opt(z, nx, es, "z"));
+  TRY(check_opt(dt_bias, (size_t)dim * 4, 4, "dt_bias"));
+  TRY(check_opt(h0, nst, 4, "h0"));
+  TRY(check_opt(dhL, nst, 4, "dhL"));
+  TRY(check_opt(ckpt, (size_t)batch * dim * nblk * dstate * 4, 4, "ckpt"));
+  TRY(check_opt(du, nx, es, "du"));
+  TRY(check_opt(ddelta, nx, es, "ddelta"));
+  TRY(check_opt(dz, nx, es, "dz"));
+  TRY(check_opt(dB, nbc, es, "dB"));
+  TRY(check_opt(dC, nbc, es, "dC"));
+  TRY(check_opt(dA, (size_t)dim * dstate * 4, 4, "dA"));
+  TRY(check_opt(dD, (size_t)dim * 4, 4, "dD"));
+  TRY(check_opt(ddt_bias, (size_t)dim * 4, 4, "ddt_bias"));
+  TRY(check_opt(dh0, nst, 4, "dh0"));
+  if (!du && !ddelta && !dA && !dB && !dC && !dD && !dz && !ddt_bias && !dh0)
+    return fail(SSM_EINVAL, "no gradient output requested");
+  if (dz && !z) return fail(SSM_EINVAL, "dz requested but z is NULL");
+
+  const BwdLayout l = layout_bwd(batch, dim, seqlen, dstate, ckpt != nullptr);
+  if (!workspace || workspace_bytes < l.total)
+    return fail(SSM_EWORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes, l.total);
+  if (reinterpret_cast<uintptr_t>(workspace) & 255)
+    return fail(SSM_EINVAL, "workspace is not 256-byte aligned");
+  TRY(check_ptr(workspace, l.total, 256, "workspace"));
+
+  char* w = reinterpret_cast<char*>(workspace);
+  float* ck_ws = reinterpret_cast<float*>(w);
+  float* part_bc = reinterpret_cast<float*>(w + l.ckpt);
+  float* part_adt = reinterpret_cast<float*>(w + l.ckpt + l.part_bc);
+  const bool vec = (seqlen * es) % 16 == 0 && aligned16(u) && aligned16(delta) && aligned16(z) &&
+                   aligned16(dout) && aligned16(du) && aligned16(ddelta) && aligned16(dz) &&
+                   aligned16(B) && aligned16(C);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+
+  const float* ck = ckpt;
+  if (!ck) {
+    ssm::FwdArgs a;
+    memset(&a, 0, sizeof(a));
+    a.u = u; a.delta = delta; a.B = B; a.C = C; a.A = A; a.dt_bias = dt_bias; a.h0 = h0;
+    a.ckpt = ck_ws;
+    a.batch = batch; a.dim = dim; a.L = seqlen; a.N = dstate;
+    a.chunk_len = (int)nblk * ssm::kBlk; a.nchunk = 1;
+    a.softplus = delta_softplus ? 1 : 0;
+    a.warps_per_b = (dim + 31) / 32;
+    a.nwarps = (long long)batch * a.warps_per_b;
+    if ((e = ssm::launch_fwd(a, io_dtype, vec, ssm::kFwdCkpt, fwd_wpb(), fwd_kmufu(), s)) != cudaSuccess)
+      return cuda_fail(e, "backward state replay pass");
+    ck = ck_ws;
+  }
+  ssm::BwdArgs b;
+  memset(&b, 0, sizeof(b));
+  b.u = u; b.delta = delta; b.z = z; b.B = B; b.C = C; b.A = A; b.D = D; b.dt_bias = dt_bias;
+  b.dout = dout; b.dhL = dhL; b.ckpt = ck;
+  b.du = du; b.ddelta = ddelta; b.dz = dz; b.dh0 = dh0;
+  b.part_bc = part_bc; b.part_adt = part_adt;
+  b.batch = batch; b.dim = dim; b.L = seqlen; b.N = dstate;
+  b.softplus = delta_softplus ? 1 : 0;
+  b.warps_per_b = (dim + 31) / 32;
+  b.nwarps = (long long)batch * b.warps_per_b;
+  b.wpb = l.wpb;
+  b.ngroups = l.ngroups;
+  if ((e = ssm::launch_bwd(b, io_dtype, vec, s)) != cudaSuccess) return cuda_fail(e, "backward pass");
+  if ((e = ssm::launch_bwd_finish(b, io_dtype, dB, dC, dA, dD, ddt_bias, s)) != cudaSuccess)
+    return cuda_fail(e, "backward reduction");
+  return SSM_OK;
+}
+
+int ssm_state_update(float* state, const void* x, const void* dt, const float* A, const void* B,
+                     const void* C, const float* D, const void* z, const float* dt_bias,
+                     int delta_softplus, void* out, int batch, int dim, int dstate,
+                     int io_dtype, void* stream) {
+  g_err[0] = 0;
+  TRY(check_dims(batch, dim, 1, dstate, io_dtype));
+  const size_t es = esize(io_dtype);
+  const size_t nx = (size_t)batch * dim * es;
+  TRY(check_ptr(state, (size_t)batch * dim * dstate * 4, 4, "state"));
+  TRY(check_ptr(x, nx, es, "x"));
+  TRY(check_ptr(dt, nx, es, "dt"));
+  TRY(check_ptr(A, (size_t)dim * dstate * 4, 4, "A"));
+  TRY(check_ptr(B, (size_t)batch * dstate * es, es, "B"));
+  TRY(check_ptr(C, (size_t)batch * dstate * es, es, "C"));
+  TRY(check_ptr(out, nx, es, "out"));
+  TRY(check_opt(D, (size_t)dim * 4, 4, "D"));
+  TRY(check_opt(z, nx, es, "z"));
+  TRY(check_opt(dt_bias, (size_t)dim * 4, 4, "dt_bias"));
+  ssm::DecodeArgs a;
+  a.state = state; a.x = x; a.dt = dt; a.z = z; a.B = B; a.C = C; a.A = A; a.D = D;
+  a.dt_bias = dt_bias; a.out = out;
+  a.batch = batch; a.dim = dim; a.N = dstate; a.softplus = delta_softplus ? 1 : 0;
+  cudaError_t e = ssm::launch_decode(a, io_dtype, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "decode step");
+  return SSM_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,113 @@
+// One-token recurrent (decode) step of the selective SSM, sm_100a.
+//
+// Generation runs the model as a recurrence that keeps only a fixed D x N state per layer and
+// costs O(1) per token ("Mamba: ..." summary page, "Sorular": no KV cache during generation;
+// mamba-minimal news page: recurrent mode for one-step-at-a-time inference).  Per channel
+// c = (b, d):
+//   Δ = softplus(dt + dt_bias_d);  h_n <- exp(Δ A_dn) h_n + Δ B_n x   (in place)
+//   out = (Σ_n C_n h_n + D_d x) * silu(z)
+//
+// The step is bound by HBM traffic on the f32 state (read + write of batch*D*N*4 bytes).
+// Four lanes share a channel, each holding 4 consecutive states as one 128-bit load/store, so
+// a warp streams 512 contiguous bytes of state per access; the partial readouts are combined
+// with two butterfly shuffles.
+#include <type_traits>
+
+#include "ssm_device.cuh"
+#include "ssm_kernels.h"
+
+namespace ssm {
+namespace {
+
+template <typename IO> __device__ __forceinline__ float ld_io(const void* p, long long i);
+template <> __device__ __forceinline__ float ld_io<float>(const void* p, long long i) {
+  return reinterpret_cast<const float*>(p)[i];
+}
+template <> __device__ __forceinline__ float ld_io<uint16_t>(const void* p, long long i) {
+  return bf16_to_f32(reinterpret_cast<const uint16_t*>(p)[i]);
+}
+template <typename IO> __device__ __forceinline__ void st_io(void* p, long long i, float v);
+template <> __device__ __forceinline__ void st_io<float>(void* p, long long i, float v) {
+  reinterpret_cast<float*>(p)[i] = v;
+}
+template <> __device__ __forceinline__ void st_io<uint16_t>(void* p, long long i, float v) {
+  reinterpret_cast<uint16_t*>(p)[i] = f32_to_bf16(v);
+}
+
+// VEC: N == 16 and the state is 16-byte aligned (one float4 per lane).
+template <typename IO, bool VEC>
+__global__ void __launch_bounds__(256) decode_kernel(const DecodeArgs a) {
+  constexpr bool kPrecise = std::is_same<IO, float>::value;
+  const long long nch = (long long)a.batch * a.dim;
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const bool act = (gid >> 2) < nch;
+  const long long ch = act ? (gid >> 2) : nch - 1;  // idle lanes shadow a valid channel
+  const int q = (int)(gid & 3);
+  const int b = (int)(ch / a.dim), d = (int)(ch % a.dim);
+  const int N = a.N;
+
+  const float xv = ld_io<IO>(a.x, ch);
+  float v = ld_io<IO>(a.dt, ch) + (a.dt_bias ? a.dt_bias[d] : 0.f);
+  const float dt = !a.softplus ? v : (kPrecise ? softplus_precise(v) : softplus_fast(v));
+  const float dx = dt * xv;
+
+  float h[4], An[4], Bn[4], Cn[4];
+  float* sp = a.state + ch * N + 4 * q;
+  if (VEC) {
+    const float4 h4 = *reinterpret_cast<const float4*>(sp);
+    h[0] = h4.x; h[1] = h4.y; h[2] = h4.z; h[3] = h4.w;
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int n = 4 * q + i;
+    const bool live = n < N;
+    if (!VEC) h[i] = live ? sp[i] : 0.f;
+    An[i] = live ? a.A[(long long)d * N + n] : 0.f;
+    Bn[i] = live ? ld_io<IO>(a.B, (long long)b * N + n) : 0.f;
+    Cn[i] = live ? ld_io<IO>(a.C, (long long)b * N + n) : 0.f;
+  }
+  float y = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float abar = kPrecise ? expf(dt * An[i]) : ex2_mufu(dt * An[i] * kLog2e);
+    h[i] = fmaf(abar, h[i], dx * Bn[i]);
+    y = fmaf(Cn[i], h[i], y);
+  }
+  y += __shfl_xor_sync(0xffffffffu, y, 1);
+  y += __shfl_xor_sync(0xffffffffu, y, 2);
+  if (!act) return;
+  if (VEC) {
+    *reinterpret_cast<float4*>(sp) = make_float4(h[0], h[1], h[2], h[3]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (4 * q + i < N) sp[i] = h[i];
+  }
+  if (q == 0) {
+    y += (a.D ? a.D[d] : 0.f) * xv;
+    if (a.z) {
+      const float zv = ld_io<IO>(a.z, ch);
+      y *= zv * (kPrecise ? sigmoid_precise(zv) : sigmoid_fast(zv));
+    }
+    st_io<IO>(a.out, ch, y);
+  }
+}
+
+template <typename IO>
+cudaError_t launch_io(const DecodeArgs& a, cudaStream_t s) {
+  const long long threads = (long long)a.batch * a.dim * 4;
+  const int tpb = 256;
+  const unsigned grid = (unsigned)((threads + tpb - 1) / tpb);
+  const bool vec = a.N == kNS && (reinterpret_cast<uintptr_t>(a.state) & 15) == 0;
+  if (vec) decode_kernel<IO, true><<<grid, tpb, 0, s>>>(a);
+  else decode_kernel<IO, false><<<grid, tpb, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const DecodeArgs& a, int io, cudaStream_t s) {
+  return io == 1 ? launch_io<uint16_t>(a, s) : launch_io<float>(a, s);
+}
+
+}  // namespace ssm

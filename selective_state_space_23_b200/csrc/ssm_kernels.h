@@ -1,0 +1,93 @@
+// Internal launch interface between the C-ABI layer (ssm_api.cu) and the kernel files.
+// Not part of the public boundary; the public declarations are in include/ssm_scan.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ssm {
+
+constexpr int kBlk = 16;   // time steps per block: one scalar / state / output phase
+constexpr int kNS = 16;    // states held per lane (dstate <= 16, padded with zeros)
+
+// kFwdOut: gated output (+ optional checkpoints / final state); kFwdSummary: per-chunk end
+// state and ΣΔ from a zero state (time-split first pass); kFwdCkpt: state recurrence only,
+// writing the state entering every 16-step block (input of the backward pass).
+enum FwdMode { kFwdOut = 0, kFwdSummary = 1, kFwdCkpt = 2 };
+
+struct FwdArgs {
+  const void* u;
+  const void* delta;
+  const void* z;        // may be NULL (no gate)
+  const void* B;
+  const void* C;
+  const float* A;
+  const float* D;       // may be NULL
+  const float* dt_bias; // may be NULL
+  const float* h0;      // may be NULL (zero initial state)
+  void* out;
+  float* hL;            // may be NULL
+  float* ckpt;          // may be NULL; [batch][dim][ceil(L/16)][N]
+  float* summ;          // summary pass: per-chunk end state from zero [S][channels][16]
+  float* dsum;          // summary pass: per-chunk sum of Δ          [S][channels]
+  const float* hin;     // output pass with S > 1: state entering each chunk [S][channels][16]
+  int batch, dim, L, N;
+  int chunk_len;        // multiple of kBlk
+  int nchunk;           // S
+  int softplus;
+  int warps_per_b;      // ceil(dim / 32)
+  long long nwarps;     // batch * warps_per_b
+};
+
+struct BwdArgs {
+  const void* u;
+  const void* delta;
+  const void* z;
+  const void* B;
+  const void* C;
+  const float* A;
+  const float* D;
+  const float* dt_bias;
+  const void* dout;
+  const float* dhL;
+  const float* ckpt;    // [batch][dim][nblk][N]
+  void* du;
+  void* ddelta;
+  void* dz;
+  float* dh0;
+  float* part_bc;       // [ngroups][batch][2][16][L] per-CTA partial sums of dB, dC
+  float* part_adt;      // [batch][dim][16 + 2] per-channel partial dA, dD, ddt_bias
+  int batch, dim, L, N;
+  int softplus;
+  int warps_per_b;
+  long long nwarps;
+  int wpb;              // warps per CTA (channels per CTA = 32 * wpb)
+  int ngroups;          // CTAs per batch row = ceil(warps_per_b / wpb)
+};
+
+struct DecodeArgs {
+  float* state;
+  const void* x;
+  const void* dt;
+  const void* z;
+  const void* B;
+  const void* C;
+  const float* A;
+  const float* D;
+  const float* dt_bias;
+  void* out;
+  int batch, dim, N;
+  int softplus;
+};
+
+// io: 0 = f32, 1 = bf16.  vec: rows are 16-byte aligned and L is a multiple of the vector width.
+cudaError_t launch_fwd(const FwdArgs& a, int io, bool vec, int mode, int wpb, int kmufu,
+                       cudaStream_t s);
+cudaError_t launch_fwd_carry(const FwdArgs& a, const float* summ, const float* dsum, float* hin,
+                             cudaStream_t s);
+cudaError_t launch_bwd(const BwdArgs& a, int io, bool vec, cudaStream_t s);
+cudaError_t launch_bwd_finish(const BwdArgs& a, int io, void* dB, void* dC, float* dA, float* dD,
+                              float* ddt_bias, cudaStream_t s);
+cudaError_t launch_decode(const DecodeArgs& a, int io, cudaStream_t s);
+
+}  // namespace ssm

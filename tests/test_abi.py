@@ -1,0 +1,99 @@
+"""The C-ABI library loads and exports every entry point include/ssm_scan.h declares; host-only
+behaviour (status strings, workspace sizes, argument validation) works without a GPU."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from selective_state_space_23_b200 import _abi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ssm_scan.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"SSM_API\s+[\w\s\*]+?\b(ssm_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(_abi.LIB_PATH):
+        from selective_state_space_23_b200 import build
+        build.build()
+    return _abi.lib()
+
+
+def test_header_declares_the_entry_points():
+    syms = declared_symbols()
+    for s in ("ssm_scan_fwd", "ssm_scan_bwd", "ssm_state_update", "ssm_scan_fwd_workspace_size",
+              "ssm_scan_bwd_workspace_size", "ssm_status_string", "ssm_last_error", "ssm_version"):
+        assert s in syms
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", _abi.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (ssm_\w+)", out))
+    assert set(declared_symbols()) <= exported
+    for s in declared_symbols():
+        assert getattr(lib, s) is not None
+    assert set(_abi.SIGNATURES) == set(declared_symbols())
+
+
+def test_build_targets_sm100a_only():
+    from selective_state_space_23_b200 import build
+    assert build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def test_status_strings(lib):
+    assert lib.ssm_status_string(0) == b"ok"
+    assert lib.ssm_status_string(1) == b"invalid argument"
+    assert lib.ssm_status_string(4).startswith(b"workspace")
+    assert lib.ssm_status_string(99) == b"unknown status"
+    assert b"sm_100a" in lib.ssm_version()
+
+
+def test_workspace_sizes(lib):
+    # 370m-shaped layer: enough channels, no time split, no scratch
+    assert lib.ssm_scan_fwd_workspace_size(8, 2048, 2048, 16, 1) == 0
+    # a long sequence over few channels needs chunk summaries
+    assert lib.ssm_scan_fwd_workspace_size(1, 256, 1 << 20, 16, 1) > 0
+    assert lib.ssm_scan_fwd_workspace_size(0, 256, 1024, 16, 1) == 0     # invalid -> 0
+    with_ck = lib.ssm_scan_bwd_workspace_size(4, 5120, 2048, 16, 1, 1)
+    without = lib.ssm_scan_bwd_workspace_size(4, 5120, 2048, 16, 1, 0)
+    assert 0 < with_ck < without
+    assert without - with_ck >= 4 * 5120 * 128 * 16 * 4
+
+
+def _fwd(lib, **kw):
+    args = dict(u=None, delta=None, A=None, B=None, C=None, D=None, z=None, dt_bias=None, sp=1,
+                h0=None, hL=None, out=None, ckpt=None, ws=None, wsb=0, batch=1, dim=64, L=256,
+                N=16, io=1, stream=None)
+    args.update(kw)
+    return lib.ssm_scan_fwd(*args.values())
+
+
+def test_invalid_arguments_are_rejected_on_the_host(lib):
+    # nothing here reaches a kernel: every call fails validation before any launch
+    assert _fwd(lib) == _abi.SSM_EINVAL                       # NULL inputs
+    assert b"NULL" in lib.ssm_last_error()
+    assert _fwd(lib, batch=0) == _abi.SSM_EINVAL
+    assert _fwd(lib, io=7) == _abi.SSM_EINVAL
+    assert _fwd(lib, N=17) == _abi.SSM_EUNSUPPORTED
+    fake = ctypes.c_void_p(0x1001)                             # misaligned for bf16
+    assert _fwd(lib, u=fake) == _abi.SSM_EINVAL
+    assert b"aligned" in lib.ssm_last_error()
+    assert lib.ssm_state_update(*([None] * 9), 1, None, 1, 1, 16, 1, None) == _abi.SSM_EINVAL
+    rc = lib.ssm_scan_bwd(*([None] * 8), 1, *([None] * 14), 0, 1, 64, 256, 16, 1, None)
+    assert rc == _abi.SSM_EINVAL
+
+
+def test_host_pageable_pointer_is_rejected(lib):
+    """A pageable host buffer must be refused before any kernel could dereference it (on a
+    machine without a GPU the pointer query itself fails, which is refused the same way)."""
+    buf = (ctypes.c_uint16 * (64 * 256))()
+    p = ctypes.cast(buf, ctypes.c_void_p)
+    assert _fwd(lib, u=p, delta=p, A=p, B=p, C=p, out=p) == _abi.SSM_EINVAL
