@@ -142,6 +142,28 @@ SSM_API int ssm_scan_bwd(const void* u, const void* delta, const float* A, const
                  float* ddt_bias, float* dh0, void* workspace, size_t workspace_bytes,
                  int batch, int dim, int seqlen, int dstate, int io_dtype, void* stream);
 
+/* Size of the static scratch array used by ssm_scan_fwd_noalloc (8 MiB per GPU). */
+#define SSM_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/*
+ * ssm_scan_fwd without a workspace, for callers that cannot allocate device memory (a process
+ * that handed all device memory to its own pool at start-up, a plugin whose host application
+ * owns every allocation, or a hot path that must not call cudaMalloc because it can synchronise
+ * the device).  The pages have no counterpart: this is a deployment variant of the forward scan.
+ * Arguments, layouts, results and errors are those of ssm_scan_fwd, minus the workspace.  The
+ * time-split scratch comes from one static device array of SSM_NOALLOC_SCRATCH_BYTES that every
+ * GPU loading the library keeps until the process exits; shapes whose plan needs more return
+ * SSM_EUNSUPPORTED (ssm_last_error() says how much) and launch nothing.  No call allocates or
+ * frees memory.  The first call on each device looks up the array's device address with that
+ * device current; make that first call before any stream capture.  All calls on a device share
+ * the array: calls whose GPU work overlaps (other streams, other host threads) race on it.
+ */
+SSM_API int ssm_scan_fwd_noalloc(const void* u, const void* delta, const float* A, const void* B,
+                                 const void* C, const float* D, const void* z,
+                                 const float* dt_bias, int delta_softplus, const float* h0,
+                                 float* hL, void* out, float* ckpt, int batch, int dim,
+                                 int seqlen, int dstate, int io_dtype, void* stream);
+
 /*
  * One-token recurrent step ("Sorular": fixed D x N state per layer, O(1) per token).
  *   state     [batch][dim][dstate] f32    IN/OUT, updated in place: h <- exp(ΔA) h + Δ B x

@@ -12,6 +12,7 @@ SSM_F32, SSM_BF16 = 0, 1
 SSM_OK, SSM_EINVAL, SSM_EUNSUPPORTED, SSM_ECUDA, SSM_EWORKSPACE = 0, 1, 2, 3, 4
 CKPT_STEPS = 16
 MAX_DSTATE = 16
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
@@ -29,6 +30,8 @@ SIGNATURES = {
     "ssm_scan_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp,
                           _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                           _i, _i, _i, _i, _i, _vp]),
+    "ssm_scan_fwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp,
+                                  _i, _i, _i, _i, _i, _vp]),
     "ssm_state_update": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp,
                               _i, _i, _i, _i, _vp]),
 }

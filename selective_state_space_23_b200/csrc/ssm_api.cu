@@ -208,6 +208,12 @@ BwdLayout layout_bwd(int batch, int dim, int seqlen, int dstate, bool have_ckpt)
 
 }  // namespace
 
+namespace ssm {
+// Records a message for ssm_last_error() on the calling thread (used by entry points that live
+// in other translation units).
+void set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+}  // namespace ssm
+
 extern "C" {
 
 const char* ssm_status_string(int status) {

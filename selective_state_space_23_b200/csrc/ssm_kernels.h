@@ -90,4 +90,7 @@ cudaError_t launch_bwd_finish(const BwdArgs& a, int io, void* dB, void* dC, floa
                               float* ddt_bias, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, int io, cudaStream_t s);
 
+// Sets the message returned by ssm_last_error() on the calling thread.
+void set_last_error(const char* msg);
+
 }  // namespace ssm
