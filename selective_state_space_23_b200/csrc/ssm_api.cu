@@ -147,9 +147,19 @@ struct FwdPlan {
   size_t ws_bytes;
 };
 
+// Lanes per channel of the forward kernel: 1 (16 states per lane), 2 (8) or 4 (4).
+int fwd_lpc() {
+  const int v = env_int("SSM_FWD_LPC", 2);
+  return (v == 1 || v == 4) ? v : 2;
+}
+int fwd_warps_per_b(int dim) {
+  const int chw = 32 / fwd_lpc();
+  return (dim + chw - 1) / chw;
+}
+
 FwdPlan plan_fwd(int batch, int dim, int seqlen) {
   const int smsp = 4 * sm_count();
-  const long long warps = (long long)batch * ((dim + 31) / 32);
+  const long long warps = (long long)batch * fwd_warps_per_b(dim);
   const int nblk = (seqlen + ssm::kBlk - 1) / ssm::kBlk;
   int S = 1;
   const int forced = env_int("SSM_FWD_SPLIT", 0);
@@ -180,11 +190,14 @@ FwdPlan plan_fwd(int batch, int dim, int seqlen) {
   return p;
 }
 
+// Launch tuning of the forward kernel (measured on B200 for the 8 x 2048 x 2048 layer; the
+// environment variables override them for experiments): one warp per CTA, and 12 of every 16
+// exponentials per lane and step pair on the MUFU unit (the rest on the FMA-pipe polynomial).
 int fwd_wpb() {
-  const int w = env_int("SSM_FWD_WPB", 4);
-  return (w == 1 || w == 2 || w == 4) ? w : 4;
+  const int w = env_int("SSM_FWD_WPB", 1);
+  return (w == 1 || w == 2 || w == 4) ? w : 1;
 }
-int fwd_kmufu() { return env_int("SSM_FWD_KMUFU", 10); }
+int fwd_kmufu() { return env_int("SSM_FWD_KMUFU", 12); }
 
 struct BwdLayout {
   size_t ckpt, part_bc, part_adt, total;
@@ -278,7 +291,8 @@ int ssm_scan_fwd(const void* u, const void* delta, const float* A, const void* B
   a.batch = batch; a.dim = dim; a.L = seqlen; a.N = dstate;
   a.chunk_len = plan.chunk_len; a.nchunk = plan.nchunk;
   a.softplus = delta_softplus ? 1 : 0;
-  a.warps_per_b = (dim + 31) / 32;
+  a.lpc = fwd_lpc();
+  a.warps_per_b = fwd_warps_per_b(dim);
   a.nwarps = (long long)batch * a.warps_per_b;
   const bool vec = (seqlen * es) % 16 == 0 && aligned16(u) && aligned16(delta) && aligned16(z) &&
                    aligned16(out) && aligned16(B) && aligned16(C);
@@ -375,7 +389,8 @@ int ssm_scan_bwd(const void* u, const void* delta, const float* A, const void* B
     a.batch = batch; a.dim = dim; a.L = seqlen; a.N = dstate;
     a.chunk_len = (int)nblk * ssm::kBlk; a.nchunk = 1;
     a.softplus = delta_softplus ? 1 : 0;
-    a.warps_per_b = (dim + 31) / 32;
+    a.lpc = fwd_lpc();
+    a.warps_per_b = fwd_warps_per_b(dim);
     a.nwarps = (long long)batch * a.warps_per_b;
     if ((e = ssm::launch_fwd(a, io_dtype, vec, ssm::kFwdCkpt, fwd_wpb(), fwd_kmufu(), s)) != cudaSuccess)
       return cuda_fail(e, "backward state replay pass");

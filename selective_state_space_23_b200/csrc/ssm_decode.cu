@@ -7,10 +7,10 @@
 //   Δ = softplus(dt + dt_bias_d);  h_n <- exp(Δ A_dn) h_n + Δ B_n x   (in place)
 //   out = (Σ_n C_n h_n + D_d x) * silu(z)
 //
-// The step is bound by HBM traffic on the f32 state (read + write of batch*D*N*4 bytes).
-// Four lanes share a channel, each holding 4 consecutive states as one 128-bit load/store, so
-// a warp streams 512 contiguous bytes of state per access; the partial readouts are combined
-// with two butterfly shuffles.
+// The step is bound by HBM traffic on the f32 state (read + write of batch*D*N*4 bytes).  For
+// N = 16 two lanes share a channel, each holding 8 consecutive states as two 128-bit accesses
+// (a warp streams 1 KB of contiguous state per access pair); the two partial readouts are
+// combined with one shuffle.  Other N use four lanes of 4 states with per-element guards.
 #include <type_traits>
 
 #include "ssm_device.cuh"
@@ -93,14 +93,84 @@ __global__ void __launch_bounds__(256) decode_kernel(const DecodeArgs a) {
   }
 }
 
+// N == 16 with 16-byte aligned tensors: two lanes per channel, 8 states each, every access a
+// 128-bit load or store (state 2 x 16 B, A 2 x 16 B, B and C 16 B of bf16 or 2 x 16 B of f32).
+template <typename IO>
+__global__ void __launch_bounds__(256) decode16_kernel(const DecodeArgs a) {
+  constexpr bool kPrecise = std::is_same<IO, float>::value;
+  const long long nch = (long long)a.batch * a.dim;
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const bool act = (gid >> 1) < nch;
+  const long long ch = act ? (gid >> 1) : nch - 1;  // idle lanes shadow a valid channel
+  const int q = (int)(gid & 1);                      // states [8q, 8q + 8)
+  const int b = (int)(ch / a.dim), d = (int)(ch % a.dim);
+
+  const float xv = ld_io<IO>(a.x, ch);
+  const float v = ld_io<IO>(a.dt, ch) + (a.dt_bias ? a.dt_bias[d] : 0.f);
+  const float dt = !a.softplus ? v : (kPrecise ? softplus_precise(v) : softplus_fast(v));
+  const float dx = dt * xv;
+
+  float* sp = a.state + ch * kNS + 8 * q;
+  const float4 h0 = reinterpret_cast<const float4*>(sp)[0];  // default caching: the state is
+  const float4 h1 = reinterpret_cast<const float4*>(sp)[1];  // reused by the next step
+  const float4* ap = reinterpret_cast<const float4*>(a.A + (long long)d * kNS + 8 * q);
+  const float4 a0 = __ldg(ap), a1 = __ldg(ap + 1);
+  float h[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+  const float An[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+  float Bn[8], Cn[8];
+  if (sizeof(IO) == 2) {
+    const uint4 bw = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.B) + (long long)b * kNS + 8 * q));
+    const uint4 cw = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.C) + (long long)b * kNS + 8 * q));
+    const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w}, cc[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      Bn[2 * i] = bf16_lo(bb[i]); Bn[2 * i + 1] = bf16_hi(bb[i]);
+      Cn[2 * i] = bf16_lo(cc[i]); Cn[2 * i + 1] = bf16_hi(cc[i]);
+    }
+  } else {
+    const float4* bp = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.B) + (long long)b * kNS + 8 * q);
+    const float4* cp = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.C) + (long long)b * kNS + 8 * q);
+    const float4 b0 = __ldg(bp), b1 = __ldg(bp + 1), c0 = __ldg(cp), c1 = __ldg(cp + 1);
+    const float bt[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+    const float ct[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) { Bn[i] = bt[i]; Cn[i] = ct[i]; }
+  }
+  float y = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float abar = kPrecise ? expf(dt * An[i]) : ex2_mufu(dt * An[i] * kLog2e);
+    h[i] = fmaf(abar, h[i], dx * Bn[i]);
+    y = fmaf(Cn[i], h[i], y);
+  }
+  y += __shfl_xor_sync(0xffffffffu, y, 1);
+  if (!act) return;
+  reinterpret_cast<float4*>(sp)[0] = make_float4(h[0], h[1], h[2], h[3]);
+  reinterpret_cast<float4*>(sp)[1] = make_float4(h[4], h[5], h[6], h[7]);
+  if (q == 0) {
+    y += (a.D ? a.D[d] : 0.f) * xv;
+    if (a.z) {
+      const float zv = ld_io<IO>(a.z, ch);
+      y *= zv * (kPrecise ? sigmoid_precise(zv) : sigmoid_fast(zv));
+    }
+    st_io<IO>(a.out, ch, y);
+  }
+}
+
 template <typename IO>
 cudaError_t launch_io(const DecodeArgs& a, cudaStream_t s) {
-  const long long threads = (long long)a.batch * a.dim * 4;
   const int tpb = 256;
-  const unsigned grid = (unsigned)((threads + tpb - 1) / tpb);
-  const bool vec = a.N == kNS && (reinterpret_cast<uintptr_t>(a.state) & 15) == 0;
-  if (vec) decode_kernel<IO, true><<<grid, tpb, 0, s>>>(a);
-  else decode_kernel<IO, false><<<grid, tpb, 0, s>>>(a);
+  const auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+  if (a.N == kNS && al16(a.state) && al16(a.A) && al16(a.B) && al16(a.C)) {
+    const long long threads = (long long)a.batch * a.dim * 2;
+    decode16_kernel<IO><<<(unsigned)((threads + tpb - 1) / tpb), tpb, 0, s>>>(a);
+  } else {
+    const long long threads = (long long)a.batch * a.dim * 4;
+    const unsigned grid = (unsigned)((threads + tpb - 1) / tpb);
+    const bool vec = a.N == kNS && al16(a.state);
+    if (vec) decode_kernel<IO, true><<<grid, tpb, 0, s>>>(a);
+    else decode_kernel<IO, false><<<grid, tpb, 0, s>>>(a);
+  }
   return cudaGetLastError();
 }
 

@@ -67,20 +67,18 @@ constexpr float kQ3 = 0.009618110954761505f;
 // 1.5 * 2^23: adding it rounds |x| < 2^22 to an integer held in the low mantissa bits.
 constexpr float kRoundMagic = 12582912.0f;
 
-// Two lanes of 2^x, x <= 127 (the exponents of the scan are Δ*A*log2(e) <= 0 when A <= 0;
-// callers route channels with a positive A entry to the MUFU path).  x below -127 is clamped
-// there, where 2^x is below the smallest normal float and the flushed result is 0.
-__device__ __forceinline__ float2 exp2_fma_x2(float2 x) {
-  x.x = fmaxf(x.x, -127.f);
-  x.y = fmaxf(x.y, -127.f);
-  const float2 t = add2(x, f2(kRoundMagic));            // t = M + rint(x)
-  const float2 r = add2(t, f2(-kRoundMagic));           // rint(x), exact
-  const float2 f = fma2(r, f2(-1.f), x);                // x - rint(x), exact, |f| <= 1/2
+// Two lanes of 2^(d*a) for |d*a| <= 126 (no range checks: the caller guarantees the range).
+// The product d*a is folded into the range reduction: t = fma(d, a, M) rounds it to an integer,
+// f = fma(d, a, -rint) recovers the fraction exactly.
+__device__ __forceinline__ float2 exp2_fma_prod_x2(float2 d, float2 a) {
+  const float2 t = fma2(d, a, f2(kRoundMagic));         // t = M + rint(d*a)
+  const float2 r = add2(t, f2(-kRoundMagic));           // rint(d*a), exact
+  const float2 f = fma2(d, a, mul2(r, f2(-1.f)));       // d*a - rint(d*a), |f| <= 1/2
   float2 q = fma2(f2(kQ3), f, f2(kQ2));
   q = fma2(q, f, f2(kQ1));
   q = fma2(q, f, f2(kQ0));
   const float2 p = fma2(q, f, f2(1.f));                 // 2^f, p(0) == 1
-  // 2^i * p: add i to the exponent field.  The low bits of t's encoding are rint(x) offset by
+  // 2^i * p: add i to the exponent field.  The low bits of t's encoding are rint(d*a) offset by
   // a constant whose bits vanish when shifted left by 23.
   float2 out;
   out.x = __int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23));
@@ -106,9 +104,28 @@ __device__ __forceinline__ float softplus_precise(float v) {
   return v > 0.f ? v + log1pf(expf(-v)) : log1pf(expf(v));
 }
 
+// two lanes of softplus_fast (same arithmetic, packed f32x2 where it applies)
+__device__ __forceinline__ float2 softplus_fast_x2(float2 v) {
+  const float2 s = mul2(v, f2(kLog2e));
+  const float2 e = make_float2(ex2_mufu(s.x), ex2_mufu(s.y));
+  const float2 onep = add2(e, f2(1.f));
+  const float2 big = mul2(make_float2(lg2_mufu(onep.x), lg2_mufu(onep.y)), f2(kLn2));
+  float2 sm = fma2(e, f2(-0.25f), f2(0.33333334f));
+  sm = fma2(e, sm, f2(-0.5f));
+  sm = fma2(e, sm, f2(1.f));
+  sm = mul2(e, sm);
+  return make_float2(v.x > 15.f ? v.x : (e.x < 0.03125f ? sm.x : big.x),
+                     v.y > 15.f ? v.y : (e.y < 0.03125f ? sm.y : big.y));
+}
+
 // logistic sigmoid 1/(1+e^-z): MUFU ex2 + rcp (relative error ~1e-7 over the whole range;
 // tanh-based forms lose relative accuracy for negative z).
 __device__ __forceinline__ float sigmoid_fast(float z) { return rcp_mufu(1.f + ex2_mufu(-z * kLog2e)); }
 __device__ __forceinline__ float sigmoid_precise(float z) { return 1.f / (1.f + expf(-z)); }
+__device__ __forceinline__ float2 sigmoid_fast_x2(float2 z) {
+  const float2 s = mul2(z, f2(-kLog2e));
+  const float2 d = add2(make_float2(ex2_mufu(s.x), ex2_mufu(s.y)), f2(1.f));
+  return make_float2(rcp_mufu(d.x), rcp_mufu(d.y));
+}
 
 }  // namespace ssm

@@ -12,15 +12,20 @@
 //
 // B200 mapping ("Donanım Duyarlı Durum Genişletme": the expanded (B, L, D, N) state never
 // leaves the chip):
-//   * one lane owns one channel and its 16 states in registers; lanes of a warp are 32
-//     consecutive d of the same batch row b, so B_t and C_t are warp-uniform;
-//   * time advances in blocks of 16 steps: 128-bit streaming loads of u, delta, z for the
-//     NEXT block are issued before the current block is computed; each warp stages the
-//     block's B/C (16 x 16 each) in shared memory as f32 and reads them back as broadcast
-//     128-bit loads;
+//   * two lanes own one channel, 8 states each in registers; a warp holds 16 consecutive d of
+//     the same batch row b, so B_t and C_t are warp-uniform;
+//   * time advances in blocks of 16 steps.  Each lane streams its half of the block (8 steps of
+//     u, delta, z: one 128-bit load each for bf16) for the NEXT block before computing the
+//     current one; the warp stages the block's B/C (16 x 16 each) in shared memory as f32 and
+//     each half-lane reads its 8 states back as broadcast 128-bit loads;
+//   * per-step scalars (Δ_t, Δ_t x_t) are computed once per channel and step, by the lane that
+//     loaded that step, and exchanged through shared memory, as are the two half readouts;
+//     the time loop itself is a short two-step body (small code, so the instruction cache holds
+//     it while several warps per scheduler hide each other's latencies);
 //   * the per-element work (Δ*A, 2^x, Δ*x*B, state FMA, C readout) runs as packed f32x2
-//     instructions; the exponentials are split between the MUFU unit (states n < KM) and a
-//     range-reduced polynomial on the FMA pipe (n >= KM) so neither unit idles;
+//     instructions; the exponentials are split between the MUFU unit and a range-reduced
+//     polynomial on the FMA pipe (KE / KO of a lane's 4 state pairs on MUFU at even / odd steps)
+//     so neither unit idles;
 //   * few channels (long sequences): the time axis is split into S chunks.  A summary pass
 //     runs every chunk but the last from a zero state and records its end state and ΣΔ; a
 //     carry pass chains the chunk states h_in(j+1) = exp(A ΣΔ_j) h_in(j) + h_end(j) (the
@@ -34,284 +39,388 @@
 namespace ssm {
 namespace {
 
-template <typename IO> struct Row { uint4 v[sizeof(IO) * kBlk / 16]; };  // 16 steps of a channel
-template <typename IO> struct Seg { uint4 v[sizeof(IO) * 8 / 16]; };     // 8 steps of a B/C row
+// E consecutive elements of one row, held as 32-bit words.
+template <typename IO, int E>
+struct Row {
+  static constexpr int kWords = E * (int)sizeof(IO) / 4;
+  uint32_t w[kWords];
+  __device__ __forceinline__ float get(int k) const {
+    if (sizeof(IO) == 4) return __uint_as_float(w[k]);
+    const uint32_t x = w[k >> 1];
+    return (k & 1) ? bf16_hi(x) : bf16_lo(x);
+  }
+  __device__ __forceinline__ void zero() {
+#pragma unroll
+    for (int i = 0; i < kWords; ++i) w[i] = 0u;
+  }
+};
 
-__device__ __forceinline__ uint32_t word(const uint4& q, int j) {
-  return j == 0 ? q.x : j == 1 ? q.y : j == 2 ? q.z : q.w;
-}
-template <typename IO> __device__ __forceinline__ float elem(const uint4* v, int k);
-template <> __device__ __forceinline__ float elem<float>(const uint4* v, int k) {
-  return __uint_as_float(word(v[k >> 2], k & 3));
-}
-template <> __device__ __forceinline__ float elem<uint16_t>(const uint4* v, int k) {
-  const uint32_t w = word(v[k >> 3], (k >> 1) & 3);
-  return (k & 1) ? bf16_hi(w) : bf16_lo(w);
-}
-
-// Load E = NV*16/sizeof(IO) consecutive elements starting at p; elements at or beyond nvalid
-// read as zero.  VEC: p is 16-byte aligned and all E elements are in bounds.
-template <typename IO, bool VEC, int NV>
-__device__ __forceinline__ void load_elems(uint4 (&v)[NV], const IO* p, int nvalid) {
+// Load E consecutive elements at p; elements at or beyond nvalid read as zero.  VEC: p is aligned
+// to E*sizeof(IO) bytes (8, 16 or 32) and all E elements are in bounds.
+template <typename IO, int E, bool VEC>
+__device__ __forceinline__ void load_row(Row<IO, E>& r, const IO* p, int nvalid) {
+  constexpr int B = E * (int)sizeof(IO);
   if (VEC) {
-    const uint4* q = reinterpret_cast<const uint4*>(p);
+    if constexpr (B == 8) {
+      const uint2 v = __ldcs(reinterpret_cast<const uint2*>(p));
+      r.w[0] = v.x;
+      r.w[1] = v.y;
+    } else {
 #pragma unroll
-    for (int i = 0; i < NV; ++i) v[i] = __ldcs(q + i);
+      for (int i = 0; i < B / 16; ++i) {
+        const uint4 v = __ldcs(reinterpret_cast<const uint4*>(p) + i);
+        r.w[4 * i] = v.x; r.w[4 * i + 1] = v.y; r.w[4 * i + 2] = v.z; r.w[4 * i + 3] = v.w;
+      }
+    }
   } else {
-    constexpr int E = NV * 16 / (int)sizeof(IO);
-    uint32_t w[NV * 4];
-#pragma unroll
-    for (int i = 0; i < NV * 4; ++i) w[i] = 0u;
+    r.zero();
     if (sizeof(IO) == 4) {
       const uint32_t* s = reinterpret_cast<const uint32_t*>(p);
 #pragma unroll
       for (int e = 0; e < E; ++e)
-        if (e < nvalid) w[e] = __ldcs(s + e);
+        if (e < nvalid) r.w[e] = __ldcs(s + e);
     } else {
       const unsigned short* s = reinterpret_cast<const unsigned short*>(p);
 #pragma unroll
       for (int e = 0; e < E; ++e)
-        if (e < nvalid) w[e >> 1] |= ((uint32_t)__ldcs(s + e)) << (16 * (e & 1));
+        if (e < nvalid) r.w[e >> 1] |= ((uint32_t)__ldcs(s + e)) << (16 * (e & 1));
     }
-#pragma unroll
-    for (int i = 0; i < NV; ++i) v[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
   }
 }
 
-template <typename IO, bool VEC>
-__device__ __forceinline__ void store_row(IO* p, const float (&o)[kBlk], int nvalid) {
+template <typename IO, int E, bool VEC>
+__device__ __forceinline__ void store_row(IO* p, const float (&o)[E], int nvalid) {
+  constexpr int B = E * (int)sizeof(IO);
+  uint32_t w[B / 4];
   if (sizeof(IO) == 2) {
-    uint32_t w[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(o[2 * i], o[2 * i + 1]);
-    if (VEC) {
-      uint4* q = reinterpret_cast<uint4*>(p);
-      __stcs(q, make_uint4(w[0], w[1], w[2], w[3]));
-      __stcs(q + 1, make_uint4(w[4], w[5], w[6], w[7]));
+    for (int i = 0; i < E / 2; ++i) w[i] = pack_bf16x2(o[2 * i], o[2 * i + 1]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < E; ++i) w[i] = __float_as_uint(o[i]);
+  }
+  if (VEC) {
+    if constexpr (B == 8) {
+      __stcs(reinterpret_cast<uint2*>(p), make_uint2(w[0], w[1]));
     } else {
-      unsigned short* s = reinterpret_cast<unsigned short*>(p);
 #pragma unroll
-      for (int e = 0; e < kBlk; ++e)
-        if (e < nvalid) s[e] = (unsigned short)(w[e >> 1] >> (16 * (e & 1)));
+      for (int i = 0; i < B / 16; ++i)
+        __stcs(reinterpret_cast<uint4*>(p) + i, make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]));
     }
+  } else if (sizeof(IO) == 2) {
+    unsigned short* s = reinterpret_cast<unsigned short*>(p);
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+      if (e < nvalid) s[e] = (unsigned short)(w[e >> 1] >> (16 * (e & 1)));
   } else {
     float* s = reinterpret_cast<float*>(p);
-    if (VEC) {
-      float4* q = reinterpret_cast<float4*>(p);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) __stcs(q + i, make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]));
-    } else {
-#pragma unroll
-      for (int e = 0; e < kBlk; ++e)
-        if (e < nvalid) s[e] = o[e];
-    }
+    for (int e = 0; e < E; ++e)
+      if (e < nvalid) s[e] = o[e];
   }
 }
 
-// One lane's scan over one time chunk.
-template <typename IO, bool VEC, int MODE, int KM>
-struct ChunkScan {
-  static constexpr bool kPrecise = std::is_same<IO, float>::value;
-  float2 al[8];   // A_dn * log2(e) (fast path) or A_dn (precise path); zero for n >= N
-  float2 hh[8];   // state
-  float Dd, bias;
-  int softplus;
-
-  __device__ __forceinline__ float step_size(float v) const {
-    if (!softplus) return v;
-    return kPrecise ? softplus_precise(v) : softplus_fast(v);
-  }
-
-  // One 16-step block.  FULL: all 16 steps valid (no per-step bound checks).
-  template <bool FULL>
-  __device__ __forceinline__ void block(const Row<IO>& cu, const Row<IO>& cd, int nvalid,
-                                        const float* sB, const float* sC, float (&yv)[kBlk],
-                                        float& dsum_blk) {
-    float dl[kBlk], du[kBlk], ux[kBlk];
-#pragma unroll
-    for (int k = 0; k < kBlk; ++k) {
-      ux[k] = elem<IO>(cu.v, k);
-      dl[k] = step_size(elem<IO>(cd.v, k) + bias);
-      du[k] = dl[k] * ux[k];
-    }
-    if (MODE == kFwdSummary) {
-      float s = 0.f;
-#pragma unroll
-      for (int k = 0; k < kBlk; ++k) s += (FULL || k < nvalid) ? dl[k] : 0.f;
-      dsum_blk = s;
-    }
-#pragma unroll
-    for (int k = 0; k < kBlk; ++k) {
-      if (!FULL && k >= nvalid) break;
-      const float2 d2 = f2(dl[k]);
-      const float2 du2 = f2(du[k]);
-      float2 y2 = make_float2(Dd * ux[k], 0.f);
-      const float4* b4p = reinterpret_cast<const float4*>(sB + k * kNS);
-      const float4* c4p = reinterpret_cast<const float4*>(sC + k * kNS);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float4 b4 = b4p[q];
-        float4 c4;
-        if (MODE == kFwdOut) c4 = c4p[q];
-#pragma unroll
-        for (int s = 0; s < 2; ++s) {
-          const int j = 2 * q + s;
-          const float2 bp = s == 0 ? make_float2(b4.x, b4.y) : make_float2(b4.z, b4.w);
-          float2 av;
-          if (kPrecise) {
-            av.x = expf(dl[k] * al[j].x);
-            av.y = expf(dl[k] * al[j].y);
-          } else {
-            const float2 x = mul2(d2, al[j]);
-            if (2 * j < KM) {
-              av.x = ex2_mufu(x.x);
-              av.y = ex2_mufu(x.y);
-            } else {
-              av = exp2_fma_x2(x);
-            }
-          }
-          hh[j] = fma2(av, hh[j], mul2(du2, bp));
-          if (MODE == kFwdOut) {
-            const float2 cp = s == 0 ? make_float2(c4.x, c4.y) : make_float2(c4.z, c4.w);
-            y2 = fma2(cp, hh[j], y2);
-          }
-        }
-      }
-      yv[k] = y2.x + y2.y;
-    }
-  }
+// Lane layout: LPC lanes (1, 2 or 4) share one channel; lane q of a channel holds states [SPL q, SPL q + SPL)
+// and owns steps [SPL q, SPL q + SPL) of every 16-step block (it loads their u, delta, z,
+// computes their Δ and writes their output).
+template <int LPC>
+struct Layout {
+  static constexpr int kSPL = kNS / LPC;       // states (and owned steps) per lane
+  static constexpr int kPPL = kSPL / 2;        // state pairs per lane
+  static constexpr int kChW = 32 / LPC;        // channels per warp
+  static constexpr int kSdStride = kChW + 1;   // entries per step in the (Δ, Δ, Δx, Δx) table
+  // floats per step in the partial-readout table: a multiple of LPC (aligned vector reads of a
+  // channel's LPC partials) chosen so that the owners' reads of different steps spread over banks
+  static constexpr int kYpStride = LPC == 1 ? 33 : (LPC == 2 ? 34 : 36);
 };
 
-template <typename IO, bool VEC, int MODE, int KM>
-__device__ __forceinline__ void run_chunk(const FwdArgs& a, ChunkScan<IO, VEC, MODE, KM>& cs,
-                                          int lane, int b, bool act, long long ch, int t_begin,
-                                          int t_end, bool last_chunk, float* sB, float* sC) {
-  const int L = a.L, N = a.N;
-  const IO* up = reinterpret_cast<const IO*>(a.u) + ch * (long long)L;
-  const IO* dp = reinterpret_cast<const IO*>(a.delta) + ch * (long long)L;
-  const IO* zp = a.z ? reinterpret_cast<const IO*>(a.z) + ch * (long long)L : nullptr;
-  IO* op = MODE == kFwdOut ? reinterpret_cast<IO*>(a.out) + ch * (long long)L : nullptr;
-  const int bc_n = lane >> 1, bc_half = lane & 1;
-  const bool bc_live = bc_n < N;
-  const IO* Bp = reinterpret_cast<const IO*>(a.B) + ((long long)b * N + (bc_live ? bc_n : 0)) * L;
-  const IO* Cp = reinterpret_cast<const IO*>(a.C) + ((long long)b * N + (bc_live ? bc_n : 0)) * L;
-  const int nblk_total = (L + kBlk - 1) / kBlk;
+// Per-warp shared memory of one 16-step block.
+template <int LPC>
+struct WarpTile {
+  float4 sB[kBlk * kNS / 4];                          // B_t,n as f32 [step][state]
+  float4 sC[kBlk * kNS / 4];                          // C_t,n
+  float4 sd[kBlk * Layout<LPC>::kSdStride];           // (Δ_t, Δ_t, Δ_t x_t, Δ_t x_t) per [step][slot]
+  float yp[kBlk * Layout<LPC>::kYpStride];            // partial readouts per [step][slot][lane]
+};
 
-  Row<IO> nu, nd, nz;
-  Seg<IO> nb, nc;
-  auto fetch = [&](int tb) {
-    const int nv = min(kBlk, t_end - tb);
-    const int nv8 = max(0, min(8, t_end - tb - 8 * bc_half));
-    if (VEC && nv == kBlk) {
-      load_elems<IO, true>(nu.v, up + tb, kBlk);
-      load_elems<IO, true>(nd.v, dp + tb, kBlk);
-      if (MODE == kFwdOut && zp) load_elems<IO, true>(nz.v, zp + tb, kBlk);
-      if (bc_live) {
-        load_elems<IO, true>(nb.v, Bp + tb + 8 * bc_half, 8);
-        if (MODE == kFwdOut) load_elems<IO, true>(nc.v, Cp + tb + 8 * bc_half, 8);
-      }
+// Per-step quantities of one lane that do not depend on the state: Ā = 2^(Δ A log2 e) and the
+// input term Δ x B.  They are computed one step ahead of the state update (the only
+// loop-carried dependency), which keeps MUFU and shared-memory latency off the critical path.
+template <int PPL>
+struct StepPrep {
+  float2 av[PPL];
+  float2 bu[PPL];
+};
+
+template <int PPL>
+__device__ __forceinline__ float4 quad(const float4* q, int i) { return q[i]; }
+
+// KP of the lane's PPL state pairs take 2^x from the MUFU unit, the others from the FMA-pipe
+// polynomial, which has no range checks: it is used only in blocks where every step satisfies
+// |Δ| max_n |A_n log2 e| <= 126 (checked once per block by a warp vote).
+template <bool PRECISE, int PPL, int KP>
+__device__ __forceinline__ void prepare_step(StepPrep<PPL>& p, const float2 (&al)[PPL], float4 dd,
+                                             const float4* bq) {
+  const float2 d2 = make_float2(dd.x, dd.y), du2 = make_float2(dd.z, dd.w);  // already paired
+  float4 bv[PPL / 2];
+#pragma unroll
+  for (int i = 0; i < PPL / 2; ++i) bv[i] = bq[i];
+#pragma unroll
+  for (int j = 0; j < PPL; ++j) {
+    const float4 bb = bv[j >> 1];
+    const float2 bp = (j & 1) ? make_float2(bb.z, bb.w) : make_float2(bb.x, bb.y);
+    if (PRECISE) {
+      p.av[j] = make_float2(expf(dd.x * al[j].x), expf(dd.x * al[j].y));
+    } else if (j < KP) {
+      const float2 x = mul2(d2, al[j]);
+      p.av[j] = make_float2(ex2_mufu(x.x), ex2_mufu(x.y));
     } else {
-      load_elems<IO, false>(nu.v, up + tb, nv);
-      load_elems<IO, false>(nd.v, dp + tb, nv);
-      if (MODE == kFwdOut && zp) load_elems<IO, false>(nz.v, zp + tb, nv);
-      if (bc_live) {
-        load_elems<IO, false>(nb.v, Bp + tb + 8 * bc_half, nv8);
-        if (MODE == kFwdOut) load_elems<IO, false>(nc.v, Cp + tb + 8 * bc_half, nv8);
-      }
+      p.av[j] = exp2_fma_prod_x2(d2, al[j]);  // block checked: |Δ A log2 e| <= 126
+    }
+    p.bu[j] = mul2(du2, bp);
+  }
+}
+
+// h <- Ā h + Δ x B for the lane's states; returns the partial readout Σ C h.
+template <bool READOUT, int PPL>
+__device__ __forceinline__ float consume_step(float2 (&hh)[PPL], const StepPrep<PPL>& p,
+                                              const float4* cq) {
+  float4 cv[PPL / 2];
+#pragma unroll
+  for (int i = 0; i < PPL / 2; ++i) cv[i] = READOUT ? cq[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+  float2 ya = make_float2(0.f, 0.f), yb = ya;
+#pragma unroll
+  for (int j = 0; j < PPL; ++j) {
+    hh[j] = fma2(p.av[j], hh[j], p.bu[j]);
+    if (READOUT) {
+      const float4 cc = cv[j >> 1];
+      const float2 cp = (j & 1) ? make_float2(cc.z, cc.w) : make_float2(cc.x, cc.y);
+      if (j & 1) yb = fma2(cp, hh[j], yb);
+      else ya = fma2(cp, hh[j], ya);
+    }
+  }
+  const float2 ys = add2(ya, yb);
+  return ys.x + ys.y;
+}
+
+// The 16-step time loop of one block, software-pipelined by one step: step k+1 is prepared while
+// step k updates the state.  A step at or beyond nvalid may be prepared from stale tile entries
+// (the index is clamped to the tile) but is never consumed.
+template <bool kPrecise, bool kReadout, int LPC, int KE, int KO>
+__device__ __forceinline__ void state_loop(WarpTile<LPC>& tile, float2 (&hh)[Layout<LPC>::kPPL],
+                                           const float2 (&al)[Layout<LPC>::kPPL], int slot, int q,
+                                           int nvalid) {
+  using Lay = Layout<LPC>;
+  constexpr int SPL = Lay::kSPL, PPL = Lay::kPPL;
+  const float4* bq = tile.sB + SPL * q / 4;
+  const float4* cq = tile.sC + SPL * q / 4;
+  const float4* sdp = tile.sd + slot;
+  float* yp = tile.yp + slot * LPC + q;
+  StepPrep<PPL> p0, p1;
+  prepare_step<kPrecise, PPL, KE>(p0, al, sdp[0], bq);
+  int k = 0;
+#pragma unroll 1
+  for (; k + 2 <= nvalid; k += 2) {
+    prepare_step<kPrecise, PPL, KO>(p1, al, sdp[(k + 1) * Lay::kSdStride], bq + (k + 1) * 4);
+    const float y0 = consume_step<kReadout, PPL>(hh, p0, cq + k * 4);
+    const int k2 = min(k + 2, kBlk - 1);
+    prepare_step<kPrecise, PPL, KE>(p0, al, sdp[k2 * Lay::kSdStride], bq + k2 * 4);
+    const float y1 = consume_step<kReadout, PPL>(hh, p1, cq + (k + 1) * 4);
+    if (kReadout) {
+      yp[k * Lay::kYpStride] = y0;
+      yp[(k + 1) * Lay::kYpStride] = y1;
+    }
+  }
+  if (k < nvalid) {  // odd number of valid steps: the last one was prepared into p0
+    const float y0 = consume_step<kReadout, PPL>(hh, p0, cq + k * 4);
+    if (kReadout) yp[k * Lay::kYpStride] = y0;
+  }
+}
+
+// Scan of one time chunk by one lane.  KE / KO: MUFU pairs on even / odd steps (the same for every
+// lane, so the lanes of a channel run identical instructions).
+template <typename IO, bool VEC, int MODE, int LPC, int KE, int KO>
+__device__ __forceinline__ void run_chunk(const FwdArgs& a, WarpTile<LPC>& tile,
+                                          float2 (&hh)[Layout<LPC>::kPPL],
+                                          const float2 (&al)[Layout<LPC>::kPPL], float Dd,
+                                          float bias, int lane, int slot, int q, int b, bool act,
+                                          long long ch, int t_begin, int t_end, bool last_chunk) {
+  using Lay = Layout<LPC>;
+  constexpr int SPL = Lay::kSPL, PPL = Lay::kPPL;
+  constexpr bool kPrecise = std::is_same<IO, float>::value;
+  constexpr bool kReadout = MODE == kFwdOut;
+  const int L = a.L, N = a.N;
+  const long long row = ch * (long long)L + SPL * q;     // this lane's steps of each block
+  const IO* up = reinterpret_cast<const IO*>(a.u) + row;
+  const IO* dp = reinterpret_cast<const IO*>(a.delta) + row;
+  const IO* zp = (kReadout && a.z) ? reinterpret_cast<const IO*>(a.z) + row : nullptr;
+  IO* op = kReadout ? reinterpret_cast<IO*>(a.out) + row : nullptr;
+  // B/C staging: lane stages state row bn, steps [8 bh, 8 bh + 8) of each block
+  const int bn = lane >> 1, bh = lane & 1;
+  const bool bc_live = bn < N;
+  const long long bcrow = ((long long)b * N + (bc_live ? bn : 0)) * L + 8 * bh;
+  const IO* Bp = reinterpret_cast<const IO*>(a.B) + bcrow;
+  const IO* Cp = reinterpret_cast<const IO*>(a.C) + bcrow;
+  const int nblk_total = (L + kBlk - 1) / kBlk;
+  float* sBw = reinterpret_cast<float*>(tile.sB);
+  float* sCw = reinterpret_cast<float*>(tile.sC);
+
+  Row<IO, SPL> nu, nd, nz;
+  Row<IO, 8> nb, nc;
+  auto fetch = [&](int tb) {
+    const int nv = max(0, min(SPL, t_end - tb - SPL * q));
+    const int nv8 = max(0, min(8, t_end - tb - 8 * bh));
+    if (VEC && nv == SPL) {
+      load_row<IO, SPL, true>(nu, up + tb, SPL);
+      load_row<IO, SPL, true>(nd, dp + tb, SPL);
+      if (zp) load_row<IO, SPL, true>(nz, zp + tb, SPL);
+    } else {
+      load_row<IO, SPL, false>(nu, up + tb, nv);
+      load_row<IO, SPL, false>(nd, dp + tb, nv);
+      if (zp) load_row<IO, SPL, false>(nz, zp + tb, nv);
     }
     if (!bc_live) {
-#pragma unroll
-      for (int i = 0; i < (int)(sizeof(nb.v) / 16); ++i) nb.v[i] = nc.v[i] = make_uint4(0, 0, 0, 0);
+      nb.zero();
+      nc.zero();
+    } else if (VEC && nv8 == 8) {
+      load_row<IO, 8, true>(nb, Bp + tb, 8);
+      if (kReadout) load_row<IO, 8, true>(nc, Cp + tb, 8);
+    } else {
+      load_row<IO, 8, false>(nb, Bp + tb, nv8);
+      if (kReadout) load_row<IO, 8, false>(nc, Cp + tb, nv8);
     }
   };
 
+  // largest |A log2 e| of the warp's states: the FMA-pipe exponential needs |Δ A log2 e| <= 126
+  float amax = 0.f;
+#pragma unroll
+  for (int j = 0; j < PPL; ++j) amax = fmaxf(amax, fmaxf(fabsf(al[j].x), fabsf(al[j].y)));
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
+
   fetch(t_begin);
-  float dsum = 0.f, dcomp = 0.f;  // Kahan-compensated ΣΔ over the chunk (summary pass)
+  float dsum = 0.f, dcomp = 0.f;  // Kahan-compensated ΣΔ of this lane's steps (summary pass)
   for (int t0 = t_begin; t0 < t_end; t0 += kBlk) {
     const int nvalid = min(kBlk, t_end - t0);
-    const Row<IO> cu = nu, cd = nd, cz = nz;
-    const Seg<IO> cb = nb, cc = nc;
+    const int nown = max(0, min(SPL, nvalid - SPL * q));
+    const Row<IO, SPL> cu = nu, cd = nd, cz = nz;
+    const Row<IO, 8> cb = nb, cc = nc;
     if (t0 + kBlk < t_end) fetch(t0 + kBlk);
 
-    // stage this block's B (and C) rows as f32 [step][state]
-    __syncwarp();
+    __syncwarp();  // the previous block's tile is no longer read
+    // stage B/C as f32 [step][state]
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      sB[(8 * bc_half + j) * kNS + bc_n] = elem<IO>(cb.v, j);
-      if (MODE == kFwdOut) sC[(8 * bc_half + j) * kNS + bc_n] = elem<IO>(cc.v, j);
+      sBw[(8 * bh + j) * kNS + bn] = cb.get(j);
+      if (kReadout) sCw[(8 * bh + j) * kNS + bn] = cc.get(j);
+    }
+    float dblk = 0.f, dabs = 0.f;  // dabs: largest |Δ| of this lane's steps (NaN propagates)
+#pragma unroll
+    for (int j = 0; j < SPL; j += 2) {
+      const float2 v = add2(make_float2(cd.get(j), cd.get(j + 1)), f2(bias));
+      float2 dl = v;
+      if (a.softplus) {
+        if (kPrecise) dl = make_float2(softplus_precise(v.x), softplus_precise(v.y));
+        else dl = softplus_fast_x2(v);
+      }
+      const float2 dx = mul2(dl, make_float2(cu.get(j), cu.get(j + 1)));
+      tile.sd[(SPL * q + j) * Lay::kSdStride + slot] = make_float4(dl.x, dl.x, dx.x, dx.x);
+      tile.sd[(SPL * q + j + 1) * Lay::kSdStride + slot] = make_float4(dl.y, dl.y, dx.y, dx.y);
+      dblk += (j < nown ? dl.x : 0.f) + (j + 1 < nown ? dl.y : 0.f);
+      dabs = fmaxf(dabs, fmaxf(fabsf(dl.x), fabsf(dl.y)));
+      if (dl.x != dl.x || dl.y != dl.y) dabs = __int_as_float(0x7f800000);  // NaN: take the checked path
+    }
+    if (MODE != kFwdSummary && a.ckpt && act) {
+      float* cp = a.ckpt + (ch * nblk_total + t0 / kBlk) * N;
+#pragma unroll
+      for (int j = 0; j < PPL; ++j) {
+        const int n0 = SPL * q + 2 * j;
+        if (n0 < N) cp[n0] = hh[j].x;
+        if (n0 + 1 < N) cp[n0 + 1] = hh[j].y;
+      }
     }
     __syncwarp();
 
-    if (MODE != kFwdSummary && a.ckpt && act) {
-      float* cp = a.ckpt + (ch * nblk_total + t0 / kBlk) * N;
-      if (N == kNS && ((reinterpret_cast<uintptr_t>(a.ckpt) & 15) == 0)) {
-        float4* c4 = reinterpret_cast<float4*>(cp);
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          c4[q] = make_float4(cs.hh[2 * q].x, cs.hh[2 * q].y, cs.hh[2 * q + 1].x, cs.hh[2 * q + 1].y);
-      } else {
-#pragma unroll
-        for (int n = 0; n < kNS; ++n)
-          if (n < N) cp[n] = (n & 1) ? cs.hh[n >> 1].y : cs.hh[n >> 1].x;
-      }
-    }
+    const bool safe = !__any_sync(0xffffffffu, !(amax * dabs <= 126.f));
+    if (kPrecise || !safe)
+      state_loop<kPrecise, kReadout, LPC, PPL, PPL>(tile, hh, al, slot, q, nvalid);
+    else
+      state_loop<kPrecise, kReadout, LPC, KE, KO>(tile, hh, al, slot, q, nvalid);
 
-    float yv[kBlk];
-    float dblk = 0.f;
-    if (nvalid == kBlk) cs.template block<true>(cu, cd, nvalid, sB, sC, yv, dblk);
-    else cs.template block<false>(cu, cd, nvalid, sB, sC, yv, dblk);
-
-    if (MODE == kFwdCkpt) {
-      // state recurrence only
-    } else if (MODE == kFwdSummary) {
+    if (MODE == kFwdSummary) {
       const float yk = dblk - dcomp;
       const float tk = dsum + yk;
       dcomp = (tk - dsum) - yk;
       dsum = tk;
-    } else {
-      float o[kBlk];
+    } else if (kReadout) {
+      __syncwarp();
+      float o[SPL];
 #pragma unroll
-      for (int k = 0; k < kBlk; ++k) {
-        float y = yv[k];
-        if (zp) {
-          const float zk = elem<IO>(cz.v, k);
-          y *= zk * (ChunkScan<IO, VEC, MODE, KM>::kPrecise ? sigmoid_precise(zk) : sigmoid_fast(zk));
+      for (int j = 0; j < SPL; j += 2) {
+        float yv[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const float* pp = tile.yp + (SPL * q + j + i) * Lay::kYpStride + slot * LPC;
+          if (LPC == 1) {
+            yv[i] = *pp;
+          } else if (LPC == 2) {
+            const float2 v = *reinterpret_cast<const float2*>(pp);
+            yv[i] = v.x + v.y;
+          } else {
+            const float4 v = *reinterpret_cast<const float4*>(pp);
+            yv[i] = (v.x + v.y) + (v.z + v.w);
+          }
         }
-        o[k] = y;
+        float2 y = fma2(f2(Dd), make_float2(cu.get(j), cu.get(j + 1)), make_float2(yv[0], yv[1]));
+        if (zp) {
+          const float2 z2 = make_float2(cz.get(j), cz.get(j + 1));
+          const float2 sg = kPrecise ? make_float2(sigmoid_precise(z2.x), sigmoid_precise(z2.y))
+                                     : sigmoid_fast_x2(z2);
+          y = mul2(y, mul2(z2, sg));
+        }
+        o[j] = y.x;
+        o[j + 1] = y.y;
       }
-      if (act) {
-        if (VEC && nvalid == kBlk) store_row<IO, true>(op + t0, o, kBlk);
-        else store_row<IO, false>(op + t0, o, nvalid);
+      if (act && nown > 0) {
+        if (VEC && nown == SPL) store_row<IO, SPL, true>(op + t0, o, SPL);
+        else store_row<IO, SPL, false>(op + t0, o, nown);
       }
     }
   }
 
-  if (!act) return;
   if (MODE == kFwdSummary) {
-    const int chunk = blockIdx.y;
-    float* sp = a.summ + ((long long)chunk * a.batch * a.dim + ch) * kNS;
+    float total = dsum;
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      reinterpret_cast<float4*>(sp)[q] =
-          make_float4(cs.hh[2 * q].x, cs.hh[2 * q].y, cs.hh[2 * q + 1].x, cs.hh[2 * q + 1].y);
-    a.dsum[(long long)chunk * a.batch * a.dim + ch] = dsum;
-  } else if (last_chunk && a.hL) {
+    for (int m = 1; m < LPC; m <<= 1) total += __shfl_xor_sync(0xffffffffu, total, m);
+    if (!act) return;
+    const int chunk = blockIdx.y;
+    float* sp = a.summ + ((long long)chunk * a.batch * a.dim + ch) * kNS + SPL * q;
+#pragma unroll
+    for (int j = 0; j < PPL; ++j) reinterpret_cast<float2*>(sp)[j] = hh[j];
+    if (q == 0) a.dsum[(long long)chunk * a.batch * a.dim + ch] = total;
+  } else if (last_chunk && a.hL && act) {
     float* hp = a.hL + ch * N;
 #pragma unroll
-    for (int n = 0; n < kNS; ++n)
-      if (n < N) hp[n] = (n & 1) ? cs.hh[n >> 1].y : cs.hh[n >> 1].x;
+    for (int j = 0; j < PPL; ++j) {
+      const int n0 = SPL * q + 2 * j;
+      if (n0 < N) hp[n0] = hh[j].x;
+      if (n0 + 1 < N) hp[n0 + 1] = hh[j].y;
+    }
   }
 }
 
-template <typename IO, bool VEC, int MODE, int KM>
-__global__ void __launch_bounds__(128, 1) fwd_kernel(const FwdArgs a) {
+template <typename IO, bool VEC, int MODE, int LPC, int KE, int KO>
+__global__ void __launch_bounds__(128) fwd_kernel(const FwdArgs a) {
+  using Lay = Layout<LPC>;
+  constexpr int SPL = Lay::kSPL, PPL = Lay::kPPL;
   extern __shared__ float4 smem4[];
-  float* smem = reinterpret_cast<float*>(smem4);
+  WarpTile<LPC>* tiles = reinterpret_cast<WarpTile<LPC>*>(smem4);
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const long long w = (long long)blockIdx.x * (blockDim.x >> 5) + wib;
   if (w >= a.nwarps) return;  // whole warp leaves together
+  const int slot = lane / LPC, q = lane % LPC;
   const int b = (int)(w / a.warps_per_b);
-  const int d = (int)(w % a.warps_per_b) * 32 + lane;
+  const int d = (int)(w % a.warps_per_b) * Lay::kChW + slot;
   const bool act = d < a.dim;
   const int dd = act ? d : a.dim - 1;  // idle lanes shadow a valid channel and store nothing
   const long long ch = (long long)b * a.dim + dd;
@@ -319,50 +428,34 @@ __global__ void __launch_bounds__(128, 1) fwd_kernel(const FwdArgs a) {
   const int t_begin = chunk * a.chunk_len;
   const int t_end = min(a.L, t_begin + a.chunk_len);
   const bool last_chunk = t_end == a.L;
-  float* sB = smem + wib * (2 * kBlk * kNS);
-  float* sC = sB + kBlk * kNS;
 
   constexpr bool kPrecise = std::is_same<IO, float>::value;
   const float ascale = kPrecise ? 1.f : kLog2e;
-  float alv[kNS], h[kNS];
   const float* Ad = a.A + (long long)dd * a.N;
-  bool nonpos = true;
-#pragma unroll
-  for (int n = 0; n < kNS; ++n) {
-    alv[n] = n < a.N ? Ad[n] * ascale : 0.f;
-    nonpos &= !(alv[n] > 0.f);
-  }
   const float* hsrc = nullptr;
+  bool hs16 = false;  // hin rows hold 16 states; h0 rows hold N
   if (MODE != kFwdSummary) {
-    if (a.hin) hsrc = a.hin + ((long long)chunk * a.batch * a.dim + ch) * kNS;
-    else if (a.h0) hsrc = a.h0 + ch * a.N;
+    if (a.hin) {
+      hsrc = a.hin + ((long long)chunk * a.batch * a.dim + ch) * kNS;
+      hs16 = true;
+    } else if (a.h0) {
+      hsrc = a.h0 + ch * a.N;
+    }
   }
+  float2 al[PPL], hh[PPL];
 #pragma unroll
-  for (int n = 0; n < kNS; ++n) h[n] = (hsrc && (a.hin || n < a.N)) ? hsrc[n] : 0.f;
+  for (int j = 0; j < PPL; ++j) {
+    const int n0 = SPL * q + 2 * j, n1 = n0 + 1;
+    al[j] = make_float2(n0 < a.N ? Ad[n0] * ascale : 0.f, n1 < a.N ? Ad[n1] * ascale : 0.f);
+    hh[j] = make_float2((hsrc && (hs16 || n0 < a.N)) ? hsrc[n0] : 0.f,
+                        (hsrc && (hs16 || n1 < a.N)) ? hsrc[n1] : 0.f);
+  }
   const float Dd = (MODE == kFwdOut && a.D) ? a.D[dd] : 0.f;
   const float bias = a.dt_bias ? a.dt_bias[dd] : 0.f;
+  WarpTile<LPC>& tile = tiles[wib];
 
-  // The FMA-pipe exponential assumes Δ*A <= 0; a warp holding any positive A entry runs
-  // every exponential on the MUFU unit instead.
-  if (kPrecise || !__all_sync(0xffffffffu, nonpos)) {
-    ChunkScan<IO, VEC, MODE, kNS> cs;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      cs.al[j] = make_float2(alv[2 * j], alv[2 * j + 1]);
-      cs.hh[j] = make_float2(h[2 * j], h[2 * j + 1]);
-    }
-    cs.Dd = Dd; cs.bias = bias; cs.softplus = a.softplus;
-    run_chunk<IO, VEC, MODE, kNS>(a, cs, lane, b, act, ch, t_begin, t_end, last_chunk, sB, sC);
-  } else {
-    ChunkScan<IO, VEC, MODE, KM> cs;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      cs.al[j] = make_float2(alv[2 * j], alv[2 * j + 1]);
-      cs.hh[j] = make_float2(h[2 * j], h[2 * j + 1]);
-    }
-    cs.Dd = Dd; cs.bias = bias; cs.softplus = a.softplus;
-    run_chunk<IO, VEC, MODE, KM>(a, cs, lane, b, act, ch, t_begin, t_end, last_chunk, sB, sC);
-  }
+  run_chunk<IO, VEC, MODE, LPC, KE, KO>(a, tile, hh, al, Dd, bias, lane, slot, q, b, act, ch, t_begin,
+                                        t_end, last_chunk);
 }
 
 // Chain the chunk summaries: h_in(0) = h0, h_in(j+1) = exp(A ΣΔ_j) h_in(j) + h_end(j).
@@ -384,24 +477,53 @@ __global__ void fwd_carry_kernel(const FwdArgs a, const float* __restrict__ summ
   }
 }
 
+template <typename IO, bool VEC, int MODE, int LPC, int KE, int KO>
+void launch_one(const FwdArgs& a, dim3 grid, dim3 block, cudaStream_t s) {
+  const size_t smem = (size_t)(block.x / 32) * sizeof(WarpTile<LPC>);
+  if (smem > 48 * 1024)
+    cudaFuncSetAttribute(fwd_kernel<IO, VEC, MODE, LPC, KE, KO>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  fwd_kernel<IO, VEC, MODE, LPC, KE, KO><<<grid, block, smem, s>>>(a);
+}
+
 template <typename IO, bool VEC, int MODE>
 cudaError_t launch_mode(const FwdArgs& a, int wpb, int kmufu, cudaStream_t s) {
   const long long ctas = (a.nwarps + wpb - 1) / wpb;
   const int nchunk_launch = MODE == kFwdSummary ? a.nchunk - 1 : a.nchunk;  // last chunk's summary is unused
   if (ctas <= 0 || nchunk_launch <= 0) return cudaSuccess;
-  dim3 grid((unsigned)ctas, (unsigned)nchunk_launch);
-  dim3 block(32 * wpb);
-  const size_t smem = (size_t)wpb * 2 * kBlk * kNS * sizeof(float);
-  if constexpr (std::is_same<IO, float>::value) {
-    fwd_kernel<IO, VEC, MODE, 16><<<grid, block, smem, s>>>(a);  // fp32 path: library expf
+  const dim3 grid((unsigned)ctas, (unsigned)nchunk_launch), block(32 * wpb);
+  if constexpr (std::is_same<IO, float>::value) {  // fp32: library expf
+    if (a.lpc == 4) launch_one<IO, VEC, MODE, 4, 2, 2>(a, grid, block, s);
+    else if (a.lpc == 1) launch_one<IO, VEC, MODE, 1, 8, 8>(a, grid, block, s);
+    else launch_one<IO, VEC, MODE, 2, 4, 4>(a, grid, block, s);
   } else if constexpr (MODE != kFwdOut) {
-    fwd_kernel<IO, VEC, MODE, 10><<<grid, block, smem, s>>>(a);
+    if (a.lpc == 4) launch_one<IO, VEC, MODE, 4, 2, 1>(a, grid, block, s);
+    else if (a.lpc == 1) launch_one<IO, VEC, MODE, 1, 7, 6>(a, grid, block, s);
+    else launch_one<IO, VEC, MODE, 2, 4, 3>(a, grid, block, s);
+  } else if (a.lpc == 4) {
+    // exponentials on the MUFU unit per lane over two steps (of 8): 4, 6 or 8
+    switch (kmufu) {
+      case 8: launch_one<IO, VEC, MODE, 4, 1, 1>(a, grid, block, s); break;
+      case 16: launch_one<IO, VEC, MODE, 4, 2, 2>(a, grid, block, s); break;
+      default: launch_one<IO, VEC, MODE, 4, 2, 1>(a, grid, block, s); break;
+    }
+  } else if (a.lpc == 1) {
+    // exponentials on the MUFU unit per lane over two steps (of 32), in units of 16/16
+    switch (kmufu) {
+      case 8: launch_one<IO, VEC, MODE, 1, 4, 4>(a, grid, block, s); break;
+      case 10: launch_one<IO, VEC, MODE, 1, 5, 5>(a, grid, block, s); break;
+      case 12: launch_one<IO, VEC, MODE, 1, 6, 6>(a, grid, block, s); break;
+      case 16: launch_one<IO, VEC, MODE, 1, 8, 8>(a, grid, block, s); break;
+      default: launch_one<IO, VEC, MODE, 1, 7, 7>(a, grid, block, s); break;
+    }
   } else {
-    switch (kmufu) {  // states whose exponential runs on the MUFU unit
-      case 8: fwd_kernel<IO, VEC, MODE, 8><<<grid, block, smem, s>>>(a); break;
-      case 12: fwd_kernel<IO, VEC, MODE, 12><<<grid, block, smem, s>>>(a); break;
-      case 16: fwd_kernel<IO, VEC, MODE, 16><<<grid, block, smem, s>>>(a); break;
-      default: fwd_kernel<IO, VEC, MODE, 10><<<grid, block, smem, s>>>(a); break;
+    // exponentials on the MUFU unit per lane over two steps (of 16): 8 ... 16
+    switch (kmufu) {
+      case 8: launch_one<IO, VEC, MODE, 2, 2, 2>(a, grid, block, s); break;
+      case 10: launch_one<IO, VEC, MODE, 2, 3, 2>(a, grid, block, s); break;
+      case 12: launch_one<IO, VEC, MODE, 2, 3, 3>(a, grid, block, s); break;
+      case 16: launch_one<IO, VEC, MODE, 2, 4, 4>(a, grid, block, s); break;
+      default: launch_one<IO, VEC, MODE, 2, 4, 3>(a, grid, block, s); break;
     }
   }
   return cudaGetLastError();

@@ -8,7 +8,7 @@
 namespace ssm {
 
 constexpr int kBlk = 16;   // time steps per block: one scalar / state / output phase
-constexpr int kNS = 16;    // states held per lane (dstate <= 16, padded with zeros)
+constexpr int kNS = 16;    // states per channel (dstate <= 16, padded with zeros)
 
 // kFwdOut: gated output (+ optional checkpoints / final state); kFwdSummary: per-chunk end
 // state and ΣΔ from a zero state (time-split first pass); kFwdCkpt: state recurrence only,
@@ -35,7 +35,8 @@ struct FwdArgs {
   int chunk_len;        // multiple of kBlk
   int nchunk;           // S
   int softplus;
-  int warps_per_b;      // ceil(dim / 32)
+  int lpc;              // lanes per channel: 1, 2 or 4 (16 / lpc states each)
+  int warps_per_b;      // ceil(dim / (32 / lpc))
   long long nwarps;     // batch * warps_per_b
 };
 
