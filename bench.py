@@ -162,18 +162,14 @@ def dist_env():
 
 
 def max_over_ranks(value: float, world: int, device) -> float:
-    if world == 1:
-        return value
-    import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device=device)
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    from selective_state_space_23_b200.dist import max_over_ranks as _max
+    return _max(value, device) if world > 1 else value
 
 
 def barrier(world: int):
+    from selective_state_space_23_b200.dist import barrier as _barrier
     if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+        _barrier()
 
 
 # ------------------------------------------------------------------ CPU oracle baseline
