@@ -206,9 +206,11 @@ struct BwdLayout {
 
 BwdLayout layout_bwd(int batch, int dim, int seqlen, int dstate, bool have_ckpt) {
   BwdLayout l;
+  // one warp per CTA: CTAs of several warps synchronise once per block for the dB/dC partials,
+  // which measured slower on B200 than writing one partial per warp
   l.wpb = env_int("SSM_BWD_WPB", 1);
   if (l.wpb < 1 || l.wpb > 4) l.wpb = 1;
-  const int warps_per_b = (dim + 31) / 32;
+  const int warps_per_b = (dim + 15) / 16;  // 16 channels per warp
   l.ngroups = (warps_per_b + l.wpb - 1) / l.wpb;
   const size_t nch = (size_t)batch * dim;
   const size_t nblk = (seqlen + ssm::kBlk - 1) / ssm::kBlk;
@@ -404,10 +406,11 @@ int ssm_scan_bwd(const void* u, const void* delta, const float* A, const void* B
   b.part_bc = part_bc; b.part_adt = part_adt;
   b.batch = batch; b.dim = dim; b.L = seqlen; b.N = dstate;
   b.softplus = delta_softplus ? 1 : 0;
-  b.warps_per_b = (dim + 31) / 32;
+  b.warps_per_b = (dim + 15) / 16;
   b.nwarps = (long long)batch * b.warps_per_b;
   b.wpb = l.wpb;
   b.ngroups = l.ngroups;
+  b.kmufu = env_int("SSM_BWD_KMUFU", 4);  // all exponentials on MUFU measured fastest
   if ((e = ssm::launch_bwd(b, io_dtype, vec, s)) != cudaSuccess) return cuda_fail(e, "backward pass");
   if ((e = ssm::launch_bwd_finish(b, io_dtype, dB, dC, dA, dD, ddt_bias, s)) != cudaSuccess)
     return cuda_fail(e, "backward reduction");

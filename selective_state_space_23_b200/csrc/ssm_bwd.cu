@@ -13,340 +13,408 @@
 //   dz_t = dout_t y_t silu'(z_t),  dh0 = Ā_0 λ_0
 // with Ā_t h_{t-1} = h_t - Δ_t B_t x_t, so the reverse sweep needs only h_t.
 //
-// Mapping: one lane per channel, 16 states in registers, time walked backwards in 16-step
-// blocks.  For each block the lane reloads the state entering the block (a checkpoint written
-// by the forward pass or by a checkpoint-only forward pass), replays the 16 steps forward and
-// parks h_t in shared memory, then runs the adjoint recurrence backwards over the block.  dB
-// and dC are sums over the channel axis: each warp transposes its 32 lanes' per-step values
-// through shared memory and sums columns; the CTA sums its warps and writes one partial per
+// Mapping: two lanes per channel, 8 states each in registers; a warp holds 16 consecutive d of
+// one batch row.  Time is walked backwards in 16-step blocks; each block is handled in two halves
+// (upper then lower 8 steps): the lanes reload the state entering the block (a checkpoint written
+// by the forward pass, or by a state-only replay pass), replay forward to the end of the half,
+// parking h_t of the half's 8 steps in shared memory, then run the adjoint recurrence backwards
+// over the half, recomputing Ā_t.  Per-step scalars (Δ, Δx, g) are computed once per (channel,
+// step) and shared through shared memory; the two half-lanes combine their sums with one shuffle.
+// dB and dC (sums over the channel axis) are transposed through shared memory two steps at a
+// time, summed with vector loads and one shuffle level, and written as one partial per
 // (CTA, b, n, t); a finishing kernel adds the partials in a fixed order (deterministic).
 #include <type_traits>
 
 #include "ssm_device.cuh"
 #include "ssm_kernels.h"
+#include "ssm_rows.cuh"
 
 namespace ssm {
 namespace {
 
-constexpr int kHsStride = kBlk * kNS + 4;  // per-lane row of parked states (+4: no bank conflicts)
-constexpr int kRedStride = 36;             // per-lane row of the transpose buffer
+constexpr int kHB = 8;                  // steps per half block = states per lane
+constexpr int kCW = 16;                 // channels per warp (two lanes per channel)
+constexpr int kTS = kCW + 1;            // padded step stride of the per-step tables
+constexpr int kParkS = kHB * kHB + 4;   // per-lane parked states: 8 steps x 8 states (+4: banks)
+constexpr int kRedS = 36;               // per-lane row of the dB/dC transpose: 2 steps x 16 (+4)
 
-struct WarpSmem {
-  float sB[kBlk * kNS];
-  float sC[kBlk * kNS];
-  float hs[32 * kHsStride];
-  float red[32 * kRedStride];
-  float wsum[kBlk * 32];
+// Per-warp shared memory of one 16-step block.
+struct BwdTile {
+  float4 sB[kBlk * kNS / 4];   // B_t,n as f32 [step][state]
+  float4 sC[kBlk * kNS / 4];   // C_t,n
+  float2 sd[kBlk * kTS];       // (Δ_t, Δ_t x_t) per [step][channel slot]
+  float sg[kBlk * kTS];        // g_t = dout_t silu(z_t)
+  float ys[kBlk * kTS];        // y_t = C_t.h_t + D x_t without D x_t (for dz)
+  float2 sS[kBlk * kTS];       // (Σ_n λ B, Σ_n A λ Ā h_{t-1}) of each step
+  float park[32 * kParkS];     // per lane: h_t of the 8 steps of the current half block
+  float red[32 * kRedS];       // dB/dC values of two steps, transposed to sum over channels
+  float wres[kBlk * 32];       // the warp's channel sums [step][half * 16 + (dB n | dC n)]
 };
 
-__device__ __forceinline__ uint32_t wd(const uint4& q, int j) {
-  return j == 0 ? q.x : j == 1 ? q.y : j == 2 ? q.z : q.w;
-}
-template <typename IO> struct Row { uint4 v[sizeof(IO) * kBlk / 16]; };
-template <typename IO> __device__ __forceinline__ float el(const Row<IO>& r, int k);
-template <> __device__ __forceinline__ float el<float>(const Row<float>& r, int k) {
-  return __uint_as_float(wd(r.v[k >> 2], k & 3));
-}
-template <> __device__ __forceinline__ float el<uint16_t>(const Row<uint16_t>& r, int k) {
-  const uint32_t w = wd(r.v[k >> 3], (k >> 1) & 3);
-  return (k & 1) ? bf16_hi(w) : bf16_lo(w);
-}
-
-template <typename IO, bool VEC>
-__device__ __forceinline__ void load_row(Row<IO>& r, const IO* p, int nvalid) {
-  if (VEC && nvalid == kBlk) {
-    const uint4* q = reinterpret_cast<const uint4*>(p);
-#pragma unroll
-    for (int i = 0; i < (int)(sizeof(r.v) / 16); ++i) r.v[i] = __ldcs(q + i);
-    return;
+// One replayed step for one lane (8 states): h <- Ā h + Δ x B.  KP of the 4 state pairs take 2^x
+// from MUFU, the rest from the FMA-pipe polynomial (only used in range-checked blocks).  Returns
+// the partial readout Σ C h over the lane's states when READOUT.
+template <bool PRECISE, bool READOUT, int KP>
+__device__ __forceinline__ float replay_step(float2 (&hh)[4], const float2 (&al)[4], float2 dd,
+                                             const float4* bq, const float4* cq) {
+  const float2 d2 = f2(dd.x), dx2 = f2(dd.y);
+  const float4 b0 = bq[0], b1 = bq[1];
+  float4 c0 = make_float4(0.f, 0.f, 0.f, 0.f), c1 = c0;
+  if (READOUT) {
+    c0 = cq[0];
+    c1 = cq[1];
   }
-  uint32_t w[sizeof(r.v) / 4];
+  float2 ya = make_float2(0.f, 0.f), yb = ya;
 #pragma unroll
-  for (int i = 0; i < (int)(sizeof(r.v) / 4); ++i) w[i] = 0u;
-  if (sizeof(IO) == 4) {
-    const uint32_t* s = reinterpret_cast<const uint32_t*>(p);
-#pragma unroll
-    for (int e = 0; e < kBlk; ++e)
-      if (e < nvalid) w[e] = s[e];
-  } else {
-    const unsigned short* s = reinterpret_cast<const unsigned short*>(p);
-#pragma unroll
-    for (int e = 0; e < kBlk; ++e)
-      if (e < nvalid) w[e >> 1] |= ((uint32_t)s[e]) << (16 * (e & 1));
-  }
-#pragma unroll
-  for (int i = 0; i < (int)(sizeof(r.v) / 16); ++i)
-    r.v[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-}
-
-template <typename IO, bool VEC>
-__device__ __forceinline__ void store_row(IO* p, const float (&o)[kBlk], int nvalid) {
-  if (sizeof(IO) == 2) {
-    uint32_t w[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(o[2 * i], o[2 * i + 1]);
-    if (VEC && nvalid == kBlk) {
-      uint4* q = reinterpret_cast<uint4*>(p);
-      __stcs(q, make_uint4(w[0], w[1], w[2], w[3]));
-      __stcs(q + 1, make_uint4(w[4], w[5], w[6], w[7]));
+  for (int j = 0; j < 4; ++j) {
+    const float4 bb = j < 2 ? b0 : b1;
+    const float2 bp = (j & 1) ? make_float2(bb.z, bb.w) : make_float2(bb.x, bb.y);
+    float2 av;
+    if (PRECISE) {
+      av = make_float2(expf(dd.x * al[j].x), expf(dd.x * al[j].y));
+    } else if (j < KP) {
+      const float2 x = mul2(d2, al[j]);
+      av = make_float2(ex2_mufu(x.x), ex2_mufu(x.y));
     } else {
-      unsigned short* s = reinterpret_cast<unsigned short*>(p);
-#pragma unroll
-      for (int e = 0; e < kBlk; ++e)
-        if (e < nvalid) s[e] = (unsigned short)(w[e >> 1] >> (16 * (e & 1)));
+      av = exp2_fma_prod_x2(d2, al[j]);
     }
-  } else {
-    float* s = reinterpret_cast<float*>(p);
-    if (VEC && nvalid == kBlk) {
-      float4* q = reinterpret_cast<float4*>(p);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) __stcs(q + i, make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]));
-    } else {
-#pragma unroll
-      for (int e = 0; e < kBlk; ++e)
-        if (e < nvalid) s[e] = o[e];
+    hh[j] = fma2(av, hh[j], mul2(dx2, bp));
+    if (READOUT) {
+      const float4 cc = j < 2 ? c0 : c1;
+      const float2 cp = (j & 1) ? make_float2(cc.z, cc.w) : make_float2(cc.x, cc.y);
+      if (j & 1) yb = fma2(cp, hh[j], yb);
+      else ya = fma2(cp, hh[j], ya);
     }
   }
+  const float2 ys = add2(ya, yb);
+  return ys.x + ys.y;
 }
 
-template <typename IO, bool VEC>
-__global__ void __launch_bounds__(128, 1) bwd_kernel(const BwdArgs a) {
+// One adjoint step for one lane: completes λ_t, forms the dB/dC contributions (into `vals`),
+// accumulates dA, Σ λB and Σ A λ Ā h_{t-1}, and advances λ <- Ā_t λ_t.
+template <bool PRECISE, int KP>
+__device__ __forceinline__ void adjoint_step(float2 (&lam)[4], float2 (&dA)[4], const float2 (&al)[4],
+                                             const float2 (&hk)[4], float2 dd, float g, float live,
+                                             const float4* bq, const float4* cq, float2 (&vals)[8],
+                                             float& S1, float& S2) {
+  const float2 d2 = f2(dd.x), ndx2 = f2(-dd.y), g2 = f2(g);
+  const float2 dxl = f2(dd.y * live), gl = f2(g * live);
+  const float4 b0 = bq[0], b1 = bq[1], c0 = cq[0], c1 = cq[1];
+  float2 s1 = make_float2(0.f, 0.f), s2 = s1;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float4 bb = j < 2 ? b0 : b1;
+    const float4 cc = j < 2 ? c0 : c1;
+    const float2 bp = (j & 1) ? make_float2(bb.z, bb.w) : make_float2(bb.x, bb.y);
+    const float2 cp = (j & 1) ? make_float2(cc.z, cc.w) : make_float2(cc.x, cc.y);
+    float2 av;
+    if (PRECISE) {
+      av = make_float2(expf(dd.x * al[j].x), expf(dd.x * al[j].y));
+    } else if (j < KP) {
+      const float2 x = mul2(d2, al[j]);
+      av = make_float2(ex2_mufu(x.x), ex2_mufu(x.y));
+    } else {
+      av = exp2_fma_prod_x2(d2, al[j]);
+    }
+    lam[j] = fma2(g2, cp, lam[j]);              // λ_t complete
+    vals[j] = mul2(lam[j], dxl);                // dB_t contribution: λ Δ x
+    vals[4 + j] = mul2(gl, hk[j]);              // dC_t contribution: g h_t
+    const float2 qv = fma2(ndx2, bp, hk[j]);    // Ā_t h_{t-1} = h_t - Δ x B
+    const float2 lq = mul2(lam[j], qv);
+    s1 = fma2(lam[j], bp, s1);
+    s2 = fma2(al[j], lq, s2);
+    dA[j] = fma2(d2, lq, dA[j]);
+    lam[j] = mul2(lam[j], av);                  // Ā_t λ_t, for step t-1
+  }
+  S1 = s1.x + s1.y;
+  S2 = s2.x + s2.y;
+}
+
+// Sum the dB/dC values of two steps over the warp's 16 channels.  Row `lane` of `red` holds the
+// lane's 32 values (step slot s = 0, 1; 8 dB then 8 dC of its half of the states).  Lane j sums
+// one 4-value quad of one step over 8 channels with vector loads, one shuffle adds the other 8,
+// and lanes 0..15 store the warp sums.
+__device__ __forceinline__ void reduce_two_steps(BwdTile& tl, int lane, int k0, int k1) {
+  __syncwarp();
+  const int quad = lane & 3, s = (lane >> 2) & 1, qq = (lane >> 3) & 1, rg = lane >> 4;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = 2 * (8 * rg + i) + qq;
+    const float4 v = *reinterpret_cast<const float4*>(tl.red + r * kRedS + s * 16 + quad * 4);
+    const float2 lo = add2(make_float2(acc.x, acc.y), make_float2(v.x, v.y));
+    const float2 hi = add2(make_float2(acc.z, acc.w), make_float2(v.z, v.w));
+    acc = make_float4(lo.x, lo.y, hi.x, hi.y);
+  }
+  acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 16);
+  acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 16);
+  acc.z += __shfl_xor_sync(0xffffffffu, acc.z, 16);
+  acc.w += __shfl_xor_sync(0xffffffffu, acc.w, 16);
+  const int kk = s == 0 ? k0 : k1;
+  if (rg == 0 && kk >= 0) *reinterpret_cast<float4*>(tl.wres + kk * 32 + qq * 16 + quad * 4) = acc;
+  __syncwarp();
+}
+
+// Replay a block from its entering state and run the adjoint over steps [lo, hi).
+template <bool PRECISE, int KP>
+__device__ __forceinline__ void half_pass(BwdTile& tl, const float2 (&hstart)[4], float2 (&lam)[4],
+                                          float2 (&dA)[4], const float2 (&al)[4], float aback,
+                                          float live, int lane, int slot, int q, int lo, int hi) {
+  const float4* bq = tl.sB + 2 * q;
+  const float4* cq = tl.sC + 2 * q;
+  float* prow = tl.park + lane * kParkS;
+  float2 hh[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) hh[j] = hstart[j];
+#pragma unroll 1
+  for (int k = 0; k < lo; ++k)
+    replay_step<PRECISE, false, KP>(hh, al, tl.sd[k * kTS + slot], bq + k * 4, cq);
+#pragma unroll 1
+  for (int k = lo; k < hi; ++k) {
+    float y = replay_step<PRECISE, true, KP>(hh, al, tl.sd[k * kTS + slot], bq + k * 4, cq + k * 4);
+    y += __shfl_xor_sync(0xffffffffu, y, 1);
+    if (q == 0) tl.ys[k * kTS + slot] = y;
+    float4* pk = reinterpret_cast<float4*>(prow + (k - lo) * kHB);
+    pk[0] = make_float4(hh[0].x, hh[0].y, hh[1].x, hh[1].y);
+    pk[1] = make_float4(hh[2].x, hh[2].y, hh[3].x, hh[3].y);
+  }
+  // adjoint, two steps at a time (hi-1, hi-2), ..., down to lo
+  float* rrow = tl.red + lane * kRedS;
+#pragma unroll 1
+  for (int k = hi - 1; k >= lo; k -= 2) {
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      const int kk = k - s;
+      float2 vals[8];
+      if (kk >= lo) {
+        const float4* pk = reinterpret_cast<const float4*>(prow + (kk - lo) * kHB);
+        const float4 h0 = pk[0], h1 = pk[1];
+        const float2 hk[4] = {make_float2(h0.x, h0.y), make_float2(h0.z, h0.w),
+                              make_float2(h1.x, h1.y), make_float2(h1.z, h1.w)};
+        float S1, S2;
+        adjoint_step<PRECISE, KP>(lam, dA, al, hk, tl.sd[kk * kTS + slot], tl.sg[kk * kTS + slot],
+                                  live, bq + kk * 4, cq + kk * 4, vals, S1, S2);
+        S1 += __shfl_xor_sync(0xffffffffu, S1, 1);
+        S2 += __shfl_xor_sync(0xffffffffu, S2, 1);
+        if (q == 0) tl.sS[kk * kTS + slot] = make_float2(S1, S2 * aback);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) vals[j] = make_float2(0.f, 0.f);
+      }
+      float4* rv = reinterpret_cast<float4*>(rrow + s * 16);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        rv[j] = make_float4(vals[2 * j].x, vals[2 * j].y, vals[2 * j + 1].x, vals[2 * j + 1].y);
+    }
+    reduce_two_steps(tl, lane, k, k - 1 >= lo ? k - 1 : -1);
+  }
+}
+
+template <typename IO, bool VEC, int KP>
+__global__ void __launch_bounds__(128) bwd_kernel(const BwdArgs a) {
   constexpr bool kPrecise = std::is_same<IO, float>::value;
   extern __shared__ float4 smem4[];
-  WarpSmem* all = reinterpret_cast<WarpSmem*>(smem4);
+  BwdTile* tiles = reinterpret_cast<BwdTile*>(smem4);
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  WarpSmem& sm = all[wib];
-  const int b = blockIdx.x / a.ngroups, g = blockIdx.x % a.ngroups;
-  const int d = (g * a.wpb + wib) * 32 + lane;
+  BwdTile& tl = tiles[wib];
+  const int slot = lane >> 1, q = lane & 1;
+  const int b = blockIdx.x / a.ngroups, grp = blockIdx.x % a.ngroups;
+  const int d = (grp * a.wpb + wib) * kCW + slot;
   const bool act = d < a.dim;
   const int dd = act ? d : a.dim - 1;
   const float live = act ? 1.f : 0.f;  // idle lanes contribute nothing to the channel sums
   const long long ch = (long long)b * a.dim + dd;
   const int L = a.L, N = a.N;
   const int nblk = (L + kBlk - 1) / kBlk;
-
   const float ascale = kPrecise ? 1.f : kLog2e;
   const float aback = kPrecise ? 1.f : kLn2;  // al * aback == A
-  float2 al[8], lam[8], dA[8];
+
+  float2 al[4], lam[4], dA[4];
+  float amax = 0.f;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int n0 = 2 * j, n1 = 2 * j + 1;
+  for (int j = 0; j < 4; ++j) {
+    const int n0 = kHB * q + 2 * j, n1 = n0 + 1;
     al[j] = make_float2(n0 < N ? a.A[(long long)dd * N + n0] * ascale : 0.f,
                         n1 < N ? a.A[(long long)dd * N + n1] * ascale : 0.f);
     lam[j] = make_float2((a.dhL && n0 < N) ? a.dhL[ch * N + n0] : 0.f,
                          (a.dhL && n1 < N) ? a.dhL[ch * N + n1] : 0.f);
     dA[j] = make_float2(0.f, 0.f);
+    amax = fmaxf(amax, fmaxf(fabsf(al[j].x), fabsf(al[j].y)));
   }
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
   const float Dd = a.D ? a.D[dd] : 0.f;
   const float bias = a.dt_bias ? a.dt_bias[dd] : 0.f;
   float dD_acc = 0.f, dbias_acc = 0.f;
 
-  const IO* up = reinterpret_cast<const IO*>(a.u) + ch * (long long)L;
-  const IO* dp = reinterpret_cast<const IO*>(a.delta) + ch * (long long)L;
-  const IO* zp = a.z ? reinterpret_cast<const IO*>(a.z) + ch * (long long)L : nullptr;
-  const IO* gp = reinterpret_cast<const IO*>(a.dout) + ch * (long long)L;
-  const int bc_n = lane >> 1, bc_half = lane & 1;
-  const bool bc_live = bc_n < N;
-  const IO* Bp = reinterpret_cast<const IO*>(a.B) + ((long long)b * N + (bc_live ? bc_n : 0)) * L;
-  const IO* Cp = reinterpret_cast<const IO*>(a.C) + ((long long)b * N + (bc_live ? bc_n : 0)) * L;
-  float* hrow = sm.hs + lane * kHsStride;
-  float* rrow = sm.red + lane * kRedStride;
+  const long long row = ch * (long long)L + kHB * q;   // this lane's 8 steps of each block
+  const IO* up = reinterpret_cast<const IO*>(a.u) + row;
+  const IO* dp = reinterpret_cast<const IO*>(a.delta) + row;
+  const IO* zp = a.z ? reinterpret_cast<const IO*>(a.z) + row : nullptr;
+  const IO* gp = reinterpret_cast<const IO*>(a.dout) + row;
+  const bool bc_live = slot < N;  // the lane also stages B/C row `slot`, steps [8 q, 8 q + 8)
+  const long long bcrow = ((long long)b * N + (bc_live ? slot : 0)) * L + kHB * q;
+  const IO* Bp = reinterpret_cast<const IO*>(a.B) + bcrow;
+  const IO* Cp = reinterpret_cast<const IO*>(a.C) + bcrow;
+  float* sBw = reinterpret_cast<float*>(tl.sB);
+  float* sCw = reinterpret_cast<float*>(tl.sC);
 
   for (int blk = nblk - 1; blk >= 0; --blk) {
     const int t0 = blk * kBlk;
     const int nvalid = min(kBlk, L - t0);
-    Row<IO> ru, rd, rz, rg;
-    load_row<IO, VEC>(ru, up + t0, nvalid);
-    load_row<IO, VEC>(rd, dp + t0, nvalid);
-    load_row<IO, VEC>(rg, gp + t0, nvalid);
-    if (zp) load_row<IO, VEC>(rz, zp + t0, nvalid);
-
-    // B, C rows of this block -> shared memory as f32 [step][state]
-    __syncwarp();
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int t = t0 + 8 * bc_half + j;
-      const bool ok = bc_live && t < L;
-      float bv = 0.f, cv = 0.f;
-      if (ok) {
-        if (sizeof(IO) == 2) {
-          bv = bf16_to_f32(reinterpret_cast<const uint16_t*>(Bp)[t]);
-          cv = bf16_to_f32(reinterpret_cast<const uint16_t*>(Cp)[t]);
-        } else {
-          bv = reinterpret_cast<const float*>(Bp)[t];
-          cv = reinterpret_cast<const float*>(Cp)[t];
-        }
-      }
-      sm.sB[(8 * bc_half + j) * kNS + bc_n] = bv;
-      sm.sC[(8 * bc_half + j) * kNS + bc_n] = cv;
+    const int nown = max(0, min(kHB, nvalid - kHB * q));
+    Row<IO, kHB> ru, rd, rz, rg, rb, rc;
+    if (VEC && nown == kHB) {
+      load_row<IO, kHB, true>(ru, up + t0, kHB);
+      load_row<IO, kHB, true>(rd, dp + t0, kHB);
+      load_row<IO, kHB, true>(rg, gp + t0, kHB);
+      if (zp) load_row<IO, kHB, true>(rz, zp + t0, kHB);
+    } else {
+      load_row<IO, kHB, false>(ru, up + t0, nown);
+      load_row<IO, kHB, false>(rd, dp + t0, nown);
+      load_row<IO, kHB, false>(rg, gp + t0, nown);
+      if (zp) load_row<IO, kHB, false>(rz, zp + t0, nown);
     }
-    __syncwarp();
-
-    // state entering the block
-    float2 hh[8];
+    if (!bc_live) {
+      rb.zero();
+      rc.zero();
+    } else if (VEC && nown == kHB) {
+      load_row<IO, kHB, true>(rb, Bp + t0, kHB);
+      load_row<IO, kHB, true>(rc, Cp + t0, kHB);
+    } else {
+      load_row<IO, kHB, false>(rb, Bp + t0, nown);
+      load_row<IO, kHB, false>(rc, Cp + t0, nown);
+    }
+    // the state entering the block
+    float2 hstart[4];
     const float* cp = a.ckpt + (ch * nblk + blk) * N;
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      hh[j] = make_float2(2 * j < N ? cp[2 * j] : 0.f, 2 * j + 1 < N ? cp[2 * j + 1] : 0.f);
+    for (int j = 0; j < 4; ++j) {
+      const int n0 = kHB * q + 2 * j;
+      hstart[j] = make_float2(n0 < N ? cp[n0] : 0.f, n0 + 1 < N ? cp[n0 + 1] : 0.f);
+    }
 
-    // per-step scalars
-    float dl[kBlk], dxu[kBlk], gg[kBlk];
+    __syncwarp();  // the previous block's tables are no longer read
 #pragma unroll
-    for (int k = 0; k < kBlk; ++k) {
-      const float v = el<IO>(rd, k) + bias;
-      dl[k] = !a.softplus ? v : (kPrecise ? softplus_precise(v) : softplus_fast(v));
-      dxu[k] = dl[k] * el<IO>(ru, k);
-      float gk = el<IO>(rg, k);
+    for (int j = 0; j < kHB; ++j) {
+      sBw[(kHB * q + j) * kNS + slot] = rb.get(j);
+      sCw[(kHB * q + j) * kNS + slot] = rc.get(j);
+    }
+    // per-step scalars of this lane's 8 steps
+    float sv[kHB], dzf[kHB];
+    float dabs = 0.f;
+#pragma unroll
+    for (int j = 0; j < kHB; j += 2) {
+      const float2 v = add2(make_float2(rd.get(j), rd.get(j + 1)), f2(bias));
+      float2 dl = v, sp = make_float2(1.f, 1.f);
+      if (a.softplus) {
+        if (kPrecise) {
+          dl = make_float2(softplus_precise(v.x), softplus_precise(v.y));
+          sp = make_float2(sigmoid_precise(v.x), sigmoid_precise(v.y));
+        } else {
+          dl = softplus_fast_x2(v);
+          sp = sigmoid_fast_x2(v);
+        }
+      }
+      const float2 dx = mul2(dl, make_float2(ru.get(j), ru.get(j + 1)));
+      const float2 go = make_float2(rg.get(j), rg.get(j + 1));
+      float2 g = go, zf = make_float2(0.f, 0.f);
       if (zp) {
-        const float zk = el<IO>(rz, k);
-        gk *= zk * (kPrecise ? sigmoid_precise(zk) : sigmoid_fast(zk));
+        const float2 z2 = make_float2(rz.get(j), rz.get(j + 1));
+        const float2 sg = kPrecise ? make_float2(sigmoid_precise(z2.x), sigmoid_precise(z2.y))
+                                   : sigmoid_fast_x2(z2);
+        g = mul2(go, mul2(z2, sg));
+        // silu'(z) = σ(z) (1 + z (1 - σ(z)))
+        zf = mul2(mul2(go, sg), fma2(z2, add2(f2(1.f), mul2(sg, f2(-1.f))), f2(1.f)));
       }
-      gg[k] = gk;
+      tl.sd[(kHB * q + j) * kTS + slot] = make_float2(dl.x, dx.x);
+      tl.sd[(kHB * q + j + 1) * kTS + slot] = make_float2(dl.y, dx.y);
+      tl.sg[(kHB * q + j) * kTS + slot] = g.x;
+      tl.sg[(kHB * q + j + 1) * kTS + slot] = g.y;
+      sv[j] = sp.x; sv[j + 1] = sp.y;
+      dzf[j] = zf.x; dzf[j + 1] = zf.y;
+      dabs = fmaxf(dabs, fmaxf(fabsf(dl.x), fabsf(dl.y)));
+      if (dl.x != dl.x || dl.y != dl.y) dabs = __int_as_float(0x7f800000);
     }
-
-    // replay the block forward, parking h_t; y_t for dz
-    float odz[kBlk];
-#pragma unroll
-    for (int k = 0; k < kBlk; ++k) {
-      if (k < nvalid) {
-        const float2 d2 = f2(dl[k]), du2 = f2(dxu[k]);
-        float2 y2 = make_float2(Dd * el<IO>(ru, k), 0.f);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          float2 av;
-          if (kPrecise) {
-            av = make_float2(expf(dl[k] * al[j].x), expf(dl[k] * al[j].y));
-          } else {
-            const float2 x = mul2(d2, al[j]);
-            av = make_float2(ex2_mufu(x.x), ex2_mufu(x.y));
-          }
-          const float2 bp = *reinterpret_cast<const float2*>(sm.sB + k * kNS + 2 * j);
-          const float2 cq = *reinterpret_cast<const float2*>(sm.sC + k * kNS + 2 * j);
-          hh[j] = fma2(av, hh[j], mul2(du2, bp));
-          y2 = fma2(cq, hh[j], y2);
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          reinterpret_cast<float4*>(hrow + k * kNS)[q] =
-              make_float4(hh[2 * q].x, hh[2 * q].y, hh[2 * q + 1].x, hh[2 * q + 1].y);
-        float dzk = 0.f;
-        if (zp) {
-          const float zk = el<IO>(rz, k);
-          const float sg = kPrecise ? sigmoid_precise(zk) : sigmoid_fast(zk);
-          dzk = el<IO>(rg, k) * (y2.x + y2.y) * sg * (1.f + zk * (1.f - sg));
-        }
-        odz[k] = dzk;
-      } else {
-        odz[k] = 0.f;
-      }
+    __syncwarp();
+    const bool safe = !__any_sync(0xffffffffu, !(amax * dabs <= 126.f));
+    for (int half = 1; half >= 0; --half) {
+      const int lo = kHB * half, hi = min(nvalid, lo + kHB);
+      if (lo >= hi) continue;
+      if (kPrecise || !safe)
+        half_pass<kPrecise, 4>(tl, hstart, lam, dA, al, aback, live, lane, slot, q, lo, hi);
+      else
+        half_pass<kPrecise, KP>(tl, hstart, lam, dA, al, aback, live, lane, slot, q, lo, hi);
     }
-    if (a.dz && zp && act) store_row<IO, VEC>(reinterpret_cast<IO*>(a.dz) + ch * (long long)L + t0, odz, nvalid);
+    __syncwarp();
 
-    // adjoint sweep, backwards over the block
+    // outputs of this lane's 8 steps
+    float odu[kHB], odd[kHB], odz[kHB];
 #pragma unroll
-    for (int k = kBlk - 1; k >= 0; --k) {
-      if (k < nvalid) {
-        float2 hk[8];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float4 v = reinterpret_cast<const float4*>(hrow + k * kNS)[q];
-          hk[2 * q] = make_float2(v.x, v.y);
-          hk[2 * q + 1] = make_float2(v.z, v.w);
-        }
-        const float2 g2 = f2(gg[k]), du2 = f2(dxu[k]), d2 = f2(dl[k]);
-        const float2 gl = f2(gg[k] * live), dul = f2(dxu[k] * live);
-        float2 s1 = make_float2(0.f, 0.f), s2 = make_float2(0.f, 0.f);
-        float2 vB[8], vC[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float2 bp = *reinterpret_cast<const float2*>(sm.sB + k * kNS + 2 * j);
-          const float2 cq = *reinterpret_cast<const float2*>(sm.sC + k * kNS + 2 * j);
-          lam[j] = fma2(g2, cq, lam[j]);                       // λ_t complete
-          vB[j] = mul2(lam[j], dul);                           // dB contribution
-          vC[j] = mul2(gl, hk[j]);                             // dC contribution
-          const float2 qv = fma2(du2, make_float2(-bp.x, -bp.y), hk[j]);  // Ā_t h_{t-1}
-          const float2 lq = mul2(lam[j], qv);
-          s1 = fma2(lam[j], bp, s1);
-          s2 = fma2(al[j], lq, s2);
-          dA[j] = fma2(d2, lq, dA[j]);
-          float2 av;
-          if (kPrecise) {
-            av = make_float2(expf(dl[k] * al[j].x), expf(dl[k] * al[j].y));
-          } else {
-            const float2 x = mul2(d2, al[j]);
-            av = make_float2(ex2_mufu(x.x), ex2_mufu(x.y));
-          }
-          lam[j] = mul2(lam[j], av);                           // Ā_t λ_t, for step t-1
-        }
-        const float S1 = s1.x + s1.y, S2 = (s2.x + s2.y) * aback;
-        const float xk = el<IO>(ru, k);
-        const float duk = dl[k] * S1 + gg[k] * Dd;
-        const float ddt = xk * S1 + S2;
-        float ddl = ddt;
-        if (a.softplus) {
-          const float v = el<IO>(rd, k) + bias;
-          ddl = ddt * (kPrecise ? sigmoid_precise(v) : sigmoid_fast(v));
-        }
-        dD_acc += gg[k] * xk;
-        dbias_acc += ddl;
-        // park du, ddelta in the (already consumed) state slot of step k
-        hrow[k * kNS + 0] = duk;
-        hrow[k * kNS + 1] = ddl;
-
-        // channel sums of dB, dC for this step: transpose through shared memory
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          reinterpret_cast<float4*>(rrow)[q] = make_float4(vB[2 * q].x, vB[2 * q].y, vB[2 * q + 1].x, vB[2 * q + 1].y);
-          reinterpret_cast<float4*>(rrow)[4 + q] = make_float4(vC[2 * q].x, vC[2 * q].y, vC[2 * q + 1].x, vC[2 * q + 1].y);
-        }
-        __syncwarp();
-        float colsum = 0.f;
-#pragma unroll
-        for (int l = 0; l < 32; ++l) colsum += sm.red[l * kRedStride + lane];
-        sm.wsum[k * 32 + lane] = colsum;
-        __syncwarp();
-      } else {
-        sm.wsum[k * 32 + lane] = 0.f;
+    for (int j = 0; j < kHB; ++j) {
+      const int k = kHB * q + j;
+      const float2 S = tl.sS[k * kTS + slot];
+      const float2 dlx = tl.sd[k * kTS + slot];
+      const float g = tl.sg[k * kTS + slot];
+      const float x = ru.get(j);
+      odz[j] = (tl.ys[k * kTS + slot] + Dd * x) * dzf[j];
+      odu[j] = dlx.x * S.x + g * Dd;
+      odd[j] = (x * S.x + S.y) * sv[j];
+      if (j < nown) {
+        dD_acc += g * x;
+        dbias_acc += odd[j];
       }
     }
-    float odu[kBlk], odd[kBlk];
-#pragma unroll
-    for (int k = 0; k < kBlk; ++k) {
-      odu[k] = hrow[k * kNS + 0];
-      odd[k] = hrow[k * kNS + 1];
-    }
-    if (act) {
-      if (a.du) store_row<IO, VEC>(reinterpret_cast<IO*>(a.du) + ch * (long long)L + t0, odu, nvalid);
-      if (a.ddelta) store_row<IO, VEC>(reinterpret_cast<IO*>(a.ddelta) + ch * (long long)L + t0, odd, nvalid);
+    if (act && nown > 0) {
+      IO* o;
+      if (a.du) {
+        o = reinterpret_cast<IO*>(a.du) + row + t0;
+        if (VEC && nown == kHB) store_row<IO, kHB, true>(o, odu, kHB); else store_row<IO, kHB, false>(o, odu, nown);
+      }
+      if (a.ddelta) {
+        o = reinterpret_cast<IO*>(a.ddelta) + row + t0;
+        if (VEC && nown == kHB) store_row<IO, kHB, true>(o, odd, kHB); else store_row<IO, kHB, false>(o, odd, nown);
+      }
+      if (a.dz && zp) {
+        o = reinterpret_cast<IO*>(a.dz) + row + t0;
+        if (VEC && nown == kHB) store_row<IO, kHB, true>(o, odz, kHB); else store_row<IO, kHB, false>(o, odz, nown);
+      }
     }
 
-    // CTA partial of dB, dC for this block: sum the warps, one value per (n, which, step)
+    // CTA partial of dB, dC for this block: add the warps' sums, one value per (step, n, which)
     __syncthreads();
     for (int p = threadIdx.x; p < kBlk * 32; p += blockDim.x) {
-      const int k = p & (kBlk - 1), j = p >> 4;   // j < 16: dB state j; j >= 16: dC state j-16
+      const int k = p & (kBlk - 1), e = p >> 4;    // e = half * 16 + (v < 8 ? dB : dC) * 8 + n
       if (k < nvalid) {
-        float s = 0.f;
-        for (int w = 0; w < a.wpb; ++w) s += all[w].wsum[k * 32 + j];
-        const long long row = ((long long)(g * a.batch + b) * 2 + (j >> 4)) * kNS + (j & 15);
-        a.part_bc[row * L + t0 + k] = s;
+        float sum = 0.f;
+        for (int w = 0; w < a.wpb; ++w) sum += tiles[w].wres[k * 32 + e];
+        const int n = 8 * (e >> 4) + (e & 7), which = (e >> 3) & 1;
+        const long long prow = ((long long)(grp * a.batch + b) * 2 + which) * kNS + n;
+        a.part_bc[prow * L + t0 + k] = sum;
       }
     }
     __syncthreads();
   }
 
+  dD_acc += __shfl_xor_sync(0xffffffffu, dD_acc, 1);
+  dbias_acc += __shfl_xor_sync(0xffffffffu, dbias_acc, 1);
   if (!act) return;
-  if (a.dh0)
 #pragma unroll
-    for (int n = 0; n < kNS; ++n)
-      if (n < N) a.dh0[ch * N + n] = (n & 1) ? lam[n >> 1].y : lam[n >> 1].x;
-  float* pa = a.part_adt + ch * (kNS + 2);
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    pa[2 * j] = dA[j].x;        // Σ λ Δ Ā h_{t-1}: no A factor, so no log2(e) rescale
-    pa[2 * j + 1] = dA[j].y;
+  for (int j = 0; j < 4; ++j) {
+    const int n0 = kHB * q + 2 * j;
+    if (a.dh0) {
+      if (n0 < N) a.dh0[ch * N + n0] = lam[j].x;
+      if (n0 + 1 < N) a.dh0[ch * N + n0 + 1] = lam[j].y;
+    }
+    float* pa = a.part_adt + ch * (kNS + 2);
+    pa[n0] = dA[j].x;  // Σ λ Δ Ā h_{t-1}: no A factor, so no log2(e) rescale
+    pa[n0 + 1] = dA[j].y;
   }
-  pa[kNS] = dD_acc;
-  pa[kNS + 1] = dbias_acc;
+  if (q == 0) {
+    float* pa = a.part_adt + ch * (kNS + 2);
+    pa[kNS] = dD_acc;
+    pa[kNS + 1] = dbias_acc;
+  }
 }
 
 // dB, dC: sum the CTA partials over groups in a fixed order; dA, dD, ddt_bias: sum over batch.
@@ -384,27 +452,27 @@ __global__ void bwd_finish_adt(const BwdArgs a, float* dA, float* dD, float* ddt
   else if (ddt_bias) ddt_bias[d] = s;
 }
 
-}  // namespace
-
-cudaError_t launch_bwd(const BwdArgs& a, int io, bool vec, cudaStream_t s) {
-  dim3 grid((unsigned)(a.batch * a.ngroups));
-  dim3 block(32 * a.wpb);
-  const size_t smem = sizeof(WarpSmem) * a.wpb;
-  if (io == 1) {
-    auto k = vec ? bwd_kernel<uint16_t, true> : bwd_kernel<uint16_t, false>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    k<<<grid, block, smem, s>>>(a);
-  } else {
-    auto k = vec ? bwd_kernel<float, true> : bwd_kernel<float, false>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    k<<<grid, block, smem, s>>>(a);
+template <typename IO, bool VEC>
+cudaError_t launch_bwd_io(const BwdArgs& a, cudaStream_t s) {
+  const dim3 grid((unsigned)(a.batch * a.ngroups)), block(32 * a.wpb);
+  const size_t smem = sizeof(BwdTile) * a.wpb;
+  auto k = bwd_kernel<IO, VEC, 2>;
+  if constexpr (!std::is_same<IO, float>::value) {
+    if (a.kmufu == 3) k = bwd_kernel<IO, VEC, 3>;
+    else if (a.kmufu == 4) k = bwd_kernel<IO, VEC, 4>;
   }
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k<<<grid, block, smem, s>>>(a);
   return cudaGetLastError();
 }
 
-size_t bwd_smem_per_warp() { return sizeof(WarpSmem); }
+}  // namespace
+
+cudaError_t launch_bwd(const BwdArgs& a, int io, bool vec, cudaStream_t s) {
+  if (io == 1) return vec ? launch_bwd_io<uint16_t, true>(a, s) : launch_bwd_io<uint16_t, false>(a, s);
+  return vec ? launch_bwd_io<float, true>(a, s) : launch_bwd_io<float, false>(a, s);
+}
 
 cudaError_t launch_bwd_finish(const BwdArgs& a, int io, void* dB, void* dC, float* dA, float* dD,
                               float* ddt_bias, cudaStream_t s) {

@@ -62,8 +62,9 @@ struct BwdArgs {
   int softplus;
   int warps_per_b;
   long long nwarps;
-  int wpb;              // warps per CTA (channels per CTA = 32 * wpb)
+  int wpb;              // warps per CTA (channels per CTA = 16 * wpb)
   int ngroups;          // CTAs per batch row = ceil(warps_per_b / wpb)
+  int kmufu;            // state pairs (of 4 per lane) whose exponential runs on MUFU: 2, 3 or 4
 };
 
 struct DecodeArgs {
