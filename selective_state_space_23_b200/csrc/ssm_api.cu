@@ -190,14 +190,19 @@ FwdPlan plan_fwd(int batch, int dim, int seqlen) {
   return p;
 }
 
-// Launch tuning of the forward kernel (measured on B200 for the 8 x 2048 x 2048 layer; the
-// environment variables override them for experiments): one warp per CTA, and 12 of every 16
-// exponentials per lane and step pair on the MUFU unit (the rest on the FMA-pipe polynomial).
+// Launch tuning of the forward kernel (measured on B200; the environment variables override it
+// for experiments): one warp per CTA.  Exponentials on the MUFU unit per lane and step pair (of
+// 16; the rest use the FMA-pipe polynomial): with fewer than 8 warps per SM (e.g. 8 x 2048
+// channels) every warp is latency-bound and the shortest instruction stream wins, so all 16 go
+// to MUFU; with more warps 14 of 16 balance the MUFU and FMA pipes best (4 x 5120 channels,
+// and the time-split 1 x 256 x 2^20 sequence).
 int fwd_wpb() {
   const int w = env_int("SSM_FWD_WPB", 1);
   return (w == 1 || w == 2 || w == 4) ? w : 1;
 }
-int fwd_kmufu() { return env_int("SSM_FWD_KMUFU", 12); }
+int fwd_kmufu(long long warps) {
+  return env_int("SSM_FWD_KMUFU", warps < 8LL * sm_count() ? 16 : 14);
+}
 
 struct BwdLayout {
   size_t ckpt, part_bc, part_adt, total;
@@ -299,7 +304,8 @@ int ssm_scan_fwd(const void* u, const void* delta, const float* A, const void* B
   const bool vec = (seqlen * es) % 16 == 0 && aligned16(u) && aligned16(delta) && aligned16(z) &&
                    aligned16(out) && aligned16(B) && aligned16(C);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int wpb = fwd_wpb(), km = fwd_kmufu();
+  const int wpb = fwd_wpb();
+  const int km = fwd_kmufu(a.nwarps * (long long)plan.nchunk);
   cudaError_t e;
   if (plan.nchunk > 1) {
     const size_t nch = (size_t)batch * dim;
@@ -394,7 +400,7 @@ int ssm_scan_bwd(const void* u, const void* delta, const float* A, const void* B
     a.lpc = fwd_lpc();
     a.warps_per_b = fwd_warps_per_b(dim);
     a.nwarps = (long long)batch * a.warps_per_b;
-    if ((e = ssm::launch_fwd(a, io_dtype, vec, ssm::kFwdCkpt, fwd_wpb(), fwd_kmufu(), s)) != cudaSuccess)
+    if ((e = ssm::launch_fwd(a, io_dtype, vec, ssm::kFwdCkpt, fwd_wpb(), fwd_kmufu(a.nwarps), s)) != cudaSuccess)
       return cuda_fail(e, "backward state replay pass");
     ck = ck_ws;
   }

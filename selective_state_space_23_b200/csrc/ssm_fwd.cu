@@ -54,13 +54,21 @@ struct Layout {
   static constexpr int kYpStride = LPC == 1 ? 33 : (LPC == 2 ? 34 : 36);
 };
 
-// Per-warp shared memory of one 16-step block.
+// Shared memory of one 16-step block of a warp.
 template <int LPC>
-struct WarpTile {
+struct BlockBuf {
   float4 sB[kBlk * kNS / 4];                          // B_t,n as f32 [step][state]
   float4 sC[kBlk * kNS / 4];                          // C_t,n
   float4 sd[kBlk * Layout<LPC>::kSdStride];           // (Δ_t, Δ_t, Δ_t x_t, Δ_t x_t) per [step][slot]
   float yp[kBlk * Layout<LPC>::kYpStride];            // partial readouts per [step][slot][lane]
+};
+
+// Per-warp shared memory: two block buffers.  While block i runs its time loop out of buffer
+// i mod 2, the lanes fill the other buffer with block i+1's per-step scalars and B/C and read
+// block i-1's partial readouts from it.
+template <int LPC>
+struct WarpTile {
+  BlockBuf<LPC> buf[2];
 };
 
 // Per-step quantities of one lane that do not depend on the state: Ā = 2^(Δ A log2 e) and the
@@ -127,7 +135,7 @@ __device__ __forceinline__ float consume_step(float2 (&hh)[PPL], const StepPrep<
 // step k updates the state.  A step at or beyond nvalid may be prepared from stale tile entries
 // (the index is clamped to the tile) but is never consumed.
 template <bool kPrecise, bool kReadout, int LPC, int KE, int KO>
-__device__ __forceinline__ void state_loop(WarpTile<LPC>& tile, float2 (&hh)[Layout<LPC>::kPPL],
+__device__ __forceinline__ void state_loop(BlockBuf<LPC>& tile, float2 (&hh)[Layout<LPC>::kPPL],
                                            const float2 (&al)[Layout<LPC>::kPPL], int slot, int q,
                                            int nvalid) {
   using Lay = Layout<LPC>;
@@ -157,7 +165,173 @@ __device__ __forceinline__ void state_loop(WarpTile<LPC>& tile, float2 (&hh)[Lay
   }
 }
 
-// Scan of one time chunk by one lane.  KE / KO: MUFU pairs on even / odd steps (the same for every
+// u, delta, z of a lane's owned steps of one block, and the B/C rows it stages.
+template <typename IO, int SPL>
+struct BlockRows {
+  Row<IO, SPL> u, d, z;
+  Row<IO, 8> b, c;
+  __device__ __forceinline__ void zero() {
+    u.zero(); d.zero(); z.zero(); b.zero(); c.zero();
+  }
+};
+
+// What one lane needs to load, prepare and finish the blocks of its chunk.
+template <typename IO, bool VEC, int MODE, int LPC>
+struct ChunkLane {
+  using Lay = Layout<LPC>;
+  static constexpr int SPL = Lay::kSPL;
+  static constexpr bool kPrecise = std::is_same<IO, float>::value;
+  static constexpr bool kReadout = MODE == kFwdOut;
+  using Rows = BlockRows<IO, SPL>;
+  using URow = Row<IO, SPL>;
+
+  const IO* up;
+  const IO* dp;
+  const IO* zp;   // null: no gate
+  const IO* Bp;
+  const IO* Cp;
+  IO* op;
+  int slot, q, bn, bh, t_end;
+  bool bc_live, softplus, act;
+  float bias, Dd;
+  float dlim;  // |Δ| < dlim keeps |Δ A log2 e| <= 126 for every state of the warp
+
+
+  // Rows of the block starting at tb; steps at or beyond t_end read as zero.
+  __device__ __forceinline__ void fetch(Rows& r, int tb) const {
+    const int nv = max(0, min(SPL, t_end - tb - SPL * q));
+    const int nv8 = max(0, min(8, t_end - tb - 8 * bh));
+    if (VEC && nv == SPL) {
+      load_row<IO, SPL, true>(r.u, up + tb, SPL);
+      load_row<IO, SPL, true>(r.d, dp + tb, SPL);
+      if (zp) load_row<IO, SPL, true>(r.z, zp + tb, SPL);
+    } else {
+      load_row<IO, SPL, false>(r.u, up + tb, nv);
+      load_row<IO, SPL, false>(r.d, dp + tb, nv);
+      if (zp) load_row<IO, SPL, false>(r.z, zp + tb, nv);
+    }
+    if (!bc_live) {
+      r.b.zero();
+      r.c.zero();
+    } else if (VEC && nv8 == 8) {
+      load_row<IO, 8, true>(r.b, Bp + tb, 8);
+      if (kReadout) load_row<IO, 8, true>(r.c, Cp + tb, 8);
+    } else {
+      load_row<IO, 8, false>(r.b, Bp + tb, nv8);
+      if (kReadout) load_row<IO, 8, false>(r.c, Cp + tb, nv8);
+    }
+  }
+
+  // Stage B_t,bn and C_t,bn of step 8 bh + j of the block as f32 [step][state].
+  __device__ __forceinline__ void stage_row(float* __restrict__ sB, float* __restrict__ sC,
+                                            const Rows& r, int j) const {
+    sB[(8 * bh + j) * kNS + bn] = r.b.get(j);
+    if (kReadout) sC[(8 * bh + j) * kNS + bn] = r.c.get(j);
+  }
+
+  // Δ and Δx of owned steps j, j+1 into the block's table.  ok stays true while every |Δ| is
+  // below dlim (false for a NaN); the summary pass also sums Δ over the valid owned steps (nown).
+  __device__ __forceinline__ void scalar_pair(float4* __restrict__ sd, const Rows& r, int j, int nown,
+                                              float& dblk, bool& ok) const {
+    const float2 v = add2(make_float2(r.d.get(j), r.d.get(j + 1)), f2(bias));
+    float2 dl = v;
+    if (softplus) {
+      if (kPrecise) dl = make_float2(softplus_precise(v.x), softplus_precise(v.y));
+      else dl = softplus_fast_x2(v);
+    }
+    const float2 dx = mul2(dl, make_float2(r.u.get(j), r.u.get(j + 1)));
+    sd[(SPL * q + j) * Lay::kSdStride + slot] = make_float4(dl.x, dl.x, dx.x, dx.x);
+    sd[(SPL * q + j + 1) * Lay::kSdStride + slot] = make_float4(dl.y, dl.y, dx.y, dx.y);
+    if (MODE == kFwdSummary) dblk += (j < nown ? dl.x : 0.f) + (j + 1 < nown ? dl.y : 0.f);
+    ok = ok && fabsf(dl.x) < dlim && fabsf(dl.y) < dlim;
+  }
+
+  // out of owned steps j, j+1: (Σ of the LPC partial readouts + D x) * silu(z).
+  __device__ __forceinline__ void output_pair(const float* __restrict__ ypb, const URow& u,
+                                              const URow& z, int j, float (&o)[SPL]) const {
+    float yv[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const float* pp = ypb + (SPL * q + j + i) * Lay::kYpStride + slot * LPC;
+      if (LPC == 1) {
+        yv[i] = *pp;
+      } else if (LPC == 2) {
+        const float2 v = *reinterpret_cast<const float2*>(pp);
+        yv[i] = v.x + v.y;
+      } else {
+        const float4 v = *reinterpret_cast<const float4*>(pp);
+        yv[i] = (v.x + v.y) + (v.z + v.w);
+      }
+    }
+    float2 y = fma2(f2(Dd), make_float2(u.get(j), u.get(j + 1)), make_float2(yv[0], yv[1]));
+    if (zp) {
+      const float2 z2 = make_float2(z.get(j), z.get(j + 1));
+      const float2 sg = kPrecise ? make_float2(sigmoid_precise(z2.x), sigmoid_precise(z2.y))
+                                 : sigmoid_fast_x2(z2);
+      y = mul2(y, mul2(z2, sg));
+    }
+    o[j] = y.x;
+    o[j + 1] = y.y;
+  }
+
+  __device__ __forceinline__ void store_out(int t0, const float (&o)[SPL], int nown) const {
+    if (!act || nown <= 0) return;
+    if (VEC && nown == SPL) store_row<IO, SPL, true>(op + t0, o, SPL);
+    else store_row<IO, SPL, false>(op + t0, o, nown);
+  }
+};
+
+// One full block (16 valid steps) with its neighbours' per-step work woven into the time loop:
+// block i+1's Δ, Δx and B/C go into `nxt`, and block i-1's outputs are finished from the partial
+// readouts in `nxt`.  A lane's SPL/2 scalar pairs and SPL/2 output pairs are spread evenly over
+// the 8 two-step iterations, so their MUFU work (softplus, sigmoid) lands between the state
+// steps' exponentials instead of forming a phase of its own.  Work for a block that does not
+// exist (no next / no previous block) runs on zeros or stale entries and is never stored.
+template <bool kPrecise, bool kReadout, int LPC, int KE, int KO, class Lane>
+__device__ __forceinline__ void interleaved_block(
+    const Lane& ln, const BlockBuf<LPC>* __restrict__ cur, float* __restrict__ cur_yp,
+    float* __restrict__ nxt_sB, float* __restrict__ nxt_sC, float4* __restrict__ nxt_sd,
+    const float* __restrict__ nxt_yp, float2 (&hh)[Layout<LPC>::kPPL],
+    const float2 (&al)[Layout<LPC>::kPPL], const typename Lane::Rows& rn, int nown_next,
+    const typename Lane::URow& pu, const typename Lane::URow& pz, float (&o)[Layout<LPC>::kSPL],
+    float& dblk, bool& ok) {
+  using Lay = Layout<LPC>;
+  constexpr int SPL = Lay::kSPL, PPL = Lay::kPPL;
+  constexpr int S8 = 8 / PPL;  // iterations per scalar (and per output) pair
+  const float4* bq = cur->sB + SPL * ln.q / 4;
+  const float4* cq = cur->sC + SPL * ln.q / 4;
+  const float4* sdp = cur->sd + ln.slot;
+  float* yp = cur_yp + ln.slot * LPC + ln.q;
+  // two steps prepared ahead: steps k+2, k+3 are prepared while k, k+1 update the state
+  StepPrep<PPL> p0, p1;
+  prepare_step<kPrecise, PPL, KE>(p0, al, sdp[0], bq);
+  prepare_step<kPrecise, PPL, KO>(p1, al, sdp[Lay::kSdStride], bq + 4);
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    const int k = 2 * m;
+    StepPrep<PPL> q0, q1;
+    if (m < 7)
+      prepare_step<kPrecise, PPL, KE>(q0, al, sdp[(k + 2) * Lay::kSdStride], bq + (k + 2) * 4);
+    const float y0 = consume_step<kReadout, PPL>(hh, p0, cq + k * 4);
+    if (m < 7)
+      prepare_step<kPrecise, PPL, KO>(q1, al, sdp[(k + 3) * Lay::kSdStride], bq + (k + 3) * 4);
+    const float y1 = consume_step<kReadout, PPL>(hh, p1, cq + (k + 1) * 4);
+    p0 = q0;
+    p1 = q1;
+    if (kReadout) {
+      yp[k * Lay::kYpStride] = y0;
+      yp[(k + 1) * Lay::kYpStride] = y1;
+    }
+    ln.stage_row(nxt_sB, nxt_sC, rn, m);
+    if (m % S8 == S8 / 2) ln.scalar_pair(nxt_sd, rn, 2 * (m / S8), nown_next, dblk, ok);
+    if (kReadout && m % S8 == 0) ln.output_pair(nxt_yp, pu, pz, 2 * (m / S8), o);
+  }
+}
+
+// Scan of one time chunk by one lane.  Blocks are processed as a three-stage pipeline: while
+// block i updates the state, block i+1's per-step scalars and B/C are prepared and block i-1's
+// outputs are finished; block i+2's rows are in flight from HBM.  A partial last block runs the
+// same stages one after another.  KE / KO: MUFU pairs on even / odd steps (the same for every
 // lane, so the lanes of a channel run identical instructions).
 template <typename IO, bool VEC, int MODE, int LPC, int KE, int KO>
 __device__ __forceinline__ void run_chunk(const FwdArgs& a, WarpTile<LPC>& tile,
@@ -166,50 +340,35 @@ __device__ __forceinline__ void run_chunk(const FwdArgs& a, WarpTile<LPC>& tile,
                                           float bias, int lane, int slot, int q, int b, bool act,
                                           long long ch, int t_begin, int t_end, bool last_chunk) {
   using Lay = Layout<LPC>;
+  using Lane = ChunkLane<IO, VEC, MODE, LPC>;
   constexpr int SPL = Lay::kSPL, PPL = Lay::kPPL;
-  constexpr bool kPrecise = std::is_same<IO, float>::value;
-  constexpr bool kReadout = MODE == kFwdOut;
+  constexpr bool kPrecise = Lane::kPrecise;
+  constexpr bool kReadout = Lane::kReadout;
   const int L = a.L, N = a.N;
-  const long long row = ch * (long long)L + SPL * q;     // this lane's steps of each block
-  const IO* up = reinterpret_cast<const IO*>(a.u) + row;
-  const IO* dp = reinterpret_cast<const IO*>(a.delta) + row;
-  const IO* zp = (kReadout && a.z) ? reinterpret_cast<const IO*>(a.z) + row : nullptr;
-  IO* op = kReadout ? reinterpret_cast<IO*>(a.out) + row : nullptr;
-  // B/C staging: lane stages state row bn, steps [8 bh, 8 bh + 8) of each block
-  const int bn = lane >> 1, bh = lane & 1;
-  const bool bc_live = bn < N;
-  const long long bcrow = ((long long)b * N + (bc_live ? bn : 0)) * L + 8 * bh;
-  const IO* Bp = reinterpret_cast<const IO*>(a.B) + bcrow;
-  const IO* Cp = reinterpret_cast<const IO*>(a.C) + bcrow;
-  const int nblk_total = (L + kBlk - 1) / kBlk;
-  float* sBw = reinterpret_cast<float*>(tile.sB);
-  float* sCw = reinterpret_cast<float*>(tile.sC);
 
-  Row<IO, SPL> nu, nd, nz;
-  Row<IO, 8> nb, nc;
-  auto fetch = [&](int tb) {
-    const int nv = max(0, min(SPL, t_end - tb - SPL * q));
-    const int nv8 = max(0, min(8, t_end - tb - 8 * bh));
-    if (VEC && nv == SPL) {
-      load_row<IO, SPL, true>(nu, up + tb, SPL);
-      load_row<IO, SPL, true>(nd, dp + tb, SPL);
-      if (zp) load_row<IO, SPL, true>(nz, zp + tb, SPL);
-    } else {
-      load_row<IO, SPL, false>(nu, up + tb, nv);
-      load_row<IO, SPL, false>(nd, dp + tb, nv);
-      if (zp) load_row<IO, SPL, false>(nz, zp + tb, nv);
-    }
-    if (!bc_live) {
-      nb.zero();
-      nc.zero();
-    } else if (VEC && nv8 == 8) {
-      load_row<IO, 8, true>(nb, Bp + tb, 8);
-      if (kReadout) load_row<IO, 8, true>(nc, Cp + tb, 8);
-    } else {
-      load_row<IO, 8, false>(nb, Bp + tb, nv8);
-      if (kReadout) load_row<IO, 8, false>(nc, Cp + tb, nv8);
-    }
-  };
+  Lane ln;
+  const long long row = ch * (long long)L + SPL * q;     // this lane's steps of each block
+  ln.up = reinterpret_cast<const IO*>(a.u) + row;
+  ln.dp = reinterpret_cast<const IO*>(a.delta) + row;
+  ln.zp = (kReadout && a.z) ? reinterpret_cast<const IO*>(a.z) + row : nullptr;
+  ln.op = kReadout ? reinterpret_cast<IO*>(a.out) + row : nullptr;
+  // B/C staging: lane stages state row bn, steps [8 bh, 8 bh + 8) of each block
+  ln.bn = lane >> 1;
+  ln.bh = lane & 1;
+  ln.bc_live = ln.bn < N;
+  const long long bcrow = ((long long)b * N + (ln.bc_live ? ln.bn : 0)) * L + 8 * ln.bh;
+  ln.Bp = reinterpret_cast<const IO*>(a.B) + bcrow;
+  ln.Cp = reinterpret_cast<const IO*>(a.C) + bcrow;
+  ln.slot = slot;
+  ln.q = q;
+  ln.t_end = t_end;
+  ln.softplus = a.softplus != 0;
+  ln.act = act;
+  ln.bias = bias;
+  ln.Dd = Dd;
+  const int nblk_total = (L + kBlk - 1) / kBlk;
+  const int nblk = (t_end - t_begin + kBlk - 1) / kBlk;
+  const auto own = [&](int nvalid) { return max(0, min(SPL, nvalid - SPL * q)); };
 
   // largest |A log2 e| of the warp's states: the FMA-pipe exponential needs |Δ A log2 e| <= 126
   float amax = 0.f;
@@ -217,39 +376,53 @@ __device__ __forceinline__ void run_chunk(const FwdArgs& a, WarpTile<LPC>& tile,
   for (int j = 0; j < PPL; ++j) amax = fmaxf(amax, fmaxf(fabsf(al[j].x), fabsf(al[j].y)));
 #pragma unroll
   for (int m = 16; m >= 1; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
+  // FLT_MAX when every A is zero (then only an infinite or NaN Δ leaves the range); 0 when some
+  // A is infinite (the block always takes the MUFU path)
+  ln.dlim = amax > 0.f ? 126.f / amax : 3.402823466e38f;
 
-  fetch(t_begin);
   float dsum = 0.f, dcomp = 0.f;  // Kahan-compensated ΣΔ of this lane's steps (summary pass)
-  for (int t0 = t_begin; t0 < t_end; t0 += kBlk) {
-    const int nvalid = min(kBlk, t_end - t0);
-    const int nown = max(0, min(SPL, nvalid - SPL * q));
-    const Row<IO, SPL> cu = nu, cd = nd, cz = nz;
-    const Row<IO, 8> cb = nb, cc = nc;
-    if (t0 + kBlk < t_end) fetch(t0 + kBlk);
+  const auto kahan = [&](float x) {
+    const float yk = x - dcomp;
+    const float tk = dsum + yk;
+    dcomp = (tk - dsum) - yk;
+    dsum = tk;
+  };
 
-    __syncwarp();  // the previous block's tile is no longer read
-    // stage B/C as f32 [step][state]
+  // prologue: block 0's scalars and B/C, block 1's rows in flight
+  typename Lane::Rows rn, rf;
+  typename Lane::URow u_cur, z_cur, pu, pz;
+  bool safe = true;
+  if (nblk > 0) {
+    ln.fetch(rn, t_begin);
+    float dblk = 0.f;
+    bool ok = true;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      sBw[(8 * bh + j) * kNS + bn] = cb.get(j);
-      if (kReadout) sCw[(8 * bh + j) * kNS + bn] = cc.get(j);
-    }
-    float dblk = 0.f, dabs = 0.f;  // dabs: largest |Δ| of this lane's steps (NaN propagates)
+    for (int j = 0; j < 8; ++j)
+      ln.stage_row(reinterpret_cast<float*>(tile.buf[0].sB), reinterpret_cast<float*>(tile.buf[0].sC),
+                   rn, j);
 #pragma unroll
-    for (int j = 0; j < SPL; j += 2) {
-      const float2 v = add2(make_float2(cd.get(j), cd.get(j + 1)), f2(bias));
-      float2 dl = v;
-      if (a.softplus) {
-        if (kPrecise) dl = make_float2(softplus_precise(v.x), softplus_precise(v.y));
-        else dl = softplus_fast_x2(v);
-      }
-      const float2 dx = mul2(dl, make_float2(cu.get(j), cu.get(j + 1)));
-      tile.sd[(SPL * q + j) * Lay::kSdStride + slot] = make_float4(dl.x, dl.x, dx.x, dx.x);
-      tile.sd[(SPL * q + j + 1) * Lay::kSdStride + slot] = make_float4(dl.y, dl.y, dx.y, dx.y);
-      dblk += (j < nown ? dl.x : 0.f) + (j + 1 < nown ? dl.y : 0.f);
-      dabs = fmaxf(dabs, fmaxf(fabsf(dl.x), fabsf(dl.y)));
-      if (dl.x != dl.x || dl.y != dl.y) dabs = __int_as_float(0x7f800000);  // NaN: take the checked path
-    }
+    for (int j = 0; j < SPL; j += 2)
+      ln.scalar_pair(tile.buf[0].sd, rn, j, own(min(kBlk, t_end - t_begin)), dblk, ok);
+    u_cur = rn.u;
+    z_cur = rn.z;
+    if (nblk > 1) ln.fetch(rn, t_begin + kBlk);
+    else rn.zero();
+    if (MODE == kFwdSummary) kahan(dblk);
+    __syncwarp();
+    safe = __all_sync(0xffffffffu, ok);
+  }
+  pu.zero();
+  pz.zero();
+
+#pragma unroll 1
+  for (int i = 0; i < nblk; ++i) {
+    const int t0 = t_begin + i * kBlk;
+    const int nvalid = min(kBlk, t_end - t0);
+    BlockBuf<LPC>& cur = tile.buf[i & 1];
+    BlockBuf<LPC>& nxt = tile.buf[(i & 1) ^ 1];
+    const bool has_next = i + 1 < nblk, has_prev = i > 0;
+    if (i + 2 < nblk) ln.fetch(rf, t0 + 2 * kBlk);
+    else rf.zero();
     if (MODE != kFwdSummary && a.ckpt && act) {
       float* cp = a.ckpt + (ch * nblk_total + t0 / kBlk) * N;
 #pragma unroll
@@ -259,53 +432,51 @@ __device__ __forceinline__ void run_chunk(const FwdArgs& a, WarpTile<LPC>& tile,
         if (n0 + 1 < N) cp[n0 + 1] = hh[j].y;
       }
     }
-    __syncwarp();
-
-    const bool safe = !__any_sync(0xffffffffu, !(amax * dabs <= 126.f));
-    if (kPrecise || !safe)
-      state_loop<kPrecise, kReadout, LPC, PPL, PPL>(tile, hh, al, slot, q, nvalid);
-    else
-      state_loop<kPrecise, kReadout, LPC, KE, KO>(tile, hh, al, slot, q, nvalid);
-
-    if (MODE == kFwdSummary) {
-      const float yk = dblk - dcomp;
-      const float tk = dsum + yk;
-      dcomp = (tk - dsum) - yk;
-      dsum = tk;
-    } else if (kReadout) {
-      __syncwarp();
-      float o[SPL];
+    const int nown_next = has_next ? own(min(kBlk, t_end - t0 - kBlk)) : 0;
+    float o[SPL];
+    float dblk = 0.f;
+    bool ok = true;
+    if (nvalid == kBlk) {
+      float* nsB = reinterpret_cast<float*>(nxt.sB);
+      float* nsC = reinterpret_cast<float*>(nxt.sC);
+      if (kPrecise || !safe)
+        interleaved_block<kPrecise, kReadout, LPC, PPL, PPL>(ln, &cur, cur.yp, nsB, nsC, nxt.sd,
+                                                             nxt.yp, hh, al, rn, nown_next, pu, pz,
+                                                             o, dblk, ok);
+      else
+        interleaved_block<kPrecise, kReadout, LPC, KE, KO>(ln, &cur, cur.yp, nsB, nsC, nxt.sd,
+                                                           nxt.yp, hh, al, rn, nown_next, pu, pz,
+                                                           o, dblk, ok);
+    } else {
+      // partial (last) block: the three stages one after another
+      if (kReadout && has_prev) {
 #pragma unroll
-      for (int j = 0; j < SPL; j += 2) {
-        float yv[2];
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const float* pp = tile.yp + (SPL * q + j + i) * Lay::kYpStride + slot * LPC;
-          if (LPC == 1) {
-            yv[i] = *pp;
-          } else if (LPC == 2) {
-            const float2 v = *reinterpret_cast<const float2*>(pp);
-            yv[i] = v.x + v.y;
-          } else {
-            const float4 v = *reinterpret_cast<const float4*>(pp);
-            yv[i] = (v.x + v.y) + (v.z + v.w);
-          }
-        }
-        float2 y = fma2(f2(Dd), make_float2(cu.get(j), cu.get(j + 1)), make_float2(yv[0], yv[1]));
-        if (zp) {
-          const float2 z2 = make_float2(cz.get(j), cz.get(j + 1));
-          const float2 sg = kPrecise ? make_float2(sigmoid_precise(z2.x), sigmoid_precise(z2.y))
-                                     : sigmoid_fast_x2(z2);
-          y = mul2(y, mul2(z2, sg));
-        }
-        o[j] = y.x;
-        o[j + 1] = y.y;
+        for (int j = 0; j < SPL; j += 2) ln.output_pair(nxt.yp, pu, pz, j, o);
       }
-      if (act && nown > 0) {
-        if (VEC && nown == SPL) store_row<IO, SPL, true>(op + t0, o, SPL);
-        else store_row<IO, SPL, false>(op + t0, o, nown);
-      }
+      if (kPrecise || !safe)
+        state_loop<kPrecise, kReadout, LPC, PPL, PPL>(cur, hh, al, slot, q, nvalid);
+      else
+        state_loop<kPrecise, kReadout, LPC, KE, KO>(cur, hh, al, slot, q, nvalid);
+      // a partial block is the last one: there is no next block to prepare
     }
+    __syncwarp();  // this block's partial readouts and the next block's table are complete
+    if (kReadout && has_prev) ln.store_out(t0 - kBlk, o, SPL);  // blocks before the last are full
+    if (MODE == kFwdSummary) kahan(dblk);
+    safe = __all_sync(0xffffffffu, ok);
+    pu = u_cur;
+    pz = z_cur;
+    u_cur = rn.u;
+    z_cur = rn.z;
+    rn = rf;
+  }
+
+  // epilogue: the last block's outputs (its u, z are now in pu, pz)
+  if (kReadout && nblk > 0) {
+    const int tl = t_begin + (nblk - 1) * kBlk;
+    float o[SPL];
+#pragma unroll
+    for (int j = 0; j < SPL; j += 2) ln.output_pair(tile.buf[(nblk - 1) & 1].yp, pu, pz, j, o);
+    ln.store_out(tl, o, own(t_end - tl));
   }
 
   if (MODE == kFwdSummary) {

@@ -86,6 +86,37 @@ def test_bf16_medium_full():
     assert_close(out, run_oracle(x)["out"], torch.bfloat16, "out")
 
 
+@pytest.mark.parametrize("kmufu", [8, 10, 12, 14, 16])
+def test_every_exponential_split(monkeypatch, kmufu):
+    """Each split of the exponentials between MUFU and the FMA-pipe polynomial (the default
+    depends on the warps per SM), on a ragged length so full and partial blocks both run."""
+    monkeypatch.setenv("SSM_FWD_KMUFU", str(kmufu))
+    w = workload("mamba370m_fwd", batch=2, dim=200, seqlen=1000)
+    x = make_inputs(w, seed=11, with_h0=True)
+    out, hL = run_gpu(on_dev(x), return_final_state=True)
+    ref = run_oracle(x)
+    assert_close(out, ref["out"], torch.bfloat16, "out")
+    assert_close(hL, ref["hL"], torch.bfloat16, "hL")
+
+
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("lpc", [1, 2, 4])
+def test_lanes_per_channel(monkeypatch, io, lpc):
+    """1, 2 or 4 lanes per channel (state split across lanes), with the time split too."""
+    monkeypatch.setenv("SSM_FWD_LPC", str(lpc))
+    w = workload("tiny_f32", batch=2, dim=40, seqlen=301, dstate=16, io_dtype=io)
+    x = make_inputs(w, seed=12, with_h0=True)
+    out, hL = run_gpu(on_dev(x), return_final_state=True)
+    ref = run_oracle(x)
+    assert_close(out, ref["out"], io, "out")
+    assert_close(hL, ref["hL"], torch.float32 if io == torch.float32 else io, "hL")
+    monkeypatch.setenv("SSM_FWD_SPLIT", "3")
+    nws = ssm.fwd_workspace_bytes(2, 40, 301, 16, io)
+    ws = torch.empty(nws, dtype=torch.uint8, device=DEV)
+    out2 = run_gpu(on_dev(x), workspace=ws)
+    assert_close(out2, ref["out"], io, "out (time split)")
+
+
 def test_positive_A_entries_use_the_exact_exponential():
     w = workload("mamba370m_fwd", batch=1, dim=64, seqlen=256)
     x = make_inputs(w, seed=4)
