@@ -58,6 +58,11 @@ def compulsory_bytes(w) -> int:
     return 4 * x + 2 * bc + w.dim * w.dstate * 4 + 2 * w.dim * 4
 
 
+def compulsory_bytes_shape(b, d, L, N, es=2) -> int:
+    """u, delta, z, out + B, C + per-channel parameters (A taken as [dim])."""
+    return 4 * b * d * L * es + 2 * b * N * L * es + 3 * d * 4
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -283,6 +288,20 @@ def bench_extras(dev):
     out["mamba2p8b_train"] = {"shape": "4x5120x2048 N16 bf16", "fwd_ms": ms_f,
                               "fwd_bwd_ms": ms_tr, "tokens_per_s": b * L / (ms_tr * 1e-3)}
     del u, de, z, dout, ws
+    torch.cuda.empty_cache()
+
+    # scalar decay (one rate per channel) on the Mamba-370m-shaped layer
+    b, d, L = 8, 2048, 2048
+    u, de, z = rnd((b, d, L)), rnd((b, d, L), 0.5), rnd((b, d, L))
+    B, C = rnd((b, N, L)), rnd((b, N, L))
+    _, D, bias = prm(d, N, 1e-3, 1e-1)
+    A1 = -(torch.rand(d, device=dev, generator=g) * 15.0 + 1.0)
+    o = torch.empty_like(u)
+    ms = timeit(lambda: ssm.ssm_scan_fwd_scalar_a(u, de, A1, B, C, D=D, z=z, dt_bias=bias, out=o), 20)
+    out["scalar_decay_fwd"] = {"shape": "8x2048x2048 N16 bf16, A [dim]", "fwd_ms": ms,
+                               "tokens_per_s": b * L / (ms * 1e-3),
+                               "hbm_gbs": compulsory_bytes_shape(b, d, L, N) / (ms * 1e-3) / 1e9}
+    del u, de, z, B, C, o
     torch.cuda.empty_cache()
 
     # long sequence

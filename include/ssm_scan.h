@@ -142,6 +142,37 @@ SSM_API int ssm_scan_bwd(const void* u, const void* delta, const float* A, const
                  float* ddt_bias, float* dh0, void* workspace, size_t workspace_bytes,
                  int batch, int dim, int seqlen, int dstate, int io_dtype, void* stream);
 
+/*
+ * Scalar decay: one rate A_d per channel shared by its N states (the restriction of the
+ * transition to a scalar that the "2024 Reading List: Neural Network" page notes for Mamba-2,
+ * section on state-space models).  The recurrence is the one above with A[d][n] = A_d:
+ *   Ā_t = exp(Δ_t A_d) (one exponential per channel and step),  h_t = Ā_t h_{t-1} + Δ_t B_t x_t,
+ *   y_t = C_t . h_t + D_d x_t,  out_t = y_t * silu(z_t).
+ * Arguments, layouts, ownership and errors are those of ssm_scan_fwd / ssm_scan_bwd except:
+ *   A   [dim] f32 (not [dim][dstate]);   dA (backward)  [dim] f32 = sum over n of dL/dA[d][n].
+ * The backward needs ssm_scan_bwd_scalar_a_workspace_size() bytes of workspace (256-byte
+ * aligned): A broadcast to [dim][dstate] and the per-state dA, followed by the workspace of
+ * ssm_scan_bwd for the same shape.  Checkpoints of ssm_scan_fwd_scalar_a feed the backward.
+ */
+SSM_API size_t ssm_scan_fwd_scalar_a_workspace_size(int batch, int dim, int seqlen, int dstate,
+                                                    int io_dtype);
+SSM_API int ssm_scan_fwd_scalar_a(const void* u, const void* delta, const float* A, const void* B,
+                                  const void* C, const float* D, const void* z,
+                                  const float* dt_bias, int delta_softplus, const float* h0,
+                                  float* hL, void* out, float* ckpt, void* workspace,
+                                  size_t workspace_bytes, int batch, int dim, int seqlen,
+                                  int dstate, int io_dtype, void* stream);
+SSM_API size_t ssm_scan_bwd_scalar_a_workspace_size(int batch, int dim, int seqlen, int dstate,
+                                                    int io_dtype, int have_ckpt);
+SSM_API int ssm_scan_bwd_scalar_a(const void* u, const void* delta, const float* A, const void* B,
+                                  const void* C, const float* D, const void* z,
+                                  const float* dt_bias, int delta_softplus, const float* h0,
+                                  const void* dout, const float* dhL, const float* ckpt, void* du,
+                                  void* ddelta, float* dA, void* dB, void* dC, float* dD, void* dz,
+                                  float* ddt_bias, float* dh0, void* workspace,
+                                  size_t workspace_bytes, int batch, int dim, int seqlen,
+                                  int dstate, int io_dtype, void* stream);
+
 /* Size of the static scratch array used by ssm_scan_fwd_noalloc (8 MiB per GPU). */
 #define SSM_NOALLOC_SCRATCH_BYTES (8u << 20)
 

@@ -16,7 +16,8 @@ import torch
 from . import _abi
 from ._abi import CKPT_STEPS, MAX_DSTATE
 
-__all__ = ["ssm_scan_fwd", "ssm_scan_bwd", "ssm_state_update", "fwd_workspace_bytes",
+__all__ = ["ssm_scan_fwd", "ssm_scan_bwd", "ssm_scan_fwd_scalar_a", "ssm_scan_bwd_scalar_a",
+           "ssm_state_update", "fwd_workspace_bytes",
            "bwd_workspace_bytes", "CKPT_STEPS", "MAX_DSTATE", "library_path"]
 
 _IO = {torch.float32: _abi.SSM_F32, torch.bfloat16: _abi.SSM_BF16}
@@ -81,19 +82,16 @@ def _workspace(nbytes, device, given):
     return torch.empty(nbytes, dtype=torch.uint8, device=device)
 
 
-def ssm_scan_fwd(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=True, h0=None,
-                 return_final_state=False, return_ckpt=False, out=None, workspace=None):
-    """Forward scan.  u, delta, z: [batch, dim, L]; B, C: [batch, N, L] (io dtype f32 or bf16);
-    A: [dim, N] f32; D, dt_bias: [dim] f32; h0: [batch, dim, N] f32.
-    Returns out, or a tuple (out, hL?, ckpt?) when those are requested."""
+def _scan_fwd(entry, u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, return_final_state,
+              return_ckpt, out, workspace, scalar_a):
     dev = u.device
     batch, dim, L = u.shape
-    N = A.shape[-1]
+    N = B.shape[1]
     io = u.dtype
     code = _io_code(io)
     _need(u, "u", (batch, dim, L), io, dev)
     _need(delta, "delta", (batch, dim, L), io, dev)
-    _need(A, "A", (dim, N), torch.float32, dev)
+    _need(A, "A", (dim,) if scalar_a else (dim, N), torch.float32, dev)
     _need(B, "B", (batch, N, L), io, dev)
     _need(C, "C", (batch, N, L), io, dev)
     _opt(D, "D", (dim,), torch.float32, dev)
@@ -107,11 +105,11 @@ def ssm_scan_fwd(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta_softplus
     nblk = (L + CKPT_STEPS - 1) // CKPT_STEPS
     ckpt = torch.empty((batch, dim, nblk, N), dtype=torch.float32, device=dev) if return_ckpt else None
     ws = _workspace(fwd_workspace_bytes(batch, dim, L, N, io), dev, workspace)
-    rc = _abi.lib().ssm_scan_fwd(
+    rc = getattr(_abi.lib(), entry)(
         _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias),
         int(bool(delta_softplus)), _ptr(h0), _ptr(hL), _ptr(out), _ptr(ckpt), _ptr(ws),
         0 if ws is None else ws.numel(), batch, dim, L, N, code, _stream(dev))
-    _abi.check(rc, "ssm_scan_fwd")
+    _abi.check(rc, entry)
     if not return_final_state and not return_ckpt:
         return out
     res = (out,)
@@ -122,18 +120,34 @@ def ssm_scan_fwd(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta_softplus
     return res
 
 
-def ssm_scan_bwd(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None, delta_softplus=True,
-                 h0=None, dhL=None, ckpt=None, workspace=None, need=None):
-    """Gradients of :func:`ssm_scan_fwd`.  Returns a dict with du, ddelta, dA, dB, dC, dD, dz,
-    ddt_bias, dh0 (entries are None when the matching input is absent or not in ``need``)."""
+def ssm_scan_fwd(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=True, h0=None,
+                 return_final_state=False, return_ckpt=False, out=None, workspace=None):
+    """Forward scan.  u, delta, z: [batch, dim, L]; B, C: [batch, N, L] (io dtype f32 or bf16);
+    A: [dim, N] f32; D, dt_bias: [dim] f32; h0: [batch, dim, N] f32.
+    Returns out, or a tuple (out, hL?, ckpt?) when those are requested."""
+    return _scan_fwd("ssm_scan_fwd", u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0,
+                     return_final_state, return_ckpt, out, workspace, False)
+
+
+def ssm_scan_fwd_scalar_a(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=True,
+                          h0=None, return_final_state=False, return_ckpt=False, out=None,
+                          workspace=None):
+    """Forward scan with one decay rate per channel: as :func:`ssm_scan_fwd` with A [dim] f32."""
+    return _scan_fwd("ssm_scan_fwd_scalar_a", u, delta, A, B, C, D, z, dt_bias, delta_softplus,
+                     h0, return_final_state, return_ckpt, out, workspace, True)
+
+
+def _scan_bwd(entry, u, delta, A, B, C, dout, D, z, dt_bias, delta_softplus, h0, dhL, ckpt,
+              workspace, need, scalar_a):
     dev = u.device
     batch, dim, L = u.shape
-    N = A.shape[-1]
+    N = B.shape[1]
     io = u.dtype
     code = _io_code(io)
     _need(u, "u", (batch, dim, L), io, dev)
     _need(delta, "delta", (batch, dim, L), io, dev)
-    _need(A, "A", (dim, N), torch.float32, dev)
+    a_shape = (dim,) if scalar_a else (dim, N)
+    _need(A, "A", a_shape, torch.float32, dev)
     _need(B, "B", (batch, N, L), io, dev)
     _need(C, "C", (batch, N, L), io, dev)
     _need(dout, "dout", (batch, dim, L), io, dev)
@@ -153,20 +167,38 @@ def ssm_scan_bwd(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None, delta_so
         "dz": e((batch, dim, L), io) if ("dz" in want and z is not None) else None,
         "dB": e((batch, N, L), io) if "dB" in want else None,
         "dC": e((batch, N, L), io) if "dC" in want else None,
-        "dA": e((dim, N), torch.float32) if "dA" in want else None,
+        "dA": e(a_shape, torch.float32) if "dA" in want else None,
         "dD": e((dim,), torch.float32) if "dD" in want else None,
         "ddt_bias": e((dim,), torch.float32) if "ddt_bias" in want else None,
         "dh0": e((batch, dim, N), torch.float32) if "dh0" in want else None,
     }
-    ws = _workspace(bwd_workspace_bytes(batch, dim, L, N, io, ckpt is not None), dev, workspace)
-    rc = _abi.lib().ssm_scan_bwd(
+    size_fn = getattr(_abi.lib(), entry + "_workspace_size")
+    nws = int(size_fn(batch, dim, L, N, code, int(ckpt is not None)))
+    ws = _workspace(nws, dev, workspace)
+    rc = getattr(_abi.lib(), entry)(
         _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias),
         int(bool(delta_softplus)), _ptr(h0), _ptr(dout), _ptr(dhL), _ptr(ckpt),
         _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]),
         _ptr(g["dD"]), _ptr(g["dz"]), _ptr(g["ddt_bias"]), _ptr(g["dh0"]),
         _ptr(ws), 0 if ws is None else ws.numel(), batch, dim, L, N, code, _stream(dev))
-    _abi.check(rc, "ssm_scan_bwd")
+    _abi.check(rc, entry)
     return g
+
+
+def ssm_scan_bwd(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None, delta_softplus=True,
+                 h0=None, dhL=None, ckpt=None, workspace=None, need=None):
+    """Gradients of :func:`ssm_scan_fwd`.  Returns a dict with du, ddelta, dA, dB, dC, dD, dz,
+    ddt_bias, dh0 (entries are None when the matching input is absent or not in ``need``)."""
+    return _scan_bwd("ssm_scan_bwd", u, delta, A, B, C, dout, D, z, dt_bias, delta_softplus, h0,
+                     dhL, ckpt, workspace, need, False)
+
+
+def ssm_scan_bwd_scalar_a(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None,
+                          delta_softplus=True, h0=None, dhL=None, ckpt=None, workspace=None,
+                          need=None):
+    """Gradients of :func:`ssm_scan_fwd_scalar_a` (dA is [dim])."""
+    return _scan_bwd("ssm_scan_bwd_scalar_a", u, delta, A, B, C, dout, D, z, dt_bias,
+                     delta_softplus, h0, dhL, ckpt, workspace, need, True)
 
 
 def ssm_state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=True,

@@ -256,11 +256,16 @@ size_t ssm_scan_fwd_workspace_size(int batch, int dim, int seqlen, int dstate, i
   return plan_fwd(batch, dim, seqlen).ws_bytes;
 }
 
-int ssm_scan_fwd(const void* u, const void* delta, const float* A, const void* B, const void* C,
-                 const float* D, const void* z, const float* dt_bias, int delta_softplus,
-                 const float* h0, float* hL, void* out, float* ckpt, void* workspace,
-                 size_t workspace_bytes, int batch, int dim, int seqlen, int dstate,
-                 int io_dtype, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Forward scan; scalar_a: A is [dim] (one decay rate per channel) instead of [dim][dstate].
+int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* B, const void* C,
+                  const float* D, const void* z, const float* dt_bias, int delta_softplus,
+                  const float* h0, float* hL, void* out, float* ckpt, void* workspace,
+                  size_t workspace_bytes, int batch, int dim, int seqlen, int dstate,
+                  int io_dtype, void* stream, bool scalar_a) {
   g_err[0] = 0;
   TRY(check_dims(batch, dim, seqlen, dstate, io_dtype));
   const size_t es = esize(io_dtype);
@@ -270,7 +275,7 @@ int ssm_scan_fwd(const void* u, const void* delta, const float* A, const void* B
   const size_t nblk = (seqlen + ssm::kBlk - 1) / ssm::kBlk;
   TRY(check_ptr(u, nx, es, "u"));
   TRY(check_ptr(delta, nx, es, "delta"));
-  TRY(check_ptr(A, (size_t)dim * dstate * 4, 4, "A"));
+  TRY(check_ptr(A, (size_t)dim * (scalar_a ? 1 : dstate) * 4, 4, "A"));
   TRY(check_ptr(B, nbc, es, "B"));
   TRY(check_ptr(C, nbc, es, "C"));
   TRY(check_ptr(out, nx, es, "out"));
@@ -298,8 +303,9 @@ int ssm_scan_fwd(const void* u, const void* delta, const float* A, const void* B
   a.batch = batch; a.dim = dim; a.L = seqlen; a.N = dstate;
   a.chunk_len = plan.chunk_len; a.nchunk = plan.nchunk;
   a.softplus = delta_softplus ? 1 : 0;
-  a.lpc = fwd_lpc();
-  a.warps_per_b = fwd_warps_per_b(dim);
+  a.scalar_a = scalar_a ? 1 : 0;
+  a.lpc = scalar_a ? 2 : fwd_lpc();
+  a.warps_per_b = (dim + 32 / a.lpc - 1) / (32 / a.lpc);
   a.nwarps = (long long)batch * a.warps_per_b;
   const bool vec = (seqlen * es) % 16 == 0 && aligned16(u) && aligned16(delta) && aligned16(z) &&
                    aligned16(out) && aligned16(B) && aligned16(C);
@@ -325,6 +331,52 @@ int ssm_scan_fwd(const void* u, const void* delta, const float* A, const void* B
   if ((e = ssm::launch_fwd(a, io_dtype, vec, ssm::kFwdOut, wpb, km, s)) != cudaSuccess)
     return cuda_fail(e, "forward pass");
   return SSM_OK;
+}
+
+// A[d] copied to every state: Af[d][n] = A[d].
+__global__ void broadcast_a_kernel(const float* __restrict__ A, float* __restrict__ Af, int dim,
+                                   int N) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < (long long)dim * N) Af[i] = A[i / N];
+}
+
+// dA[d] = sum over n of dAf[d][n], in the order n = 0 .. N-1.
+__global__ void reduce_da_kernel(const float* __restrict__ dAf, float* __restrict__ dA, int dim,
+                                 int N) {
+  const int d = blockIdx.x * blockDim.x + threadIdx.x;
+  if (d >= dim) return;
+  float acc = 0.f;
+  for (int n = 0; n < N; ++n) acc += dAf[(long long)d * N + n];
+  dA[d] = acc;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ssm_scan_fwd(const void* u, const void* delta, const float* A, const void* B, const void* C,
+                 const float* D, const void* z, const float* dt_bias, int delta_softplus,
+                 const float* h0, float* hL, void* out, float* ckpt, void* workspace,
+                 size_t workspace_bytes, int batch, int dim, int seqlen, int dstate,
+                 int io_dtype, void* stream) {
+  return scan_fwd_impl(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, hL, out, ckpt,
+                       workspace, workspace_bytes, batch, dim, seqlen, dstate, io_dtype, stream,
+                       false);
+}
+
+size_t ssm_scan_fwd_scalar_a_workspace_size(int batch, int dim, int seqlen, int dstate,
+                                            int io_dtype) {
+  return ssm_scan_fwd_workspace_size(batch, dim, seqlen, dstate, io_dtype);
+}
+
+int ssm_scan_fwd_scalar_a(const void* u, const void* delta, const float* A, const void* B,
+                          const void* C, const float* D, const void* z, const float* dt_bias,
+                          int delta_softplus, const float* h0, float* hL, void* out, float* ckpt,
+                          void* workspace, size_t workspace_bytes, int batch, int dim, int seqlen,
+                          int dstate, int io_dtype, void* stream) {
+  return scan_fwd_impl(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, hL, out, ckpt,
+                       workspace, workspace_bytes, batch, dim, seqlen, dstate, io_dtype, stream,
+                       true);
 }
 
 size_t ssm_scan_bwd_workspace_size(int batch, int dim, int seqlen, int dstate, int io_dtype,
@@ -420,6 +472,52 @@ int ssm_scan_bwd(const void* u, const void* delta, const float* A, const void* B
   if ((e = ssm::launch_bwd(b, io_dtype, vec, s)) != cudaSuccess) return cuda_fail(e, "backward pass");
   if ((e = ssm::launch_bwd_finish(b, io_dtype, dB, dC, dA, dD, ddt_bias, s)) != cudaSuccess)
     return cuda_fail(e, "backward reduction");
+  return SSM_OK;
+}
+
+size_t ssm_scan_bwd_scalar_a_workspace_size(int batch, int dim, int seqlen, int dstate,
+                                            int io_dtype, int have_ckpt) {
+  const size_t base = ssm_scan_bwd_workspace_size(batch, dim, seqlen, dstate, io_dtype, have_ckpt);
+  if (base == 0) return 0;
+  return align_up((size_t)dim * dstate * 4) * 2 + base;
+}
+
+int ssm_scan_bwd_scalar_a(const void* u, const void* delta, const float* A, const void* B,
+                          const void* C, const float* D, const void* z, const float* dt_bias,
+                          int delta_softplus, const float* h0, const void* dout, const float* dhL,
+                          const float* ckpt, void* du, void* ddelta, float* dA, void* dB, void* dC,
+                          float* dD, void* dz, float* ddt_bias, float* dh0, void* workspace,
+                          size_t workspace_bytes, int batch, int dim, int seqlen, int dstate,
+                          int io_dtype, void* stream) {
+  g_err[0] = 0;
+  TRY(check_dims(batch, dim, seqlen, dstate, io_dtype));
+  TRY(check_ptr(A, (size_t)dim * 4, 4, "A"));
+  TRY(check_opt(dA, (size_t)dim * 4, 4, "dA"));
+  const size_t head = align_up((size_t)dim * dstate * 4);
+  const size_t need = ssm_scan_bwd_scalar_a_workspace_size(batch, dim, seqlen, dstate, io_dtype,
+                                                           ckpt != nullptr);
+  if (!workspace || workspace_bytes < need)
+    return fail(SSM_EWORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes, need);
+  if (reinterpret_cast<uintptr_t>(workspace) & 255)
+    return fail(SSM_EINVAL, "workspace is not 256-byte aligned");
+  TRY(check_ptr(workspace, need, 256, "workspace"));
+  char* w = reinterpret_cast<char*>(workspace);
+  float* Af = reinterpret_cast<float*>(w);          // A broadcast to [dim][dstate]
+  float* dAf = reinterpret_cast<float*>(w + head);  // dA per state, summed into dA[d] at the end
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long long n = (long long)dim * dstate;
+  broadcast_a_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(A, Af, dim, dstate);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "decay broadcast");
+  const int rc = ssm_scan_bwd(u, delta, Af, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL,
+                              ckpt, du, ddelta, dA ? dAf : nullptr, dB, dC, dD, dz, ddt_bias, dh0,
+                              w + 2 * head, workspace_bytes - 2 * head, batch, dim, seqlen, dstate,
+                              io_dtype, stream);
+  if (rc != SSM_OK) return rc;
+  if (dA) {
+    reduce_da_kernel<<<(unsigned)((dim + 255) / 256), 256, 0, s>>>(dAf, dA, dim, dstate);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "decay gradient sum");
+  }
   return SSM_OK;
 }
 

@@ -26,6 +26,10 @@
 //     instructions; the exponentials are split between the MUFU unit and a range-reduced
 //     polynomial on the FMA pipe (KE / KO of a lane's 4 state pairs on MUFU at even / odd steps)
 //     so neither unit idles;
+//   * scalar decay (one A_d per channel shared by its N states, the Mamba-2 restriction noted on
+//     the "2024 Reading List: Neural Network" page, section on state-space models): Ā_t =
+//     exp(Δ_t A_d) is computed once per (channel, step) with Δ_t and Δ_t x_t, so the time loop
+//     runs no exponential at all (template KE = KO = -1);
 //   * few channels (long sequences): the time axis is split into S chunks.  A summary pass
 //     runs every chunk but the last from a zero state and records its end state and ΣΔ; a
 //     carry pass chains the chunk states h_in(j+1) = exp(A ΣΔ_j) h_in(j) + h_end(j) (the
@@ -85,7 +89,8 @@ __device__ __forceinline__ float4 quad(const float4* q, int i) { return q[i]; }
 
 // KP of the lane's PPL state pairs take 2^x from the MUFU unit, the others from the FMA-pipe
 // polynomial, which has no range checks: it is used only in blocks where every step satisfies
-// |Δ| max_n |A_n log2 e| <= 126 (checked once per block by a warp vote).
+// |Δ| max_n |A_n log2 e| <= 126 (checked once per block by a warp vote).  KP < 0: scalar decay,
+// Ā is already in the table.
 template <bool PRECISE, int PPL, int KP>
 __device__ __forceinline__ void prepare_step(StepPrep<PPL>& p, const float2 (&al)[PPL], float4 dd,
                                              const float4* bq) {
@@ -97,7 +102,9 @@ __device__ __forceinline__ void prepare_step(StepPrep<PPL>& p, const float2 (&al
   for (int j = 0; j < PPL; ++j) {
     const float4 bb = bv[j >> 1];
     const float2 bp = (j & 1) ? make_float2(bb.z, bb.w) : make_float2(bb.x, bb.y);
-    if (PRECISE) {
+    if (KP < 0) {
+      p.av[j] = d2;  // scalar decay: the table holds (Ā, Ā, Δx, Δx)
+    } else if (PRECISE) {
       p.av[j] = make_float2(expf(dd.x * al[j].x), expf(dd.x * al[j].y));
     } else if (j < KP) {
       const float2 x = mul2(d2, al[j]);
@@ -176,7 +183,7 @@ struct BlockRows {
 };
 
 // What one lane needs to load, prepare and finish the blocks of its chunk.
-template <typename IO, bool VEC, int MODE, int LPC>
+template <typename IO, bool VEC, int MODE, int LPC, bool SA>
 struct ChunkLane {
   using Lay = Layout<LPC>;
   static constexpr int SPL = Lay::kSPL;
@@ -195,6 +202,7 @@ struct ChunkLane {
   bool bc_live, softplus, act;
   float bias, Dd;
   float dlim;  // |Δ| < dlim keeps |Δ A log2 e| <= 126 for every state of the warp
+  float a1;    // scalar decay: A_d (times log2 e on the bf16 path)
 
 
   // Rows of the block starting at tb; steps at or beyond t_end read as zero.
@@ -240,8 +248,13 @@ struct ChunkLane {
       else dl = softplus_fast_x2(v);
     }
     const float2 dx = mul2(dl, make_float2(r.u.get(j), r.u.get(j + 1)));
-    sd[(SPL * q + j) * Lay::kSdStride + slot] = make_float4(dl.x, dl.x, dx.x, dx.x);
-    sd[(SPL * q + j + 1) * Lay::kSdStride + slot] = make_float4(dl.y, dl.y, dx.y, dx.y);
+    float2 tv = dl;  // table entry: Δ, or Ā = exp(Δ A_d) for a scalar decay
+    if (SA) {
+      if (kPrecise) tv = make_float2(expf(dl.x * a1), expf(dl.y * a1));
+      else tv = make_float2(ex2_mufu(dl.x * a1), ex2_mufu(dl.y * a1));
+    }
+    sd[(SPL * q + j) * Lay::kSdStride + slot] = make_float4(tv.x, tv.x, dx.x, dx.x);
+    sd[(SPL * q + j + 1) * Lay::kSdStride + slot] = make_float4(tv.y, tv.y, dx.y, dx.y);
     if (MODE == kFwdSummary) dblk += (j < nown ? dl.x : 0.f) + (j + 1 < nown ? dl.y : 0.f);
     ok = ok && fabsf(dl.x) < dlim && fabsf(dl.y) < dlim;
   }
@@ -340,7 +353,8 @@ __device__ __forceinline__ void run_chunk(const FwdArgs& a, WarpTile<LPC>& tile,
                                           float bias, int lane, int slot, int q, int b, bool act,
                                           long long ch, int t_begin, int t_end, bool last_chunk) {
   using Lay = Layout<LPC>;
-  using Lane = ChunkLane<IO, VEC, MODE, LPC>;
+  using Lane = ChunkLane<IO, VEC, MODE, LPC, (KE < 0)>;
+  constexpr int KS = KE < 0 ? -1 : Layout<LPC>::kPPL;  // exponentials of an unchecked block
   constexpr int SPL = Lay::kSPL, PPL = Lay::kPPL;
   constexpr bool kPrecise = Lane::kPrecise;
   constexpr bool kReadout = Lane::kReadout;
@@ -366,6 +380,7 @@ __device__ __forceinline__ void run_chunk(const FwdArgs& a, WarpTile<LPC>& tile,
   ln.act = act;
   ln.bias = bias;
   ln.Dd = Dd;
+  ln.a1 = al[0].x;
   const int nblk_total = (L + kBlk - 1) / kBlk;
   const int nblk = (t_end - t_begin + kBlk - 1) / kBlk;
   const auto own = [&](int nvalid) { return max(0, min(SPL, nvalid - SPL * q)); };
@@ -440,7 +455,7 @@ __device__ __forceinline__ void run_chunk(const FwdArgs& a, WarpTile<LPC>& tile,
       float* nsB = reinterpret_cast<float*>(nxt.sB);
       float* nsC = reinterpret_cast<float*>(nxt.sC);
       if (kPrecise || !safe)
-        interleaved_block<kPrecise, kReadout, LPC, PPL, PPL>(ln, &cur, cur.yp, nsB, nsC, nxt.sd,
+        interleaved_block<kPrecise, kReadout, LPC, KS, KS>(ln, &cur, cur.yp, nsB, nsC, nxt.sd,
                                                              nxt.yp, hh, al, rn, nown_next, pu, pz,
                                                              o, dblk, ok);
       else
@@ -454,7 +469,7 @@ __device__ __forceinline__ void run_chunk(const FwdArgs& a, WarpTile<LPC>& tile,
         for (int j = 0; j < SPL; j += 2) ln.output_pair(nxt.yp, pu, pz, j, o);
       }
       if (kPrecise || !safe)
-        state_loop<kPrecise, kReadout, LPC, PPL, PPL>(cur, hh, al, slot, q, nvalid);
+        state_loop<kPrecise, kReadout, LPC, KS, KS>(cur, hh, al, slot, q, nvalid);
       else
         state_loop<kPrecise, kReadout, LPC, KE, KO>(cur, hh, al, slot, q, nvalid);
       // a partial block is the last one: there is no next block to prepare
@@ -522,7 +537,7 @@ __global__ void __launch_bounds__(128) fwd_kernel(const FwdArgs a) {
 
   constexpr bool kPrecise = std::is_same<IO, float>::value;
   const float ascale = kPrecise ? 1.f : kLog2e;
-  const float* Ad = a.A + (long long)dd * a.N;
+  const float* Ad = a.A + (long long)dd * (KE < 0 ? 1 : a.N);
   const float* hsrc = nullptr;
   bool hs16 = false;  // hin rows hold 16 states; h0 rows hold N
   if (MODE != kFwdSummary) {
@@ -537,7 +552,10 @@ __global__ void __launch_bounds__(128) fwd_kernel(const FwdArgs a) {
 #pragma unroll
   for (int j = 0; j < PPL; ++j) {
     const int n0 = SPL * q + 2 * j, n1 = n0 + 1;
-    al[j] = make_float2(n0 < a.N ? Ad[n0] * ascale : 0.f, n1 < a.N ? Ad[n1] * ascale : 0.f);
+    if (KE < 0)
+      al[j] = f2(Ad[0] * ascale);  // one decay rate for every state
+    else
+      al[j] = make_float2(n0 < a.N ? Ad[n0] * ascale : 0.f, n1 < a.N ? Ad[n1] * ascale : 0.f);
     hh[j] = make_float2((hsrc && (hs16 || n0 < a.N)) ? hsrc[n0] : 0.f,
                         (hsrc && (hs16 || n1 < a.N)) ? hsrc[n1] : 0.f);
   }
@@ -559,7 +577,7 @@ __global__ void fwd_carry_kernel(const FwdArgs a, const float* __restrict__ summ
   const long long ch = i / kNS;
   const int n = (int)(i % kNS);
   const int d = (int)(ch % a.dim);
-  const float An = n < a.N ? a.A[(long long)d * a.N + n] : 0.f;
+  const float An = n >= a.N ? 0.f : (a.scalar_a ? a.A[d] : a.A[(long long)d * a.N + n]);
   float h = (a.h0 && n < a.N) ? a.h0[ch * a.N + n] : 0.f;
   for (int j = 0; j < a.nchunk; ++j) {
     hin[((long long)j * nch + ch) * kNS + n] = h;
@@ -583,7 +601,9 @@ cudaError_t launch_mode(const FwdArgs& a, int wpb, int kmufu, cudaStream_t s) {
   const int nchunk_launch = MODE == kFwdSummary ? a.nchunk - 1 : a.nchunk;  // last chunk's summary is unused
   if (ctas <= 0 || nchunk_launch <= 0) return cudaSuccess;
   const dim3 grid((unsigned)ctas, (unsigned)nchunk_launch), block(32 * wpb);
-  if constexpr (std::is_same<IO, float>::value) {  // fp32: library expf
+  if (a.scalar_a) {  // two lanes per channel, no exponential in the time loop
+    launch_one<IO, VEC, MODE, 2, -1, -1>(a, grid, block, s);
+  } else if constexpr (std::is_same<IO, float>::value) {  // fp32: library expf
     if (a.lpc == 4) launch_one<IO, VEC, MODE, 4, 2, 2>(a, grid, block, s);
     else if (a.lpc == 1) launch_one<IO, VEC, MODE, 1, 8, 8>(a, grid, block, s);
     else launch_one<IO, VEC, MODE, 2, 4, 4>(a, grid, block, s);

@@ -21,7 +21,7 @@ struct FwdArgs {
   const void* z;        // may be NULL (no gate)
   const void* B;
   const void* C;
-  const float* A;
+  const float* A;       // [dim][N], or [dim] when scalar_a
   const float* D;       // may be NULL
   const float* dt_bias; // may be NULL
   const float* h0;      // may be NULL (zero initial state)
@@ -35,6 +35,7 @@ struct FwdArgs {
   int chunk_len;        // multiple of kBlk
   int nchunk;           // S
   int softplus;
+  int scalar_a;         // one decay rate A_d per channel, shared by its N states
   int lpc;              // lanes per channel: 1, 2 or 4 (16 / lpc states each)
   int warps_per_b;      // ceil(dim / (32 / lpc))
   long long nwarps;     // batch * warps_per_b

@@ -6,7 +6,8 @@ Recipe (every workload):
   u, z, B, C, dout ~ N(0, 1);  delta (raw step input) ~ N(0, 0.5^2);
   dt ~ log-uniform on [dt_min, dt_max] per channel d, dt_bias = inv_softplus(dt) so that a zero
   raw delta gives a step of exactly dt (inv_softplus(y) = y + log(-expm1(-y)));
-  A[d, n] = -(n + 1) (S4D-real initialisation);  D ~ N(0, 1).
+  A[d, n] = -(n + 1) (S4D-real initialisation);  D ~ N(0, 1);
+  scalar decay (one rate per channel): A[d] = -U(1, 16), the range of Mamba-2's initial rates.
 io tensors are drawn in float32 and rounded once to the io dtype (bf16: round-to-nearest-even);
 the oracle reads the rounded values.  numpy's PCG64 generator, seeded per tensor name, so each
 tensor is reproducible on its own and on any machine.
@@ -73,10 +74,10 @@ def _io(x: np.ndarray, dtype: torch.dtype) -> torch.Tensor:
 
 
 def make_inputs(w: Workload, seed: int = 0, with_dout: bool = False, with_h0: bool = False,
-                gate: bool = True, step: int = None) -> dict:
+                gate: bool = True, step: int = None, scalar_a: bool = False) -> dict:
     """CPU tensors for one call.  Scan layout: u, delta, z, dout [batch, dim, L];
     B, C [batch, N, L].  Decode (step is not None): x, dt, z [batch, dim]; B, C [batch, N],
-    drawn independently for each step index."""
+    drawn independently for each step index.  scalar_a: A is [dim] (one decay rate per channel)."""
     b, d, L, N = w.batch, w.dim, w.seqlen, w.dstate
     tag = "" if step is None else f"/step{step}"
     shape_x = (b, d, L) if step is None else (b, d)
@@ -92,7 +93,10 @@ def make_inputs(w: Workload, seed: int = 0, with_dout: bool = False, with_h0: bo
     lo, hi = np.log(w.dt_min), np.log(w.dt_max)
     dt = np.exp(_rng(seed, "dt").uniform(lo, hi, size=(d,)))
     out["dt_bias"] = torch.from_numpy(inv_softplus(dt).astype(np.float32))
-    out["A"] = torch.from_numpy(-np.tile(np.arange(1, N + 1, dtype=np.float32), (d, 1)))
+    if scalar_a:
+        out["A"] = torch.from_numpy(-_rng(seed, "A").uniform(1.0, 16.0, size=(d,)).astype(np.float32))
+    else:
+        out["A"] = torch.from_numpy(-np.tile(np.arange(1, N + 1, dtype=np.float32), (d, 1)))
     out["D"] = torch.from_numpy(_normal(seed, "D", (d,)))
     if with_h0:
         out["h0"] = torch.from_numpy(_normal(seed, "h0", (b, d, N), 0.5))

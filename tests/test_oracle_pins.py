@@ -8,6 +8,8 @@ Every test builds its expected value independently (a different formula or libra
   * the gating special case of the "Seçim Mekanizması (S6)" section (N=1, A=-1, B=1);
   * the Δ limits of the "Sorular" section (small Δ keeps the state, large Δ resets it);
   * chunked-vs-sequential state passing, superposition, decode-vs-scan;
+  * the scalar decay (one A per channel, the Mamba-2 restriction in the reading-list notes) as
+    a masked Gram-matrix product, and its rate gradient by central differences;
   * central finite differences of the forward pass for every gradient.
 """
 import numpy as np
@@ -248,6 +250,63 @@ def test_gradients_by_finite_differences(gate, softplus):
             num[i] = (loss_and_grads(dict(c, **{key: xp}), dout, dhL, softplus)
                       - loss_and_grads(dict(c, **{key: xm}), dout, dhL, softplus)) / (2 * eps)
         np.testing.assert_allclose(g[gname], num, rtol=2e-6, atol=2e-7, err_msg=gname)
+
+
+# ------------------------------------------------------------------ scalar decay (one A per channel)
+def scalar_decay_matrix_form(c, a_d, softplus=True):
+    """Scalar decay as one masked matrix product per channel: y = (M o (C^T B)) (Δ u) with
+    M[t, s] = exp(a_d (cs[t+1] - cs[s+1])) for s <= t, plus the decayed h0 and D u.  The N-state
+    dot products C_t . B_s form a Gram matrix, so no recurrence is run."""
+    u, B, C = c["u"], c["B"], c["C"]
+    batch, dim, L = u.shape
+    v = c["delta"] + c["dt_bias"][None, :, None]
+    dt = softplus_ref(v) if softplus else v
+    out = np.zeros_like(u)
+    tri = np.tril(np.ones((L, L), bool))
+    for b in range(batch):
+        G = C[b].T @ B[b]                                  # G[t, s] = C_t . B_s
+        for d in range(dim):
+            cs = np.cumsum(dt[b, d])                       # cs[t] = sum_{r<=t} Δ_r
+            M = np.where(tri, np.exp(a_d[d] * (cs[:, None] - cs[None, :])), 0.0)
+            y = (M * G) @ (dt[b, d] * u[b, d])
+            if c["h0"] is not None:
+                y += np.exp(a_d[d] * cs) * (C[b].T @ c["h0"][b, d])
+            y += c["D"][d] * u[b, d]
+            if c["z"] is not None:
+                zz = c["z"][b, d]
+                y = y * zz * expit(zz)
+            out[b, d] = y
+    return out
+
+
+def test_scalar_decay_matrix_form():
+    """The oracle with A[d, n] = a_d for every n against the masked-matrix (dual) form."""
+    c = rand_case(batch=2, dim=3, L=48, N=16, seed=61)
+    a_d = -np.exp(np.random.default_rng(62).standard_normal(3))
+    c["A"] = np.repeat(a_d[:, None], 16, 1)
+    np.testing.assert_allclose(run(c)["out"], scalar_decay_matrix_form(c, a_d),
+                               rtol=1e-10, atol=1e-11)
+
+
+def test_scalar_decay_gradient_is_the_state_sum():
+    """dL/da_d of a shared rate equals the sum over n of the oracle's per-state dA[d, n]
+    (chain rule through A[d, n] = a_d), checked against central differences in a_d."""
+    c = rand_case(batch=2, dim=2, L=6, N=4, seed=63)
+    a_d = np.array([-0.7, -2.1])
+    c["A"] = np.repeat(a_d[:, None], 4, 1)
+    r = np.random.default_rng(64)
+    dout = r.standard_normal(c["u"].shape)
+    dhL = r.standard_normal(c["h0"].shape)
+    g = oracle.scan_bwd(c["u"], c["delta"], c["A"], c["B"], c["C"], dout, D=c["D"], z=c["z"],
+                        dt_bias=c["dt_bias"], h0=c["h0"], dhL=dhL)
+    eps = 1e-6
+    for d in range(2):
+        ap, am = a_d.copy(), a_d.copy()
+        ap[d] += eps
+        am[d] -= eps
+        lp = loss_and_grads(dict(c, A=np.repeat(ap[:, None], 4, 1)), dout, dhL)
+        lm = loss_and_grads(dict(c, A=np.repeat(am[:, None], 4, 1)), dout, dhL)
+        np.testing.assert_allclose(g["dA"][d].sum(), (lp - lm) / (2 * eps), rtol=2e-6, atol=2e-7)
 
 
 def test_planted_mistake_is_caught():
