@@ -173,6 +173,40 @@ SSM_API int ssm_scan_bwd_scalar_a(const void* u, const void* delta, const float*
                                   size_t workspace_bytes, int batch, int dim, int seqlen,
                                   int dstate, int io_dtype, void* stream);
 
+/*
+ * Variants of the scan selected by a bit mask (the _ex entry points; 0 = ssm_scan_fwd/_bwd):
+ *   SSM_SCALAR_A  A (and dA) is [dim]: one decay rate per channel, as ssm_scan_fwd_scalar_a.
+ *   SSM_REVERSE   the scan runs backwards in time, t = L-1 down to 0:
+ *                   h_t = exp(Δ_t A) h_{t+1} + Δ_t B_t x_t  (h0 enters at t = L-1; hL is the
+ *                   state after t = 0),  y_t = C_t . h_t + D x_t,
+ *                 the anti-causal half of a bidirectional layer ("2024 Reading List: Neural
+ *                 Network", Hydra notes: a forward and a backward scan whose outputs are summed).
+ *                 Every tensor keeps its layout; the kernels read and write the time rows
+ *                 mirrored.  Checkpoints are indexed by blocks of 16 steps in scan order
+ *                 (block k holds the state before scan steps 16k .. 16k+15, i.e. before time
+ *                 index L-1-16k), and only feed ssm_scan_bwd_ex with the same flags.
+ * Any other bit is rejected with SSM_EINVAL.  Arguments are those of ssm_scan_fwd /
+ * ssm_scan_bwd plus flags.
+ */
+#define SSM_SCALAR_A 1
+#define SSM_REVERSE 2
+SSM_API size_t ssm_scan_fwd_ex_workspace_size(int batch, int dim, int seqlen, int dstate,
+                                              int io_dtype, int flags);
+SSM_API int ssm_scan_fwd_ex(const void* u, const void* delta, const float* A, const void* B,
+                            const void* C, const float* D, const void* z, const float* dt_bias,
+                            int delta_softplus, const float* h0, float* hL, void* out, float* ckpt,
+                            void* workspace, size_t workspace_bytes, int batch, int dim,
+                            int seqlen, int dstate, int io_dtype, int flags, void* stream);
+SSM_API size_t ssm_scan_bwd_ex_workspace_size(int batch, int dim, int seqlen, int dstate,
+                                              int io_dtype, int have_ckpt, int flags);
+SSM_API int ssm_scan_bwd_ex(const void* u, const void* delta, const float* A, const void* B,
+                            const void* C, const float* D, const void* z, const float* dt_bias,
+                            int delta_softplus, const float* h0, const void* dout,
+                            const float* dhL, const float* ckpt, void* du, void* ddelta, float* dA,
+                            void* dB, void* dC, float* dD, void* dz, float* ddt_bias, float* dh0,
+                            void* workspace, size_t workspace_bytes, int batch, int dim,
+                            int seqlen, int dstate, int io_dtype, int flags, void* stream);
+
 /* Size of the static scratch array used by ssm_scan_fwd_noalloc (8 MiB per GPU). */
 #define SSM_NOALLOC_SCRATCH_BYTES (8u << 20)
 

@@ -14,6 +14,10 @@ The arithmetic lives in ``ssm_oracle.c`` (plain double-precision loops, cited th
                          finite differences of ``scan_fwd`` (parity of the gradient formulas
                          themselves is otherwise unpinned by the pages).
   * ``state_update``  -- one recurrent (decode) step of the same recurrence, in place.
+  * ``reverse=True``  -- the scan backwards in time (t = L-1 .. 0), the anti-causal half of a
+                         bidirectional layer ("2024 Reading List: Neural Network", Hydra notes):
+                         by definition the forward scan of the time-reversed sequences, so it is
+                         written as exactly that (reverse the time axis, scan, reverse back).
 
 All arrays are numpy float64, C-contiguous; layouts as in ``ssm_oracle.c``.
 """
@@ -68,14 +72,32 @@ def _chans(channels):
     return c, c.ctypes.data_as(_i64p), int(c.size)
 
 
+def _flip(x):
+    """Time axis (the last one) reversed, or None."""
+    return None if x is None else np.ascontiguousarray(np.asarray(x, dtype=np.float64)[..., ::-1])
+
+
 def scan_fwd(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=True,
-             h0=None, zoh=False, channels=None, nthreads=0, out=None, ypre=False):
+             h0=None, zoh=False, channels=None, nthreads=0, out=None, ypre=False, reverse=False):
     """Forward selective scan in fp64.
 
     u, delta, z: [batch, dim, L]; B, C: [batch, N, L]; A: [dim, N]; D, dt_bias: [dim];
     h0: [batch, dim, N].  ``channels``: optional flat indices b*dim+d to compute (others
-    left as in ``out``, default zeros).  Returns dict(out, hL[, ypre]).
+    left as in ``out``, default zeros).  ``reverse``: scan from t = L-1 down to 0 (h0 enters
+    at t = L-1, hL is the state after t = 0).  Returns dict(out, hL[, ypre]).
     """
+    if reverse:
+        res = scan_fwd(_flip(u), _flip(delta), A, _flip(B), _flip(C), D=D, z=_flip(z),
+                       dt_bias=dt_bias, delta_softplus=delta_softplus, h0=h0, zoh=zoh,
+                       channels=channels, nthreads=nthreads,
+                       out=None if out is None else _flip(out), ypre=ypre)
+        res["out"] = _flip(res["out"])
+        if out is not None:
+            out[...] = res["out"]
+            res["out"] = out
+        if ypre:
+            res["ypre"] = _flip(res["ypre"])
+        return res
     u = _arr(u)
     batch, dim, L = u.shape
     A = _arr(A)
@@ -106,12 +128,20 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=Tru
 
 
 def scan_bwd(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None, delta_softplus=True,
-             h0=None, dhL=None, channels=None, nthreads=0):
+             h0=None, dhL=None, channels=None, nthreads=0, reverse=False):
     """Gradients of :func:`scan_fwd` (Euler input term) w.r.t. every input, in fp64.
 
     Returns dict(du, ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0).  With ``channels`` the
     summed gradients (dA, dB, dC, dD, ddt_bias) hold only those channels' contributions.
+    ``reverse``: gradients of the reverse scan (time-indexed gradients reversed back).
     """
+    if reverse:
+        g = scan_bwd(_flip(u), _flip(delta), A, _flip(B), _flip(C), _flip(dout), D=D, z=_flip(z),
+                     dt_bias=dt_bias, delta_softplus=delta_softplus, h0=h0, dhL=dhL,
+                     channels=channels, nthreads=nthreads)
+        for k in ("du", "ddelta", "dz", "dB", "dC"):
+            g[k] = _flip(g[k])
+        return g
     u = _arr(u)
     batch, dim, L = u.shape
     A = _arr(A)

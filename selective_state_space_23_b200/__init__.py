@@ -82,8 +82,8 @@ def _workspace(nbytes, device, given):
     return torch.empty(nbytes, dtype=torch.uint8, device=device)
 
 
-def _scan_fwd(entry, u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, return_final_state,
-              return_ckpt, out, workspace, scalar_a):
+def _scan_fwd(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, return_final_state,
+              return_ckpt, out, workspace, scalar_a, reverse):
     dev = u.device
     batch, dim, L = u.shape
     N = B.shape[1]
@@ -104,12 +104,14 @@ def _scan_fwd(entry, u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, retur
     hL = torch.empty((batch, dim, N), dtype=torch.float32, device=dev) if return_final_state else None
     nblk = (L + CKPT_STEPS - 1) // CKPT_STEPS
     ckpt = torch.empty((batch, dim, nblk, N), dtype=torch.float32, device=dev) if return_ckpt else None
-    ws = _workspace(fwd_workspace_bytes(batch, dim, L, N, io), dev, workspace)
-    rc = getattr(_abi.lib(), entry)(
+    flags = (_abi.SSM_SCALAR_A if scalar_a else 0) | (_abi.SSM_REVERSE if reverse else 0)
+    nws = int(_abi.lib().ssm_scan_fwd_ex_workspace_size(batch, dim, L, N, code, flags))
+    ws = _workspace(nws, dev, workspace)
+    rc = _abi.lib().ssm_scan_fwd_ex(
         _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias),
         int(bool(delta_softplus)), _ptr(h0), _ptr(hL), _ptr(out), _ptr(ckpt), _ptr(ws),
-        0 if ws is None else ws.numel(), batch, dim, L, N, code, _stream(dev))
-    _abi.check(rc, entry)
+        0 if ws is None else ws.numel(), batch, dim, L, N, code, flags, _stream(dev))
+    _abi.check(rc, "ssm_scan_fwd_ex")
     if not return_final_state and not return_ckpt:
         return out
     res = (out,)
@@ -121,24 +123,25 @@ def _scan_fwd(entry, u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, retur
 
 
 def ssm_scan_fwd(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=True, h0=None,
-                 return_final_state=False, return_ckpt=False, out=None, workspace=None):
+                 return_final_state=False, return_ckpt=False, out=None, workspace=None,
+                 reverse=False):
     """Forward scan.  u, delta, z: [batch, dim, L]; B, C: [batch, N, L] (io dtype f32 or bf16);
-    A: [dim, N] f32; D, dt_bias: [dim] f32; h0: [batch, dim, N] f32.
-    Returns out, or a tuple (out, hL?, ckpt?) when those are requested."""
-    return _scan_fwd("ssm_scan_fwd", u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0,
-                     return_final_state, return_ckpt, out, workspace, False)
+    A: [dim, N] f32; D, dt_bias: [dim] f32; h0: [batch, dim, N] f32.  reverse: scan from
+    t = L-1 down to 0.  Returns out, or a tuple (out, hL?, ckpt?) when those are requested."""
+    return _scan_fwd(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, return_final_state,
+                     return_ckpt, out, workspace, False, reverse)
 
 
 def ssm_scan_fwd_scalar_a(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=True,
                           h0=None, return_final_state=False, return_ckpt=False, out=None,
-                          workspace=None):
+                          workspace=None, reverse=False):
     """Forward scan with one decay rate per channel: as :func:`ssm_scan_fwd` with A [dim] f32."""
-    return _scan_fwd("ssm_scan_fwd_scalar_a", u, delta, A, B, C, D, z, dt_bias, delta_softplus,
-                     h0, return_final_state, return_ckpt, out, workspace, True)
+    return _scan_fwd(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, return_final_state,
+                     return_ckpt, out, workspace, True, reverse)
 
 
-def _scan_bwd(entry, u, delta, A, B, C, dout, D, z, dt_bias, delta_softplus, h0, dhL, ckpt,
-              workspace, need, scalar_a):
+def _scan_bwd(u, delta, A, B, C, dout, D, z, dt_bias, delta_softplus, h0, dhL, ckpt,
+              workspace, need, scalar_a, reverse):
     dev = u.device
     batch, dim, L = u.shape
     N = B.shape[1]
@@ -172,33 +175,34 @@ def _scan_bwd(entry, u, delta, A, B, C, dout, D, z, dt_bias, delta_softplus, h0,
         "ddt_bias": e((dim,), torch.float32) if "ddt_bias" in want else None,
         "dh0": e((batch, dim, N), torch.float32) if "dh0" in want else None,
     }
-    size_fn = getattr(_abi.lib(), entry + "_workspace_size")
-    nws = int(size_fn(batch, dim, L, N, code, int(ckpt is not None)))
+    flags = (_abi.SSM_SCALAR_A if scalar_a else 0) | (_abi.SSM_REVERSE if reverse else 0)
+    nws = int(_abi.lib().ssm_scan_bwd_ex_workspace_size(batch, dim, L, N, code,
+                                                         int(ckpt is not None), flags))
     ws = _workspace(nws, dev, workspace)
-    rc = getattr(_abi.lib(), entry)(
+    rc = _abi.lib().ssm_scan_bwd_ex(
         _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias),
         int(bool(delta_softplus)), _ptr(h0), _ptr(dout), _ptr(dhL), _ptr(ckpt),
         _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]),
         _ptr(g["dD"]), _ptr(g["dz"]), _ptr(g["ddt_bias"]), _ptr(g["dh0"]),
-        _ptr(ws), 0 if ws is None else ws.numel(), batch, dim, L, N, code, _stream(dev))
-    _abi.check(rc, entry)
+        _ptr(ws), 0 if ws is None else ws.numel(), batch, dim, L, N, code, flags, _stream(dev))
+    _abi.check(rc, "ssm_scan_bwd_ex")
     return g
 
 
 def ssm_scan_bwd(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None, delta_softplus=True,
-                 h0=None, dhL=None, ckpt=None, workspace=None, need=None):
+                 h0=None, dhL=None, ckpt=None, workspace=None, need=None, reverse=False):
     """Gradients of :func:`ssm_scan_fwd`.  Returns a dict with du, ddelta, dA, dB, dC, dD, dz,
     ddt_bias, dh0 (entries are None when the matching input is absent or not in ``need``)."""
-    return _scan_bwd("ssm_scan_bwd", u, delta, A, B, C, dout, D, z, dt_bias, delta_softplus, h0,
-                     dhL, ckpt, workspace, need, False)
+    return _scan_bwd(u, delta, A, B, C, dout, D, z, dt_bias, delta_softplus, h0, dhL, ckpt,
+                     workspace, need, False, reverse)
 
 
 def ssm_scan_bwd_scalar_a(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None,
                           delta_softplus=True, h0=None, dhL=None, ckpt=None, workspace=None,
-                          need=None):
+                          need=None, reverse=False):
     """Gradients of :func:`ssm_scan_fwd_scalar_a` (dA is [dim])."""
-    return _scan_bwd("ssm_scan_bwd_scalar_a", u, delta, A, B, C, dout, D, z, dt_bias,
-                     delta_softplus, h0, dhL, ckpt, workspace, need, True)
+    return _scan_bwd(u, delta, A, B, C, dout, D, z, dt_bias, delta_softplus, h0, dhL, ckpt,
+                     workspace, need, True, reverse)
 
 
 def ssm_state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=True,

@@ -13,6 +13,7 @@ SSM_OK, SSM_EINVAL, SSM_EUNSUPPORTED, SSM_ECUDA, SSM_EWORKSPACE = 0, 1, 2, 3, 4
 CKPT_STEPS = 16
 MAX_DSTATE = 16
 NOALLOC_SCRATCH_BYTES = 8 << 20
+SSM_SCALAR_A, SSM_REVERSE = 1, 2
 
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
@@ -37,6 +38,13 @@ SIGNATURES = {
     "ssm_scan_bwd_scalar_a": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp,
                                    _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                                    _i, _i, _i, _i, _i, _vp]),
+    "ssm_scan_fwd_ex_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "ssm_scan_fwd_ex": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp,
+                             _vp, _sz, _i, _i, _i, _i, _i, _i, _vp]),
+    "ssm_scan_bwd_ex_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "ssm_scan_bwd_ex": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp,
+                             _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                             _i, _i, _i, _i, _i, _i, _vp]),
     "ssm_scan_fwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp,
                                   _i, _i, _i, _i, _i, _vp]),
     "ssm_state_update": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp,

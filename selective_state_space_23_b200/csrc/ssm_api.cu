@@ -260,13 +260,16 @@ size_t ssm_scan_fwd_workspace_size(int batch, int dim, int seqlen, int dstate, i
 
 namespace {
 
-// Forward scan; scalar_a: A is [dim] (one decay rate per channel) instead of [dim][dstate].
+// Forward scan.  flags: SSM_SCALAR_A (A is [dim], one decay rate per channel, instead of
+// [dim][dstate]) and SSM_REVERSE (scan from t = L-1 down to 0).
 int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* B, const void* C,
                   const float* D, const void* z, const float* dt_bias, int delta_softplus,
                   const float* h0, float* hL, void* out, float* ckpt, void* workspace,
                   size_t workspace_bytes, int batch, int dim, int seqlen, int dstate,
-                  int io_dtype, void* stream, bool scalar_a) {
+                  int io_dtype, void* stream, int flags) {
   g_err[0] = 0;
+  if (flags & ~(SSM_SCALAR_A | SSM_REVERSE)) return fail(SSM_EINVAL, "unknown flags 0x%x", flags);
+  const bool scalar_a = (flags & SSM_SCALAR_A) != 0;
   TRY(check_dims(batch, dim, seqlen, dstate, io_dtype));
   const size_t es = esize(io_dtype);
   const size_t nx = (size_t)batch * dim * seqlen * es;
@@ -304,6 +307,7 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
   a.chunk_len = plan.chunk_len; a.nchunk = plan.nchunk;
   a.softplus = delta_softplus ? 1 : 0;
   a.scalar_a = scalar_a ? 1 : 0;
+  a.reverse = (flags & SSM_REVERSE) ? 1 : 0;
   a.lpc = scalar_a ? 2 : fwd_lpc();
   a.warps_per_b = (dim + 32 / a.lpc - 1) / (32 / a.lpc);
   a.nwarps = (long long)batch * a.warps_per_b;
@@ -360,8 +364,23 @@ int ssm_scan_fwd(const void* u, const void* delta, const float* A, const void* B
                  size_t workspace_bytes, int batch, int dim, int seqlen, int dstate,
                  int io_dtype, void* stream) {
   return scan_fwd_impl(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, hL, out, ckpt,
+                       workspace, workspace_bytes, batch, dim, seqlen, dstate, io_dtype, stream, 0);
+}
+
+size_t ssm_scan_fwd_ex_workspace_size(int batch, int dim, int seqlen, int dstate, int io_dtype,
+                                      int flags) {
+  (void)flags;  // the time-split scratch does not depend on the variant
+  return ssm_scan_fwd_workspace_size(batch, dim, seqlen, dstate, io_dtype);
+}
+
+int ssm_scan_fwd_ex(const void* u, const void* delta, const float* A, const void* B,
+                    const void* C, const float* D, const void* z, const float* dt_bias,
+                    int delta_softplus, const float* h0, float* hL, void* out, float* ckpt,
+                    void* workspace, size_t workspace_bytes, int batch, int dim, int seqlen,
+                    int dstate, int io_dtype, int flags, void* stream) {
+  return scan_fwd_impl(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, hL, out, ckpt,
                        workspace, workspace_bytes, batch, dim, seqlen, dstate, io_dtype, stream,
-                       false);
+                       flags);
 }
 
 size_t ssm_scan_fwd_scalar_a_workspace_size(int batch, int dim, int seqlen, int dstate,
@@ -376,7 +395,7 @@ int ssm_scan_fwd_scalar_a(const void* u, const void* delta, const float* A, cons
                           int dstate, int io_dtype, void* stream) {
   return scan_fwd_impl(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, hL, out, ckpt,
                        workspace, workspace_bytes, batch, dim, seqlen, dstate, io_dtype, stream,
-                       true);
+                       SSM_SCALAR_A);
 }
 
 size_t ssm_scan_bwd_workspace_size(int batch, int dim, int seqlen, int dstate, int io_dtype,
@@ -385,13 +404,18 @@ size_t ssm_scan_bwd_workspace_size(int batch, int dim, int seqlen, int dstate, i
   return layout_bwd(batch, dim, seqlen, dstate, have_ckpt != 0).total;
 }
 
-int ssm_scan_bwd(const void* u, const void* delta, const float* A, const void* B, const void* C,
-                 const float* D, const void* z, const float* dt_bias, int delta_softplus,
-                 const float* h0, const void* dout, const float* dhL, const float* ckpt,
-                 void* du, void* ddelta, float* dA, void* dB, void* dC, float* dD, void* dz,
-                 float* ddt_bias, float* dh0, void* workspace, size_t workspace_bytes,
-                 int batch, int dim, int seqlen, int dstate, int io_dtype, void* stream) {
-  g_err[0] = 0;
+}  // extern "C"
+
+namespace {
+
+// Backward of the per-state-decay scan (A is [dim][dstate]); reverse: of the reverse scan.
+int scan_bwd_core(const void* u, const void* delta, const float* A, const void* B, const void* C,
+                  const float* D, const void* z, const float* dt_bias, int delta_softplus,
+                  const float* h0, const void* dout, const float* dhL, const float* ckpt,
+                  void* du, void* ddelta, float* dA, void* dB, void* dC, float* dD, void* dz,
+                  float* ddt_bias, float* dh0, void* workspace, size_t workspace_bytes,
+                  int batch, int dim, int seqlen, int dstate, int io_dtype, void* stream,
+                  bool reverse) {
   TRY(check_dims(batch, dim, seqlen, dstate, io_dtype));
   const size_t es = esize(io_dtype);
   const size_t nx = (size_t)batch * dim * seqlen * es;
@@ -449,6 +473,7 @@ int ssm_scan_bwd(const void* u, const void* delta, const float* A, const void* B
     a.batch = batch; a.dim = dim; a.L = seqlen; a.N = dstate;
     a.chunk_len = (int)nblk * ssm::kBlk; a.nchunk = 1;
     a.softplus = delta_softplus ? 1 : 0;
+    a.reverse = reverse ? 1 : 0;
     a.lpc = fwd_lpc();
     a.warps_per_b = fwd_warps_per_b(dim);
     a.nwarps = (long long)batch * a.warps_per_b;
@@ -464,6 +489,7 @@ int ssm_scan_bwd(const void* u, const void* delta, const float* A, const void* B
   b.part_bc = part_bc; b.part_adt = part_adt;
   b.batch = batch; b.dim = dim; b.L = seqlen; b.N = dstate;
   b.softplus = delta_softplus ? 1 : 0;
+  b.reverse = reverse ? 1 : 0;
   b.warps_per_b = (dim + 15) / 16;
   b.nwarps = (long long)batch * b.warps_per_b;
   b.wpb = l.wpb;
@@ -475,27 +501,51 @@ int ssm_scan_bwd(const void* u, const void* delta, const float* A, const void* B
   return SSM_OK;
 }
 
-size_t ssm_scan_bwd_scalar_a_workspace_size(int batch, int dim, int seqlen, int dstate,
-                                            int io_dtype, int have_ckpt) {
+}  // namespace
+
+extern "C" {
+
+int ssm_scan_bwd(const void* u, const void* delta, const float* A, const void* B, const void* C,
+                 const float* D, const void* z, const float* dt_bias, int delta_softplus,
+                 const float* h0, const void* dout, const float* dhL, const float* ckpt,
+                 void* du, void* ddelta, float* dA, void* dB, void* dC, float* dD, void* dz,
+                 float* ddt_bias, float* dh0, void* workspace, size_t workspace_bytes,
+                 int batch, int dim, int seqlen, int dstate, int io_dtype, void* stream) {
+  g_err[0] = 0;
+  return scan_bwd_core(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL, ckpt, du,
+                       ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, workspace, workspace_bytes,
+                       batch, dim, seqlen, dstate, io_dtype, stream, false);
+}
+
+size_t ssm_scan_bwd_ex_workspace_size(int batch, int dim, int seqlen, int dstate, int io_dtype,
+                                      int have_ckpt, int flags) {
+  if (flags & ~(SSM_SCALAR_A | SSM_REVERSE)) return 0;
   const size_t base = ssm_scan_bwd_workspace_size(batch, dim, seqlen, dstate, io_dtype, have_ckpt);
-  if (base == 0) return 0;
+  if (base == 0 || !(flags & SSM_SCALAR_A)) return base;
   return align_up((size_t)dim * dstate * 4) * 2 + base;
 }
 
-int ssm_scan_bwd_scalar_a(const void* u, const void* delta, const float* A, const void* B,
-                          const void* C, const float* D, const void* z, const float* dt_bias,
-                          int delta_softplus, const float* h0, const void* dout, const float* dhL,
-                          const float* ckpt, void* du, void* ddelta, float* dA, void* dB, void* dC,
-                          float* dD, void* dz, float* ddt_bias, float* dh0, void* workspace,
-                          size_t workspace_bytes, int batch, int dim, int seqlen, int dstate,
-                          int io_dtype, void* stream) {
+int ssm_scan_bwd_ex(const void* u, const void* delta, const float* A, const void* B,
+                    const void* C, const float* D, const void* z, const float* dt_bias,
+                    int delta_softplus, const float* h0, const void* dout, const float* dhL,
+                    const float* ckpt, void* du, void* ddelta, float* dA, void* dB, void* dC,
+                    float* dD, void* dz, float* ddt_bias, float* dh0, void* workspace,
+                    size_t workspace_bytes, int batch, int dim, int seqlen, int dstate,
+                    int io_dtype, int flags, void* stream) {
   g_err[0] = 0;
+  if (flags & ~(SSM_SCALAR_A | SSM_REVERSE)) return fail(SSM_EINVAL, "unknown flags 0x%x", flags);
+  const bool reverse = (flags & SSM_REVERSE) != 0;
   TRY(check_dims(batch, dim, seqlen, dstate, io_dtype));
+  if (!(flags & SSM_SCALAR_A))
+    return scan_bwd_core(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL, ckpt,
+                         du, ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, workspace,
+                         workspace_bytes, batch, dim, seqlen, dstate, io_dtype, stream, reverse);
+  // scalar decay: broadcast A over the states, run the per-state backward, sum dA over n
   TRY(check_ptr(A, (size_t)dim * 4, 4, "A"));
   TRY(check_opt(dA, (size_t)dim * 4, 4, "dA"));
   const size_t head = align_up((size_t)dim * dstate * 4);
-  const size_t need = ssm_scan_bwd_scalar_a_workspace_size(batch, dim, seqlen, dstate, io_dtype,
-                                                           ckpt != nullptr);
+  const size_t need = ssm_scan_bwd_ex_workspace_size(batch, dim, seqlen, dstate, io_dtype,
+                                                     ckpt != nullptr, flags);
   if (!workspace || workspace_bytes < need)
     return fail(SSM_EWORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes, need);
   if (reinterpret_cast<uintptr_t>(workspace) & 255)
@@ -509,16 +559,34 @@ int ssm_scan_bwd_scalar_a(const void* u, const void* delta, const float* A, cons
   broadcast_a_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(A, Af, dim, dstate);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decay broadcast");
-  const int rc = ssm_scan_bwd(u, delta, Af, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL,
-                              ckpt, du, ddelta, dA ? dAf : nullptr, dB, dC, dD, dz, ddt_bias, dh0,
-                              w + 2 * head, workspace_bytes - 2 * head, batch, dim, seqlen, dstate,
-                              io_dtype, stream);
+  const int rc = scan_bwd_core(u, delta, Af, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL,
+                               ckpt, du, ddelta, dA ? dAf : nullptr, dB, dC, dD, dz, ddt_bias,
+                               dh0, w + 2 * head, workspace_bytes - 2 * head, batch, dim, seqlen,
+                               dstate, io_dtype, stream, reverse);
   if (rc != SSM_OK) return rc;
   if (dA) {
     reduce_da_kernel<<<(unsigned)((dim + 255) / 256), 256, 0, s>>>(dAf, dA, dim, dstate);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "decay gradient sum");
   }
   return SSM_OK;
+}
+
+size_t ssm_scan_bwd_scalar_a_workspace_size(int batch, int dim, int seqlen, int dstate,
+                                            int io_dtype, int have_ckpt) {
+  return ssm_scan_bwd_ex_workspace_size(batch, dim, seqlen, dstate, io_dtype, have_ckpt,
+                                        SSM_SCALAR_A);
+}
+
+int ssm_scan_bwd_scalar_a(const void* u, const void* delta, const float* A, const void* B,
+                          const void* C, const float* D, const void* z, const float* dt_bias,
+                          int delta_softplus, const float* h0, const void* dout, const float* dhL,
+                          const float* ckpt, void* du, void* ddelta, float* dA, void* dB, void* dC,
+                          float* dD, void* dz, float* ddt_bias, float* dh0, void* workspace,
+                          size_t workspace_bytes, int batch, int dim, int seqlen, int dstate,
+                          int io_dtype, void* stream) {
+  return ssm_scan_bwd_ex(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL, ckpt,
+                         du, ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, workspace, workspace_bytes,
+                         batch, dim, seqlen, dstate, io_dtype, SSM_SCALAR_A, stream);
 }
 
 int ssm_state_update(float* state, const void* x, const void* dt, const float* A, const void* B,

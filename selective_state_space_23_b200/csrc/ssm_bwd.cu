@@ -247,13 +247,16 @@ __global__ void __launch_bounds__(128) bwd_kernel(const BwdArgs a) {
   const float bias = a.dt_bias ? a.dt_bias[dd] : 0.f;
   float dD_acc = 0.f, dbias_acc = 0.f;
 
-  const long long row = ch * (long long)L + kHB * q;   // this lane's 8 steps of each block
+  // time rows at step 0 in scan order (mirrored for a reverse scan); the lane owns steps
+  // [8 q, 8 q + 8) of each block
+  const long long row = ch * (long long)L;
+  const bool rev = a.reverse != 0;
   const IO* up = reinterpret_cast<const IO*>(a.u) + row;
   const IO* dp = reinterpret_cast<const IO*>(a.delta) + row;
   const IO* zp = a.z ? reinterpret_cast<const IO*>(a.z) + row : nullptr;
   const IO* gp = reinterpret_cast<const IO*>(a.dout) + row;
   const bool bc_live = slot < N;  // the lane also stages B/C row `slot`, steps [8 q, 8 q + 8)
-  const long long bcrow = ((long long)b * N + (bc_live ? slot : 0)) * L + kHB * q;
+  const long long bcrow = ((long long)b * N + (bc_live ? slot : 0)) * L;
   const IO* Bp = reinterpret_cast<const IO*>(a.B) + bcrow;
   const IO* Cp = reinterpret_cast<const IO*>(a.C) + bcrow;
   float* sBw = reinterpret_cast<float*>(tl.sB);
@@ -264,26 +267,27 @@ __global__ void __launch_bounds__(128) bwd_kernel(const BwdArgs a) {
     const int nvalid = min(kBlk, L - t0);
     const int nown = max(0, min(kHB, nvalid - kHB * q));
     Row<IO, kHB> ru, rd, rz, rg, rb, rc;
+    const int tq = t0 + kHB * q;
     if (VEC && nown == kHB) {
-      load_row<IO, kHB, true>(ru, up + t0, kHB);
-      load_row<IO, kHB, true>(rd, dp + t0, kHB);
-      load_row<IO, kHB, true>(rg, gp + t0, kHB);
-      if (zp) load_row<IO, kHB, true>(rz, zp + t0, kHB);
+      load_steps<IO, kHB, true>(ru, up, L, tq, kHB, rev);
+      load_steps<IO, kHB, true>(rd, dp, L, tq, kHB, rev);
+      load_steps<IO, kHB, true>(rg, gp, L, tq, kHB, rev);
+      if (zp) load_steps<IO, kHB, true>(rz, zp, L, tq, kHB, rev);
     } else {
-      load_row<IO, kHB, false>(ru, up + t0, nown);
-      load_row<IO, kHB, false>(rd, dp + t0, nown);
-      load_row<IO, kHB, false>(rg, gp + t0, nown);
-      if (zp) load_row<IO, kHB, false>(rz, zp + t0, nown);
+      load_steps<IO, kHB, false>(ru, up, L, tq, nown, rev);
+      load_steps<IO, kHB, false>(rd, dp, L, tq, nown, rev);
+      load_steps<IO, kHB, false>(rg, gp, L, tq, nown, rev);
+      if (zp) load_steps<IO, kHB, false>(rz, zp, L, tq, nown, rev);
     }
     if (!bc_live) {
       rb.zero();
       rc.zero();
     } else if (VEC && nown == kHB) {
-      load_row<IO, kHB, true>(rb, Bp + t0, kHB);
-      load_row<IO, kHB, true>(rc, Cp + t0, kHB);
+      load_steps<IO, kHB, true>(rb, Bp, L, tq, kHB, rev);
+      load_steps<IO, kHB, true>(rc, Cp, L, tq, kHB, rev);
     } else {
-      load_row<IO, kHB, false>(rb, Bp + t0, nown);
-      load_row<IO, kHB, false>(rc, Cp + t0, nown);
+      load_steps<IO, kHB, false>(rb, Bp, L, tq, nown, rev);
+      load_steps<IO, kHB, false>(rc, Cp, L, tq, nown, rev);
     }
     // the state entering the block
     float2 hstart[4];
@@ -366,19 +370,14 @@ __global__ void __launch_bounds__(128) bwd_kernel(const BwdArgs a) {
       }
     }
     if (act && nown > 0) {
-      IO* o;
-      if (a.du) {
-        o = reinterpret_cast<IO*>(a.du) + row + t0;
-        if (VEC && nown == kHB) store_row<IO, kHB, true>(o, odu, kHB); else store_row<IO, kHB, false>(o, odu, nown);
-      }
-      if (a.ddelta) {
-        o = reinterpret_cast<IO*>(a.ddelta) + row + t0;
-        if (VEC && nown == kHB) store_row<IO, kHB, true>(o, odd, kHB); else store_row<IO, kHB, false>(o, odd, nown);
-      }
-      if (a.dz && zp) {
-        o = reinterpret_cast<IO*>(a.dz) + row + t0;
-        if (VEC && nown == kHB) store_row<IO, kHB, true>(o, odz, kHB); else store_row<IO, kHB, false>(o, odz, nown);
-      }
+      const auto put = [&](void* base, const float (&v)[kHB]) {
+        IO* o = reinterpret_cast<IO*>(base) + row;
+        if (VEC && nown == kHB) store_steps<IO, kHB, true>(o, v, L, tq, kHB, rev);
+        else store_steps<IO, kHB, false>(o, v, L, tq, nown, rev);
+      };
+      if (a.du) put(a.du, odu);
+      if (a.ddelta) put(a.ddelta, odd);
+      if (a.dz && zp) put(a.dz, odz);
     }
 
     // CTA partial of dB, dC for this block: add the warps' sums, one value per (step, n, which)
@@ -434,7 +433,7 @@ __global__ void bwd_finish_bc(const BwdArgs a, IO* dB, IO* dC) {
     s += a.part_bc[(((long long)(g * a.batch + b) * 2 + which) * kNS + n) * a.L + t];
   IO* dst = which == 0 ? dB : dC;
   if (!dst) return;
-  const long long o = ((long long)b * a.N + n) * a.L + t;
+  const long long o = ((long long)b * a.N + n) * a.L + (a.reverse ? a.L - 1 - t : t);
   if (sizeof(IO) == 2) reinterpret_cast<uint16_t*>(dst)[o] = f32_to_bf16(s);
   else reinterpret_cast<float*>(dst)[o] = s;
 }

@@ -30,6 +30,9 @@
 //     the "2024 Reading List: Neural Network" page, section on state-space models): Ā_t =
 //     exp(Δ_t A_d) is computed once per (channel, step) with Δ_t and Δ_t x_t, so the time loop
 //     runs no exponential at all (template KE = KO = -1);
+//   * reverse scan (the anti-causal direction of a bidirectional layer, "2024 Reading List:
+//     Neural Network", Hydra notes): the same recurrence in mirrored time; every time row is
+//     read and written mirrored (step t of the scan is row index L-1-t), nothing else changes;
 //   * few channels (long sequences): the time axis is split into S chunks.  A summary pass
 //     runs every chunk but the last from a zero state and records its end state and ΣΔ; a
 //     carry pass chains the chunk states h_in(j+1) = exp(A ΣΔ_j) h_in(j) + h_end(j) (the
@@ -192,14 +195,15 @@ struct ChunkLane {
   using Rows = BlockRows<IO, SPL>;
   using URow = Row<IO, SPL>;
 
+  // time rows at step 0 (scan order; a reverse scan reads and writes them mirrored)
   const IO* up;
   const IO* dp;
   const IO* zp;   // null: no gate
   const IO* Bp;
   const IO* Cp;
   IO* op;
-  int slot, q, bn, bh, t_end;
-  bool bc_live, softplus, act;
+  int slot, q, bn, bh, t_end, L;
+  bool bc_live, softplus, act, rev;
   float bias, Dd;
   float dlim;  // |Δ| < dlim keeps |Δ A log2 e| <= 126 for every state of the warp
   float a1;    // scalar decay: A_d (times log2 e on the bf16 path)
@@ -207,26 +211,27 @@ struct ChunkLane {
 
   // Rows of the block starting at tb; steps at or beyond t_end read as zero.
   __device__ __forceinline__ void fetch(Rows& r, int tb) const {
-    const int nv = max(0, min(SPL, t_end - tb - SPL * q));
-    const int nv8 = max(0, min(8, t_end - tb - 8 * bh));
+    const int tq = tb + SPL * q, t8 = tb + 8 * bh;
+    const int nv = max(0, min(SPL, t_end - tq));
+    const int nv8 = max(0, min(8, t_end - t8));
     if (VEC && nv == SPL) {
-      load_row<IO, SPL, true>(r.u, up + tb, SPL);
-      load_row<IO, SPL, true>(r.d, dp + tb, SPL);
-      if (zp) load_row<IO, SPL, true>(r.z, zp + tb, SPL);
+      load_steps<IO, SPL, true>(r.u, up, L, tq, SPL, rev);
+      load_steps<IO, SPL, true>(r.d, dp, L, tq, SPL, rev);
+      if (zp) load_steps<IO, SPL, true>(r.z, zp, L, tq, SPL, rev);
     } else {
-      load_row<IO, SPL, false>(r.u, up + tb, nv);
-      load_row<IO, SPL, false>(r.d, dp + tb, nv);
-      if (zp) load_row<IO, SPL, false>(r.z, zp + tb, nv);
+      load_steps<IO, SPL, false>(r.u, up, L, tq, nv, rev);
+      load_steps<IO, SPL, false>(r.d, dp, L, tq, nv, rev);
+      if (zp) load_steps<IO, SPL, false>(r.z, zp, L, tq, nv, rev);
     }
     if (!bc_live) {
       r.b.zero();
       r.c.zero();
     } else if (VEC && nv8 == 8) {
-      load_row<IO, 8, true>(r.b, Bp + tb, 8);
-      if (kReadout) load_row<IO, 8, true>(r.c, Cp + tb, 8);
+      load_steps<IO, 8, true>(r.b, Bp, L, t8, 8, rev);
+      if (kReadout) load_steps<IO, 8, true>(r.c, Cp, L, t8, 8, rev);
     } else {
-      load_row<IO, 8, false>(r.b, Bp + tb, nv8);
-      if (kReadout) load_row<IO, 8, false>(r.c, Cp + tb, nv8);
+      load_steps<IO, 8, false>(r.b, Bp, L, t8, nv8, rev);
+      if (kReadout) load_steps<IO, 8, false>(r.c, Cp, L, t8, nv8, rev);
     }
   }
 
@@ -289,8 +294,8 @@ struct ChunkLane {
 
   __device__ __forceinline__ void store_out(int t0, const float (&o)[SPL], int nown) const {
     if (!act || nown <= 0) return;
-    if (VEC && nown == SPL) store_row<IO, SPL, true>(op + t0, o, SPL);
-    else store_row<IO, SPL, false>(op + t0, o, nown);
+    if (VEC && nown == SPL) store_steps<IO, SPL, true>(op, o, L, t0 + SPL * q, SPL, rev);
+    else store_steps<IO, SPL, false>(op, o, L, t0 + SPL * q, nown, rev);
   }
 };
 
@@ -361,7 +366,7 @@ __device__ __forceinline__ void run_chunk(const FwdArgs& a, WarpTile<LPC>& tile,
   const int L = a.L, N = a.N;
 
   Lane ln;
-  const long long row = ch * (long long)L + SPL * q;     // this lane's steps of each block
+  const long long row = ch * (long long)L;  // the lane owns steps [SPL q, SPL q + SPL) of each block
   ln.up = reinterpret_cast<const IO*>(a.u) + row;
   ln.dp = reinterpret_cast<const IO*>(a.delta) + row;
   ln.zp = (kReadout && a.z) ? reinterpret_cast<const IO*>(a.z) + row : nullptr;
@@ -370,12 +375,14 @@ __device__ __forceinline__ void run_chunk(const FwdArgs& a, WarpTile<LPC>& tile,
   ln.bn = lane >> 1;
   ln.bh = lane & 1;
   ln.bc_live = ln.bn < N;
-  const long long bcrow = ((long long)b * N + (ln.bc_live ? ln.bn : 0)) * L + 8 * ln.bh;
+  const long long bcrow = ((long long)b * N + (ln.bc_live ? ln.bn : 0)) * L;
   ln.Bp = reinterpret_cast<const IO*>(a.B) + bcrow;
   ln.Cp = reinterpret_cast<const IO*>(a.C) + bcrow;
   ln.slot = slot;
   ln.q = q;
   ln.t_end = t_end;
+  ln.L = L;
+  ln.rev = a.reverse != 0;
   ln.softplus = a.softplus != 0;
   ln.act = act;
   ln.bias = bias;

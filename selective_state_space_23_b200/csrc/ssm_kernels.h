@@ -36,6 +36,7 @@ struct FwdArgs {
   int nchunk;           // S
   int softplus;
   int scalar_a;         // one decay rate A_d per channel, shared by its N states
+  int reverse;          // scan runs from t = L-1 down to 0 (time rows read/written mirrored)
   int lpc;              // lanes per channel: 1, 2 or 4 (16 / lpc states each)
   int warps_per_b;      // ceil(dim / (32 / lpc))
   long long nwarps;     // batch * warps_per_b
@@ -66,6 +67,7 @@ struct BwdArgs {
   int wpb;              // warps per CTA (channels per CTA = 16 * wpb)
   int ngroups;          // CTAs per batch row = ceil(warps_per_b / wpb)
   int kmufu;            // state pairs (of 4 per lane) whose exponential runs on MUFU: 2, 3 or 4
+  int reverse;          // gradients of the reverse scan (time rows read/written mirrored)
 };
 
 struct DecodeArgs {

@@ -1,6 +1,7 @@
 // Row I/O helpers shared by the scan kernels: E consecutive io elements of one row held as
 // 32-bit words, loaded with streaming 128-bit (or 64-bit) loads when aligned, stored back with
-// round-to-nearest-even bf16 packing.
+// round-to-nearest-even bf16 packing; the load_steps / store_steps forms address the row in scan
+// order, which is the row's own order or (reverse scan) its mirror image.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -88,6 +89,66 @@ __device__ __forceinline__ void store_row(IO* p, const float (&o)[E], int nvalid
 #pragma unroll
     for (int e = 0; e < E; ++e)
       if (e < nvalid) s[e] = o[e];
+  }
+}
+
+// Element order of a row reversed in place (row k <- row E-1-k).
+template <typename IO, int E>
+__device__ __forceinline__ void reverse_row(Row<IO, E>& r) {
+  constexpr int W = Row<IO, E>::kWords;
+  uint32_t t[W];
+#pragma unroll
+  for (int i = 0; i < W; ++i) t[i] = r.w[W - 1 - i];
+#pragma unroll
+  for (int i = 0; i < W; ++i) r.w[i] = sizeof(IO) == 2 ? __byte_perm(t[i], 0u, 0x1032) : t[i];
+}
+
+// E consecutive steps [tau, tau + E) of one time row in scan order.  In reverse order (rev) the
+// scan's step tau is stored at row index L-1-tau, so the E steps are the row's elements
+// [L-tau-E, L-tau) read backwards.  Steps at or beyond nvalid read as zero.  VEC: the row
+// segment is aligned as load_row requires and all E steps are valid.
+template <typename IO, int E, bool VEC>
+__device__ __forceinline__ void load_steps(Row<IO, E>& r, const IO* row, int L, int tau, int nvalid,
+                                           bool rev) {
+  if (!rev) {
+    load_row<IO, E, VEC>(r, row + tau, nvalid);
+  } else if (VEC) {
+    load_row<IO, E, true>(r, row + (L - tau - E), E);
+    reverse_row(r);
+  } else {
+    r.zero();
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      if (e < nvalid) {
+        if (sizeof(IO) == 4)
+          r.w[e] = __ldcs(reinterpret_cast<const uint32_t*>(row) + (L - 1 - tau - e));
+        else
+          r.w[e >> 1] |= ((uint32_t)__ldcs(reinterpret_cast<const unsigned short*>(row) +
+                                           (L - 1 - tau - e))) << (16 * (e & 1));
+      }
+    }
+  }
+}
+
+// Store E values of steps [tau, tau + E) (only the first nvalid) to a time row in scan order.
+template <typename IO, int E, bool VEC>
+__device__ __forceinline__ void store_steps(IO* row, const float (&o)[E], int L, int tau, int nvalid,
+                                            bool rev) {
+  if (!rev) {
+    store_row<IO, E, VEC>(row + tau, o, nvalid);
+  } else if (VEC) {
+    float rv[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) rv[e] = o[E - 1 - e];
+    store_row<IO, E, true>(row + (L - tau - E), rv, E);
+  } else {
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      if (e < nvalid) {
+        if (sizeof(IO) == 4) reinterpret_cast<float*>(row)[L - 1 - tau - e] = o[e];
+        else reinterpret_cast<uint16_t*>(row)[L - 1 - tau - e] = f32_to_bf16(o[e]);
+      }
+    }
   }
 }
 

@@ -10,6 +10,9 @@ Every test builds its expected value independently (a different formula or libra
   * chunked-vs-sequential state passing, superposition, decode-vs-scan;
   * the scalar decay (one A per channel, the Mamba-2 restriction in the reading-list notes) as
     a masked Gram-matrix product, and its rate gradient by central differences;
+  * the reverse scan (Hydra notes: the anti-causal half of a bidirectional layer) against the
+    anti-causal quadratic form, a two-step closed form of its final state, and central
+    differences of its gradients;
   * central finite differences of the forward pass for every gradient.
 """
 import numpy as np
@@ -307,6 +310,79 @@ def test_scalar_decay_gradient_is_the_state_sum():
         lp = loss_and_grads(dict(c, A=np.repeat(ap[:, None], 4, 1)), dout, dhL)
         lm = loss_and_grads(dict(c, A=np.repeat(am[:, None], 4, 1)), dout, dhL)
         np.testing.assert_allclose(g["dA"][d].sum(), (lp - lm) / (2 * eps), rtol=2e-6, atol=2e-7)
+
+
+# ------------------------------------------------------------------ reverse scan
+def quadratic_form_reverse(c, softplus=True):
+    """Anti-causal form: y_t = sum_{s>=t} C_t . exp(A sum_{r=t}^{s-1} Δ_r) Δ_s B_s u_s
+    + C_t . exp(A sum_{r=t}^{L-1} Δ_r) h0 + D u_t, then * silu(z_t) (h0 enters at t = L-1)."""
+    u, A, B, C = c["u"], c["A"], c["B"], c["C"]
+    batch, dim, L = u.shape
+    v = c["delta"] + c["dt_bias"][None, :, None]
+    dt = softplus_ref(v) if softplus else v
+    out = np.zeros_like(u)
+    for b in range(batch):
+        for d in range(dim):
+            cs = np.concatenate([[0.0], np.cumsum(dt[b, d])])  # cs[k] = sum_{r<k} Δ_r
+            for t in range(L):
+                y = 0.0
+                for s_ in range(t, L):
+                    decay = np.exp(A[d] * (cs[s_] - cs[t]))
+                    y += np.sum(C[b, :, t] * decay * dt[b, d, s_] * B[b, :, s_]) * u[b, d, s_]
+                if c["h0"] is not None:
+                    y += np.sum(C[b, :, t] * np.exp(A[d] * (cs[L] - cs[t])) * c["h0"][b, d])
+                y += c["D"][d] * u[b, d, t]
+                if c["z"] is not None:
+                    zz = c["z"][b, d, t]
+                    y *= zz * expit(zz)
+                out[b, d, t] = y
+    return out
+
+
+@pytest.mark.parametrize("gate,h0", [(True, True), (False, False)])
+def test_reverse_quadratic_form(gate, h0):
+    c = rand_case(batch=2, dim=3, L=9, N=3, gate=gate, h0=h0, seed=71)
+    got = run(c, reverse=True)["out"]
+    np.testing.assert_allclose(got, quadratic_form_reverse(c), rtol=1e-11, atol=1e-12)
+    # a reverse scan is not the forward scan: the pin tells them apart
+    assert not np.allclose(run(c)["out"], got, rtol=1e-3)
+
+
+def test_reverse_final_state_single_step_chain():
+    """hL of the reverse scan is the state after t = 0: for L = 2 it is
+    a_0 (a_1 h0 + b_1) + b_0 with a_t = exp(Δ_t A), b_t = Δ_t B_t u_t."""
+    c = rand_case(batch=1, dim=2, L=2, N=4, seed=72)
+    dt = softplus_ref(c["delta"] + c["dt_bias"][None, :, None])[0]          # [d, t]
+    a = np.exp(dt[:, :, None] * c["A"][:, None, :])                         # [d, t, n]
+    bt = dt[:, :, None] * c["B"][0].T[None] * c["u"][0][:, :, None]          # [d, t, n]
+    h = a[:, 0] * (a[:, 1] * c["h0"][0] + bt[:, 1]) + bt[:, 0]
+    np.testing.assert_allclose(run(c, reverse=True)["hL"][0], h, rtol=1e-13, atol=1e-14)
+
+
+def test_reverse_gradients_by_finite_differences():
+    c = rand_case(batch=1, dim=2, L=5, N=3, seed=73)
+    r = np.random.default_rng(74)
+    dout = r.standard_normal(c["u"].shape)
+    dhL = r.standard_normal(c["h0"].shape)
+    g = oracle.scan_bwd(c["u"], c["delta"], c["A"], c["B"], c["C"], dout, D=c["D"], z=c["z"],
+                        dt_bias=c["dt_bias"], h0=c["h0"], dhL=dhL, reverse=True)
+
+    def loss(cc):
+        res = run(cc, reverse=True)
+        return np.sum(res["out"] * dout) + np.sum(res["hL"] * dhL)
+
+    eps = 1e-6
+    for key, gname in (("u", "du"), ("delta", "ddelta"), ("B", "dB"), ("C", "dC"), ("z", "dz"),
+                       ("A", "dA"), ("h0", "dh0")):
+        x = c[key]
+        num = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            i = it.multi_index
+            xp = x.copy(); xp[i] += eps
+            xm = x.copy(); xm[i] -= eps
+            num[i] = (loss(dict(c, **{key: xp})) - loss(dict(c, **{key: xm}))) / (2 * eps)
+        np.testing.assert_allclose(g[gname], num, rtol=2e-6, atol=2e-7, err_msg=gname)
 
 
 def test_planted_mistake_is_caught():
