@@ -185,11 +185,16 @@ SSM_API int ssm_scan_bwd_scalar_a(const void* u, const void* delta, const float*
  *                 mirrored.  Checkpoints are indexed by blocks of 16 steps in scan order
  *                 (block k holds the state before scan steps 16k .. 16k+15, i.e. before time
  *                 index L-1-16k), and only feed ssm_scan_bwd_ex with the same flags.
+ *   SSM_ZOH       the zero-order-hold input term of the discretisation ("Yöntem":
+ *                 B̄ = (ΔA)^{-1}(exp(ΔA) - I) ΔB): h_t = Ā h_{t-1} + c B_t x_t with
+ *                 c = (exp(Δ_t A) - 1)/A per state (c -> Δ_t as A -> 0) instead of Δ_t.
+ *                 Combines with the other flags.
  * Any other bit is rejected with SSM_EINVAL.  Arguments are those of ssm_scan_fwd /
  * ssm_scan_bwd plus flags.
  */
 #define SSM_SCALAR_A 1
 #define SSM_REVERSE 2
+#define SSM_ZOH 4
 SSM_API size_t ssm_scan_fwd_ex_workspace_size(int batch, int dim, int seqlen, int dstate,
                                               int io_dtype, int flags);
 SSM_API int ssm_scan_fwd_ex(const void* u, const void* delta, const float* A, const void* B,

@@ -9,7 +9,8 @@ The arithmetic lives in ``ssm_oracle.c`` (plain double-precision loops, cited th
                          out_t = y_t * silu(z_t); Δ_t = softplus(delta_t + dt_bias).
                          ("Mamba: Linear-Time Sequence Modeling with Selective State Spaces",
                          summary page, sections "Yöntem" and "Seçim Mekanizması (S6)").
-  * ``scan_bwd``      -- gradients of ``scan_fwd`` by the chain rule (reverse-time adjoint).
+  * ``scan_bwd``      -- gradients of ``scan_fwd`` by the chain rule (reverse-time adjoint),
+                         for the Euler input term and for the ZOH one (``zoh=True``).
                          The pages give no gradient formula: this function is pinned only by
                          finite differences of ``scan_fwd`` (parity of the gradient formulas
                          themselves is otherwise unpinned by the pages).
@@ -128,8 +129,9 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=Tru
 
 
 def scan_bwd(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None, delta_softplus=True,
-             h0=None, dhL=None, channels=None, nthreads=0, reverse=False):
-    """Gradients of :func:`scan_fwd` (Euler input term) w.r.t. every input, in fp64.
+             h0=None, dhL=None, channels=None, nthreads=0, reverse=False, zoh=False):
+    """Gradients of :func:`scan_fwd` (Euler input term, or ZOH with ``zoh``) w.r.t. every
+    input, in fp64.
 
     Returns dict(du, ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0).  With ``channels`` the
     summed gradients (dA, dB, dC, dD, ddt_bias) hold only those channels' contributions.
@@ -138,7 +140,7 @@ def scan_bwd(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None, delta_softpl
     if reverse:
         g = scan_bwd(_flip(u), _flip(delta), A, _flip(B), _flip(C), _flip(dout), D=D, z=_flip(z),
                      dt_bias=dt_bias, delta_softplus=delta_softplus, h0=h0, dhL=dhL,
-                     channels=channels, nthreads=nthreads)
+                     channels=channels, nthreads=nthreads, zoh=zoh)
         for k in ("du", "ddelta", "dz", "dB", "dC"):
             g[k] = _flip(g[k])
         return g
@@ -165,7 +167,7 @@ def scan_bwd(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None, delta_softpl
     keep, cp, nc = _chans(channels)
     rc = _lib().oracle_scan_bwd(
         batch, dim, L, N, _p(u), _p(delta), _p(A), _p(B), _p(C), _p(D), _p(z), _p(dt_bias),
-        int(bool(delta_softplus)), _p(h0), _p(dout), _p(dhL),
+        int(bool(delta_softplus)), int(bool(zoh)), _p(h0), _p(dout), _p(dhL),
         _p(g["du"]), _p(g["ddelta"]), _p(g["dA"]), _p(g["dB"]), _p(g["dC"]), _p(g["dD"]),
         _p(g["dz"]), _p(g["ddt_bias"]), _p(g["dh0"]), cp, ctypes.c_int64(nc), int(nthreads))
     if rc != 0:

@@ -22,7 +22,7 @@
  *
  * Readings taken where the pages are silent (each is listed in the design notes):
  *   - Input term: B̄ x_t = Δ_t * B_t * x_t (first-order/Euler form).  The exact ZOH
- *     input term (exp(ΔA)-1)/A * B_t * x_t is available with zoh=1 (forward only).
+ *     input term (exp(ΔA)-1)/A * B_t * x_t is available with zoh=1 (forward and backward).
  *   - A is a general real [D][N] matrix (diagonal state matrix per channel).
  *   - softplus(v) = log(1 + exp(v)), evaluated in the overflow-safe form.
  *   - The skip term D*x_t is added to y_t before the gate; z == NULL means no gate.
@@ -68,6 +68,26 @@ static double input_coef(double dt, double a_dn, int zoh) {
   if (!zoh) return dt;                 /* B̄ x = Δ B x */
   if (a_dn == 0.0) return dt;          /* limit of (exp(ΔA)-1)/A as A -> 0 */
   return expm1(dt * a_dn) / a_dn;      /* ZOH: (ΔA)^-1 (exp(ΔA) - 1) Δ  for diagonal A */
+}
+
+/* d/dΔ and d/dA of the input coefficient.  Euler: (1, 0).  ZOH, c = (e^{ΔA} - 1)/A:
+ * dc/dΔ = e^{ΔA};  dc/dA = (Δ e^{ΔA} - c)/A = Δ^2 ψ(ΔA) with ψ(y) = (y e^y - e^y + 1)/y^2,
+ * evaluated by its Taylor series Σ_{k>=2} (k-1) y^{k-2}/k! = 1/2 + y/3 + y^2/8 + y^3/30 + ...
+ * where the direct form cancels (|ΔA| < 1e-2; truncation after y^5 < 1e-15 relative). */
+static void input_coef_grad(double dt, double a_dn, int zoh, double* d_dt, double* d_da) {
+  if (!zoh) {
+    *d_dt = 1.0;
+    *d_da = 0.0;
+    return;
+  }
+  const double y = dt * a_dn;
+  *d_dt = exp(y);
+  if (fabs(y) < 1e-2) {
+    const double psi = 0.5 + y * (1.0 / 3.0 + y * (1.0 / 8.0 + y * (1.0 / 30.0 + y * (1.0 / 144.0 + y / 840.0))));
+    *d_da = dt * dt * psi;
+  } else {
+    *d_da = (dt * exp(y) - expm1(y) / a_dn) / a_dn;
+  }
 }
 
 static int nthreads_or_default(int nthreads) {
@@ -142,18 +162,19 @@ int oracle_scan_fwd(int batch, int dim, int seqlen, int dstate,
 }
 
 /*
- * Backward pass of the forward scan above (Euler input term), by the chain rule through
- * the same recurrence run in reverse time.  The pages state only that the backward pass
+ * Backward pass of the forward scan above, by the chain rule through the same recurrence run
+ * in reverse time.  Written for the Euler input term (c = Δ); with zoh=1 the coefficient is
+ * c_n = (e^{ΔA_n} - 1)/A_n and the terms below take c_n, dc/dΔ and dc/dA in place of Δ, 1, 0.  The pages state only that the backward pass
  * recomputes the intermediate states instead of storing them; the oracle simply keeps
  * the whole per-channel state history in host memory.
  *
  *   g_t      = dout_t * silu(z_t)                    (dL/dy_t)
  *   λ_t      = g_t C_t + Ā_{t+1} λ_{t+1},  λ_{L-1} = g_{L-1} C_{L-1} + dhL
  *   dC_t    += g_t h_t            dB_t += λ_t Δ_t x_t          (summed over channels d)
- *   du_t     = g_t D + Δ_t Σ_n λ_t B_t
- *   dΔ_t     = Σ_n λ_t (A Ā_t h_{t-1} + B_t x_t)
+ *   du_t     = g_t D + Σ_n λ_t c_n B_t              (c_n = Δ_t for the Euler term)
+ *   dΔ_t     = Σ_n λ_t (A Ā_t h_{t-1} + dc/dΔ B_t x_t)
  *   ddelta_t = dΔ_t * sigmoid(delta_t + dt_bias)  (softplus' ; 1 without softplus)
- *   dA      += λ_t Δ_t Ā_t h_{t-1}     dD += g_t x_t     ddt_bias += ddelta_t
+ *   dA      += λ_t (Δ_t Ā_t h_{t-1} + dc/dA B_t x_t)     dD += g_t x_t     ddt_bias += ddelta_t
  *   dz_t     = dout_t y_t silu'(z_t)   dh0 = Ā_0 λ_0
  *
  * Gradients dB, dC, dA, dD, ddt_bias are ACCUMULATED (+=) into the given arrays, which the
@@ -163,7 +184,7 @@ int oracle_scan_fwd(int batch, int dim, int seqlen, int dstate,
 int oracle_scan_bwd(int batch, int dim, int seqlen, int dstate,
                     const double* u, const double* delta, const double* A,
                     const double* B, const double* C, const double* Dskip,
-                    const double* z, const double* dt_bias, int delta_softplus,
+                    const double* z, const double* dt_bias, int delta_softplus, int zoh,
                     const double* h0, const double* dout, const double* dhL,
                     double* du, double* ddelta, double* dA, double* dB, double* dC,
                     double* dD, double* dz, double* ddt_bias, double* dh0,
@@ -213,7 +234,7 @@ int oracle_scan_bwd(int batch, int dim, int seqlen, int dstate,
         for (int n = 0; n < dstate; ++n) {
           const double hp = hist[(size_t)t * dstate + n];
           hist[(size_t)(t + 1) * dstate + n] =
-              exp(dt * Ad[n]) * hp + dt * Bb[(int64_t)n * seqlen + t] * uc[t];
+              exp(dt * Ad[n]) * hp + input_coef(dt, Ad[n], zoh) * Bb[(int64_t)n * seqlen + t] * uc[t];
         }
       }
       /* reverse */
@@ -233,22 +254,26 @@ int oracle_scan_bwd(int batch, int dim, int seqlen, int dstate,
         } else if (dz) {
           dz[ch * seqlen + t] = 0.0;
         }
-        double s1 = 0.0, s2 = 0.0;
+        double s1 = 0.0, s2 = 0.0, s3 = 0.0;
         for (int n = 0; n < dstate; ++n) {
           const double Bt = Bb[(int64_t)n * seqlen + t];
           const double Ct = Cb[(int64_t)n * seqlen + t];
           const double abar = exp(dt * Ad[n]);
+          const double c = input_coef(dt, Ad[n], zoh);
+          double c_dt, c_da;
+          input_coef_grad(dt, Ad[n], zoh, &c_dt, &c_da);
           lam[n] += g * Ct;                                /* λ_t complete */
           const double q = abar * hp[n];                   /* Ā_t h_{t-1} */
-          accB[(size_t)b * dstate * seqlen + (size_t)n * seqlen + t] += lam[n] * dt * x;
+          accB[(size_t)b * dstate * seqlen + (size_t)n * seqlen + t] += lam[n] * c * x;
           accC[(size_t)b * dstate * seqlen + (size_t)n * seqlen + t] += g * ht[n];
-          accA[(size_t)d * dstate + n] += lam[n] * dt * q;
-          s1 += lam[n] * Bt;
+          accA[(size_t)d * dstate + n] += lam[n] * (dt * q + c_da * Bt * x);
+          s1 += lam[n] * c * Bt;
           s2 += lam[n] * Ad[n] * q;
+          s3 += lam[n] * c_dt * Bt;
           lam[n] *= abar;                                  /* becomes Ā_t λ_t for step t-1 */
         }
-        if (du) du[ch * seqlen + t] = g * skip + dt * s1;
-        const double ddt = x * s1 + s2;
+        if (du) du[ch * seqlen + t] = g * skip + s1;
+        const double ddt = x * s3 + s2;
         const double ddl = delta_softplus ? ddt * sp_sigmoid(dc[t] + bias) : ddt;
         if (ddelta) ddelta[ch * seqlen + t] = ddl;
         accD[d] += g * x;

@@ -82,8 +82,13 @@ def _workspace(nbytes, device, given):
     return torch.empty(nbytes, dtype=torch.uint8, device=device)
 
 
+def _flags(scalar_a, reverse, zoh):
+    return ((_abi.SSM_SCALAR_A if scalar_a else 0) | (_abi.SSM_REVERSE if reverse else 0)
+            | (_abi.SSM_ZOH if zoh else 0))
+
+
 def _scan_fwd(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, return_final_state,
-              return_ckpt, out, workspace, scalar_a, reverse):
+              return_ckpt, out, workspace, scalar_a, reverse, zoh):
     dev = u.device
     batch, dim, L = u.shape
     N = B.shape[1]
@@ -104,7 +109,7 @@ def _scan_fwd(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, return_final
     hL = torch.empty((batch, dim, N), dtype=torch.float32, device=dev) if return_final_state else None
     nblk = (L + CKPT_STEPS - 1) // CKPT_STEPS
     ckpt = torch.empty((batch, dim, nblk, N), dtype=torch.float32, device=dev) if return_ckpt else None
-    flags = (_abi.SSM_SCALAR_A if scalar_a else 0) | (_abi.SSM_REVERSE if reverse else 0)
+    flags = _flags(scalar_a, reverse, zoh)
     nws = int(_abi.lib().ssm_scan_fwd_ex_workspace_size(batch, dim, L, N, code, flags))
     ws = _workspace(nws, dev, workspace)
     rc = _abi.lib().ssm_scan_fwd_ex(
@@ -124,24 +129,25 @@ def _scan_fwd(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, return_final
 
 def ssm_scan_fwd(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=True, h0=None,
                  return_final_state=False, return_ckpt=False, out=None, workspace=None,
-                 reverse=False):
+                 reverse=False, zoh=False):
     """Forward scan.  u, delta, z: [batch, dim, L]; B, C: [batch, N, L] (io dtype f32 or bf16);
     A: [dim, N] f32; D, dt_bias: [dim] f32; h0: [batch, dim, N] f32.  reverse: scan from
-    t = L-1 down to 0.  Returns out, or a tuple (out, hL?, ckpt?) when those are requested."""
+    t = L-1 down to 0.  zoh: zero-order-hold input term (e^{ΔA} - 1)/A B x instead of Δ B x.
+    Returns out, or a tuple (out, hL?, ckpt?) when those are requested."""
     return _scan_fwd(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, return_final_state,
-                     return_ckpt, out, workspace, False, reverse)
+                     return_ckpt, out, workspace, False, reverse, zoh)
 
 
 def ssm_scan_fwd_scalar_a(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=True,
                           h0=None, return_final_state=False, return_ckpt=False, out=None,
-                          workspace=None, reverse=False):
+                          workspace=None, reverse=False, zoh=False):
     """Forward scan with one decay rate per channel: as :func:`ssm_scan_fwd` with A [dim] f32."""
     return _scan_fwd(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, return_final_state,
-                     return_ckpt, out, workspace, True, reverse)
+                     return_ckpt, out, workspace, True, reverse, zoh)
 
 
 def _scan_bwd(u, delta, A, B, C, dout, D, z, dt_bias, delta_softplus, h0, dhL, ckpt,
-              workspace, need, scalar_a, reverse):
+              workspace, need, scalar_a, reverse, zoh):
     dev = u.device
     batch, dim, L = u.shape
     N = B.shape[1]
@@ -175,7 +181,7 @@ def _scan_bwd(u, delta, A, B, C, dout, D, z, dt_bias, delta_softplus, h0, dhL, c
         "ddt_bias": e((dim,), torch.float32) if "ddt_bias" in want else None,
         "dh0": e((batch, dim, N), torch.float32) if "dh0" in want else None,
     }
-    flags = (_abi.SSM_SCALAR_A if scalar_a else 0) | (_abi.SSM_REVERSE if reverse else 0)
+    flags = _flags(scalar_a, reverse, zoh)
     nws = int(_abi.lib().ssm_scan_bwd_ex_workspace_size(batch, dim, L, N, code,
                                                          int(ckpt is not None), flags))
     ws = _workspace(nws, dev, workspace)
@@ -190,19 +196,20 @@ def _scan_bwd(u, delta, A, B, C, dout, D, z, dt_bias, delta_softplus, h0, dhL, c
 
 
 def ssm_scan_bwd(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None, delta_softplus=True,
-                 h0=None, dhL=None, ckpt=None, workspace=None, need=None, reverse=False):
+                 h0=None, dhL=None, ckpt=None, workspace=None, need=None, reverse=False,
+                 zoh=False):
     """Gradients of :func:`ssm_scan_fwd`.  Returns a dict with du, ddelta, dA, dB, dC, dD, dz,
     ddt_bias, dh0 (entries are None when the matching input is absent or not in ``need``)."""
     return _scan_bwd(u, delta, A, B, C, dout, D, z, dt_bias, delta_softplus, h0, dhL, ckpt,
-                     workspace, need, False, reverse)
+                     workspace, need, False, reverse, zoh)
 
 
 def ssm_scan_bwd_scalar_a(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None,
                           delta_softplus=True, h0=None, dhL=None, ckpt=None, workspace=None,
-                          need=None, reverse=False):
+                          need=None, reverse=False, zoh=False):
     """Gradients of :func:`ssm_scan_fwd_scalar_a` (dA is [dim])."""
     return _scan_bwd(u, delta, A, B, C, dout, D, z, dt_bias, delta_softplus, h0, dhL, ckpt,
-                     workspace, need, True, reverse)
+                     workspace, need, True, reverse, zoh)
 
 
 def ssm_state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=True,

@@ -268,7 +268,8 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
                   size_t workspace_bytes, int batch, int dim, int seqlen, int dstate,
                   int io_dtype, void* stream, int flags) {
   g_err[0] = 0;
-  if (flags & ~(SSM_SCALAR_A | SSM_REVERSE)) return fail(SSM_EINVAL, "unknown flags 0x%x", flags);
+  if (flags & ~(SSM_SCALAR_A | SSM_REVERSE | SSM_ZOH))
+    return fail(SSM_EINVAL, "unknown flags 0x%x", flags);
   const bool scalar_a = (flags & SSM_SCALAR_A) != 0;
   TRY(check_dims(batch, dim, seqlen, dstate, io_dtype));
   const size_t es = esize(io_dtype);
@@ -308,7 +309,8 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
   a.softplus = delta_softplus ? 1 : 0;
   a.scalar_a = scalar_a ? 1 : 0;
   a.reverse = (flags & SSM_REVERSE) ? 1 : 0;
-  a.lpc = scalar_a ? 2 : fwd_lpc();
+  a.zoh = (flags & SSM_ZOH) ? 1 : 0;
+  a.lpc = (scalar_a || a.zoh) ? 2 : fwd_lpc();
   a.warps_per_b = (dim + 32 / a.lpc - 1) / (32 / a.lpc);
   a.nwarps = (long long)batch * a.warps_per_b;
   const bool vec = (seqlen * es) % 16 == 0 && aligned16(u) && aligned16(delta) && aligned16(z) &&
@@ -415,7 +417,7 @@ int scan_bwd_core(const void* u, const void* delta, const float* A, const void* 
                   void* du, void* ddelta, float* dA, void* dB, void* dC, float* dD, void* dz,
                   float* ddt_bias, float* dh0, void* workspace, size_t workspace_bytes,
                   int batch, int dim, int seqlen, int dstate, int io_dtype, void* stream,
-                  bool reverse) {
+                  bool reverse, bool zoh) {
   TRY(check_dims(batch, dim, seqlen, dstate, io_dtype));
   const size_t es = esize(io_dtype);
   const size_t nx = (size_t)batch * dim * seqlen * es;
@@ -474,7 +476,8 @@ int scan_bwd_core(const void* u, const void* delta, const float* A, const void* 
     a.chunk_len = (int)nblk * ssm::kBlk; a.nchunk = 1;
     a.softplus = delta_softplus ? 1 : 0;
     a.reverse = reverse ? 1 : 0;
-    a.lpc = fwd_lpc();
+    a.zoh = zoh ? 1 : 0;
+    a.lpc = zoh ? 2 : fwd_lpc();
     a.warps_per_b = fwd_warps_per_b(dim);
     a.nwarps = (long long)batch * a.warps_per_b;
     if ((e = ssm::launch_fwd(a, io_dtype, vec, ssm::kFwdCkpt, fwd_wpb(), fwd_kmufu(a.nwarps), s)) != cudaSuccess)
@@ -490,6 +493,7 @@ int scan_bwd_core(const void* u, const void* delta, const float* A, const void* 
   b.batch = batch; b.dim = dim; b.L = seqlen; b.N = dstate;
   b.softplus = delta_softplus ? 1 : 0;
   b.reverse = reverse ? 1 : 0;
+  b.zoh = zoh ? 1 : 0;
   b.warps_per_b = (dim + 15) / 16;
   b.nwarps = (long long)batch * b.warps_per_b;
   b.wpb = l.wpb;
@@ -514,12 +518,12 @@ int ssm_scan_bwd(const void* u, const void* delta, const float* A, const void* B
   g_err[0] = 0;
   return scan_bwd_core(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL, ckpt, du,
                        ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, workspace, workspace_bytes,
-                       batch, dim, seqlen, dstate, io_dtype, stream, false);
+                       batch, dim, seqlen, dstate, io_dtype, stream, false, false);
 }
 
 size_t ssm_scan_bwd_ex_workspace_size(int batch, int dim, int seqlen, int dstate, int io_dtype,
                                       int have_ckpt, int flags) {
-  if (flags & ~(SSM_SCALAR_A | SSM_REVERSE)) return 0;
+  if (flags & ~(SSM_SCALAR_A | SSM_REVERSE | SSM_ZOH)) return 0;
   const size_t base = ssm_scan_bwd_workspace_size(batch, dim, seqlen, dstate, io_dtype, have_ckpt);
   if (base == 0 || !(flags & SSM_SCALAR_A)) return base;
   return align_up((size_t)dim * dstate * 4) * 2 + base;
@@ -533,13 +537,15 @@ int ssm_scan_bwd_ex(const void* u, const void* delta, const float* A, const void
                     size_t workspace_bytes, int batch, int dim, int seqlen, int dstate,
                     int io_dtype, int flags, void* stream) {
   g_err[0] = 0;
-  if (flags & ~(SSM_SCALAR_A | SSM_REVERSE)) return fail(SSM_EINVAL, "unknown flags 0x%x", flags);
-  const bool reverse = (flags & SSM_REVERSE) != 0;
+  if (flags & ~(SSM_SCALAR_A | SSM_REVERSE | SSM_ZOH))
+    return fail(SSM_EINVAL, "unknown flags 0x%x", flags);
+  const bool reverse = (flags & SSM_REVERSE) != 0, zoh = (flags & SSM_ZOH) != 0;
   TRY(check_dims(batch, dim, seqlen, dstate, io_dtype));
   if (!(flags & SSM_SCALAR_A))
     return scan_bwd_core(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL, ckpt,
                          du, ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, workspace,
-                         workspace_bytes, batch, dim, seqlen, dstate, io_dtype, stream, reverse);
+                         workspace_bytes, batch, dim, seqlen, dstate, io_dtype, stream, reverse,
+                         zoh);
   // scalar decay: broadcast A over the states, run the per-state backward, sum dA over n
   TRY(check_ptr(A, (size_t)dim * 4, 4, "A"));
   TRY(check_opt(dA, (size_t)dim * 4, 4, "dA"));
@@ -562,7 +568,7 @@ int ssm_scan_bwd_ex(const void* u, const void* delta, const float* A, const void
   const int rc = scan_bwd_core(u, delta, Af, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL,
                                ckpt, du, ddelta, dA ? dAf : nullptr, dB, dC, dD, dz, ddt_bias,
                                dh0, w + 2 * head, workspace_bytes - 2 * head, batch, dim, seqlen,
-                               dstate, io_dtype, stream, reverse);
+                               dstate, io_dtype, stream, reverse, zoh);
   if (rc != SSM_OK) return rc;
   if (dA) {
     reduce_da_kernel<<<(unsigned)((dim + 255) / 256), 256, 0, s>>>(dAf, dA, dim, dstate);

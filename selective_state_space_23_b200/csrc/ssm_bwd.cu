@@ -11,7 +11,11 @@
 //   dΔ_t = Σ_n λ_t (A Ā_t h_{t-1} + B_t x_t),   ddelta_t = dΔ_t * sigmoid(delta_t + dt_bias)
 //   dA   = Σ_{b,t} λ_t Δ_t Ā_t h_{t-1},  dD = Σ_{b,t} g_t x_t,  ddt_bias = Σ_{b,t} ddelta_t
 //   dz_t = dout_t y_t silu'(z_t),  dh0 = Ā_0 λ_0
-// with Ā_t h_{t-1} = h_t - Δ_t B_t x_t, so the reverse sweep needs only h_t.
+// with Ā_t h_{t-1} = h_t - Δ_t B_t x_t, so the reverse sweep needs only h_t.  With the
+// zero-order-hold input term ("Yöntem": B̄ = (ΔA)^{-1}(e^{ΔA} - I) ΔB) the coefficient of B_t x_t
+// is c = (e^{ΔA} - 1)/A per state instead of Δ: dB_t = Σ_d λ_t c x_t, du_t = g_t D + Σ_n λ_t c B_t,
+// dΔ_t = Σ_n λ_t Ā_t (A h_{t-1} + B_t x_t) (dc/dΔ = Ā) and dA gains λ_t (dc/dA) B_t x_t with
+// dc/dA = (Δ Ā - c)/A, or Δ^2 (1/2 + y/3 + y^2/8) for |y = ΔA| < 0.01 where that form cancels.
 //
 // Mapping: two lanes per channel, 8 states each in registers; a warp holds 16 consecutive d of
 // one batch row.  Time is walked backwards in 16-step blocks; each block is handled in two halves
@@ -51,13 +55,30 @@ struct BwdTile {
   float wres[kBlk * 32];       // the warp's channel sums [step][half * 16 + (dB n | dC n)]
 };
 
+// Ā and the ZOH coefficient c = (e^{ΔA} - 1)/A of two states: library expf/expm1f on the fp32
+// path, the FMA-pipe form (zoh_coef_x2) on the bf16 path.  al = A (fp32) or A log2 e (bf16).
+template <bool PRECISE, bool CLAMP>
+__device__ __forceinline__ void zoh_pair(float2 d2, float2 al, float2 ra, float2& av, float2& c) {
+  if (PRECISE) {
+    const float2 y = mul2(d2, al);
+    av = make_float2(expf(y.x), expf(y.y));
+    c = mul2(make_float2(expm1f(y.x), expm1f(y.y)), ra);
+  } else {
+    zoh_coef_x2<CLAMP>(d2, al, ra, av, c);
+  }
+}
+
+__device__ __forceinline__ float2 dx2_of(float2 dd) { return f2(dd.y); }
+
 // One replayed step for one lane (8 states): h <- Ā h + Δ x B.  KP of the 4 state pairs take 2^x
 // from MUFU, the rest from the FMA-pipe polynomial (only used in range-checked blocks).  Returns
 // the partial readout Σ C h over the lane's states when READOUT.
 template <bool PRECISE, bool READOUT, int KP>
-__device__ __forceinline__ float replay_step(float2 (&hh)[4], const float2 (&al)[4], float2 dd,
-                                             const float4* bq, const float4* cq) {
-  const float2 d2 = f2(dd.x), dx2 = f2(dd.y);
+__device__ __forceinline__ float replay_step(float2 (&hh)[4], const float2 (&al)[4],
+                                             const float2 (&ra)[4], float2 dd, const float4* bq,
+                                             const float4* cq) {
+  constexpr bool kZoh = KP == kKpZoh || KP == kKpZohClamped;
+  const float2 d2 = f2(dd.x), dx2 = f2(dd.y);  // (Δ, Δx), or (Δ, x) with the ZOH term
   const float4 b0 = bq[0], b1 = bq[1];
   float4 c0 = make_float4(0.f, 0.f, 0.f, 0.f), c1 = c0;
   if (READOUT) {
@@ -69,8 +90,12 @@ __device__ __forceinline__ float replay_step(float2 (&hh)[4], const float2 (&al)
   for (int j = 0; j < 4; ++j) {
     const float4 bb = j < 2 ? b0 : b1;
     const float2 bp = (j & 1) ? make_float2(bb.z, bb.w) : make_float2(bb.x, bb.y);
-    float2 av;
-    if (PRECISE) {
+    float2 av, bx = dx2;
+    if (kZoh) {
+      float2 c;
+      zoh_pair<PRECISE, KP == kKpZohClamped>(d2, al[j], ra[j], av, c);
+      bx = mul2(c, dx2);
+    } else if (PRECISE) {
       av = make_float2(expf(dd.x * al[j].x), expf(dd.x * al[j].y));
     } else if (j < KP) {
       const float2 x = mul2(d2, al[j]);
@@ -78,7 +103,7 @@ __device__ __forceinline__ float replay_step(float2 (&hh)[4], const float2 (&al)
     } else {
       av = exp2_fma_prod_x2(d2, al[j]);
     }
-    hh[j] = fma2(av, hh[j], mul2(dx2, bp));
+    hh[j] = fma2(av, hh[j], mul2(bx, bp));
     if (READOUT) {
       const float4 cc = j < 2 ? c0 : c1;
       const float2 cp = (j & 1) ? make_float2(cc.z, cc.w) : make_float2(cc.x, cc.y);
@@ -94,13 +119,15 @@ __device__ __forceinline__ float replay_step(float2 (&hh)[4], const float2 (&al)
 // accumulates dA, Σ λB and Σ A λ Ā h_{t-1}, and advances λ <- Ā_t λ_t.
 template <bool PRECISE, int KP>
 __device__ __forceinline__ void adjoint_step(float2 (&lam)[4], float2 (&dA)[4], const float2 (&al)[4],
+                                             const float2 (&ra)[4], float aback,
                                              const float2 (&hk)[4], float2 dd, float g, float live,
                                              const float4* bq, const float4* cq, float2 (&vals)[8],
-                                             float& S1, float& S2) {
+                                             float& S1, float& S2, float& S3) {
+  constexpr bool kZoh = KP == kKpZoh || KP == kKpZohClamped;
   const float2 d2 = f2(dd.x), ndx2 = f2(-dd.y), g2 = f2(g);
   const float2 dxl = f2(dd.y * live), gl = f2(g * live);
   const float4 b0 = bq[0], b1 = bq[1], c0 = cq[0], c1 = cq[1];
-  float2 s1 = make_float2(0.f, 0.f), s2 = s1;
+  float2 s1 = make_float2(0.f, 0.f), s2 = s1, s3 = s1;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const float4 bb = j < 2 ? b0 : b1;
@@ -108,6 +135,28 @@ __device__ __forceinline__ void adjoint_step(float2 (&lam)[4], float2 (&dA)[4], 
     const float2 bp = (j & 1) ? make_float2(bb.z, bb.w) : make_float2(bb.x, bb.y);
     const float2 cp = (j & 1) ? make_float2(cc.z, cc.w) : make_float2(cc.x, cc.y);
     float2 av;
+    if (kZoh) {
+      // (Δ, x) in dd; c = (e^{ΔA} - 1)/A per state
+      float2 c;
+      zoh_pair<PRECISE, KP == kKpZohClamped>(d2, al[j], ra[j], av, c);
+      lam[j] = fma2(g2, cp, lam[j]);                        // λ_t complete
+      const float2 cx = mul2(c, dx2_of(dd));
+      vals[j] = mul2(lam[j], mul2(cx, f2(live)));           // dB_t contribution: λ c x
+      vals[4 + j] = mul2(gl, hk[j]);                        // dC_t contribution: g h_t
+      const float2 qv = fma2(make_float2(-cx.x, -cx.y), bp, hk[j]);  // Ā h_{t-1} = h_t - c x B
+      const float2 lq = mul2(lam[j], qv);
+      s1 = fma2(mul2(lam[j], c), bp, s1);                   // Σ λ c B        (du)
+      s2 = fma2(al[j], lq, s2);                             // Σ A λ Ā h_{t-1} (dΔ, / aback)
+      s3 = fma2(mul2(lam[j], av), bp, s3);                  // Σ λ Ā B        (dΔ, times x)
+      // dc/dA: direct form, or its series where |ΔA| < 0.01
+      const float2 y = mul2(mul2(d2, al[j]), f2(aback));
+      const float2 ser = mul2(mul2(d2, d2), fma2(fma2(y, f2(0.125f), f2(1.f / 3.f)), y, f2(0.5f)));
+      const float2 dir = mul2(fma2(d2, av, make_float2(-c.x, -c.y)), ra[j]);
+      const float2 dcda = make_float2(fabsf(y.x) < 1e-2f ? ser.x : dir.x, fabsf(y.y) < 1e-2f ? ser.y : dir.y);
+      dA[j] = fma2(d2, lq, fma2(mul2(lam[j], mul2(dcda, dx2_of(dd))), bp, dA[j]));
+      lam[j] = mul2(lam[j], av);                            // Ā_t λ_t, for step t-1
+      continue;
+    }
     if (PRECISE) {
       av = make_float2(expf(dd.x * al[j].x), expf(dd.x * al[j].y));
     } else if (j < KP) {
@@ -128,6 +177,7 @@ __device__ __forceinline__ void adjoint_step(float2 (&lam)[4], float2 (&dA)[4], 
   }
   S1 = s1.x + s1.y;
   S2 = s2.x + s2.y;
+  S3 = s3.x + s3.y;
 }
 
 // Sum the dB/dC values of two steps over the warp's 16 channels.  Row `lane` of `red` holds the
@@ -158,8 +208,10 @@ __device__ __forceinline__ void reduce_two_steps(BwdTile& tl, int lane, int k0, 
 // Replay a block from its entering state and run the adjoint over steps [lo, hi).
 template <bool PRECISE, int KP>
 __device__ __forceinline__ void half_pass(BwdTile& tl, const float2 (&hstart)[4], float2 (&lam)[4],
-                                          float2 (&dA)[4], const float2 (&al)[4], float aback,
+                                          float2 (&dA)[4], const float2 (&al)[4],
+                                          const float2 (&ra)[4], float aback,
                                           float live, int lane, int slot, int q, int lo, int hi) {
+  constexpr bool kZoh = KP == kKpZoh || KP == kKpZohClamped;
   const float4* bq = tl.sB + 2 * q;
   const float4* cq = tl.sC + 2 * q;
   float* prow = tl.park + lane * kParkS;
@@ -168,10 +220,10 @@ __device__ __forceinline__ void half_pass(BwdTile& tl, const float2 (&hstart)[4]
   for (int j = 0; j < 4; ++j) hh[j] = hstart[j];
 #pragma unroll 1
   for (int k = 0; k < lo; ++k)
-    replay_step<PRECISE, false, KP>(hh, al, tl.sd[k * kTS + slot], bq + k * 4, cq);
+    replay_step<PRECISE, false, KP>(hh, al, ra, tl.sd[k * kTS + slot], bq + k * 4, cq);
 #pragma unroll 1
   for (int k = lo; k < hi; ++k) {
-    float y = replay_step<PRECISE, true, KP>(hh, al, tl.sd[k * kTS + slot], bq + k * 4, cq + k * 4);
+    float y = replay_step<PRECISE, true, KP>(hh, al, ra, tl.sd[k * kTS + slot], bq + k * 4, cq + k * 4);
     y += __shfl_xor_sync(0xffffffffu, y, 1);
     if (q == 0) tl.ys[k * kTS + slot] = y;
     float4* pk = reinterpret_cast<float4*>(prow + (k - lo) * kHB);
@@ -191,12 +243,15 @@ __device__ __forceinline__ void half_pass(BwdTile& tl, const float2 (&hstart)[4]
         const float4 h0 = pk[0], h1 = pk[1];
         const float2 hk[4] = {make_float2(h0.x, h0.y), make_float2(h0.z, h0.w),
                               make_float2(h1.x, h1.y), make_float2(h1.z, h1.w)};
-        float S1, S2;
-        adjoint_step<PRECISE, KP>(lam, dA, al, hk, tl.sd[kk * kTS + slot], tl.sg[kk * kTS + slot],
-                                  live, bq + kk * 4, cq + kk * 4, vals, S1, S2);
+        float S1, S2, S3;
+        const float2 dd = tl.sd[kk * kTS + slot];
+        adjoint_step<PRECISE, KP>(lam, dA, al, ra, aback, hk, dd, tl.sg[kk * kTS + slot],
+                                  live, bq + kk * 4, cq + kk * 4, vals, S1, S2, S3);
+        // Euler: (Σ λ B, Σ A λ Ā h_{t-1}); ZOH: (Σ λ c B, x Σ λ Ā B + Σ A λ Ā h_{t-1})
+        float T = kZoh ? fmaf(dd.y, S3, S2 * aback) : S2 * aback;
         S1 += __shfl_xor_sync(0xffffffffu, S1, 1);
-        S2 += __shfl_xor_sync(0xffffffffu, S2, 1);
-        if (q == 0) tl.sS[kk * kTS + slot] = make_float2(S1, S2 * aback);
+        T += __shfl_xor_sync(0xffffffffu, T, 1);
+        if (q == 0) tl.sS[kk * kTS + slot] = make_float2(S1, T);
       } else {
 #pragma unroll
         for (int j = 0; j < 8; ++j) vals[j] = make_float2(0.f, 0.f);
@@ -229,13 +284,18 @@ __global__ void __launch_bounds__(128) bwd_kernel(const BwdArgs a) {
   const float ascale = kPrecise ? 1.f : kLog2e;
   const float aback = kPrecise ? 1.f : kLn2;  // al * aback == A
 
-  float2 al[4], lam[4], dA[4];
+  // ZOH: ra = 1/A, with |A| < 1e-20 taken as -1e-20 (the A -> 0 limit, c = Δ)
+  constexpr bool kZoh = KP == kKpZoh;
+  float2 al[4], ra[4], lam[4], dA[4];
   float amax = 0.f;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const int n0 = kHB * q + 2 * j, n1 = n0 + 1;
-    al[j] = make_float2(n0 < N ? a.A[(long long)dd * N + n0] * ascale : 0.f,
-                        n1 < N ? a.A[(long long)dd * N + n1] * ascale : 0.f);
+    float2 av = make_float2(n0 < N ? a.A[(long long)dd * N + n0] : 0.f,
+                            n1 < N ? a.A[(long long)dd * N + n1] : 0.f);
+    if (kZoh) av = make_float2(zoh_rate(av.x), zoh_rate(av.y));
+    al[j] = mul2(av, f2(ascale));
+    ra[j] = kZoh ? make_float2(1.f / av.x, 1.f / av.y) : f2(0.f);
     lam[j] = make_float2((a.dhL && n0 < N) ? a.dhL[ch * N + n0] : 0.f,
                          (a.dhL && n1 < N) ? a.dhL[ch * N + n1] : 0.f);
     dA[j] = make_float2(0.f, 0.f);
@@ -320,7 +380,9 @@ __global__ void __launch_bounds__(128) bwd_kernel(const BwdArgs a) {
           sp = sigmoid_fast_x2(v);
         }
       }
-      const float2 dx = mul2(dl, make_float2(ru.get(j), ru.get(j + 1)));
+      // (Δ, Δx), or (Δ, x) with the ZOH term (its coefficient is per state)
+      const float2 xv = make_float2(ru.get(j), ru.get(j + 1));
+      const float2 dx = kZoh ? xv : mul2(dl, xv);
       const float2 go = make_float2(rg.get(j), rg.get(j + 1));
       float2 g = go, zf = make_float2(0.f, 0.f);
       if (zp) {
@@ -345,10 +407,12 @@ __global__ void __launch_bounds__(128) bwd_kernel(const BwdArgs a) {
     for (int half = 1; half >= 0; --half) {
       const int lo = kHB * half, hi = min(nvalid, lo + kHB);
       if (lo >= hi) continue;
-      if (kPrecise || !safe)
-        half_pass<kPrecise, 4>(tl, hstart, lam, dA, al, aback, live, lane, slot, q, lo, hi);
+      // blocks that fail the range vote: MUFU exponentials, or the clamped ZOH form
+      constexpr int KS = kZoh ? kKpZohClamped : 4;
+      if (!safe || (kPrecise && !kZoh))
+        half_pass<kPrecise, KS>(tl, hstart, lam, dA, al, ra, aback, live, lane, slot, q, lo, hi);
       else
-        half_pass<kPrecise, KP>(tl, hstart, lam, dA, al, aback, live, lane, slot, q, lo, hi);
+        half_pass<kPrecise, KP>(tl, hstart, lam, dA, al, ra, aback, live, lane, slot, q, lo, hi);
     }
     __syncwarp();
 
@@ -362,8 +426,8 @@ __global__ void __launch_bounds__(128) bwd_kernel(const BwdArgs a) {
       const float g = tl.sg[k * kTS + slot];
       const float x = ru.get(j);
       odz[j] = (tl.ys[k * kTS + slot] + Dd * x) * dzf[j];
-      odu[j] = dlx.x * S.x + g * Dd;
-      odd[j] = (x * S.x + S.y) * sv[j];
+      odu[j] = (kZoh ? S.x : dlx.x * S.x) + g * Dd;
+      odd[j] = (kZoh ? S.y : x * S.x + S.y) * sv[j];
       if (j < nown) {
         dD_acc += g * x;
         dbias_acc += odd[j];
@@ -456,7 +520,9 @@ cudaError_t launch_bwd_io(const BwdArgs& a, cudaStream_t s) {
   const dim3 grid((unsigned)(a.batch * a.ngroups)), block(32 * a.wpb);
   const size_t smem = sizeof(BwdTile) * a.wpb;
   auto k = bwd_kernel<IO, VEC, 2>;
-  if constexpr (!std::is_same<IO, float>::value) {
+  if (a.zoh) {
+    k = bwd_kernel<IO, VEC, kKpZoh>;  // ZOH coefficient on the FMA pipe
+  } else if constexpr (!std::is_same<IO, float>::value) {
     if (a.kmufu == 3) k = bwd_kernel<IO, VEC, 3>;
     else if (a.kmufu == 4) k = bwd_kernel<IO, VEC, 4>;
   }

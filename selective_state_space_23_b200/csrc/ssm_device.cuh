@@ -86,6 +86,41 @@ __device__ __forceinline__ float2 exp2_fma_prod_x2(float2 d, float2 a) {
   return out;
 }
 
+// Zero-order-hold input coefficient, two lanes: Ā = e^{ΔA} and g = (e^{ΔA} - 1)/A, from
+// x = Δ a with a = A log2 e and ra = 1/A.  With x = i + f (i = rint(x), |f| <= 1/2) and
+// 2^f = 1 + f q(f) (the cubic above), e^{ΔA} - 1 = 2^i f q(f) + (2^i - 1): as ΔA -> 0 the
+// relative accuracy of f q(f) carries over, where Ā - 1 would cancel.  2^i is built in the
+// exponent field.  CLAMP limits x to [-126, 126] (Ā -> 0 and g -> -1/A below; above, the true
+// values overflow f32 anyway); otherwise the caller guarantees |x| <= 126.
+template <bool CLAMP>
+__device__ __forceinline__ void zoh_coef_x2(float2 d, float2 a, float2 ra, float2& abar, float2& g) {
+  float2 t, f;
+  if (CLAMP) {
+    float2 x = mul2(d, a);
+    x = make_float2(fminf(fmaxf(x.x, -126.f), 126.f), fminf(fmaxf(x.y, -126.f), 126.f));
+    t = add2(x, f2(kRoundMagic));                           // M + rint(x)
+    const float2 rn = add2(f2(kRoundMagic), make_float2(-t.x, -t.y));  // -rint(x), exact
+    f = add2(x, rn);
+  } else {
+    t = fma2(d, a, f2(kRoundMagic));
+    const float2 rn = add2(f2(kRoundMagic), make_float2(-t.x, -t.y));
+    f = fma2(d, a, rn);                                     // Δ a - rint(Δ a), exact
+  }
+  float2 q = fma2(f2(kQ3), f, f2(kQ2));
+  q = fma2(q, f, f2(kQ1));
+  q = fma2(q, f, f2(kQ0));
+  const float2 fq = mul2(f, q);                             // 2^f - 1
+  float2 s;                                                 // 2^i: i added to the exponent of 1
+  s.x = __int_as_float(0x3f800000 + (__float_as_int(t.x) << 23));
+  s.y = __int_as_float(0x3f800000 + (__float_as_int(t.y) << 23));
+  abar = fma2(fq, s, s);
+  g = mul2(fma2(fq, s, add2(s, f2(-1.f))), ra);
+}
+
+// A rate that the zero-order-hold coefficient divides by: |A| below 1e-20 is taken as -1e-20
+// (then Ā = 1 and g = Δ to f32 precision, the A -> 0 limit, with no division by zero).
+__device__ __forceinline__ float zoh_rate(float A) { return fabsf(A) < 1e-20f ? -1e-20f : A; }
+
 // ---------------------------------------------------------------- step size and gate
 // softplus(v) = log(1 + e^v) to ~5e-6 relative error, for the bf16 path.
 //   v > 15          : v (the remainder e^-v < 3.1e-7 of v)

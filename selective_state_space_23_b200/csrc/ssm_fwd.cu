@@ -92,10 +92,12 @@ __device__ __forceinline__ float4 quad(const float4* q, int i) { return q[i]; }
 
 // KP of the lane's PPL state pairs take 2^x from the MUFU unit, the others from the FMA-pipe
 // polynomial, which has no range checks: it is used only in blocks where every step satisfies
-// |Δ| max_n |A_n log2 e| <= 126 (checked once per block by a warp vote).  KP < 0: scalar decay,
-// Ā is already in the table.
+// |Δ| max_n |A_n log2 e| <= 126 (checked once per block by a warp vote).  Negative KP select the
+// variants: kKpScalar / kKpScalarZoh (scalar decay, Ā already in the table), kKpZoh /
+// kKpZohClamped (zero-order-hold input term per state; the clamped form for unchecked blocks).
 template <bool PRECISE, int PPL, int KP>
-__device__ __forceinline__ void prepare_step(StepPrep<PPL>& p, const float2 (&al)[PPL], float4 dd,
+__device__ __forceinline__ void prepare_step(StepPrep<PPL>& p, const float2 (&al)[PPL],
+                                             const float2 (&ra)[PPL], float4 dd,
                                              const float4* bq) {
   const float2 d2 = make_float2(dd.x, dd.y), du2 = make_float2(dd.z, dd.w);  // already paired
   float4 bv[PPL / 2];
@@ -105,8 +107,20 @@ __device__ __forceinline__ void prepare_step(StepPrep<PPL>& p, const float2 (&al
   for (int j = 0; j < PPL; ++j) {
     const float4 bb = bv[j >> 1];
     const float2 bp = (j & 1) ? make_float2(bb.z, bb.w) : make_float2(bb.x, bb.y);
-    if (KP < 0) {
-      p.av[j] = d2;  // scalar decay: the table holds (Ā, Ā, Δx, Δx)
+    if (KP == kKpScalar || KP == kKpScalarZoh) {
+      p.av[j] = d2;  // scalar decay: the table holds (Ā, Ā, b x, b x), b = Δ or the ZOH coefficient
+    } else if (KP == kKpZoh || KP == kKpZohClamped) {
+      // ZOH per state: the table holds (Δ, Δ, x, x); B̄ x = (e^{ΔA} - 1)/A B x
+      float2 g;
+      if (PRECISE) {
+        const float2 y = mul2(d2, al[j]);
+        p.av[j] = make_float2(expf(y.x), expf(y.y));
+        g = mul2(make_float2(expm1f(y.x), expm1f(y.y)), ra[j]);
+      } else {
+        zoh_coef_x2<KP == kKpZohClamped>(d2, al[j], ra[j], p.av[j], g);
+      }
+      p.bu[j] = mul2(mul2(g, du2), bp);
+      continue;
     } else if (PRECISE) {
       p.av[j] = make_float2(expf(dd.x * al[j].x), expf(dd.x * al[j].y));
     } else if (j < KP) {
@@ -146,7 +160,8 @@ __device__ __forceinline__ float consume_step(float2 (&hh)[PPL], const StepPrep<
 // (the index is clamped to the tile) but is never consumed.
 template <bool kPrecise, bool kReadout, int LPC, int KE, int KO>
 __device__ __forceinline__ void state_loop(BlockBuf<LPC>& tile, float2 (&hh)[Layout<LPC>::kPPL],
-                                           const float2 (&al)[Layout<LPC>::kPPL], int slot, int q,
+                                           const float2 (&al)[Layout<LPC>::kPPL],
+                                           const float2 (&ra)[Layout<LPC>::kPPL], int slot, int q,
                                            int nvalid) {
   using Lay = Layout<LPC>;
   constexpr int SPL = Lay::kSPL, PPL = Lay::kPPL;
@@ -155,14 +170,14 @@ __device__ __forceinline__ void state_loop(BlockBuf<LPC>& tile, float2 (&hh)[Lay
   const float4* sdp = tile.sd + slot;
   float* yp = tile.yp + slot * LPC + q;
   StepPrep<PPL> p0, p1;
-  prepare_step<kPrecise, PPL, KE>(p0, al, sdp[0], bq);
+  prepare_step<kPrecise, PPL, KE>(p0, al, ra, sdp[0], bq);
   int k = 0;
 #pragma unroll 1
   for (; k + 2 <= nvalid; k += 2) {
-    prepare_step<kPrecise, PPL, KO>(p1, al, sdp[(k + 1) * Lay::kSdStride], bq + (k + 1) * 4);
+    prepare_step<kPrecise, PPL, KO>(p1, al, ra, sdp[(k + 1) * Lay::kSdStride], bq + (k + 1) * 4);
     const float y0 = consume_step<kReadout, PPL>(hh, p0, cq + k * 4);
     const int k2 = min(k + 2, kBlk - 1);
-    prepare_step<kPrecise, PPL, KE>(p0, al, sdp[k2 * Lay::kSdStride], bq + k2 * 4);
+    prepare_step<kPrecise, PPL, KE>(p0, al, ra, sdp[k2 * Lay::kSdStride], bq + k2 * 4);
     const float y1 = consume_step<kReadout, PPL>(hh, p1, cq + (k + 1) * 4);
     if (kReadout) {
       yp[k * Lay::kYpStride] = y0;
@@ -186,8 +201,10 @@ struct BlockRows {
 };
 
 // What one lane needs to load, prepare and finish the blocks of its chunk.
-template <typename IO, bool VEC, int MODE, int LPC, bool SA>
+template <typename IO, bool VEC, int MODE, int LPC, int KV>
 struct ChunkLane {
+  static constexpr bool SA = KV == kKpScalar || KV == kKpScalarZoh;   // scalar decay
+  static constexpr bool ZOH = KV == kKpZoh || KV == kKpZohClamped || KV == kKpScalarZoh;
   using Lay = Layout<LPC>;
   static constexpr int SPL = Lay::kSPL;
   static constexpr bool kPrecise = std::is_same<IO, float>::value;
@@ -207,6 +224,7 @@ struct ChunkLane {
   float bias, Dd;
   float dlim;  // |Δ| < dlim keeps |Δ A log2 e| <= 126 for every state of the warp
   float a1;    // scalar decay: A_d (times log2 e on the bf16 path)
+  float ra1;   // scalar decay with the ZOH input term: 1 / A_d
 
 
   // Rows of the block starting at tb; steps at or beyond t_end read as zero.
@@ -252,11 +270,23 @@ struct ChunkLane {
       if (kPrecise) dl = make_float2(softplus_precise(v.x), softplus_precise(v.y));
       else dl = softplus_fast_x2(v);
     }
-    const float2 dx = mul2(dl, make_float2(r.u.get(j), r.u.get(j + 1)));
-    float2 tv = dl;  // table entry: Δ, or Ā = exp(Δ A_d) for a scalar decay
-    if (SA) {
+    const float2 xv = make_float2(r.u.get(j), r.u.get(j + 1));
+    // table entry (tv, tv, dx, dx): Euler (Δ, Δx); ZOH (Δ, x); scalar decay (Ā, Δx) or, with
+    // the ZOH input term, (Ā, g x) with g = (e^{Δ A_d} - 1)/A_d
+    float2 tv = dl, dx = ZOH && !SA ? xv : mul2(dl, xv);
+    if (SA && !ZOH) {
       if (kPrecise) tv = make_float2(expf(dl.x * a1), expf(dl.y * a1));
       else tv = make_float2(ex2_mufu(dl.x * a1), ex2_mufu(dl.y * a1));
+    } else if (SA) {
+      float2 g;
+      if (kPrecise) {
+        const float2 y = mul2(dl, f2(a1));
+        tv = make_float2(expf(y.x), expf(y.y));
+        g = mul2(make_float2(expm1f(y.x), expm1f(y.y)), f2(ra1));
+      } else {
+        zoh_coef_x2<true>(dl, f2(a1), f2(ra1), tv, g);
+      }
+      dx = mul2(g, xv);
     }
     sd[(SPL * q + j) * Lay::kSdStride + slot] = make_float4(tv.x, tv.x, dx.x, dx.x);
     sd[(SPL * q + j + 1) * Lay::kSdStride + slot] = make_float4(tv.y, tv.y, dx.y, dx.y);
@@ -310,7 +340,8 @@ __device__ __forceinline__ void interleaved_block(
     const Lane& ln, const BlockBuf<LPC>* __restrict__ cur, float* __restrict__ cur_yp,
     float* __restrict__ nxt_sB, float* __restrict__ nxt_sC, float4* __restrict__ nxt_sd,
     const float* __restrict__ nxt_yp, float2 (&hh)[Layout<LPC>::kPPL],
-    const float2 (&al)[Layout<LPC>::kPPL], const typename Lane::Rows& rn, int nown_next,
+    const float2 (&al)[Layout<LPC>::kPPL], const float2 (&ra)[Layout<LPC>::kPPL],
+    const typename Lane::Rows& rn, int nown_next,
     const typename Lane::URow& pu, const typename Lane::URow& pz, float (&o)[Layout<LPC>::kSPL],
     float& dblk, bool& ok) {
   using Lay = Layout<LPC>;
@@ -322,17 +353,17 @@ __device__ __forceinline__ void interleaved_block(
   float* yp = cur_yp + ln.slot * LPC + ln.q;
   // two steps prepared ahead: steps k+2, k+3 are prepared while k, k+1 update the state
   StepPrep<PPL> p0, p1;
-  prepare_step<kPrecise, PPL, KE>(p0, al, sdp[0], bq);
-  prepare_step<kPrecise, PPL, KO>(p1, al, sdp[Lay::kSdStride], bq + 4);
+  prepare_step<kPrecise, PPL, KE>(p0, al, ra, sdp[0], bq);
+  prepare_step<kPrecise, PPL, KO>(p1, al, ra, sdp[Lay::kSdStride], bq + 4);
 #pragma unroll
   for (int m = 0; m < 8; ++m) {
     const int k = 2 * m;
     StepPrep<PPL> q0, q1;
     if (m < 7)
-      prepare_step<kPrecise, PPL, KE>(q0, al, sdp[(k + 2) * Lay::kSdStride], bq + (k + 2) * 4);
+      prepare_step<kPrecise, PPL, KE>(q0, al, ra, sdp[(k + 2) * Lay::kSdStride], bq + (k + 2) * 4);
     const float y0 = consume_step<kReadout, PPL>(hh, p0, cq + k * 4);
     if (m < 7)
-      prepare_step<kPrecise, PPL, KO>(q1, al, sdp[(k + 3) * Lay::kSdStride], bq + (k + 3) * 4);
+      prepare_step<kPrecise, PPL, KO>(q1, al, ra, sdp[(k + 3) * Lay::kSdStride], bq + (k + 3) * 4);
     const float y1 = consume_step<kReadout, PPL>(hh, p1, cq + (k + 1) * 4);
     p0 = q0;
     p1 = q1;
@@ -354,12 +385,14 @@ __device__ __forceinline__ void interleaved_block(
 template <typename IO, bool VEC, int MODE, int LPC, int KE, int KO>
 __device__ __forceinline__ void run_chunk(const FwdArgs& a, WarpTile<LPC>& tile,
                                           float2 (&hh)[Layout<LPC>::kPPL],
-                                          const float2 (&al)[Layout<LPC>::kPPL], float Dd,
+                                          const float2 (&al)[Layout<LPC>::kPPL],
+                                          const float2 (&ra)[Layout<LPC>::kPPL], float Dd,
                                           float bias, int lane, int slot, int q, int b, bool act,
                                           long long ch, int t_begin, int t_end, bool last_chunk) {
   using Lay = Layout<LPC>;
-  using Lane = ChunkLane<IO, VEC, MODE, LPC, (KE < 0)>;
-  constexpr int KS = KE < 0 ? -1 : Layout<LPC>::kPPL;  // exponentials of an unchecked block
+  using Lane = ChunkLane<IO, VEC, MODE, LPC, (KE < 0 ? KE : 0)>;
+  // exponentials of a block that failed the range vote
+  constexpr int KS = KE == kKpZoh ? kKpZohClamped : (KE < 0 ? KE : Layout<LPC>::kPPL);
   constexpr int SPL = Lay::kSPL, PPL = Lay::kPPL;
   constexpr bool kPrecise = Lane::kPrecise;
   constexpr bool kReadout = Lane::kReadout;
@@ -388,6 +421,7 @@ __device__ __forceinline__ void run_chunk(const FwdArgs& a, WarpTile<LPC>& tile,
   ln.bias = bias;
   ln.Dd = Dd;
   ln.a1 = al[0].x;
+  ln.ra1 = ra[0].x;
   const int nblk_total = (L + kBlk - 1) / kBlk;
   const int nblk = (t_end - t_begin + kBlk - 1) / kBlk;
   const auto own = [&](int nvalid) { return max(0, min(SPL, nvalid - SPL * q)); };
@@ -463,11 +497,11 @@ __device__ __forceinline__ void run_chunk(const FwdArgs& a, WarpTile<LPC>& tile,
       float* nsC = reinterpret_cast<float*>(nxt.sC);
       if (kPrecise || !safe)
         interleaved_block<kPrecise, kReadout, LPC, KS, KS>(ln, &cur, cur.yp, nsB, nsC, nxt.sd,
-                                                             nxt.yp, hh, al, rn, nown_next, pu, pz,
+                                                             nxt.yp, hh, al, ra, rn, nown_next, pu, pz,
                                                              o, dblk, ok);
       else
         interleaved_block<kPrecise, kReadout, LPC, KE, KO>(ln, &cur, cur.yp, nsB, nsC, nxt.sd,
-                                                           nxt.yp, hh, al, rn, nown_next, pu, pz,
+                                                           nxt.yp, hh, al, ra, rn, nown_next, pu, pz,
                                                            o, dblk, ok);
     } else {
       // partial (last) block: the three stages one after another
@@ -476,9 +510,9 @@ __device__ __forceinline__ void run_chunk(const FwdArgs& a, WarpTile<LPC>& tile,
         for (int j = 0; j < SPL; j += 2) ln.output_pair(nxt.yp, pu, pz, j, o);
       }
       if (kPrecise || !safe)
-        state_loop<kPrecise, kReadout, LPC, KS, KS>(cur, hh, al, slot, q, nvalid);
+        state_loop<kPrecise, kReadout, LPC, KS, KS>(cur, hh, al, ra, slot, q, nvalid);
       else
-        state_loop<kPrecise, kReadout, LPC, KE, KO>(cur, hh, al, slot, q, nvalid);
+        state_loop<kPrecise, kReadout, LPC, KE, KO>(cur, hh, al, ra, slot, q, nvalid);
       // a partial block is the last one: there is no next block to prepare
     }
     __syncwarp();  // this block's partial readouts and the next block's table are complete
@@ -544,7 +578,9 @@ __global__ void __launch_bounds__(128) fwd_kernel(const FwdArgs a) {
 
   constexpr bool kPrecise = std::is_same<IO, float>::value;
   const float ascale = kPrecise ? 1.f : kLog2e;
-  const float* Ad = a.A + (long long)dd * (KE < 0 ? 1 : a.N);
+  constexpr bool kSA = KE == kKpScalar || KE == kKpScalarZoh;
+  constexpr bool kZOH = KE == kKpZoh || KE == kKpScalarZoh;
+  const float* Ad = a.A + (long long)dd * (kSA ? 1 : a.N);
   const float* hsrc = nullptr;
   bool hs16 = false;  // hin rows hold 16 states; h0 rows hold N
   if (MODE != kFwdSummary) {
@@ -555,14 +591,17 @@ __global__ void __launch_bounds__(128) fwd_kernel(const FwdArgs a) {
       hsrc = a.h0 + ch * a.N;
     }
   }
-  float2 al[PPL], hh[PPL];
+  // al = A log2 e (A on the fp32 path); ra = 1/A for the ZOH coefficient, with |A| < 1e-20
+  // taken as -1e-20 (the A -> 0 limit, g = Δ)
+  float2 al[PPL], ra[PPL], hh[PPL];
 #pragma unroll
   for (int j = 0; j < PPL; ++j) {
     const int n0 = SPL * q + 2 * j, n1 = n0 + 1;
-    if (KE < 0)
-      al[j] = f2(Ad[0] * ascale);  // one decay rate for every state
-    else
-      al[j] = make_float2(n0 < a.N ? Ad[n0] * ascale : 0.f, n1 < a.N ? Ad[n1] * ascale : 0.f);
+    float2 av = kSA ? f2(Ad[0])  // one decay rate for every state
+                    : make_float2(n0 < a.N ? Ad[n0] : 0.f, n1 < a.N ? Ad[n1] : 0.f);
+    if (kZOH) av = make_float2(zoh_rate(av.x), zoh_rate(av.y));
+    al[j] = mul2(av, f2(ascale));
+    ra[j] = kZOH ? make_float2(1.f / av.x, 1.f / av.y) : f2(0.f);
     hh[j] = make_float2((hsrc && (hs16 || n0 < a.N)) ? hsrc[n0] : 0.f,
                         (hsrc && (hs16 || n1 < a.N)) ? hsrc[n1] : 0.f);
   }
@@ -570,8 +609,8 @@ __global__ void __launch_bounds__(128) fwd_kernel(const FwdArgs a) {
   const float bias = a.dt_bias ? a.dt_bias[dd] : 0.f;
   WarpTile<LPC>& tile = tiles[wib];
 
-  run_chunk<IO, VEC, MODE, LPC, KE, KO>(a, tile, hh, al, Dd, bias, lane, slot, q, b, act, ch, t_begin,
-                                        t_end, last_chunk);
+  run_chunk<IO, VEC, MODE, LPC, KE, KO>(a, tile, hh, al, ra, Dd, bias, lane, slot, q, b, act, ch,
+                                        t_begin, t_end, last_chunk);
 }
 
 // Chain the chunk summaries: h_in(0) = h0, h_in(j+1) = exp(A ΣΔ_j) h_in(j) + h_end(j).
@@ -608,8 +647,12 @@ cudaError_t launch_mode(const FwdArgs& a, int wpb, int kmufu, cudaStream_t s) {
   const int nchunk_launch = MODE == kFwdSummary ? a.nchunk - 1 : a.nchunk;  // last chunk's summary is unused
   if (ctas <= 0 || nchunk_launch <= 0) return cudaSuccess;
   const dim3 grid((unsigned)ctas, (unsigned)nchunk_launch), block(32 * wpb);
-  if (a.scalar_a) {  // two lanes per channel, no exponential in the time loop
-    launch_one<IO, VEC, MODE, 2, -1, -1>(a, grid, block, s);
+  if (a.scalar_a && a.zoh) {  // two lanes per channel, no exponential in the time loop
+    launch_one<IO, VEC, MODE, 2, kKpScalarZoh, kKpScalarZoh>(a, grid, block, s);
+  } else if (a.scalar_a) {
+    launch_one<IO, VEC, MODE, 2, kKpScalar, kKpScalar>(a, grid, block, s);
+  } else if (a.zoh) {  // per-state ZOH coefficient on the FMA pipe
+    launch_one<IO, VEC, MODE, 2, kKpZoh, kKpZoh>(a, grid, block, s);
   } else if constexpr (std::is_same<IO, float>::value) {  // fp32: library expf
     if (a.lpc == 4) launch_one<IO, VEC, MODE, 4, 2, 2>(a, grid, block, s);
     else if (a.lpc == 1) launch_one<IO, VEC, MODE, 1, 8, 8>(a, grid, block, s);

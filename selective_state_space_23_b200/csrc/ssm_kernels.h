@@ -15,6 +15,13 @@ constexpr int kNS = 16;    // states per channel (dstate <= 16, padded with zero
 // writing the state entering every 16-step block (input of the backward pass).
 enum FwdMode { kFwdOut = 0, kFwdSummary = 1, kFwdCkpt = 2 };
 
+// Variant codes passed in place of a MUFU pair count (template KE = KO of the forward kernel,
+// KP of the backward kernel).
+constexpr int kKpScalar = -1;      // one decay rate per channel, first-order input term
+constexpr int kKpZoh = -2;         // zero-order-hold input term, range-checked block
+constexpr int kKpZohClamped = -3;  // zero-order-hold input term, exponent range clamped
+constexpr int kKpScalarZoh = -4;   // one decay rate per channel, zero-order-hold input term
+
 struct FwdArgs {
   const void* u;
   const void* delta;
@@ -37,6 +44,7 @@ struct FwdArgs {
   int softplus;
   int scalar_a;         // one decay rate A_d per channel, shared by its N states
   int reverse;          // scan runs from t = L-1 down to 0 (time rows read/written mirrored)
+  int zoh;              // zero-order-hold input term (e^{ΔA} - 1)/A B x instead of Δ B x
   int lpc;              // lanes per channel: 1, 2 or 4 (16 / lpc states each)
   int warps_per_b;      // ceil(dim / (32 / lpc))
   long long nwarps;     // batch * warps_per_b
@@ -68,6 +76,7 @@ struct BwdArgs {
   int ngroups;          // CTAs per batch row = ceil(warps_per_b / wpb)
   int kmufu;            // state pairs (of 4 per lane) whose exponential runs on MUFU: 2, 3 or 4
   int reverse;          // gradients of the reverse scan (time rows read/written mirrored)
+  int zoh;              // gradients of the zero-order-hold input term
 };
 
 struct DecodeArgs {

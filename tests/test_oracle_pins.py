@@ -220,23 +220,29 @@ def test_channel_subset_matches_full():
 
 
 # ------------------------------------------------------------------ gradients
-def loss_and_grads(c, dout, dhL, softplus=True):
-    res = run(c, delta_softplus=softplus)
+def loss_and_grads(c, dout, dhL, softplus=True, zoh=False):
+    res = run(c, delta_softplus=softplus, zoh=zoh)
     loss = np.sum(res["out"] * dout) + np.sum(res["hL"] * dhL)
     return loss
 
 
-@pytest.mark.parametrize("gate,softplus", [(True, True), (False, True), (True, False)])
-def test_gradients_by_finite_differences(gate, softplus):
+@pytest.mark.parametrize("gate,softplus,zoh", [(True, True, False), (False, True, False),
+                                               (True, False, False), (True, True, True),
+                                               (False, False, True)])
+def test_gradients_by_finite_differences(gate, softplus, zoh):
     c = rand_case(batch=2, dim=2, L=5, N=3, gate=gate, seed=31)
     if not softplus:
         c["delta"] = np.abs(c["delta"]) + 0.1
         c["dt_bias"] = np.full(2, 0.05)
+    if zoh:
+        c["A"][0, 1] = 0.0        # the A -> 0 limit of the ZOH coefficient
+        c["A"][1, 2] = -3e-4      # |ΔA| small: the series branch of dc/dA
     r = np.random.default_rng(5)
     dout = r.standard_normal(c["u"].shape)
     dhL = r.standard_normal(c["h0"].shape)
     g = oracle.scan_bwd(c["u"], c["delta"], c["A"], c["B"], c["C"], dout, D=c["D"], z=c["z"],
-                        dt_bias=c["dt_bias"], delta_softplus=softplus, h0=c["h0"], dhL=dhL)
+                        dt_bias=c["dt_bias"], delta_softplus=softplus, h0=c["h0"], dhL=dhL,
+                        zoh=zoh)
     names = {"u": "du", "delta": "ddelta", "A": "dA", "B": "dB", "C": "dC", "D": "dD",
              "dt_bias": "ddt_bias", "h0": "dh0"}
     if gate:
@@ -250,8 +256,8 @@ def test_gradients_by_finite_differences(gate, softplus):
             i = it.multi_index
             xp = x.copy(); xp[i] += eps
             xm = x.copy(); xm[i] -= eps
-            num[i] = (loss_and_grads(dict(c, **{key: xp}), dout, dhL, softplus)
-                      - loss_and_grads(dict(c, **{key: xm}), dout, dhL, softplus)) / (2 * eps)
+            num[i] = (loss_and_grads(dict(c, **{key: xp}), dout, dhL, softplus, zoh)
+                      - loss_and_grads(dict(c, **{key: xm}), dout, dhL, softplus, zoh)) / (2 * eps)
         np.testing.assert_allclose(g[gname], num, rtol=2e-6, atol=2e-7, err_msg=gname)
 
 
