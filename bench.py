@@ -75,7 +75,7 @@ def load_peaks():
 
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for f in ("ssm_fwd.cu", "ssm_device.cuh", "ssm_kernels.h", "ssm_rows.cuh"):
+    for f in ("ssm_fwd_impl.cuh", "ssm_fwd_bf16.cu", "ssm_device.cuh", "ssm_kernels.h", "ssm_rows.cuh"):
         with open(os.path.join(ROOT, "selective_state_space_23_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]

@@ -1,617 +1,18 @@
-// Forward selective scan (S6), sm_100a.
-//
-// What is computed (per channel c = (b, d), time t, state n < N):
-//   Δ_t   = softplus(delta_t + dt_bias_d)          (or delta_t + dt_bias_d without softplus)
-//   Ā     = exp(Δ_t A_dn)                          ZOH discretisation of the diagonal A
-//   h_t,n = Ā h_{t-1},n + Δ_t B_t,n x_t            input term Δ B x
-//   y_t   = Σ_n C_t,n h_t,n + D_d x_t ;  out_t = y_t * silu(z_t)
-// "Mamba: Linear-Time Sequence Modeling with Selective State Spaces" (summary page), sections
-// "Yöntem" (discretisation and recurrence) and "Seçim Mekanizması (S6)" (input-dependent B, C,
-// Δ); the state is updated before it is read out, as in the sequential loop quoted on the
-// mamba-minimal news page.
-//
-// B200 mapping ("Donanım Duyarlı Durum Genişletme": the expanded (B, L, D, N) state never
-// leaves the chip):
-//   * two lanes own one channel, 8 states each in registers; a warp holds 16 consecutive d of
-//     the same batch row b, so B_t and C_t are warp-uniform;
-//   * time advances in blocks of 16 steps.  Each lane streams its half of the block (8 steps of
-//     u, delta, z: one 128-bit load each for bf16) for the NEXT block before computing the
-//     current one; the warp stages the block's B/C (16 x 16 each) in shared memory as f32 and
-//     each half-lane reads its 8 states back as broadcast 128-bit loads;
-//   * per-step scalars (Δ_t, Δ_t x_t) are computed once per channel and step, by the lane that
-//     loaded that step, and exchanged through shared memory, as are the two half readouts;
-//     the time loop itself is a short two-step body (small code, so the instruction cache holds
-//     it while several warps per scheduler hide each other's latencies);
-//   * the per-element work (Δ*A, 2^x, Δ*x*B, state FMA, C readout) runs as packed f32x2
-//     instructions; the exponentials are split between the MUFU unit and a range-reduced
-//     polynomial on the FMA pipe (KE / KO of a lane's 4 state pairs on MUFU at even / odd steps)
-//     so neither unit idles;
-//   * scalar decay (one A_d per channel shared by its N states, the Mamba-2 restriction noted on
-//     the "2024 Reading List: Neural Network" page, section on state-space models): Ā_t =
-//     exp(Δ_t A_d) is computed once per (channel, step) with Δ_t and Δ_t x_t, so the time loop
-//     runs no exponential at all (template KE = KO = -1);
-//   * reverse scan (the anti-causal direction of a bidirectional layer, "2024 Reading List:
-//     Neural Network", Hydra notes): the same recurrence in mirrored time; every time row is
-//     read and written mirrored (step t of the scan is row index L-1-t), nothing else changes;
-//   * few channels (long sequences): the time axis is split into S chunks.  A summary pass
-//     runs every chunk but the last from a zero state and records its end state and ΣΔ; a
-//     carry pass chains the chunk states h_in(j+1) = exp(A ΣΔ_j) h_in(j) + h_end(j) (the
-//     associative combine of the linear recurrence, "paralel ilişkisel tarama"); the output
-//     pass then reruns each chunk from its true entering state.
-#include <type_traits>
-
+// Forward selective scan (S6), sm_100a: dispatch over io type and direction, and the carry pass
+// of the time split.  The kernels and their design notes are in ssm_fwd_impl.cuh.
 #include "ssm_device.cuh"
 #include "ssm_kernels.h"
-#include "ssm_rows.cuh"
 
 namespace ssm {
+
+cudaError_t launch_fwd_bf16(const FwdArgs& a, bool vec, int mode, int wpb, int kmufu, cudaStream_t s);
+cudaError_t launch_fwd_f32(const FwdArgs& a, bool vec, int mode, int wpb, int kmufu, cudaStream_t s);
+cudaError_t launch_fwd_rev_bf16(const FwdArgs& a, bool vec, int mode, int wpb, int kmufu,
+                                cudaStream_t s);
+cudaError_t launch_fwd_rev_f32(const FwdArgs& a, bool vec, int mode, int wpb, int kmufu,
+                               cudaStream_t s);
+
 namespace {
-
-// Lane layout: LPC lanes (1, 2 or 4) share one channel; lane q of a channel holds states [SPL q, SPL q + SPL)
-// and owns steps [SPL q, SPL q + SPL) of every 16-step block (it loads their u, delta, z,
-// computes their Δ and writes their output).
-template <int LPC>
-struct Layout {
-  static constexpr int kSPL = kNS / LPC;       // states (and owned steps) per lane
-  static constexpr int kPPL = kSPL / 2;        // state pairs per lane
-  static constexpr int kChW = 32 / LPC;        // channels per warp
-  static constexpr int kSdStride = kChW + 1;   // entries per step in the (Δ, Δ, Δx, Δx) table
-  // floats per step in the partial-readout table: a multiple of LPC (aligned vector reads of a
-  // channel's LPC partials) chosen so that the owners' reads of different steps spread over banks
-  static constexpr int kYpStride = LPC == 1 ? 33 : (LPC == 2 ? 34 : 36);
-};
-
-// Shared memory of one 16-step block of a warp.
-template <int LPC>
-struct BlockBuf {
-  float4 sB[kBlk * kNS / 4];                          // B_t,n as f32 [step][state]
-  float4 sC[kBlk * kNS / 4];                          // C_t,n
-  float4 sd[kBlk * Layout<LPC>::kSdStride];           // (Δ_t, Δ_t, Δ_t x_t, Δ_t x_t) per [step][slot]
-  float yp[kBlk * Layout<LPC>::kYpStride];            // partial readouts per [step][slot][lane]
-};
-
-// Per-warp shared memory: two block buffers.  While block i runs its time loop out of buffer
-// i mod 2, the lanes fill the other buffer with block i+1's per-step scalars and B/C and read
-// block i-1's partial readouts from it.
-template <int LPC>
-struct WarpTile {
-  BlockBuf<LPC> buf[2];
-};
-
-// Per-step quantities of one lane that do not depend on the state: Ā = 2^(Δ A log2 e) and the
-// input term Δ x B.  They are computed one step ahead of the state update (the only
-// loop-carried dependency), which keeps MUFU and shared-memory latency off the critical path.
-template <int PPL>
-struct StepPrep {
-  float2 av[PPL];
-  float2 bu[PPL];
-};
-
-template <int PPL>
-__device__ __forceinline__ float4 quad(const float4* q, int i) { return q[i]; }
-
-// KP of the lane's PPL state pairs take 2^x from the MUFU unit, the others from the FMA-pipe
-// polynomial, which has no range checks: it is used only in blocks where every step satisfies
-// |Δ| max_n |A_n log2 e| <= 126 (checked once per block by a warp vote).  Negative KP select the
-// variants: kKpScalar / kKpScalarZoh (scalar decay, Ā already in the table), kKpZoh /
-// kKpZohClamped (zero-order-hold input term per state; the clamped form for unchecked blocks).
-template <bool PRECISE, int PPL, int KP>
-__device__ __forceinline__ void prepare_step(StepPrep<PPL>& p, const float2 (&al)[PPL],
-                                             const float2 (&ra)[PPL], float4 dd,
-                                             const float4* bq) {
-  const float2 d2 = make_float2(dd.x, dd.y), du2 = make_float2(dd.z, dd.w);  // already paired
-  float4 bv[PPL / 2];
-#pragma unroll
-  for (int i = 0; i < PPL / 2; ++i) bv[i] = bq[i];
-#pragma unroll
-  for (int j = 0; j < PPL; ++j) {
-    const float4 bb = bv[j >> 1];
-    const float2 bp = (j & 1) ? make_float2(bb.z, bb.w) : make_float2(bb.x, bb.y);
-    if (KP == kKpScalar || KP == kKpScalarZoh) {
-      p.av[j] = d2;  // scalar decay: the table holds (Ā, Ā, b x, b x), b = Δ or the ZOH coefficient
-    } else if (KP == kKpZoh || KP == kKpZohClamped) {
-      // ZOH per state: the table holds (Δ, Δ, x, x); B̄ x = (e^{ΔA} - 1)/A B x
-      float2 g;
-      if (PRECISE) {
-        const float2 y = mul2(d2, al[j]);
-        p.av[j] = make_float2(expf(y.x), expf(y.y));
-        g = mul2(make_float2(expm1f(y.x), expm1f(y.y)), ra[j]);
-      } else {
-        zoh_coef_x2<KP == kKpZohClamped>(d2, al[j], ra[j], p.av[j], g);
-      }
-      p.bu[j] = mul2(mul2(g, du2), bp);
-      continue;
-    } else if (PRECISE) {
-      p.av[j] = make_float2(expf(dd.x * al[j].x), expf(dd.x * al[j].y));
-    } else if (j < KP) {
-      const float2 x = mul2(d2, al[j]);
-      p.av[j] = make_float2(ex2_mufu(x.x), ex2_mufu(x.y));
-    } else {
-      p.av[j] = exp2_fma_prod_x2(d2, al[j]);  // block checked: |Δ A log2 e| <= 126
-    }
-    p.bu[j] = mul2(du2, bp);
-  }
-}
-
-// h <- Ā h + Δ x B for the lane's states; returns the partial readout Σ C h.
-template <bool READOUT, int PPL>
-__device__ __forceinline__ float consume_step(float2 (&hh)[PPL], const StepPrep<PPL>& p,
-                                              const float4* cq) {
-  float4 cv[PPL / 2];
-#pragma unroll
-  for (int i = 0; i < PPL / 2; ++i) cv[i] = READOUT ? cq[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-  float2 ya = make_float2(0.f, 0.f), yb = ya;
-#pragma unroll
-  for (int j = 0; j < PPL; ++j) {
-    hh[j] = fma2(p.av[j], hh[j], p.bu[j]);
-    if (READOUT) {
-      const float4 cc = cv[j >> 1];
-      const float2 cp = (j & 1) ? make_float2(cc.z, cc.w) : make_float2(cc.x, cc.y);
-      if (j & 1) yb = fma2(cp, hh[j], yb);
-      else ya = fma2(cp, hh[j], ya);
-    }
-  }
-  const float2 ys = add2(ya, yb);
-  return ys.x + ys.y;
-}
-
-// The 16-step time loop of one block, software-pipelined by one step: step k+1 is prepared while
-// step k updates the state.  A step at or beyond nvalid may be prepared from stale tile entries
-// (the index is clamped to the tile) but is never consumed.
-template <bool kPrecise, bool kReadout, int LPC, int KE, int KO>
-__device__ __forceinline__ void state_loop(BlockBuf<LPC>& tile, float2 (&hh)[Layout<LPC>::kPPL],
-                                           const float2 (&al)[Layout<LPC>::kPPL],
-                                           const float2 (&ra)[Layout<LPC>::kPPL], int slot, int q,
-                                           int nvalid) {
-  using Lay = Layout<LPC>;
-  constexpr int SPL = Lay::kSPL, PPL = Lay::kPPL;
-  const float4* bq = tile.sB + SPL * q / 4;
-  const float4* cq = tile.sC + SPL * q / 4;
-  const float4* sdp = tile.sd + slot;
-  float* yp = tile.yp + slot * LPC + q;
-  StepPrep<PPL> p0, p1;
-  prepare_step<kPrecise, PPL, KE>(p0, al, ra, sdp[0], bq);
-  int k = 0;
-#pragma unroll 1
-  for (; k + 2 <= nvalid; k += 2) {
-    prepare_step<kPrecise, PPL, KO>(p1, al, ra, sdp[(k + 1) * Lay::kSdStride], bq + (k + 1) * 4);
-    const float y0 = consume_step<kReadout, PPL>(hh, p0, cq + k * 4);
-    const int k2 = min(k + 2, kBlk - 1);
-    prepare_step<kPrecise, PPL, KE>(p0, al, ra, sdp[k2 * Lay::kSdStride], bq + k2 * 4);
-    const float y1 = consume_step<kReadout, PPL>(hh, p1, cq + (k + 1) * 4);
-    if (kReadout) {
-      yp[k * Lay::kYpStride] = y0;
-      yp[(k + 1) * Lay::kYpStride] = y1;
-    }
-  }
-  if (k < nvalid) {  // odd number of valid steps: the last one was prepared into p0
-    const float y0 = consume_step<kReadout, PPL>(hh, p0, cq + k * 4);
-    if (kReadout) yp[k * Lay::kYpStride] = y0;
-  }
-}
-
-// u, delta, z of a lane's owned steps of one block, and the B/C rows it stages.
-template <typename IO, int SPL>
-struct BlockRows {
-  Row<IO, SPL> u, d, z;
-  Row<IO, 8> b, c;
-  __device__ __forceinline__ void zero() {
-    u.zero(); d.zero(); z.zero(); b.zero(); c.zero();
-  }
-};
-
-// What one lane needs to load, prepare and finish the blocks of its chunk.
-template <typename IO, bool VEC, int MODE, int LPC, int KV>
-struct ChunkLane {
-  static constexpr bool SA = KV == kKpScalar || KV == kKpScalarZoh;   // scalar decay
-  static constexpr bool ZOH = KV == kKpZoh || KV == kKpZohClamped || KV == kKpScalarZoh;
-  using Lay = Layout<LPC>;
-  static constexpr int SPL = Lay::kSPL;
-  static constexpr bool kPrecise = std::is_same<IO, float>::value;
-  static constexpr bool kReadout = MODE == kFwdOut;
-  using Rows = BlockRows<IO, SPL>;
-  using URow = Row<IO, SPL>;
-
-  // time rows at step 0 (scan order; a reverse scan reads and writes them mirrored)
-  const IO* up;
-  const IO* dp;
-  const IO* zp;   // null: no gate
-  const IO* Bp;
-  const IO* Cp;
-  IO* op;
-  int slot, q, bn, bh, t_end, L;
-  bool bc_live, softplus, act, rev;
-  float bias, Dd;
-  float dlim;  // |Δ| < dlim keeps |Δ A log2 e| <= 126 for every state of the warp
-  float a1;    // scalar decay: A_d (times log2 e on the bf16 path)
-  float ra1;   // scalar decay with the ZOH input term: 1 / A_d
-
-
-  // Rows of the block starting at tb; steps at or beyond t_end read as zero.
-  __device__ __forceinline__ void fetch(Rows& r, int tb) const {
-    const int tq = tb + SPL * q, t8 = tb + 8 * bh;
-    const int nv = max(0, min(SPL, t_end - tq));
-    const int nv8 = max(0, min(8, t_end - t8));
-    if (VEC && nv == SPL) {
-      load_steps<IO, SPL, true>(r.u, up, L, tq, SPL, rev);
-      load_steps<IO, SPL, true>(r.d, dp, L, tq, SPL, rev);
-      if (zp) load_steps<IO, SPL, true>(r.z, zp, L, tq, SPL, rev);
-    } else {
-      load_steps<IO, SPL, false>(r.u, up, L, tq, nv, rev);
-      load_steps<IO, SPL, false>(r.d, dp, L, tq, nv, rev);
-      if (zp) load_steps<IO, SPL, false>(r.z, zp, L, tq, nv, rev);
-    }
-    if (!bc_live) {
-      r.b.zero();
-      r.c.zero();
-    } else if (VEC && nv8 == 8) {
-      load_steps<IO, 8, true>(r.b, Bp, L, t8, 8, rev);
-      if (kReadout) load_steps<IO, 8, true>(r.c, Cp, L, t8, 8, rev);
-    } else {
-      load_steps<IO, 8, false>(r.b, Bp, L, t8, nv8, rev);
-      if (kReadout) load_steps<IO, 8, false>(r.c, Cp, L, t8, nv8, rev);
-    }
-  }
-
-  // Stage B_t,bn and C_t,bn of step 8 bh + j of the block as f32 [step][state].
-  __device__ __forceinline__ void stage_row(float* __restrict__ sB, float* __restrict__ sC,
-                                            const Rows& r, int j) const {
-    sB[(8 * bh + j) * kNS + bn] = r.b.get(j);
-    if (kReadout) sC[(8 * bh + j) * kNS + bn] = r.c.get(j);
-  }
-
-  // Δ and Δx of owned steps j, j+1 into the block's table.  ok stays true while every |Δ| is
-  // below dlim (false for a NaN); the summary pass also sums Δ over the valid owned steps (nown).
-  __device__ __forceinline__ void scalar_pair(float4* __restrict__ sd, const Rows& r, int j, int nown,
-                                              float& dblk, bool& ok) const {
-    const float2 v = add2(make_float2(r.d.get(j), r.d.get(j + 1)), f2(bias));
-    float2 dl = v;
-    if (softplus) {
-      if (kPrecise) dl = make_float2(softplus_precise(v.x), softplus_precise(v.y));
-      else dl = softplus_fast_x2(v);
-    }
-    const float2 xv = make_float2(r.u.get(j), r.u.get(j + 1));
-    // table entry (tv, tv, dx, dx): Euler (Δ, Δx); ZOH (Δ, x); scalar decay (Ā, Δx) or, with
-    // the ZOH input term, (Ā, g x) with g = (e^{Δ A_d} - 1)/A_d
-    float2 tv = dl, dx = ZOH && !SA ? xv : mul2(dl, xv);
-    if (SA && !ZOH) {
-      if (kPrecise) tv = make_float2(expf(dl.x * a1), expf(dl.y * a1));
-      else tv = make_float2(ex2_mufu(dl.x * a1), ex2_mufu(dl.y * a1));
-    } else if (SA) {
-      float2 g;
-      if (kPrecise) {
-        const float2 y = mul2(dl, f2(a1));
-        tv = make_float2(expf(y.x), expf(y.y));
-        g = mul2(make_float2(expm1f(y.x), expm1f(y.y)), f2(ra1));
-      } else {
-        zoh_coef_x2<true>(dl, f2(a1), f2(ra1), tv, g);
-      }
-      dx = mul2(g, xv);
-    }
-    sd[(SPL * q + j) * Lay::kSdStride + slot] = make_float4(tv.x, tv.x, dx.x, dx.x);
-    sd[(SPL * q + j + 1) * Lay::kSdStride + slot] = make_float4(tv.y, tv.y, dx.y, dx.y);
-    if (MODE == kFwdSummary) dblk += (j < nown ? dl.x : 0.f) + (j + 1 < nown ? dl.y : 0.f);
-    ok = ok && fabsf(dl.x) < dlim && fabsf(dl.y) < dlim;
-  }
-
-  // out of owned steps j, j+1: (Σ of the LPC partial readouts + D x) * silu(z).
-  __device__ __forceinline__ void output_pair(const float* __restrict__ ypb, const URow& u,
-                                              const URow& z, int j, float (&o)[SPL]) const {
-    float yv[2];
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const float* pp = ypb + (SPL * q + j + i) * Lay::kYpStride + slot * LPC;
-      if (LPC == 1) {
-        yv[i] = *pp;
-      } else if (LPC == 2) {
-        const float2 v = *reinterpret_cast<const float2*>(pp);
-        yv[i] = v.x + v.y;
-      } else {
-        const float4 v = *reinterpret_cast<const float4*>(pp);
-        yv[i] = (v.x + v.y) + (v.z + v.w);
-      }
-    }
-    float2 y = fma2(f2(Dd), make_float2(u.get(j), u.get(j + 1)), make_float2(yv[0], yv[1]));
-    if (zp) {
-      const float2 z2 = make_float2(z.get(j), z.get(j + 1));
-      const float2 sg = kPrecise ? make_float2(sigmoid_precise(z2.x), sigmoid_precise(z2.y))
-                                 : sigmoid_fast_x2(z2);
-      y = mul2(y, mul2(z2, sg));
-    }
-    o[j] = y.x;
-    o[j + 1] = y.y;
-  }
-
-  __device__ __forceinline__ void store_out(int t0, const float (&o)[SPL], int nown) const {
-    if (!act || nown <= 0) return;
-    if (VEC && nown == SPL) store_steps<IO, SPL, true>(op, o, L, t0 + SPL * q, SPL, rev);
-    else store_steps<IO, SPL, false>(op, o, L, t0 + SPL * q, nown, rev);
-  }
-};
-
-// One full block (16 valid steps) with its neighbours' per-step work woven into the time loop:
-// block i+1's Δ, Δx and B/C go into `nxt`, and block i-1's outputs are finished from the partial
-// readouts in `nxt`.  A lane's SPL/2 scalar pairs and SPL/2 output pairs are spread evenly over
-// the 8 two-step iterations, so their MUFU work (softplus, sigmoid) lands between the state
-// steps' exponentials instead of forming a phase of its own.  Work for a block that does not
-// exist (no next / no previous block) runs on zeros or stale entries and is never stored.
-template <bool kPrecise, bool kReadout, int LPC, int KE, int KO, class Lane>
-__device__ __forceinline__ void interleaved_block(
-    const Lane& ln, const BlockBuf<LPC>* __restrict__ cur, float* __restrict__ cur_yp,
-    float* __restrict__ nxt_sB, float* __restrict__ nxt_sC, float4* __restrict__ nxt_sd,
-    const float* __restrict__ nxt_yp, float2 (&hh)[Layout<LPC>::kPPL],
-    const float2 (&al)[Layout<LPC>::kPPL], const float2 (&ra)[Layout<LPC>::kPPL],
-    const typename Lane::Rows& rn, int nown_next,
-    const typename Lane::URow& pu, const typename Lane::URow& pz, float (&o)[Layout<LPC>::kSPL],
-    float& dblk, bool& ok) {
-  using Lay = Layout<LPC>;
-  constexpr int SPL = Lay::kSPL, PPL = Lay::kPPL;
-  constexpr int S8 = 8 / PPL;  // iterations per scalar (and per output) pair
-  const float4* bq = cur->sB + SPL * ln.q / 4;
-  const float4* cq = cur->sC + SPL * ln.q / 4;
-  const float4* sdp = cur->sd + ln.slot;
-  float* yp = cur_yp + ln.slot * LPC + ln.q;
-  // two steps prepared ahead: steps k+2, k+3 are prepared while k, k+1 update the state
-  StepPrep<PPL> p0, p1;
-  prepare_step<kPrecise, PPL, KE>(p0, al, ra, sdp[0], bq);
-  prepare_step<kPrecise, PPL, KO>(p1, al, ra, sdp[Lay::kSdStride], bq + 4);
-#pragma unroll
-  for (int m = 0; m < 8; ++m) {
-    const int k = 2 * m;
-    StepPrep<PPL> q0, q1;
-    if (m < 7)
-      prepare_step<kPrecise, PPL, KE>(q0, al, ra, sdp[(k + 2) * Lay::kSdStride], bq + (k + 2) * 4);
-    const float y0 = consume_step<kReadout, PPL>(hh, p0, cq + k * 4);
-    if (m < 7)
-      prepare_step<kPrecise, PPL, KO>(q1, al, ra, sdp[(k + 3) * Lay::kSdStride], bq + (k + 3) * 4);
-    const float y1 = consume_step<kReadout, PPL>(hh, p1, cq + (k + 1) * 4);
-    p0 = q0;
-    p1 = q1;
-    if (kReadout) {
-      yp[k * Lay::kYpStride] = y0;
-      yp[(k + 1) * Lay::kYpStride] = y1;
-    }
-    ln.stage_row(nxt_sB, nxt_sC, rn, m);
-    if (m % S8 == S8 / 2) ln.scalar_pair(nxt_sd, rn, 2 * (m / S8), nown_next, dblk, ok);
-    if (kReadout && m % S8 == 0) ln.output_pair(nxt_yp, pu, pz, 2 * (m / S8), o);
-  }
-}
-
-// Scan of one time chunk by one lane.  Blocks are processed as a three-stage pipeline: while
-// block i updates the state, block i+1's per-step scalars and B/C are prepared and block i-1's
-// outputs are finished; block i+2's rows are in flight from HBM.  A partial last block runs the
-// same stages one after another.  KE / KO: MUFU pairs on even / odd steps (the same for every
-// lane, so the lanes of a channel run identical instructions).
-template <typename IO, bool VEC, int MODE, int LPC, int KE, int KO>
-__device__ __forceinline__ void run_chunk(const FwdArgs& a, WarpTile<LPC>& tile,
-                                          float2 (&hh)[Layout<LPC>::kPPL],
-                                          const float2 (&al)[Layout<LPC>::kPPL],
-                                          const float2 (&ra)[Layout<LPC>::kPPL], float Dd,
-                                          float bias, int lane, int slot, int q, int b, bool act,
-                                          long long ch, int t_begin, int t_end, bool last_chunk) {
-  using Lay = Layout<LPC>;
-  using Lane = ChunkLane<IO, VEC, MODE, LPC, (KE < 0 ? KE : 0)>;
-  // exponentials of a block that failed the range vote
-  constexpr int KS = KE == kKpZoh ? kKpZohClamped : (KE < 0 ? KE : Layout<LPC>::kPPL);
-  constexpr int SPL = Lay::kSPL, PPL = Lay::kPPL;
-  constexpr bool kPrecise = Lane::kPrecise;
-  constexpr bool kReadout = Lane::kReadout;
-  const int L = a.L, N = a.N;
-
-  Lane ln;
-  const long long row = ch * (long long)L;  // the lane owns steps [SPL q, SPL q + SPL) of each block
-  ln.up = reinterpret_cast<const IO*>(a.u) + row;
-  ln.dp = reinterpret_cast<const IO*>(a.delta) + row;
-  ln.zp = (kReadout && a.z) ? reinterpret_cast<const IO*>(a.z) + row : nullptr;
-  ln.op = kReadout ? reinterpret_cast<IO*>(a.out) + row : nullptr;
-  // B/C staging: lane stages state row bn, steps [8 bh, 8 bh + 8) of each block
-  ln.bn = lane >> 1;
-  ln.bh = lane & 1;
-  ln.bc_live = ln.bn < N;
-  const long long bcrow = ((long long)b * N + (ln.bc_live ? ln.bn : 0)) * L;
-  ln.Bp = reinterpret_cast<const IO*>(a.B) + bcrow;
-  ln.Cp = reinterpret_cast<const IO*>(a.C) + bcrow;
-  ln.slot = slot;
-  ln.q = q;
-  ln.t_end = t_end;
-  ln.L = L;
-  ln.rev = a.reverse != 0;
-  ln.softplus = a.softplus != 0;
-  ln.act = act;
-  ln.bias = bias;
-  ln.Dd = Dd;
-  ln.a1 = al[0].x;
-  ln.ra1 = ra[0].x;
-  const int nblk_total = (L + kBlk - 1) / kBlk;
-  const int nblk = (t_end - t_begin + kBlk - 1) / kBlk;
-  const auto own = [&](int nvalid) { return max(0, min(SPL, nvalid - SPL * q)); };
-
-  // largest |A log2 e| of the warp's states: the FMA-pipe exponential needs |Δ A log2 e| <= 126
-  float amax = 0.f;
-#pragma unroll
-  for (int j = 0; j < PPL; ++j) amax = fmaxf(amax, fmaxf(fabsf(al[j].x), fabsf(al[j].y)));
-#pragma unroll
-  for (int m = 16; m >= 1; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
-  // FLT_MAX when every A is zero (then only an infinite or NaN Δ leaves the range); 0 when some
-  // A is infinite (the block always takes the MUFU path)
-  ln.dlim = amax > 0.f ? 126.f / amax : 3.402823466e38f;
-
-  float dsum = 0.f, dcomp = 0.f;  // Kahan-compensated ΣΔ of this lane's steps (summary pass)
-  const auto kahan = [&](float x) {
-    const float yk = x - dcomp;
-    const float tk = dsum + yk;
-    dcomp = (tk - dsum) - yk;
-    dsum = tk;
-  };
-
-  // prologue: block 0's scalars and B/C, block 1's rows in flight
-  typename Lane::Rows rn, rf;
-  typename Lane::URow u_cur, z_cur, pu, pz;
-  bool safe = true;
-  if (nblk > 0) {
-    ln.fetch(rn, t_begin);
-    float dblk = 0.f;
-    bool ok = true;
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-      ln.stage_row(reinterpret_cast<float*>(tile.buf[0].sB), reinterpret_cast<float*>(tile.buf[0].sC),
-                   rn, j);
-#pragma unroll
-    for (int j = 0; j < SPL; j += 2)
-      ln.scalar_pair(tile.buf[0].sd, rn, j, own(min(kBlk, t_end - t_begin)), dblk, ok);
-    u_cur = rn.u;
-    z_cur = rn.z;
-    if (nblk > 1) ln.fetch(rn, t_begin + kBlk);
-    else rn.zero();
-    if (MODE == kFwdSummary) kahan(dblk);
-    __syncwarp();
-    safe = __all_sync(0xffffffffu, ok);
-  }
-  pu.zero();
-  pz.zero();
-
-#pragma unroll 1
-  for (int i = 0; i < nblk; ++i) {
-    const int t0 = t_begin + i * kBlk;
-    const int nvalid = min(kBlk, t_end - t0);
-    BlockBuf<LPC>& cur = tile.buf[i & 1];
-    BlockBuf<LPC>& nxt = tile.buf[(i & 1) ^ 1];
-    const bool has_next = i + 1 < nblk, has_prev = i > 0;
-    if (i + 2 < nblk) ln.fetch(rf, t0 + 2 * kBlk);
-    else rf.zero();
-    if (MODE != kFwdSummary && a.ckpt && act) {
-      float* cp = a.ckpt + (ch * nblk_total + t0 / kBlk) * N;
-#pragma unroll
-      for (int j = 0; j < PPL; ++j) {
-        const int n0 = SPL * q + 2 * j;
-        if (n0 < N) cp[n0] = hh[j].x;
-        if (n0 + 1 < N) cp[n0 + 1] = hh[j].y;
-      }
-    }
-    const int nown_next = has_next ? own(min(kBlk, t_end - t0 - kBlk)) : 0;
-    float o[SPL];
-    float dblk = 0.f;
-    bool ok = true;
-    if (nvalid == kBlk) {
-      float* nsB = reinterpret_cast<float*>(nxt.sB);
-      float* nsC = reinterpret_cast<float*>(nxt.sC);
-      if (kPrecise || !safe)
-        interleaved_block<kPrecise, kReadout, LPC, KS, KS>(ln, &cur, cur.yp, nsB, nsC, nxt.sd,
-                                                             nxt.yp, hh, al, ra, rn, nown_next, pu, pz,
-                                                             o, dblk, ok);
-      else
-        interleaved_block<kPrecise, kReadout, LPC, KE, KO>(ln, &cur, cur.yp, nsB, nsC, nxt.sd,
-                                                           nxt.yp, hh, al, ra, rn, nown_next, pu, pz,
-                                                           o, dblk, ok);
-    } else {
-      // partial (last) block: the three stages one after another
-      if (kReadout && has_prev) {
-#pragma unroll
-        for (int j = 0; j < SPL; j += 2) ln.output_pair(nxt.yp, pu, pz, j, o);
-      }
-      if (kPrecise || !safe)
-        state_loop<kPrecise, kReadout, LPC, KS, KS>(cur, hh, al, ra, slot, q, nvalid);
-      else
-        state_loop<kPrecise, kReadout, LPC, KE, KO>(cur, hh, al, ra, slot, q, nvalid);
-      // a partial block is the last one: there is no next block to prepare
-    }
-    __syncwarp();  // this block's partial readouts and the next block's table are complete
-    if (kReadout && has_prev) ln.store_out(t0 - kBlk, o, SPL);  // blocks before the last are full
-    if (MODE == kFwdSummary) kahan(dblk);
-    safe = __all_sync(0xffffffffu, ok);
-    pu = u_cur;
-    pz = z_cur;
-    u_cur = rn.u;
-    z_cur = rn.z;
-    rn = rf;
-  }
-
-  // epilogue: the last block's outputs (its u, z are now in pu, pz)
-  if (kReadout && nblk > 0) {
-    const int tl = t_begin + (nblk - 1) * kBlk;
-    float o[SPL];
-#pragma unroll
-    for (int j = 0; j < SPL; j += 2) ln.output_pair(tile.buf[(nblk - 1) & 1].yp, pu, pz, j, o);
-    ln.store_out(tl, o, own(t_end - tl));
-  }
-
-  if (MODE == kFwdSummary) {
-    float total = dsum;
-#pragma unroll
-    for (int m = 1; m < LPC; m <<= 1) total += __shfl_xor_sync(0xffffffffu, total, m);
-    if (!act) return;
-    const int chunk = blockIdx.y;
-    float* sp = a.summ + ((long long)chunk * a.batch * a.dim + ch) * kNS + SPL * q;
-#pragma unroll
-    for (int j = 0; j < PPL; ++j) reinterpret_cast<float2*>(sp)[j] = hh[j];
-    if (q == 0) a.dsum[(long long)chunk * a.batch * a.dim + ch] = total;
-  } else if (last_chunk && a.hL && act) {
-    float* hp = a.hL + ch * N;
-#pragma unroll
-    for (int j = 0; j < PPL; ++j) {
-      const int n0 = SPL * q + 2 * j;
-      if (n0 < N) hp[n0] = hh[j].x;
-      if (n0 + 1 < N) hp[n0 + 1] = hh[j].y;
-    }
-  }
-}
-
-template <typename IO, bool VEC, int MODE, int LPC, int KE, int KO>
-__global__ void __launch_bounds__(128) fwd_kernel(const FwdArgs a) {
-  using Lay = Layout<LPC>;
-  constexpr int SPL = Lay::kSPL, PPL = Lay::kPPL;
-  extern __shared__ float4 smem4[];
-  WarpTile<LPC>* tiles = reinterpret_cast<WarpTile<LPC>*>(smem4);
-  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  const long long w = (long long)blockIdx.x * (blockDim.x >> 5) + wib;
-  if (w >= a.nwarps) return;  // whole warp leaves together
-  const int slot = lane / LPC, q = lane % LPC;
-  const int b = (int)(w / a.warps_per_b);
-  const int d = (int)(w % a.warps_per_b) * Lay::kChW + slot;
-  const bool act = d < a.dim;
-  const int dd = act ? d : a.dim - 1;  // idle lanes shadow a valid channel and store nothing
-  const long long ch = (long long)b * a.dim + dd;
-  const int chunk = blockIdx.y;
-  const int t_begin = chunk * a.chunk_len;
-  const int t_end = min(a.L, t_begin + a.chunk_len);
-  const bool last_chunk = t_end == a.L;
-
-  constexpr bool kPrecise = std::is_same<IO, float>::value;
-  const float ascale = kPrecise ? 1.f : kLog2e;
-  constexpr bool kSA = KE == kKpScalar || KE == kKpScalarZoh;
-  constexpr bool kZOH = KE == kKpZoh || KE == kKpScalarZoh;
-  const float* Ad = a.A + (long long)dd * (kSA ? 1 : a.N);
-  const float* hsrc = nullptr;
-  bool hs16 = false;  // hin rows hold 16 states; h0 rows hold N
-  if (MODE != kFwdSummary) {
-    if (a.hin) {
-      hsrc = a.hin + ((long long)chunk * a.batch * a.dim + ch) * kNS;
-      hs16 = true;
-    } else if (a.h0) {
-      hsrc = a.h0 + ch * a.N;
-    }
-  }
-  // al = A log2 e (A on the fp32 path); ra = 1/A for the ZOH coefficient, with |A| < 1e-20
-  // taken as -1e-20 (the A -> 0 limit, g = Δ)
-  float2 al[PPL], ra[PPL], hh[PPL];
-#pragma unroll
-  for (int j = 0; j < PPL; ++j) {
-    const int n0 = SPL * q + 2 * j, n1 = n0 + 1;
-    float2 av = kSA ? f2(Ad[0])  // one decay rate for every state
-                    : make_float2(n0 < a.N ? Ad[n0] : 0.f, n1 < a.N ? Ad[n1] : 0.f);
-    if (kZOH) av = make_float2(zoh_rate(av.x), zoh_rate(av.y));
-    al[j] = mul2(av, f2(ascale));
-    ra[j] = kZOH ? make_float2(1.f / av.x, 1.f / av.y) : f2(0.f);
-    hh[j] = make_float2((hsrc && (hs16 || n0 < a.N)) ? hsrc[n0] : 0.f,
-                        (hsrc && (hs16 || n1 < a.N)) ? hsrc[n1] : 0.f);
-  }
-  const float Dd = (MODE == kFwdOut && a.D) ? a.D[dd] : 0.f;
-  const float bias = a.dt_bias ? a.dt_bias[dd] : 0.f;
-  WarpTile<LPC>& tile = tiles[wib];
-
-  run_chunk<IO, VEC, MODE, LPC, KE, KO>(a, tile, hh, al, ra, Dd, bias, lane, slot, q, b, act, ch,
-                                        t_begin, t_end, last_chunk);
-}
 
 // Chain the chunk summaries: h_in(0) = h0, h_in(j+1) = exp(A ΣΔ_j) h_in(j) + h_end(j).
 // One thread per (channel, state).
@@ -632,81 +33,16 @@ __global__ void fwd_carry_kernel(const FwdArgs a, const float* __restrict__ summ
   }
 }
 
-template <typename IO, bool VEC, int MODE, int LPC, int KE, int KO>
-void launch_one(const FwdArgs& a, dim3 grid, dim3 block, cudaStream_t s) {
-  const size_t smem = (size_t)(block.x / 32) * sizeof(WarpTile<LPC>);
-  if (smem > 48 * 1024)
-    cudaFuncSetAttribute(fwd_kernel<IO, VEC, MODE, LPC, KE, KO>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  fwd_kernel<IO, VEC, MODE, LPC, KE, KO><<<grid, block, smem, s>>>(a);
-}
-
-template <typename IO, bool VEC, int MODE>
-cudaError_t launch_mode(const FwdArgs& a, int wpb, int kmufu, cudaStream_t s) {
-  const long long ctas = (a.nwarps + wpb - 1) / wpb;
-  const int nchunk_launch = MODE == kFwdSummary ? a.nchunk - 1 : a.nchunk;  // last chunk's summary is unused
-  if (ctas <= 0 || nchunk_launch <= 0) return cudaSuccess;
-  const dim3 grid((unsigned)ctas, (unsigned)nchunk_launch), block(32 * wpb);
-  if (a.scalar_a && a.zoh) {  // two lanes per channel, no exponential in the time loop
-    launch_one<IO, VEC, MODE, 2, kKpScalarZoh, kKpScalarZoh>(a, grid, block, s);
-  } else if (a.scalar_a) {
-    launch_one<IO, VEC, MODE, 2, kKpScalar, kKpScalar>(a, grid, block, s);
-  } else if (a.zoh) {  // per-state ZOH coefficient on the FMA pipe
-    launch_one<IO, VEC, MODE, 2, kKpZoh, kKpZoh>(a, grid, block, s);
-  } else if constexpr (std::is_same<IO, float>::value) {  // fp32: library expf
-    if (a.lpc == 4) launch_one<IO, VEC, MODE, 4, 2, 2>(a, grid, block, s);
-    else if (a.lpc == 1) launch_one<IO, VEC, MODE, 1, 8, 8>(a, grid, block, s);
-    else launch_one<IO, VEC, MODE, 2, 4, 4>(a, grid, block, s);
-  } else if constexpr (MODE != kFwdOut) {
-    if (a.lpc == 4) launch_one<IO, VEC, MODE, 4, 2, 1>(a, grid, block, s);
-    else if (a.lpc == 1) launch_one<IO, VEC, MODE, 1, 7, 6>(a, grid, block, s);
-    else launch_one<IO, VEC, MODE, 2, 4, 3>(a, grid, block, s);
-  } else if (a.lpc == 4) {
-    // exponentials on the MUFU unit per lane over two steps (of 8): 4, 6 or 8
-    switch (kmufu) {
-      case 8: launch_one<IO, VEC, MODE, 4, 1, 1>(a, grid, block, s); break;
-      case 16: launch_one<IO, VEC, MODE, 4, 2, 2>(a, grid, block, s); break;
-      default: launch_one<IO, VEC, MODE, 4, 2, 1>(a, grid, block, s); break;
-    }
-  } else if (a.lpc == 1) {
-    // exponentials on the MUFU unit per lane over two steps (of 32), in units of 16/16
-    switch (kmufu) {
-      case 8: launch_one<IO, VEC, MODE, 1, 4, 4>(a, grid, block, s); break;
-      case 10: launch_one<IO, VEC, MODE, 1, 5, 5>(a, grid, block, s); break;
-      case 12: launch_one<IO, VEC, MODE, 1, 6, 6>(a, grid, block, s); break;
-      case 16: launch_one<IO, VEC, MODE, 1, 8, 8>(a, grid, block, s); break;
-      default: launch_one<IO, VEC, MODE, 1, 7, 7>(a, grid, block, s); break;
-    }
-  } else {
-    // exponentials on the MUFU unit per lane over two steps (of 16): 8 ... 16
-    switch (kmufu) {
-      case 8: launch_one<IO, VEC, MODE, 2, 2, 2>(a, grid, block, s); break;
-      case 10: launch_one<IO, VEC, MODE, 2, 3, 2>(a, grid, block, s); break;
-      case 12: launch_one<IO, VEC, MODE, 2, 3, 3>(a, grid, block, s); break;
-      case 16: launch_one<IO, VEC, MODE, 2, 4, 4>(a, grid, block, s); break;
-      default: launch_one<IO, VEC, MODE, 2, 4, 3>(a, grid, block, s); break;
-    }
-  }
-  return cudaGetLastError();
-}
-
 }  // namespace
-
-template <typename IO, bool VEC>
-cudaError_t launch_io(const FwdArgs& a, int mode, int wpb, int kmufu, cudaStream_t s) {
-  switch (mode) {
-    case kFwdOut: return launch_mode<IO, VEC, kFwdOut>(a, wpb, kmufu, s);
-    case kFwdSummary: return launch_mode<IO, VEC, kFwdSummary>(a, wpb, kmufu, s);
-    default: return launch_mode<IO, VEC, kFwdCkpt>(a, wpb, kmufu, s);
-  }
-}
 
 cudaError_t launch_fwd(const FwdArgs& a, int io, bool vec, int mode, int wpb, int kmufu,
                        cudaStream_t s) {
-  if (io == 1) return vec ? launch_io<uint16_t, true>(a, mode, wpb, kmufu, s)
-                          : launch_io<uint16_t, false>(a, mode, wpb, kmufu, s);
-  return vec ? launch_io<float, true>(a, mode, wpb, 16, s)
-             : launch_io<float, false>(a, mode, wpb, 16, s);
+  // fp32: library expf for every state (the MUFU split does not apply)
+  if (a.reverse)
+    return io == 1 ? launch_fwd_rev_bf16(a, vec, mode, wpb, kmufu, s)
+                   : launch_fwd_rev_f32(a, vec, mode, wpb, 16, s);
+  return io == 1 ? launch_fwd_bf16(a, vec, mode, wpb, kmufu, s)
+                 : launch_fwd_f32(a, vec, mode, wpb, 16, s);
 }
 
 cudaError_t launch_fwd_carry(const FwdArgs& a, const float* summ, const float* dsum, float* hin,

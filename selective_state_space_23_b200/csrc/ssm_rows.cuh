@@ -106,28 +106,33 @@ __device__ __forceinline__ void reverse_row(Row<IO, E>& r) {
 // E consecutive steps [tau, tau + E) of one time row in scan order.  In reverse order (rev) the
 // scan's step tau is stored at row index L-1-tau, so the E steps are the row's elements
 // [L-tau-E, L-tau) read backwards.  Steps at or beyond nvalid read as zero.  VEC: the row
-// segment is aligned as load_row requires and all E steps are valid.
-template <typename IO, int E, bool VEC>
+// segment is aligned as load_row requires and all E steps are valid.  REORDER = false leaves a
+// reversed segment in row order (reverse_row later puts it in scan order), so that a prefetch
+// does not wait for its data at the load.
+template <typename IO, int E, bool VEC, bool REORDER = true>
 __device__ __forceinline__ void load_steps(Row<IO, E>& r, const IO* row, int L, int tau, int nvalid,
                                            bool rev) {
   if (!rev) {
     load_row<IO, E, VEC>(r, row + tau, nvalid);
-  } else if (VEC) {
-    load_row<IO, E, true>(r, row + (L - tau - E), E);
-    reverse_row(r);
+    return;
+  }
+  const long long base = (long long)L - tau - E;  // row index of the segment's first element
+  if (VEC) {
+    load_row<IO, E, true>(r, row + base, E);
   } else {
     r.zero();
 #pragma unroll
     for (int e = 0; e < E; ++e) {
-      if (e < nvalid) {
+      if (e >= E - nvalid) {  // scan step E-1-e is valid
         if (sizeof(IO) == 4)
-          r.w[e] = __ldcs(reinterpret_cast<const uint32_t*>(row) + (L - 1 - tau - e));
+          r.w[e] = __ldcs(reinterpret_cast<const uint32_t*>(row) + (base + e));
         else
           r.w[e >> 1] |= ((uint32_t)__ldcs(reinterpret_cast<const unsigned short*>(row) +
-                                           (L - 1 - tau - e))) << (16 * (e & 1));
+                                           (base + e))) << (16 * (e & 1));
       }
     }
   }
+  if (REORDER) reverse_row(r);
 }
 
 // Store E values of steps [tau, tau + E) (only the first nvalid) to a time row in scan order.
