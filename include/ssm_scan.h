@@ -190,27 +190,36 @@ SSM_API int ssm_scan_bwd_scalar_a(const void* u, const void* delta, const float*
  *                 c = (exp(Δ_t A) - 1)/A per state (c -> Δ_t as A -> 0) instead of Δ_t.
  *                 Combines with the other flags.
  * Any other bit is rejected with SSM_EINVAL.  Arguments are those of ssm_scan_fwd /
- * ssm_scan_bwd plus flags.
+ * ssm_scan_bwd plus flags and bc_groups:
+ *   bc_groups     B, C (and dB, dC) are [batch][bc_groups][dstate][L]: the per-token B_t, C_t
+ *                 of the selection mechanism ("Seçim Mekanizması (S6)") computed once per group
+ *                 of dim / bc_groups consecutive channels instead of once for all channels (the
+ *                 grouping Mamba-2 uses; 1 = shared by every channel).  dim must be a multiple of
+ *                 bc_groups (else SSM_EINVAL) and dim / bc_groups a multiple of 16 (the channels
+ *                 of one warp share a group; else SSM_EUNSUPPORTED).
  */
 #define SSM_SCALAR_A 1
 #define SSM_REVERSE 2
 #define SSM_ZOH 4
 SSM_API size_t ssm_scan_fwd_ex_workspace_size(int batch, int dim, int seqlen, int dstate,
-                                              int io_dtype, int flags);
+                                              int bc_groups, int io_dtype, int flags);
 SSM_API int ssm_scan_fwd_ex(const void* u, const void* delta, const float* A, const void* B,
                             const void* C, const float* D, const void* z, const float* dt_bias,
                             int delta_softplus, const float* h0, float* hL, void* out, float* ckpt,
                             void* workspace, size_t workspace_bytes, int batch, int dim,
-                            int seqlen, int dstate, int io_dtype, int flags, void* stream);
+                            int seqlen, int dstate, int bc_groups, int io_dtype, int flags,
+                            void* stream);
 SSM_API size_t ssm_scan_bwd_ex_workspace_size(int batch, int dim, int seqlen, int dstate,
-                                              int io_dtype, int have_ckpt, int flags);
+                                              int bc_groups, int io_dtype, int have_ckpt,
+                                              int flags);
 SSM_API int ssm_scan_bwd_ex(const void* u, const void* delta, const float* A, const void* B,
                             const void* C, const float* D, const void* z, const float* dt_bias,
                             int delta_softplus, const float* h0, const void* dout,
                             const float* dhL, const float* ckpt, void* du, void* ddelta, float* dA,
                             void* dB, void* dC, float* dD, void* dz, float* ddt_bias, float* dh0,
                             void* workspace, size_t workspace_bytes, int batch, int dim,
-                            int seqlen, int dstate, int io_dtype, int flags, void* stream);
+                            int seqlen, int dstate, int bc_groups, int io_dtype, int flags,
+                            void* stream);
 
 /* Size of the static scratch array used by ssm_scan_fwd_noalloc (8 MiB per GPU). */
 #define SSM_NOALLOC_SCRATCH_BYTES (8u << 20)

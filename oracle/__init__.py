@@ -15,6 +15,8 @@ The arithmetic lives in ``ssm_oracle.c`` (plain double-precision loops, cited th
                          finite differences of ``scan_fwd`` (parity of the gradient formulas
                          themselves is otherwise unpinned by the pages).
   * ``state_update``  -- one recurrent (decode) step of the same recurrence, in place.
+  * grouped B/C      -- B, C of shape [batch, G, N, L]: each group of dim/G channels is an
+                         independent scan with its own B, C, run as exactly that.
   * ``reverse=True``  -- the scan backwards in time (t = L-1 .. 0), the anti-causal half of a
                          bidirectional layer ("2024 Reading List: Neural Network", Hydra notes):
                          by definition the forward scan of the time-reversed sequences, so it is
@@ -78,6 +80,48 @@ def _flip(x):
     return None if x is None else np.ascontiguousarray(np.asarray(x, dtype=np.float64)[..., ::-1])
 
 
+_PER_CHANNEL = {"u", "delta", "z", "dout"}  # [batch, dim, L]
+_PER_D = {"A", "D", "dt_bias"}             # [dim, ...]
+_PER_BD = {"h0", "dhL"}                    # [batch, dim, N]
+
+
+def _grouped(fn, u, delta, A, B, C, *rest, **kw):
+    """Grouped B/C ([batch, G, N, L]): channel d uses group d // (dim // G).  By definition each
+    group is an independent scan over its channels with its own B, C; run it per group and
+    assemble the results (dB, dC per group; every other output per channel)."""
+    u = np.asarray(u, dtype=np.float64)
+    batch, dim, L = u.shape
+    G = np.shape(B)[1]
+    if dim % G:
+        raise ValueError(f"dim {dim} is not a multiple of {G} groups")
+    per = dim // G
+    args = {"u": u, "delta": delta, "A": A}
+    if rest:
+        args["dout"] = rest[0]
+    parts = []
+    for g in range(G):
+        sl = slice(g * per, (g + 1) * per)
+        pick = lambda k, v: (None if v is None else
+                             np.asarray(v)[:, sl] if k in _PER_CHANNEL or k in _PER_BD else
+                             np.asarray(v)[sl] if k in _PER_D else v)
+        pos = [pick(k, args[k]) for k in ("u", "delta", "A")]
+        pos += [np.asarray(B)[:, g], np.asarray(C)[:, g]]
+        if "dout" in args:
+            pos.append(pick("dout", args["dout"]))
+        parts.append(fn(*pos, **{k: pick(k, v) for k, v in kw.items()}))
+    res = {}
+    for k in parts[0]:
+        if parts[0][k] is None:
+            res[k] = None
+        elif k in ("dB", "dC"):
+            res[k] = np.stack([p[k] for p in parts], 1)
+        elif k in ("dA", "dD", "ddt_bias"):
+            res[k] = np.concatenate([p[k] for p in parts], 0)
+        else:
+            res[k] = np.concatenate([p[k] for p in parts], 1)
+    return res
+
+
 def scan_fwd(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=True,
              h0=None, zoh=False, channels=None, nthreads=0, out=None, ypre=False, reverse=False):
     """Forward selective scan in fp64.
@@ -87,6 +131,10 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=Tru
     left as in ``out``, default zeros).  ``reverse``: scan from t = L-1 down to 0 (h0 enters
     at t = L-1, hL is the state after t = 0).  Returns dict(out, hL[, ypre]).
     """
+    if np.ndim(B) == 4:
+        return _grouped(scan_fwd, u, delta, A, B, C, D=D, z=z, dt_bias=dt_bias,
+                        delta_softplus=delta_softplus, h0=h0, zoh=zoh, nthreads=nthreads,
+                        ypre=ypre, reverse=reverse)
     if reverse:
         res = scan_fwd(_flip(u), _flip(delta), A, _flip(B), _flip(C), D=D, z=_flip(z),
                        dt_bias=dt_bias, delta_softplus=delta_softplus, h0=h0, zoh=zoh,
@@ -137,6 +185,10 @@ def scan_bwd(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None, delta_softpl
     summed gradients (dA, dB, dC, dD, ddt_bias) hold only those channels' contributions.
     ``reverse``: gradients of the reverse scan (time-indexed gradients reversed back).
     """
+    if np.ndim(B) == 4:
+        return _grouped(scan_bwd, u, delta, A, B, C, dout, D=D, z=z, dt_bias=dt_bias,
+                        delta_softplus=delta_softplus, h0=h0, dhL=dhL, nthreads=nthreads,
+                        reverse=reverse, zoh=zoh)
     if reverse:
         g = scan_bwd(_flip(u), _flip(delta), A, _flip(B), _flip(C), _flip(dout), D=D, z=_flip(z),
                      dt_bias=dt_bias, delta_softplus=delta_softplus, h0=h0, dhL=dhL,

@@ -82,6 +82,17 @@ def _workspace(nbytes, device, given):
     return torch.empty(nbytes, dtype=torch.uint8, device=device)
 
 
+def _bc_layout(B, batch, L):
+    """(groups, N, shape) of the B/C layout: [batch, N, L] (one group) or [batch, G, N, L]."""
+    if not isinstance(B, torch.Tensor):
+        raise TypeError("B must be a torch.Tensor")
+    if B.dim() == 3:
+        return 1, B.shape[1], (batch, B.shape[1], L)
+    if B.dim() == 4:
+        return B.shape[1], B.shape[2], (batch, B.shape[1], B.shape[2], L)
+    raise ValueError(f"B must be [batch, N, L] or [batch, groups, N, L], got {tuple(B.shape)}")
+
+
 def _flags(scalar_a, reverse, zoh):
     return ((_abi.SSM_SCALAR_A if scalar_a else 0) | (_abi.SSM_REVERSE if reverse else 0)
             | (_abi.SSM_ZOH if zoh else 0))
@@ -91,14 +102,14 @@ def _scan_fwd(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, return_final
               return_ckpt, out, workspace, scalar_a, reverse, zoh):
     dev = u.device
     batch, dim, L = u.shape
-    N = B.shape[1]
+    G, N, bc_shape = _bc_layout(B, batch, L)
     io = u.dtype
     code = _io_code(io)
     _need(u, "u", (batch, dim, L), io, dev)
     _need(delta, "delta", (batch, dim, L), io, dev)
     _need(A, "A", (dim,) if scalar_a else (dim, N), torch.float32, dev)
-    _need(B, "B", (batch, N, L), io, dev)
-    _need(C, "C", (batch, N, L), io, dev)
+    _need(B, "B", bc_shape, io, dev)
+    _need(C, "C", bc_shape, io, dev)
     _opt(D, "D", (dim,), torch.float32, dev)
     _opt(z, "z", (batch, dim, L), io, dev)
     _opt(dt_bias, "dt_bias", (dim,), torch.float32, dev)
@@ -110,12 +121,12 @@ def _scan_fwd(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, return_final
     nblk = (L + CKPT_STEPS - 1) // CKPT_STEPS
     ckpt = torch.empty((batch, dim, nblk, N), dtype=torch.float32, device=dev) if return_ckpt else None
     flags = _flags(scalar_a, reverse, zoh)
-    nws = int(_abi.lib().ssm_scan_fwd_ex_workspace_size(batch, dim, L, N, code, flags))
+    nws = int(_abi.lib().ssm_scan_fwd_ex_workspace_size(batch, dim, L, N, G, code, flags))
     ws = _workspace(nws, dev, workspace)
     rc = _abi.lib().ssm_scan_fwd_ex(
         _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias),
         int(bool(delta_softplus)), _ptr(h0), _ptr(hL), _ptr(out), _ptr(ckpt), _ptr(ws),
-        0 if ws is None else ws.numel(), batch, dim, L, N, code, flags, _stream(dev))
+        0 if ws is None else ws.numel(), batch, dim, L, N, G, code, flags, _stream(dev))
     _abi.check(rc, "ssm_scan_fwd_ex")
     if not return_final_state and not return_ckpt:
         return out
@@ -130,8 +141,8 @@ def _scan_fwd(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, return_final
 def ssm_scan_fwd(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=True, h0=None,
                  return_final_state=False, return_ckpt=False, out=None, workspace=None,
                  reverse=False, zoh=False):
-    """Forward scan.  u, delta, z: [batch, dim, L]; B, C: [batch, N, L] (io dtype f32 or bf16);
-    A: [dim, N] f32; D, dt_bias: [dim] f32; h0: [batch, dim, N] f32.  reverse: scan from
+    """Forward scan.  u, delta, z: [batch, dim, L]; B, C: [batch, N, L] or, grouped, [batch, G,
+    N, L] (channel d uses group d // (dim // G)) (io dtype f32 or bf16); A: [dim, N] f32; D, dt_bias: [dim] f32; h0: [batch, dim, N] f32.  reverse: scan from
     t = L-1 down to 0.  zoh: zero-order-hold input term (e^{ΔA} - 1)/A B x instead of Δ B x.
     Returns out, or a tuple (out, hL?, ckpt?) when those are requested."""
     return _scan_fwd(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, return_final_state,
@@ -150,15 +161,15 @@ def _scan_bwd(u, delta, A, B, C, dout, D, z, dt_bias, delta_softplus, h0, dhL, c
               workspace, need, scalar_a, reverse, zoh):
     dev = u.device
     batch, dim, L = u.shape
-    N = B.shape[1]
+    G, N, bc_shape = _bc_layout(B, batch, L)
     io = u.dtype
     code = _io_code(io)
     _need(u, "u", (batch, dim, L), io, dev)
     _need(delta, "delta", (batch, dim, L), io, dev)
     a_shape = (dim,) if scalar_a else (dim, N)
     _need(A, "A", a_shape, torch.float32, dev)
-    _need(B, "B", (batch, N, L), io, dev)
-    _need(C, "C", (batch, N, L), io, dev)
+    _need(B, "B", bc_shape, io, dev)
+    _need(C, "C", bc_shape, io, dev)
     _need(dout, "dout", (batch, dim, L), io, dev)
     _opt(D, "D", (dim,), torch.float32, dev)
     _opt(z, "z", (batch, dim, L), io, dev)
@@ -174,15 +185,15 @@ def _scan_bwd(u, delta, A, B, C, dout, D, z, dt_bias, delta_softplus, h0, dhL, c
         "du": e((batch, dim, L), io) if "du" in want else None,
         "ddelta": e((batch, dim, L), io) if "ddelta" in want else None,
         "dz": e((batch, dim, L), io) if ("dz" in want and z is not None) else None,
-        "dB": e((batch, N, L), io) if "dB" in want else None,
-        "dC": e((batch, N, L), io) if "dC" in want else None,
+        "dB": e(bc_shape, io) if "dB" in want else None,
+        "dC": e(bc_shape, io) if "dC" in want else None,
         "dA": e(a_shape, torch.float32) if "dA" in want else None,
         "dD": e((dim,), torch.float32) if "dD" in want else None,
         "ddt_bias": e((dim,), torch.float32) if "ddt_bias" in want else None,
         "dh0": e((batch, dim, N), torch.float32) if "dh0" in want else None,
     }
     flags = _flags(scalar_a, reverse, zoh)
-    nws = int(_abi.lib().ssm_scan_bwd_ex_workspace_size(batch, dim, L, N, code,
+    nws = int(_abi.lib().ssm_scan_bwd_ex_workspace_size(batch, dim, L, N, G, code,
                                                          int(ckpt is not None), flags))
     ws = _workspace(nws, dev, workspace)
     rc = _abi.lib().ssm_scan_bwd_ex(
@@ -190,7 +201,8 @@ def _scan_bwd(u, delta, A, B, C, dout, D, z, dt_bias, delta_softplus, h0, dhL, c
         int(bool(delta_softplus)), _ptr(h0), _ptr(dout), _ptr(dhL), _ptr(ckpt),
         _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]),
         _ptr(g["dD"]), _ptr(g["dz"]), _ptr(g["ddt_bias"]), _ptr(g["dh0"]),
-        _ptr(ws), 0 if ws is None else ws.numel(), batch, dim, L, N, code, flags, _stream(dev))
+        _ptr(ws), 0 if ws is None else ws.numel(), batch, dim, L, N, G, code, flags,
+        _stream(dev))
     _abi.check(rc, "ssm_scan_bwd_ex")
     return g
 

@@ -136,6 +136,17 @@ int check_dims(int batch, int dim, int seqlen, int dstate, int io) {
 }
 
 size_t esize(int io) { return io == SSM_BF16 ? 2 : 4; }
+
+// B/C groups: dim must split into groups of whole warps (16 channels each).
+int check_groups(int dim, int bc_groups) {
+  if (bc_groups < 1) return fail(SSM_EINVAL, "bc_groups must be >= 1, got %d", bc_groups);
+  if (bc_groups == 1) return SSM_OK;
+  if (dim % bc_groups != 0) return fail(SSM_EINVAL, "dim %d is not a multiple of bc_groups %d", dim, bc_groups);
+  if ((dim / bc_groups) % 16 != 0)
+    return fail(SSM_EUNSUPPORTED, "grouped B/C needs dim / bc_groups to be a multiple of 16 (got %d)",
+                dim / bc_groups);
+  return SSM_OK;
+}
 size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
 
 bool aligned16(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
@@ -209,11 +220,12 @@ struct BwdLayout {
   int wpb, ngroups;
 };
 
-BwdLayout layout_bwd(int batch, int dim, int seqlen, int dstate, bool have_ckpt) {
+BwdLayout layout_bwd(int batch, int dim, int seqlen, int dstate, bool have_ckpt, int bc_groups) {
   BwdLayout l;
   // one warp per CTA: CTAs of several warps synchronise once per block for the dB/dC partials,
-  // which measured slower on B200 than writing one partial per warp
-  l.wpb = env_int("SSM_BWD_WPB", 1);
+  // which measured slower on B200 than writing one partial per warp (and with grouped B/C every
+  // CTA must lie inside one group)
+  l.wpb = bc_groups > 1 ? 1 : env_int("SSM_BWD_WPB", 1);
   if (l.wpb < 1 || l.wpb > 4) l.wpb = 1;
   const int warps_per_b = (dim + 15) / 16;  // 16 channels per warp
   l.ngroups = (warps_per_b + l.wpb - 1) / l.wpb;
@@ -266,15 +278,16 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
                   const float* D, const void* z, const float* dt_bias, int delta_softplus,
                   const float* h0, float* hL, void* out, float* ckpt, void* workspace,
                   size_t workspace_bytes, int batch, int dim, int seqlen, int dstate,
-                  int io_dtype, void* stream, int flags) {
+                  int io_dtype, void* stream, int flags, int bc_groups) {
   g_err[0] = 0;
   if (flags & ~(SSM_SCALAR_A | SSM_REVERSE | SSM_ZOH))
     return fail(SSM_EINVAL, "unknown flags 0x%x", flags);
   const bool scalar_a = (flags & SSM_SCALAR_A) != 0;
   TRY(check_dims(batch, dim, seqlen, dstate, io_dtype));
+  TRY(check_groups(dim, bc_groups));
   const size_t es = esize(io_dtype);
   const size_t nx = (size_t)batch * dim * seqlen * es;
-  const size_t nbc = (size_t)batch * dstate * seqlen * es;
+  const size_t nbc = (size_t)batch * bc_groups * dstate * seqlen * es;
   const size_t nst = (size_t)batch * dim * dstate * 4;
   const size_t nblk = (seqlen + ssm::kBlk - 1) / ssm::kBlk;
   TRY(check_ptr(u, nx, es, "u"));
@@ -310,7 +323,8 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
   a.scalar_a = scalar_a ? 1 : 0;
   a.reverse = (flags & SSM_REVERSE) ? 1 : 0;
   a.zoh = (flags & SSM_ZOH) ? 1 : 0;
-  a.lpc = (scalar_a || a.zoh) ? 2 : fwd_lpc();
+  a.bc_groups = bc_groups;
+  a.lpc = (scalar_a || a.zoh || bc_groups > 1) ? 2 : fwd_lpc();
   a.warps_per_b = (dim + 32 / a.lpc - 1) / (32 / a.lpc);
   a.nwarps = (long long)batch * a.warps_per_b;
   const bool vec = (seqlen * es) % 16 == 0 && aligned16(u) && aligned16(delta) && aligned16(z) &&
@@ -366,12 +380,13 @@ int ssm_scan_fwd(const void* u, const void* delta, const float* A, const void* B
                  size_t workspace_bytes, int batch, int dim, int seqlen, int dstate,
                  int io_dtype, void* stream) {
   return scan_fwd_impl(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, hL, out, ckpt,
-                       workspace, workspace_bytes, batch, dim, seqlen, dstate, io_dtype, stream, 0);
+                       workspace, workspace_bytes, batch, dim, seqlen, dstate, io_dtype, stream, 0, 1);
 }
 
-size_t ssm_scan_fwd_ex_workspace_size(int batch, int dim, int seqlen, int dstate, int io_dtype,
-                                      int flags) {
+size_t ssm_scan_fwd_ex_workspace_size(int batch, int dim, int seqlen, int dstate, int bc_groups,
+                                      int io_dtype, int flags) {
   (void)flags;  // the time-split scratch does not depend on the variant
+  if (bc_groups < 1) return 0;
   return ssm_scan_fwd_workspace_size(batch, dim, seqlen, dstate, io_dtype);
 }
 
@@ -379,10 +394,10 @@ int ssm_scan_fwd_ex(const void* u, const void* delta, const float* A, const void
                     const void* C, const float* D, const void* z, const float* dt_bias,
                     int delta_softplus, const float* h0, float* hL, void* out, float* ckpt,
                     void* workspace, size_t workspace_bytes, int batch, int dim, int seqlen,
-                    int dstate, int io_dtype, int flags, void* stream) {
+                    int dstate, int bc_groups, int io_dtype, int flags, void* stream) {
   return scan_fwd_impl(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, hL, out, ckpt,
                        workspace, workspace_bytes, batch, dim, seqlen, dstate, io_dtype, stream,
-                       flags);
+                       flags, bc_groups);
 }
 
 size_t ssm_scan_fwd_scalar_a_workspace_size(int batch, int dim, int seqlen, int dstate,
@@ -397,13 +412,13 @@ int ssm_scan_fwd_scalar_a(const void* u, const void* delta, const float* A, cons
                           int dstate, int io_dtype, void* stream) {
   return scan_fwd_impl(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, hL, out, ckpt,
                        workspace, workspace_bytes, batch, dim, seqlen, dstate, io_dtype, stream,
-                       SSM_SCALAR_A);
+                       SSM_SCALAR_A, 1);
 }
 
 size_t ssm_scan_bwd_workspace_size(int batch, int dim, int seqlen, int dstate, int io_dtype,
                                    int have_ckpt) {
   if (check_dims(batch, dim, seqlen, dstate, io_dtype) != SSM_OK) return 0;
-  return layout_bwd(batch, dim, seqlen, dstate, have_ckpt != 0).total;
+  return layout_bwd(batch, dim, seqlen, dstate, have_ckpt != 0, 1).total;
 }
 
 }  // extern "C"
@@ -417,11 +432,12 @@ int scan_bwd_core(const void* u, const void* delta, const float* A, const void* 
                   void* du, void* ddelta, float* dA, void* dB, void* dC, float* dD, void* dz,
                   float* ddt_bias, float* dh0, void* workspace, size_t workspace_bytes,
                   int batch, int dim, int seqlen, int dstate, int io_dtype, void* stream,
-                  bool reverse, bool zoh) {
+                  bool reverse, bool zoh, int bc_groups) {
   TRY(check_dims(batch, dim, seqlen, dstate, io_dtype));
+  TRY(check_groups(dim, bc_groups));
   const size_t es = esize(io_dtype);
   const size_t nx = (size_t)batch * dim * seqlen * es;
-  const size_t nbc = (size_t)batch * dstate * seqlen * es;
+  const size_t nbc = (size_t)batch * bc_groups * dstate * seqlen * es;
   const size_t nst = (size_t)batch * dim * dstate * 4;
   const size_t nblk = (seqlen + ssm::kBlk - 1) / ssm::kBlk;
   TRY(check_ptr(u, nx, es, "u"));
@@ -449,7 +465,7 @@ int scan_bwd_core(const void* u, const void* delta, const float* A, const void* 
     return fail(SSM_EINVAL, "no gradient output requested");
   if (dz && !z) return fail(SSM_EINVAL, "dz requested but z is NULL");
 
-  const BwdLayout l = layout_bwd(batch, dim, seqlen, dstate, ckpt != nullptr);
+  const BwdLayout l = layout_bwd(batch, dim, seqlen, dstate, ckpt != nullptr, bc_groups);
   if (!workspace || workspace_bytes < l.total)
     return fail(SSM_EWORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes, l.total);
   if (reinterpret_cast<uintptr_t>(workspace) & 255)
@@ -477,8 +493,9 @@ int scan_bwd_core(const void* u, const void* delta, const float* A, const void* 
     a.softplus = delta_softplus ? 1 : 0;
     a.reverse = reverse ? 1 : 0;
     a.zoh = zoh ? 1 : 0;
-    a.lpc = zoh ? 2 : fwd_lpc();
-    a.warps_per_b = fwd_warps_per_b(dim);
+    a.bc_groups = bc_groups;
+    a.lpc = (zoh || bc_groups > 1) ? 2 : fwd_lpc();
+    a.warps_per_b = (dim + 32 / a.lpc - 1) / (32 / a.lpc);
     a.nwarps = (long long)batch * a.warps_per_b;
     if ((e = ssm::launch_fwd(a, io_dtype, vec, ssm::kFwdCkpt, fwd_wpb(), fwd_kmufu(a.nwarps), s)) != cudaSuccess)
       return cuda_fail(e, "backward state replay pass");
@@ -494,6 +511,7 @@ int scan_bwd_core(const void* u, const void* delta, const float* A, const void* 
   b.softplus = delta_softplus ? 1 : 0;
   b.reverse = reverse ? 1 : 0;
   b.zoh = zoh ? 1 : 0;
+  b.bc_groups = bc_groups;
   b.warps_per_b = (dim + 15) / 16;
   b.nwarps = (long long)batch * b.warps_per_b;
   b.wpb = l.wpb;
@@ -518,13 +536,15 @@ int ssm_scan_bwd(const void* u, const void* delta, const float* A, const void* B
   g_err[0] = 0;
   return scan_bwd_core(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL, ckpt, du,
                        ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, workspace, workspace_bytes,
-                       batch, dim, seqlen, dstate, io_dtype, stream, false, false);
+                       batch, dim, seqlen, dstate, io_dtype, stream, false, false, 1);
 }
 
-size_t ssm_scan_bwd_ex_workspace_size(int batch, int dim, int seqlen, int dstate, int io_dtype,
-                                      int have_ckpt, int flags) {
+size_t ssm_scan_bwd_ex_workspace_size(int batch, int dim, int seqlen, int dstate, int bc_groups,
+                                      int io_dtype, int have_ckpt, int flags) {
   if (flags & ~(SSM_SCALAR_A | SSM_REVERSE | SSM_ZOH)) return 0;
-  const size_t base = ssm_scan_bwd_workspace_size(batch, dim, seqlen, dstate, io_dtype, have_ckpt);
+  if (check_dims(batch, dim, seqlen, dstate, io_dtype) != SSM_OK) return 0;
+  if (check_groups(dim, bc_groups) != SSM_OK) return 0;
+  const size_t base = layout_bwd(batch, dim, seqlen, dstate, have_ckpt != 0, bc_groups).total;
   if (base == 0 || !(flags & SSM_SCALAR_A)) return base;
   return align_up((size_t)dim * dstate * 4) * 2 + base;
 }
@@ -535,7 +555,7 @@ int ssm_scan_bwd_ex(const void* u, const void* delta, const float* A, const void
                     const float* ckpt, void* du, void* ddelta, float* dA, void* dB, void* dC,
                     float* dD, void* dz, float* ddt_bias, float* dh0, void* workspace,
                     size_t workspace_bytes, int batch, int dim, int seqlen, int dstate,
-                    int io_dtype, int flags, void* stream) {
+                    int bc_groups, int io_dtype, int flags, void* stream) {
   g_err[0] = 0;
   if (flags & ~(SSM_SCALAR_A | SSM_REVERSE | SSM_ZOH))
     return fail(SSM_EINVAL, "unknown flags 0x%x", flags);
@@ -545,13 +565,13 @@ int ssm_scan_bwd_ex(const void* u, const void* delta, const float* A, const void
     return scan_bwd_core(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL, ckpt,
                          du, ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, workspace,
                          workspace_bytes, batch, dim, seqlen, dstate, io_dtype, stream, reverse,
-                         zoh);
+                         zoh, bc_groups);
   // scalar decay: broadcast A over the states, run the per-state backward, sum dA over n
   TRY(check_ptr(A, (size_t)dim * 4, 4, "A"));
   TRY(check_opt(dA, (size_t)dim * 4, 4, "dA"));
   const size_t head = align_up((size_t)dim * dstate * 4);
-  const size_t need = ssm_scan_bwd_ex_workspace_size(batch, dim, seqlen, dstate, io_dtype,
-                                                     ckpt != nullptr, flags);
+  const size_t need = ssm_scan_bwd_ex_workspace_size(batch, dim, seqlen, dstate, bc_groups,
+                                                     io_dtype, ckpt != nullptr, flags);
   if (!workspace || workspace_bytes < need)
     return fail(SSM_EWORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes, need);
   if (reinterpret_cast<uintptr_t>(workspace) & 255)
@@ -568,7 +588,7 @@ int ssm_scan_bwd_ex(const void* u, const void* delta, const float* A, const void
   const int rc = scan_bwd_core(u, delta, Af, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL,
                                ckpt, du, ddelta, dA ? dAf : nullptr, dB, dC, dD, dz, ddt_bias,
                                dh0, w + 2 * head, workspace_bytes - 2 * head, batch, dim, seqlen,
-                               dstate, io_dtype, stream, reverse, zoh);
+                               dstate, io_dtype, stream, reverse, zoh, bc_groups);
   if (rc != SSM_OK) return rc;
   if (dA) {
     reduce_da_kernel<<<(unsigned)((dim + 255) / 256), 256, 0, s>>>(dAf, dA, dim, dstate);
@@ -579,7 +599,7 @@ int ssm_scan_bwd_ex(const void* u, const void* delta, const float* A, const void
 
 size_t ssm_scan_bwd_scalar_a_workspace_size(int batch, int dim, int seqlen, int dstate,
                                             int io_dtype, int have_ckpt) {
-  return ssm_scan_bwd_ex_workspace_size(batch, dim, seqlen, dstate, io_dtype, have_ckpt,
+  return ssm_scan_bwd_ex_workspace_size(batch, dim, seqlen, dstate, 1, io_dtype, have_ckpt,
                                         SSM_SCALAR_A);
 }
 
@@ -592,7 +612,7 @@ int ssm_scan_bwd_scalar_a(const void* u, const void* delta, const float* A, cons
                           int io_dtype, void* stream) {
   return ssm_scan_bwd_ex(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL, ckpt,
                          du, ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, workspace, workspace_bytes,
-                         batch, dim, seqlen, dstate, io_dtype, SSM_SCALAR_A, stream);
+                         batch, dim, seqlen, dstate, 1, io_dtype, SSM_SCALAR_A, stream);
 }
 
 int ssm_state_update(float* state, const void* x, const void* dt, const float* A, const void* B,

@@ -316,7 +316,8 @@ __global__ void __launch_bounds__(128) bwd_kernel(const BwdArgs a) {
   const IO* zp = a.z ? reinterpret_cast<const IO*>(a.z) + row : nullptr;
   const IO* gp = reinterpret_cast<const IO*>(a.dout) + row;
   const bool bc_live = slot < N;  // the lane also stages B/C row `slot`, steps [8 q, 8 q + 8)
-  const long long bcrow = ((long long)b * N + (bc_live ? slot : 0)) * L;
+  const int gbc = ((grp * a.wpb + wib) * kCW) / (a.dim / a.bc_groups);  // the warp's B/C group
+  const long long bcrow = (((long long)b * a.bc_groups + gbc) * N + (bc_live ? slot : 0)) * L;
   const IO* Bp = reinterpret_cast<const IO*>(a.B) + bcrow;
   const IO* Cp = reinterpret_cast<const IO*>(a.C) + bcrow;
   float* sBw = reinterpret_cast<float*>(tl.sB);
@@ -480,10 +481,11 @@ __global__ void __launch_bounds__(128) bwd_kernel(const BwdArgs a) {
   }
 }
 
-// dB, dC: sum the CTA partials over groups in a fixed order; dA, dD, ddt_bias: sum over batch.
+// dB, dC: sum the partials of the CTAs of one B/C group in a fixed order; dA, dD, ddt_bias: sum
+// over batch.
 template <typename IO>
 __global__ void bwd_finish_bc(const BwdArgs a, IO* dB, IO* dC) {
-  const long long total = (long long)a.batch * 2 * a.N * a.L;
+  const long long total = (long long)a.batch * a.bc_groups * 2 * a.N * a.L;
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= total) return;
   const int t = (int)(i % a.L);
@@ -491,13 +493,16 @@ __global__ void bwd_finish_bc(const BwdArgs a, IO* dB, IO* dC) {
   const int n = (int)(r % a.N);
   r /= a.N;
   const int which = (int)(r % 2);
-  const int b = (int)(r / 2);
+  r /= 2;
+  const int gb = (int)(r % a.bc_groups);
+  const int b = (int)(r / a.bc_groups);
+  const int per = a.ngroups / a.bc_groups;  // CTAs per B/C group (whole groups of channels)
   float s = 0.f;
-  for (int g = 0; g < a.ngroups; ++g)
+  for (int g = gb * per; g < (gb + 1) * per; ++g)
     s += a.part_bc[(((long long)(g * a.batch + b) * 2 + which) * kNS + n) * a.L + t];
   IO* dst = which == 0 ? dB : dC;
   if (!dst) return;
-  const long long o = ((long long)b * a.N + n) * a.L + (a.reverse ? a.L - 1 - t : t);
+  const long long o = (((long long)b * a.bc_groups + gb) * a.N + n) * a.L + (a.reverse ? a.L - 1 - t : t);
   if (sizeof(IO) == 2) reinterpret_cast<uint16_t*>(dst)[o] = f32_to_bf16(s);
   else reinterpret_cast<float*>(dst)[o] = s;
 }
@@ -542,7 +547,7 @@ cudaError_t launch_bwd(const BwdArgs& a, int io, bool vec, cudaStream_t s) {
 cudaError_t launch_bwd_finish(const BwdArgs& a, int io, void* dB, void* dC, float* dA, float* dD,
                               float* ddt_bias, cudaStream_t s) {
   const int tpb = 256;
-  const long long nbc = (long long)a.batch * 2 * a.N * a.L;
+  const long long nbc = (long long)a.batch * a.bc_groups * 2 * a.N * a.L;
   if (io == 1)
     bwd_finish_bc<uint16_t><<<(unsigned)((nbc + tpb - 1) / tpb), tpb, 0, s>>>(
         a, reinterpret_cast<uint16_t*>(dB), reinterpret_cast<uint16_t*>(dC));

@@ -401,8 +401,9 @@ __device__ __forceinline__ void run_chunk(const FwdArgs& a, WarpTile<LPC>& tile,
                                           float2 (&hh)[Layout<LPC>::kPPL],
                                           const float2 (&al)[Layout<LPC>::kPPL],
                                           const float2 (&ra)[Layout<LPC>::kPPL], float Dd,
-                                          float bias, int lane, int slot, int q, int b, bool act,
-                                          long long ch, int t_begin, int t_end, bool last_chunk) {
+                                          float bias, int lane, int slot, int q, int b, int gbc,
+                                          bool act, long long ch, int t_begin, int t_end,
+                                          bool last_chunk) {
   using Lay = Layout<LPC>;
   using Lane = ChunkLane<IO, VEC, MODE, LPC, (KE < 0 ? KE : 0), REV>;
   // exponentials of a block that failed the range vote
@@ -422,7 +423,8 @@ __device__ __forceinline__ void run_chunk(const FwdArgs& a, WarpTile<LPC>& tile,
   ln.bn = lane >> 1;
   ln.bh = lane & 1;
   ln.bc_live = ln.bn < N;
-  const long long bcrow = ((long long)b * N + (ln.bc_live ? ln.bn : 0)) * L;
+  // the warp's B/C group: gbc of bc_groups for this batch row
+  const long long bcrow = (((long long)b * a.bc_groups + gbc) * N + (ln.bc_live ? ln.bn : 0)) * L;
   ln.Bp = reinterpret_cast<const IO*>(a.B) + bcrow;
   ln.Cp = reinterpret_cast<const IO*>(a.C) + bcrow;
   ln.slot = slot;
@@ -586,7 +588,9 @@ __global__ void __launch_bounds__(128) fwd_kernel(const FwdArgs a) {
   if (w >= a.nwarps) return;  // whole warp leaves together
   const int slot = lane / LPC, q = lane % LPC;
   const int b = (int)(w / a.warps_per_b);
-  const int d = (int)(w % a.warps_per_b) * Lay::kChW + slot;
+  const int d0 = (int)(w % a.warps_per_b) * Lay::kChW;  // the warp's first channel
+  const int d = d0 + slot;
+  const int gbc = d0 / (a.dim / a.bc_groups);         // all channels of a warp share B/C
   const bool act = d < a.dim;
   const int dd = act ? d : a.dim - 1;  // idle lanes shadow a valid channel and store nothing
   const long long ch = (long long)b * a.dim + dd;
@@ -628,8 +632,8 @@ __global__ void __launch_bounds__(128) fwd_kernel(const FwdArgs a) {
   const float bias = a.dt_bias ? a.dt_bias[dd] : 0.f;
   WarpTile<LPC>& tile = tiles[wib];
 
-  run_chunk<IO, VEC, MODE, LPC, KE, KO, REV>(a, tile, hh, al, ra, Dd, bias, lane, slot, q, b, act,
-                                             ch, t_begin, t_end, last_chunk);
+  run_chunk<IO, VEC, MODE, LPC, KE, KO, REV>(a, tile, hh, al, ra, Dd, bias, lane, slot, q, b, gbc,
+                                             act, ch, t_begin, t_end, last_chunk);
 }
 
 template <typename IO, bool VEC, int MODE, int LPC, int KE, int KO, bool REV>

@@ -45,6 +45,7 @@ struct FwdArgs {
   int scalar_a;         // one decay rate A_d per channel, shared by its N states
   int reverse;          // scan runs from t = L-1 down to 0 (time rows read/written mirrored)
   int zoh;              // zero-order-hold input term (e^{ΔA} - 1)/A B x instead of Δ B x
+  int bc_groups;        // B, C are [batch][bc_groups][N][L]; channel d uses group d / (dim / bc_groups)
   int lpc;              // lanes per channel: 1, 2 or 4 (16 / lpc states each)
   int warps_per_b;      // ceil(dim / (32 / lpc))
   long long nwarps;     // batch * warps_per_b
@@ -77,6 +78,7 @@ struct BwdArgs {
   int kmufu;            // state pairs (of 4 per lane) whose exponential runs on MUFU: 2, 3 or 4
   int reverse;          // gradients of the reverse scan (time rows read/written mirrored)
   int zoh;              // gradients of the zero-order-hold input term
+  int bc_groups;        // B, C (and dB, dC) are [batch][bc_groups][N][L]
 };
 
 struct DecodeArgs {

@@ -10,6 +10,8 @@ Every test builds its expected value independently (a different formula or libra
   * chunked-vs-sequential state passing, superposition, decode-vs-scan;
   * the scalar decay (one A per channel, the Mamba-2 restriction in the reading-list notes) as
     a masked Gram-matrix product, and its rate gradient by central differences;
+  * grouped B/C (one B_t, C_t per group of channels) against the quadratic form of each group,
+    and its gradients by central differences;
   * the reverse scan (Hydra notes: the anti-causal half of a bidirectional layer) against the
     anti-causal quadratic form, a two-step closed form of its final state, and central
     differences of its gradients;
@@ -388,6 +390,48 @@ def test_reverse_gradients_by_finite_differences():
             xp = x.copy(); xp[i] += eps
             xm = x.copy(); xm[i] -= eps
             num[i] = (loss(dict(c, **{key: xp})) - loss(dict(c, **{key: xm}))) / (2 * eps)
+        np.testing.assert_allclose(g[gname], num, rtol=2e-6, atol=2e-7, err_msg=gname)
+
+
+# ------------------------------------------------------------------ grouped B/C
+def test_grouped_bc_quadratic_form():
+    """B, C of shape [batch, G, N, L]: channel d reads group d // (dim // G); each group against
+    the brute-force quadratic form of its own channels."""
+    c = rand_case(batch=2, dim=6, L=7, N=3, seed=81)
+    r = np.random.default_rng(82)
+    Bg = r.standard_normal((2, 3, 3, 7))
+    Cg = r.standard_normal((2, 3, 3, 7))
+    got = oracle.scan_fwd(c["u"], c["delta"], c["A"], Bg, Cg, D=c["D"], z=c["z"],
+                          dt_bias=c["dt_bias"], h0=c["h0"])["out"]
+    for g in range(3):
+        sl = slice(2 * g, 2 * g + 2)
+        cg = dict(c, u=c["u"][:, sl], delta=c["delta"][:, sl], A=c["A"][sl], D=c["D"][sl],
+                  z=c["z"][:, sl], dt_bias=c["dt_bias"][sl], h0=c["h0"][:, sl],
+                  B=Bg[:, g], C=Cg[:, g])
+        np.testing.assert_allclose(got[:, sl], quadratic_form(cg), rtol=1e-11, atol=1e-12)
+
+
+def test_grouped_bc_gradients_by_finite_differences():
+    c = rand_case(batch=1, dim=4, L=5, N=2, seed=83)
+    r = np.random.default_rng(84)
+    c["B"] = r.standard_normal((1, 2, 2, 5))
+    c["C"] = r.standard_normal((1, 2, 2, 5))
+    dout = r.standard_normal(c["u"].shape)
+    dhL = r.standard_normal(c["h0"].shape)
+    g = oracle.scan_bwd(c["u"], c["delta"], c["A"], c["B"], c["C"], dout, D=c["D"], z=c["z"],
+                        dt_bias=c["dt_bias"], h0=c["h0"], dhL=dhL)
+    assert g["dB"].shape == (1, 2, 2, 5)
+    eps = 1e-6
+    for key, gname in (("B", "dB"), ("C", "dC"), ("u", "du"), ("A", "dA"), ("h0", "dh0")):
+        x = c[key]
+        num = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            i = it.multi_index
+            xp = x.copy(); xp[i] += eps
+            xm = x.copy(); xm[i] -= eps
+            num[i] = (loss_and_grads(dict(c, **{key: xp}), dout, dhL)
+                      - loss_and_grads(dict(c, **{key: xm}), dout, dhL)) / (2 * eps)
         np.testing.assert_allclose(g[gname], num, rtol=2e-6, atol=2e-7, err_msg=gname)
 
 
