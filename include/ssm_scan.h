@@ -256,6 +256,19 @@ SSM_API int ssm_state_update(float* state, const void* x, const void* dt, const 
                      int delta_softplus, void* out, int batch, int dim, int dstate,
                      int io_dtype, void* stream);
 
+/*
+ * ssm_state_update with the variants of the scan: flags SSM_SCALAR_A (A is [dim]) and SSM_ZOH
+ * (the zero-order-hold input coefficient); B, C are [batch][bc_groups][dstate] (channel d uses
+ * group d / (dim / bc_groups); dim / bc_groups a multiple of 16 when bc_groups > 1).  A decode
+ * step runs forward in time: SSM_REVERSE is rejected with SSM_EINVAL, as is any unknown bit.
+ * Calling it L times reproduces ssm_scan_fwd_ex with the same flags and groups.
+ */
+SSM_API int ssm_state_update_ex(float* state, const void* x, const void* dt, const float* A,
+                                const void* B, const void* C, const float* D, const void* z,
+                                const float* dt_bias, int delta_softplus, void* out, int batch,
+                                int dim, int dstate, int bc_groups, int io_dtype, int flags,
+                                void* stream);
+
 #ifdef __cplusplus
 }
 #endif

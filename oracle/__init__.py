@@ -231,13 +231,29 @@ def scan_bwd(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None, delta_softpl
 
 
 def state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=True,
-                 nthreads=0):
+                 nthreads=0, zoh=False):
     """One decode step.  ``state`` [batch, dim, N] float64 is updated IN PLACE (it must be a
-    C-contiguous float64 array).  x, dt, z: [batch, dim]; B, C: [batch, N].  Returns out."""
+    C-contiguous float64 array).  x, dt, z: [batch, dim]; B, C: [batch, N], or [batch, G, N]
+    (grouped: each group of dim/G channels is an independent step with its own B, C).
+    ``zoh``: zero-order-hold input coefficient.  Returns out."""
     if not (isinstance(state, np.ndarray) and state.dtype == np.float64
             and state.flags["C_CONTIGUOUS"]):
         raise TypeError("state must be a C-contiguous float64 numpy array (updated in place)")
     batch, dim, N = state.shape
+    if np.ndim(B) == 3:
+        G = np.shape(B)[1]
+        per = dim // G
+        out = np.zeros((batch, dim))
+        for g in range(G):
+            sl = slice(g * per, (g + 1) * per)
+            st = np.ascontiguousarray(state[:, sl])
+            cut = lambda v, ax: None if v is None else (np.asarray(v)[:, sl] if ax else np.asarray(v)[sl])
+            out[:, sl] = state_update(st, cut(x, 1), cut(dt, 1), np.asarray(A)[sl],
+                                      np.asarray(B)[:, g], np.asarray(C)[:, g], D=cut(D, 0),
+                                      z=cut(z, 1), dt_bias=cut(dt_bias, 0),
+                                      delta_softplus=delta_softplus, nthreads=nthreads, zoh=zoh)
+            state[:, sl] = st
+        return out
     x = _arr(x, (batch, dim))
     dt = _arr(dt, (batch, dim))
     A = _arr(A, (dim, N))
@@ -249,7 +265,7 @@ def state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, delta_soft
     out = np.zeros((batch, dim))
     rc = _lib().oracle_state_update(
         batch, dim, N, _p(state), _p(x), _p(dt), _p(A), _p(B), _p(C), _p(D), _p(z),
-        _p(dt_bias), int(bool(delta_softplus)), _p(out), int(nthreads))
+        _p(dt_bias), int(bool(delta_softplus)), int(bool(zoh)), _p(out), int(nthreads))
     if rc != 0:
         raise RuntimeError(f"oracle_state_update failed ({rc})")
     return out

@@ -306,7 +306,7 @@ int oracle_scan_bwd(int batch, int dim, int seqlen, int dstate,
 int oracle_state_update(int batch, int dim, int dstate, double* state,
                         const double* x, const double* dt_raw, const double* A,
                         const double* B, const double* C, const double* Dskip,
-                        const double* z, const double* dt_bias, int delta_softplus,
+                        const double* z, const double* dt_bias, int delta_softplus, int zoh,
                         double* out, int nthreads) {
   if (!state || !x || !dt_raw || !A || !B || !C || !out) return -1;
   const int64_t nall = (int64_t)batch * dim;
@@ -318,7 +318,8 @@ int oracle_state_update(int batch, int dim, int dstate, double* state,
     double y = 0.0;
     for (int n = 0; n < dstate; ++n) {
       double* h = state + ch * dstate + n;
-      *h = exp(dt * A[(int64_t)d * dstate + n]) * (*h) + dt * B[(int64_t)b * dstate + n] * x[ch];
+      const double a_dn = A[(int64_t)d * dstate + n];
+      *h = exp(dt * a_dn) * (*h) + input_coef(dt, a_dn, zoh) * B[(int64_t)b * dstate + n] * x[ch];
       y += C[(int64_t)b * dstate + n] * (*h);
     }
     y += (Dskip ? Dskip[d] : 0.0) * x[ch];

@@ -225,27 +225,34 @@ def ssm_scan_bwd_scalar_a(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None,
 
 
 def ssm_state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=True,
-                     out=None):
+                     out=None, scalar_a=False, zoh=False):
     """One decode step; ``state`` [batch, dim, N] f32 is updated in place.  x, dt, z:
-    [batch, dim]; B, C: [batch, N] (io dtype).  Returns out [batch, dim]."""
+    [batch, dim]; B, C: [batch, N] or, grouped, [batch, G, N] (io dtype); A: [dim, N] f32, or
+    [dim] with ``scalar_a``; ``zoh``: zero-order-hold input coefficient.  Returns out [batch, dim]."""
     dev = state.device
     batch, dim, N = state.shape
     io = x.dtype
     code = _io_code(io)
+    if not isinstance(B, torch.Tensor):
+        raise TypeError("B must be a torch.Tensor")
+    G = B.shape[1] if B.dim() == 3 else 1
+    bc_shape = (batch, G, N) if B.dim() == 3 else (batch, N)
     _need(state, "state", (batch, dim, N), torch.float32, dev)
     _need(x, "x", (batch, dim), io, dev)
     _need(dt, "dt", (batch, dim), io, dev)
-    _need(A, "A", (dim, N), torch.float32, dev)
-    _need(B, "B", (batch, N), io, dev)
-    _need(C, "C", (batch, N), io, dev)
+    _need(A, "A", (dim,) if scalar_a else (dim, N), torch.float32, dev)
+    _need(B, "B", bc_shape, io, dev)
+    _need(C, "C", bc_shape, io, dev)
     _opt(D, "D", (dim,), torch.float32, dev)
     _opt(z, "z", (batch, dim), io, dev)
     _opt(dt_bias, "dt_bias", (dim,), torch.float32, dev)
     if out is None:
         out = torch.empty((batch, dim), dtype=io, device=dev)
     _need(out, "out", (batch, dim), io, dev)
-    rc = _abi.lib().ssm_state_update(
+    flags = _flags(scalar_a, False, zoh)
+    rc = _abi.lib().ssm_state_update_ex(
         _ptr(state), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
-        _ptr(dt_bias), int(bool(delta_softplus)), _ptr(out), batch, dim, N, code, _stream(dev))
-    _abi.check(rc, "ssm_state_update")
+        _ptr(dt_bias), int(bool(delta_softplus)), _ptr(out), batch, dim, N, G, code, flags,
+        _stream(dev))
+    _abi.check(rc, "ssm_state_update_ex")
     return out

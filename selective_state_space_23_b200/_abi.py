@@ -49,6 +49,8 @@ SIGNATURES = {
                                   _i, _i, _i, _i, _i, _vp]),
     "ssm_state_update": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp,
                               _i, _i, _i, _i, _vp]),
+    "ssm_state_update_ex": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp,
+                                 _i, _i, _i, _i, _i, _i, _vp]),
 }
 
 _lib = None

@@ -615,20 +615,25 @@ int ssm_scan_bwd_scalar_a(const void* u, const void* delta, const float* A, cons
                          batch, dim, seqlen, dstate, 1, io_dtype, SSM_SCALAR_A, stream);
 }
 
-int ssm_state_update(float* state, const void* x, const void* dt, const float* A, const void* B,
-                     const void* C, const float* D, const void* z, const float* dt_bias,
-                     int delta_softplus, void* out, int batch, int dim, int dstate,
-                     int io_dtype, void* stream) {
+int ssm_state_update_ex(float* state, const void* x, const void* dt, const float* A,
+                        const void* B, const void* C, const float* D, const void* z,
+                        const float* dt_bias, int delta_softplus, void* out, int batch, int dim,
+                        int dstate, int bc_groups, int io_dtype, int flags, void* stream) {
   g_err[0] = 0;
+  if (flags & ~(SSM_SCALAR_A | SSM_ZOH))
+    return fail(SSM_EINVAL, "unsupported flags 0x%x for a decode step", flags);
   TRY(check_dims(batch, dim, 1, dstate, io_dtype));
+  TRY(check_groups(dim, bc_groups));
+  const bool scalar_a = (flags & SSM_SCALAR_A) != 0;
   const size_t es = esize(io_dtype);
   const size_t nx = (size_t)batch * dim * es;
+  const size_t nbc = (size_t)batch * bc_groups * dstate * es;
   TRY(check_ptr(state, (size_t)batch * dim * dstate * 4, 4, "state"));
   TRY(check_ptr(x, nx, es, "x"));
   TRY(check_ptr(dt, nx, es, "dt"));
-  TRY(check_ptr(A, (size_t)dim * dstate * 4, 4, "A"));
-  TRY(check_ptr(B, (size_t)batch * dstate * es, es, "B"));
-  TRY(check_ptr(C, (size_t)batch * dstate * es, es, "C"));
+  TRY(check_ptr(A, (size_t)dim * (scalar_a ? 1 : dstate) * 4, 4, "A"));
+  TRY(check_ptr(B, nbc, es, "B"));
+  TRY(check_ptr(C, nbc, es, "C"));
   TRY(check_ptr(out, nx, es, "out"));
   TRY(check_opt(D, (size_t)dim * 4, 4, "D"));
   TRY(check_opt(z, nx, es, "z"));
@@ -637,9 +642,20 @@ int ssm_state_update(float* state, const void* x, const void* dt, const float* A
   a.state = state; a.x = x; a.dt = dt; a.z = z; a.B = B; a.C = C; a.A = A; a.D = D;
   a.dt_bias = dt_bias; a.out = out;
   a.batch = batch; a.dim = dim; a.N = dstate; a.softplus = delta_softplus ? 1 : 0;
+  a.scalar_a = scalar_a ? 1 : 0;
+  a.zoh = (flags & SSM_ZOH) ? 1 : 0;
+  a.bc_groups = bc_groups;
   cudaError_t e = ssm::launch_decode(a, io_dtype, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode step");
   return SSM_OK;
+}
+
+int ssm_state_update(float* state, const void* x, const void* dt, const float* A, const void* B,
+                     const void* C, const float* D, const void* z, const float* dt_bias,
+                     int delta_softplus, void* out, int batch, int dim, int dstate,
+                     int io_dtype, void* stream) {
+  return ssm_state_update_ex(state, x, dt, A, B, C, D, z, dt_bias, delta_softplus, out, batch,
+                             dim, dstate, 1, io_dtype, 0, stream);
 }
 
 }  // extern "C"

@@ -7,6 +7,10 @@
 //   Δ = softplus(dt + dt_bias_d);  h_n <- exp(Δ A_dn) h_n + Δ B_n x   (in place)
 //   out = (Σ_n C_n h_n + D_d x) * silu(z)
 //
+// Variants (the same recurrence as the scan's): one decay rate A_d per channel (A is [dim]); the
+// zero-order-hold input coefficient c = (e^{ΔA} - 1)/A (library expm1f: the step is memory-bound,
+// so the accurate form costs nothing); B, C per group of channels ([batch][groups][N]).
+//
 // The step is bound by HBM traffic on the f32 state (read + write of batch*D*N*4 bytes).  For
 // N = 16 two lanes share a channel, each holding 8 consecutive states as two 128-bit accesses
 // (a warp streams 1 KB of contiguous state per access pair); the two partial readouts are
@@ -34,6 +38,12 @@ template <> __device__ __forceinline__ void st_io<uint16_t>(void* p, long long i
   reinterpret_cast<uint16_t*>(p)[i] = f32_to_bf16(v);
 }
 
+// Input coefficient of B x: Δ, or with the ZOH term (e^{ΔA} - 1)/A (Δ as A -> 0).
+__device__ __forceinline__ float decode_coef(float dt, float An, bool zoh) {
+  if (!zoh) return dt;
+  return fabsf(An) < 1e-20f ? dt : expm1f(dt * An) / An;
+}
+
 // VEC: N == 16 and the state is 16-byte aligned (one float4 per lane).
 template <typename IO, bool VEC>
 __global__ void __launch_bounds__(256) decode_kernel(const DecodeArgs a) {
@@ -53,6 +63,7 @@ __global__ void __launch_bounds__(256) decode_kernel(const DecodeArgs a) {
 
   float h[4], An[4], Bn[4], Cn[4];
   float* sp = a.state + ch * N + 4 * q;
+  const long long bc = ((long long)b * a.bc_groups + d / (a.dim / a.bc_groups)) * N;
   if (VEC) {
     const float4 h4 = *reinterpret_cast<const float4*>(sp);
     h[0] = h4.x; h[1] = h4.y; h[2] = h4.z; h[3] = h4.w;
@@ -62,15 +73,16 @@ __global__ void __launch_bounds__(256) decode_kernel(const DecodeArgs a) {
     const int n = 4 * q + i;
     const bool live = n < N;
     if (!VEC) h[i] = live ? sp[i] : 0.f;
-    An[i] = live ? a.A[(long long)d * N + n] : 0.f;
-    Bn[i] = live ? ld_io<IO>(a.B, (long long)b * N + n) : 0.f;
-    Cn[i] = live ? ld_io<IO>(a.C, (long long)b * N + n) : 0.f;
+    An[i] = live ? a.A[a.scalar_a ? (long long)d : (long long)d * N + n] : 0.f;
+    Bn[i] = live ? ld_io<IO>(a.B, bc + n) : 0.f;
+    Cn[i] = live ? ld_io<IO>(a.C, bc + n) : 0.f;
   }
   float y = 0.f;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const float abar = kPrecise ? expf(dt * An[i]) : ex2_mufu(dt * An[i] * kLog2e);
-    h[i] = fmaf(abar, h[i], dx * Bn[i]);
+    const float abar = (kPrecise || a.zoh) ? expf(dt * An[i]) : ex2_mufu(dt * An[i] * kLog2e);
+    const float bx = a.zoh ? decode_coef(dt, An[i], true) * xv : dx;
+    h[i] = fmaf(abar, h[i], bx * Bn[i]);
     y = fmaf(Cn[i], h[i], y);
   }
   y += __shfl_xor_sync(0xffffffffu, y, 1);
@@ -113,14 +125,24 @@ __global__ void __launch_bounds__(256) decode16_kernel(const DecodeArgs a) {
   float* sp = a.state + ch * kNS + 8 * q;
   const float4 h0 = reinterpret_cast<const float4*>(sp)[0];  // default caching: the state is
   const float4 h1 = reinterpret_cast<const float4*>(sp)[1];  // reused by the next step
-  const float4* ap = reinterpret_cast<const float4*>(a.A + (long long)d * kNS + 8 * q);
-  const float4 a0 = __ldg(ap), a1 = __ldg(ap + 1);
   float h[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-  const float An[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+  float An[8];
+  if (a.scalar_a) {
+    const float ad = __ldg(a.A + d);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) An[i] = ad;
+  } else {
+    const float4* ap = reinterpret_cast<const float4*>(a.A + (long long)d * kNS + 8 * q);
+    const float4 a0 = __ldg(ap), a1 = __ldg(ap + 1);
+    const float at[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) An[i] = at[i];
+  }
+  const long long bc = ((long long)b * a.bc_groups + d / (a.dim / a.bc_groups)) * kNS + 8 * q;
   float Bn[8], Cn[8];
   if (sizeof(IO) == 2) {
-    const uint4 bw = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.B) + (long long)b * kNS + 8 * q));
-    const uint4 cw = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.C) + (long long)b * kNS + 8 * q));
+    const uint4 bw = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.B) + bc));
+    const uint4 cw = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.C) + bc));
     const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w}, cc[4] = {cw.x, cw.y, cw.z, cw.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -128,8 +150,8 @@ __global__ void __launch_bounds__(256) decode16_kernel(const DecodeArgs a) {
       Cn[2 * i] = bf16_lo(cc[i]); Cn[2 * i + 1] = bf16_hi(cc[i]);
     }
   } else {
-    const float4* bp = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.B) + (long long)b * kNS + 8 * q);
-    const float4* cp = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.C) + (long long)b * kNS + 8 * q);
+    const float4* bp = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.B) + bc);
+    const float4* cp = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.C) + bc);
     const float4 b0 = __ldg(bp), b1 = __ldg(bp + 1), c0 = __ldg(cp), c1 = __ldg(cp + 1);
     const float bt[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
     const float ct[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
@@ -139,8 +161,9 @@ __global__ void __launch_bounds__(256) decode16_kernel(const DecodeArgs a) {
   float y = 0.f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float abar = kPrecise ? expf(dt * An[i]) : ex2_mufu(dt * An[i] * kLog2e);
-    h[i] = fmaf(abar, h[i], dx * Bn[i]);
+    const float abar = (kPrecise || a.zoh) ? expf(dt * An[i]) : ex2_mufu(dt * An[i] * kLog2e);
+    const float bx = a.zoh ? decode_coef(dt, An[i], true) * xv : dx;
+    h[i] = fmaf(abar, h[i], bx * Bn[i]);
     y = fmaf(Cn[i], h[i], y);
   }
   y += __shfl_xor_sync(0xffffffffu, y, 1);
@@ -161,7 +184,7 @@ template <typename IO>
 cudaError_t launch_io(const DecodeArgs& a, cudaStream_t s) {
   const int tpb = 256;
   const auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
-  if (a.N == kNS && al16(a.state) && al16(a.A) && al16(a.B) && al16(a.C)) {
+  if (a.N == kNS && al16(a.state) && (a.scalar_a || al16(a.A)) && al16(a.B) && al16(a.C)) {
     const long long threads = (long long)a.batch * a.dim * 2;
     decode16_kernel<IO><<<(unsigned)((threads + tpb - 1) / tpb), tpb, 0, s>>>(a);
   } else {

@@ -94,6 +94,9 @@ struct DecodeArgs {
   void* out;
   int batch, dim, N;
   int softplus;
+  int scalar_a;   // A is [dim]: one decay rate per channel
+  int zoh;        // zero-order-hold input coefficient (e^{ΔA} - 1)/A instead of Δ
+  int bc_groups;  // B, C are [batch][bc_groups][N]; channel d uses group d / (dim / bc_groups)
 };
 
 // io: 0 = f32, 1 = bf16.  vec: rows are 16-byte aligned and L is a multiple of the vector width.

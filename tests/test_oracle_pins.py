@@ -210,6 +210,27 @@ def test_decode_steps_equal_scan():
     np.testing.assert_allclose(state, full["hL"], rtol=1e-13, atol=1e-14)
 
 
+@pytest.mark.parametrize("zoh,groups", [(True, 1), (False, 2), (True, 2)])
+def test_decode_steps_equal_scan_variants(zoh, groups):
+    """The decode step with the ZOH coefficient and with grouped B/C reproduces the scan (whose
+    ZOH form is pinned by the gating case and finite differences, and grouped form by the
+    per-group quadratic form)."""
+    c = rand_case(batch=2, dim=4, L=9, N=3, seed=25)
+    c["A"][1, 2] = 0.0  # the A -> 0 limit of the ZOH coefficient
+    if groups > 1:
+        r = np.random.default_rng(26)
+        c["B"] = r.standard_normal((2, groups, 3, 9))
+        c["C"] = r.standard_normal((2, groups, 3, 9))
+    full = run(c, zoh=zoh)
+    state = np.ascontiguousarray(c["h0"].copy())
+    for t in range(9):
+        o = oracle.state_update(state, c["u"][..., t], c["delta"][..., t], c["A"], c["B"][..., t],
+                                c["C"][..., t], D=c["D"], z=c["z"][..., t], dt_bias=c["dt_bias"],
+                                zoh=zoh)
+        np.testing.assert_allclose(o, full["out"][..., t], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(state, full["hL"], rtol=1e-12, atol=1e-13)
+
+
 def test_channel_subset_matches_full():
     c = rand_case(batch=2, dim=5, L=10, N=3, seed=23)
     full = run(c)
