@@ -189,6 +189,10 @@ SSM_API int ssm_scan_bwd_scalar_a(const void* u, const void* delta, const float*
  *                 B̄ = (ΔA)^{-1}(exp(ΔA) - I) ΔB): h_t = Ā h_{t-1} + c B_t x_t with
  *                 c = (exp(Δ_t A) - 1)/A per state (c -> Δ_t as A -> 0) instead of Δ_t.
  *                 Combines with the other flags.
+ *   SSM_CHANNELS_LAST  the (B, L, D) layout: u, delta, z, out, dout, du, ddelta, dz are
+ *                 [batch][L][dim] and B, C, dB, dC are [batch][L][bc_groups][dstate] (the
+ *                 projections' own output layout), read and written with element accesses;
+ *                 everything else as above.
  * Any other bit is rejected with SSM_EINVAL.  Arguments are those of ssm_scan_fwd /
  * ssm_scan_bwd plus flags and bc_groups:
  *   bc_groups     B, C (and dB, dC) are [batch][bc_groups][dstate][L]: the per-token B_t, C_t
@@ -201,6 +205,7 @@ SSM_API int ssm_scan_bwd_scalar_a(const void* u, const void* delta, const float*
 #define SSM_SCALAR_A 1
 #define SSM_REVERSE 2
 #define SSM_ZOH 4
+#define SSM_CHANNELS_LAST 8
 SSM_API size_t ssm_scan_fwd_ex_workspace_size(int batch, int dim, int seqlen, int dstate,
                                               int bc_groups, int io_dtype, int flags);
 SSM_API int ssm_scan_fwd_ex(const void* u, const void* delta, const float* A, const void* B,

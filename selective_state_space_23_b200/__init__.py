@@ -82,10 +82,17 @@ def _workspace(nbytes, device, given):
     return torch.empty(nbytes, dtype=torch.uint8, device=device)
 
 
-def _bc_layout(B, batch, L):
-    """(groups, N, shape) of the B/C layout: [batch, N, L] (one group) or [batch, G, N, L]."""
+def _bc_layout(B, batch, L, channels_last=False):
+    """(groups, N, shape) of the B/C layout: [batch, N, L] (one group) or [batch, G, N, L];
+    channels last: [batch, L, N] or [batch, L, G, N]."""
     if not isinstance(B, torch.Tensor):
         raise TypeError("B must be a torch.Tensor")
+    if channels_last:
+        if B.dim() == 3:
+            return 1, B.shape[2], (batch, L, B.shape[2])
+        if B.dim() == 4:
+            return B.shape[2], B.shape[3], (batch, L, B.shape[2], B.shape[3])
+        raise ValueError(f"B must be [batch, L, N] or [batch, L, groups, N], got {tuple(B.shape)}")
     if B.dim() == 3:
         return 1, B.shape[1], (batch, B.shape[1], L)
     if B.dim() == 4:
@@ -93,34 +100,38 @@ def _bc_layout(B, batch, L):
     raise ValueError(f"B must be [batch, N, L] or [batch, groups, N, L], got {tuple(B.shape)}")
 
 
-def _flags(scalar_a, reverse, zoh):
+def _flags(scalar_a, reverse, zoh, channels_last=False):
     return ((_abi.SSM_SCALAR_A if scalar_a else 0) | (_abi.SSM_REVERSE if reverse else 0)
-            | (_abi.SSM_ZOH if zoh else 0))
+            | (_abi.SSM_ZOH if zoh else 0) | (_abi.SSM_CHANNELS_LAST if channels_last else 0))
 
 
 def _scan_fwd(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, return_final_state,
-              return_ckpt, out, workspace, scalar_a, reverse, zoh):
+              return_ckpt, out, workspace, scalar_a, reverse, zoh, channels_last=False):
     dev = u.device
-    batch, dim, L = u.shape
-    G, N, bc_shape = _bc_layout(B, batch, L)
+    if channels_last:
+        batch, L, dim = u.shape
+    else:
+        batch, dim, L = u.shape
+    xs = (batch, L, dim) if channels_last else (batch, dim, L)
+    G, N, bc_shape = _bc_layout(B, batch, L, channels_last)
     io = u.dtype
     code = _io_code(io)
-    _need(u, "u", (batch, dim, L), io, dev)
-    _need(delta, "delta", (batch, dim, L), io, dev)
+    _need(u, "u", xs, io, dev)
+    _need(delta, "delta", xs, io, dev)
     _need(A, "A", (dim,) if scalar_a else (dim, N), torch.float32, dev)
     _need(B, "B", bc_shape, io, dev)
     _need(C, "C", bc_shape, io, dev)
     _opt(D, "D", (dim,), torch.float32, dev)
-    _opt(z, "z", (batch, dim, L), io, dev)
+    _opt(z, "z", xs, io, dev)
     _opt(dt_bias, "dt_bias", (dim,), torch.float32, dev)
     _opt(h0, "h0", (batch, dim, N), torch.float32, dev)
     if out is None:
-        out = torch.empty((batch, dim, L), dtype=io, device=dev)
-    _need(out, "out", (batch, dim, L), io, dev)
+        out = torch.empty(xs, dtype=io, device=dev)
+    _need(out, "out", xs, io, dev)
     hL = torch.empty((batch, dim, N), dtype=torch.float32, device=dev) if return_final_state else None
     nblk = (L + CKPT_STEPS - 1) // CKPT_STEPS
     ckpt = torch.empty((batch, dim, nblk, N), dtype=torch.float32, device=dev) if return_ckpt else None
-    flags = _flags(scalar_a, reverse, zoh)
+    flags = _flags(scalar_a, reverse, zoh, channels_last)
     nws = int(_abi.lib().ssm_scan_fwd_ex_workspace_size(batch, dim, L, N, G, code, flags))
     ws = _workspace(nws, dev, workspace)
     rc = _abi.lib().ssm_scan_fwd_ex(
@@ -140,39 +151,44 @@ def _scan_fwd(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, return_final
 
 def ssm_scan_fwd(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=True, h0=None,
                  return_final_state=False, return_ckpt=False, out=None, workspace=None,
-                 reverse=False, zoh=False):
+                 reverse=False, zoh=False, channels_last=False):
     """Forward scan.  u, delta, z: [batch, dim, L]; B, C: [batch, N, L] or, grouped, [batch, G,
     N, L] (channel d uses group d // (dim // G)) (io dtype f32 or bf16); A: [dim, N] f32; D, dt_bias: [dim] f32; h0: [batch, dim, N] f32.  reverse: scan from
     t = L-1 down to 0.  zoh: zero-order-hold input term (e^{ΔA} - 1)/A B x instead of Δ B x.
-    Returns out, or a tuple (out, hL?, ckpt?) when those are requested."""
+    channels_last: the (B, L, D) layout (u, delta, z, out [batch, L, dim]; B, C [batch, L, N]
+    or [batch, L, G, N]).  Returns out, or a tuple (out, hL?, ckpt?) when those are requested."""
     return _scan_fwd(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, return_final_state,
-                     return_ckpt, out, workspace, False, reverse, zoh)
+                     return_ckpt, out, workspace, False, reverse, zoh, channels_last)
 
 
 def ssm_scan_fwd_scalar_a(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=True,
                           h0=None, return_final_state=False, return_ckpt=False, out=None,
-                          workspace=None, reverse=False, zoh=False):
+                          workspace=None, reverse=False, zoh=False, channels_last=False):
     """Forward scan with one decay rate per channel: as :func:`ssm_scan_fwd` with A [dim] f32."""
     return _scan_fwd(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, return_final_state,
-                     return_ckpt, out, workspace, True, reverse, zoh)
+                     return_ckpt, out, workspace, True, reverse, zoh, channels_last)
 
 
 def _scan_bwd(u, delta, A, B, C, dout, D, z, dt_bias, delta_softplus, h0, dhL, ckpt,
-              workspace, need, scalar_a, reverse, zoh):
+              workspace, need, scalar_a, reverse, zoh, channels_last=False):
     dev = u.device
-    batch, dim, L = u.shape
-    G, N, bc_shape = _bc_layout(B, batch, L)
+    if channels_last:
+        batch, L, dim = u.shape
+    else:
+        batch, dim, L = u.shape
+    xs = (batch, L, dim) if channels_last else (batch, dim, L)
+    G, N, bc_shape = _bc_layout(B, batch, L, channels_last)
     io = u.dtype
     code = _io_code(io)
-    _need(u, "u", (batch, dim, L), io, dev)
-    _need(delta, "delta", (batch, dim, L), io, dev)
+    _need(u, "u", xs, io, dev)
+    _need(delta, "delta", xs, io, dev)
     a_shape = (dim,) if scalar_a else (dim, N)
     _need(A, "A", a_shape, torch.float32, dev)
     _need(B, "B", bc_shape, io, dev)
     _need(C, "C", bc_shape, io, dev)
-    _need(dout, "dout", (batch, dim, L), io, dev)
+    _need(dout, "dout", xs, io, dev)
     _opt(D, "D", (dim,), torch.float32, dev)
-    _opt(z, "z", (batch, dim, L), io, dev)
+    _opt(z, "z", xs, io, dev)
     _opt(dt_bias, "dt_bias", (dim,), torch.float32, dev)
     _opt(h0, "h0", (batch, dim, N), torch.float32, dev)
     _opt(dhL, "dhL", (batch, dim, N), torch.float32, dev)
@@ -182,9 +198,9 @@ def _scan_bwd(u, delta, A, B, C, dout, D, z, dt_bias, delta_softplus, h0, dhL, c
                                                 "ddt_bias", "dh0"}
     e = lambda shape, dt: torch.empty(shape, dtype=dt, device=dev)
     g = {
-        "du": e((batch, dim, L), io) if "du" in want else None,
-        "ddelta": e((batch, dim, L), io) if "ddelta" in want else None,
-        "dz": e((batch, dim, L), io) if ("dz" in want and z is not None) else None,
+        "du": e(xs, io) if "du" in want else None,
+        "ddelta": e(xs, io) if "ddelta" in want else None,
+        "dz": e(xs, io) if ("dz" in want and z is not None) else None,
         "dB": e(bc_shape, io) if "dB" in want else None,
         "dC": e(bc_shape, io) if "dC" in want else None,
         "dA": e(a_shape, torch.float32) if "dA" in want else None,
@@ -192,7 +208,7 @@ def _scan_bwd(u, delta, A, B, C, dout, D, z, dt_bias, delta_softplus, h0, dhL, c
         "ddt_bias": e((dim,), torch.float32) if "ddt_bias" in want else None,
         "dh0": e((batch, dim, N), torch.float32) if "dh0" in want else None,
     }
-    flags = _flags(scalar_a, reverse, zoh)
+    flags = _flags(scalar_a, reverse, zoh, channels_last)
     nws = int(_abi.lib().ssm_scan_bwd_ex_workspace_size(batch, dim, L, N, G, code,
                                                          int(ckpt is not None), flags))
     ws = _workspace(nws, dev, workspace)
@@ -209,19 +225,19 @@ def _scan_bwd(u, delta, A, B, C, dout, D, z, dt_bias, delta_softplus, h0, dhL, c
 
 def ssm_scan_bwd(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None, delta_softplus=True,
                  h0=None, dhL=None, ckpt=None, workspace=None, need=None, reverse=False,
-                 zoh=False):
+                 zoh=False, channels_last=False):
     """Gradients of :func:`ssm_scan_fwd`.  Returns a dict with du, ddelta, dA, dB, dC, dD, dz,
     ddt_bias, dh0 (entries are None when the matching input is absent or not in ``need``)."""
     return _scan_bwd(u, delta, A, B, C, dout, D, z, dt_bias, delta_softplus, h0, dhL, ckpt,
-                     workspace, need, False, reverse, zoh)
+                     workspace, need, False, reverse, zoh, channels_last)
 
 
 def ssm_scan_bwd_scalar_a(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None,
                           delta_softplus=True, h0=None, dhL=None, ckpt=None, workspace=None,
-                          need=None, reverse=False, zoh=False):
+                          need=None, reverse=False, zoh=False, channels_last=False):
     """Gradients of :func:`ssm_scan_fwd_scalar_a` (dA is [dim])."""
     return _scan_bwd(u, delta, A, B, C, dout, D, z, dt_bias, delta_softplus, h0, dhL, ckpt,
-                     workspace, need, True, reverse, zoh)
+                     workspace, need, True, reverse, zoh, channels_last)
 
 
 def ssm_state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=True,

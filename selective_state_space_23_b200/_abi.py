@@ -13,7 +13,7 @@ SSM_OK, SSM_EINVAL, SSM_EUNSUPPORTED, SSM_ECUDA, SSM_EWORKSPACE = 0, 1, 2, 3, 4
 CKPT_STEPS = 16
 MAX_DSTATE = 16
 NOALLOC_SCRATCH_BYTES = 8 << 20
-SSM_SCALAR_A, SSM_REVERSE, SSM_ZOH = 1, 2, 4
+SSM_SCALAR_A, SSM_REVERSE, SSM_ZOH, SSM_CHANNELS_LAST = 1, 2, 4, 8
 
 _vp = ctypes.c_void_p
 _i = ctypes.c_int

@@ -280,7 +280,7 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
                   size_t workspace_bytes, int batch, int dim, int seqlen, int dstate,
                   int io_dtype, void* stream, int flags, int bc_groups) {
   g_err[0] = 0;
-  if (flags & ~(SSM_SCALAR_A | SSM_REVERSE | SSM_ZOH))
+  if (flags & ~(SSM_SCALAR_A | SSM_REVERSE | SSM_ZOH | SSM_CHANNELS_LAST))
     return fail(SSM_EINVAL, "unknown flags 0x%x", flags);
   const bool scalar_a = (flags & SSM_SCALAR_A) != 0;
   TRY(check_dims(batch, dim, seqlen, dstate, io_dtype));
@@ -327,8 +327,11 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
   a.lpc = (scalar_a || a.zoh || bc_groups > 1) ? 2 : fwd_lpc();
   a.warps_per_b = (dim + 32 / a.lpc - 1) / (32 / a.lpc);
   a.nwarps = (long long)batch * a.warps_per_b;
-  const bool vec = (seqlen * es) % 16 == 0 && aligned16(u) && aligned16(delta) && aligned16(z) &&
-                   aligned16(out) && aligned16(B) && aligned16(C);
+  a.channels_last = (flags & SSM_CHANNELS_LAST) ? 1 : 0;
+  // 128-bit row accesses need rows along L; the channels-last layout takes element accesses
+  const bool vec = !a.channels_last && (seqlen * es) % 16 == 0 && aligned16(u) &&
+                   aligned16(delta) && aligned16(z) && aligned16(out) && aligned16(B) &&
+                   aligned16(C);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int wpb = fwd_wpb();
   const int km = fwd_kmufu(a.nwarps * (long long)plan.nchunk);
@@ -432,7 +435,7 @@ int scan_bwd_core(const void* u, const void* delta, const float* A, const void* 
                   void* du, void* ddelta, float* dA, void* dB, void* dC, float* dD, void* dz,
                   float* ddt_bias, float* dh0, void* workspace, size_t workspace_bytes,
                   int batch, int dim, int seqlen, int dstate, int io_dtype, void* stream,
-                  bool reverse, bool zoh, int bc_groups) {
+                  bool reverse, bool zoh, int bc_groups, bool channels_last = false) {
   TRY(check_dims(batch, dim, seqlen, dstate, io_dtype));
   TRY(check_groups(dim, bc_groups));
   const size_t es = esize(io_dtype);
@@ -476,9 +479,9 @@ int scan_bwd_core(const void* u, const void* delta, const float* A, const void* 
   float* ck_ws = reinterpret_cast<float*>(w);
   float* part_bc = reinterpret_cast<float*>(w + l.ckpt);
   float* part_adt = reinterpret_cast<float*>(w + l.ckpt + l.part_bc);
-  const bool vec = (seqlen * es) % 16 == 0 && aligned16(u) && aligned16(delta) && aligned16(z) &&
-                   aligned16(dout) && aligned16(du) && aligned16(ddelta) && aligned16(dz) &&
-                   aligned16(B) && aligned16(C);
+  const bool vec = !channels_last && (seqlen * es) % 16 == 0 && aligned16(u) &&
+                   aligned16(delta) && aligned16(z) && aligned16(dout) && aligned16(du) &&
+                   aligned16(ddelta) && aligned16(dz) && aligned16(B) && aligned16(C);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
 
@@ -494,6 +497,7 @@ int scan_bwd_core(const void* u, const void* delta, const float* A, const void* 
     a.reverse = reverse ? 1 : 0;
     a.zoh = zoh ? 1 : 0;
     a.bc_groups = bc_groups;
+    a.channels_last = channels_last ? 1 : 0;
     a.lpc = (zoh || bc_groups > 1) ? 2 : fwd_lpc();
     a.warps_per_b = (dim + 32 / a.lpc - 1) / (32 / a.lpc);
     a.nwarps = (long long)batch * a.warps_per_b;
@@ -512,6 +516,7 @@ int scan_bwd_core(const void* u, const void* delta, const float* A, const void* 
   b.reverse = reverse ? 1 : 0;
   b.zoh = zoh ? 1 : 0;
   b.bc_groups = bc_groups;
+  b.channels_last = channels_last ? 1 : 0;
   b.warps_per_b = (dim + 15) / 16;
   b.nwarps = (long long)batch * b.warps_per_b;
   b.wpb = l.wpb;
@@ -541,7 +546,7 @@ int ssm_scan_bwd(const void* u, const void* delta, const float* A, const void* B
 
 size_t ssm_scan_bwd_ex_workspace_size(int batch, int dim, int seqlen, int dstate, int bc_groups,
                                       int io_dtype, int have_ckpt, int flags) {
-  if (flags & ~(SSM_SCALAR_A | SSM_REVERSE | SSM_ZOH)) return 0;
+  if (flags & ~(SSM_SCALAR_A | SSM_REVERSE | SSM_ZOH | SSM_CHANNELS_LAST)) return 0;
   if (check_dims(batch, dim, seqlen, dstate, io_dtype) != SSM_OK) return 0;
   if (check_groups(dim, bc_groups) != SSM_OK) return 0;
   const size_t base = layout_bwd(batch, dim, seqlen, dstate, have_ckpt != 0, bc_groups).total;
@@ -557,15 +562,16 @@ int ssm_scan_bwd_ex(const void* u, const void* delta, const float* A, const void
                     size_t workspace_bytes, int batch, int dim, int seqlen, int dstate,
                     int bc_groups, int io_dtype, int flags, void* stream) {
   g_err[0] = 0;
-  if (flags & ~(SSM_SCALAR_A | SSM_REVERSE | SSM_ZOH))
+  if (flags & ~(SSM_SCALAR_A | SSM_REVERSE | SSM_ZOH | SSM_CHANNELS_LAST))
     return fail(SSM_EINVAL, "unknown flags 0x%x", flags);
   const bool reverse = (flags & SSM_REVERSE) != 0, zoh = (flags & SSM_ZOH) != 0;
+  const bool cl = (flags & SSM_CHANNELS_LAST) != 0;
   TRY(check_dims(batch, dim, seqlen, dstate, io_dtype));
   if (!(flags & SSM_SCALAR_A))
     return scan_bwd_core(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL, ckpt,
                          du, ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, workspace,
                          workspace_bytes, batch, dim, seqlen, dstate, io_dtype, stream, reverse,
-                         zoh, bc_groups);
+                         zoh, bc_groups, cl);
   // scalar decay: broadcast A over the states, run the per-state backward, sum dA over n
   TRY(check_ptr(A, (size_t)dim * 4, 4, "A"));
   TRY(check_opt(dA, (size_t)dim * 4, 4, "dA"));
@@ -588,7 +594,7 @@ int ssm_scan_bwd_ex(const void* u, const void* delta, const float* A, const void
   const int rc = scan_bwd_core(u, delta, Af, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL,
                                ckpt, du, ddelta, dA ? dAf : nullptr, dB, dC, dD, dz, ddt_bias,
                                dh0, w + 2 * head, workspace_bytes - 2 * head, batch, dim, seqlen,
-                               dstate, io_dtype, stream, reverse, zoh, bc_groups);
+                               dstate, io_dtype, stream, reverse, zoh, bc_groups, cl);
   if (rc != SSM_OK) return rc;
   if (dA) {
     reduce_da_kernel<<<(unsigned)((dim + 255) / 256), 256, 0, s>>>(dAf, dA, dim, dstate);

@@ -309,7 +309,9 @@ __global__ void __launch_bounds__(128) bwd_kernel(const BwdArgs a) {
 
   // time rows at step 0 in scan order (mirrored for a reverse scan); the lane owns steps
   // [8 q, 8 q + 8) of each block
-  const long long row = ch * (long long)L;
+  const bool cl = a.channels_last != 0;  // [batch][L][dim] rows: element stride dim
+  const long long row = cl ? (long long)b * L * a.dim + dd : ch * (long long)L;
+  const long long ts_x = cl ? a.dim : 1, ts_bc = cl ? (long long)a.bc_groups * N : 1;
   const bool rev = a.reverse != 0;
   const IO* up = reinterpret_cast<const IO*>(a.u) + row;
   const IO* dp = reinterpret_cast<const IO*>(a.delta) + row;
@@ -317,7 +319,8 @@ __global__ void __launch_bounds__(128) bwd_kernel(const BwdArgs a) {
   const IO* gp = reinterpret_cast<const IO*>(a.dout) + row;
   const bool bc_live = slot < N;  // the lane also stages B/C row `slot`, steps [8 q, 8 q + 8)
   const int gbc = ((grp * a.wpb + wib) * kCW) / (a.dim / a.bc_groups);  // the warp's B/C group
-  const long long bcrow = (((long long)b * a.bc_groups + gbc) * N + (bc_live ? slot : 0)) * L;
+  const long long bcrow = cl ? ((long long)b * L * a.bc_groups + gbc) * N + (bc_live ? slot : 0)
+                             : (((long long)b * a.bc_groups + gbc) * N + (bc_live ? slot : 0)) * L;
   const IO* Bp = reinterpret_cast<const IO*>(a.B) + bcrow;
   const IO* Cp = reinterpret_cast<const IO*>(a.C) + bcrow;
   float* sBw = reinterpret_cast<float*>(tl.sB);
@@ -335,10 +338,10 @@ __global__ void __launch_bounds__(128) bwd_kernel(const BwdArgs a) {
       load_steps<IO, kHB, true>(rg, gp, L, tq, kHB, rev);
       if (zp) load_steps<IO, kHB, true>(rz, zp, L, tq, kHB, rev);
     } else {
-      load_steps<IO, kHB, false>(ru, up, L, tq, nown, rev);
-      load_steps<IO, kHB, false>(rd, dp, L, tq, nown, rev);
-      load_steps<IO, kHB, false>(rg, gp, L, tq, nown, rev);
-      if (zp) load_steps<IO, kHB, false>(rz, zp, L, tq, nown, rev);
+      load_steps<IO, kHB, false>(ru, up, L, tq, nown, rev, ts_x);
+      load_steps<IO, kHB, false>(rd, dp, L, tq, nown, rev, ts_x);
+      load_steps<IO, kHB, false>(rg, gp, L, tq, nown, rev, ts_x);
+      if (zp) load_steps<IO, kHB, false>(rz, zp, L, tq, nown, rev, ts_x);
     }
     if (!bc_live) {
       rb.zero();
@@ -347,8 +350,8 @@ __global__ void __launch_bounds__(128) bwd_kernel(const BwdArgs a) {
       load_steps<IO, kHB, true>(rb, Bp, L, tq, kHB, rev);
       load_steps<IO, kHB, true>(rc, Cp, L, tq, kHB, rev);
     } else {
-      load_steps<IO, kHB, false>(rb, Bp, L, tq, nown, rev);
-      load_steps<IO, kHB, false>(rc, Cp, L, tq, nown, rev);
+      load_steps<IO, kHB, false>(rb, Bp, L, tq, nown, rev, ts_bc);
+      load_steps<IO, kHB, false>(rc, Cp, L, tq, nown, rev, ts_bc);
     }
     // the state entering the block
     float2 hstart[4];
@@ -438,7 +441,7 @@ __global__ void __launch_bounds__(128) bwd_kernel(const BwdArgs a) {
       const auto put = [&](void* base, const float (&v)[kHB]) {
         IO* o = reinterpret_cast<IO*>(base) + row;
         if (VEC && nown == kHB) store_steps<IO, kHB, true>(o, v, L, tq, kHB, rev);
-        else store_steps<IO, kHB, false>(o, v, L, tq, nown, rev);
+        else store_steps<IO, kHB, false>(o, v, L, tq, nown, rev, ts_x);
       };
       if (a.du) put(a.du, odu);
       if (a.ddelta) put(a.ddelta, odd);
@@ -502,7 +505,9 @@ __global__ void bwd_finish_bc(const BwdArgs a, IO* dB, IO* dC) {
     s += a.part_bc[(((long long)(g * a.batch + b) * 2 + which) * kNS + n) * a.L + t];
   IO* dst = which == 0 ? dB : dC;
   if (!dst) return;
-  const long long o = (((long long)b * a.bc_groups + gb) * a.N + n) * a.L + (a.reverse ? a.L - 1 - t : t);
+  const long long tm = a.reverse ? a.L - 1 - t : t;  // time index of scan step t
+  const long long o = a.channels_last ? (((long long)b * a.L + tm) * a.bc_groups + gb) * a.N + n
+                                      : (((long long)b * a.bc_groups + gb) * a.N + n) * a.L + tm;
   if (sizeof(IO) == 2) reinterpret_cast<uint16_t*>(dst)[o] = f32_to_bf16(s);
   else reinterpret_cast<float*>(dst)[o] = s;
 }

@@ -228,6 +228,7 @@ struct ChunkLane {
   float dlim;  // |Δ| < dlim keeps |Δ A log2 e| <= 126 for every state of the warp
   float a1;    // scalar decay: A_d (times log2 e on the bf16 path)
   float ra1;   // scalar decay with the ZOH input term: 1 / A_d
+  long long ts_x, ts_bc;  // element strides of the u/delta/z/out rows and of the B/C rows
 
 
   // Rows of the block starting at tb; steps at or beyond t_end read as zero.  A reverse scan's
@@ -241,9 +242,9 @@ struct ChunkLane {
       load_steps<IO, SPL, true, false>(r.d, dp, L, tq, SPL, rev);
       if (zp) load_steps<IO, SPL, true, false>(r.z, zp, L, tq, SPL, rev);
     } else {
-      load_steps<IO, SPL, false, false>(r.u, up, L, tq, nv, rev);
-      load_steps<IO, SPL, false, false>(r.d, dp, L, tq, nv, rev);
-      if (zp) load_steps<IO, SPL, false, false>(r.z, zp, L, tq, nv, rev);
+      load_steps<IO, SPL, false, false>(r.u, up, L, tq, nv, rev, ts_x);
+      load_steps<IO, SPL, false, false>(r.d, dp, L, tq, nv, rev, ts_x);
+      if (zp) load_steps<IO, SPL, false, false>(r.z, zp, L, tq, nv, rev, ts_x);
     }
     if (!bc_live) {
       r.b.zero();
@@ -252,8 +253,8 @@ struct ChunkLane {
       load_steps<IO, 8, true, false>(r.b, Bp, L, t8, 8, rev);
       if (kReadout) load_steps<IO, 8, true, false>(r.c, Cp, L, t8, 8, rev);
     } else {
-      load_steps<IO, 8, false, false>(r.b, Bp, L, t8, nv8, rev);
-      if (kReadout) load_steps<IO, 8, false, false>(r.c, Cp, L, t8, nv8, rev);
+      load_steps<IO, 8, false, false>(r.b, Bp, L, t8, nv8, rev, ts_bc);
+      if (kReadout) load_steps<IO, 8, false, false>(r.c, Cp, L, t8, nv8, rev, ts_bc);
     }
   }
 
@@ -339,7 +340,7 @@ struct ChunkLane {
   __device__ __forceinline__ void store_out(int t0, const float (&o)[SPL], int nown) const {
     if (!act || nown <= 0) return;
     if (VEC && nown == SPL) store_steps<IO, SPL, true>(op, o, L, t0 + SPL * q, SPL, rev);
-    else store_steps<IO, SPL, false>(op, o, L, t0 + SPL * q, nown, rev);
+    else store_steps<IO, SPL, false>(op, o, L, t0 + SPL * q, nown, rev, ts_x);
   }
 };
 
@@ -414,7 +415,12 @@ __device__ __forceinline__ void run_chunk(const FwdArgs& a, WarpTile<LPC>& tile,
   const int L = a.L, N = a.N;
 
   Lane ln;
-  const long long row = ch * (long long)L;  // the lane owns steps [SPL q, SPL q + SPL) of each block
+  // time rows at step 0; the lane owns steps [SPL q, SPL q + SPL) of each block.  Rows run along
+  // L ([batch][dim][L]), or across it with stride dim for the channels-last layout.
+  const bool cl = a.channels_last != 0;
+  const long long row = cl ? (long long)b * L * a.dim + (ch - (long long)b * a.dim) : ch * (long long)L;
+  ln.ts_x = cl ? a.dim : 1;
+  ln.ts_bc = cl ? (long long)a.bc_groups * N : 1;
   ln.up = reinterpret_cast<const IO*>(a.u) + row;
   ln.dp = reinterpret_cast<const IO*>(a.delta) + row;
   ln.zp = (kReadout && a.z) ? reinterpret_cast<const IO*>(a.z) + row : nullptr;
@@ -424,7 +430,9 @@ __device__ __forceinline__ void run_chunk(const FwdArgs& a, WarpTile<LPC>& tile,
   ln.bh = lane & 1;
   ln.bc_live = ln.bn < N;
   // the warp's B/C group: gbc of bc_groups for this batch row
-  const long long bcrow = (((long long)b * a.bc_groups + gbc) * N + (ln.bc_live ? ln.bn : 0)) * L;
+  const int bn_row = ln.bc_live ? ln.bn : 0;
+  const long long bcrow = cl ? ((long long)b * L * a.bc_groups + gbc) * N + bn_row
+                             : (((long long)b * a.bc_groups + gbc) * N + bn_row) * L;
   ln.Bp = reinterpret_cast<const IO*>(a.B) + bcrow;
   ln.Cp = reinterpret_cast<const IO*>(a.C) + bcrow;
   ln.slot = slot;

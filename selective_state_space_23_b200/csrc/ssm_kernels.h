@@ -46,6 +46,7 @@ struct FwdArgs {
   int reverse;          // scan runs from t = L-1 down to 0 (time rows read/written mirrored)
   int zoh;              // zero-order-hold input term (e^{ΔA} - 1)/A B x instead of Δ B x
   int bc_groups;        // B, C are [batch][bc_groups][N][L]; channel d uses group d / (dim / bc_groups)
+  int channels_last;    // u, delta, z, out are [batch][L][dim] and B, C [batch][L][bc_groups][N]
   int lpc;              // lanes per channel: 1, 2 or 4 (16 / lpc states each)
   int warps_per_b;      // ceil(dim / (32 / lpc))
   long long nwarps;     // batch * warps_per_b
@@ -79,6 +80,7 @@ struct BwdArgs {
   int reverse;          // gradients of the reverse scan (time rows read/written mirrored)
   int zoh;              // gradients of the zero-order-hold input term
   int bc_groups;        // B, C (and dB, dC) are [batch][bc_groups][N][L]
+  int channels_last;    // time rows strided: [batch][L][dim] and [batch][L][bc_groups][N]
 };
 
 struct DecodeArgs {

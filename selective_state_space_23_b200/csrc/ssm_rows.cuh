@@ -109,50 +109,62 @@ __device__ __forceinline__ void reverse_row(Row<IO, E>& r) {
 // segment is aligned as load_row requires and all E steps are valid.  REORDER = false leaves a
 // reversed segment in row order (reverse_row later puts it in scan order), so that a prefetch
 // does not wait for its data at the load.
+// ts: the row's element stride (1 for rows along L; the channel count for a [batch][L][dim]
+// layout); only the element paths (VEC = false) take a stride other than 1.
 template <typename IO, int E, bool VEC, bool REORDER = true>
 __device__ __forceinline__ void load_steps(Row<IO, E>& r, const IO* row, int L, int tau, int nvalid,
-                                           bool rev) {
-  if (!rev) {
-    load_row<IO, E, VEC>(r, row + tau, nvalid);
-    return;
-  }
-  const long long base = (long long)L - tau - E;  // row index of the segment's first element
-  if (VEC) {
-    load_row<IO, E, true>(r, row + base, E);
-  } else {
-    r.zero();
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      if (e >= E - nvalid) {  // scan step E-1-e is valid
-        if (sizeof(IO) == 4)
-          r.w[e] = __ldcs(reinterpret_cast<const uint32_t*>(row) + (base + e));
-        else
-          r.w[e >> 1] |= ((uint32_t)__ldcs(reinterpret_cast<const unsigned short*>(row) +
-                                           (base + e))) << (16 * (e & 1));
-      }
+                                           bool rev, long long ts = 1) {
+  if (VEC || ts == 1) {
+    if (!rev) {
+      load_row<IO, E, VEC>(r, row + tau, nvalid);
+      return;
+    }
+    if (VEC) {
+      load_row<IO, E, true>(r, row + ((long long)L - tau - E), E);
+      if (REORDER) reverse_row(r);
+      return;
     }
   }
-  if (REORDER) reverse_row(r);
+  // element accesses: step tau + e (scan order) lives at row index i(e)
+  r.zero();
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    // a mirrored segment kept in row order (REORDER = false) places scan step E-1-e in slot e
+    const int sstep = (rev && !REORDER) ? E - 1 - e : e;
+    if (sstep < nvalid) {
+      const long long i = (rev ? (long long)L - 1 - tau - sstep : (long long)tau + sstep) * ts;
+      if (sizeof(IO) == 4)
+        r.w[e] = __ldcs(reinterpret_cast<const uint32_t*>(row) + i);
+      else
+        r.w[e >> 1] |= ((uint32_t)__ldcs(reinterpret_cast<const unsigned short*>(row) + i))
+                       << (16 * (e & 1));
+    }
+  }
 }
 
 // Store E values of steps [tau, tau + E) (only the first nvalid) to a time row in scan order.
 template <typename IO, int E, bool VEC>
 __device__ __forceinline__ void store_steps(IO* row, const float (&o)[E], int L, int tau, int nvalid,
-                                            bool rev) {
-  if (!rev) {
-    store_row<IO, E, VEC>(row + tau, o, nvalid);
-  } else if (VEC) {
-    float rv[E];
+                                            bool rev, long long ts = 1) {
+  if (VEC || ts == 1) {
+    if (!rev) {
+      store_row<IO, E, VEC>(row + tau, o, nvalid);
+      return;
+    }
+    if (VEC) {
+      float rv[E];
 #pragma unroll
-    for (int e = 0; e < E; ++e) rv[e] = o[E - 1 - e];
-    store_row<IO, E, true>(row + (L - tau - E), rv, E);
-  } else {
+      for (int e = 0; e < E; ++e) rv[e] = o[E - 1 - e];
+      store_row<IO, E, true>(row + ((long long)L - tau - E), rv, E);
+      return;
+    }
+  }
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      if (e < nvalid) {
-        if (sizeof(IO) == 4) reinterpret_cast<float*>(row)[L - 1 - tau - e] = o[e];
-        else reinterpret_cast<uint16_t*>(row)[L - 1 - tau - e] = f32_to_bf16(o[e]);
-      }
+  for (int e = 0; e < E; ++e) {
+    if (e < nvalid) {
+      const long long i = (rev ? (long long)L - 1 - tau - e : (long long)tau + e) * ts;
+      if (sizeof(IO) == 4) reinterpret_cast<float*>(row)[i] = o[e];
+      else reinterpret_cast<uint16_t*>(row)[i] = f32_to_bf16(o[e]);
     }
   }
 }
