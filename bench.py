@@ -301,7 +301,25 @@ def bench_extras(dev):
     out["scalar_decay_fwd"] = {"shape": "8x2048x2048 N16 bf16, A [dim]", "fwd_ms": ms,
                                "tokens_per_s": b * L / (ms * 1e-3),
                                "hbm_gbs": compulsory_bytes_shape(b, d, L, N) / (ms * 1e-3) / 1e9}
-    del u, de, z, B, C, o
+
+    # the other variants of the forward scan on the same layer
+    A, D, bias = prm(d, N, 1e-3, 1e-1)
+    Bg, Cg = rnd((b, 4, N, L)), rnd((b, 4, N, L))
+    uc, dec, zc = (t.transpose(1, 2).contiguous() for t in (u, de, z))
+    Bc, Cc = B.transpose(1, 2).contiguous(), C.transpose(1, 2).contiguous()
+    oc = torch.empty_like(uc)
+    var = {
+        "default": lambda: ssm.ssm_scan_fwd(u, de, A, B, C, D=D, z=z, dt_bias=bias, out=o),
+        "zoh": lambda: ssm.ssm_scan_fwd(u, de, A, B, C, D=D, z=z, dt_bias=bias, out=o, zoh=True),
+        "reverse": lambda: ssm.ssm_scan_fwd(u, de, A, B, C, D=D, z=z, dt_bias=bias, out=o,
+                                            reverse=True),
+        "groups4": lambda: ssm.ssm_scan_fwd(u, de, A, Bg, Cg, D=D, z=z, dt_bias=bias, out=o),
+        "channels_last": lambda: ssm.ssm_scan_fwd(uc, dec, A, Bc, Cc, D=D, z=zc, dt_bias=bias,
+                                                  out=oc, channels_last=True),
+    }
+    out["variants_fwd_ms"] = {"shape": "8x2048x2048 N16 bf16",
+                              **{k: timeit(f, 20) for k, f in var.items()}}
+    del u, de, z, B, C, o, Bg, Cg, uc, dec, zc, Bc, Cc, oc
     torch.cuda.empty_cache()
 
     # long sequence
