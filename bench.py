@@ -419,19 +419,20 @@ def main():
     ms_step = total_ms / K
     value = world * w.tokens / (ms_step * 1e-3)
 
-    # end to end through the public call with host buffers: pinned H2D of the step's inputs,
-    # the scan, D2H of the output, every step
+    # end to end through the public host-memory call (ssm_scan_fwd_host): every step copies the
+    # inputs from pinned host memory, scans and copies the output back, pipelined over batch rows
     hx = {k: v.pin_memory() for k, v in x.items()}
     hout = torch.empty_like(x["u"]).pin_memory()
     names_in = ("u", "delta", "z", "B", "C")
     h2d = sum(hx[k].numel() * hx[k].element_size() for k in names_in)
     d2h = hout.numel() * hout.element_size()
+    hws = torch.empty(max(1, ssm.fwd_host_workspace_bytes(w.batch, w.dim, w.seqlen, w.dstate,
+                                                          w.io_dtype)), dtype=torch.uint8,
+                      device=dev)
 
     def e2e_step():
-        for k in names_in:
-            xd[k].copy_(hx[k], non_blocking=True)
-        step()
-        hout.copy_(out, non_blocking=True)
+        ssm.ssm_scan_fwd_host(hx["u"], hx["delta"], xd["A"], hx["B"], hx["C"], D=xd["D"],
+                              z=hx["z"], dt_bias=xd["dt_bias"], out=hout, workspace=hws)
 
     e2e_ms = e2e_value = None
     if args.e2e_steps > 0:

@@ -226,6 +226,30 @@ SSM_API int ssm_scan_bwd_ex(const void* u, const void* delta, const float* A, co
                             int seqlen, int dstate, int bc_groups, int io_dtype, int flags,
                             void* stream);
 
+/*
+ * ssm_scan_fwd from and to HOST memory.  The pages have no counterpart: this is the call a user
+ * makes when sequences live in host memory.  The batch is cut into chunks of rows that flow
+ * through three streams (host-to-device copies, the scan, device-to-host copies), so the copies
+ * of one chunk overlap the scan of another and the two copy directions overlap each other.
+ *   u, delta, z, out  [batch][dim][L] io       HOST (page-locked memory lets the copies overlap;
+ *   B, C              [batch][N][L] io         HOST   pageable memory works but serialises them)
+ *   h0, hL            [batch][dim][N] f32      HOST, or NULL
+ *   A, D, dt_bias     as for ssm_scan_fwd      DEVICE (model parameters stay on the GPU)
+ *   workspace         DEVICE, 256-byte aligned, ssm_scan_fwd_host_workspace_size() bytes
+ * Asynchronous with respect to the host: the output is complete once `stream` has reached this
+ * point (e.g. after cudaStreamSynchronize(stream)); work queued on `stream` before the call runs
+ * first.  The three streams and their events are created on a device's first call and kept until
+ * the process exits; calls from several host threads on one device are serialised while they
+ * enqueue.  Errors as for ssm_scan_fwd; a copy failure returns SSM_ECUDA.
+ */
+SSM_API size_t ssm_scan_fwd_host_workspace_size(int batch, int dim, int seqlen, int dstate,
+                                                int io_dtype);
+SSM_API int ssm_scan_fwd_host(const void* u, const void* delta, const float* A, const void* B,
+                              const void* C, const float* D, const void* z, const float* dt_bias,
+                              int delta_softplus, const float* h0, float* hL, void* out,
+                              void* workspace, size_t workspace_bytes, int batch, int dim,
+                              int seqlen, int dstate, int io_dtype, void* stream);
+
 /* Size of the static scratch array used by ssm_scan_fwd_noalloc (8 MiB per GPU). */
 #define SSM_NOALLOC_SCRATCH_BYTES (8u << 20)
 

@@ -17,6 +17,7 @@ from . import _abi
 from ._abi import CKPT_STEPS, MAX_DSTATE
 
 __all__ = ["ssm_scan_fwd", "ssm_scan_bwd", "ssm_scan_fwd_scalar_a", "ssm_scan_bwd_scalar_a",
+           "ssm_scan_fwd_host", "fwd_host_workspace_bytes",
            "ssm_state_update", "fwd_workspace_bytes",
            "bwd_workspace_bytes", "CKPT_STEPS", "MAX_DSTATE", "library_path"]
 
@@ -238,6 +239,54 @@ def ssm_scan_bwd_scalar_a(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None,
     """Gradients of :func:`ssm_scan_fwd_scalar_a` (dA is [dim])."""
     return _scan_bwd(u, delta, A, B, C, dout, D, z, dt_bias, delta_softplus, h0, dhL, ckpt,
                      workspace, need, True, reverse, zoh, channels_last)
+
+
+def _host(t, name, shape, dtype):
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor) or t.device.type != "cpu":
+        raise ValueError(f"{name} must be a CPU tensor")
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)}")
+
+
+def ssm_scan_fwd_host(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=True,
+                      h0=None, return_final_state=False, out=None, workspace=None):
+    """Forward scan from and to host memory: u, delta, z, B, C (and h0) are CPU tensors (pinned
+    memory lets the copies overlap the scan), A, D, dt_bias live on the GPU.  The batch flows
+    through copy-in, scan and copy-out streams in chunks of rows.  Returns out (CPU), or
+    (out, hL) with ``return_final_state``; both are complete once the current stream of A's
+    device has reached this call."""
+    dev = A.device
+    batch, dim, L = u.shape
+    N = A.shape[-1]
+    io = u.dtype
+    code = _io_code(io)
+    for t, n, shp in ((u, "u", (batch, dim, L)), (delta, "delta", (batch, dim, L)),
+                      (z, "z", (batch, dim, L)), (B, "B", (batch, N, L)), (C, "C", (batch, N, L))):
+        _host(t, n, shp, io)
+    _host(h0, "h0", (batch, dim, N), torch.float32)
+    _need(A, "A", (dim, N), torch.float32, dev)
+    _opt(D, "D", (dim,), torch.float32, dev)
+    _opt(dt_bias, "dt_bias", (dim,), torch.float32, dev)
+    pin = u.is_pinned()
+    if out is None:
+        out = torch.empty((batch, dim, L), dtype=io, pin_memory=pin)
+    _host(out, "out", (batch, dim, L), io)
+    hL = torch.empty((batch, dim, N), dtype=torch.float32, pin_memory=pin) if return_final_state else None
+    nws = int(_abi.lib().ssm_scan_fwd_host_workspace_size(batch, dim, L, N, code))
+    ws = _workspace(nws, dev, workspace)
+    rc = _abi.lib().ssm_scan_fwd_host(
+        _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias),
+        int(bool(delta_softplus)), _ptr(h0), _ptr(hL), _ptr(out), _ptr(ws),
+        0 if ws is None else ws.numel(), batch, dim, L, N, code, _stream(dev))
+    _abi.check(rc, "ssm_scan_fwd_host")
+    return (out, hL) if return_final_state else out
+
+
+def fwd_host_workspace_bytes(batch, dim, seqlen, dstate, dtype) -> int:
+    return int(_abi.lib().ssm_scan_fwd_host_workspace_size(batch, dim, seqlen, dstate,
+                                                            _io_code(dtype)))
 
 
 def ssm_state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=True,

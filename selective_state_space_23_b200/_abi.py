@@ -45,6 +45,9 @@ SIGNATURES = {
     "ssm_scan_bwd_ex": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp,
                              _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                              _i, _i, _i, _i, _i, _i, _i, _vp]),
+    "ssm_scan_fwd_host_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
+    "ssm_scan_fwd_host": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _sz,
+                               _i, _i, _i, _i, _i, _vp]),
     "ssm_scan_fwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp,
                                   _i, _i, _i, _i, _i, _vp]),
     "ssm_state_update": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp,
