@@ -202,18 +202,20 @@ FwdPlan plan_fwd(int batch, int dim, int seqlen) {
 }
 
 // Launch tuning of the forward kernel (measured on B200; the environment variables override it
-// for experiments): one warp per CTA.  Exponentials on the MUFU unit per lane and step pair (of
-// 16; the rest use the FMA-pipe polynomial): with fewer than 8 warps per SM (e.g. 8 x 2048
-// channels) every warp is latency-bound and the shortest instruction stream wins, so all 16 go
-// to MUFU; with more warps 14 of 16 balance the MUFU and FMA pipes best (4 x 5120 channels,
-// and the time-split 1 x 256 x 2^20 sequence).
+// for experiments): one warp per CTA; 14 of every 16 exponentials per lane and step pair on the
+// MUFU unit, the rest on the FMA-pipe polynomial (best on 8 x 2048 and 4 x 5120 channels and on
+// the time-split 1 x 256 x 2^20 sequence).
 int fwd_wpb() {
   const int w = env_int("SSM_FWD_WPB", 1);
   return (w == 1 || w == 2 || w == 4) ? w : 1;
 }
 int fwd_kmufu(long long warps) {
-  return env_int("SSM_FWD_KMUFU", warps < 8LL * sm_count() ? 16 : 14);
+  (void)warps;
+  return env_int("SSM_FWD_KMUFU", 14);
 }
+
+// The output kernel's 255-register form pays off below 8 warps per SM (SSM_FWD_WIDE=0/1 forces it).
+int fwd_wide(long long warps) { return env_int("SSM_FWD_WIDE", warps < 8LL * sm_count() ? 1 : 0); }
 
 struct BwdLayout {
   size_t ckpt, part_bc, part_adt, total;
@@ -335,6 +337,7 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int wpb = fwd_wpb();
   const int km = fwd_kmufu(a.nwarps * (long long)plan.nchunk);
+  a.wide = fwd_wide(a.nwarps * (long long)plan.nchunk);
   cudaError_t e;
   if (plan.nchunk > 1) {
     const size_t nch = (size_t)batch * dim;

@@ -586,7 +586,7 @@ __device__ __forceinline__ void run_chunk(const FwdArgs& a, WarpTile<LPC>& tile,
 }
 
 template <typename IO, bool VEC, int MODE, int LPC, int KE, int KO, bool REV>
-__global__ void __launch_bounds__(128) fwd_kernel(const FwdArgs a) {
+__device__ __forceinline__ void fwd_body(const FwdArgs& a) {
   using Lay = Layout<LPC>;
   constexpr int SPL = Lay::kSPL, PPL = Lay::kPPL;
   extern __shared__ float4 smem4[];
@@ -644,13 +644,30 @@ __global__ void __launch_bounds__(128) fwd_kernel(const FwdArgs a) {
                                              act, ch, t_begin, t_end, last_chunk);
 }
 
+// The kernel, compiled for two register budgets.  fwd_kernel leaves the choice to the compiler
+// (about 160 registers); fwd_kernel_wide promises at most 128 threads and one CTA per SM, so the
+// compiler may use up to 255 registers and keeps more of each block's independent work in flight.
+// Measured on B200: with fewer than 8 warps per SM (8 x 2048 channels: 1.7 per scheduler) the
+// wide form is 5 % faster; with more warps (4 x 5120 channels, or the time-split 2^20 sequence)
+// the default form is faster (the wide one 17 % and 3 % slower).
 template <typename IO, bool VEC, int MODE, int LPC, int KE, int KO, bool REV>
+__global__ void __launch_bounds__(128) fwd_kernel(const FwdArgs a) {
+  fwd_body<IO, VEC, MODE, LPC, KE, KO, REV>(a);
+}
+
+template <typename IO, bool VEC, int MODE, int LPC, int KE, int KO, bool REV>
+__global__ void __launch_bounds__(128, 1) fwd_kernel_wide(const FwdArgs a) {
+  fwd_body<IO, VEC, MODE, LPC, KE, KO, REV>(a);
+}
+
+template <typename IO, bool VEC, int MODE, int LPC, int KE, int KO, bool REV, bool WIDE = false>
 void launch_one(const FwdArgs& a, dim3 grid, dim3 block, cudaStream_t s) {
   const size_t smem = (size_t)(block.x / 32) * sizeof(WarpTile<LPC>);
+  auto k = WIDE ? fwd_kernel_wide<IO, VEC, MODE, LPC, KE, KO, REV>
+                : fwd_kernel<IO, VEC, MODE, LPC, KE, KO, REV>;
   if (smem > 48 * 1024)
-    cudaFuncSetAttribute(fwd_kernel<IO, VEC, MODE, LPC, KE, KO, REV>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  fwd_kernel<IO, VEC, MODE, LPC, KE, KO, REV><<<grid, block, smem, s>>>(a);
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  k<<<grid, block, smem, s>>>(a);
 }
 
 template <typename IO, bool VEC, int MODE, bool REV>
@@ -688,6 +705,13 @@ cudaError_t launch_mode(const FwdArgs& a, int wpb, int kmufu, cudaStream_t s) {
       case 12: launch_one<IO, VEC, MODE, 1, 6, 6, REV>(a, grid, block, s); break;
       case 16: launch_one<IO, VEC, MODE, 1, 8, 8, REV>(a, grid, block, s); break;
       default: launch_one<IO, VEC, MODE, 1, 7, 7, REV>(a, grid, block, s); break;
+    }
+  } else if (a.wide && (kmufu == 12 || kmufu == 14 || kmufu == 16)) {
+    // few warps per SM: the 255-register form
+    switch (kmufu) {
+      case 12: launch_one<IO, VEC, MODE, 2, 3, 3, REV, true>(a, grid, block, s); break;
+      case 16: launch_one<IO, VEC, MODE, 2, 4, 4, REV, true>(a, grid, block, s); break;
+      default: launch_one<IO, VEC, MODE, 2, 4, 3, REV, true>(a, grid, block, s); break;
     }
   } else {
     // exponentials on the MUFU unit per lane over two steps (of 16): 8 ... 16

@@ -48,6 +48,7 @@ struct FwdArgs {
   int bc_groups;        // B, C are [batch][bc_groups][N][L]; channel d uses group d / (dim / bc_groups)
   int channels_last;    // u, delta, z, out are [batch][L][dim] and B, C [batch][L][bc_groups][N]
   int lpc;              // lanes per channel: 1, 2 or 4 (16 / lpc states each)
+  int wide;             // few warps per SM: the 255-register form of the output kernel
   int warps_per_b;      // ceil(dim / (32 / lpc))
   long long nwarps;     // batch * warps_per_b
 };

@@ -99,6 +99,21 @@ def test_every_exponential_split(monkeypatch, kmufu):
     assert_close(hL, ref["hL"], torch.bfloat16, "hL")
 
 
+@pytest.mark.parametrize("wide", [0, 1])
+@pytest.mark.parametrize("kmufu", [12, 14, 16])
+def test_both_register_budgets(monkeypatch, wide, kmufu):
+    """The output kernel's default and 255-register forms (chosen by warps per SM) agree with the
+    oracle, on a ragged length, and with each other bitwise."""
+    monkeypatch.setenv("SSM_FWD_KMUFU", str(kmufu))
+    w = workload("mamba370m_fwd", batch=2, dim=160, seqlen=777)
+    x = make_inputs(w, seed=13, with_h0=True)
+    monkeypatch.setenv("SSM_FWD_WIDE", str(wide))
+    out = run_gpu(on_dev(x))
+    assert_close(out, run_oracle(x)["out"], torch.bfloat16, "out")
+    monkeypatch.setenv("SSM_FWD_WIDE", str(1 - wide))
+    assert torch.equal(out, run_gpu(on_dev(x)))
+
+
 @pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("lpc", [1, 2, 4])
 def test_lanes_per_channel(monkeypatch, io, lpc):
