@@ -97,3 +97,61 @@ def test_host_pageable_pointer_is_rejected(lib):
     buf = (ctypes.c_uint16 * (64 * 256))()
     p = ctypes.cast(buf, ctypes.c_void_p)
     assert _fwd(lib, u=p, delta=p, A=p, B=p, C=p, out=p) == _abi.SSM_EINVAL
+
+
+def _fwd_ex(lib, flags=0, groups=1, **kw):
+    args = dict(u=None, delta=None, A=None, B=None, C=None, D=None, z=None, dt_bias=None, sp=1,
+                h0=None, hL=None, out=None, ckpt=None, ws=None, wsb=0, batch=1, dim=64, L=256,
+                N=16, groups=groups, io=1, flags=flags, stream=None)
+    args.update(kw)
+    return lib.ssm_scan_fwd_ex(*args.values())
+
+
+def _bwd_ex(lib, flags=0, groups=1, dim=64):
+    return lib.ssm_scan_bwd_ex(*([None] * 8), 1, *([None] * 14), 0, 1, dim, 256, 16, groups, 1,
+                               flags, None)
+
+
+def test_variant_flags_and_groups_are_checked_on_the_host(lib):
+    """The _ex entry points refuse unknown flag bits and unusable B/C groupings before touching
+    any pointer (nothing here needs a GPU)."""
+    known = _abi.SSM_SCALAR_A | _abi.SSM_REVERSE | _abi.SSM_ZOH | _abi.SSM_CHANNELS_LAST
+    assert _fwd_ex(lib, flags=16) == _abi.SSM_EINVAL
+    assert b"flags" in lib.ssm_last_error()
+    assert _bwd_ex(lib, flags=32) == _abi.SSM_EINVAL
+    assert _fwd_ex(lib, groups=0) == _abi.SSM_EINVAL
+    assert _fwd_ex(lib, groups=3) == _abi.SSM_EINVAL               # 64 channels, 3 groups
+    assert _fwd_ex(lib, groups=8) == _abi.SSM_EUNSUPPORTED         # 8 channels per group
+    assert b"multiple of 16" in lib.ssm_last_error()
+    assert _bwd_ex(lib, groups=8) == _abi.SSM_EUNSUPPORTED
+    # known flags with valid groups get past these checks (and stop at the NULL inputs)
+    assert _fwd_ex(lib, flags=known, groups=4) == _abi.SSM_EINVAL
+    assert b"NULL" in lib.ssm_last_error()
+    assert lib.ssm_scan_fwd_ex_workspace_size(1, 256, 1 << 20, 16, 1, 1, known) > 0
+    assert lib.ssm_scan_bwd_ex_workspace_size(4, 5120, 2048, 16, 8, 1, 1, 0) > 0
+    assert lib.ssm_scan_bwd_ex_workspace_size(4, 64, 2048, 16, 8, 1, 1, 0) == 0   # bad groups
+    # the scalar decay adds the broadcast rate and per-state dA to the backward's workspace
+    base = lib.ssm_scan_bwd_ex_workspace_size(4, 5120, 2048, 16, 1, 1, 1, 0)
+    sa = lib.ssm_scan_bwd_ex_workspace_size(4, 5120, 2048, 16, 1, 1, 1, _abi.SSM_SCALAR_A)
+    assert sa - base == 2 * 5120 * 16 * 4
+
+
+def test_decode_variants_refuse_the_reverse_flag(lib):
+    rc = lib.ssm_state_update_ex(*([None] * 9), 1, None, 1, 64, 16, 1, 1, _abi.SSM_REVERSE, None)
+    assert rc == _abi.SSM_EINVAL
+    rc = lib.ssm_state_update_ex(*([None] * 9), 1, None, 1, 64, 16, 8, 1, 0, None)
+    assert rc == _abi.SSM_EUNSUPPORTED                              # 8 channels per group
+
+
+def test_host_memory_call_checks_shape_and_workspace(lib):
+    assert lib.ssm_scan_fwd_host_workspace_size(0, 64, 256, 16, 1) == 0
+    need = lib.ssm_scan_fwd_host_workspace_size(8, 2048, 2048, 16, 1)
+    assert need >= 2 * 4 * 2048 * 2048 * 2                          # two slots of u, delta, z, out
+    buf = (ctypes.c_uint16 * 16)()
+    p = ctypes.cast(buf, ctypes.c_void_p)
+    rc = lib.ssm_scan_fwd_host(p, p, None, p, p, None, None, None, 1, None, None, p, None, 0,
+                               8, 2048, 2048, 16, 1, None)
+    assert rc == _abi.SSM_EWORKSPACE
+    rc = lib.ssm_scan_fwd_host(None, p, None, p, p, None, None, None, 1, None, None, p, None, 0,
+                               8, 2048, 2048, 16, 1, None)
+    assert rc == _abi.SSM_EINVAL
