@@ -330,6 +330,15 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
   a.warps_per_b = (dim + 32 / a.lpc - 1) / (32 / a.lpc);
   a.nwarps = (long long)batch * a.warps_per_b;
   a.channels_last = (flags & SSM_CHANNELS_LAST) ? 1 : 0;
+  if (a.channels_last) {
+    a.lpc = 2;
+    a.warps_per_b = (dim + 15) / 16;
+    a.nwarps = (long long)batch * a.warps_per_b;
+    // 16-byte tiles of 8 channels (or states) per lane: every warp full, rows 16-byte aligned
+    a.cl_tile = dim % 16 == 0 && dstate == 16 && (dim * es) % 16 == 0 && aligned16(u) &&
+                aligned16(delta) && aligned16(z) && aligned16(out) && aligned16(B) &&
+                aligned16(C);
+  }
   // 128-bit row accesses need rows along L; the channels-last layout takes element accesses
   const bool vec = !a.channels_last && (seqlen * es) % 16 == 0 && aligned16(u) &&
                    aligned16(delta) && aligned16(z) && aligned16(out) && aligned16(B) &&

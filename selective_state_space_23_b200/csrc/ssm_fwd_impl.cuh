@@ -80,6 +80,9 @@ struct WarpTile {
   BlockBuf<LPC> buf[2];
 };
 
+// Elements of the per-warp channels-last scratch: 5 input tiles and 1 output tile of 16 x 16.
+constexpr int kClScratch = 6 * 256;
+
 // Per-step quantities of one lane that do not depend on the state: Ā = 2^(Δ A log2 e) and the
 // input term Δ x B.  They are computed one step ahead of the state update (the only
 // loop-carried dependency), which keeps MUFU and shared-memory latency off the critical path.
@@ -229,11 +232,28 @@ struct ChunkLane {
   float a1;    // scalar decay: A_d (times log2 e on the bf16 path)
   float ra1;   // scalar decay with the ZOH input term: 1 / A_d
   long long ts_x, ts_bc;  // element strides of the u/delta/z/out rows and of the B/C rows
+  // channels-last tiles (element paths only): each lane moves one step of 8 consecutive
+  // channels (or states) with one 16-byte access, and a per-warp scratch turns the warp's
+  // [16 steps][16 channels] tile into per-lane rows and back
+  bool clt;
+  const IO* tu;   // u at (b, t = 0, channel d0 + 8 (lane & 1)); delta, z, out at the same offset
+  const IO* td;
+  const IO* tz;
+  IO* to;
+  const IO* tB;   // B at (b, t = 0, group, state 8 (lane & 1)); C likewise
+  const IO* tC;
+  IO* xs;         // the warp's scratch: 6 tiles of 16 x 16 elements
 
 
   // Rows of the block starting at tb; steps at or beyond t_end read as zero.  A reverse scan's
   // rows stay in row order until reorder() (called once the loads have landed).
   __device__ __forceinline__ void fetch(Rows& r, int tb) const {
+    if constexpr (!VEC && SPL == 8) {
+      if (clt) {
+        fetch_tile(r, tb);
+        return;
+      }
+    }
     const int tq = tb + SPL * q, t8 = tb + 8 * bh;
     const int nv = max(0, min(SPL, t_end - tq));
     const int nv8 = max(0, min(8, t_end - t8));
@@ -258,8 +278,70 @@ struct ChunkLane {
     }
   }
 
-  // Reverse scan: put fetched rows in scan order.
+  // Channels-last tile of the block starting at tb: lane l loads scan step l/2 of 8 consecutive
+  // channels (u, delta, z) and states (B, C) -- one 16-byte access each (two for fp32) -- into
+  // its row words, in the order reorder() transposes them from.
+  __device__ __forceinline__ void fetch_tile(Rows& r, int tb) const {
+    const int lane = 2 * slot + q, st = lane >> 1;
+    const bool ok = tb + st < t_end;
+    const long long tr = REV ? (long long)L - 1 - (tb + st) : (long long)(tb + st);
+    const auto ld = [&](Row<IO, 8>& w, const IO* base, long long stride) {
+      if (!ok) {
+        w.zero();
+        return;
+      }
+      const uint4* p = reinterpret_cast<const uint4*>(base + tr * stride);
+#pragma unroll
+      for (int i = 0; i < Row<IO, 8>::kWords / 4; ++i) {
+        const uint4 v = __ldcs(p + i);
+        w.w[4 * i] = v.x; w.w[4 * i + 1] = v.y; w.w[4 * i + 2] = v.z; w.w[4 * i + 3] = v.w;
+      }
+    };
+    ld(r.u, tu, ts_x);
+    ld(r.d, td, ts_x);
+    if (zp) ld(r.z, tz, ts_x);
+    ld(r.b, tB, ts_bc);
+    if (kReadout) ld(r.c, tC, ts_bc);
+  }
+
+  // Element e of a row, as raw io bits.
+  static __device__ __forceinline__ uint32_t elem(const Row<IO, 8>& w, int e) {
+    if (sizeof(IO) == 4) return w.w[e];
+    return (w.w[e >> 1] >> (16 * (e & 1))) & 0xffffu;
+  }
+
+  // Transpose one [16 steps][16 columns] tile held as lane pieces (step lane/2, columns
+  // 8 (lane & 1) .. + 7) into per-lane rows (column lane/2, steps 8 (lane & 1) .. + 7).
+  __device__ __forceinline__ void transpose_in(Row<IO, 8>& w, IO* T) const {
+    const int lane = 2 * slot + q, st = lane >> 1, h = lane & 1;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const uint32_t v = elem(w, e);
+      if (sizeof(IO) == 4) reinterpret_cast<uint32_t*>(T)[(8 * h + e) * 16 + st] = v;
+      else reinterpret_cast<uint16_t*>(T)[(8 * h + e) * 16 + st] = (uint16_t)v;
+    }
+    __syncwarp();
+    const uint4* p = reinterpret_cast<const uint4*>(T + st * 16 + 8 * h);
+#pragma unroll
+    for (int i = 0; i < Row<IO, 8>::kWords / 4; ++i) {
+      const uint4 v = p[i];
+      w.w[4 * i] = v.x; w.w[4 * i + 1] = v.y; w.w[4 * i + 2] = v.z; w.w[4 * i + 3] = v.w;
+    }
+  }
+
+  // Reverse scan: put fetched rows in scan order; channels-last tiles: transpose them into rows.
   __device__ __forceinline__ void reorder(Rows& r) const {
+    if constexpr (!VEC && SPL == 8) {
+      if (clt) {
+        __syncwarp();  // the scratch's previous reads are done
+        transpose_in(r.u, xs);
+        transpose_in(r.d, xs + 256);
+        if (zp) transpose_in(r.z, xs + 512);
+        transpose_in(r.b, xs + 768);
+        if (kReadout) transpose_in(r.c, xs + 1024);
+        return;
+      }
+    }
     if constexpr (!REV) return;
     reverse_row(r.u);
     reverse_row(r.d);
@@ -338,6 +420,42 @@ struct ChunkLane {
   }
 
   __device__ __forceinline__ void store_out(int t0, const float (&o)[SPL], int nown) const {
+    if constexpr (!VEC && SPL == 8) {
+      if (clt) {  // every lane takes part: the tile goes out through the scratch
+        IO* T = xs + 1280;
+        const int lane = 2 * slot + q, st = lane >> 1, h = lane & 1;
+        __syncwarp();
+        {  // the lane's row (16 or 32 bytes) into the scratch, rounded as the output
+          uint32_t rw[Row<IO, 8>::kWords];
+#pragma unroll
+          for (int i = 0; i < Row<IO, 8>::kWords; ++i)
+            rw[i] = sizeof(IO) == 4 ? __float_as_uint(o[i]) : pack_bf16x2(o[2 * i], o[2 * i + 1]);
+          uint4* p = reinterpret_cast<uint4*>(T + slot * 16 + 8 * q);
+#pragma unroll
+          for (int i = 0; i < Row<IO, 8>::kWords / 4; ++i)
+            p[i] = make_uint4(rw[4 * i], rw[4 * i + 1], rw[4 * i + 2], rw[4 * i + 3]);
+        }
+        __syncwarp();
+        uint32_t wv[Row<IO, 8>::kWords];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {  // step st of columns 8 h .. 8 h + 7
+          uint32_t v;
+          if (sizeof(IO) == 4) v = reinterpret_cast<const uint32_t*>(T)[(8 * h + e) * 16 + st];
+          else v = reinterpret_cast<const uint16_t*>(T)[(8 * h + e) * 16 + st];
+          if (sizeof(IO) == 4) wv[e] = v;
+          else if (e & 1) wv[e >> 1] |= v << 16;
+          else wv[e >> 1] = v;
+        }
+        if (t0 + st < t_end) {
+          const long long tr = REV ? (long long)L - 1 - (t0 + st) : (long long)(t0 + st);
+          uint4* p = reinterpret_cast<uint4*>(to + tr * ts_x);
+#pragma unroll
+          for (int i = 0; i < Row<IO, 8>::kWords / 4; ++i)
+            __stcs(p + i, make_uint4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]));
+        }
+        return;
+      }
+    }
     if (!act || nown <= 0) return;
     if (VEC && nown == SPL) store_steps<IO, SPL, true>(op, o, L, t0 + SPL * q, SPL, rev);
     else store_steps<IO, SPL, false>(op, o, L, t0 + SPL * q, nown, rev, ts_x);
@@ -404,7 +522,7 @@ __device__ __forceinline__ void run_chunk(const FwdArgs& a, WarpTile<LPC>& tile,
                                           const float2 (&ra)[Layout<LPC>::kPPL], float Dd,
                                           float bias, int lane, int slot, int q, int b, int gbc,
                                           bool act, long long ch, int t_begin, int t_end,
-                                          bool last_chunk) {
+                                          bool last_chunk, IO* xs) {
   using Lay = Layout<LPC>;
   using Lane = ChunkLane<IO, VEC, MODE, LPC, (KE < 0 ? KE : 0), REV>;
   // exponentials of a block that failed the range vote
@@ -435,6 +553,19 @@ __device__ __forceinline__ void run_chunk(const FwdArgs& a, WarpTile<LPC>& tile,
                              : (((long long)b * a.bc_groups + gbc) * N + bn_row) * L;
   ln.Bp = reinterpret_cast<const IO*>(a.B) + bcrow;
   ln.Cp = reinterpret_cast<const IO*>(a.C) + bcrow;
+  ln.clt = a.cl_tile != 0;
+  if (ln.clt) {  // channels-last tiles: the warp's first channel, this lane's half of 16 columns
+    const int d0 = (int)(ch - (long long)b * a.dim) - slot, h = lane & 1;
+    const long long xrow = (long long)b * L * a.dim + d0 + 8 * h;
+    ln.tu = reinterpret_cast<const IO*>(a.u) + xrow;
+    ln.td = reinterpret_cast<const IO*>(a.delta) + xrow;
+    ln.tz = a.z ? reinterpret_cast<const IO*>(a.z) + xrow : nullptr;
+    ln.to = kReadout ? reinterpret_cast<IO*>(a.out) + xrow : nullptr;
+    const long long brow = ((long long)b * L * a.bc_groups + gbc) * N + 8 * h;
+    ln.tB = reinterpret_cast<const IO*>(a.B) + brow;
+    ln.tC = reinterpret_cast<const IO*>(a.C) + brow;
+  }
+  ln.xs = xs;
   ln.slot = slot;
   ln.q = q;
   ln.t_end = t_end;
@@ -640,8 +771,11 @@ __device__ __forceinline__ void fwd_body(const FwdArgs& a) {
   const float bias = a.dt_bias ? a.dt_bias[dd] : 0.f;
   WarpTile<LPC>& tile = tiles[wib];
 
+  // channels-last scratch (element instantiations): 6 tiles of 16 x 16 per warp after the tiles
+  IO* xs = VEC ? nullptr
+               : reinterpret_cast<IO*>(tiles + (blockDim.x >> 5)) + (size_t)wib * kClScratch;
   run_chunk<IO, VEC, MODE, LPC, KE, KO, REV>(a, tile, hh, al, ra, Dd, bias, lane, slot, q, b, gbc,
-                                             act, ch, t_begin, t_end, last_chunk);
+                                             act, ch, t_begin, t_end, last_chunk, xs);
 }
 
 // The kernel, compiled for two register budgets.  fwd_kernel leaves the choice to the compiler
@@ -662,7 +796,8 @@ __global__ void __launch_bounds__(128, 1) fwd_kernel_wide(const FwdArgs a) {
 
 template <typename IO, bool VEC, int MODE, int LPC, int KE, int KO, bool REV, bool WIDE = false>
 void launch_one(const FwdArgs& a, dim3 grid, dim3 block, cudaStream_t s) {
-  const size_t smem = (size_t)(block.x / 32) * sizeof(WarpTile<LPC>);
+  const size_t smem =
+      (size_t)(block.x / 32) * (sizeof(WarpTile<LPC>) + (VEC ? 0 : kClScratch * sizeof(IO)));
   auto k = WIDE ? fwd_kernel_wide<IO, VEC, MODE, LPC, KE, KO, REV>
                 : fwd_kernel<IO, VEC, MODE, LPC, KE, KO, REV>;
   if (smem > 48 * 1024)

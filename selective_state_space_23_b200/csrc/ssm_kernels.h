@@ -47,6 +47,7 @@ struct FwdArgs {
   int zoh;              // zero-order-hold input term (e^{ΔA} - 1)/A B x instead of Δ B x
   int bc_groups;        // B, C are [batch][bc_groups][N][L]; channel d uses group d / (dim / bc_groups)
   int channels_last;    // u, delta, z, out are [batch][L][dim] and B, C [batch][L][bc_groups][N]
+  int cl_tile;          // channels-last rows moved as 16-byte tiles (dim % 16 == 0, N == 16, aligned)
   int lpc;              // lanes per channel: 1, 2 or 4 (16 / lpc states each)
   int wide;             // few warps per SM: the 255-register form of the output kernel
   int warps_per_b;      // ceil(dim / (32 / lpc))

@@ -146,25 +146,27 @@ __device__ __forceinline__ void load_steps(Row<IO, E>& r, const IO* row, int L, 
 template <typename IO, int E, bool VEC>
 __device__ __forceinline__ void store_steps(IO* row, const float (&o)[E], int L, int tau, int nvalid,
                                             bool rev, long long ts = 1) {
-  if (VEC || ts == 1) {
+  if constexpr (VEC) {
     if (!rev) {
-      store_row<IO, E, VEC>(row + tau, o, nvalid);
-      return;
-    }
-    if (VEC) {
+      store_row<IO, E, true>(row + tau, o, nvalid);
+    } else {
       float rv[E];
 #pragma unroll
       for (int e = 0; e < E; ++e) rv[e] = o[E - 1 - e];
       store_row<IO, E, true>(row + ((long long)L - tau - E), rv, E);
+    }
+  } else {
+    if (!rev && ts == 1) {
+      store_row<IO, E, false>(row + tau, o, nvalid);
       return;
     }
-  }
 #pragma unroll
-  for (int e = 0; e < E; ++e) {
-    if (e < nvalid) {
-      const long long i = (rev ? (long long)L - 1 - tau - e : (long long)tau + e) * ts;
-      if (sizeof(IO) == 4) reinterpret_cast<float*>(row)[i] = o[e];
-      else reinterpret_cast<uint16_t*>(row)[i] = f32_to_bf16(o[e]);
+    for (int e = 0; e < E; ++e) {
+      if (e < nvalid) {
+        const long long i = (rev ? (long long)L - 1 - tau - e : (long long)tau + e) * ts;
+        if (sizeof(IO) == 4) reinterpret_cast<float*>(row)[i] = o[e];
+        else reinterpret_cast<uint16_t*>(row)[i] = f32_to_bf16(o[e]);
+      }
     }
   }
 }
