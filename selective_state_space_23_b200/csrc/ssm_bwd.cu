@@ -54,6 +54,7 @@ struct BwdTile {
   float red[32 * kRedS];       // dB/dC values of two steps, transposed to sum over channels
   float wres[kBlk * 32];       // the warp's channel sums [step][half * 16 + (dB n | dC n)]
 };
+static_assert(sizeof(BwdTile) % 16 == 0, "per-warp tiles keep 16-byte alignment");
 
 // Ā and the ZOH coefficient c = (e^{ΔA} - 1)/A of two states: library expf/expm1f on the fp32
 // path, the FMA-pipe form (zoh_coef_x2) on the bf16 path.  al = A (fp32) or A log2 e (bf16).
@@ -265,6 +266,84 @@ __device__ __forceinline__ void half_pass(BwdTile& tl, const float2 (&hstart)[4]
   }
 }
 
+// ---- channels-last tiles (element instantiations): lane l moves scan step l/2 of 8 consecutive
+// channels (or B/C states) with one 16-byte access (two for fp32), and a per-warp 16 x 16 scratch
+// tile, reused for every operand, turns the warp's [16 steps][16 columns] tile into per-lane rows
+// (column l/2, steps 8 (l & 1) .. + 7) and back.
+constexpr int kClTile = 256;  // elements of the scratch tile, [column][step]
+
+template <typename IO>
+__device__ __forceinline__ void cl_load_piece(Row<IO, kHB>& w, const IO* base, long long stride,
+                                              long long tr, bool ok) {
+  if (!ok) {
+    w.zero();
+    return;
+  }
+  const uint4* p = reinterpret_cast<const uint4*>(base + tr * stride);
+#pragma unroll
+  for (int i = 0; i < Row<IO, kHB>::kWords / 4; ++i) {
+    const uint4 v = __ldcs(p + i);
+    w.w[4 * i] = v.x; w.w[4 * i + 1] = v.y; w.w[4 * i + 2] = v.z; w.w[4 * i + 3] = v.w;
+  }
+}
+
+template <typename IO>
+__device__ __forceinline__ void cl_transpose_in(Row<IO, kHB>& w, IO* T, int lane) {
+  const int st = lane >> 1, h = lane & 1;
+#pragma unroll
+  for (int e = 0; e < kHB; ++e) {
+    if (sizeof(IO) == 4) reinterpret_cast<uint32_t*>(T)[(8 * h + e) * 16 + st] = w.w[e];
+    else reinterpret_cast<uint16_t*>(T)[(8 * h + e) * 16 + st] = (uint16_t)(w.w[e >> 1] >> (16 * (e & 1)));
+  }
+  __syncwarp();
+  const uint4* p = reinterpret_cast<const uint4*>(T + st * 16 + 8 * h);
+#pragma unroll
+  for (int i = 0; i < Row<IO, kHB>::kWords / 4; ++i) {
+    const uint4 v = p[i];
+    w.w[4 * i] = v.x; w.w[4 * i + 1] = v.y; w.w[4 * i + 2] = v.z; w.w[4 * i + 3] = v.w;
+  }
+  __syncwarp();  // the tile is free for the next operand
+}
+
+// The lane's row (column lane/2, steps 8 (lane & 1) .. + 7) goes out as step `st` of its 8
+// columns; ok: that step exists; tr: its time row.
+template <typename IO>
+__device__ __forceinline__ void cl_store_piece(IO* base, long long stride, const float (&o)[kHB],
+                                               IO* T, int lane, long long tr, bool ok) {
+  const int st = lane >> 1, h = lane & 1;
+  __syncwarp();  // the scratch's previous reads are done
+  {
+    uint32_t rw[Row<IO, kHB>::kWords];
+#pragma unroll
+    for (int i = 0; i < Row<IO, kHB>::kWords; ++i)
+      rw[i] = sizeof(IO) == 4 ? __float_as_uint(o[i]) : pack_bf16x2(o[2 * i], o[2 * i + 1]);
+    uint4* p = reinterpret_cast<uint4*>(T + st * 16 + 8 * h);
+#pragma unroll
+    for (int i = 0; i < Row<IO, kHB>::kWords / 4; ++i)
+      p[i] = make_uint4(rw[4 * i], rw[4 * i + 1], rw[4 * i + 2], rw[4 * i + 3]);
+  }
+  __syncwarp();
+  uint32_t wv[Row<IO, kHB>::kWords];
+#pragma unroll
+  for (int e = 0; e < kHB; ++e) {
+    uint32_t v;
+    if (sizeof(IO) == 4) v = reinterpret_cast<const uint32_t*>(T)[(8 * h + e) * 16 + st];
+    else v = reinterpret_cast<const uint16_t*>(T)[(8 * h + e) * 16 + st];
+    if (sizeof(IO) == 4) wv[e] = v;
+    else if (e & 1) wv[e >> 1] |= v << 16;
+    else wv[e >> 1] = v;
+  }
+  if (!ok) return;
+  uint4* p = reinterpret_cast<uint4*>(base + tr * stride);
+#pragma unroll
+  for (int i = 0; i < Row<IO, kHB>::kWords / 4; ++i)
+    __stcs(p + i, make_uint4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]));
+}
+
+__device__ __forceinline__ bool al16p(const void* p) {
+  return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15) == 0;
+}
+
 template <typename IO, bool VEC, int KP>
 __global__ void __launch_bounds__(128) bwd_kernel(const BwdArgs a) {
   constexpr bool kPrecise = std::is_same<IO, float>::value;
@@ -323,6 +402,15 @@ __global__ void __launch_bounds__(128) bwd_kernel(const BwdArgs a) {
                              : (((long long)b * a.bc_groups + gbc) * N + (bc_live ? slot : 0)) * L;
   const IO* Bp = reinterpret_cast<const IO*>(a.B) + bcrow;
   const IO* Cp = reinterpret_cast<const IO*>(a.C) + bcrow;
+  // channels-last tiles: the warp's 16 channels all exist, N == 16, every time row 16-byte aligned
+  const bool clt = !VEC && cl && a.dim % kCW == 0 && (grp * a.wpb + wib + 1) * kCW <= a.dim &&
+                   N == kNS && (a.dim * sizeof(IO)) % 16 == 0 &&
+                   al16p(a.u) && al16p(a.delta) && al16p(a.z) && al16p(a.dout) && al16p(a.du) &&
+                   al16p(a.ddelta) && al16p(a.dz) && al16p(a.B) && al16p(a.C);
+  IO* xs = VEC ? nullptr
+               : reinterpret_cast<IO*>(tiles + (blockDim.x >> 5)) + (size_t)wib * kClTile;
+  const long long xrow = (long long)b * L * a.dim + (grp * a.wpb + wib) * kCW + 8 * (lane & 1);
+  const long long xbc = ((long long)b * L * a.bc_groups + gbc) * N + 8 * (lane & 1);
   float* sBw = reinterpret_cast<float*>(tl.sB);
   float* sCw = reinterpret_cast<float*>(tl.sC);
 
@@ -337,13 +425,32 @@ __global__ void __launch_bounds__(128) bwd_kernel(const BwdArgs a) {
       load_steps<IO, kHB, true>(rd, dp, L, tq, kHB, rev);
       load_steps<IO, kHB, true>(rg, gp, L, tq, kHB, rev);
       if (zp) load_steps<IO, kHB, true>(rz, zp, L, tq, kHB, rev);
+    } else if (clt) {
+      const int st = lane >> 1;
+      const bool ok = st < nvalid;
+      const long long tr = rev ? (long long)L - 1 - (t0 + st) : (long long)(t0 + st);
+      cl_load_piece<IO>(ru, reinterpret_cast<const IO*>(a.u) + xrow, a.dim, tr, ok);
+      cl_load_piece<IO>(rd, reinterpret_cast<const IO*>(a.delta) + xrow, a.dim, tr, ok);
+      cl_load_piece<IO>(rg, reinterpret_cast<const IO*>(a.dout) + xrow, a.dim, tr, ok);
+      if (zp) cl_load_piece<IO>(rz, reinterpret_cast<const IO*>(a.z) + xrow, a.dim, tr, ok);
+      cl_load_piece<IO>(rb, reinterpret_cast<const IO*>(a.B) + xbc, ts_bc, tr, ok);
+      cl_load_piece<IO>(rc, reinterpret_cast<const IO*>(a.C) + xbc, ts_bc, tr, ok);
+      __syncwarp();  // the scratch's previous reads are done
+      cl_transpose_in<IO>(ru, xs, lane);
+      cl_transpose_in<IO>(rd, xs, lane);
+      cl_transpose_in<IO>(rg, xs, lane);
+      if (zp) cl_transpose_in<IO>(rz, xs, lane);
+      cl_transpose_in<IO>(rb, xs, lane);
+      cl_transpose_in<IO>(rc, xs, lane);
     } else {
       load_steps<IO, kHB, false>(ru, up, L, tq, nown, rev, ts_x);
       load_steps<IO, kHB, false>(rd, dp, L, tq, nown, rev, ts_x);
       load_steps<IO, kHB, false>(rg, gp, L, tq, nown, rev, ts_x);
       if (zp) load_steps<IO, kHB, false>(rz, zp, L, tq, nown, rev, ts_x);
     }
-    if (!bc_live) {
+    if (clt) {
+      // B/C rows came with the tile
+    } else if (!bc_live) {
       rb.zero();
       rc.zero();
     } else if (VEC && nown == kHB) {
@@ -437,7 +544,15 @@ __global__ void __launch_bounds__(128) bwd_kernel(const BwdArgs a) {
         dbias_acc += odd[j];
       }
     }
-    if (act && nown > 0) {
+    if (clt) {  // every lane takes part: the tiles go out through the scratch
+      const int st = lane >> 1;
+      const bool ok = st < nvalid;
+      const long long tr = rev ? (long long)L - 1 - (t0 + st) : (long long)(t0 + st);
+      IO* T = xs;
+      if (a.du) cl_store_piece<IO>(reinterpret_cast<IO*>(a.du) + xrow, a.dim, odu, T, lane, tr, ok);
+      if (a.ddelta) cl_store_piece<IO>(reinterpret_cast<IO*>(a.ddelta) + xrow, a.dim, odd, T, lane, tr, ok);
+      if (a.dz && zp) cl_store_piece<IO>(reinterpret_cast<IO*>(a.dz) + xrow, a.dim, odz, T, lane, tr, ok);
+    } else if (act && nown > 0) {
       const auto put = [&](void* base, const float (&v)[kHB]) {
         IO* o = reinterpret_cast<IO*>(base) + row;
         if (VEC && nown == kHB) store_steps<IO, kHB, true>(o, v, L, tq, kHB, rev);
@@ -528,7 +643,10 @@ __global__ void bwd_finish_adt(const BwdArgs a, float* dA, float* dD, float* ddt
 template <typename IO, bool VEC>
 cudaError_t launch_bwd_io(const BwdArgs& a, cudaStream_t s) {
   const dim3 grid((unsigned)(a.batch * a.ngroups)), block(32 * a.wpb);
-  const size_t smem = sizeof(BwdTile) * a.wpb;
+  // the channels-last scratch tile exists only in channels-last launches (the kernel's tile test
+  // requires the layout flag)
+  const size_t smem =
+      (sizeof(BwdTile) + (!VEC && a.channels_last ? kClTile * sizeof(IO) : 0)) * a.wpb;
   auto k = bwd_kernel<IO, VEC, 2>;
   if (a.zoh) {
     k = bwd_kernel<IO, VEC, kKpZoh>;  // ZOH coefficient on the FMA pipe

@@ -85,12 +85,17 @@ def test_forward_variants_equal_default_layout(monkeypatch, reverse, zoh, groups
     assert torch.equal(a.transpose(1, 2), b)
 
 
-@pytest.mark.parametrize("io,L,use_ckpt", [(torch.float32, 333, False), (torch.bfloat16, 256, True),
-                                           (torch.bfloat16, 101, False)])
-def test_backward(io, L, use_ckpt):
-    w = workload("tiny_f32", batch=2, dim=80, seqlen=L, io_dtype=io)
+# dim a multiple of 16 with N = 16 takes the 16-byte tile loads and stores; dim = 72 or N = 5
+# takes the element-stride path
+@pytest.mark.parametrize("io,dim,N,L,use_ckpt", [(torch.float32, 80, 16, 333, False),
+                                                 (torch.bfloat16, 80, 16, 256, True),
+                                                 (torch.bfloat16, 80, 16, 101, False),
+                                                 (torch.bfloat16, 72, 16, 101, False),
+                                                 (torch.float32, 80, 5, 64, False)])
+def test_backward(io, dim, N, L, use_ckpt):
+    w = workload("tiny_f32", batch=2, dim=dim, seqlen=L, dstate=N, io_dtype=io)
     x = make_inputs(w, seed=74, with_dout=True, with_h0=True)
-    dhL = torch.randn((2, 80, 16), generator=torch.Generator().manual_seed(13))
+    dhL = torch.randn((2, dim, N), generator=torch.Generator().manual_seed(13))
     xc = on_dev(to_cl(x))
     ck = None
     if use_ckpt:
@@ -123,6 +128,25 @@ def test_backward_grouped_reverse_zoh_equals_default_layout():
                           z=xd["z"], dt_bias=xd["dt_bias"], h0=xd["h0"], **kw)
     gc = ssm.ssm_scan_bwd(xc["u"], xc["delta"], xc["A"], xc["B"], xc["C"], xc["dout"], D=xc["D"],
                           z=xc["z"], dt_bias=xc["dt_bias"], h0=xc["h0"], channels_last=True, **kw)
+    for k in GRADS:
+        a = gc[k]
+        if k in ("du", "ddelta", "dz"):
+            a = a.transpose(1, 2)
+        elif k in ("dB", "dC"):
+            a = from_cl_bc(a)
+        assert torch.equal(a, gd[k]), k
+
+
+@pytest.mark.parametrize("io,dim,L", [(torch.bfloat16, 48, 77), (torch.float32, 48, 16),
+                                      (torch.bfloat16, 32, 1)])
+def test_backward_tiles_equal_default_layout(io, dim, L):
+    w = workload("tiny_f32", batch=3, dim=dim, seqlen=L, io_dtype=io)
+    x = make_inputs(w, seed=77, with_dout=True, with_h0=True)
+    xd, xc = on_dev(x), on_dev(to_cl(x))
+    gd = ssm.ssm_scan_bwd(xd["u"], xd["delta"], xd["A"], xd["B"], xd["C"], xd["dout"], D=xd["D"],
+                          z=xd["z"], dt_bias=xd["dt_bias"], h0=xd["h0"])
+    gc = ssm.ssm_scan_bwd(xc["u"], xc["delta"], xc["A"], xc["B"], xc["C"], xc["dout"], D=xc["D"],
+                          z=xc["z"], dt_bias=xc["dt_bias"], h0=xc["h0"], channels_last=True)
     for k in GRADS:
         a = gc[k]
         if k in ("du", "ddelta", "dz"):
