@@ -477,7 +477,12 @@ def main():
         cb_desc = "skipped (--no-baseline)"
     else:
         cb_value, cb_cores, cb_desc, _ = oracle_sample_time(w, seed=0)
-    extras = {} if args.no_extras else bench_extras(dev)
+    extras = {}
+    if not args.no_extras:
+        try:  # side measurements: a failure here is reported, it does not cost the main line
+            extras = bench_extras(dev)
+        except Exception as e:  # noqa: BLE001
+            extras = {"error": f"{type(e).__name__}: {e}"[:300]}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
