@@ -1,5 +1,7 @@
-"""Multi-process host logic on CPU (gloo, world size 2): batch sharding needs no exchange (the
-oracle on each rank's rows reproduces the whole batch), and timing reduces to the max over ranks."""
+"""Multi-process host logic on CPU (gloo, world size 2): batch sharding needs no exchange in the
+forward (the oracle on each rank's rows reproduces the whole batch), the backward's parameter
+gradients are the all-reduced sums of the ranks' partial gradients, and timing reduces to the
+max over ranks."""
 import os
 import socket
 
@@ -9,7 +11,8 @@ import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
-from selective_state_space_23_b200.dist import barrier, max_over_ranks, shard_rows
+from selective_state_space_23_b200.dist import (allreduce_param_grads, barrier, max_over_ranks,
+                                                shard_rows)
 
 
 def test_shard_rows_partition():
@@ -83,3 +86,71 @@ def test_two_ranks_shard_without_exchange_and_time_is_max():
 
 def test_max_over_ranks_single_process():
     assert max_over_ranks(3.25) == 3.25
+
+
+BWD_SHAPE = dict(batch=5, dim=6, seqlen=37, dstate=4)
+
+
+def _bwd_inputs():
+    from selective_state_space_23_b200.inputs import make_inputs, to_f64, workload
+    w = workload("tiny_f32", **BWD_SHAPE)
+    return {k: to_f64(v) for k, v in make_inputs(w, seed=5, with_h0=True, with_dout=True).items()}
+
+
+def _bwd(oracle, x, b0, b1):
+    sl = lambda k: x[k][b0:b1]
+    return oracle.scan_bwd(sl("u"), sl("delta"), x["A"], sl("B"), sl("C"), sl("dout"), D=x["D"],
+                           z=sl("z"), dt_bias=x["dt_bias"], h0=sl("h0"), nthreads=1)
+
+
+def _bwd_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import oracle
+        x = _bwd_inputs()
+        b0, b1 = shard_rows(BWD_SHAPE["batch"], world, rank)
+        g = _bwd(oracle, x, b0, b1)
+        part = {k: torch.from_numpy(np.ascontiguousarray(g[k])) for k in ("dA", "dD", "ddt_bias")}
+        before = {k: v.clone() for k, v in part.items()}
+        allreduce_param_grads(part)
+        rows = {k: g[k] for k in ("du", "ddelta", "dz", "dB", "dC", "dh0")}
+        q.put((rank, (b0, b1), {k: v.numpy() for k, v in part.items()},
+               {k: v.numpy() for k, v in before.items()}, rows))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_backward_param_grads_allreduced():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_bwd_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    res.sort(key=lambda r: r[0])
+    import oracle
+    x = _bwd_inputs()
+    full = _bwd(oracle, x, 0, BWD_SHAPE["batch"])
+    for k in ("dA", "dD", "ddt_bias"):
+        # every rank holds the whole-batch gradient, and it is the sum of the two partials
+        for r in res:
+            np.testing.assert_allclose(r[2][k], full[k], rtol=1e-12, atol=1e-12)
+        np.testing.assert_array_equal(res[0][2][k], res[1][2][k])
+        np.testing.assert_array_equal(res[0][2][k], res[0][3][k] + res[1][3][k])
+        # a rank's partial alone is not the whole-batch gradient
+        assert not np.allclose(res[0][3][k], full[k])
+    # the row gradients need no exchange: each rank's rows are the whole batch's rows
+    for k in ("du", "ddelta", "dz", "dB", "dC", "dh0"):
+        got = np.concatenate([r[4][k] for r in res], 0)
+        np.testing.assert_array_equal(got, full[k])
+
+
+def test_allreduce_param_grads_without_group_is_identity():
+    g = {"dA": torch.ones(3, 2), "dD": None}
+    out = allreduce_param_grads(g)
+    assert out is g and torch.equal(g["dA"], torch.ones(3, 2)) and g["dD"] is None
