@@ -191,8 +191,11 @@ SSM_API int ssm_scan_bwd_scalar_a(const void* u, const void* delta, const float*
  *                 Combines with the other flags.
  *   SSM_CHANNELS_LAST  the (B, L, D) layout: u, delta, z, out, dout, du, ddelta, dz are
  *                 [batch][L][dim] and B, C, dB, dC are [batch][L][bc_groups][dstate] (the
- *                 projections' own output layout), read and written with element accesses;
- *                 everything else as above.
+ *                 projections' own output layout); everything else as above.  With
+ *                 dim % 16 == 0, dstate == 16 and 16-byte aligned tensors each warp moves
+ *                 16-byte pieces (8 consecutive channels or states of one step) and transposes
+ *                 them through shared memory; otherwise it uses element accesses (slower, same
+ *                 results).
  * Any other bit is rejected with SSM_EINVAL.  Arguments are those of ssm_scan_fwd /
  * ssm_scan_bwd plus flags and bc_groups:
  *   bc_groups     B, C (and dB, dC) are [batch][bc_groups][dstate][L]: the per-token B_t, C_t
