@@ -58,6 +58,15 @@ def _opt(t, name, shape, dtype, device):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _on_gpu(t, name):
+    """The tensor's device, which must be a CUDA device (the library has no host path)."""
+    if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+        where = t.device if isinstance(t, torch.Tensor) else type(t).__name__
+        raise ValueError(f"{name} must be a CUDA tensor, got {where} (host tensors: "
+                         "ssm_scan_fwd_host)")
+    return t.device
+
+
 def _io_code(dtype):
     if dtype not in _IO:
         raise TypeError(f"io dtype must be float32 or bfloat16, got {dtype}")
@@ -108,7 +117,7 @@ def _flags(scalar_a, reverse, zoh, channels_last=False):
 
 def _scan_fwd(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, return_final_state,
               return_ckpt, out, workspace, scalar_a, reverse, zoh, channels_last=False):
-    dev = u.device
+    dev = _on_gpu(u, "u")
     if channels_last:
         batch, L, dim = u.shape
     else:
@@ -172,7 +181,7 @@ def ssm_scan_fwd_scalar_a(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta
 
 def _scan_bwd(u, delta, A, B, C, dout, D, z, dt_bias, delta_softplus, h0, dhL, ckpt,
               workspace, need, scalar_a, reverse, zoh, channels_last=False):
-    dev = u.device
+    dev = _on_gpu(u, "u")
     if channels_last:
         batch, L, dim = u.shape
     else:
@@ -257,7 +266,7 @@ def ssm_scan_fwd_host(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta_sof
     through copy-in, scan and copy-out streams in chunks of rows.  Returns out (CPU), or
     (out, hL) with ``return_final_state``; both are complete once the current stream of A's
     device has reached this call."""
-    dev = A.device
+    dev = _on_gpu(A, "A")
     batch, dim, L = u.shape
     N = A.shape[-1]
     io = u.dtype
@@ -294,7 +303,7 @@ def ssm_state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, delta_
     """One decode step; ``state`` [batch, dim, N] f32 is updated in place.  x, dt, z:
     [batch, dim]; B, C: [batch, N] or, grouped, [batch, G, N] (io dtype); A: [dim, N] f32, or
     [dim] with ``scalar_a``; ``zoh``: zero-order-hold input coefficient.  Returns out [batch, dim]."""
-    dev = state.device
+    dev = _on_gpu(state, "state")
     batch, dim, N = state.shape
     io = x.dtype
     code = _io_code(io)

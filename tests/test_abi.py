@@ -155,3 +155,25 @@ def test_host_memory_call_checks_shape_and_workspace(lib):
     rc = lib.ssm_scan_fwd_host(None, p, None, p, p, None, None, None, 1, None, None, p, None, 0,
                                8, 2048, 2048, 16, 1, None)
     assert rc == _abi.SSM_EINVAL
+
+
+def test_binding_rejects_host_tensors_before_any_cuda_call():
+    """The Python entry points refuse CPU tensors with a ValueError of their own (they never
+    reach the CUDA runtime or the library with a host pointer)."""
+    import torch
+    import selective_state_space_23_b200 as ssm
+    from selective_state_space_23_b200.inputs import make_inputs, workload
+    x = make_inputs(workload("tiny_f32"), seed=0, with_dout=True)
+    calls = {
+        "fwd": lambda: ssm.ssm_scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"]),
+        "fwd_cl": lambda: ssm.ssm_scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"],
+                                           channels_last=True),
+        "bwd": lambda: ssm.ssm_scan_bwd(x["u"], x["delta"], x["A"], x["B"], x["C"], x["dout"]),
+        "decode": lambda: ssm.ssm_state_update(torch.zeros(1, 64, 16), x["u"][:, :, 0],
+                                               x["delta"][:, :, 0], x["A"], x["B"][:, :, 0],
+                                               x["C"][:, :, 0]),
+        "host": lambda: ssm.ssm_scan_fwd_host(x["u"], x["delta"], x["A"], x["B"], x["C"]),
+    }
+    for name, f in calls.items():
+        with pytest.raises(ValueError, match="must be a CUDA tensor"):
+            f()
