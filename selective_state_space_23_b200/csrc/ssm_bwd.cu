@@ -266,7 +266,7 @@ __device__ __forceinline__ void half_pass(BwdTile& tl, const float2 (&hstart)[4]
   }
 }
 
-// ---- channels-last tiles (element instantiations): lane l moves scan step l/2 of 8 consecutive
+// ---- channels-last tiles (the kernel's VEC = false forms): lane l moves step l/2 of 8 consecutive
 // channels (or B/C states) with one 16-byte access (two for fp32), and a per-warp 16 x 16 scratch
 // tile, reused for every operand, turns the warp's [16 steps][16 columns] tile into per-lane rows
 // (column l/2, steps 8 (l & 1) .. + 7) and back.
