@@ -202,6 +202,32 @@ def oracle_sample_time(w, seed: int, target_s: float = 3.0):
     return w.tokens / full_s, cores, desc, dt
 
 
+def oracle_single_core(w, seed: int, nd: int = 256):
+    """The same oracle on one thread over an nd-channel sample: (tokens/s extrapolated, sample)."""
+    import oracle
+    x = make_inputs(w, seed=seed)
+    sel = np.arange(min(nd, w.dim))
+    f = {k: v.to(torch.float64).numpy() for k, v in x.items()}
+    t0 = time.perf_counter()
+    oracle.scan_fwd(f["u"][:, sel], f["delta"][:, sel], f["A"][sel], f["B"], f["C"],
+                    D=f["D"][sel], z=f["z"][:, sel], dt_bias=f["dt_bias"][sel], nthreads=1)
+    dt = time.perf_counter() - t0
+    return w.tokens / (dt * w.dim / len(sel)), (f"1 thread, {w.batch}x{len(sel)} channels "
+                                                f"({dt:.2f} s), extrapolated by channel count")
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for ln in fh:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
@@ -472,13 +498,15 @@ def main():
     alu_peak = alu_peak_elems_per_s(sms, peaks["sm_max_mhz"])
     alu_ach = elems / (kern_ms * 1e-3)
     traffic = recorded_traffic()
-    if args.no_baseline:
+    if args.no_baseline or world > 1:
         cb_value = cb_cores = None
-        cb_desc = "skipped (--no-baseline)"
+        cb_desc = "skipped (--no-baseline)" if args.no_baseline else "timed at N=1 only"
+        sc_value, sc_desc = None, cb_desc
     else:
         cb_value, cb_cores, cb_desc, _ = oracle_sample_time(w, seed=0)
-    extras = {}
-    if not args.no_extras:
+        sc_value, sc_desc = oracle_single_core(w, seed=0)
+    extras = {} if world == 1 else {"skipped": "the side measurements run at N=1 only"}
+    if not args.no_extras and world == 1:
         try:  # side measurements: a failure here is reported, it does not cost the main line
             extras = bench_extras(dev)
         except Exception as e:  # noqa: BLE001
@@ -502,7 +530,8 @@ def main():
                              "bytes_per_launch": byts},
                      "kernel_ms": kern_ms},
         "cpu_baseline": {"value": cb_value, "unit": UNIT, "cores": cb_cores, "kind": "oracle",
-                         "sample": cb_desc},
+                         "sample": cb_desc, "cpu_model": cpu_model(),
+                         "single_core": {"value": sc_value, "unit": UNIT, "sample": sc_desc}},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},
         "gpu_launches": K * launches_per_step,
