@@ -5,7 +5,8 @@ Every test builds its expected value independently (a different formula or libra
     page, Hydra notes: sequence mixing of an SSM is a structured, data-dependent matrix;
   * closed forms: L = 1, the geometric series for constant inputs, the LTI causal convolution
     (mamba-minimal news page: a time-invariant SSM can run as one global convolution);
-  * the gating special case of the "Seçim Mekanizması (S6)" section (N=1, A=-1, B=1);
+  * the gating special case of the "Seçim Mekanizması (S6)" section (N=1, A=-1, B=1), and the
+    ZOH input term against the hold integral of the "Yöntem" discretisation (Gauss-Legendre);
   * the Δ limits of the "Sorular" section (small Δ keeps the state, large Δ resets it);
   * chunked-vs-sequential state passing, superposition, decode-vs-scan;
   * the scalar decay (one A per channel, the Mamba-2 restriction in the reading-list notes) as
@@ -155,6 +156,48 @@ def test_gating_reduction():
             h = (1 - g[t]) * h + inp
             ref.append(h)
         np.testing.assert_allclose(res["out"][0, 0], ref, rtol=1e-12, atol=1e-14)
+
+
+def hold_integral(dt, a, nodes=24):
+    """Zero-order hold of a diagonal entry: the integral of exp(a tau) over tau in [0, dt],
+    by Gauss-Legendre quadrature (not the closed form (exp(a dt) - 1)/a)."""
+    x, w = np.polynomial.legendre.leggauss(nodes)
+    tau = 0.5 * dt * (x + 1.0)
+    return 0.5 * dt * np.sum(w * np.exp(a * tau))
+
+
+def test_zoh_quadratic_form_from_the_hold_integral():
+    """With the ZOH input term ("Yöntem": B̄ = (ΔA)^{-1}(exp(ΔA) - I) ΔB, i.e. the input held
+    constant over the step and integrated through exp(A tau)), every output is
+    y_t = sum_{s<=t} C_t . (prod_{r=s+1..t} exp(Δ_r A)) (int_0^{Δ_s} exp(A tau) dtau) B_s u_s
+          + C_t . (prod_{r<=t} exp(Δ_r A)) h0 + D u_t, gated.  A holds an exact zero and a
+    tiny rate, where the hold integral is Δ."""
+    c = rand_case(batch=2, dim=3, L=8, N=3, seed=21)
+    c["A"][0, 0] = 0.0
+    c["A"][1, 1] = -1e-9
+    u, A, B, C = c["u"], c["A"], c["B"], c["C"]
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    dt = softplus_ref(c["delta"] + c["dt_bias"][None, :, None])
+    want = np.zeros_like(u)
+    for b in range(batch):
+        for d in range(dim):
+            cs = np.concatenate([[0.0], np.cumsum(dt[b, d])])
+            hold = np.array([[hold_integral(dt[b, d, s], A[d, n]) for n in range(N)]
+                             for s in range(L)])                      # [s, n]
+            for t in range(L):
+                y = 0.0
+                for s in range(t + 1):
+                    decay = np.exp(A[d] * (cs[t + 1] - cs[s + 1]))
+                    y += np.sum(C[b, :, t] * decay * hold[s] * B[b, :, s]) * u[b, d, s]
+                y += np.sum(C[b, :, t] * np.exp(A[d] * cs[t + 1]) * c["h0"][b, d])
+                y += c["D"][d] * u[b, d, t]
+                zz = c["z"][b, d, t]
+                want[b, d, t] = y * zz * expit(zz)
+    got = run(c, zoh=True)["out"]
+    np.testing.assert_allclose(got, want, rtol=1e-11, atol=1e-12)
+    # and the Euler input term differs from it (the two forms are not confused)
+    assert not np.allclose(run(c)["out"], want, rtol=1e-6, atol=1e-8)
 
 
 def test_delta_limits():
