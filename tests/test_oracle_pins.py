@@ -499,6 +499,38 @@ def test_grouped_bc_gradients_by_finite_differences():
         np.testing.assert_allclose(g[gname], num, rtol=2e-6, atol=2e-7, err_msg=gname)
 
 
+def test_combined_variants_gradients_by_finite_differences():
+    """Reverse scan, ZOH input term and grouped B/C at once (the variants compose in the
+    oracle's wrappers): every gradient against central differences of the same forward."""
+    c = rand_case(batch=1, dim=4, L=5, N=2, seed=91)
+    r = np.random.default_rng(92)
+    c["B"] = r.standard_normal((1, 2, 2, 5))
+    c["C"] = r.standard_normal((1, 2, 2, 5))
+    c["A"][2, 0] = 0.0                     # the A -> 0 limit of the ZOH coefficient
+    dout = r.standard_normal(c["u"].shape)
+    dhL = r.standard_normal(c["h0"].shape)
+    kw = dict(reverse=True, zoh=True)
+    g = oracle.scan_bwd(c["u"], c["delta"], c["A"], c["B"], c["C"], dout, D=c["D"], z=c["z"],
+                        dt_bias=c["dt_bias"], h0=c["h0"], dhL=dhL, **kw)
+
+    def loss(cc):
+        res = run(cc, **kw)
+        return np.sum(res["out"] * dout) + np.sum(res["hL"] * dhL)
+
+    eps = 1e-6
+    for key, gname in (("u", "du"), ("delta", "ddelta"), ("A", "dA"), ("B", "dB"), ("C", "dC"),
+                       ("D", "dD"), ("z", "dz"), ("dt_bias", "ddt_bias"), ("h0", "dh0")):
+        x = c[key]
+        num = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            i = it.multi_index
+            xp = x.copy(); xp[i] += eps
+            xm = x.copy(); xm[i] -= eps
+            num[i] = (loss(dict(c, **{key: xp})) - loss(dict(c, **{key: xm}))) / (2 * eps)
+        np.testing.assert_allclose(g[gname], num, rtol=2e-6, atol=2e-7, err_msg=gname)
+
+
 def test_planted_mistake_is_caught():
     """A plausible oracle mistake (reading out h_{t-1} instead of h_t) must fail the pins:
     emulate it by shifting the readout and check the quadratic form tells the two apart."""
