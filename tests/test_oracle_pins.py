@@ -499,6 +499,39 @@ def test_grouped_bc_gradients_by_finite_differences():
         np.testing.assert_allclose(g[gname], num, rtol=2e-6, atol=2e-7, err_msg=gname)
 
 
+def test_combined_variants_forward_quadratic_form():
+    """Reverse scan + ZOH input term + grouped B/C at once, against the anti-causal quadratic
+    form with the hold integral as input coefficient and each channel's group of B/C:
+    h_t = sum_{s>=t} (prod_{r=t..s-1} exp(Δ_r A)) hold(Δ_s) B_s u_s + (prod_{r>=t} exp(Δ_r A)) h0."""
+    c = rand_case(batch=2, dim=4, L=7, N=3, seed=93)
+    r = np.random.default_rng(94)
+    G = 2
+    Bg = r.standard_normal((2, G, 3, 7))
+    Cg = r.standard_normal((2, G, 3, 7))
+    c["A"][1, 2] = 0.0
+    u, A = c["u"], c["A"]
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    dt = softplus_ref(c["delta"] + c["dt_bias"][None, :, None])
+    want = np.zeros_like(u)
+    for b in range(batch):
+        for d in range(dim):
+            g = d // (dim // G)
+            B, C = Bg[b, g], Cg[b, g]                                   # [n, t]
+            cs = np.concatenate([[0.0], np.cumsum(dt[b, d])])          # cs[k] = sum_{r<k} Δ_r
+            for t in range(L):
+                h = np.exp(A[d] * (cs[L] - cs[t])) * c["h0"][b, d]
+                for s_ in range(t, L):
+                    hold = np.array([hold_integral(dt[b, d, s_], A[d, n]) for n in range(N)])
+                    h = h + np.exp(A[d] * (cs[s_] - cs[t])) * hold * B[:, s_] * u[b, d, s_]
+                y = np.sum(C[:, t] * h) + c["D"][d] * u[b, d, t]
+                zz = c["z"][b, d, t]
+                want[b, d, t] = y * zz * expit(zz)
+    got = oracle.scan_fwd(u, c["delta"], A, Bg, Cg, D=c["D"], z=c["z"], dt_bias=c["dt_bias"],
+                          h0=c["h0"], reverse=True, zoh=True)["out"]
+    np.testing.assert_allclose(got, want, rtol=1e-11, atol=1e-12)
+
+
 def test_combined_variants_gradients_by_finite_differences():
     """Reverse scan, ZOH input term and grouped B/C at once (the variants compose in the
     oracle's wrappers): every gradient against central differences of the same forward."""
