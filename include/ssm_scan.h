@@ -265,8 +265,9 @@ SSM_API int ssm_scan_fwd_host(const void* u, const void* delta, const float* A, 
  * time-split scratch comes from one static device array of SSM_NOALLOC_SCRATCH_BYTES that every
  * GPU loading the library keeps until the process exits; shapes whose plan needs more return
  * SSM_EUNSUPPORTED (ssm_last_error() says how much) and launch nothing.  No call allocates or
- * frees memory.  The first call on each device looks up the array's device address with that
- * device current; make that first call before any stream capture.  All calls on a device share
+ * frees memory.  The first call on each device (and the first after that device's context
+ * changes, e.g. after cudaDeviceReset) looks up the array's device address with that device
+ * current; make that first call before any stream capture.  All calls on a device share
  * the array: calls whose GPU work overlaps (other streams, other host threads) race on it.
  */
 SSM_API int ssm_scan_fwd_noalloc(const void* u, const void* delta, const float* A, const void* B,

@@ -29,10 +29,36 @@ static __device__ __align__(256) unsigned char g_fwd_scratch[SSM_NOALLOC_SCRATCH
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_scratch_addr[kMaxDevices] = {nullptr};
+void* g_scratch_ctx[kMaxDevices] = {nullptr};
+
+// cuCtxGetCurrent, reached through the runtime so that the library does not link libcuda.
+typedef int (*PFN_ctxGetCurrent)(void**);
+PFN_ctxGetCurrent ctx_get_current_fn() {
+  static PFN_ctxGetCurrent fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_ctxGetCurrent>(p);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
+void* current_context() {
+  void* ctx = nullptr;
+  PFN_ctxGetCurrent fn = ctx_get_current_fn();
+  if (!fn || fn(&ctx) != 0) return nullptr;
+  return ctx;
+}
 
 // Device address of the scratch array on the current device.  In host code the symbol name is
-// only a host-side handle, so the address is looked up once per device with that device
-// current and cached.
+// only a host-side handle, so the address is looked up with that device current.  It is cached
+// per device together with the context it belongs to: if the context changes (after
+// cudaDeviceReset, for instance, the module is loaded again and the array may move), or if the
+// context cannot be identified, the address is looked up again.
 int scratch_on_current_device(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -47,7 +73,8 @@ int scratch_on_current_device(void** out) {
     return SSM_EUNSUPPORTED;
   }
   std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_scratch_addr[dev]) {
+  void* ctx = current_context();
+  if (!g_scratch_addr[dev] || !ctx || ctx != g_scratch_ctx[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_fwd_scratch);
     if (e != cudaSuccess || !p) {
@@ -55,9 +82,11 @@ int scratch_on_current_device(void** out) {
       snprintf(msg, sizeof(msg), "ssm_scan_fwd_noalloc: cudaGetSymbolAddress failed: %s",
                cudaGetErrorString(e));
       ssm::set_last_error(msg);
+      g_scratch_addr[dev] = nullptr;
       return SSM_ECUDA;
     }
     g_scratch_addr[dev] = p;
+    g_scratch_ctx[dev] = current_context();  // the lookup made the device's context current
   }
   *out = g_scratch_addr[dev];
   return SSM_OK;

@@ -41,3 +41,30 @@ def assert_close(got, ref, io_dtype, name="", scale=1.0):
         m = np.max(np.abs(g - ref) / np.maximum(1.0, np.abs(ref)))
         assert m <= tol["max_abs"] * scale, f"{name}: max normalised error {m:.3e}"
     return e
+
+
+def bf16_ulp(x):
+    """Spacing of bfloat16 numbers at |x| (8 significant bits; normal range)."""
+    a = np.maximum(np.abs(np.asarray(x, dtype=np.float64)), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(a)) - 7)
+
+
+def assert_bf16_elementwise(got, ref, name="", ulps=2.0, floor_rel=1e-3):
+    """Element-wise check of a bf16 output against the unrounded fp64 oracle value:
+    |got - ref| <= ulps * ulp_bf16(ref) + floor_rel * rms(ref).
+
+    A correct kernel computes in f32 and rounds once at the store, so it lands within one bf16
+    ulp of the exact value unless f32 error flips the rounding; two ulps leave room for that.
+    The floor (a thousandth of the output's rms, a quarter of a bf16 ulp at that scale) covers
+    outputs that are small only because their terms cancel, where f32 error is absolute."""
+    g = f64(got) if isinstance(got, torch.Tensor) else np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert g.shape == ref.shape, (name, g.shape, ref.shape)
+    rms = float(np.sqrt(np.mean(ref * ref))) if ref.size else 0.0
+    bound = ulps * bf16_ulp(ref) + floor_rel * rms
+    err = np.abs(g - ref)
+    bad = err > bound
+    if bad.any():
+        i = np.unravel_index(np.argmax(err - bound), err.shape)
+        raise AssertionError(f"{name}: {int(bad.sum())} elements beyond {ulps} bf16 ulp "
+                             f"(worst at {i}: got {g[i]!r}, ref {ref[i]!r})")

@@ -285,6 +285,61 @@ def test_channel_subset_matches_full():
     assert not flat_sub[0].any()
 
 
+def _bwd(c, dout, dhL, channels=None):
+    return oracle.scan_bwd(c["u"], c["delta"], c["A"], c["B"], c["C"], dout, D=c["D"], z=c["z"],
+                           dt_bias=c["dt_bias"], h0=c["h0"], dhL=dhL, channels=channels)
+
+
+def _one_channel(c, dout, dhL, b, d):
+    """The problem restricted to the single channel (b, d): a 1 x 1 scan with that channel's
+    rows, parameters and batch row of B, C."""
+    one = dict(u=c["u"][b:b + 1, d:d + 1], delta=c["delta"][b:b + 1, d:d + 1],
+               A=c["A"][d:d + 1], B=c["B"][b:b + 1], C=c["C"][b:b + 1], D=c["D"][d:d + 1],
+               z=c["z"][b:b + 1, d:d + 1], dt_bias=c["dt_bias"][d:d + 1],
+               h0=c["h0"][b:b + 1, d:d + 1])
+    return one, dout[b:b + 1, d:d + 1], dhL[b:b + 1, d:d + 1]
+
+
+def test_backward_channel_subset():
+    """The channel-subset mode of the backward (used to check large workloads on sampled
+    channels): per-channel gradients equal the full run's; the summed gradients of one listed
+    channel equal those of the 1 x 1 problem cut out of the inputs (the unsubsetted code path on
+    a different problem); and the summed gradients of a partition of the channels add up to the
+    full run's (every channel contributes exactly its own share, once)."""
+    batch, dim, L, N = 2, 5, 9, 3
+    c = rand_case(batch=batch, dim=dim, L=L, N=N, seed=29)
+    r = np.random.default_rng(30)
+    dout = r.standard_normal((batch, dim, L))
+    dhL = r.standard_normal((batch, dim, N))
+    full = _bwd(c, dout, dhL)
+    sub_idx = [1, 7, 9]                                  # flat b * dim + d
+    sub = _bwd(c, dout, dhL, channels=sub_idx)
+    for k in ("du", "ddelta", "dz", "dh0"):
+        fs, ss = full[k].reshape(batch * dim, -1), sub[k].reshape(batch * dim, -1)
+        for ch in sub_idx:
+            np.testing.assert_array_equal(ss[ch], fs[ch], err_msg=k)
+    # one listed channel: its share equals the whole gradient of the cut-out 1 x 1 problem
+    for ch in (7, 3):
+        b, d = divmod(ch, dim)
+        g1 = _bwd(*_one_channel(c, dout, dhL, b, d))
+        gs = _bwd(c, dout, dhL, channels=[ch])
+        np.testing.assert_allclose(gs["dA"][d], g1["dA"][0], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(gs["dD"][d], g1["dD"][0], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(gs["ddt_bias"][d], g1["ddt_bias"][0], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(gs["dB"][b], g1["dB"][0], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(gs["dC"][b], g1["dC"][0], rtol=1e-12, atol=1e-14)
+        # nothing outside the listed channel's d (for dA, dD, ddt_bias) or row b (for dB, dC)
+        others = [i for i in range(dim) if i != d]
+        assert not gs["dA"][others].any() and not gs["dD"][others].any()
+        assert not gs["ddt_bias"][others].any()
+        assert not gs["dB"][1 - b].any() and not gs["dC"][1 - b].any()
+    # a partition of the channels: the shares add up to the full sums
+    rest = [i for i in range(batch * dim) if i not in sub_idx]
+    other = _bwd(c, dout, dhL, channels=rest)
+    for k in ("dA", "dB", "dC", "dD", "ddt_bias"):
+        np.testing.assert_allclose(sub[k] + other[k], full[k], rtol=1e-12, atol=1e-13, err_msg=k)
+
+
 # ------------------------------------------------------------------ gradients
 def loss_and_grads(c, dout, dhL, softplus=True, zoh=False):
     res = run(c, delta_softplus=softplus, zoh=zoh)

@@ -33,13 +33,16 @@ def _noalloc(x, out, hL, batch, dim, L, N, io_code):
 
 @pytest.mark.parametrize("io", [torch.bfloat16, torch.float32])
 def test_noalloc_matches_workspace_entry_point_twice(monkeypatch, io):
-    monkeypatch.delenv("SSM_FWD_SPLIT", raising=False)
-    batch, dim, L, N = 1, 64, 16384, 16          # few channels: the plan splits time
-    need = ssm.fwd_workspace_bytes(batch, dim, L, N, io)
-    assert 0 < need <= _abi.NOALLOC_SCRATCH_BYTES
-    w = workload("long_seq_1m", batch=batch, dim=dim, seqlen=L, dstate=N, io_dtype=io)
+    """Two calls in a row with different time splits and lengths: the second call's chunk
+    boundaries move, so words the first call left in the array lie under the second call's
+    reads; the second call must write every word it reads first."""
+    batch, dim, N = 1, 64, 16                    # few channels: the plan splits time
     code = _abi.SSM_BF16 if io == torch.bfloat16 else _abi.SSM_F32
-    for call, seed in enumerate((11, 12)):      # two calls in a row, different inputs
+    for call, (seed, L, split) in enumerate(((11, 16384, "16"), (12, 12000, "3"))):
+        monkeypatch.setenv("SSM_FWD_SPLIT", split)
+        need = ssm.fwd_workspace_bytes(batch, dim, L, N, io)
+        assert 0 < need <= _abi.NOALLOC_SCRATCH_BYTES
+        w = workload("long_seq_1m", batch=batch, dim=dim, seqlen=L, dstate=N, io_dtype=io)
         x = {k: v.to(DEV) for k, v in make_inputs(w, seed=seed, with_h0=True).items()}
         ref, ref_hL = ssm.ssm_scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], D=x["D"], z=x["z"],
                                        dt_bias=x["dt_bias"], h0=x["h0"], return_final_state=True)
