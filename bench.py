@@ -73,9 +73,13 @@ def load_peaks():
     return dict(FALLBACK_PEAKS)
 
 
+# Sources of the kernel that runs the benchmark step (the one-lane-per-channel forward kernel)
+KERNEL_SOURCES = ("ssm_fwd_lane.cuh", "ssm_fwd_lane_bf16.cu", "ssm_device.cuh", "ssm_kernels.h")
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for f in ("ssm_fwd_impl.cuh", "ssm_fwd_bf16.cu", "ssm_device.cuh", "ssm_kernels.h", "ssm_rows.cuh"):
+    for f in KERNEL_SOURCES:
         with open(os.path.join(ROOT, "selective_state_space_23_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -178,42 +182,45 @@ def barrier(world: int):
 
 
 # ------------------------------------------------------------------ CPU oracle baseline
-def oracle_sample_time(w, seed: int, target_s: float = 3.0):
-    """Time the fp64 oracle (as it stands) on a channel sample of the workload; return
-    (tokens_per_s_extrapolated, cores, description).  The sample grows until it takes about
-    target_s seconds or covers the whole workload."""
+# Both arms time the same thing: the fp64 oracle, as it stands, on the first REF_CHANNELS
+# channels of every batch row of the workload (full L and N), with the oracle's default thread
+# count; the full-width throughput is that sample's measured time scaled by dim / REF_CHANNELS.
+REF_CHANNELS = int(os.environ.get("SSM_REF_CHANNELS", "512"))
+
+
+def oracle_sample(w, seed: int = 0, nd: int = REF_CHANNELS, nthreads: int = 0):
+    """A callable running the oracle forward on nd channels (all batch rows) of the workload."""
     import oracle
     x = make_inputs(w, seed=seed)
     f = {k: v.to(torch.float64).numpy() for k, v in x.items()}
-    cores = oracle.max_threads()
-    nd = min(w.dim, 64)
-    while True:
-        sel = np.arange(nd)
-        t0 = time.perf_counter()
-        oracle.scan_fwd(f["u"][:, sel], f["delta"][:, sel], f["A"][sel], f["B"], f["C"],
-                        D=f["D"][sel], z=f["z"][:, sel], dt_bias=f["dt_bias"][sel])
-        dt = time.perf_counter() - t0
-        if dt >= target_s or nd >= w.dim:
-            break
-        nd = min(w.dim, max(nd * 2, int(nd * target_s / max(dt, 1e-3))))
-    full_s = dt * w.dim / nd
-    desc = (f"oracle fp64 on {w.batch}x{nd} of {w.batch}x{w.dim} channels x L {w.seqlen} x N "
-            f"{w.dstate} ({dt:.2f} s), extrapolated by channel count")
-    return w.tokens / full_s, cores, desc, dt
-
-
-def oracle_single_core(w, seed: int, nd: int = 256):
-    """The same oracle on one thread over an nd-channel sample: (tokens/s extrapolated, sample)."""
-    import oracle
-    x = make_inputs(w, seed=seed)
     sel = np.arange(min(nd, w.dim))
-    f = {k: v.to(torch.float64).numpy() for k, v in x.items()}
+    sub = dict(u=np.ascontiguousarray(f["u"][:, sel]), delta=np.ascontiguousarray(f["delta"][:, sel]),
+               A=f["A"][sel], B=f["B"], C=f["C"], D=f["D"][sel],
+               z=np.ascontiguousarray(f["z"][:, sel]), dt_bias=f["dt_bias"][sel])
+    run = lambda: oracle.scan_fwd(sub["u"], sub["delta"], sub["A"], sub["B"], sub["C"], D=sub["D"],
+                                  z=sub["z"], dt_bias=sub["dt_bias"], nthreads=nthreads)
+    return run, len(sel)
+
+
+def oracle_timing(w, warmup: int, steps: int, nthreads: int = 0):
+    """Measured seconds per sample run (mean over `steps` after `warmup`), the sample's channel
+    count, the threads used and the full-width tokens/s extrapolated by channel count."""
+    import oracle
+    run, nd = oracle_sample(w, nthreads=nthreads)
+    for _ in range(warmup):
+        run()
     t0 = time.perf_counter()
-    oracle.scan_fwd(f["u"][:, sel], f["delta"][:, sel], f["A"][sel], f["B"], f["C"],
-                    D=f["D"][sel], z=f["z"][:, sel], dt_bias=f["dt_bias"][sel], nthreads=1)
-    dt = time.perf_counter() - t0
-    return w.tokens / (dt * w.dim / len(sel)), (f"1 thread, {w.batch}x{len(sel)} channels "
-                                                f"({dt:.2f} s), extrapolated by channel count")
+    for _ in range(steps):
+        run()
+    per_run = (time.perf_counter() - t0) / steps
+    cores = nthreads if nthreads > 0 else oracle.max_threads()
+    return per_run, nd, cores, w.tokens / (per_run * w.dim / nd)
+
+
+def sample_desc(w, nd, per_run, steps):
+    return (f"oracle fp64 on {w.batch}x{nd} of {w.batch}x{w.dim} channels (L {w.seqlen}, N "
+            f"{w.dstate}): measured {per_run * 1e3:.1f} ms per run (mean of {steps}); tokens/s "
+            f"= {w.batch}x{w.seqlen} tokens / (that time x {w.dim}/{nd})")
 
 
 def cpu_model() -> str:
@@ -232,34 +239,19 @@ def run_reference(args, rank, world):
     if rank != 0:
         return 0
     w = workload(WORKLOAD)
-    # warm-up steps (untimed), then K timed steps; each step a bounded channel sample
-    import oracle
-    x = make_inputs(w, seed=0)
-    f = {k: v.to(torch.float64).numpy() for k, v in x.items()}
-    cores = oracle.max_threads()
-    nd = int(os.environ.get("SSM_REF_CHANNELS", "128"))
-    sel = np.arange(nd)
-    sub = dict(u=f["u"][:, sel], delta=f["delta"][:, sel], A=f["A"][sel], B=f["B"], C=f["C"],
-               D=f["D"][sel], z=f["z"][:, sel], dt_bias=f["dt_bias"][sel])
-    run = lambda: oracle.scan_fwd(sub["u"], sub["delta"], sub["A"], sub["B"], sub["C"], D=sub["D"],
-                                  z=sub["z"], dt_bias=sub["dt_bias"])
-    for _ in range(args.warmup):
-        run()
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        run()
-    el = time.perf_counter() - t0
-    per_step_full = el / args.steps * w.dim / nd
-    value = w.tokens / per_step_full
-    sample = (f"each step: oracle fp64 on {w.batch}x{nd} of {w.batch}x{w.dim} channels "
-              f"(L {w.seqlen}, N {w.dstate}); throughput extrapolated by channel count")
+    # W untimed warm-up runs, then K timed runs of the bounded channel sample
+    per_run, nd, cores, value = oracle_timing(w, args.warmup, args.steps)
+    sample = sample_desc(w, nd, per_run, args.steps)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step_full * 1e3,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_run * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded)",
         "config": {"workload": f"{WORKLOAD}: batch 8 x dim 2048 x L 2048, N 16, bf16 io rounded then f64",
-                   "global_batch": w.batch, "seq_len": w.seqlen, "parallelism": "host cores"},
+                   "global_batch": w.batch, "seq_len": w.seqlen, "parallelism": "host cores",
+                   "step": f"one oracle run over {w.batch}x{nd} of the {w.batch}x{w.dim} channels "
+                           "(ms_per_step is its measured time; value is extrapolated to the full "
+                           "width by channel count)"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -503,8 +495,11 @@ def main():
         cb_desc = "skipped (--no-baseline)" if args.no_baseline else "timed at N=1 only"
         sc_value, sc_desc = None, cb_desc
     else:
-        cb_value, cb_cores, cb_desc, _ = oracle_sample_time(w, seed=0)
-        sc_value, sc_desc = oracle_single_core(w, seed=0)
+        reps = 5
+        per_run, nd, cb_cores, cb_value = oracle_timing(w, 1, reps)
+        cb_desc = sample_desc(w, nd, per_run, reps)
+        per1, nd1, _, sc_value = oracle_timing(w, 0, 1, nthreads=1)
+        sc_desc = sample_desc(w, nd1, per1, 1) + " (1 thread)"
     extras = {} if world == 1 else {"skipped": "the side measurements run at N=1 only"}
     if not args.no_extras and world == 1:
         try:  # side measurements: a failure here is reported, it does not cost the main line
@@ -531,6 +526,7 @@ def main():
                      "kernel_ms": kern_ms},
         "cpu_baseline": {"value": cb_value, "unit": UNIT, "cores": cb_cores, "kind": "oracle",
                          "sample": cb_desc, "cpu_model": cpu_model(),
+                         "same_as": "the --impl reference arm (same sample, threads and oracle)",
                          "single_core": {"value": sc_value, "unit": UNIT, "sample": sc_desc}},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},

@@ -302,6 +302,17 @@ SSM_API int ssm_state_update_ex(float* state, const void* x, const void* dt, con
                                 int dim, int dstate, int bc_groups, int io_dtype, int flags,
                                 void* stream);
 
+/*
+ * Number of bounded waits that ran out on the current device since the library was loaded
+ * (the pages have no counterpart: this reports on the library's own kernels).  The streamed
+ * decode step waits on shared-memory barriers for its bulk copies; each wait gives up after a
+ * fixed number of polls, counts a timeout here, lets the copies in flight land and returns
+ * (that call's outputs are then incomplete).  0 means every wait completed.  Synchronises with
+ * the device (it reads a device counter).  Returns SSM_OK, or SSM_EINVAL for a NULL pointer,
+ * or SSM_ECUDA if the counter cannot be read.
+ */
+SSM_API int ssm_wait_timeouts(unsigned int* count);
+
 #ifdef __cplusplus
 }
 #endif

@@ -54,6 +54,7 @@ SIGNATURES = {
                               _i, _i, _i, _i, _vp]),
     "ssm_state_update_ex": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp,
                                  _i, _i, _i, _i, _i, _i, _vp]),
+    "ssm_wait_timeouts": (_i, [ctypes.POINTER(ctypes.c_uint)]),
 }
 
 _lib = None
@@ -78,6 +79,13 @@ def lib() -> ctypes.CDLL:
 
 def last_error() -> str:
     return lib().ssm_last_error().decode()
+
+
+def wait_timeouts() -> int:
+    """Bounded waits that ran out in the library's kernels on the current device (0 = none)."""
+    n = ctypes.c_uint(0)
+    check(lib().ssm_wait_timeouts(ctypes.byref(n)), "ssm_wait_timeouts")
+    return int(n.value)
 
 
 def check(rc: int, what: str) -> None:

@@ -14,8 +14,8 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD_DIR = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libssm_b200.so")
 SOURCES = ["ssm_api.cu", "ssm_fwd.cu", "ssm_fwd_bf16.cu", "ssm_fwd_f32.cu", "ssm_fwd_rev_bf16.cu",
-           "ssm_fwd_rev_f32.cu", "ssm_bwd.cu", "ssm_decode.cu", "ssm_noalloc.cu", "ssm_host.cu"]
-HEADERS = ["ssm_device.cuh", "ssm_kernels.h", "ssm_rows.cuh", "ssm_fwd_impl.cuh"]
+           "ssm_fwd_rev_f32.cu", "ssm_fwd_lane_bf16.cu", "ssm_fwd_lane_f32.cu", "ssm_bwd.cu", "ssm_bwd_hist.cu", "ssm_decode.cu", "ssm_noalloc.cu", "ssm_host.cu"]
+HEADERS = ["ssm_device.cuh", "ssm_kernels.h", "ssm_rows.cuh", "ssm_fwd_impl.cuh", "ssm_fwd_lane.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
@@ -27,6 +27,35 @@ def _inputs():
             + [os.path.join(ROOT, "include", "ssm_scan.h")])
 
 
+def _deps(path: str, seen=None) -> set:
+    """The file and every file it #includes with quotes, recursively (paths resolved relative to
+    the including file)."""
+    seen = set() if seen is None else seen
+    path = os.path.normpath(path)
+    if path in seen or not os.path.exists(path):
+        return seen
+    seen.add(path)
+    with open(path, encoding="utf-8") as fh:
+        for line in fh:
+            line = line.strip()
+            if line.startswith("#include \""):
+                inc = line.split('"')[1]
+                _deps(os.path.join(os.path.dirname(path), inc), seen)
+    return seen
+
+
+def _obj(src: str) -> str:
+    return os.path.join(BUILD_DIR, os.path.splitext(src)[0] + ".o")
+
+
+def _obj_stale(src: str) -> bool:
+    obj = _obj(src)
+    if not os.path.exists(obj):
+        return True
+    t = os.path.getmtime(obj)
+    return any(os.path.getmtime(p) > t for p in _deps(os.path.join(CSRC, src)))
+
+
 def _stale() -> bool:
     if not os.path.exists(LIB):
         return True
@@ -35,7 +64,7 @@ def _stale() -> bool:
 
 
 def _compile(src: str, verbose: bool) -> str:
-    obj = os.path.join(BUILD_DIR, os.path.splitext(src)[0] + ".o")
+    obj = _obj(src)
     cmd = [NVCC, *ARCH, *FLAGS, "-c", os.path.join(CSRC, src), "-o", obj]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
@@ -52,8 +81,10 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if not force and not _stale():
         return LIB
     os.makedirs(BUILD_DIR, exist_ok=True)
-    with cf.ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose), SOURCES))
+    todo = [s for s in SOURCES if force or _obj_stale(s)]  # objects older than their includes
+    with cf.ThreadPoolExecutor(max_workers=max(1, len(todo))) as ex:
+        list(ex.map(lambda s: _compile(s, verbose), todo))
+    objs = [_obj(s) for s in SOURCES]
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = [NVCC, *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", tmp, *objs, "-cudart", "static"]
     r = subprocess.run(cmd, capture_output=True, text=True)

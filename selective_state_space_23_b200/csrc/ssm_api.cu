@@ -158,19 +158,23 @@ struct FwdPlan {
   size_t ws_bytes;
 };
 
-// Lanes per channel of the forward kernel: 1 (16 states per lane), 2 (8) or 4 (4).
-int fwd_lpc() {
-  const int v = env_int("SSM_FWD_LPC", 2);
-  return (v == 1 || v == 4) ? v : 2;
-}
-int fwd_warps_per_b(int dim) {
-  const int chw = 32 / fwd_lpc();
-  return (dim + chw - 1) / chw;
+// Lanes per channel of the general forward kernel (8 states per lane).
+int fwd_lpc() { return 2; }
+
+// Kernel family of the forward scan: the one-lane-per-channel kernel (ssm_fwd_lane.cuh) serves
+// the default variant whenever its rows allow 16-byte copies; SSM_FWD_KERNEL=pair forces the
+// general kernel (ssm_fwd_impl.cuh), which serves every variant and layout.
+bool fwd_lane_allowed() {
+  const char* v = getenv("SSM_FWD_KERNEL");
+  return !(v && strcmp(v, "pair") == 0);
 }
 
-FwdPlan plan_fwd(int batch, int dim, int seqlen) {
+// Channels per warp of each kernel family.
+int fwd_chw(bool lane) { return lane ? 32 : 32 / fwd_lpc(); }
+
+FwdPlan plan_fwd(int batch, int dim, int seqlen, int chw) {
   const int smsp = 4 * sm_count();
-  const long long warps = (long long)batch * fwd_warps_per_b(dim);
+  const long long warps = (long long)batch * ((dim + chw - 1) / chw);
   const int nblk = (seqlen + ssm::kBlk - 1) / ssm::kBlk;
   int S = 1;
   const int forced = env_int("SSM_FWD_SPLIT", 0);
@@ -199,6 +203,14 @@ FwdPlan plan_fwd(int batch, int dim, int seqlen) {
   const size_t nch = (size_t)batch * dim;
   p.ws_bytes = align_up(p.nchunk * nch * ssm::kNS * 4) * 2 + align_up(p.nchunk * nch * 4);
   return p;
+}
+
+// Workspace that covers the plan of either kernel family (the family is chosen per call, from
+// the pointers' alignment too).
+size_t fwd_ws_bytes(int batch, int dim, int seqlen) {
+  const size_t a = plan_fwd(batch, dim, seqlen, fwd_chw(false)).ws_bytes;
+  const size_t b = plan_fwd(batch, dim, seqlen, fwd_chw(true)).ws_bytes;
+  return a > b ? a : b;
 }
 
 // Launch tuning of the forward kernel (measured on B200; the environment variables override it
@@ -267,7 +279,7 @@ const char* ssm_version(void) { return "ssm_b200 0.1 (sm_100a)"; }
 
 size_t ssm_scan_fwd_workspace_size(int batch, int dim, int seqlen, int dstate, int io_dtype) {
   if (check_dims(batch, dim, seqlen, dstate, io_dtype) != SSM_OK) return 0;
-  return plan_fwd(batch, dim, seqlen).ws_bytes;
+  return fwd_ws_bytes(batch, dim, seqlen);
 }
 
 }  // extern "C"
@@ -306,7 +318,15 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
   TRY(check_opt(ckpt, (size_t)batch * dim * nblk * dstate * 4, 4, "ckpt"));
   if (out == u || out == delta || out == z) return fail(SSM_EINVAL, "out aliases an input");
 
-  FwdPlan plan = plan_fwd(batch, dim, seqlen);
+  const bool zoh = (flags & SSM_ZOH) != 0, reverse = (flags & SSM_REVERSE) != 0;
+  const bool channels_last = (flags & SSM_CHANNELS_LAST) != 0;
+  // 128-bit row accesses need rows along L; the channels-last layout takes element accesses
+  const bool vec = !channels_last && (seqlen * es) % 16 == 0 && aligned16(u) &&
+                   aligned16(delta) && aligned16(z) && aligned16(out) && aligned16(B) &&
+                   aligned16(C);
+  const bool lane = fwd_lane_allowed() && vec && !scalar_a && !zoh && !reverse &&
+                    (bc_groups == 1 || (dim / bc_groups) % 32 == 0);
+  FwdPlan plan = plan_fwd(batch, dim, seqlen, fwd_chw(lane));
   if (plan.nchunk > 1 && (!workspace || workspace_bytes < plan.ws_bytes ||
                           (reinterpret_cast<uintptr_t>(workspace) & 255))) {
     plan.nchunk = 1;  // not enough scratch: same result without the time split
@@ -328,21 +348,19 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
   a.bc_groups = bc_groups;
   a.lpc = (scalar_a || a.zoh || bc_groups > 1) ? 2 : fwd_lpc();
   a.warps_per_b = (dim + 32 / a.lpc - 1) / (32 / a.lpc);
-  a.nwarps = (long long)batch * a.warps_per_b;
-  a.channels_last = (flags & SSM_CHANNELS_LAST) ? 1 : 0;
-  if (a.channels_last) {
+  a.channels_last = channels_last ? 1 : 0;
+  if (lane) {
+    a.lpc = 1;
+    a.warps_per_b = (dim + 31) / 32;
+  } else if (a.channels_last) {
     a.lpc = 2;
     a.warps_per_b = (dim + 15) / 16;
-    a.nwarps = (long long)batch * a.warps_per_b;
     // 16-byte tiles of 8 channels (or states) per lane: every warp full, rows 16-byte aligned
     a.cl_tile = dim % 16 == 0 && dstate == 16 && (dim * es) % 16 == 0 && aligned16(u) &&
                 aligned16(delta) && aligned16(z) && aligned16(out) && aligned16(B) &&
                 aligned16(C);
   }
-  // 128-bit row accesses need rows along L; the channels-last layout takes element accesses
-  const bool vec = !a.channels_last && (seqlen * es) % 16 == 0 && aligned16(u) &&
-                   aligned16(delta) && aligned16(z) && aligned16(out) && aligned16(B) &&
-                   aligned16(C);
+  a.nwarps = (long long)batch * a.warps_per_b;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int wpb = fwd_wpb();
   const int km = fwd_kmufu(a.nwarps * (long long)plan.nchunk);
@@ -357,14 +375,16 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
     ssm::FwdArgs as = a;
     as.summ = summ; as.dsum = dsum;
     as.out = nullptr; as.hL = nullptr; as.ckpt = nullptr; as.h0 = nullptr;
-    if ((e = ssm::launch_fwd(as, io_dtype, vec, ssm::kFwdSummary, wpb, km, s)) != cudaSuccess)
-      return cuda_fail(e, "forward summary pass");
+    e = lane ? ssm::launch_fwd_lane(as, io_dtype, ssm::kFwdSummary, km, s)
+             : ssm::launch_fwd(as, io_dtype, vec, ssm::kFwdSummary, wpb, km, s);
+    if (e != cudaSuccess) return cuda_fail(e, "forward summary pass");
     if ((e = ssm::launch_fwd_carry(a, summ, dsum, hin, s)) != cudaSuccess)
       return cuda_fail(e, "forward carry pass");
     a.hin = hin;
   }
-  if ((e = ssm::launch_fwd(a, io_dtype, vec, ssm::kFwdOut, wpb, km, s)) != cudaSuccess)
-    return cuda_fail(e, "forward pass");
+  e = lane ? ssm::launch_fwd_lane(a, io_dtype, ssm::kFwdOut, km, s)
+           : ssm::launch_fwd(a, io_dtype, vec, ssm::kFwdOut, wpb, km, s);
+  if (e != cudaSuccess) return cuda_fail(e, "forward pass");
   return SSM_OK;
 }
 
@@ -510,11 +530,15 @@ int scan_bwd_core(const void* u, const void* delta, const float* A, const void* 
     a.zoh = zoh ? 1 : 0;
     a.bc_groups = bc_groups;
     a.channels_last = channels_last ? 1 : 0;
-    a.lpc = (zoh || bc_groups > 1) ? 2 : fwd_lpc();
-    a.warps_per_b = (dim + 32 / a.lpc - 1) / (32 / a.lpc);
+    const bool lane = fwd_lane_allowed() && vec && !reverse && !zoh &&
+                      (bc_groups == 1 || (dim / bc_groups) % 32 == 0);
+    a.lpc = lane ? 1 : ((zoh || bc_groups > 1) ? 2 : fwd_lpc());
+    a.warps_per_b = (dim + fwd_chw(lane) - 1) / fwd_chw(lane);
+    if (!lane) a.warps_per_b = (dim + 32 / a.lpc - 1) / (32 / a.lpc);
     a.nwarps = (long long)batch * a.warps_per_b;
-    if ((e = ssm::launch_fwd(a, io_dtype, vec, ssm::kFwdCkpt, fwd_wpb(), fwd_kmufu(a.nwarps), s)) != cudaSuccess)
-      return cuda_fail(e, "backward state replay pass");
+    e = lane ? ssm::launch_fwd_lane(a, io_dtype, ssm::kFwdCkpt, fwd_kmufu(a.nwarps), s)
+             : ssm::launch_fwd(a, io_dtype, vec, ssm::kFwdCkpt, fwd_wpb(), fwd_kmufu(a.nwarps), s);
+    if (e != cudaSuccess) return cuda_fail(e, "backward state replay pass");
     ck = ck_ws;
   }
   ssm::BwdArgs b;
@@ -534,7 +558,24 @@ int scan_bwd_core(const void* u, const void* delta, const float* A, const void* 
   b.wpb = l.wpb;
   b.ngroups = l.ngroups;
   b.kmufu = env_int("SSM_BWD_KMUFU", 4);  // all exponentials on MUFU measured fastest
-  if ((e = ssm::launch_bwd(b, io_dtype, vec, s)) != cudaSuccess) return cuda_fail(e, "backward pass");
+  // the default variant with N = 16 and rows of whole 8-step pieces: the state history in
+  // registers (ssm_bwd_hist.cu); SSM_BWD_KERNEL=pair forces the general kernel
+  const char* bk = getenv("SSM_BWD_KERNEL");
+  bool hist = !(bk && strcmp(bk, "pair") == 0) && vec && !reverse && !zoh && !channels_last &&
+              dstate == ssm::kNS && seqlen % 8 == 0 && aligned16(ck) && aligned16(dhL) &&
+              aligned16(dh0);
+  if (hist) {
+    int w = env_int("SSM_BWD_WPB", 0);
+    if (w != 2 && w != 4) w = ssm::bwd_hist_pick_wpb(io_dtype, batch, dim);
+    if (bc_groups > 1 && (dim / bc_groups) % (16 * w) != 0) w = 2;
+    if (bc_groups > 1 && (dim / bc_groups) % (16 * w) != 0) hist = false;
+    if (hist) {
+      b.wpb = w;
+      b.ngroups = (b.warps_per_b + w - 1) / w;
+    }
+  }
+  e = hist ? ssm::launch_bwd_hist(b, io_dtype, s) : ssm::launch_bwd(b, io_dtype, vec, s);
+  if (e != cudaSuccess) return cuda_fail(e, "backward pass");
   if ((e = ssm::launch_bwd_finish(b, io_dtype, dB, dC, dA, dD, ddt_bias, s)) != cudaSuccess)
     return cuda_fail(e, "backward reduction");
   return SSM_OK;
@@ -665,6 +706,16 @@ int ssm_state_update_ex(float* state, const void* x, const void* dt, const float
   a.bc_groups = bc_groups;
   cudaError_t e = ssm::launch_decode(a, io_dtype, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode step");
+  return SSM_OK;
+}
+
+int ssm_wait_timeouts(unsigned int* count) {
+  g_err[0] = 0;
+  if (!count) return fail(SSM_EINVAL, "count is NULL");
+  if (ssm::decode_wait_timeouts(count) != 0) {
+    cudaError_t e = cudaGetLastError();
+    return cuda_fail(e, "reading the wait-timeout counter");
+  }
   return SSM_OK;
 }
 

@@ -15,6 +15,8 @@
 // N = 16 two lanes share a channel, each holding 8 consecutive states as two 128-bit accesses
 // (a warp streams 1 KB of contiguous state per access pair); the two partial readouts are
 // combined with one shuffle.  Other N use four lanes of 4 states with per-element guards.
+#include <stdlib.h>
+
 #include <type_traits>
 
 #include "ssm_device.cuh"
@@ -36,6 +38,13 @@ template <> __device__ __forceinline__ void st_io<float>(void* p, long long i, f
 }
 template <> __device__ __forceinline__ void st_io<uint16_t>(void* p, long long i, float v) {
   reinterpret_cast<uint16_t*>(p)[i] = f32_to_bf16(v);
+}
+
+// SSM_DECODE_STREAM=0 selects the per-thread form of the N = 16 decode step instead of the
+// streamed one (for measurements; both compute the same arithmetic).
+bool getenv_stream_enabled() {
+  const char* v = getenv("SSM_DECODE_STREAM");
+  return !(v && v[0] == '0');
 }
 
 // Input coefficient of B x: Δ, or with the ZOH term (e^{ΔA} - 1)/A (Δ as A -> 0).
@@ -180,10 +189,212 @@ __global__ void __launch_bounds__(256) decode16_kernel(const DecodeArgs a) {
   }
 }
 
+// ---------------------------------------------------------------- streamed form
+// The state is the step's only large operand (batch x dim x 16 f32, read and written once).  A
+// thread that loads its channel's 64 bytes and waits for them keeps few bytes in flight per
+// SM.  Here persistent CTAs stream tiles of kTile consecutive channels through a kStages-deep
+// shared-memory ring with bulk asynchronous copies (one cp.async.bulk per operand and tile,
+// completing on the stage's mbarrier), so kStages tiles per CTA are in flight with no register
+// cost.  A CTA keeps one block of kTile channels d and walks down the batch rows, so its rows of
+// A (and D, dt_bias) are loaded once.  Every wait on an mbarrier is bounded: after kSpinLimit
+// polls the kernel counts a timeout in g_wait_timeouts (read by ssm_wait_timeouts()), waits
+// (bounded again) for the copies it issued, and returns.
+constexpr int kTile = 128;                 // channels per tile (2 threads each)
+constexpr int kStages = 4;
+constexpr int kStreamThreads = 2 * kTile;
+constexpr long long kSpinLimit = 1LL << 22;
+
+__device__ unsigned int g_wait_timeouts = 0;
+
+template <typename IO>
+struct StreamStage {
+  float state[kTile * kNS];
+  IO x[kTile], dt[kTile], z[kTile];
+  IO B[kNS], C[kNS];
+};
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_expect(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+// true when the phase with this parity has completed; false after kSpinLimit polls
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  for (long long i = 0; i < kSpinLimit; ++i) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+// bytes (a multiple of 16) from global src to shared dst (both 16-byte aligned), counted on bar
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+          smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+template <typename IO>
+__global__ void __launch_bounds__(kStreamThreads) decode_stream_kernel(const __grid_constant__ DecodeArgs a,
+                                                                       int rows_per_cta) {
+  constexpr bool kPrecise = std::is_same<IO, float>::value;
+  extern __shared__ float4 smem_dec[];
+  StreamStage<IO>* st = reinterpret_cast<StreamStage<IO>*>(smem_dec);
+  __shared__ __align__(8) uint64_t bars[kStages];
+  const int tid = threadIdx.x;
+  const int nblk_d = a.dim / kTile;
+  const int dblk = blockIdx.x % nblk_d;
+  const int b0 = (blockIdx.x / nblk_d) * rows_per_cta;
+  const int nrows = min(rows_per_cta, a.batch - b0);
+  if (nrows <= 0) return;
+  const int d0 = dblk * kTile;
+  const int gbc = d0 / (a.dim / a.bc_groups);  // the tile's channels share one B/C group
+  const int cl = tid >> 1, q = tid & 1;        // channel in the tile, half of its states
+  const int d = d0 + cl;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&bars[s]);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  __syncthreads();
+
+  const size_t es = sizeof(IO);
+  const auto issue = [&](int r, int stage) {  // batch row b0 + r into stage
+    StreamStage<IO>& sg = st[stage];
+    const long long c0 = (long long)(b0 + r) * a.dim + d0;
+    const uint32_t bytes = (uint32_t)(kTile * kNS * 4 + (a.z ? 3 : 2) * kTile * es + 2 * kNS * es);
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+    mbar_expect(&bars[stage], bytes);
+    bulk_load(sg.state, a.state + c0 * kNS, kTile * kNS * 4, &bars[stage]);
+    bulk_load(sg.x, reinterpret_cast<const IO*>(a.x) + c0, kTile * es, &bars[stage]);
+    bulk_load(sg.dt, reinterpret_cast<const IO*>(a.dt) + c0, kTile * es, &bars[stage]);
+    if (a.z) bulk_load(sg.z, reinterpret_cast<const IO*>(a.z) + c0, kTile * es, &bars[stage]);
+    const long long bc = ((long long)(b0 + r) * a.bc_groups + gbc) * kNS;
+    bulk_load(sg.B, reinterpret_cast<const IO*>(a.B) + bc, kNS * es, &bars[stage]);
+    bulk_load(sg.C, reinterpret_cast<const IO*>(a.C) + bc, kNS * es, &bars[stage]);
+  };
+  if (tid == 0)
+    for (int r = 0; r < kStages && r < nrows; ++r) issue(r, r);
+
+  // per-channel parameters, once for every batch row of the CTA
+  float An[8];
+  if (a.scalar_a) {
+    const float ad = __ldg(a.A + d);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) An[i] = ad;
+  } else {
+    const float4* ap = reinterpret_cast<const float4*>(a.A + (long long)d * kNS + 8 * q);
+    const float4 a0 = __ldg(ap), a1 = __ldg(ap + 1);
+    An[0] = a0.x; An[1] = a0.y; An[2] = a0.z; An[3] = a0.w;
+    An[4] = a1.x; An[5] = a1.y; An[6] = a1.z; An[7] = a1.w;
+  }
+  const float bias = a.dt_bias ? a.dt_bias[d] : 0.f;
+  const float Dd = a.D ? a.D[d] : 0.f;
+
+  bool ok = true;
+  int r = 0;
+  for (; r < nrows; ++r) {
+    const int stage = r % kStages;
+    const bool landed = mbar_wait(&bars[stage], (uint32_t)((r / kStages) & 1));
+    if (!__syncthreads_and(landed)) {  // the whole CTA stops together
+      ok = false;
+      break;
+    }
+    const StreamStage<IO>& sg = st[stage];
+    const float xv = ld_io<IO>(sg.x, cl);
+    const float v = ld_io<IO>(sg.dt, cl) + bias;
+    const float dt = !a.softplus ? v : (kPrecise ? softplus_precise(v) : softplus_fast(v));
+    const float dx = dt * xv;
+    const float4 h0 = reinterpret_cast<const float4*>(sg.state + cl * kNS + 8 * q)[0];
+    const float4 h1 = reinterpret_cast<const float4*>(sg.state + cl * kNS + 8 * q)[1];
+    float h[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+    float y = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float Bn = ld_io<IO>(sg.B, 8 * q + i), Cn = ld_io<IO>(sg.C, 8 * q + i);
+      const float abar = (kPrecise || a.zoh) ? expf(dt * An[i]) : ex2_mufu(dt * An[i] * kLog2e);
+      const float bx = a.zoh ? decode_coef(dt, An[i], true) * xv : dx;
+      h[i] = fmaf(abar, h[i], bx * Bn);
+      y = fmaf(Cn, h[i], y);
+    }
+    y += __shfl_xor_sync(0xffffffffu, y, 1);
+    const float zv = a.z ? ld_io<IO>(sg.z, cl) : 0.f;
+    __syncthreads();  // every thread has read this stage
+    if (tid == 0 && r + kStages < nrows) issue(r + kStages, stage);
+    const long long ch = (long long)(b0 + r) * a.dim + d;
+    float4* sp = reinterpret_cast<float4*>(a.state + ch * kNS + 8 * q);
+    sp[0] = make_float4(h[0], h[1], h[2], h[3]);
+    sp[1] = make_float4(h[4], h[5], h[6], h[7]);
+    if (q == 0) {
+      y += Dd * xv;
+      if (a.z) y *= zv * (kPrecise ? sigmoid_precise(zv) : sigmoid_fast(zv));
+      st_io<IO>(a.out, ch, y);
+    }
+  }
+  if (!ok) {
+    // a copy never completed: record it, wait (bounded) for the copies still in flight so none
+    // lands after the CTA's shared memory is released, and stop
+    if (tid == 0) atomicAdd(&g_wait_timeouts, 1u);
+    for (int rr = r; rr < nrows && rr < r + kStages; ++rr)
+      mbar_wait(&bars[rr % kStages], (uint32_t)((rr / kStages) & 1));
+  }
+}
+
+template <typename IO>
+cudaError_t launch_stream(const DecodeArgs& a, cudaStream_t s) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int nblk_d = a.dim / kTile;
+  // 2 to 4 resident CTAs per SM, each walking a run of batch rows; the run length is chosen so
+  // that the CTAs spread evenly over the SMs
+  int rows = a.batch, grid = nblk_d;
+  double best = -1.0;
+  for (int k = 2; k <= 4; ++k) {
+    const int g = max(1, min(a.batch, (int)((double)k * sms / nblk_d + 0.5)));
+    const int rw = (a.batch + g - 1) / g;
+    const int ng = (a.batch + rw - 1) / rw;
+    const int gr = nblk_d * ng;
+    const double eff = (double)gr / ((double)sms * ((gr + sms - 1) / sms)) *
+                       ((double)a.batch / ((double)ng * rw));
+    if (eff > best) {
+      best = eff;
+      rows = rw;
+      grid = gr;
+    }
+  }
+  const size_t smem = kStages * sizeof(StreamStage<IO>);
+  auto k = decode_stream_kernel<IO>;
+  if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  k<<<grid, kStreamThreads, smem, s>>>(a, rows);
+  return cudaGetLastError();
+}
+
 template <typename IO>
 cudaError_t launch_io(const DecodeArgs& a, cudaStream_t s) {
   const int tpb = 256;
   const auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+  // the streamed form: 16 states, whole tiles of channels inside one batch row and one B/C
+  // group, every bulk copy 16-byte aligned and a multiple of 16 bytes
+  const bool stream_ok = a.N == kNS && a.dim % kTile == 0 &&
+                         (a.bc_groups == 1 || (a.dim / a.bc_groups) % kTile == 0) &&
+                         al16(a.state) && (a.scalar_a || al16(a.A)) && al16(a.B) && al16(a.C) &&
+                         al16(a.x) && al16(a.dt) && (a.z == nullptr || al16(a.z)) &&
+                         kNS * sizeof(IO) % 16 == 0 && getenv_stream_enabled();
+  if (stream_ok) return launch_stream<IO>(a, s);
   if (a.N == kNS && al16(a.state) && (a.scalar_a || al16(a.A)) && al16(a.B) && al16(a.C)) {
     const long long threads = (long long)a.batch * a.dim * 2;
     decode16_kernel<IO><<<(unsigned)((threads + tpb - 1) / tpb), tpb, 0, s>>>(a);
@@ -201,6 +412,10 @@ cudaError_t launch_io(const DecodeArgs& a, cudaStream_t s) {
 
 cudaError_t launch_decode(const DecodeArgs& a, int io, cudaStream_t s) {
   return io == 1 ? launch_io<uint16_t>(a, s) : launch_io<float>(a, s);
+}
+
+int decode_wait_timeouts(unsigned int* out) {
+  return cudaMemcpyFromSymbol(out, g_wait_timeouts, sizeof(unsigned int)) == cudaSuccess ? 0 : -1;
 }
 
 }  // namespace ssm

@@ -818,45 +818,17 @@ cudaError_t launch_mode(const FwdArgs& a, int wpb, int kmufu, cudaStream_t s) {
   } else if (a.zoh) {  // per-state ZOH coefficient on the FMA pipe
     launch_one<IO, VEC, MODE, 2, kKpZoh, kKpZoh, REV>(a, grid, block, s);
   } else if constexpr (std::is_same<IO, float>::value) {  // fp32: library expf
-    if (a.lpc == 4) launch_one<IO, VEC, MODE, 4, 2, 2, REV>(a, grid, block, s);
-    else if (a.lpc == 1) launch_one<IO, VEC, MODE, 1, 8, 8, REV>(a, grid, block, s);
-    else launch_one<IO, VEC, MODE, 2, 4, 4, REV>(a, grid, block, s);
+    launch_one<IO, VEC, MODE, 2, 4, 4, REV>(a, grid, block, s);
   } else if constexpr (MODE != kFwdOut) {
-    if (a.lpc == 4) launch_one<IO, VEC, MODE, 4, 2, 1, REV>(a, grid, block, s);
-    else if (a.lpc == 1) launch_one<IO, VEC, MODE, 1, 7, 6, REV>(a, grid, block, s);
-    else launch_one<IO, VEC, MODE, 2, 4, 3, REV>(a, grid, block, s);
-  } else if (a.lpc == 4) {
-    // exponentials on the MUFU unit per lane over two steps (of 8): 4, 6 or 8
-    switch (kmufu) {
-      case 8: launch_one<IO, VEC, MODE, 4, 1, 1, REV>(a, grid, block, s); break;
-      case 16: launch_one<IO, VEC, MODE, 4, 2, 2, REV>(a, grid, block, s); break;
-      default: launch_one<IO, VEC, MODE, 4, 2, 1, REV>(a, grid, block, s); break;
-    }
-  } else if (a.lpc == 1) {
-    // exponentials on the MUFU unit per lane over two steps (of 32), in units of 16/16
-    switch (kmufu) {
-      case 8: launch_one<IO, VEC, MODE, 1, 4, 4, REV>(a, grid, block, s); break;
-      case 10: launch_one<IO, VEC, MODE, 1, 5, 5, REV>(a, grid, block, s); break;
-      case 12: launch_one<IO, VEC, MODE, 1, 6, 6, REV>(a, grid, block, s); break;
-      case 16: launch_one<IO, VEC, MODE, 1, 8, 8, REV>(a, grid, block, s); break;
-      default: launch_one<IO, VEC, MODE, 1, 7, 7, REV>(a, grid, block, s); break;
-    }
-  } else if (a.wide && (kmufu == 12 || kmufu == 14 || kmufu == 16)) {
-    // few warps per SM: the 255-register form
-    switch (kmufu) {
-      case 12: launch_one<IO, VEC, MODE, 2, 3, 3, REV, true>(a, grid, block, s); break;
-      case 16: launch_one<IO, VEC, MODE, 2, 4, 4, REV, true>(a, grid, block, s); break;
-      default: launch_one<IO, VEC, MODE, 2, 4, 3, REV, true>(a, grid, block, s); break;
-    }
+    launch_one<IO, VEC, MODE, 2, 4, 3, REV>(a, grid, block, s);
+  } else if (a.wide) {
+    // few warps per SM: the 255-register form; exponentials on MUFU per lane over two steps
+    // (of 16): 14, or 16 with SSM_FWD_KMUFU=16
+    if (kmufu == 16) launch_one<IO, VEC, MODE, 2, 4, 4, REV, true>(a, grid, block, s);
+    else launch_one<IO, VEC, MODE, 2, 4, 3, REV, true>(a, grid, block, s);
   } else {
-    // exponentials on the MUFU unit per lane over two steps (of 16): 8 ... 16
-    switch (kmufu) {
-      case 8: launch_one<IO, VEC, MODE, 2, 2, 2, REV>(a, grid, block, s); break;
-      case 10: launch_one<IO, VEC, MODE, 2, 3, 2, REV>(a, grid, block, s); break;
-      case 12: launch_one<IO, VEC, MODE, 2, 3, 3, REV>(a, grid, block, s); break;
-      case 16: launch_one<IO, VEC, MODE, 2, 4, 4, REV>(a, grid, block, s); break;
-      default: launch_one<IO, VEC, MODE, 2, 4, 3, REV>(a, grid, block, s); break;
-    }
+    if (kmufu == 16) launch_one<IO, VEC, MODE, 2, 4, 4, REV>(a, grid, block, s);
+    else launch_one<IO, VEC, MODE, 2, 4, 3, REV>(a, grid, block, s);
   }
   return cudaGetLastError();
 }

@@ -106,12 +106,25 @@ struct DecodeArgs {
 // io: 0 = f32, 1 = bf16.  vec: rows are 16-byte aligned and L is a multiple of the vector width.
 cudaError_t launch_fwd(const FwdArgs& a, int io, bool vec, int mode, int wpb, int kmufu,
                        cudaStream_t s);
+// The one-lane-per-channel forward kernel (default variant only: no scalar_a, zoh, reverse or
+// channels_last; rows allow 16-byte copies; a.warps_per_b = ceil(dim / 32); dim / bc_groups a
+// multiple of 32).
+cudaError_t launch_fwd_lane(const FwdArgs& a, int io, int mode, int kmufu, cudaStream_t s);
 cudaError_t launch_fwd_carry(const FwdArgs& a, const float* summ, const float* dsum, float* hin,
                              cudaStream_t s);
 cudaError_t launch_bwd(const BwdArgs& a, int io, bool vec, cudaStream_t s);
+// The backward of the default variant with the state history in registers (ssm_bwd_hist.cu):
+// N = 16, forward direction, no ZOH, [batch][dim][L] rows with L % 8 == 0 and 16-byte aligned
+// tensors and checkpoints; a.wpb = 2 or 4 warps per CTA (bwd_hist_pick_wpb), a.ngroups =
+// ceil(ceil(dim / 16) / a.wpb), each CTA inside one B/C group.
+cudaError_t launch_bwd_hist(const BwdArgs& a, int io, cudaStream_t s);
+int bwd_hist_pick_wpb(int io, int batch, int dim);
 cudaError_t launch_bwd_finish(const BwdArgs& a, int io, void* dB, void* dC, float* dA, float* dD,
                               float* ddt_bias, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, int io, cudaStream_t s);
+// Number of bounded waits that ran out in the streamed decode kernel since the library was loaded
+// on the current device (0 when every copy completed); -1 if the count could not be read.
+int decode_wait_timeouts(unsigned int* out);
 
 // Sets the message returned by ssm_last_error() on the calling thread.
 void set_last_error(const char* msg);

@@ -177,3 +177,8 @@ def test_binding_rejects_host_tensors_before_any_cuda_call():
     for name, f in calls.items():
         with pytest.raises(ValueError, match="must be a CUDA tensor"):
             f()
+
+
+def test_wait_timeout_query_rejects_null(lib):
+    assert lib.ssm_wait_timeouts(None) == _abi.SSM_EINVAL
+    assert b"NULL" in lib.ssm_last_error()

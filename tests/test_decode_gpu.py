@@ -92,3 +92,46 @@ def test_decode_b256_workload_sampled_channels():
         if t % 64 == 0 or t == steps - 1:
             assert_close(out[sel_b][:, sel_d.to(DEV)], ro, torch.bfloat16, f"out {t}")
             assert_close(state[sel_b][:, sel_d.to(DEV)], ref_state, torch.bfloat16, f"state {t}")
+
+
+@pytest.mark.parametrize("io", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("variant", ["plain", "no_gate", "groups", "scalar_a", "zoh"])
+def test_streamed_decode_matches_oracle_and_per_thread_form(monkeypatch, io, variant):
+    """dim a multiple of 128 with N = 16 takes the streamed form (bulk copies of 128-channel
+    tiles through a shared-memory ring): step by step against the oracle, bitwise against the
+    per-thread form (the same arithmetic), and no bounded wait ran out."""
+    from selective_state_space_23_b200 import _abi
+    batch, dim, N = 7, 384, 16
+    groups = 3 if variant == "groups" else 1
+    w = workload("decode_b256", batch=batch * groups, dim=dim, dstate=N, io_dtype=io)
+    r = np.random.default_rng(5)
+    state0 = (0.5 * r.standard_normal((batch, dim, N))).astype(np.float32)
+    st_a = torch.from_numpy(state0).to(DEV)
+    st_b = st_a.clone()
+    ref = state0.astype(np.float64).copy()
+    kw = dict(scalar_a=variant == "scalar_a", zoh=variant == "zoh")
+    for t in range(12):
+        x = make_inputs(w, seed=7, step=t, gate=variant != "no_gate", scalar_a=kw["scalar_a"])
+        x = {k: (v[:batch] if k in ("x", "dt", "z") else v) for k, v in x.items()}
+        if groups > 1:  # [batch, G, N]: draw G rows of B, C per batch row
+            x["B"] = x["B"].reshape(batch, groups, N)
+            x["C"] = x["C"].reshape(batch, groups, N)
+        else:
+            x["B"], x["C"] = x["B"][:batch], x["C"][:batch]
+        xd = {k: v.to(DEV) for k, v in x.items()}
+        monkeypatch.delenv("SSM_DECODE_STREAM", raising=False)
+        out_a = ssm.ssm_state_update(st_a, xd["x"], xd["dt"], xd["A"], xd["B"], xd["C"], D=xd["D"],
+                                     z=xd.get("z"), dt_bias=xd["dt_bias"], **kw)
+        monkeypatch.setenv("SSM_DECODE_STREAM", "0")
+        out_b = ssm.ssm_state_update(st_b, xd["x"], xd["dt"], xd["A"], xd["B"], xd["C"], D=xd["D"],
+                                     z=xd.get("z"), dt_bias=xd["dt_bias"], **kw)
+        A_ref = f64(x["A"])
+        if kw["scalar_a"]:
+            A_ref = np.repeat(A_ref[:, None], N, axis=1)
+        ro = oracle.state_update(ref, f64(x["x"]), f64(x["dt"]), A_ref, f64(x["B"]), f64(x["C"]),
+                                 D=f64(x["D"]), z=None if "z" not in x else f64(x["z"]),
+                                 dt_bias=f64(x["dt_bias"]), zoh=kw["zoh"])
+        assert torch.equal(out_a, out_b) and torch.equal(st_a, st_b), f"step {t}"
+        assert_close(out_a, ro, io, f"out step {t}")
+        assert_close(st_a, ref, torch.float32 if io == torch.float32 else io, f"state step {t}")
+    assert _abi.wait_timeouts() == 0

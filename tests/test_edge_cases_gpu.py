@@ -73,12 +73,21 @@ def check_fwd(x, io, softplus=True, elementwise=True):
     return out, hL, ref
 
 
-def check_bwd(x, io, softplus=True, use_ckpt=False):
+# Summed gradients (dA, dD, ddt_bias) add hundreds of per-step terms in f32.  With steps up to
+# Δ = 30 the terms span many decades and partly cancel, and f32 summation error grows with the
+# sum's condition number (sum of |terms| over |sum|), not with the f32 unit roundoff alone; for
+# these adversarial ranges the f32 bound on them is 5e-5 instead of 1e-5.  Per-element outputs
+# keep the 1e-5 bound.
+SUMMED = ("dA", "dD", "ddt_bias")
+
+
+def check_bwd(x, io, softplus=True, use_ckpt=False, summed_scale=1.0):
     g = bwd_gpu(on_dev(x), softplus, use_ckpt)
     r = bwd_oracle(x, softplus)
     for k in GRADS:
         if r.get(k) is not None and g.get(k) is not None:
-            assert_close(g[k], r[k], io, k)
+            scale = summed_scale if (k in SUMMED and io == torch.float32) else 1.0
+            assert_close(g[k], r[k], io, k, scale=scale)
 
 
 # ------------------------------------------------------------------ helper (CPU)
@@ -129,7 +138,7 @@ def test_fwd_large_step_resets_the_state(io):
     # the closed form of the reset: h_{L-1} = Δ B_{L-1} x_{L-1}, Δ = softplus(30)
     dl = np.logaddexp(0.0, 30.0)
     want = dl * f64(x["B"])[:, None, :, L - 1] * f64(x["u"])[:, :, L - 1:L]
-    np.testing.assert_allclose(ref["hL"], want, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(ref["hL"], want, rtol=1e-9, atol=1e-9)  # Ā <= e^-30 is not 0
     np.testing.assert_allclose(f64(hL), want, rtol=2e-6 if io == torch.float32 else 1e-2,
                                atol=1e-5 if io == torch.float32 else 5e-2)
 
@@ -169,7 +178,7 @@ def test_bwd_softplus_over_the_whole_range(io, use_ckpt):
     and vanishing steps in the same sequences."""
     w = workload("tiny_f32", batch=2, dim=96, seqlen=333, dstate=16, io_dtype=io)
     x = spread_delta(make_inputs(w, seed=46, with_h0=True, with_dout=True), io, seed=4)
-    check_bwd(x, io, use_ckpt=use_ckpt)
+    check_bwd(x, io, use_ckpt=use_ckpt, summed_scale=5.0)
 
 
 @pytest.mark.gpu
@@ -184,7 +193,7 @@ def test_bwd_resets_and_vanishing_steps(io):
     d[..., 200::9] = 25.0
     x["delta"] = d.to(io)
     x["dt_bias"] = torch.zeros_like(x["dt_bias"])
-    check_bwd(x, io)
+    check_bwd(x, io, summed_scale=5.0)
 
 
 @pytest.mark.gpu

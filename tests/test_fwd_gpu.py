@@ -42,7 +42,8 @@ def run_oracle(x, softplus=True, sel=None):
 
 @pytest.fixture(autouse=True)
 def _clean_env(monkeypatch):
-    monkeypatch.delenv("SSM_FWD_SPLIT", raising=False)
+    for k in ("SSM_FWD_SPLIT", "SSM_FWD_KERNEL", "SSM_FWD_KMUFU"):
+        monkeypatch.delenv(k, raising=False)
     yield
 
 
@@ -86,10 +87,13 @@ def test_bf16_medium_full():
     assert_close(out, run_oracle(x)["out"], torch.bfloat16, "out")
 
 
-@pytest.mark.parametrize("kmufu", [8, 10, 12, 14, 16])
-def test_every_exponential_split(monkeypatch, kmufu):
-    """Each split of the exponentials between MUFU and the FMA-pipe polynomial (the default
-    depends on the warps per SM), on a ragged length so full and partial blocks both run."""
+@pytest.mark.parametrize("kernel,kmufu", [("lane", k) for k in (10, 11, 12, 13, 14, 15, 16)] +
+                         [("pair", k) for k in (14, 16)])
+def test_every_exponential_split(monkeypatch, kernel, kmufu):
+    """Each split of the exponentials between MUFU and the FMA-pipe polynomial, in both kernel
+    families (one lane per channel; two lanes per channel), on a length that is not a multiple
+    of the 16-step block so full and partial blocks both run."""
+    monkeypatch.setenv("SSM_FWD_KERNEL", kernel)
     monkeypatch.setenv("SSM_FWD_KMUFU", str(kmufu))
     w = workload("mamba370m_fwd", batch=2, dim=200, seqlen=1000)
     x = make_inputs(w, seed=11, with_h0=True)
@@ -100,10 +104,11 @@ def test_every_exponential_split(monkeypatch, kmufu):
 
 
 @pytest.mark.parametrize("wide", [0, 1])
-@pytest.mark.parametrize("kmufu", [12, 14, 16])
+@pytest.mark.parametrize("kmufu", [14, 16])
 def test_both_register_budgets(monkeypatch, wide, kmufu):
     """The output kernel's default and 255-register forms (chosen by warps per SM) agree with the
-    oracle, on a ragged length, and with each other bitwise."""
+    oracle, on a ragged length, and with each other bitwise (two-lanes-per-channel kernel)."""
+    monkeypatch.setenv("SSM_FWD_KERNEL", "pair")
     monkeypatch.setenv("SSM_FWD_KMUFU", str(kmufu))
     w = workload("mamba370m_fwd", batch=2, dim=160, seqlen=777)
     x = make_inputs(w, seed=13, with_h0=True)
@@ -115,10 +120,10 @@ def test_both_register_budgets(monkeypatch, wide, kmufu):
 
 
 @pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
-@pytest.mark.parametrize("lpc", [1, 2, 4])
-def test_lanes_per_channel(monkeypatch, io, lpc):
-    """1, 2 or 4 lanes per channel (state split across lanes), with the time split too."""
-    monkeypatch.setenv("SSM_FWD_LPC", str(lpc))
+def test_general_kernel_with_and_without_time_split(monkeypatch, io):
+    """The general (two-lanes-per-channel) kernel on the default variant, with the time split
+    too (it serves rows that do not allow 16-byte copies, and every other variant)."""
+    monkeypatch.setenv("SSM_FWD_KERNEL", "pair")
     w = workload("tiny_f32", batch=2, dim=40, seqlen=301, dstate=16, io_dtype=io)
     x = make_inputs(w, seed=12, with_h0=True)
     out, hL = run_gpu(on_dev(x), return_final_state=True)
