@@ -260,8 +260,12 @@ def run_reference(args, rank, world):
 
 
 # ------------------------------------------------------------------ our arm
-def bench_extras(dev):
-    """Timing of the other hot-path calls on their workloads (inputs drawn on the GPU)."""
+EXTRAS = ("train", "scalar_decay", "variants", "long_seq", "decode")
+
+
+def bench_extras(dev, which=EXTRAS):
+    """Timing of the other hot-path calls on their workloads (inputs drawn on the GPU); `which`
+    selects the measurements."""
     import selective_state_space_23_b200 as ssm
     g = torch.Generator(device=dev).manual_seed(1)
     out = {}
@@ -287,7 +291,22 @@ def bench_extras(dev):
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / reps
 
+    N = 16
     # training step (forward with checkpoints + backward) on the Mamba-2.8B-shaped layer
+    if "train" in which:
+        out.update(_train_step(dev, rnd, prm, timeit))
+    if "scalar_decay" in which or "variants" in which:
+        out.update(_variants(dev, rnd, prm, timeit, g, which))
+    if "long_seq" in which:
+        out.update(_long_seq(dev, rnd, prm, timeit))
+    if "decode" in which:
+        out.update(_decode(dev, rnd, prm, timeit))
+    return out
+
+
+def _train_step(dev, rnd, prm, timeit):
+    import selective_state_space_23_b200 as ssm
+    out = {}
     b, d, L, N = 4, 5120, 2048, 16
     u, de, z, dout = rnd((b, d, L)), rnd((b, d, L), 0.5), rnd((b, d, L)), rnd((b, d, L))
     B, C = rnd((b, N, L)), rnd((b, N, L))
@@ -307,7 +326,13 @@ def bench_extras(dev):
                               "fwd_bwd_ms": ms_tr, "tokens_per_s": b * L / (ms_tr * 1e-3)}
     del u, de, z, dout, ws
     torch.cuda.empty_cache()
+    return out
 
+
+def _variants(dev, rnd, prm, timeit, g, which):
+    import selective_state_space_23_b200 as ssm
+    out = {}
+    N = 16
     # scalar decay (one rate per channel) on the Mamba-370m-shaped layer
     b, d, L = 8, 2048, 2048
     u, de, z = rnd((b, d, L)), rnd((b, d, L), 0.5), rnd((b, d, L))
@@ -315,10 +340,13 @@ def bench_extras(dev):
     _, D, bias = prm(d, N, 1e-3, 1e-1)
     A1 = -(torch.rand(d, device=dev, generator=g) * 15.0 + 1.0)
     o = torch.empty_like(u)
-    ms = timeit(lambda: ssm.ssm_scan_fwd_scalar_a(u, de, A1, B, C, D=D, z=z, dt_bias=bias, out=o), 20)
-    out["scalar_decay_fwd"] = {"shape": "8x2048x2048 N16 bf16, A [dim]", "fwd_ms": ms,
-                               "tokens_per_s": b * L / (ms * 1e-3),
-                               "hbm_gbs": compulsory_bytes_shape(b, d, L, N) / (ms * 1e-3) / 1e9}
+    if "scalar_decay" in which:
+        ms = timeit(lambda: ssm.ssm_scan_fwd_scalar_a(u, de, A1, B, C, D=D, z=z, dt_bias=bias, out=o), 20)
+        out["scalar_decay_fwd"] = {"shape": "8x2048x2048 N16 bf16, A [dim]", "fwd_ms": ms,
+                                   "tokens_per_s": b * L / (ms * 1e-3),
+                                   "hbm_gbs": compulsory_bytes_shape(b, d, L, N) / (ms * 1e-3) / 1e9}
+        if "variants" not in which:
+            return out
 
     # the other variants of the forward scan on the same layer
     A, D, bias = prm(d, N, 1e-3, 1e-1)
@@ -326,8 +354,16 @@ def bench_extras(dev):
     uc, dec, zc = (t.transpose(1, 2).contiguous() for t in (u, de, z))
     Bc, Cc = B.transpose(1, 2).contiguous(), C.transpose(1, 2).contiguous()
     oc = torch.empty_like(uc)
+    def general_kernel():  # the default variant in the two-lanes-per-channel kernel
+        os.environ["SSM_FWD_KERNEL"] = "pair"
+        try:
+            ssm.ssm_scan_fwd(u, de, A, B, C, D=D, z=z, dt_bias=bias, out=o)
+        finally:
+            del os.environ["SSM_FWD_KERNEL"]
+
     var = {
         "default": lambda: ssm.ssm_scan_fwd(u, de, A, B, C, D=D, z=z, dt_bias=bias, out=o),
+        "default_general_kernel": general_kernel,
         "zoh": lambda: ssm.ssm_scan_fwd(u, de, A, B, C, D=D, z=z, dt_bias=bias, out=o, zoh=True),
         "reverse": lambda: ssm.ssm_scan_fwd(u, de, A, B, C, D=D, z=z, dt_bias=bias, out=o,
                                             reverse=True),
@@ -339,7 +375,13 @@ def bench_extras(dev):
                               **{k: timeit(f, 20) for k, f in var.items()}}
     del u, de, z, B, C, o, Bg, Cg, uc, dec, zc, Bc, Cc, oc
     torch.cuda.empty_cache()
+    return out
 
+
+def _long_seq(dev, rnd, prm, timeit):
+    import selective_state_space_23_b200 as ssm
+    out = {}
+    N = 16
     # long sequence
     b, d, L = 1, 256, 1 << 20
     u, de, z = rnd((b, d, L)), rnd((b, d, L), 0.5), rnd((b, d, L))
@@ -352,7 +394,13 @@ def bench_extras(dev):
                           "tokens_per_s": b * L / (ms * 1e-3), "hbm_gbs": byt / (ms * 1e-3) / 1e9}
     del u, de, z, B, C, ws
     torch.cuda.empty_cache()
+    return out
 
+
+def _decode(dev, rnd, prm, timeit):
+    import selective_state_space_23_b200 as ssm
+    out = {}
+    N = 16
     # decode: 256 x 5120 x 16 state.  The 84 MB state fits in L2 (126 MB), so L2 is flushed
     # before every step by READING 256 MB (clean lines: no write-back lands inside the step) and
     # the state comes from HBM; the flush is timed separately and subtracted
@@ -385,6 +433,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--extras", default=",".join(EXTRAS),
+                    help="comma-separated side measurements to run: " + ",".join(EXTRAS))
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-baseline", action="store_true", help="skip the CPU oracle timing")
     args = ap.parse_args()
@@ -503,7 +553,7 @@ def main():
     extras = {} if world == 1 else {"skipped": "the side measurements run at N=1 only"}
     if not args.no_extras and world == 1:
         try:  # side measurements: a failure here is reported, it does not cost the main line
-            extras = bench_extras(dev)
+            extras = bench_extras(dev, tuple(x for x in args.extras.split(",") if x))
         except Exception as e:  # noqa: BLE001
             extras = {"error": f"{type(e).__name__}: {e}"[:300]}
     line = {

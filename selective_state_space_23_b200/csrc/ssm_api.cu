@@ -137,13 +137,16 @@ int check_dims(int batch, int dim, int seqlen, int dstate, int io) {
 
 size_t esize(int io) { return io == SSM_BF16 ? 2 : 4; }
 
-// B/C groups: dim must split into groups of whole warps (16 channels each).
+// B/C groups: dim must split into groups of whole warps (16 channels each), or into single
+// channels (bc_groups == dim: B/C per channel).
 int check_groups(int dim, int bc_groups) {
   if (bc_groups < 1) return fail(SSM_EINVAL, "bc_groups must be >= 1, got %d", bc_groups);
-  if (bc_groups == 1) return SSM_OK;
+  if (bc_groups == 1 || bc_groups == dim) return SSM_OK;
   if (dim % bc_groups != 0) return fail(SSM_EINVAL, "dim %d is not a multiple of bc_groups %d", dim, bc_groups);
   if ((dim / bc_groups) % 16 != 0)
-    return fail(SSM_EUNSUPPORTED, "grouped B/C needs dim / bc_groups to be a multiple of 16 (got %d)",
+    return fail(SSM_EUNSUPPORTED,
+                "grouped B/C needs dim / bc_groups to be a multiple of 16, or bc_groups == dim "
+                "(got %d channels per group)",
                 dim / bc_groups);
   return SSM_OK;
 }
@@ -324,9 +327,14 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
   const bool vec = !channels_last && (seqlen * es) % 16 == 0 && aligned16(u) &&
                    aligned16(delta) && aligned16(z) && aligned16(out) && aligned16(B) &&
                    aligned16(C);
-  const bool lane = fwd_lane_allowed() && vec && !scalar_a && !zoh && !reverse &&
+  // B/C per channel (bc_groups == dim > 1): the per-state kernel of ssm_pcbc.cu, no time split
+  const bool pcbc = bc_groups == dim && bc_groups > 1;
+  if (pcbc && (scalar_a || zoh || reverse || channels_last))
+    return fail(SSM_EUNSUPPORTED, "B/C per channel combines with no other variant flag");
+  const bool lane = !pcbc && fwd_lane_allowed() && vec && !scalar_a && !zoh && !reverse &&
                     (bc_groups == 1 || (dim / bc_groups) % 32 == 0);
   FwdPlan plan = plan_fwd(batch, dim, seqlen, fwd_chw(lane));
+  if (pcbc) plan.nchunk = 1;
   if (plan.nchunk > 1 && (!workspace || workspace_bytes < plan.ws_bytes ||
                           (reinterpret_cast<uintptr_t>(workspace) & 255))) {
     plan.nchunk = 1;  // not enough scratch: same result without the time split
@@ -366,6 +374,15 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
   const int km = fwd_kmufu(a.nwarps * (long long)plan.nchunk);
   a.wide = fwd_wide(a.nwarps * (long long)plan.nchunk);
   cudaError_t e;
+  if (pcbc) {
+    plan.chunk_len = (int)nblk * ssm::kBlk;
+    a.chunk_len = plan.chunk_len; a.nchunk = 1;
+    const bool pvec = (seqlen * es) % 16 == 0 && aligned16(u) && aligned16(delta) &&
+                      aligned16(z) && aligned16(out) && aligned16(B) && aligned16(C);
+    if ((e = ssm::launch_fwd_pcbc(a, io_dtype, pvec, ssm::kFwdOut, s)) != cudaSuccess)
+      return cuda_fail(e, "forward pass (B/C per channel)");
+    return SSM_OK;
+  }
   if (plan.nchunk > 1) {
     const size_t nch = (size_t)batch * dim;
     char* w = reinterpret_cast<char*>(workspace);
@@ -517,7 +534,26 @@ int scan_bwd_core(const void* u, const void* delta, const float* A, const void* 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
 
+  const bool pcbc = bc_groups == dim && bc_groups > 1;
+  if (pcbc && (reverse || zoh || channels_last))
+    return fail(SSM_EUNSUPPORTED, "B/C per channel combines with no other variant flag");
+  const bool pvec = (seqlen * es) % 16 == 0 && aligned16(u) && aligned16(delta) &&
+                    aligned16(z) && aligned16(dout) && aligned16(du) && aligned16(ddelta) &&
+                    aligned16(dz) && aligned16(B) && aligned16(C) && aligned16(dB) && aligned16(dC);
   const float* ck = ckpt;
+  if (!ck && pcbc) {
+    ssm::FwdArgs a;
+    memset(&a, 0, sizeof(a));
+    a.u = u; a.delta = delta; a.B = B; a.C = C; a.A = A; a.dt_bias = dt_bias; a.h0 = h0;
+    a.ckpt = ck_ws;
+    a.batch = batch; a.dim = dim; a.L = seqlen; a.N = dstate;
+    a.chunk_len = (int)nblk * ssm::kBlk; a.nchunk = 1;
+    a.softplus = delta_softplus ? 1 : 0;
+    a.bc_groups = bc_groups;
+    if ((e = ssm::launch_fwd_pcbc(a, io_dtype, pvec, ssm::kFwdCkpt, s)) != cudaSuccess)
+      return cuda_fail(e, "backward state replay pass (B/C per channel)");
+    ck = ck_ws;
+  }
   if (!ck) {
     ssm::FwdArgs a;
     memset(&a, 0, sizeof(a));
@@ -558,6 +594,13 @@ int scan_bwd_core(const void* u, const void* delta, const float* A, const void* 
   b.wpb = l.wpb;
   b.ngroups = l.ngroups;
   b.kmufu = env_int("SSM_BWD_KMUFU", 4);  // all exponentials on MUFU measured fastest
+  if (pcbc) {
+    if ((e = ssm::launch_bwd_pcbc(b, io_dtype, pvec, dB, dC, s)) != cudaSuccess)
+      return cuda_fail(e, "backward pass (B/C per channel)");
+    if ((e = ssm::launch_bwd_finish_adt(b, dA, dD, ddt_bias, s)) != cudaSuccess)
+      return cuda_fail(e, "backward reduction");
+    return SSM_OK;
+  }
   // the default variant with N = 16 and rows of whole 8-step pieces: the state history in
   // registers (ssm_bwd_hist.cu); SSM_BWD_KERNEL=pair forces the general kernel
   const char* bk = getenv("SSM_BWD_KERNEL");

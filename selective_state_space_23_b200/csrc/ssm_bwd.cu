@@ -679,6 +679,12 @@ cudaError_t launch_bwd_finish(const BwdArgs& a, int io, void* dB, void* dC, floa
         a, reinterpret_cast<float*>(dB), reinterpret_cast<float*>(dC));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  return launch_bwd_finish_adt(a, dA, dD, ddt_bias, s);
+}
+
+cudaError_t launch_bwd_finish_adt(const BwdArgs& a, float* dA, float* dD, float* ddt_bias,
+                                  cudaStream_t s) {
+  const int tpb = 256;
   const long long nadt = (long long)a.dim * (kNS + 2);
   bwd_finish_adt<<<(unsigned)((nadt + tpb - 1) / tpb), tpb, 0, s>>>(a, dA, dD, ddt_bias);
   return cudaGetLastError();

@@ -119,6 +119,13 @@ cudaError_t launch_bwd(const BwdArgs& a, int io, bool vec, cudaStream_t s);
 // ceil(ceil(dim / 16) / a.wpb), each CTA inside one B/C group.
 cudaError_t launch_bwd_hist(const BwdArgs& a, int io, cudaStream_t s);
 int bwd_hist_pick_wpb(int io, int batch, int dim);
+// B/C per channel (bc_groups == dim, ssm_pcbc.cu): forward (mode kFwdOut or kFwdCkpt) and
+// backward (writes du, ddelta, dz, dB, dC, dh0 and the per-channel dA/dD/ddt_bias partials).
+cudaError_t launch_fwd_pcbc(const FwdArgs& a, int io, bool vec, int mode, cudaStream_t s);
+cudaError_t launch_bwd_pcbc(const BwdArgs& a, int io, bool vec, void* dB, void* dC, cudaStream_t s);
+// dA, dD, ddt_bias from the per-channel partials (the second half of launch_bwd_finish).
+cudaError_t launch_bwd_finish_adt(const BwdArgs& a, float* dA, float* dD, float* ddt_bias,
+                                  cudaStream_t s);
 cudaError_t launch_bwd_finish(const BwdArgs& a, int io, void* dB, void* dC, float* dA, float* dD,
                               float* ddt_bias, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, int io, cudaStream_t s);

@@ -48,10 +48,11 @@ def run_fwd(x, cl, **kw):
 
 @pytest.fixture(autouse=True)
 def _clean_env(monkeypatch):
-    # the channels-last layout runs in the general (two-lanes-per-channel) kernel; the default
+    # the channels-last layout runs in the general (two-lanes-per-channel) kernels; the default
     # layout is compared with it bitwise, so it runs there too
     monkeypatch.delenv("SSM_FWD_SPLIT", raising=False)
     monkeypatch.setenv("SSM_FWD_KERNEL", "pair")
+    monkeypatch.setenv("SSM_BWD_KERNEL", "pair")
     yield
 
 

@@ -61,10 +61,11 @@ def test_matches_device_call(pin, batch, dim, L, io):
 
 
 def test_bitwise_when_no_time_split(monkeypatch):
-    """5120 channels fill the GPU one row at a time: no chunk and no full call splits time (and
-    the exponential split is pinned, as the default depends on the warps per launch)."""
+    """Two rows of 5120 channels (the host call's chunk for a batch of 16) fill the GPU: no chunk
+    and no full call splits time, so the host call and the device call run the same kernel
+    launches on the same rows (the exponential split is pinned too)."""
     monkeypatch.setenv("SSM_FWD_KMUFU", "16")
-    w = workload("mamba2p8b_train", batch=8, seqlen=256)
+    w = workload("mamba2p8b_train", batch=16, seqlen=256)
     x = make_inputs(w, seed=95)
     assert torch.equal(host_result(x, True), device_result(x).cpu())
 
