@@ -354,8 +354,8 @@ def _variants(dev, rnd, prm, timeit, g, which):
     uc, dec, zc = (t.transpose(1, 2).contiguous() for t in (u, de, z))
     Bc, Cc = B.transpose(1, 2).contiguous(), C.transpose(1, 2).contiguous()
     oc = torch.empty_like(uc)
-    def general_kernel():  # the default variant in the two-lanes-per-channel kernel
-        os.environ["SSM_FWD_KERNEL"] = "pair"
+    def lane_kernel():  # the default variant in the one-lane-per-channel kernel
+        os.environ["SSM_FWD_KERNEL"] = "lane"
         try:
             ssm.ssm_scan_fwd(u, de, A, B, C, D=D, z=z, dt_bias=bias, out=o)
         finally:
@@ -363,7 +363,7 @@ def _variants(dev, rnd, prm, timeit, g, which):
 
     var = {
         "default": lambda: ssm.ssm_scan_fwd(u, de, A, B, C, D=D, z=z, dt_bias=bias, out=o),
-        "default_general_kernel": general_kernel,
+        "default_lane_kernel": lane_kernel,
         "zoh": lambda: ssm.ssm_scan_fwd(u, de, A, B, C, D=D, z=z, dt_bias=bias, out=o, zoh=True),
         "reverse": lambda: ssm.ssm_scan_fwd(u, de, A, B, C, D=D, z=z, dt_bias=bias, out=o,
                                             reverse=True),

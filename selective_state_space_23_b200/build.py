@@ -56,13 +56,6 @@ def _obj_stale(src: str) -> bool:
     return any(os.path.getmtime(p) > t for p in _deps(os.path.join(CSRC, src)))
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
-        return True
-    t = os.path.getmtime(LIB)
-    return any(os.path.getmtime(p) > t for p in _inputs())
-
-
 def _compile(src: str, verbose: bool) -> str:
     obj = _obj(src)
     cmd = [NVCC, *ARCH, *FLAGS, "-c", os.path.join(CSRC, src), "-o", obj]
@@ -77,14 +70,18 @@ def _compile(src: str, verbose: bool) -> str:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every kernel source for sm_100a and link the shared library; return its path."""
-    if not force and not _stale():
-        return LIB
+    """Compile every kernel source for sm_100a and link the shared library; return its path.
+    Objects are recompiled when they are older than any file they include; the library is
+    relinked when an object was rebuilt or is newer than it."""
     os.makedirs(BUILD_DIR, exist_ok=True)
     todo = [s for s in SOURCES if force or _obj_stale(s)]  # objects older than their includes
-    with cf.ThreadPoolExecutor(max_workers=max(1, len(todo))) as ex:
-        list(ex.map(lambda s: _compile(s, verbose), todo))
+    if todo:
+        with cf.ThreadPoolExecutor(max_workers=len(todo)) as ex:
+            list(ex.map(lambda s: _compile(s, verbose), todo))
     objs = [_obj(s) for s in SOURCES]
+    if (not todo and os.path.exists(LIB)
+            and all(os.path.getmtime(o) <= os.path.getmtime(LIB) for o in objs)):
+        return LIB
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = [NVCC, *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", tmp, *objs, "-cudart", "static"]
     r = subprocess.run(cmd, capture_output=True, text=True)

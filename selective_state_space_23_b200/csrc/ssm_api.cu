@@ -164,12 +164,15 @@ struct FwdPlan {
 // Lanes per channel of the general forward kernel (8 states per lane).
 int fwd_lpc() { return 2; }
 
-// Kernel family of the forward scan: the one-lane-per-channel kernel (ssm_fwd_lane.cuh) serves
-// the default variant whenever its rows allow 16-byte copies; SSM_FWD_KERNEL=pair forces the
-// general kernel (ssm_fwd_impl.cuh), which serves every variant and layout.
+// Kernel family of the forward scan.  The general two-lanes-per-channel kernel
+// (ssm_fwd_impl.cuh) serves every variant and layout and is the default: measured on B200 it is
+// faster than the one-lane-per-channel kernel (ssm_fwd_lane.cuh) on every workload here (8 x 2048
+// x 2048: 263 against 314 us), whose single warp per scheduler leaves fixed-latency dependencies
+// exposed.  SSM_FWD_KERNEL=lane selects the latter for the default variant when its rows allow
+// 16-byte copies.
 bool fwd_lane_allowed() {
   const char* v = getenv("SSM_FWD_KERNEL");
-  return !(v && strcmp(v, "pair") == 0);
+  return v && strcmp(v, "lane") == 0;
 }
 
 // Channels per warp of each kernel family.

@@ -25,7 +25,10 @@
 //     butterfly: lanes whose channel slot has bit 3 set hold their 8 states rotated by 4, so the
 //     butterfly's first level (8 of its 15 shuffles) needs no selects; the CTA's warps are then
 //     added in shared memory in a fixed order and written as one partial per (CTA, b, n, t),
-//     which the finishing kernel of ssm_bwd.cu sums in a fixed order (bitwise reproducible).
+//     which the finishing kernel of ssm_bwd.cu sums in a fixed order (bitwise reproducible);
+//   * 16.6 KB of shared memory per warp (the step outputs reuse the step scalars' slots), so a
+//     CTA of 4 warps leaves room for 3 per SM: the 320 CTAs of a 4 x 5120-channel row set run
+//     in one wave.
 #include <type_traits>
 
 #include "ssm_device.cuh"
@@ -48,9 +51,8 @@ struct HGeo {
   static constexpr int kSlotBytes = kRowsBytes + kRawBytes + kCkBytes;
   static constexpr int kWarpBytes = 2 * kSlotBytes          // ring: this block and the next
                                     + 2 * kBCS * 4          // B/C tile as f32
-                                    + kBlk * kCW * 16       // per-step scalars
-                                    + kBlk * kCW * 16       // per-step outputs
-                                    + 2 * kBlk * 32 * 4;    // dB/dC warp sums, two blocks
+                                    + kBlk * kCW * 16       // per-step scalars, then outputs
+                                    + kBlk * 32 * 4;        // dB/dC warp sums of the block
 };
 
 // 16 bytes from global to shared; src_bytes < 16 zero-fills the rest (0: nothing is read).
@@ -126,9 +128,10 @@ struct HistBwd {
   __device__ __forceinline__ float4* table() const {
     return reinterpret_cast<float4*>(wsm + 2 * G::kSlotBytes + 2 * kBCS * 4);
   }
-  __device__ __forceinline__ float4* outs() const { return table() + kBlk * kCW; }
-  __device__ __forceinline__ float* red(int blk) const {
-    return reinterpret_cast<float*>(outs() + kBlk * kCW) + (blk & 1) * kBlk * 32;
+  // the outputs of step k replace its scalars once both lanes of the channel have read them
+  __device__ __forceinline__ float4* outs() const { return table(); }
+  __device__ __forceinline__ float* red() const {
+    return reinterpret_cast<float*>(table() + kBlk * kCW);
   }
 
   // Copies of block blk: the lane's 8 steps (8 q ..) of its channel's u, delta, z, dout; its
@@ -247,6 +250,7 @@ struct HistBwd {
     s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
     s2 += __shfl_xor_sync(0xffffffffu, s2, 1);
     y += __shfl_xor_sync(0xffffffffu, y, 1);
+    __syncwarp();  // both lanes of the channel have read the scalars of step k
     if (q == half) {
       const float aback = kPrecise ? 1.f : kLn2;  // al * aback = A
       const float du = fmaf(sc.z, Dd, sc.x * s1);
@@ -284,7 +288,7 @@ struct HistBwd {
     const float send = b0 ? v[0] : v[8];
     const float tot = keep + __shfl_xor_sync(0xffffffffu, send, 2);
     const int n = 8 * q + ((2 * (int)b2 + (int)b1 + 4 * rot) & 7);
-    red(blkcur)[k * 32 + (int)b0 * 16 + n] = tot;
+    red()[k * 32 + (int)b0 * 16 + n] = tot;
   }
 
   int blkcur;
@@ -453,7 +457,7 @@ __global__ void __launch_bounds__(32 * W) bwd_hist_kernel(const __grid_constant_
       for (int w = 0; w < W; ++w) {
         const float* rw = reinterpret_cast<const float*>(
             reinterpret_cast<const unsigned char*>(redw0) + (size_t)w * G::kWarpBytes +
-            2 * G::kSlotBytes + 2 * kBCS * 4 + 2 * kBlk * kCW * 16) + (blk & 1) * kBlk * 32;
+            2 * G::kSlotBytes + 2 * kBCS * 4 + kBlk * kCW * 16);
 #pragma unroll
         for (int i = 0; i < 4; ++i) sum[i] += rw[(4 * tq + i) * 32 + e];
       }
@@ -462,6 +466,7 @@ __global__ void __launch_bounds__(32 * W) bwd_hist_kernel(const __grid_constant_
       *reinterpret_cast<float4*>(a.part_bc + prow * a.L + t0 + 4 * tq) =
           make_float4(sum[0], sum[1], sum[2], sum[3]);
     }
+    __syncthreads();  // the warps' sums are read before the next block writes them again
   }
 
   dD_acc += __shfl_xor_sync(0xffffffffu, dD_acc, 1);

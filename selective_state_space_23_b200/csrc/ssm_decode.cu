@@ -289,30 +289,29 @@ __global__ void __launch_bounds__(kStreamThreads) decode_stream_kernel(const __g
   if (tid == 0)
     for (int r = 0; r < kStages && r < nrows; ++r) issue(r, r);
 
-  // per-channel parameters, once for every batch row of the CTA
+  // per-channel parameters, once for every batch row of the CTA (A times log2 e for the MUFU
+  // exponential of the bf16 path)
+  const float ascale = (kPrecise || a.zoh) ? 1.f : kLog2e;
   float An[8];
   if (a.scalar_a) {
-    const float ad = __ldg(a.A + d);
+    const float ad = __ldg(a.A + d) * ascale;
 #pragma unroll
     for (int i = 0; i < 8; ++i) An[i] = ad;
   } else {
     const float4* ap = reinterpret_cast<const float4*>(a.A + (long long)d * kNS + 8 * q);
     const float4 a0 = __ldg(ap), a1 = __ldg(ap + 1);
-    An[0] = a0.x; An[1] = a0.y; An[2] = a0.z; An[3] = a0.w;
-    An[4] = a1.x; An[5] = a1.y; An[6] = a1.z; An[7] = a1.w;
+    An[0] = a0.x * ascale; An[1] = a0.y * ascale; An[2] = a0.z * ascale; An[3] = a0.w * ascale;
+    An[4] = a1.x * ascale; An[5] = a1.y * ascale; An[6] = a1.z * ascale; An[7] = a1.w * ascale;
   }
   const float bias = a.dt_bias ? a.dt_bias[d] : 0.f;
   const float Dd = a.D ? a.D[d] : 0.f;
 
-  bool ok = true;
+  // one barrier per row: it carries every thread's "row r + 1 has landed" and marks the end of
+  // every thread's reads of row r, after which row r's stage is refilled
+  bool ok = __syncthreads_and(mbar_wait(&bars[0], 0u));
   int r = 0;
-  for (; r < nrows; ++r) {
+  for (; ok && r < nrows; ++r) {
     const int stage = r % kStages;
-    const bool landed = mbar_wait(&bars[stage], (uint32_t)((r / kStages) & 1));
-    if (!__syncthreads_and(landed)) {  // the whole CTA stops together
-      ok = false;
-      break;
-    }
     const StreamStage<IO>& sg = st[stage];
     const float xv = ld_io<IO>(sg.x, cl);
     const float v = ld_io<IO>(sg.dt, cl) + bias;
@@ -321,19 +320,36 @@ __global__ void __launch_bounds__(kStreamThreads) decode_stream_kernel(const __g
     const float4 h0 = reinterpret_cast<const float4*>(sg.state + cl * kNS + 8 * q)[0];
     const float4 h1 = reinterpret_cast<const float4*>(sg.state + cl * kNS + 8 * q)[1];
     float h[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+    float Bn[8], Cn[8];
+    if constexpr (sizeof(IO) == 2) {
+      const uint4 bw = *reinterpret_cast<const uint4*>(sg.B + 8 * q);
+      const uint4 cw = *reinterpret_cast<const uint4*>(sg.C + 8 * q);
+      const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w}, cc[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        Bn[2 * i] = bf16_lo(bb[i]); Bn[2 * i + 1] = bf16_hi(bb[i]);
+        Cn[2 * i] = bf16_lo(cc[i]); Cn[2 * i + 1] = bf16_hi(cc[i]);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        Bn[i] = ld_io<IO>(sg.B, 8 * q + i);
+        Cn[i] = ld_io<IO>(sg.C, 8 * q + i);
+      }
+    }
     float y = 0.f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const float Bn = ld_io<IO>(sg.B, 8 * q + i), Cn = ld_io<IO>(sg.C, 8 * q + i);
-      const float abar = (kPrecise || a.zoh) ? expf(dt * An[i]) : ex2_mufu(dt * An[i] * kLog2e);
+      const float abar = (kPrecise || a.zoh) ? expf(dt * An[i]) : ex2_mufu(dt * An[i]);
       const float bx = a.zoh ? decode_coef(dt, An[i], true) * xv : dx;
-      h[i] = fmaf(abar, h[i], bx * Bn);
-      y = fmaf(Cn, h[i], y);
+      h[i] = fmaf(abar, h[i], bx * Bn[i]);
+      y = fmaf(Cn[i], h[i], y);
     }
     y += __shfl_xor_sync(0xffffffffu, y, 1);
     const float zv = a.z ? ld_io<IO>(sg.z, cl) : 0.f;
-    __syncthreads();  // every thread has read this stage
-    if (tid == 0 && r + kStages < nrows) issue(r + kStages, stage);
+    const bool landed = r + 1 >= nrows || mbar_wait(&bars[(r + 1) % kStages], (uint32_t)(((r + 1) / kStages) & 1));
+    ok = __syncthreads_and(landed);
+    if (ok && tid == 0 && r + kStages < nrows) issue(r + kStages, stage);
     const long long ch = (long long)(b0 + r) * a.dim + d;
     float4* sp = reinterpret_cast<float4*>(a.state + ch * kNS + 8 * q);
     sp[0] = make_float4(h[0], h[1], h[2], h[3]);
@@ -346,9 +362,10 @@ __global__ void __launch_bounds__(kStreamThreads) decode_stream_kernel(const __g
   }
   if (!ok) {
     // a copy never completed: record it, wait (bounded) for the copies still in flight so none
-    // lands after the CTA's shared memory is released, and stop
+    // lands after the CTA's shared memory is released, and stop.  Rows before the failed one
+    // are complete; the failed row and the ones after it are not written.
     if (tid == 0) atomicAdd(&g_wait_timeouts, 1u);
-    for (int rr = r; rr < nrows && rr < r + kStages; ++rr)
+    for (int rr = r; rr < nrows && rr < r + kStages; ++rr)  // r: the row that did not land
       mbar_wait(&bars[rr % kStages], (uint32_t)((rr / kStages) & 1));
   }
 }

@@ -419,9 +419,13 @@ __global__ void __launch_bounds__(32, 1) fwd_lane_kernel(const __grid_constant__
     if (MODE == kFwdSummary) kahan(dsum);
     cp_wait<kStages - 3>();  // block i+1 has landed (this lane's copies)
     __syncwarp();            // ... and every other lane's
-    const bool fast = !kPrecise && __all_sync(0xffffffffu, m <= dlim);
-    if (fast) sc.template body<KE, KO>(i, h, al, dl, du, m, dsum);
-    else sc.template body<8, 8>(i, h, al, dl, du, m, dsum);
+    if constexpr (kPrecise || (KE == 8 && KO == 8)) {
+      sc.template body<8, 8>(i, h, al, dl, du, m, dsum);  // every exponential on MUFU: no vote
+    } else {
+      const bool fast = __all_sync(0xffffffffu, m <= dlim);
+      if (fast) sc.template body<KE, KO>(i, h, al, dl, du, m, dsum);
+      else sc.template body<8, 8>(i, h, al, dl, du, m, dsum);
+    }
     __syncwarp();  // slot i-1 and B/C buffer i&1 are free for reuse
   }
   cp_wait<0>();

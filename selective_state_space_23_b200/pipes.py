@@ -30,14 +30,14 @@ def measure(iters: int = 4096, ctas_per_sm: int = 4, threads: int = 256) -> dict
     f = lib.ssm_pipe_probe
     f.restype = ctypes.c_int
     f.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                  ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]
+                  ctypes.POINTER(ctypes.c_double)]
     out = {"ctas_per_sm": ctas_per_sm, "threads_per_cta": threads, "iters": iters}
     for kind, name in ((0, "ffma_fp32_ops"), (1, "ffma2_fp32_ops"), (2, "mufu_ex2")):
-        cyc, ops = ctypes.c_double(), ctypes.c_double()
-        rc = f(kind, iters, ctas_per_sm, threads, ctypes.byref(cyc), ctypes.byref(ops))
+        rate = ctypes.c_double()
+        rc = f(kind, iters, ctas_per_sm, threads, ctypes.byref(rate))
         if rc != 0:
             raise RuntimeError(f"pipe probe {name} failed ({rc})")
-        out[name + "_per_clk_per_sm"] = ops.value * ctas_per_sm / cyc.value
+        out[name + "_per_clk_per_sm"] = rate.value
     return out
 
 

@@ -124,3 +124,21 @@ def test_mamba2p8b_train_step_full_size():
     r0 = oracle_grads(x, channels=list(range(5120)))  # batch row 0, every channel
     for k in ("dB", "dC"):
         assert_close(g[k][0], r0[k][0], torch.bfloat16, k)
+
+
+@pytest.mark.parametrize("fwd_kernel", ["pair", "lane"])
+@pytest.mark.parametrize("bwd_kernel", ["pair", "hist"])
+def test_kernel_families(monkeypatch, fwd_kernel, bwd_kernel):
+    """Every pairing of the forward kernel that writes the checkpoints (or replays the states
+    when none are given) with the backward kernel that consumes them: the one-lane-per-channel
+    or two-lanes-per-channel forward, and the register-history or general backward."""
+    monkeypatch.setenv("SSM_FWD_KERNEL", fwd_kernel)
+    if bwd_kernel == "pair":
+        monkeypatch.setenv("SSM_BWD_KERNEL", "pair")
+    else:
+        monkeypatch.delenv("SSM_BWD_KERNEL", raising=False)
+    w = workload("mamba2p8b_train", batch=2, dim=96, seqlen=312)
+    x = make_inputs(w, seed=14, with_dout=True, with_h0=True)
+    r = oracle_grads(x)
+    for use_ckpt in (False, True):
+        compare(gpu_grads(on_dev(x), use_ckpt=use_ckpt), r, torch.bfloat16)

@@ -74,8 +74,9 @@ def test_fma_polynomial_and_mufu_within_bounds(monkeypatch):
     assert rate_err.max() < 2e-3  # limited by the f32 spacing of a near 1, not by the polynomial
 
 
-@pytest.mark.parametrize("L", [1, 8])
-def test_exact_one_when_step_is_zero(L):
+@pytest.mark.parametrize("L,kernel", [(1, "pair"), (8, "pair"), (8, "lane")])
+def test_exact_one_when_step_is_zero(monkeypatch, L, kernel):
+    monkeypatch.setenv("SSM_FWD_KERNEL", kernel)
     dim, N = 64, 16
     A = -torch.rand((dim, N)) * 10
     a_gpu, _ = run(torch.zeros(dim), A, L=L)
@@ -87,7 +88,7 @@ def test_lane_kernel_exponentials_within_bounds(monkeypatch):
     (states 0..7) take MUFU and states 8..15 the polynomial.  A warp (32 channels) any of whose
     lanes has a step beyond the polynomial's range runs the block with every exponential on
     MUFU."""
-    monkeypatch.delenv("SSM_FWD_KERNEL", raising=False)
+    monkeypatch.setenv("SSM_FWD_KERNEL", "lane")
     monkeypatch.setenv("SSM_FWD_KMUFU", "8")
     r = np.random.default_rng(1)
     dim, N = 4096, 16
