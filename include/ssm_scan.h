@@ -60,6 +60,8 @@ extern "C" {
 #define SSM_CKPT_STEPS 16
 /* Largest supported dstate (N). */
 #define SSM_MAX_DSTATE 16
+/* Largest dstate of the scalar-decay forward scan (SSM_SCALAR_A; N = 32, 64 or 128 above 16). */
+#define SSM_MAX_DSTATE_SCALAR 128
 
 typedef enum { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype;
 

@@ -123,13 +123,13 @@ int check_opt(const void* p, size_t bytes, size_t align, const char* name) {
     if (_rc != SSM_OK) return _rc; \
   } while (0)
 
-int check_dims(int batch, int dim, int seqlen, int dstate, int io) {
+int check_dims(int batch, int dim, int seqlen, int dstate, int io, int max_dstate = SSM_MAX_DSTATE) {
   if (batch <= 0 || dim <= 0 || seqlen <= 0 || dstate <= 0)
     return fail(SSM_EINVAL, "sizes must be positive (batch=%d dim=%d seqlen=%d dstate=%d)", batch,
                 dim, seqlen, dstate);
   if (io != SSM_F32 && io != SSM_BF16) return fail(SSM_EINVAL, "io_dtype %d is not SSM_F32/SSM_BF16", io);
-  if (dstate > SSM_MAX_DSTATE)
-    return fail(SSM_EUNSUPPORTED, "dstate %d > %d is not implemented", dstate, SSM_MAX_DSTATE);
+  if (dstate > max_dstate)
+    return fail(SSM_EUNSUPPORTED, "dstate %d > %d is not implemented", dstate, max_dstate);
   if ((long long)batch * ((dim + 31) / 32) > (1LL << 30))
     return fail(SSM_EUNSUPPORTED, "batch*dim too large for one launch");
   return SSM_OK;
@@ -303,7 +303,8 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
   if (flags & ~(SSM_SCALAR_A | SSM_REVERSE | SSM_ZOH | SSM_CHANNELS_LAST))
     return fail(SSM_EINVAL, "unknown flags 0x%x", flags);
   const bool scalar_a = (flags & SSM_SCALAR_A) != 0;
-  TRY(check_dims(batch, dim, seqlen, dstate, io_dtype));
+  // scalar decay takes N up to 128 (the chunked matrix form, ssm_ssd.cu); per-state decay 16
+  TRY(check_dims(batch, dim, seqlen, dstate, io_dtype, scalar_a ? SSM_MAX_DSTATE_SCALAR : SSM_MAX_DSTATE));
   TRY(check_groups(dim, bc_groups));
   const size_t es = esize(io_dtype);
   const size_t nx = (size_t)batch * dim * seqlen * es;
@@ -330,6 +331,29 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
   const bool vec = !channels_last && (seqlen * es) % 16 == 0 && aligned16(u) &&
                    aligned16(delta) && aligned16(z) && aligned16(out) && aligned16(B) &&
                    aligned16(C);
+  // scalar decay with N > 16: the chunked matrix form on the tensor cores (bf16, N = 32, 64 or
+  // 128, forward direction, [batch][dim][L] rows, B/C shared by each 64-channel tile)
+  if (dstate > SSM_MAX_DSTATE) {
+    if (io_dtype != SSM_BF16 || (dstate != 32 && dstate != 64 && dstate != 128) || zoh ||
+        reverse || channels_last || ckpt ||
+        !(bc_groups == 1 || (dim % bc_groups == 0 && (dim / bc_groups) % 64 == 0)))
+      return fail(SSM_EUNSUPPORTED,
+                  "scalar decay with dstate %d > %d needs bf16 io, dstate 32, 64 or 128, the "
+                  "forward direction without ZOH, the default layout, no checkpoints and B/C "
+                  "groups of whole 64-channel tiles", dstate, SSM_MAX_DSTATE);
+    ssm::FwdArgs a;
+    memset(&a, 0, sizeof(a));
+    a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
+    a.A = A; a.D = D; a.dt_bias = dt_bias; a.h0 = h0; a.out = out; a.hL = hL;
+    a.batch = batch; a.dim = dim; a.L = seqlen; a.N = dstate;
+    a.softplus = delta_softplus ? 1 : 0;
+    a.scalar_a = 1;
+    a.bc_groups = bc_groups;
+    a.rows16 = vec ? 1 : 0;
+    cudaError_t e = ssm::launch_ssd_fwd(a, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "forward pass (chunked matrix form)");
+    return SSM_OK;
+  }
   // B/C per channel (bc_groups == dim > 1): the per-state kernel of ssm_pcbc.cu, no time split
   const bool pcbc = bc_groups == dim && bc_groups > 1;
   if (pcbc && (scalar_a || zoh || reverse || channels_last))

@@ -82,14 +82,16 @@ __global__ void __launch_bounds__(256) decode_kernel(const DecodeArgs a) {
     const int n = 4 * q + i;
     const bool live = n < N;
     if (!VEC) h[i] = live ? sp[i] : 0.f;
-    An[i] = live ? a.A[a.scalar_a ? (long long)d : (long long)d * N + n] : 0.f;
+    // A times log2 e for the MUFU exponential (every decode form rounds the same product)
+    An[i] = live ? a.A[a.scalar_a ? (long long)d : (long long)d * N + n] * ((kPrecise || a.zoh) ? 1.f : kLog2e)
+                 : 0.f;
     Bn[i] = live ? ld_io<IO>(a.B, bc + n) : 0.f;
     Cn[i] = live ? ld_io<IO>(a.C, bc + n) : 0.f;
   }
   float y = 0.f;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const float abar = (kPrecise || a.zoh) ? expf(dt * An[i]) : ex2_mufu(dt * An[i] * kLog2e);
+    const float abar = (kPrecise || a.zoh) ? expf(dt * An[i]) : ex2_mufu(dt * An[i]);
     const float bx = a.zoh ? decode_coef(dt, An[i], true) * xv : dx;
     h[i] = fmaf(abar, h[i], bx * Bn[i]);
     y = fmaf(Cn[i], h[i], y);
@@ -135,9 +137,11 @@ __global__ void __launch_bounds__(256) decode16_kernel(const DecodeArgs a) {
   const float4 h0 = reinterpret_cast<const float4*>(sp)[0];  // default caching: the state is
   const float4 h1 = reinterpret_cast<const float4*>(sp)[1];  // reused by the next step
   float h[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+  // A times log2 e for the MUFU exponential (every decode form rounds the same product)
+  const float ascale = (kPrecise || a.zoh) ? 1.f : kLog2e;
   float An[8];
   if (a.scalar_a) {
-    const float ad = __ldg(a.A + d);
+    const float ad = __ldg(a.A + d) * ascale;
 #pragma unroll
     for (int i = 0; i < 8; ++i) An[i] = ad;
   } else {
@@ -145,7 +149,7 @@ __global__ void __launch_bounds__(256) decode16_kernel(const DecodeArgs a) {
     const float4 a0 = __ldg(ap), a1 = __ldg(ap + 1);
     const float at[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) An[i] = at[i];
+    for (int i = 0; i < 8; ++i) An[i] = at[i] * ascale;
   }
   const long long bc = ((long long)b * a.bc_groups + d / (a.dim / a.bc_groups)) * kNS + 8 * q;
   float Bn[8], Cn[8];
@@ -170,7 +174,7 @@ __global__ void __launch_bounds__(256) decode16_kernel(const DecodeArgs a) {
   float y = 0.f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float abar = (kPrecise || a.zoh) ? expf(dt * An[i]) : ex2_mufu(dt * An[i] * kLog2e);
+    const float abar = (kPrecise || a.zoh) ? expf(dt * An[i]) : ex2_mufu(dt * An[i]);
     const float bx = a.zoh ? decode_coef(dt, An[i], true) * xv : dx;
     h[i] = fmaf(abar, h[i], bx * Bn[i]);
     y = fmaf(Cn[i], h[i], y);

@@ -50,6 +50,7 @@ struct FwdArgs {
   int cl_tile;          // channels-last rows moved as 16-byte tiles (dim % 16 == 0, N == 16, aligned)
   int lpc;              // lanes per channel: 1, 2 or 4 (16 / lpc states each)
   int wide;             // few warps per SM: the 255-register form of the output kernel
+  int rows16;           // rows along L in aligned 16-byte pieces (L * es % 16 == 0, aligned tensors)
   int warps_per_b;      // ceil(dim / (32 / lpc))
   long long nwarps;     // batch * warps_per_b
 };
@@ -110,6 +111,10 @@ cudaError_t launch_fwd(const FwdArgs& a, int io, bool vec, int mode, int wpb, in
 // channels_last; rows allow 16-byte copies; a.warps_per_b = ceil(dim / 32); dim / bc_groups a
 // multiple of 32).
 cudaError_t launch_fwd_lane(const FwdArgs& a, int io, int mode, int kmufu, cudaStream_t s);
+// Scalar decay with N = 32, 64 or 128 (bf16 io): the chunked matrix form on the tensor cores
+// (ssm_ssd.cu).  B, C shared by each CTA's 64 channels (bc_groups == 1 or dim / bc_groups a
+// multiple of 64); a.rows16 selects 16-byte row accesses.
+cudaError_t launch_ssd_fwd(const FwdArgs& a, cudaStream_t s);
 cudaError_t launch_fwd_carry(const FwdArgs& a, const float* summ, const float* dsum, float* hin,
                              cudaStream_t s);
 cudaError_t launch_bwd(const BwdArgs& a, int io, bool vec, cudaStream_t s);

@@ -1,0 +1,113 @@
+"""Scalar decay with large state sizes (N = 32, 64, 128; the Mamba-2 setting of the "2024 Reading
+List: Neural Network" page): the chunked matrix form on the tensor cores, through the C ABI,
+against the fp64 oracle run with A broadcast over the states.  Ragged lengths, partial channel
+tiles, options, grouped B/C, the Mamba-370m layer shape on sampled channels, and steps large
+enough that chunks leave the factorised form's range and take its exact sequential pass."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import selective_state_space_23_b200 as ssm
+from selective_state_space_23_b200.inputs import make_inputs, workload
+
+from _parity import assert_close, f64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def inputs(batch, dim, L, N, seed, gate=True, groups=1):
+    w = workload("mamba370m_fwd", batch=batch, dim=dim, seqlen=L, dstate=N)
+    x = make_inputs(w, seed=seed, with_h0=True, gate=gate, scalar_a=True)
+    if groups > 1:
+        wg = workload("mamba370m_fwd", batch=batch * groups, dim=1, seqlen=L, dstate=N)
+        xg = make_inputs(wg, seed=seed + 500)
+        x["B"] = xg["B"].reshape(batch, groups, N, L).contiguous()
+        x["C"] = xg["C"].reshape(batch, groups, N, L).contiguous()
+    return x
+
+
+def gpu(x, softplus=True):
+    xd = {k: v.to(DEV) for k, v in x.items()}
+    return ssm.ssm_scan_fwd_scalar_a(xd["u"], xd["delta"], xd["A"], xd["B"], xd["C"], D=xd.get("D"),
+                                     z=xd.get("z"), dt_bias=xd.get("dt_bias"),
+                                     delta_softplus=softplus, h0=xd.get("h0"),
+                                     return_final_state=True)
+
+
+def ref(x, softplus=True, channels=None):
+    c = lambda k: None if x.get(k) is None else f64(x[k])
+    N = x["B"].shape[-2]
+    A = np.repeat(c("A")[:, None], N, axis=1)
+    return oracle.scan_fwd(c("u"), c("delta"), A, c("B"), c("C"), D=c("D"), z=c("z"),
+                           dt_bias=c("dt_bias"), delta_softplus=softplus, h0=c("h0"),
+                           channels=channels)
+
+
+@pytest.mark.parametrize("N", [32, 64, 128])
+@pytest.mark.parametrize("shape", [(2, 128, 256), (1, 96, 200), (2, 64, 17)])
+def test_matches_oracle(N, shape):
+    batch, dim, L = shape
+    x = inputs(batch, dim, L, N, seed=61)
+    out, hL = gpu(x)
+    r = ref(x)
+    assert_close(out, r["out"], torch.bfloat16, "out")
+    assert_close(hL, r["hL"], torch.bfloat16, "hL")
+
+
+@pytest.mark.parametrize("N", [64, 128])
+def test_without_gate_bias_softplus(N):
+    x = inputs(2, 64, 160, N, seed=62, gate=False)
+    x["delta"] = (x["delta"].float().abs() * 0.05 + 1e-3).to(torch.bfloat16)
+    del x["dt_bias"], x["D"]
+    out, hL = gpu(x, softplus=False)
+    r = ref(x, softplus=False)
+    assert_close(out, r["out"], torch.bfloat16, "out")
+    assert_close(hL, r["hL"], torch.bfloat16, "hL")
+
+
+def test_grouped_bc():
+    x = inputs(2, 256, 128, 64, seed=63, groups=2)  # 128 channels per group
+    out, hL = gpu(x)
+    r = ref(x)
+    assert_close(out, r["out"], torch.bfloat16, "out")
+
+
+@pytest.mark.parametrize("N", [64, 128])
+def test_large_steps_take_the_sequential_pass(N):
+    """v = delta + dt_bias over [-30, 30]: many chunks exceed |A| S <= 80 and are computed by
+    the exact sequential pass, next to chunks in the factorised form."""
+    x = inputs(2, 128, 200, N, seed=64)
+    v = np.random.default_rng(3).uniform(-30, 30, size=x["delta"].shape).astype(np.float32)
+    x["delta"] = torch.from_numpy(v).to(torch.bfloat16)
+    x["dt_bias"] = torch.zeros_like(x["dt_bias"])
+    out, hL = gpu(x)
+    r = ref(x)
+    assert_close(out, r["out"], torch.bfloat16, "out")
+    assert_close(hL, r["hL"], torch.bfloat16, "hL")
+
+
+@pytest.mark.parametrize("N", [64, 128])
+def test_mamba370m_shape_sampled(N):
+    """8 x 2048 x 2048 (the Mamba-370m layer shape) with N states: every output of 32 sampled
+    channels per batch row, and their final states."""
+    x = inputs(8, 2048, 2048, N, seed=65)
+    out, hL = gpu(x)
+    torch.cuda.synchronize()
+    sel = list(range(0, 2048, 64))
+    chans = [b * 2048 + d for b in range(8) for d in sel]
+    r = ref(x, channels=chans)
+    idx = torch.as_tensor(sel, device=DEV)
+    assert_close(out.index_select(1, idx), r["out"][:, sel], torch.bfloat16, "out")
+    assert_close(hL.index_select(1, idx), r["hL"][:, sel], torch.bfloat16, "hL")
+
+
+def test_unsupported_requests_are_refused():
+    x = inputs(1, 64, 32, 48, seed=66)
+    with pytest.raises(RuntimeError):
+        gpu(x)  # N = 48
+    x = inputs(1, 64, 32, 64, seed=67)
+    x = {k: (v.float() if v.dtype == torch.bfloat16 else v) for k, v in x.items()}
+    with pytest.raises(RuntimeError):
+        gpu(x)  # f32 io
