@@ -73,8 +73,8 @@ def load_peaks():
     return dict(FALLBACK_PEAKS)
 
 
-# Sources of the kernel that runs the benchmark step (the one-lane-per-channel forward kernel)
-KERNEL_SOURCES = ("ssm_fwd_lane.cuh", "ssm_fwd_lane_bf16.cu", "ssm_device.cuh", "ssm_kernels.h")
+# Sources of the kernel that runs the benchmark step (the general two-lanes forward kernel)
+KERNEL_SOURCES = ("ssm_fwd_impl.cuh", "ssm_fwd_bf16.cu", "ssm_device.cuh", "ssm_kernels.h", "ssm_rows.cuh")
 
 
 def kernel_source_hash() -> str:
@@ -260,7 +260,7 @@ def run_reference(args, rank, world):
 
 
 # ------------------------------------------------------------------ our arm
-EXTRAS = ("train", "scalar_decay", "variants", "long_seq", "decode")
+EXTRAS = ("train", "scalar_decay", "variants", "long_seq", "decode", "ssd")
 
 
 def bench_extras(dev, which=EXTRAS):
@@ -301,6 +301,31 @@ def bench_extras(dev, which=EXTRAS):
         out.update(_long_seq(dev, rnd, prm, timeit))
     if "decode" in which:
         out.update(_decode(dev, rnd, prm, timeit))
+    if "ssd" in which:
+        out.update(_ssd(dev, rnd, prm, timeit, g))
+    return out
+
+
+def _ssd(dev, rnd, prm, timeit, g):
+    """Scalar decay with 64 and 128 states on the Mamba-370m-shaped layer (the chunked matrix
+    form on the tensor cores)."""
+    import selective_state_space_23_b200 as ssm
+    out = {}
+    b, d, L = 8, 2048, 2048
+    u, de, z = rnd((b, d, L)), rnd((b, d, L), 0.5), rnd((b, d, L))
+    _, D, bias = prm(d, 16, 1e-3, 1e-1)
+    A1 = -(torch.rand(d, device=dev, generator=g) * 15.0 + 1.0)
+    o = torch.empty_like(u)
+    res = {"shape": "8x2048x2048 bf16, A [dim]"}
+    for N in (64, 128):
+        B, C = rnd((b, N, L)), rnd((b, N, L))
+        ms = timeit(lambda: ssm.ssm_scan_fwd_scalar_a(u, de, A1, B, C, D=D, z=z, dt_bias=bias, out=o), 10)
+        # the chunk products per 16 steps and 64 channels: C B^T, mask(G) X', C H, B^T X''
+        flops = 2.0 * b * (L // 16) * (d // 64) * (16 * 16 * N + 16 * 16 * 64 + 16 * N * 64 + N * 16 * 64)
+        res[f"N{N}"] = {"fwd_ms": ms, "tokens_per_s": b * L / (ms * 1e-3),
+                        "hbm_gbs": (4 * b * d * L * 2 + 2 * b * N * L * 2) / (ms * 1e-3) / 1e9,
+                        "mma_tflops": flops / (ms * 1e-3) / 1e12}
+    out["scalar_decay_large_n"] = res
     return out
 
 

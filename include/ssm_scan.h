@@ -30,7 +30,8 @@
  *     dout, du, ddelta, dz, dB, dC, x, dt): SSM_F32 or SSM_BF16.  A, D, dt_bias, h0, hL, ckpt,
  *     dhL, dh0, dA, dD, ddt_bias and state are always float32.
  *   - All tensors are dense and row-major (last index contiguous), with the layouts given per
- *     argument.  1 <= dstate <= 16 (SSM_EUNSUPPORTED above).
+ *     argument.  1 <= dstate <= 16 (SSM_EUNSUPPORTED above), except the scalar-decay forward
+ *     scan, which also takes dstate 32, 64 and 128.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream) and the call
  *     returns without synchronising.  A launch failure is reported by the return value; an
  *     error raised later by the device is reported by CUDA on the stream as usual.
@@ -68,7 +69,7 @@ typedef enum { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype;
 typedef enum {
   SSM_OK = 0,
   SSM_EINVAL = 1,        /* invalid argument; nothing was launched */
-  SSM_EUNSUPPORTED = 2,  /* valid request this build does not implement (e.g. dstate > 16) */
+  SSM_EUNSUPPORTED = 2,  /* valid request this build does not implement (e.g. dstate 48) */
   SSM_ECUDA = 3,         /* a CUDA runtime call or kernel launch failed */
   SSM_EWORKSPACE = 4     /* workspace NULL or smaller than the size function returned */
 } ssm_status;
@@ -155,6 +156,13 @@ SSM_API int ssm_scan_bwd(const void* u, const void* delta, const float* A, const
  * The backward needs ssm_scan_bwd_scalar_a_workspace_size() bytes of workspace (256-byte
  * aligned): A broadcast to [dim][dstate] and the per-state dA, followed by the workspace of
  * ssm_scan_bwd for the same shape.  Checkpoints of ssm_scan_fwd_scalar_a feed the backward.
+ * dstate may be up to SSM_MAX_DSTATE_SCALAR in the forward scan: above 16 it runs in the chunked
+ * matrix form (per 16-step chunk and 64-channel tile, the products C B^T, masked with the decay
+ * factors, times the step-scaled inputs, plus C times the entering state: the structured-matrix
+ * view of the scan in the Mamba-2 notes of the same page) on the tensor cores.  That form takes
+ * bf16 io, dstate 32, 64 or 128, the forward direction without SSM_ZOH, the default layout, no
+ * checkpoints, and B/C groups of whole 64-channel tiles; other requests with dstate > 16, and the
+ * backward with dstate > 16, return SSM_EUNSUPPORTED.
  */
 SSM_API size_t ssm_scan_fwd_scalar_a_workspace_size(int batch, int dim, int seqlen, int dstate,
                                                     int io_dtype);
@@ -206,6 +214,9 @@ SSM_API int ssm_scan_bwd_scalar_a(const void* u, const void* delta, const float*
  *                 grouping Mamba-2 uses; 1 = shared by every channel).  dim must be a multiple of
  *                 bc_groups (else SSM_EINVAL) and dim / bc_groups a multiple of 16 (the channels
  *                 of one warp share a group; else SSM_EUNSUPPORTED).
+ *                 bc_groups == dim gives B, C (and dB, dC) per channel, [batch][dim][dstate][L]
+ *                 (B_t, C_t computed from each channel's own input); dB, dC are then per channel,
+ *                 not summed over d.  Per-channel B/C combines with no flag (SSM_EUNSUPPORTED).
  */
 #define SSM_SCALAR_A 1
 #define SSM_REVERSE 2
@@ -294,7 +305,8 @@ SSM_API int ssm_state_update(float* state, const void* x, const void* dt, const 
 /*
  * ssm_state_update with the variants of the scan: flags SSM_SCALAR_A (A is [dim]) and SSM_ZOH
  * (the zero-order-hold input coefficient); B, C are [batch][bc_groups][dstate] (channel d uses
- * group d / (dim / bc_groups); dim / bc_groups a multiple of 16 when bc_groups > 1).  A decode
+ * group d / (dim / bc_groups); dim / bc_groups a multiple of 16 when 1 < bc_groups < dim;
+ * bc_groups == dim gives B, C per channel, [batch][dim][dstate]).  A decode
  * step runs forward in time: SSM_REVERSE is rejected with SSM_EINVAL, as is any unknown bit.
  * Calling it L times reproduces ssm_scan_fwd_ex with the same flags and groups.
  */
