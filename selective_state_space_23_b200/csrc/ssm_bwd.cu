@@ -397,7 +397,8 @@ __global__ void __launch_bounds__(128) bwd_kernel(const BwdArgs a) {
   const IO* zp = a.z ? reinterpret_cast<const IO*>(a.z) + row : nullptr;
   const IO* gp = reinterpret_cast<const IO*>(a.dout) + row;
   const bool bc_live = slot < N;  // the lane also stages B/C row `slot`, steps [8 q, 8 q + 8)
-  const int gbc = ((grp * a.wpb + wib) * kCW) / (a.dim / a.bc_groups);  // the warp's B/C group
+  // the warp's B/C group (a warp wholly past dim shadows the last channel's)
+  const int gbc = min((grp * a.wpb + wib) * kCW, a.dim - 1) / (a.dim / a.bc_groups);
   const long long bcrow = cl ? ((long long)b * L * a.bc_groups + gbc) * N + (bc_live ? slot : 0)
                              : (((long long)b * a.bc_groups + gbc) * N + (bc_live ? slot : 0)) * L;
   const IO* Bp = reinterpret_cast<const IO*>(a.B) + bcrow;

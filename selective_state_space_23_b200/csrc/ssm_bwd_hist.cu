@@ -114,7 +114,7 @@ struct HistBwd {
 
   const BwdArgs& a;
   unsigned char* wsm;  // this warp's shared memory
-  int lane, s, q, rot, b, d0w, L, nblk;
+  int lane, s, q, rot, b, d0w, gbc, L, nblk;
   long long ch;
   bool act;
   int qlo, qhi;        // offsets of the lane's two state quads in a B/C tile row
@@ -161,7 +161,7 @@ struct HistBwd {
       const int n = lane >> 1, hh = lane & 1;
       const long long tb = (long long)blk * kBlk + 8 * hh;
       const bool have_bc = tb < L;
-      const long long bcrow = (((long long)b * a.bc_groups + d0w / (a.dim / a.bc_groups)) * kNS + n) * L +
+      const long long bcrow = (((long long)b * a.bc_groups + gbc) * kNS + n) * L +
                               (have_bc ? tb : 0);
       const int nbc = have_bc ? 16 : 0;
       unsigned char* raw = sl + G::kRowsBytes;
@@ -333,6 +333,8 @@ __global__ void __launch_bounds__(32 * W) bwd_hist_kernel(const __grid_constant_
   hb.rot = (hb.s >> 3) & 1;
   hb.b = b;
   hb.d0w = (grp * W + wib) * kCW;
+  // the warp's B/C group; a warp wholly past dim (last CTA of a row) shadows the last channel's
+  hb.gbc = min(hb.d0w, a.dim - 1) / (a.dim / a.bc_groups);
   const int d = hb.d0w + hb.s;
   hb.act = d < a.dim;
   const int dd = hb.act ? d : a.dim - 1;
