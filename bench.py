@@ -417,7 +417,15 @@ def _long_seq(dev, rnd, prm, timeit):
     byt = 4 * b * d * L * 2 + 2 * b * N * L * 2
     out["long_seq_1m"] = {"shape": "1x256x1048576 N16 bf16", "fwd_ms": ms,
                           "tokens_per_s": b * L / (ms * 1e-3), "hbm_gbs": byt / (ms * 1e-3) / 1e9}
-    del u, de, z, B, C, ws
+    # backward of the same sequence (time-split history backward) from the forward's checkpoints
+    _, ck = ssm.ssm_scan_fwd(u, de, A, B, C, D=D, z=z, dt_bias=bias, return_ckpt=True, workspace=ws)
+    dout = rnd((b, d, L))
+    wsb = torch.empty(ssm.bwd_workspace_bytes(b, d, L, N, torch.bfloat16, True), dtype=torch.uint8,
+                      device=dev)
+    ms_b = timeit(lambda: ssm.ssm_scan_bwd(u, de, A, B, C, dout, D=D, z=z, dt_bias=bias, ckpt=ck,
+                                           workspace=wsb), 5)
+    out["long_seq_1m"]["bwd_ms"] = ms_b
+    del u, de, z, B, C, ws, ck, dout, wsb
     torch.cuda.empty_cache()
     return out
 

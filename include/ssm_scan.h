@@ -327,6 +327,75 @@ SSM_API int ssm_state_update_ex(float* state, const void* x, const void* dt, con
  */
 SSM_API int ssm_wait_timeouts(unsigned int* count);
 
+/*
+ * General element strides.  The entry points above take dense tensors (the layouts given per
+ * argument, or the (B, L, D) layout of SSM_CHANNELS_LAST).  These take each io tensor with its
+ * own element strides, e.g. views cut out of a larger projection output, transposed views, or B
+ * and C broadcast over the batch with stride 0 ("Seçim Mekanizması (S6)": the selective
+ * parameters come from projections of the input, in whatever layout those produce).  Strides
+ * are in elements, one per index of the tensor's logical shape:
+ *   [batch][dim][L] tensors (u, delta, z, out, dout, du, ddelta, dz): (batch, dim, t)
+ *   [batch][bc_groups][dstate][L] tensors (B, C, dB, dC): (batch, group, state, t)
+ * Strides must be >= 0; an output's strides must not map two of its elements to one address
+ * (SSM_EINVAL otherwise).  Each tensor's allocation must hold every element the strides reach.
+ * A tensor whose strides are the dense ones is used in place; any other is gathered into (or,
+ * for an output, scattered from) a dense copy in the workspace by the library's own copy kernel
+ * around the dense call, so the results equal those of the dense entry points bitwise.  f32
+ * tensors (A, D, dt_bias, h0, hL, ckpt, dhL, dA, dD, ddt_bias, dh0) stay dense.  flags:
+ * SSM_SCALAR_A, SSM_REVERSE, SSM_ZOH (SSM_CHANNELS_LAST is one set of strides: SSM_EINVAL).
+ * The workspace holds the dense copies followed by the dense call's workspace; its size does not
+ * depend on the strides.
+ */
+typedef struct ssm_strides {
+  long long u[3], delta[3], z[3], out[3];      /* forward tensors: (batch, dim, t) */
+  long long dout[3], du[3], ddelta[3], dz[3];  /* backward tensors: (batch, dim, t) */
+  long long B[4], C[4], dB[4], dC[4];          /* (batch, group, state, t) */
+} ssm_strides;
+
+SSM_API size_t ssm_scan_fwd_strided_workspace_size(int batch, int dim, int seqlen, int dstate,
+                                                   int bc_groups, int io_dtype, int flags);
+SSM_API int ssm_scan_fwd_strided(const void* u, const void* delta, const float* A, const void* B,
+                                 const void* C, const float* D, const void* z,
+                                 const float* dt_bias, int delta_softplus, const float* h0,
+                                 float* hL, void* out, float* ckpt, void* workspace,
+                                 size_t workspace_bytes, int batch, int dim, int seqlen,
+                                 int dstate, int bc_groups, int io_dtype, int flags,
+                                 const ssm_strides* strides, void* stream);
+SSM_API size_t ssm_scan_bwd_strided_workspace_size(int batch, int dim, int seqlen, int dstate,
+                                                   int bc_groups, int io_dtype, int have_ckpt,
+                                                   int flags);
+SSM_API int ssm_scan_bwd_strided(const void* u, const void* delta, const float* A, const void* B,
+                                 const void* C, const float* D, const void* z,
+                                 const float* dt_bias, int delta_softplus, const float* h0,
+                                 const void* dout, const float* dhL, const float* ckpt, void* du,
+                                 void* ddelta, float* dA, void* dB, void* dC, float* dD, void* dz,
+                                 float* ddt_bias, float* dh0, void* workspace,
+                                 size_t workspace_bytes, int batch, int dim, int seqlen,
+                                 int dstate, int bc_groups, int io_dtype, int flags,
+                                 const ssm_strides* strides, void* stream);
+
+/*
+ * The decode step with general element strides (same rules as above):
+ *   state (batch, dim, state) f32, updated in place;  x, dt, z, out (batch, dim) io;
+ *   B, C (batch, group, state) io.
+ * flags: SSM_SCALAR_A, SSM_ZOH.  Needs ssm_state_update_strided_workspace_size() bytes of
+ * workspace (256-byte aligned) for the dense copies.
+ */
+typedef struct ssm_decode_strides {
+  long long state[3];
+  long long x[2], dt[2], z[2], out[2];
+  long long B[3], C[3];
+} ssm_decode_strides;
+
+SSM_API size_t ssm_state_update_strided_workspace_size(int batch, int dim, int dstate,
+                                                       int bc_groups, int io_dtype);
+SSM_API int ssm_state_update_strided(float* state, const void* x, const void* dt, const float* A,
+                                     const void* B, const void* C, const float* D, const void* z,
+                                     const float* dt_bias, int delta_softplus, void* out,
+                                     void* workspace, size_t workspace_bytes, int batch, int dim,
+                                     int dstate, int bc_groups, int io_dtype, int flags,
+                                     const ssm_decode_strides* strides, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -8,6 +8,9 @@ allocated here with torch.  Work is enqueued on the current torch CUDA stream.
   ssm_scan_fwd      forward selective scan (gated output, optional final state / checkpoints)
   ssm_scan_bwd      gradients of ssm_scan_fwd, recomputing the states
   ssm_state_update  one-token recurrent step, state updated in place
+
+with variants (``*_scalar_a``, flags), the host-memory forward ``ssm_scan_fwd_host`` and the
+``*_strided`` forms that take io tensors with arbitrary element strides.
 """
 import ctypes
 
@@ -18,7 +21,8 @@ from ._abi import CKPT_STEPS, MAX_DSTATE
 
 __all__ = ["ssm_scan_fwd", "ssm_scan_bwd", "ssm_scan_fwd_scalar_a", "ssm_scan_bwd_scalar_a",
            "ssm_scan_fwd_host", "fwd_host_workspace_bytes",
-           "ssm_state_update", "fwd_workspace_bytes",
+           "ssm_state_update", "fwd_workspace_bytes", "ssm_scan_fwd_strided",
+           "ssm_scan_bwd_strided", "ssm_state_update_strided",
            "bwd_workspace_bytes", "CKPT_STEPS", "MAX_DSTATE", "library_path"]
 
 _IO = {torch.float32: _abi.SSM_F32, torch.bfloat16: _abi.SSM_BF16}
@@ -329,4 +333,184 @@ def ssm_state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, delta_
         _ptr(dt_bias), int(bool(delta_softplus)), _ptr(out), batch, dim, N, G, code, flags,
         _stream(dev))
     _abi.check(rc, "ssm_state_update_ex")
+    return out
+
+
+# ------------------------------------------------------------------ general element strides
+def _view(t, name, shape, dtype, device):
+    """A tensor of the given logical shape with any non-negative element strides."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _bc_view(B, batch, L):
+    """(groups, N, strides (batch, group, state, t)) of B/C given as [batch, N, L] or
+    [batch, G, N, L] with any strides."""
+    if B.dim() == 3:
+        return 1, B.shape[1], (B.stride(0), 0, B.stride(1), B.stride(2))
+    if B.dim() == 4:
+        return B.shape[1], B.shape[2], tuple(B.stride())
+    raise ValueError(f"B must be [batch, N, L] or [batch, groups, N, L], got {tuple(B.shape)}")
+
+
+def _set(arr, vals):
+    for i, v in enumerate(vals):
+        arr[i] = v
+
+
+def ssm_scan_fwd_strided(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=True,
+                         h0=None, return_final_state=False, out=None, workspace=None,
+                         scalar_a=False, reverse=False, zoh=False):
+    """:func:`ssm_scan_fwd` for io tensors with arbitrary (non-negative) element strides: u,
+    delta, z (and ``out``, if given) [batch, dim, L]; B, C [batch, N, L] or [batch, G, N, L]
+    (e.g. expanded over the batch with stride 0).  Results equal the dense call's bitwise."""
+    dev = _on_gpu(u, "u")
+    batch, dim, L = u.shape
+    io = u.dtype
+    code = _io_code(io)
+    G, N, sbc = _bc_view(B, batch, L)
+    xs = (batch, dim, L)
+    bshape = tuple(B.shape)
+    for t, n in ((u, "u"), (delta, "delta")):
+        _view(t, n, xs, io, dev)
+    if z is not None:
+        _view(z, "z", xs, io, dev)
+    _view(B, "B", bshape, io, dev)
+    _view(C, "C", bshape, io, dev)
+    _need(A, "A", (dim,) if scalar_a else (dim, N), torch.float32, dev)
+    _opt(D, "D", (dim,), torch.float32, dev)
+    _opt(dt_bias, "dt_bias", (dim,), torch.float32, dev)
+    _opt(h0, "h0", (batch, dim, N), torch.float32, dev)
+    if out is None:
+        out = torch.empty(xs, dtype=io, device=dev)
+    _view(out, "out", xs, io, dev)
+    hL = torch.empty((batch, dim, N), dtype=torch.float32, device=dev) if return_final_state else None
+    st = _abi.Strides()
+    _set(st.u, u.stride())
+    _set(st.delta, delta.stride())
+    if z is not None:
+        _set(st.z, z.stride())
+    _set(st.out, out.stride())
+    _set(st.B, sbc)
+    _set(st.C, _bc_view(C, batch, L)[2])
+    flags = _flags(scalar_a, reverse, zoh)
+    nws = int(_abi.lib().ssm_scan_fwd_strided_workspace_size(batch, dim, L, N, G, code, flags))
+    ws = _workspace(nws, dev, workspace)
+    rc = _abi.lib().ssm_scan_fwd_strided(
+        _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias),
+        int(bool(delta_softplus)), _ptr(h0), _ptr(hL), _ptr(out), None, _ptr(ws),
+        0 if ws is None else ws.numel(), batch, dim, L, N, G, code, flags, ctypes.byref(st),
+        _stream(dev))
+    _abi.check(rc, "ssm_scan_fwd_strided")
+    return (out, hL) if return_final_state else out
+
+
+def ssm_scan_bwd_strided(u, delta, A, B, C, dout, D=None, z=None, dt_bias=None,
+                         delta_softplus=True, h0=None, dhL=None, grads=None, workspace=None,
+                         scalar_a=False, reverse=False, zoh=False):
+    """:func:`ssm_scan_bwd` for io tensors with arbitrary element strides (u, delta, z, dout,
+    B, C as in :func:`ssm_scan_fwd_strided`).  ``grads`` may supply any of du, ddelta, dz, dB,
+    dC as strided output tensors (the others are allocated dense).  Returns the gradient dict."""
+    dev = _on_gpu(u, "u")
+    batch, dim, L = u.shape
+    io = u.dtype
+    code = _io_code(io)
+    G, N, sbc = _bc_view(B, batch, L)
+    xs = (batch, dim, L)
+    bshape = tuple(B.shape)
+    for t, n in ((u, "u"), (delta, "delta"), (dout, "dout")):
+        _view(t, n, xs, io, dev)
+    if z is not None:
+        _view(z, "z", xs, io, dev)
+    _view(B, "B", bshape, io, dev)
+    _view(C, "C", bshape, io, dev)
+    a_shape = (dim,) if scalar_a else (dim, N)
+    _need(A, "A", a_shape, torch.float32, dev)
+    _opt(D, "D", (dim,), torch.float32, dev)
+    _opt(dt_bias, "dt_bias", (dim,), torch.float32, dev)
+    _opt(h0, "h0", (batch, dim, N), torch.float32, dev)
+    _opt(dhL, "dhL", (batch, dim, N), torch.float32, dev)
+    given = dict(grads or {})
+    e = lambda shape, dt: torch.empty(shape, dtype=dt, device=dev)
+    g = {"du": given.get("du", e(xs, io)), "ddelta": given.get("ddelta", e(xs, io)),
+         "dz": given.get("dz", e(xs, io)) if z is not None else None,
+         "dB": given.get("dB", e(bshape, io)), "dC": given.get("dC", e(bshape, io)),
+         "dA": e(a_shape, torch.float32), "dD": e((dim,), torch.float32),
+         "ddt_bias": e((dim,), torch.float32), "dh0": e((batch, dim, N), torch.float32)}
+    for k in ("du", "ddelta", "dz"):
+        if g[k] is not None:
+            _view(g[k], k, xs, io, dev)
+    for k in ("dB", "dC"):
+        _view(g[k], k, bshape, io, dev)
+    st = _abi.Strides()
+    for k, t in (("u", u), ("delta", delta), ("z", z), ("dout", dout), ("du", g["du"]),
+                 ("ddelta", g["ddelta"]), ("dz", g["dz"])):
+        if t is not None:
+            _set(getattr(st, k), t.stride())
+    for k, t in (("B", B), ("C", C), ("dB", g["dB"]), ("dC", g["dC"])):
+        _set(getattr(st, k), _bc_view(t, batch, L)[2])
+    flags = _flags(scalar_a, reverse, zoh)
+    nws = int(_abi.lib().ssm_scan_bwd_strided_workspace_size(batch, dim, L, N, G, code, 0, flags))
+    ws = _workspace(nws, dev, workspace)
+    rc = _abi.lib().ssm_scan_bwd_strided(
+        _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias),
+        int(bool(delta_softplus)), _ptr(h0), _ptr(dout), _ptr(dhL), None,
+        _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]),
+        _ptr(g["dD"]), _ptr(g["dz"]), _ptr(g["ddt_bias"]), _ptr(g["dh0"]),
+        _ptr(ws), 0 if ws is None else ws.numel(), batch, dim, L, N, G, code, flags,
+        ctypes.byref(st), _stream(dev))
+    _abi.check(rc, "ssm_scan_bwd_strided")
+    return g
+
+
+def ssm_state_update_strided(state, x, dt, A, B, C, D=None, z=None, dt_bias=None,
+                             delta_softplus=True, out=None, scalar_a=False, zoh=False,
+                             workspace=None):
+    """:func:`ssm_state_update` for tensors with arbitrary element strides: state [batch, dim,
+    N] f32 (updated in place), x, dt, z, out [batch, dim], B, C [batch, N] or [batch, G, N]."""
+    dev = _on_gpu(state, "state")
+    batch, dim, N = state.shape
+    io = x.dtype
+    code = _io_code(io)
+    if not isinstance(B, torch.Tensor):
+        raise TypeError("B must be a torch.Tensor")
+    G = B.shape[1] if B.dim() == 3 else 1
+    bshape = tuple(B.shape)
+    sbc = lambda t: tuple(t.stride()) if t.dim() == 3 else (t.stride(0), 0, t.stride(1))
+    _view(state, "state", (batch, dim, N), torch.float32, dev)
+    for t, n in ((x, "x"), (dt, "dt")):
+        _view(t, n, (batch, dim), io, dev)
+    if z is not None:
+        _view(z, "z", (batch, dim), io, dev)
+    _view(B, "B", bshape, io, dev)
+    _view(C, "C", bshape, io, dev)
+    _need(A, "A", (dim,) if scalar_a else (dim, N), torch.float32, dev)
+    _opt(D, "D", (dim,), torch.float32, dev)
+    _opt(dt_bias, "dt_bias", (dim,), torch.float32, dev)
+    if out is None:
+        out = torch.empty((batch, dim), dtype=io, device=dev)
+    _view(out, "out", (batch, dim), io, dev)
+    st = _abi.DecodeStrides()
+    _set(st.state, state.stride())
+    _set(st.x, x.stride())
+    _set(st.dt, dt.stride())
+    if z is not None:
+        _set(st.z, z.stride())
+    _set(st.out, out.stride())
+    _set(st.B, sbc(B))
+    _set(st.C, sbc(C))
+    nws = int(_abi.lib().ssm_state_update_strided_workspace_size(batch, dim, N, G, code))
+    ws = _workspace(nws, dev, workspace)
+    rc = _abi.lib().ssm_state_update_strided(
+        _ptr(state), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+        _ptr(dt_bias), int(bool(delta_softplus)), _ptr(out), _ptr(ws),
+        0 if ws is None else ws.numel(), batch, dim, N, G, code, _flags(scalar_a, False, zoh),
+        ctypes.byref(st), _stream(dev))
+    _abi.check(rc, "ssm_state_update_strided")
     return out

@@ -18,6 +18,21 @@ SSM_SCALAR_A, SSM_REVERSE, SSM_ZOH, SSM_CHANNELS_LAST = 1, 2, 4, 8
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
 _sz = ctypes.c_size_t
+_ll3 = ctypes.c_longlong * 3
+_ll4 = ctypes.c_longlong * 4
+_ll2 = ctypes.c_longlong * 2
+
+
+class Strides(ctypes.Structure):
+    """ssm_strides: element strides of every io tensor of a strided scan call."""
+    _fields_ = [(n, _ll3) for n in ("u", "delta", "z", "out", "dout", "du", "ddelta", "dz")] + \
+               [(n, _ll4) for n in ("B", "C", "dB", "dC")]
+
+
+class DecodeStrides(ctypes.Structure):
+    """ssm_decode_strides: element strides of the tensors of a strided decode step."""
+    _fields_ = [("state", _ll3)] + [(n, _ll2) for n in ("x", "dt", "z", "out")] + \
+               [(n, _ll3) for n in ("B", "C")]
 
 # name -> (restype, argtypes)
 SIGNATURES = {
@@ -55,6 +70,18 @@ SIGNATURES = {
     "ssm_state_update_ex": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp,
                                  _i, _i, _i, _i, _i, _i, _vp]),
     "ssm_wait_timeouts": (_i, [ctypes.POINTER(ctypes.c_uint)]),
+    "ssm_scan_fwd_strided_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "ssm_scan_fwd_strided": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp,
+                                  _vp, _sz, _i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(Strides),
+                                  _vp]),
+    "ssm_scan_bwd_strided_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i]),
+    "ssm_scan_bwd_strided": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp,
+                                  _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                                  _i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(Strides), _vp]),
+    "ssm_state_update_strided_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
+    "ssm_state_update_strided": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp,
+                                      _sz, _i, _i, _i, _i, _i, _i,
+                                      ctypes.POINTER(DecodeStrides), _vp]),
 }
 
 _lib = None

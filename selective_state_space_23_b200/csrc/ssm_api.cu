@@ -236,11 +236,35 @@ int fwd_kmufu(long long warps) {
 int fwd_wide(long long warps) { return env_int("SSM_FWD_WIDE", warps < 8LL * sm_count() ? 1 : 0); }
 
 struct BwdLayout {
-  size_t ckpt, part_bc, part_adt, total;
+  size_t ckpt, part_bc, part_adt, split, fwd_ws, total;
   int wpb, ngroups;
+  int nsplit;  // the most time chunks the history backward may take for this shape
 };
 
-BwdLayout layout_bwd(int batch, int dim, int seqlen, int dstate, bool have_ckpt, int bc_groups) {
+// Time split of the register-history backward: when its CTAs (batch rows x channel groups) fill
+// less than one wave, time is cut into chunks of whole 16-step blocks so that about one wave of
+// CTAs runs (SSM_BWD_SPLIT overrides).  Returns the number of chunks (1: none); *bpc = blocks
+// per chunk.
+int plan_bwd_split(int batch, int dim, int seqlen, int wpb, int ctas_per_sm, int* bpc) {
+  const int nblk = (seqlen + ssm::kBlk - 1) / ssm::kBlk;
+  const long long ctas = (long long)batch * (((dim + 15) / 16 + wpb - 1) / wpb);
+  const long long slots = (long long)sm_count() * ctas_per_sm;
+  long long S = env_int("SSM_BWD_SPLIT", 0);
+  if (S <= 0) S = ctas >= slots ? 1 : (slots + ctas - 1) / ctas;
+  S = S < 1 ? 1 : (S > nblk ? nblk : S);
+  *bpc = (int)((nblk + S - 1) / S);
+  return (nblk + *bpc - 1) / *bpc;
+}
+
+// Whether the history backward (and so its time split) can serve this request, judged from the
+// shape and flags alone (the pointers' alignment is checked at the call).
+bool bwd_hist_shape(int dim, int seqlen, int dstate, int bc_groups, int flags) {
+  return !(flags & (SSM_REVERSE | SSM_ZOH | SSM_CHANNELS_LAST)) && dstate == ssm::kNS &&
+         seqlen % 8 == 0 && !(bc_groups == dim && bc_groups > 1);
+}
+
+BwdLayout layout_bwd(int batch, int dim, int seqlen, int dstate, bool have_ckpt, int bc_groups,
+                     int io_dtype, int flags) {
   BwdLayout l;
   // one warp per CTA: CTAs of several warps synchronise once per block for the dB/dC partials,
   // which measured slower on B200 than writing one partial per warp (and with grouped B/C every
@@ -253,8 +277,19 @@ BwdLayout layout_bwd(int batch, int dim, int seqlen, int dstate, bool have_ckpt,
   const size_t nblk = (seqlen + ssm::kBlk - 1) / ssm::kBlk;
   l.ckpt = have_ckpt ? 0 : align_up(nch * nblk * dstate * 4);
   l.part_bc = align_up((size_t)l.ngroups * batch * 2 * ssm::kNS * seqlen * 4);
-  l.part_adt = align_up(nch * (ssm::kNS + 2) * 4);
-  l.total = l.ckpt + l.part_bc + l.part_adt;
+  // 4 warps per CTA give the fewest CTAs, hence the most chunks
+  int bpc = 0;
+  l.nsplit = bwd_hist_shape(dim, seqlen, dstate, bc_groups, flags)
+                 ? plan_bwd_split(batch, dim, seqlen, 4, ssm::bwd_hist_ctas_per_sm(io_dtype, 4), &bpc)
+                 : 1;
+  l.part_adt = align_up((size_t)l.nsplit * nch * (ssm::kNS + 2) * 4);
+  // chunk summaries and entering adjoints [nsplit][nch][16], chunk ΣΔ [nsplit][nch]
+  l.split = l.nsplit > 1 ? 2 * align_up((size_t)l.nsplit * nch * ssm::kNS * 4) +
+                               align_up((size_t)l.nsplit * nch * 4)
+                         : 0;
+  // the replay pass without checkpoints takes the forward's own time split
+  l.fwd_ws = have_ckpt ? 0 : fwd_ws_bytes(batch, dim, seqlen);
+  l.total = l.ckpt + l.part_bc + l.part_adt + l.split + l.fwd_ws;
   return l;
 }
 
@@ -264,6 +299,11 @@ namespace ssm {
 // Records a message for ssm_last_error() on the calling thread (used by entry points that live
 // in other translation units).
 void set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+// The pointer validation of the entry points, for entry points in other translation units: the
+// pointer is usable by kernels on the current device and its allocation holds `bytes` bytes.
+int check_device_ptr(const void* p, size_t bytes, size_t align, const char* name) {
+  return check_ptr(p, bytes, align, name);
+}
 }  // namespace ssm
 
 extern "C" {
@@ -497,7 +537,7 @@ int ssm_scan_fwd_scalar_a(const void* u, const void* delta, const float* A, cons
 size_t ssm_scan_bwd_workspace_size(int batch, int dim, int seqlen, int dstate, int io_dtype,
                                    int have_ckpt) {
   if (check_dims(batch, dim, seqlen, dstate, io_dtype) != SSM_OK) return 0;
-  return layout_bwd(batch, dim, seqlen, dstate, have_ckpt != 0, 1).total;
+  return layout_bwd(batch, dim, seqlen, dstate, have_ckpt != 0, 1, io_dtype, 0).total;
 }
 
 }  // extern "C"
@@ -544,7 +584,10 @@ int scan_bwd_core(const void* u, const void* delta, const float* A, const void* 
     return fail(SSM_EINVAL, "no gradient output requested");
   if (dz && !z) return fail(SSM_EINVAL, "dz requested but z is NULL");
 
-  const BwdLayout l = layout_bwd(batch, dim, seqlen, dstate, ckpt != nullptr, bc_groups);
+  const int lflags = (reverse ? SSM_REVERSE : 0) | (zoh ? SSM_ZOH : 0) |
+                     (channels_last ? SSM_CHANNELS_LAST : 0);
+  const BwdLayout l = layout_bwd(batch, dim, seqlen, dstate, ckpt != nullptr, bc_groups,
+                                 io_dtype, lflags);
   if (!workspace || workspace_bytes < l.total)
     return fail(SSM_EWORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes, l.total);
   if (reinterpret_cast<uintptr_t>(workspace) & 255)
@@ -555,6 +598,9 @@ int scan_bwd_core(const void* u, const void* delta, const float* A, const void* 
   float* ck_ws = reinterpret_cast<float*>(w);
   float* part_bc = reinterpret_cast<float*>(w + l.ckpt);
   float* part_adt = reinterpret_cast<float*>(w + l.ckpt + l.part_bc);
+  char* split_ws = w + l.ckpt + l.part_bc + l.part_adt;
+  char* fwd_ws = split_ws + l.split;
+  const size_t nch = (size_t)batch * dim;
   const bool vec = !channels_last && (seqlen * es) % 16 == 0 && aligned16(u) &&
                    aligned16(delta) && aligned16(z) && aligned16(dout) && aligned16(du) &&
                    aligned16(ddelta) && aligned16(dz) && aligned16(B) && aligned16(C);
@@ -599,8 +645,31 @@ int scan_bwd_core(const void* u, const void* delta, const float* A, const void* 
     a.warps_per_b = (dim + fwd_chw(lane) - 1) / fwd_chw(lane);
     if (!lane) a.warps_per_b = (dim + 32 / a.lpc - 1) / (32 / a.lpc);
     a.nwarps = (long long)batch * a.warps_per_b;
-    e = lane ? ssm::launch_fwd_lane(a, io_dtype, ssm::kFwdCkpt, fwd_kmufu(a.nwarps), s)
-             : ssm::launch_fwd(a, io_dtype, vec, ssm::kFwdCkpt, fwd_wpb(), fwd_kmufu(a.nwarps), s);
+    // with few channels the replay takes the forward's time split (summary, carry, replay)
+    FwdPlan plan = plan_fwd(batch, dim, seqlen, fwd_chw(lane));
+    if (plan.nchunk > 1 && plan.ws_bytes > l.fwd_ws) {
+      plan.nchunk = 1;
+      plan.chunk_len = (int)nblk * ssm::kBlk;
+    }
+    a.chunk_len = plan.chunk_len;
+    a.nchunk = plan.nchunk;
+    const int km = fwd_kmufu(a.nwarps * (long long)plan.nchunk);
+    if (plan.nchunk > 1) {
+      float* summ = reinterpret_cast<float*>(fwd_ws);
+      float* hin = reinterpret_cast<float*>(fwd_ws + align_up(plan.nchunk * nch * ssm::kNS * 4));
+      float* dsum = reinterpret_cast<float*>(fwd_ws + 2 * align_up(plan.nchunk * nch * ssm::kNS * 4));
+      ssm::FwdArgs as = a;
+      as.summ = summ; as.dsum = dsum;
+      as.ckpt = nullptr; as.h0 = nullptr;
+      e = lane ? ssm::launch_fwd_lane(as, io_dtype, ssm::kFwdSummary, km, s)
+               : ssm::launch_fwd(as, io_dtype, vec, ssm::kFwdSummary, fwd_wpb(), km, s);
+      if (e != cudaSuccess) return cuda_fail(e, "backward replay summary pass");
+      if ((e = ssm::launch_fwd_carry(a, summ, dsum, hin, s)) != cudaSuccess)
+        return cuda_fail(e, "backward replay carry pass");
+      a.hin = hin;
+    }
+    e = lane ? ssm::launch_fwd_lane(a, io_dtype, ssm::kFwdCkpt, km, s)
+             : ssm::launch_fwd(a, io_dtype, vec, ssm::kFwdCkpt, fwd_wpb(), km, s);
     if (e != cudaSuccess) return cuda_fail(e, "backward state replay pass");
     ck = ck_ws;
   }
@@ -642,6 +711,32 @@ int scan_bwd_core(const void* u, const void* delta, const float* A, const void* 
     if (hist) {
       b.wpb = w;
       b.ngroups = (b.warps_per_b + w - 1) / w;
+      // time split when the CTAs fill less than a wave: adjoint summaries of chunks 1 .. S-1,
+      // chained from dhL by the carry pass, give each chunk the adjoint entering it
+      int bpc = 0;
+      int S = plan_bwd_split(batch, dim, seqlen, w, ssm::bwd_hist_ctas_per_sm(io_dtype, w), &bpc);
+      if (S > l.nsplit) {
+        bpc = (int)((nblk + l.nsplit - 1) / l.nsplit);
+        S = (int)((nblk + bpc - 1) / bpc);
+      }
+      if (S > 1) {
+        b.nsplit = S;
+        b.blk_per_chunk = bpc;
+        const size_t sz = align_up((size_t)l.nsplit * nch * ssm::kNS * 4);
+        float* summ = reinterpret_cast<float*>(split_ws);
+        float* lam_in = reinterpret_cast<float*>(split_ws + sz);
+        float* dsum = reinterpret_cast<float*>(split_ws + 2 * sz);
+        if ((e = ssm::launch_bwd_summary(b, io_dtype, summ, dsum, s)) != cudaSuccess)
+          return cuda_fail(e, "backward summary pass");
+        ssm::FwdArgs c;
+        memset(&c, 0, sizeof(c));
+        c.A = A; c.h0 = dhL;
+        c.batch = batch; c.dim = dim; c.N = dstate;
+        c.nchunk = S;
+        if ((e = ssm::launch_fwd_carry(c, summ, dsum, lam_in, s)) != cudaSuccess)
+          return cuda_fail(e, "backward carry pass");
+        b.lam_in = lam_in;
+      }
     }
   }
   e = hist ? ssm::launch_bwd_hist(b, io_dtype, s) : ssm::launch_bwd(b, io_dtype, vec, s);
@@ -672,7 +767,8 @@ size_t ssm_scan_bwd_ex_workspace_size(int batch, int dim, int seqlen, int dstate
   if (flags & ~(SSM_SCALAR_A | SSM_REVERSE | SSM_ZOH | SSM_CHANNELS_LAST)) return 0;
   if (check_dims(batch, dim, seqlen, dstate, io_dtype) != SSM_OK) return 0;
   if (check_groups(dim, bc_groups) != SSM_OK) return 0;
-  const size_t base = layout_bwd(batch, dim, seqlen, dstate, have_ckpt != 0, bc_groups).total;
+  const size_t base = layout_bwd(batch, dim, seqlen, dstate, have_ckpt != 0, bc_groups, io_dtype,
+                                 flags & ~SSM_SCALAR_A).total;
   if (base == 0 || !(flags & SSM_SCALAR_A)) return base;
   return align_up((size_t)dim * dstate * 4) * 2 + base;
 }

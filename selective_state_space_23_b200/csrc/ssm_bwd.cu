@@ -635,7 +635,10 @@ __global__ void bwd_finish_adt(const BwdArgs a, float* dA, float* dD, float* ddt
   const int d = (int)(i / (kNS + 2)), j = (int)(i % (kNS + 2));
   if (j < kNS && j >= a.N) return;
   float s = 0.f;
-  for (int b = 0; b < a.batch; ++b) s += a.part_adt[((long long)b * a.dim + d) * (kNS + 2) + j];
+  const int nsplit = a.nsplit > 1 ? a.nsplit : 1;  // chunks of a time-split backward
+  for (int c = 0; c < nsplit; ++c)
+    for (int b = 0; b < a.batch; ++b)
+      s += a.part_adt[(((long long)c * a.batch + b) * a.dim + d) * (kNS + 2) + j];
   if (j < kNS) { if (dA) dA[(long long)d * a.N + j] = s; }
   else if (j == kNS) { if (dD) dD[d] = s; }
   else if (ddt_bias) ddt_bias[d] = s;

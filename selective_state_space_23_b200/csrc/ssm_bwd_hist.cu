@@ -341,6 +341,14 @@ __global__ void __launch_bounds__(32 * W) bwd_hist_kernel(const __grid_constant_
   hb.ch = (long long)b * a.dim + dd;
   hb.L = a.L;
   hb.nblk = (a.L + kBlk - 1) / kBlk;
+  // time split: this CTA walks the blocks of chunk blockIdx.y only
+  const int chunk = blockIdx.y;
+  const bool split = a.nsplit > 1;
+  const int blk_lo = split ? chunk * a.blk_per_chunk : 0;
+  const int blk_hi = split ? min(hb.nblk, blk_lo + a.blk_per_chunk) : hb.nblk;
+  const long long nch = (long long)a.batch * a.dim;
+  // the adjoint entering the chunk from later time (dhL for the last chunk, or none)
+  const float* lam0 = split ? a.lam_in + (long long)(a.nsplit - 1 - chunk) * nch * kNS : a.dhL;
   hb.qlo = 8 * hb.q + 4 * hb.rot;
   hb.qhi = 8 * hb.q + 4 * (1 - hb.rot);
   const float live = hb.act ? 1.f : 0.f;  // idle lanes add nothing to the channel sums
@@ -354,8 +362,8 @@ __global__ void __launch_bounds__(32 * W) bwd_hist_kernel(const __grid_constant_
   for (int jj = 0; jj < 4; ++jj) {
     const int n0 = 8 * q + ((2 * jj + 4 * rot) & 7);
     al[jj] = make_float2(a.A[(long long)dd * kNS + n0] * ascale, a.A[(long long)dd * kNS + n0 + 1] * ascale);
-    lam[jj] = a.dhL ? make_float2(a.dhL[hb.ch * kNS + n0], a.dhL[hb.ch * kNS + n0 + 1])
-                    : make_float2(0.f, 0.f);
+    lam[jj] = lam0 ? make_float2(lam0[hb.ch * kNS + n0], lam0[hb.ch * kNS + n0 + 1])
+                   : make_float2(0.f, 0.f);
     dA[jj] = make_float2(0.f, 0.f);
     amax = fmaxf(amax, fmaxf(fabsf(al[jj].x), fabsf(al[jj].y)));
   }
@@ -364,10 +372,10 @@ __global__ void __launch_bounds__(32 * W) bwd_hist_kernel(const __grid_constant_
   float dD_acc = 0.f, db_acc = 0.f;
   const float* redw0 = reinterpret_cast<const float*>(reinterpret_cast<unsigned char*>(smem_bh));
 
-  hb.issue(hb.nblk - 1);
-  for (int blk = hb.nblk - 1; blk >= 0; --blk) {
+  hb.issue(blk_hi - 1);
+  for (int blk = blk_hi - 1; blk >= blk_lo; --blk) {
     hb.blkcur = blk;
-    hb.issue(blk - 1);   // the next (earlier) block's copies run while this one computes
+    hb.issue(blk > blk_lo ? blk - 1 : -1);  // the next (earlier) block's copies run meanwhile
     cp_wait_all_but1();  // this block's copies have landed
     __syncwarp();
     hb.convert_bc(blk);
@@ -474,11 +482,11 @@ __global__ void __launch_bounds__(32 * W) bwd_hist_kernel(const __grid_constant_
   dD_acc += __shfl_xor_sync(0xffffffffu, dD_acc, 1);
   db_acc += __shfl_xor_sync(0xffffffffu, db_acc, 1);
   if (!hb.act) return;
-  float* pa = a.part_adt + hb.ch * (kNS + 2);
+  float* pa = a.part_adt + ((long long)(split ? chunk : 0) * nch + hb.ch) * (kNS + 2);
 #pragma unroll
   for (int jj = 0; jj < 4; ++jj) {
     const int n0 = 8 * q + ((2 * jj + 4 * rot) & 7);
-    if (a.dh0) {
+    if (a.dh0 && chunk == 0) {
       a.dh0[hb.ch * kNS + n0] = lam[jj].x;
       a.dh0[hb.ch * kNS + n0 + 1] = lam[jj].y;
     }
@@ -491,9 +499,99 @@ __global__ void __launch_bounds__(32 * W) bwd_hist_kernel(const __grid_constant_
   }
 }
 
+// 8 consecutive steps of a row from global memory (16-byte aligned).
+template <typename IO>
+__device__ __forceinline__ void load8(const IO* p, float (&v)[8]) {
+  if constexpr (sizeof(IO) == 2) {
+    const uint4 q = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = bf16_lo(w[i]);
+      v[2 * i + 1] = bf16_hi(w[i]);
+    }
+  } else {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+}
+
+// Adjoint summary of chunk c >= 1 of a time-split backward.  The adjoint recurrence is linear in
+// what enters a chunk from later time: if μ_in enters at the chunk's end, the adjoint leaving its
+// first step is exp(A ΣΔ) μ_in + m, where m is what leaves when nothing enters.  This kernel walks
+// the chunk backwards from zero (λ <- g_t C_t + λ, then λ <- Ā_t λ, as the history backward does)
+// to get m, and sums Δ over the chunk (Kahan-compensated); the forward carry pass then chains the
+// chunks' maps from the last chunk to the first, starting from dhL.  Two threads per channel (8
+// states each); rows are read in 8-step pieces.
+template <typename IO>
+__global__ void __launch_bounds__(128) bwd_summary_kernel(const __grid_constant__ BwdArgs a,
+                                                          float* __restrict__ summ,
+                                                          float* __restrict__ dsum) {
+  constexpr bool kPrecise = std::is_same<IO, float>::value;
+  const long long nch = (long long)a.batch * a.dim;
+  const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long ch = tid >> 1;
+  const int q = (int)(tid & 1);
+  if (ch >= nch) return;
+  const int chunk = blockIdx.y + 1;
+  const long long slot = a.nsplit - 1 - chunk;
+  const int b = (int)(ch / a.dim), d = (int)(ch % a.dim);
+  const int gbc = d / (a.dim / a.bc_groups);
+  const float ascale = kPrecise ? 1.f : kLog2e;
+  float al[8], lam[8];
+#pragma unroll
+  for (int n = 0; n < 8; ++n) {
+    al[n] = a.A[(long long)d * kNS + 8 * q + n] * ascale;
+    lam[n] = 0.f;
+  }
+  const float bias = a.dt_bias ? a.dt_bias[d] : 0.f;
+  const long long L = a.L;
+  const int t_lo = chunk * a.blk_per_chunk * kBlk;
+  const int t_hi = min(a.L, t_lo + a.blk_per_chunk * kBlk);  // L % 8 == 0: whole 8-step pieces
+  const IO* dp = reinterpret_cast<const IO*>(a.delta) + ch * L;
+  const IO* zp = a.z ? reinterpret_cast<const IO*>(a.z) + ch * L : nullptr;
+  const IO* gp = reinterpret_cast<const IO*>(a.dout) + ch * L;
+  const IO* cp = reinterpret_cast<const IO*>(a.C) + (((long long)b * a.bc_groups + gbc) * kNS + 8 * q) * L;
+  float dsm = 0.f, dcomp = 0.f;
+  for (int t0 = t_hi - 8; t0 >= t_lo; t0 -= 8) {
+    float dv[8], zv[8], gv[8], cv[8][8];
+    load8<IO>(dp + t0, dv);
+    if (zp) load8<IO>(zp + t0, zv);
+    load8<IO>(gp + t0, gv);
+#pragma unroll
+    for (int n = 0; n < 8; ++n) load8<IO>(cp + n * L + t0, cv[n]);
+#pragma unroll
+    for (int j = 7; j >= 0; --j) {
+      const float v = dv[j] + bias;
+      const float dl = !a.softplus ? v : (kPrecise ? softplus_precise(v) : softplus_fast(v));
+      float g = gv[j];
+      if (zp) {
+        const float sg = kPrecise ? sigmoid_precise(zv[j]) : sigmoid_fast(zv[j]);
+        g = g * (zv[j] * sg);
+      }
+      const float yk = dl - dcomp;  // Kahan step
+      const float tk = dsm + yk;
+      dcomp = (tk - dsm) - yk;
+      dsm = tk;
+#pragma unroll
+      for (int n = 0; n < 8; ++n) {
+        lam[n] = fmaf(g, cv[n][j], lam[n]);
+        lam[n] *= kPrecise ? expf(dl * al[n]) : ex2_mufu(dl * al[n]);
+      }
+    }
+  }
+  float* o = summ + (slot * nch + ch) * kNS + 8 * q;
+#pragma unroll
+  for (int n = 0; n < 8; ++n) o[n] = lam[n];
+  if (q == 0) dsum[slot * nch + ch] = dsm;
+}
+
 template <typename IO, int W>
 cudaError_t launch_hist_io(const BwdArgs& a, cudaStream_t s) {
-  const dim3 grid((unsigned)(a.batch * a.ngroups)), block(32 * W);
+  const dim3 grid((unsigned)(a.batch * a.ngroups), (unsigned)(a.nsplit > 1 ? a.nsplit : 1)),
+      block(32 * W);
   const size_t smem = (size_t)W * HGeo<IO>::kWarpBytes;
   auto k = bwd_hist_kernel<IO, W, 4>;
   if constexpr (!std::is_same<IO, float>::value) {
@@ -539,6 +637,34 @@ int pick_wpb_io(int batch, int dim) {
 
 int bwd_hist_pick_wpb(int io, int batch, int dim) {
   return io == 1 ? pick_wpb_io<uint16_t>(batch, dim) : pick_wpb_io<float>(batch, dim);
+}
+
+namespace {
+template <typename IO>
+int ctas_per_sm_io(int wpb) {
+  int occ = 0;
+  const size_t smem = (size_t)wpb * HGeo<IO>::kWarpBytes;
+  auto k = wpb == 2 ? bwd_hist_kernel<IO, 2, 4> : bwd_hist_kernel<IO, 4, 4>;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, 32 * wpb, smem) != cudaSuccess) {
+    cudaGetLastError();
+    return 1;
+  }
+  return occ < 1 ? 1 : occ;
+}
+}  // namespace
+
+int bwd_hist_ctas_per_sm(int io, int wpb) {
+  return io == 1 ? ctas_per_sm_io<uint16_t>(wpb) : ctas_per_sm_io<float>(wpb);
+}
+
+cudaError_t launch_bwd_summary(const BwdArgs& a, int io, float* summ, float* dsum, cudaStream_t s) {
+  if (a.nsplit <= 1) return cudaSuccess;
+  const long long threads = 2LL * a.batch * a.dim;
+  const dim3 grid((unsigned)((threads + 127) / 128), (unsigned)(a.nsplit - 1)), block(128);
+  if (io == 1) bwd_summary_kernel<uint16_t><<<grid, block, 0, s>>>(a, summ, dsum);
+  else bwd_summary_kernel<float><<<grid, block, 0, s>>>(a, summ, dsum);
+  return cudaGetLastError();
 }
 
 }  // namespace ssm

@@ -72,7 +72,7 @@ struct BwdArgs {
   void* dz;
   float* dh0;
   float* part_bc;       // [ngroups][batch][2][16][L] per-CTA partial sums of dB, dC
-  float* part_adt;      // [batch][dim][16 + 2] per-channel partial dA, dD, ddt_bias
+  float* part_adt;      // [nsplit][batch][dim][16 + 2] per-channel (and chunk) partial dA, dD, ddt_bias
   int batch, dim, L, N;
   int softplus;
   int warps_per_b;
@@ -84,6 +84,12 @@ struct BwdArgs {
   int zoh;              // gradients of the zero-order-hold input term
   int bc_groups;        // B, C (and dB, dC) are [batch][bc_groups][N][L]
   int channels_last;    // time rows strided: [batch][L][dim] and [batch][L][bc_groups][N]
+  // time split of the register-history backward (nsplit <= 1: none): chunk c covers blocks
+  // [c blk_per_chunk, (c + 1) blk_per_chunk); lam_in [nsplit][batch][dim][16] holds the adjoint
+  // entering each chunk from later time, in reverse chunk order (slot nsplit-1-c)
+  int nsplit;
+  int blk_per_chunk;
+  const float* lam_in;
 };
 
 struct DecodeArgs {
@@ -122,8 +128,17 @@ cudaError_t launch_bwd(const BwdArgs& a, int io, bool vec, cudaStream_t s);
 // N = 16, forward direction, no ZOH, [batch][dim][L] rows with L % 8 == 0 and 16-byte aligned
 // tensors and checkpoints; a.wpb = 2 or 4 warps per CTA (bwd_hist_pick_wpb), a.ngroups =
 // ceil(ceil(dim / 16) / a.wpb), each CTA inside one B/C group.
+// With a.nsplit > 1 the CTAs of chunk c (grid.y) start from the adjoint in a.lam_in and write
+// chunk c's part of part_adt; only chunk 0 writes dh0.
 cudaError_t launch_bwd_hist(const BwdArgs& a, int io, cudaStream_t s);
 int bwd_hist_pick_wpb(int io, int batch, int dim);
+// The adjoint summaries of chunks 1 .. nsplit-1 for the time-split history backward: for chunk c,
+// the adjoint leaving its first step when none enters at its end (summ [slot][batch][dim][16])
+// and its ΣΔ (dsum [slot][batch][dim]), stored at slot nsplit-1-c so that the forward carry pass
+// (launch_fwd_carry, with dhL in place of h0) chains them from the last chunk to the first.
+cudaError_t launch_bwd_summary(const BwdArgs& a, int io, float* summ, float* dsum, cudaStream_t s);
+// Number of CTAs of the history backward that one SM holds at once for this shape.
+int bwd_hist_ctas_per_sm(int io, int wpb);
 // B/C per channel (bc_groups == dim, ssm_pcbc.cu): forward (mode kFwdOut or kFwdCkpt) and
 // backward (writes du, ddelta, dz, dB, dC, dh0 and the per-channel dA/dD/ddt_bias partials).
 cudaError_t launch_fwd_pcbc(const FwdArgs& a, int io, bool vec, int mode, cudaStream_t s);
@@ -140,5 +155,8 @@ int decode_wait_timeouts(unsigned int* out);
 
 // Sets the message returned by ssm_last_error() on the calling thread.
 void set_last_error(const char* msg);
+// The entry points' pointer check (device-accessible on the current device, allocation holds
+// `bytes` bytes, `align`-byte aligned); returns an ssm_status and sets the error message.
+int check_device_ptr(const void* p, size_t bytes, size_t align, const char* name);
 
 }  // namespace ssm

@@ -182,3 +182,26 @@ def test_binding_rejects_host_tensors_before_any_cuda_call():
 def test_wait_timeout_query_rejects_null(lib):
     assert lib.ssm_wait_timeouts(None) == _abi.SSM_EINVAL
     assert b"NULL" in lib.ssm_last_error()
+
+
+def test_strided_entry_points_check_on_the_host(lib):
+    """The strided forms refuse a missing stride table, the channels-last flag (a layout the
+    strides already express) and a missing workspace before any pointer is touched."""
+    st = _abi.Strides()
+    assert lib.ssm_scan_fwd_strided_workspace_size(2, 64, 256, 16, 1, 1, 0) > 0
+    assert lib.ssm_scan_fwd_strided_workspace_size(2, 64, 256, 16, 1, 1,
+                                                   _abi.SSM_CHANNELS_LAST) == 0
+    assert lib.ssm_scan_bwd_strided_workspace_size(2, 64, 256, 16, 1, 1, 0, 0) > 0
+    assert lib.ssm_state_update_strided_workspace_size(2, 64, 16, 1, 1) > 0
+    args = [None] * 8 + [1] + [None] * 5 + [0, 2, 64, 256, 16, 1, 1]
+    assert lib.ssm_scan_fwd_strided(*args, 0, None, None) == _abi.SSM_EINVAL   # strides NULL
+    assert lib.ssm_scan_fwd_strided(*args, _abi.SSM_CHANNELS_LAST, ctypes.byref(st),
+                                    None) == _abi.SSM_EINVAL
+    assert lib.ssm_scan_fwd_strided(*args, 0, ctypes.byref(st), None) == _abi.SSM_EWORKSPACE
+    bargs = [None] * 8 + [1] + [None] * 14 + [0, 2, 64, 256, 16, 1, 1, 0]
+    assert lib.ssm_scan_bwd_strided(*bargs, None, None) == _abi.SSM_EINVAL
+    dst = _abi.DecodeStrides()
+    dargs = [None] * 9 + [1, None, None, 0, 2, 64, 16, 1, 1]
+    assert lib.ssm_state_update_strided(*dargs, _abi.SSM_REVERSE, ctypes.byref(dst),
+                                        None) == _abi.SSM_EINVAL
+    assert lib.ssm_state_update_strided(*dargs, 0, ctypes.byref(dst), None) == _abi.SSM_EWORKSPACE

@@ -176,6 +176,8 @@ BWD_CASES = {
     "history_w4": ({"SSM_BWD_WPB": "4"}, 2, 96, 312, 16, torch.bfloat16, 1, 0),
     "history_w2": ({"SSM_BWD_WPB": "2"}, 2, 72 + 8, 312, 16, torch.bfloat16, 1, 0),
     "history_f32": ({}, 2, 96, 200, 16, torch.float32, 1, 0),
+    "history_split3": ({"SSM_BWD_SPLIT": "3"}, 2, 96, 312, 16, torch.bfloat16, 1, 0),
+    "history_split7_f32": ({"SSM_BWD_SPLIT": "7"}, 1, 80, 200, 16, torch.float32, 1, 0),
     "general": ({"SSM_BWD_KERNEL": "pair"}, 2, 96, 312, 16, torch.bfloat16, 1, 0),
     "general_wpb2": ({"SSM_BWD_KERNEL": "pair", "SSM_BWD_WPB": "2"}, 2, 80, 250, 16,
                      torch.bfloat16, 1, 0),
@@ -190,7 +192,7 @@ BWD_CASES = {
 @pytest.mark.parametrize("case", sorted(BWD_CASES))
 def test_backward_stays_inside_its_tensors(monkeypatch, case):
     env, batch, dim, L, N, io, G, flags = BWD_CASES[case]
-    for k in ("SSM_FWD_KERNEL", "SSM_BWD_KERNEL", "SSM_BWD_WPB"):
+    for k in ("SSM_FWD_KERNEL", "SSM_BWD_KERNEL", "SSM_BWD_WPB", "SSM_BWD_SPLIT"):
         monkeypatch.delenv(k, raising=False)
     for k, v in env.items():
         monkeypatch.setenv(k, v)
