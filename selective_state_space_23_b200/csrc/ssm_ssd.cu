@@ -4,25 +4,42 @@
 // With one decay rate A_d per channel (the Mamba-2 restriction noted on the "2024 Reading List:
 // Neural Network" page, section on state-space models, where the scalar transition is what lets
 // the state grow to N = 64..128), the scan h_t = e^{Δ_t A_d} h_{t-1} + Δ_t x_t B_t,
-// y_t = C_t . h_t + D_d x_t, out_t = y_t silu(z_t) has, over a chunk of T steps with cumulative
-// steps S_t = Σ_{r <= t} Δ_r (from the chunk start) and state h_in entering the chunk,
+// y_t = C_t . h_t + D_d x_t, out_t = y_t silu(z_t) has, over a chunk of T = 16 steps with
+// cumulative steps S_t = Σ_{r <= t} Δ_r (from the chunk start) and state h_in entering it,
 //   y_t   = Σ_{s <= t} (C_t . B_s) e^{A (S_t - S_s)} Δ_s x_s  +  e^{A S_t} (C_t . h_in)  +  D x_t
 //   h_out = e^{A S_{T-1}} h_in + Σ_s e^{A (S_{T-1} - S_s)} Δ_s x_s B_s,
 // the masked-matrix ("state-space duality") form of the scan, whose products over states and
 // steps are dense contractions.  Because A is a scalar per channel, the decay factor is rank one
-// in (t, s) for every channel: e^{A (S_t - S_s)} = P_t Q_s with P_t = e^{A (S_t - S_m)},
-// Q_s = 1 / P_s about the chunk's middle step m.  So with B, C shared by the channels of a batch
-// row the chunk is four matrix products over a tile of 64 channels:
-//   G  = C B^T                  [T x T]   (K = N)
-//   Y1 = mask(G) X',  X'[s][d]  = Q_s Δ_s x_s                 [T x 64]  (K = T)
-//   Y2 = C H_in                                                 [T x 64]  (K = N)
-//   U  = B^T X'',  X''[s][d] = e^{A (S_{T-1} - S_s)} Δ_s x_s  [N x 64]  (K = T)
-// and y = P Y1 + e^{A S_t} Y2 + D x,  h_out = e^{A S_{T-1}} h_in + U.  The products run as
-// warp-level bf16 tensor-core MMAs (m16n8k16, f32 accumulation); the state H stays in shared
-// memory in f32 (a bf16 copy feeds Y2).  P_t and Q_s grow as e^{|A| S} inside a chunk: a channel
-// whose chunk would leave the safe range (|A| S_{T-1} > 80, or a non-finite step) is computed for
-// that chunk by an exact sequential pass instead (its columns of the products are ignored).
+// in (t, s) for each channel: e^{A (S_t - S_s)} = P_t Q_s with P_t = e^{A (S_t - S_m)} and
+// Q_s = 1 / P_s about the chunk's middle step m.  With B, C shared by the channels of a batch
+// row, a warp's 16 channels take per chunk four tensor-core products (bf16 in, f32 accumulate):
+//   G   = C B^T                     [16 t x 16 s]   K = N    (masked to s <= t)
+//   Y1' = X1' mask(G)^T              [16 d x 16 t]   K = 16,  X1'[d][s] = Q_s Δ_s x_s
+//   Y2' = H' C^T                     [16 d x 16 t]   K = N,   H' = h_in transposed [d][n]
+//   U'  = X2' B                      [16 d x N]      K = 16,  X2'[d][s] = e^{A (S_end - S_s)} Δ_s x_s
+// and y = P Y1 + e^{A S_t} Y2 + D x,  H' <- e^{A S_end} H' + U'.
+//
+// B200 mapping (one warp = 16 channels, a CTA = W warps of one batch row and B/C group):
+//   * the transposed state H' [16 d][N] lives in the warp's MMA accumulator registers (f32) for
+//     the whole sequence: the U' product accumulates straight into it, and its accumulator
+//     layout is also the A-operand layout of Y2' (packed to bf16), so the state never touches
+//     shared memory;
+//   * G's accumulators are, after the mask, the B operand of Y1' (no shared-memory round trip);
+//   * the chunk's B, C tiles ([N][16 steps], as stored in HBM) stream into a 4-stage
+//     shared-memory ring by cp.async and are read with ldmatrix (.trans where the product needs
+//     them transposed): rows padded to 48 bytes, conflict-free; one CTA barrier per chunk;
+//   * each lane's elementwise work covers exactly the (channel, step) pairs it holds in the
+//     accumulators: channels g, g+8 and steps 2tg, 2tg+1, 2tg+8, 2tg+9 of the chunk
+//     (g = lane / 4, tg = lane % 4); the cumulative steps S_t are a scan over the 4 lanes of a
+//     quad (warp shuffles); u, delta, z are prefetched one chunk ahead into registers;
+//   * P_t and Q_s grow as e^{|A| S} inside a chunk: a channel whose chunk would leave the safe
+//     range (|A| |S_t - S_m| > 60 or |A| |S_t| > 80, or a non-finite step) takes no part in that
+//     chunk's products (its inputs are zeroed, its state kept) and is computed for that chunk by
+//     an exact sequential pass over its states held by the quad instead.
+// The products are small (K = 16 or N per 16-step chunk) and carry the sequence's dependency from
+// chunk to chunk, so they run as warp-level mma.sync.m16n8k16 rather than tcgen05 tiles.
 #include <stdint.h>
+#include <stdlib.h>
 
 #include "ssm_device.cuh"
 #include "ssm_kernels.h"
@@ -30,15 +47,15 @@
 namespace ssm {
 namespace {
 
-constexpr int kT = 16;        // steps per chunk (one MMA k-step)
-constexpr int kDB = 64;       // channels per CTA
-constexpr int kThreads = 128; // 4 warps, 16 channels each in the products
-constexpr int kPadH = 8;      // bf16 row padding of the [*][N] and [*][T] operand tiles
+constexpr int kT = 16;       // steps per chunk (one MMA k-step)
+constexpr int kLdS = 24;     // bf16 per shared tile row: 16 steps + 8 pad (48-byte rows)
+constexpr int kStages = 4;   // B/C ring depth (chunks)
 
-__device__ __forceinline__ uint32_t ld32(const uint16_t* p) {
-  return *reinterpret_cast<const uint32_t*>(p);
-}
-__device__ __forceinline__ uint16_t to_bf16(float x) { return f32_to_bf16(x); }
+template <int N>
+struct SsdStage {
+  uint16_t Bs[N * kLdS];  // B of the chunk as [n][t]
+  uint16_t Cs[N * kLdS];  // C of the chunk as [n][t]
+};
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -49,295 +66,383 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// One 16 x 8 output tile: D += A[16 x K] B[K x 8].  A row-major at a (row stride lda elements);
-// B given as its transpose [8][K] at b (row stride ldb), i.e. the MMA's column-major operand.
-template <int K>
-__device__ __forceinline__ void mma_tile(float (&d)[4], const uint16_t* a, int lda,
-                                         const uint16_t* b, int ldb, int lane) {
-  const int g = lane >> 2, tg = lane & 3;
-#pragma unroll
-  for (int k0 = 0; k0 < K; k0 += 16) {
-    const uint16_t* ar = a + g * lda + k0 + 2 * tg;
-    const uint16_t* br = b + g * ldb + k0 + 2 * tg;
-    mma16816(d, ld32(ar), ld32(ar + 8 * lda), ld32(ar + 8), ld32(ar + 8 * lda + 8), ld32(br),
-             ld32(br + 8));
-  }
+// Four 8x8 bf16 matrices from shared memory; lane i gives the address of row i % 8 of matrix
+// i / 8.  Plain: lane l receives (row l / 4, cols 2 (l % 4), +1) of each; .trans: the transpose.
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
+  const uint32_t a = (uint32_t)__cvta_generic_to_shared(p);
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(a));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* p) {
+  const uint32_t a = (uint32_t)__cvta_generic_to_shared(p);
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(a));
+}
+// The lane's row address for the four 8x8 blocks (rows n0 .. n0+7 | n0+8 .., cols 0..7 | 8..15)
+// of a [n][t] tile: matrix m = lane / 8 covers rows n0 + 8 (m / 2) .., cols 8 (m % 2) ..
+__device__ __forceinline__ const uint16_t* blk(const uint16_t* tile, int n0, int lane) {
+  return tile + (n0 + ((lane >> 4) << 3) + (lane & 7)) * kLdS + (((lane >> 3) & 1) << 3);
 }
 
-template <int N>
-struct SsdSmem {
-  static constexpr int kLdN = N + kPadH;    // [*][N] tiles
-  static constexpr int kLdT = kT + kPadH;   // [*][T] tiles
-  float H[kDB * N];              // state, [d][n], f32
-  uint16_t Hb[kDB * kLdN];       // bf16 copy of H (B operand of Y2: [d][n])
-  uint16_t Ct[kT * kLdN];        // C as [t][n] (A operand of G and Y2)
-  uint16_t Bt[kT * kLdN];        // B as [s][n] (B operand of G)
-  uint16_t Bn[N * kLdT];         // B as [n][s] (A operand of U)
-  uint16_t Gm[kT * kLdT];        // mask(G) as [t][s] (A operand of Y1)
-  uint16_t X1[kDB * kLdT];       // X'  as [d][s]
-  uint16_t X2[kDB * kLdT];       // X'' as [d][s]
-  float P[kDB * kT], E[kDB * kT], Ux[kDB * kT], Gt[kDB * kT], Dl[kDB * kT], Xs[kDB * kT];
-  float Eend[kDB], Dskip[kDB];
-  int fb[kDB];
-  uint16_t Y[kDB * kT];          // gated outputs of the chunk, [d][t]
+__device__ __forceinline__ void cp16(void* smem, const void* gmem) {
+  const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int K>
+__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(K) : "memory"); }
+
+// u, delta, z of the lane's two channels and four steps of one chunk, as bf16 pairs:
+// w[c][0] = steps 2tg, 2tg+1 and w[c][1] = steps 2tg+8, 2tg+9 of channel c.
+struct ChunkIn {
+  uint32_t u[2][2], dl[2][2], z[2][2];
 };
 
-template <int N>
-__global__ void __launch_bounds__(kThreads) ssd_fwd_kernel(const __grid_constant__ FwdArgs a) {
-  using SM = SsdSmem<N>;
+__device__ __forceinline__ uint32_t ld_pair(const uint16_t* p, long long t, int L, bool vec) {
+  if (vec) return __ldg(reinterpret_cast<const uint32_t*>(p + t));
+  const uint32_t lo = t < L ? (uint32_t)__ldg(p + t) : 0u;
+  const uint32_t hi = t + 1 < L ? (uint32_t)__ldg(p + t + 1) : 0u;
+  return lo | (hi << 16);
+}
+
+template <int N, int W>
+__global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__ FwdArgs a) {
+  constexpr int kNT = N / 8;  // n8 tiles of the state
   extern __shared__ float4 smem_ssd[];
-  SM& sm = *reinterpret_cast<SM*>(smem_ssd);
+  SsdStage<N>* ring = reinterpret_cast<SsdStage<N>*>(smem_ssd);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nblk_d = (a.dim + kDB - 1) / kDB;
-  const int b = blockIdx.x / nblk_d;
-  const int d0 = (blockIdx.x % nblk_d) * kDB;
+  const int g = lane >> 2, tg = lane & 3;
+  const int tiles_d = (a.dim + 16 * W - 1) / (16 * W);
+  const int b = blockIdx.x / tiles_d;
+  const int d0 = (blockIdx.x % tiles_d) * 16 * W;
   const int L = a.L;
+  const int nchunk = (L + kT - 1) / kT;
   const int gbc = d0 / (a.dim / a.bc_groups);
   const uint16_t* Bg = reinterpret_cast<const uint16_t*>(a.B) + ((long long)b * a.bc_groups + gbc) * N * (long long)L;
   const uint16_t* Cg = reinterpret_cast<const uint16_t*>(a.C) + ((long long)b * a.bc_groups + gbc) * N * (long long)L;
 
-  // per-channel constants (threads 0..63 own channel d0 + tid in the elementwise phases)
-  const int dl = tid & (kDB - 1);
-  const bool own = tid < kDB;
-  const int d = min(d0 + dl, a.dim - 1);
-  const bool dact = d0 + dl < a.dim;
-  const long long row = ((long long)b * a.dim + d) * L;
-  const float Ad = a.A[d];
-  const float bias = a.dt_bias ? a.dt_bias[d] : 0.f;
-  const float Dd = a.D ? a.D[d] : 0.f;
+  // the lane's two channels (rows g and g + 8 of the warp's 16); idle ones shadow the last
+  int dch[2];
+  bool act[2];
+  long long row[2];
+  float al[2], bias[2], Dd[2];
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    const int d = d0 + 16 * warp + g + 8 * c;
+    act[c] = d < a.dim;
+    dch[c] = act[c] ? d : a.dim - 1;
+    row[c] = ((long long)b * a.dim + dch[c]) * L;
+    al[c] = a.A[dch[c]] * kLog2e;
+    bias[c] = a.dt_bias ? a.dt_bias[dch[c]] : 0.f;
+    Dd[c] = a.D ? a.D[dch[c]] : 0.f;
+  }
+  const uint16_t* up = reinterpret_cast<const uint16_t*>(a.u);
+  const uint16_t* dp = reinterpret_cast<const uint16_t*>(a.delta);
+  const uint16_t* zp = reinterpret_cast<const uint16_t*>(a.z);
+  uint16_t* op = reinterpret_cast<uint16_t*>(a.out);
 
-  // initial state
-  for (int i = tid; i < kDB * N; i += kThreads) {
-    const int dd = i / N, n = i % N;
-    const int dg = d0 + dd;
-    sm.H[i] = (a.h0 && dg < a.dim) ? a.h0[((long long)b * a.dim + dg) * N + n] : 0.f;
+  // the transposed state H'[d][n] in accumulator layout: Ht[nt][0..1] = channel g, states
+  // 8 nt + 2 tg + {0, 1}; Ht[nt][2..3] = channel g + 8, same states
+  float Ht[kNT][4];
+#pragma unroll
+  for (int nt = 0; nt < kNT; ++nt) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int c = e >> 1, n = 8 * nt + 2 * tg + (e & 1);
+      Ht[nt][e] = a.h0 ? a.h0[((long long)b * a.dim + dch[c]) * N + n] : 0.f;
+    }
   }
 
-  for (int t0 = 0; t0 < L; t0 += kT) {
-    const int nv = min(kT, L - t0);
-    __syncthreads();  // the previous chunk's reads of every table are done
-    // ---- phase A: channel scalars (threads 0..63) and the B/C tiles (threads 64..127)
-    if (own) {
-      // the chunk's 16 steps of u, delta, z: two 16-byte pieces per row when aligned
-      uint32_t uw[8], dw[8], zw[8];
-      const auto load16 = [&](const void* base, uint32_t (&w)[8]) {
-        const uint16_t* p = reinterpret_cast<const uint16_t*>(base) + row + t0;
-        if (nv == kT && a.rows16) {
-          const uint4 v0 = reinterpret_cast<const uint4*>(p)[0], v1 = reinterpret_cast<const uint4*>(p)[1];
-          w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
-          w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+  // B/C tiles of chunk k into ring slot k % kStages: 16-byte cp.async pieces when rows allow
+  // them, else element loads (ragged tail, unaligned rows) with zeros past L
+  const auto issue = [&](int k) {
+    if (k < nchunk) {
+      SsdStage<N>& st = ring[k % kStages];
+      const int t0 = k * kT;
+      if (a.rows16 && t0 + kT <= L) {
+        for (int p = tid; p < 4 * N; p += 32 * W) {
+          const int which = p / (2 * N), rem = p % (2 * N), n = rem >> 1, h = rem & 1;
+          const uint16_t* src = (which ? Cg : Bg) + (long long)n * L + t0 + 8 * h;
+          uint16_t* dst = (which ? st.Cs : st.Bs) + n * kLdS + 8 * h;
+          cp16(dst, src);
+        }
+      } else {
+        for (int p = tid; p < 2 * N * kT; p += 32 * W) {
+          const int which = p / (N * kT), rem = p % (N * kT), n = rem / kT, t = rem % kT;
+          const uint16_t* src = (which ? Cg : Bg) + (long long)n * L + t0 + t;
+          (which ? st.Cs : st.Bs)[n * kLdS + t] = t0 + t < L ? *src : (uint16_t)0;
+        }
+      }
+    }
+    cp_commit();
+  };
+  const bool vec_rows = a.rows16 != 0;
+  const auto load_in = [&](int k, ChunkIn& in) {
+    const int t0 = k * kT;
+    const bool vec = vec_rows && t0 + kT <= L;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const long long t = t0 + 2 * tg + 8 * hh;
+        in.u[c][hh] = ld_pair(up + row[c], t, L, vec);
+        in.dl[c][hh] = ld_pair(dp + row[c], t, L, vec);
+        in.z[c][hh] = zp ? ld_pair(zp + row[c], t, L, vec) : 0u;
+      }
+    }
+  };
+
+#pragma unroll
+  for (int k = 0; k < kStages - 1; ++k) issue(k);
+  ChunkIn nxt;
+  load_in(0, nxt);
+
+  for (int k = 0; k < nchunk; ++k) {
+    cp_wait<kStages - 2>();  // chunk k's B/C tiles have landed (this thread's copies)
+    __syncthreads();         // ... every thread's; and every warp is done with chunk k - 1's slot
+    issue(k + kStages - 1);  // into the slot chunk k - 1 used
+    const ChunkIn cur = nxt;
+    if (k + 1 < nchunk) load_in(k + 1, nxt);
+    const SsdStage<N>& st = ring[k % kStages];
+    const int t0 = k * kT;
+
+    // ---- per (channel, step): Δ, Δx, gate; index j: steps 2tg, 2tg+1, 2tg+8, 2tg+9
+    float dl[2][4], xv[2][4], gt[2][4], uv[2][4];
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t wu = cur.u[c][j >> 1], wd = cur.dl[c][j >> 1], wz = cur.z[c][j >> 1];
+        const float u = (j & 1) ? bf16_hi(wu) : bf16_lo(wu);
+        const float v = ((j & 1) ? bf16_hi(wd) : bf16_lo(wd)) + bias[c];
+        const int t = t0 + 2 * tg + (j & 1) + 8 * (j >> 1);
+        const bool live = t < L;
+        const float D = a.softplus ? softplus_fast(v) : v;
+        dl[c][j] = live ? D : 0.f;
+        uv[c][j] = live ? u : 0.f;
+        xv[c][j] = dl[c][j] * uv[c][j];
+        if (zp) {
+          const float z = (j & 1) ? bf16_hi(wz) : bf16_lo(wz);
+          gt[c][j] = z * sigmoid_fast(z);
         } else {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) w[i] = 0u;
-          for (int e = 0; e < nv; ++e) w[e >> 1] |= (uint32_t)p[e] << (16 * (e & 1));
-        }
-      };
-      load16(a.u, uw);
-      load16(a.delta, dw);
-      if (a.z) load16(a.z, zw);
-      float S = 0.f;
-      float mx = 0.f;
-      bool bad = false;
-#pragma unroll
-      for (int t = 0; t < kT; ++t) {
-        float Dv = 0.f, xv = 0.f, gv = 1.f;
-        if (t < nv) {
-          const float u = (t & 1) ? bf16_hi(uw[t >> 1]) : bf16_lo(uw[t >> 1]);
-          const float v = ((t & 1) ? bf16_hi(dw[t >> 1]) : bf16_lo(dw[t >> 1])) + bias;
-          Dv = a.softplus ? softplus_fast(v) : v;
-          xv = Dv * u;
-          if (a.z) {
-            const float zv = (t & 1) ? bf16_hi(zw[t >> 1]) : bf16_lo(zw[t >> 1]);
-            gv = zv * sigmoid_fast(zv);
-          }
-          sm.Ux[dl * kT + t] = u;  // x_t for the D skip
-        } else {
-          sm.Ux[dl * kT + t] = 0.f;
-        }
-        S += Dv;
-        bad = bad || !(Dv == Dv) || fabsf(Dv) > 3.0e38f;
-        sm.Dl[dl * kT + t] = S;   // cumulative step S_t
-        sm.Xs[dl * kT + t] = xv;  // Δ_t x_t
-        sm.Gt[dl * kT + t] = gv;  // silu(z_t)
-        mx = fmaxf(mx, fabsf(S));
-      }
-      sm.fb[dl] = (bad || fabsf(Ad) * mx > 80.f) ? 1 : 0;
-      sm.Dskip[dl] = Dd;
-    } else {
-      const int i0 = tid - kDB;  // 64 threads load N rows x 16 steps of B and of C
-      for (int i = i0; i < N * 2; i += kThreads - kDB) {
-        const int n = i >> 1, h = i & 1;  // steps 8 h .. 8 h + 7 of state row n
-        uint32_t bw[4] = {0u, 0u, 0u, 0u}, cw[4] = {0u, 0u, 0u, 0u};
-        const long long off = (long long)n * L + t0 + 8 * h;
-        if (8 * h + 8 <= nv && ((off & 7) == 0) && a.rows16) {  // aligned 16-byte pieces
-          const uint4 vb = *reinterpret_cast<const uint4*>(Bg + off);
-          const uint4 vc = *reinterpret_cast<const uint4*>(Cg + off);
-          bw[0] = vb.x; bw[1] = vb.y; bw[2] = vb.z; bw[3] = vb.w;
-          cw[0] = vc.x; cw[1] = vc.y; cw[2] = vc.z; cw[3] = vc.w;
-        } else {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            if (8 * h + e < nv) {
-              bw[e >> 1] |= (uint32_t)Bg[off + e] << (16 * (e & 1));
-              cw[e >> 1] |= (uint32_t)Cg[off + e] << (16 * (e & 1));
-            }
-          }
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const uint16_t vb = (uint16_t)(bw[e >> 1] >> (16 * (e & 1)));
-          const uint16_t vc = (uint16_t)(cw[e >> 1] >> (16 * (e & 1)));
-          const int s = 8 * h + e;
-          sm.Bn[n * SM::kLdT + s] = vb;
-          sm.Bt[s * SM::kLdN + n] = vb;
-          sm.Ct[s * SM::kLdN + n] = vc;
+          gt[c][j] = 1.f;
         }
       }
     }
-    __syncthreads();
-    // ---- phase B: decay factors and scaled inputs (threads 0..63); bf16 copy of the state
-    if (own) {
-      const float Sm = sm.Dl[dl * kT + kT / 2 - 1], Send = sm.Dl[dl * kT + kT - 1];
-      const bool fbk = sm.fb[dl] != 0;
-      const float eAm = expf(Ad * Sm), eEnd_m = expf(Ad * (Send - Sm));
+    // ---- cumulative steps over the chunk: scans over the quad's lanes (lane tg holds the
+    // pairs (2tg, 2tg+1) of the low and of the high 8 steps)
+    float S[2][4], Sm[2], Se[2];
+    bool fb[2];
 #pragma unroll
-      for (int t = 0; t < kT; ++t) {
-        const float S = sm.Dl[dl * kT + t];
-        const float P = expf(Ad * (S - Sm));                 // e^{A (S_t - S_m)}
-        const float Q = expf(Ad * (Sm - S));                 // 1 / P_t
-        const float x = sm.Xs[dl * kT + t];
-        sm.P[dl * kT + t] = P;
-        sm.E[dl * kT + t] = eAm * P;                         // e^{A S_t}
-        sm.X1[dl * SM::kLdT + t] = to_bf16(fbk ? 0.f : Q * x);
-        sm.X2[dl * SM::kLdT + t] = to_bf16(fbk ? 0.f : eEnd_m * Q * x);  // e^{A (S_end - S_t)} x
-      }
-      sm.Eend[dl] = expf(Ad * Send);
-    }
-    for (int i = tid; i < kDB * N; i += kThreads) {
-      const int dd = i / N, n = i % N;
-      sm.Hb[dd * SM::kLdN + n] = to_bf16(sm.H[i]);
-    }
-    __syncthreads();
-    // ---- phase C: the products.  Warps 0, 1: G; every warp: its 16 channels of Y2 and U
-    if (warp < 2) {
-      float g[4] = {0.f, 0.f, 0.f, 0.f};
-      mma_tile<N>(g, sm.Ct, SM::kLdN, sm.Bt + (8 * warp) * SM::kLdN, SM::kLdN, lane);
-      const int r = lane >> 2, c = 8 * warp + 2 * (lane & 3);
-      // mask: s <= t
-      sm.Gm[r * SM::kLdT + c] = to_bf16(c <= r ? g[0] : 0.f);
-      sm.Gm[r * SM::kLdT + c + 1] = to_bf16(c + 1 <= r ? g[1] : 0.f);
-      sm.Gm[(r + 8) * SM::kLdT + c] = to_bf16(c <= r + 8 ? g[2] : 0.f);
-      sm.Gm[(r + 8) * SM::kLdT + c + 1] = to_bf16(c + 1 <= r + 8 ? g[3] : 0.f);
-    }
-    float y2[2][4];
+    for (int c = 0; c < 2; ++c) {
+      const float p = dl[c][0] + dl[c][1], q = dl[c][2] + dl[c][3];
+      float ip = p, iq = q;
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      y2[j][0] = y2[j][1] = y2[j][2] = y2[j][3] = 0.f;
-      mma_tile<N>(y2[j], sm.Ct, SM::kLdN, sm.Hb + (16 * warp + 8 * j) * SM::kLdN, SM::kLdN, lane);
-    }
-    // U = B^T X'': rows n (N / 16 tiles), columns the warp's 16 channels; h_out = e^{A S_end} h + U
-#pragma unroll
-    for (int mt = 0; mt < N / 16; ++mt) {
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        float u4[4] = {0.f, 0.f, 0.f, 0.f};
-        mma_tile<kT>(u4, sm.Bn + (16 * mt) * SM::kLdT, SM::kLdT,
-                     sm.X2 + (16 * warp + 8 * j) * SM::kLdT, SM::kLdT, lane);
-        const int n = 16 * mt + (lane >> 2), dd = 16 * warp + 8 * j + 2 * (lane & 3);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int nn = n + (e >> 1) * 8, dc = dd + (e & 1);
-          if (!sm.fb[dc]) sm.H[dc * N + nn] = fmaf(sm.Eend[dc], sm.H[dc * N + nn], u4[e]);
+      for (int off = 1; off < 4; off <<= 1) {
+        const float np = __shfl_up_sync(0xffffffffu, ip, off, 4);
+        const float nq = __shfl_up_sync(0xffffffffu, iq, off, 4);
+        if (tg >= off) {
+          ip += np;
+          iq += nq;
         }
       }
-    }
-    __syncthreads();  // Gm is complete
-    // Y1 = mask(G) X' and the outputs of the warp's 16 channels
+      const float lo_total = __shfl_sync(0xffffffffu, ip, 3, 4);
+      const float hi_total = __shfl_sync(0xffffffffu, iq, 3, 4);
+      S[c][0] = ip - p + dl[c][0];
+      S[c][1] = ip;
+      S[c][2] = lo_total + iq - q + dl[c][2];
+      S[c][3] = lo_total + iq;
+      Sm[c] = lo_total;  // S at step 7, the chunk's middle
+      Se[c] = lo_total + hi_total;
+      float mrel = 0.f, mabs = 0.f;
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      float y1[4] = {0.f, 0.f, 0.f, 0.f};
-      mma_tile<kT>(y1, sm.Gm, SM::kLdT, sm.X1 + (16 * warp + 8 * j) * SM::kLdT, SM::kLdT, lane);
-      const int t = lane >> 2, dd = 16 * warp + 8 * j + 2 * (lane & 3);
+      for (int j = 0; j < 4; ++j) {
+        mrel = fmaxf(mrel, fabsf(S[c][j] - Sm[c]));
+        mabs = fmaxf(mabs, fabsf(S[c][j]));
+      }
+      // NaN-safe: a non-finite step fails the comparisons
+      int ok = (fabsf(al[c]) * kLn2 * mrel <= 60.f && fabsf(al[c]) * kLn2 * mabs <= 80.f) ? 1 : 0;
+      ok &= __shfl_xor_sync(0xffffffffu, ok, 1, 4);
+      ok &= __shfl_xor_sync(0xffffffffu, ok, 2, 4);
+      fb[c] = ok == 0;
+    }
+    // ---- decay factors and the scaled inputs (A operands of Y1' and U')
+    float P[2][4], E[2][4], scale[2];
+    uint32_t x1[4], x2[4];  // A fragments: {row g k lo, row g+8 k lo, row g k hi, row g+8 k hi}
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const float eAm = ex2_mufu(Sm[c] * al[c]);
+      const float eEm = ex2_mufu((Se[c] - Sm[c]) * al[c]);
+      scale[c] = fb[c] ? 1.f : ex2_mufu(Se[c] * al[c]);
+      float q1[4], q2[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float r = (S[c][j] - Sm[c]) * al[c];
+        P[c][j] = ex2_mufu(r);
+        E[c][j] = eAm * P[c][j];
+        const float Q = ex2_mufu(-r);
+        q1[j] = fb[c] ? 0.f : Q * xv[c][j];
+        q2[j] = fb[c] ? 0.f : eEm * q1[j];
+      }
+      x1[c] = pack_bf16x2(q1[0], q1[1]);
+      x1[2 + c] = pack_bf16x2(q1[2], q1[3]);
+      x2[c] = pack_bf16x2(q2[0], q2[1]);
+      x2[2 + c] = pack_bf16x2(q2[2], q2[3]);
+    }
+
+    // ---- G = C B^T and Y2' = H' C^T, sharing the C fragments of each 16-state k-step
+    float G[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // s tiles 0..7, 8..15
+    float Y2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // t tiles 0..7, 8..15
+#pragma unroll
+    for (int kk = 0; kk < N / 16; ++kk) {
+      uint32_t cf[4], bf[4];
+      ldsm_x4_t(cf, blk(st.Cs, 16 * kk, lane));  // {t0-7|n lo, t8-15|n lo, t0-7|n hi, t8-15|n hi}
+      ldsm_x4_t(bf, blk(st.Bs, 16 * kk, lane));  // {s0-7|n lo, s8-15|n lo, s0-7|n hi, s8-15|n hi}
+      mma16816(G[0], cf[0], cf[1], cf[2], cf[3], bf[0], bf[2]);
+      mma16816(G[1], cf[0], cf[1], cf[2], cf[3], bf[1], bf[3]);
+      const uint32_t h0 = pack_bf16x2(Ht[2 * kk][0], Ht[2 * kk][1]);
+      const uint32_t h1 = pack_bf16x2(Ht[2 * kk][2], Ht[2 * kk][3]);
+      const uint32_t h2 = pack_bf16x2(Ht[2 * kk + 1][0], Ht[2 * kk + 1][1]);
+      const uint32_t h3 = pack_bf16x2(Ht[2 * kk + 1][2], Ht[2 * kk + 1][3]);
+      mma16816(Y2[0], h0, h1, h2, h3, cf[0], cf[2]);
+      mma16816(Y2[1], h0, h1, h2, h3, cf[1], cf[3]);
+    }
+    // ---- H' <- e^{A S_end} H' + X2' B   (fb channels: scale 1, zero inputs: unchanged)
+#pragma unroll
+    for (int nt = 0; nt < kNT; nt += 2) {
+      uint32_t bn[4];
+      ldsm_x4(bn, blk(st.Bs, 8 * nt, lane));  // {n tile nt: s lo, s hi; n tile nt+1: s lo, s hi}
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int tt = t + (e >> 1) * 8, dc = dd + (e & 1);
-        if (sm.fb[dc]) continue;
-        const int k = dc * kT + tt;
-        const float y = fmaf(sm.P[k], y1[e], fmaf(sm.E[k], y2[j][e], sm.Dskip[dc] * sm.Ux[k]));
-        sm.Y[k] = to_bf16(y * sm.Gt[k]);
+        Ht[nt][e] *= scale[e >> 1];
+        Ht[nt + 1][e] *= scale[e >> 1];
+      }
+      mma16816(Ht[nt], x2[0], x2[1], x2[2], x2[3], bn[0], bn[1]);
+      mma16816(Ht[nt + 1], x2[0], x2[1], x2[2], x2[3], bn[2], bn[3]);
+    }
+    // ---- Y1' = X1' mask(G)^T: G's accumulators (rows t, cols s) are the B fragments
+    // (k = s, n = t) once masked to s <= t
+    float Y1[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    {
+      const int s0 = 2 * tg, r0 = g;
+      const auto m = [](float v, int s, int t) { return s <= t ? v : 0.f; };
+      // t tile 0: rows t = g; t tile 1: rows t = g + 8
+      const uint32_t b00 = pack_bf16x2(m(G[0][0], s0, r0), m(G[0][1], s0 + 1, r0));
+      const uint32_t b01 = pack_bf16x2(m(G[1][0], s0 + 8, r0), m(G[1][1], s0 + 9, r0));
+      const uint32_t b10 = pack_bf16x2(m(G[0][2], s0, r0 + 8), m(G[0][3], s0 + 1, r0 + 8));
+      const uint32_t b11 = pack_bf16x2(m(G[1][2], s0 + 8, r0 + 8), m(G[1][3], s0 + 9, r0 + 8));
+      mma16816(Y1[0], x1[0], x1[1], x1[2], x1[3], b00, b01);
+      mma16816(Y1[1], x1[0], x1[1], x1[2], x1[3], b10, b11);
+    }
+    // ---- outputs: y = P Y1 + e^{A S_t} Y2 + D x, gated.  Accumulator (tile T, e): channel
+    // e / 2, step index j = 2 T + e % 2
+    float yo[2][4];
+#pragma unroll
+    for (int T = 0; T < 2; ++T) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int c = e >> 1, j = 2 * T + (e & 1);
+        const float y = fmaf(P[c][j], Y1[T][e], fmaf(E[c][j], Y2[T][e], Dd[c] * uv[c][j]));
+        yo[c][j] = y * gt[c][j];
       }
     }
-    __syncthreads();
-    // ---- phase D: channels whose chunk left the factorization's range: exact sequential pass
-    if (own && sm.fb[dl]) {
-      float prevS = 0.f;
-      for (int t = 0; t < nv; ++t) {
-        const float S = sm.Dl[dl * kT + t];
-        const float ab = expf(Ad * (S - prevS));
-        prevS = S;
-        const float x = sm.Xs[dl * kT + t];
-        float y = 0.f;
-        for (int n = 0; n < N; ++n) {
-          const float hb = fmaf(ab, sm.H[dl * N + n], x * bf16_to_f32(sm.Bt[t * SM::kLdN + n]));
-          sm.H[dl * N + n] = hb;
-          y = fmaf(bf16_to_f32(sm.Ct[t * SM::kLdN + n]), hb, y);
+    // ---- channels outside the factorisation's range this chunk: exact sequential pass over
+    // the states the quad holds (rare; warp-uniform branch, per-channel predicates)
+    if (__any_sync(0xffffffffu, fb[0] || fb[1])) {
+      const int qb = lane & ~3;
+#pragma unroll
+      for (int t = 0; t < kT; ++t) {
+        const int to = (t & 7) >> 1, jo = (t & 1) + 2 * (t >> 3);  // owner lane, its index
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const float dt = __shfl_sync(0xffffffffu, dl[c][jo], qb | to);
+          const float xt = __shfl_sync(0xffffffffu, xv[c][jo], qb | to);
+          const float ab = ex2_mufu(dt * al[c]);
+          float yp = 0.f;
+#pragma unroll
+          for (int nt = 0; nt < kNT; ++nt) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int n = 8 * nt + 2 * tg + e;
+              const float bv = bf16_to_f32(st.Bs[n * kLdS + t]);
+              const float cv = bf16_to_f32(st.Cs[n * kLdS + t]);
+              float& h = Ht[nt][2 * c + e];
+              if (fb[c]) h = fmaf(ab, h, xt * bv);
+              yp = fmaf(cv, h, yp);
+            }
+          }
+          yp += __shfl_xor_sync(0xffffffffu, yp, 1);
+          yp += __shfl_xor_sync(0xffffffffu, yp, 2);
+          if (fb[c] && tg == to) yo[c][jo] = fmaf(Dd[c], uv[c][jo], yp) * gt[c][jo];
         }
-        sm.Y[dl * kT + t] = to_bf16(fmaf(Dd, sm.Ux[dl * kT + t], y) * sm.Gt[dl * kT + t]);
       }
     }
-    __syncthreads();
-    // ---- outputs of the chunk
-    if (own && dact) {
-      uint16_t* o = reinterpret_cast<uint16_t*>(a.out) + row + t0;
-      if (nv == kT && ((row + t0) & 7) == 0 && a.rows16) {
-        const uint4* src = reinterpret_cast<const uint4*>(sm.Y + dl * kT);
-        reinterpret_cast<uint4*>(o)[0] = src[0];
-        reinterpret_cast<uint4*>(o)[1] = src[1];
-      } else {
-        for (int t = 0; t < nv; ++t) o[t] = sm.Y[dl * kT + t];
+    // ---- store the chunk's outputs (bf16 pairs of steps)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      if (!act[c]) continue;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const long long t = t0 + 2 * tg + 8 * hh;
+        const uint32_t w = pack_bf16x2(yo[c][2 * hh], yo[c][2 * hh + 1]);
+        if (vec_rows && t0 + kT <= L) {
+          *reinterpret_cast<uint32_t*>(op + row[c] + t) = w;
+        } else {
+          if (t < L) op[row[c] + t] = (uint16_t)(w & 0xffffu);
+          if (t + 1 < L) op[row[c] + t + 1] = (uint16_t)(w >> 16);
+        }
       }
     }
   }
-  __syncthreads();
+  cp_wait<0>();
   if (a.hL) {
-    for (int i = tid; i < kDB * N; i += kThreads) {
-      const int dd = i / N, n = i % N;
-      const int dg = d0 + dd;
-      if (dg < a.dim) a.hL[((long long)b * a.dim + dg) * N + n] = sm.H[i];
+#pragma unroll
+    for (int nt = 0; nt < kNT; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int c = e >> 1, n = 8 * nt + 2 * tg + (e & 1);
+        if (act[c]) a.hL[((long long)b * a.dim + dch[c]) * N + n] = Ht[nt][e];
+      }
     }
   }
+}
+
+template <int N, int W>
+cudaError_t launch_n(const FwdArgs& a, cudaStream_t s) {
+  const unsigned grid = (unsigned)((long long)a.batch * ((a.dim + 16 * W - 1) / (16 * W)));
+  const size_t smem = kStages * sizeof(SsdStage<N>);
+  auto k = ssd_fwd_kernel<N, W>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k<<<grid, 32 * W, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+template <int N>
+cudaError_t launch_w(const FwdArgs& a, cudaStream_t s) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // 2 warps per CTA (32 channels) when 64-channel CTAs would leave fewer than 2 per SM
+  // (SSM_SSD_WPB=2 or 4 forces the choice)
+  const long long ctas4 = (long long)a.batch * ((a.dim + 63) / 64);
+  bool two = ctas4 < 2LL * sms;
+  const char* env = getenv("SSM_SSD_WPB");
+  if (env && (atoi(env) == 2 || atoi(env) == 4)) two = atoi(env) == 2;
+  return two ? launch_n<N, 2>(a, s) : launch_n<N, 4>(a, s);
 }
 
 }  // namespace
 
 cudaError_t launch_ssd_fwd(const FwdArgs& a, cudaStream_t s) {
-  const unsigned grid = (unsigned)((long long)a.batch * ((a.dim + kDB - 1) / kDB));
   switch (a.N) {
-    case 32: {
-      auto k = ssd_fwd_kernel<32>;
-      const size_t sm = sizeof(SsdSmem<32>);
-      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-      k<<<grid, kThreads, sm, s>>>(a);
-      break;
-    }
-    case 64: {
-      auto k = ssd_fwd_kernel<64>;
-      const size_t sm = sizeof(SsdSmem<64>);
-      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-      k<<<grid, kThreads, sm, s>>>(a);
-      break;
-    }
-    case 128: {
-      auto k = ssd_fwd_kernel<128>;
-      const size_t sm = sizeof(SsdSmem<128>);
-      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-      k<<<grid, kThreads, sm, s>>>(a);
-      break;
-    }
-    default:
-      return cudaErrorInvalidValue;
+    case 32: return launch_w<32>(a, s);
+    case 64: return launch_w<64>(a, s);
+    case 128: return launch_w<128>(a, s);
+    default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 }  // namespace ssm

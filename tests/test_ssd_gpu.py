@@ -45,9 +45,12 @@ def ref(x, softplus=True, channels=None):
                            channels=channels)
 
 
+@pytest.mark.parametrize("wpb", ["2", "4"])
 @pytest.mark.parametrize("N", [32, 64, 128])
-@pytest.mark.parametrize("shape", [(2, 128, 256), (1, 96, 200), (2, 64, 17)])
-def test_matches_oracle(N, shape):
+@pytest.mark.parametrize("shape", [(2, 128, 256), (1, 96, 200), (2, 64, 17), (1, 40, 45)])
+def test_matches_oracle(monkeypatch, wpb, N, shape):
+    """Both CTA widths (32 or 64 channels), partial channel tiles, ragged time tails."""
+    monkeypatch.setenv("SSM_SSD_WPB", wpb)
     batch, dim, L = shape
     x = inputs(batch, dim, L, N, seed=61)
     out, hL = gpu(x)
