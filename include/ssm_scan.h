@@ -328,6 +328,36 @@ SSM_API int ssm_state_update_ex(float* state, const void* x, const void* dt, con
 SSM_API int ssm_wait_timeouts(unsigned int* count);
 
 /*
+ * Sequence split (a long sequence cut into consecutive segments, e.g. one per GPU).  The scan is
+ * a composition of affine maps of the state ("Temel Fikirler": the recurrence is a parallel
+ * associative scan): a segment with steps Δ_t maps the state entering it to
+ *   h_out = exp(A ΣΔ) h_in + hend,
+ * where hend is the segment's end state from a zero state (per state n: exp(A_n ΣΔ)).
+ *
+ * ssm_scan_fwd_summary: the map of one segment.  Arguments as ssm_scan_fwd_ex (flags
+ *   SSM_SCALAR_A and SSM_ZOH; shared or grouped B/C), plus
+ *     hend  [batch][dim][dstate] f32   OUT: the state after the segment from a zero state
+ *     dsum  [batch][dim] f32 or NULL   OUT: ΣΔ over the segment (Kahan-summed in f32)
+ *   and ssm_scan_fwd_summary_workspace_size() bytes of workspace (256-byte aligned).
+ * ssm_scan_chain: the state entering each of nseg consecutive segments,
+ *     hin[0] = h0 (zero if NULL),  hin[r+1] = exp(A dsum[r]) hin[r] + hend[r],
+ *   hend, hin [nseg][batch][dim][dstate] f32, dsum [nseg][batch][dim] f32, A as for the scan
+ *   (flags: SSM_SCALAR_A).  Running each segment's forward scan from its hin[r] gives the
+ *   full-sequence results, up to rounding.
+ * Errors as for the scans.
+ */
+SSM_API size_t ssm_scan_fwd_summary_workspace_size(int batch, int dim, int seqlen, int dstate,
+                                                   int bc_groups, int io_dtype, int flags);
+SSM_API int ssm_scan_fwd_summary(const void* u, const void* delta, const float* A, const void* B,
+                                 const void* C, const float* dt_bias, int delta_softplus,
+                                 float* hend, float* dsum, void* workspace,
+                                 size_t workspace_bytes, int batch, int dim, int seqlen,
+                                 int dstate, int bc_groups, int io_dtype, int flags, void* stream);
+SSM_API int ssm_scan_chain(const float* hend, const float* dsum, const float* A, const float* h0,
+                           float* hin, int nseg, int batch, int dim, int dstate, int flags,
+                           void* stream);
+
+/*
  * General element strides.  The entry points above take dense tensors (the layouts given per
  * argument, or the (B, L, D) layout of SSM_CHANNELS_LAST).  These take each io tensor with its
  * own element strides, e.g. views cut out of a larger projection output, transposed views, or B

@@ -22,7 +22,8 @@ from ._abi import CKPT_STEPS, MAX_DSTATE
 __all__ = ["ssm_scan_fwd", "ssm_scan_bwd", "ssm_scan_fwd_scalar_a", "ssm_scan_bwd_scalar_a",
            "ssm_scan_fwd_host", "fwd_host_workspace_bytes",
            "ssm_state_update", "fwd_workspace_bytes", "ssm_scan_fwd_strided",
-           "ssm_scan_bwd_strided", "ssm_state_update_strided",
+           "ssm_scan_bwd_strided", "ssm_state_update_strided", "ssm_scan_fwd_summary",
+           "ssm_scan_chain",
            "bwd_workspace_bytes", "CKPT_STEPS", "MAX_DSTATE", "library_path"]
 
 _IO = {torch.float32: _abi.SSM_F32, torch.bfloat16: _abi.SSM_BF16}
@@ -514,3 +515,50 @@ def ssm_state_update_strided(state, x, dt, A, B, C, D=None, z=None, dt_bias=None
         ctypes.byref(st), _stream(dev))
     _abi.check(rc, "ssm_state_update_strided")
     return out
+
+
+# ------------------------------------------------------------------ sequence split
+def ssm_scan_fwd_summary(u, delta, A, B, C, dt_bias=None, delta_softplus=True, scalar_a=False,
+                         zoh=False, workspace=None):
+    """The affine map of one sequence segment: returns (hend [batch, dim, N], dsum [batch, dim]),
+    the state after the segment from a zero state and ΣΔ over it, so that the segment maps an
+    entering state h to exp(A dsum) h + hend."""
+    dev = _on_gpu(u, "u")
+    batch, dim, L = u.shape
+    io = u.dtype
+    code = _io_code(io)
+    G, N, bc_shape = _bc_layout(B, batch, L)
+    _need(u, "u", (batch, dim, L), io, dev)
+    _need(delta, "delta", (batch, dim, L), io, dev)
+    _need(A, "A", (dim,) if scalar_a else (dim, N), torch.float32, dev)
+    _need(B, "B", bc_shape, io, dev)
+    _need(C, "C", bc_shape, io, dev)
+    _opt(dt_bias, "dt_bias", (dim,), torch.float32, dev)
+    hend = torch.empty((batch, dim, N), dtype=torch.float32, device=dev)
+    dsum = torch.empty((batch, dim), dtype=torch.float32, device=dev)
+    flags = _flags(scalar_a, False, zoh)
+    nws = int(_abi.lib().ssm_scan_fwd_summary_workspace_size(batch, dim, L, N, G, code, flags))
+    ws = _workspace(nws, dev, workspace)
+    rc = _abi.lib().ssm_scan_fwd_summary(
+        _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(dt_bias), int(bool(delta_softplus)),
+        _ptr(hend), _ptr(dsum), _ptr(ws), 0 if ws is None else ws.numel(), batch, dim, L, N, G,
+        code, flags, _stream(dev))
+    _abi.check(rc, "ssm_scan_fwd_summary")
+    return hend, dsum
+
+
+def ssm_scan_chain(hend, dsum, A, h0=None, scalar_a=False):
+    """The state entering each of S consecutive segments given their maps (hend [S, batch, dim,
+    N], dsum [S, batch, dim], as from :func:`ssm_scan_fwd_summary`) and the state h0 entering the
+    first: returns hin [S, batch, dim, N]."""
+    dev = _on_gpu(hend, "hend")
+    S, batch, dim, N = hend.shape
+    _need(hend, "hend", (S, batch, dim, N), torch.float32, dev)
+    _need(dsum, "dsum", (S, batch, dim), torch.float32, dev)
+    _need(A, "A", (dim,) if scalar_a else (dim, N), torch.float32, dev)
+    _opt(h0, "h0", (batch, dim, N), torch.float32, dev)
+    hin = torch.empty_like(hend)
+    rc = _abi.lib().ssm_scan_chain(_ptr(hend), _ptr(dsum), _ptr(A), _ptr(h0), _ptr(hin), S, batch,
+                                   dim, N, _flags(scalar_a, False, False), _stream(dev))
+    _abi.check(rc, "ssm_scan_chain")
+    return hin

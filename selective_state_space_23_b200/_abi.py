@@ -78,6 +78,10 @@ SIGNATURES = {
     "ssm_scan_bwd_strided": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp,
                                   _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                                   _i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(Strides), _vp]),
+    "ssm_scan_fwd_summary_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "ssm_scan_fwd_summary": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _sz,
+                                  _i, _i, _i, _i, _i, _i, _i, _vp]),
+    "ssm_scan_chain": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
     "ssm_state_update_strided_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "ssm_state_update_strided": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp,
                                       _sz, _i, _i, _i, _i, _i, _i,

@@ -472,6 +472,58 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
   return SSM_OK;
 }
 
+// Time chunks of a whole-sequence summary and its scratch: the forward's plan with one more
+// chunk slot (summaries, entering states, ΣΔ).
+FwdPlan plan_summary(int batch, int dim, int seqlen) {
+  FwdPlan p = plan_fwd(batch, dim, seqlen, fwd_chw(false));
+  const size_t nch = (size_t)batch * dim;
+  const size_t slots = (size_t)p.nchunk + 1;
+  p.ws_bytes = 2 * align_up(slots * nch * ssm::kNS * 4) + align_up(slots * nch * 4);
+  return p;
+}
+
+// The end state from zero of a whole sequence, out of the carry's entering states (16-state
+// rows) into [batch][dim][N], and each channel's ΣΔ summed (Kahan) over the S chunk summaries.
+__global__ void summary_finish_kernel(const float* __restrict__ hin_end,
+                                      const float* __restrict__ dsum, int S, long long nch, int N,
+                                      float* __restrict__ hend, float* __restrict__ dsum_out) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= nch * N) return;
+  const long long ch = i / N;
+  const int n = (int)(i % N);
+  hend[i] = hin_end[ch * ssm::kNS + n];
+  if (n == 0 && dsum_out) {
+    float acc = 0.f, comp = 0.f;
+    for (int j = 0; j < S; ++j) {
+      const float y = dsum[(long long)j * nch + ch] - comp;
+      const float t = acc + y;
+      comp = (t - acc) - y;
+      acc = t;
+    }
+    dsum_out[ch] = acc;
+  }
+}
+
+// The state entering each of nseg consecutive segments: hin[0] = h0 (zero without one) and
+// hin[r + 1] = exp(A ΣΔ_r) hin[r] + hend[r], the composition of the segments' affine maps in
+// order (one thread per (channel, state), the segments in sequence).
+__global__ void chain_kernel(const float* __restrict__ hend, const float* __restrict__ dsum,
+                             const float* __restrict__ A, int scalar_a,
+                             const float* __restrict__ h0, float* __restrict__ hin, int nseg,
+                             long long nch, int dim, int N) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= nch * N) return;
+  const long long ch = i / N;
+  const int n = (int)(i % N), d = (int)(ch % dim);
+  const float An = scalar_a ? A[d] : A[(long long)d * N + n];
+  const long long stride = nch * N;
+  float h = h0 ? h0[i] : 0.f;
+  for (int r = 0; r < nseg; ++r) {
+    hin[(long long)r * stride + i] = h;
+    h = fmaf(expf(An * dsum[(long long)r * nch + ch]), h, hend[(long long)r * stride + i]);
+  }
+}
+
 // A[d] copied to every state: Af[d][n] = A[d].
 __global__ void broadcast_a_kernel(const float* __restrict__ A, float* __restrict__ Af, int dim,
                                    int N) {
@@ -838,6 +890,108 @@ int ssm_scan_bwd_scalar_a(const void* u, const void* delta, const float* A, cons
   return ssm_scan_bwd_ex(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL, ckpt,
                          du, ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, workspace, workspace_bytes,
                          batch, dim, seqlen, dstate, 1, io_dtype, SSM_SCALAR_A, stream);
+}
+
+// Whole-sequence summary of the forward scan (the segment map of a sequence split across GPUs):
+// the state after the sequence from a zero state and each channel's ΣΔ.  Runs the forward's
+// summary pass over the planner's time chunks (one more chunk slot than chunks, so the carry
+// pass's last entering state is the sequence's end state), the carry pass from zero, and a
+// finishing kernel.
+size_t ssm_scan_fwd_summary_workspace_size(int batch, int dim, int seqlen, int dstate,
+                                           int bc_groups, int io_dtype, int flags) {
+  if (flags & ~(SSM_SCALAR_A | SSM_ZOH)) return 0;
+  if (check_dims(batch, dim, seqlen, dstate, io_dtype) != SSM_OK) return 0;
+  if (check_groups(dim, bc_groups) != SSM_OK) return 0;
+  return plan_summary(batch, dim, seqlen).ws_bytes;
+}
+
+int ssm_scan_fwd_summary(const void* u, const void* delta, const float* A, const void* B,
+                         const void* C, const float* dt_bias, int delta_softplus, float* hend,
+                         float* dsum, void* workspace, size_t workspace_bytes, int batch,
+                         int dim, int seqlen, int dstate, int bc_groups, int io_dtype, int flags,
+                         void* stream) {
+  g_err[0] = 0;
+  if (flags & ~(SSM_SCALAR_A | SSM_ZOH))
+    return fail(SSM_EINVAL, "unsupported flags 0x%x for a sequence summary", flags);
+  TRY(check_dims(batch, dim, seqlen, dstate, io_dtype));
+  TRY(check_groups(dim, bc_groups));
+  if (bc_groups == dim && bc_groups > 1)
+    return fail(SSM_EUNSUPPORTED, "sequence summaries take shared or grouped B/C");
+  const bool scalar_a = (flags & SSM_SCALAR_A) != 0;
+  const size_t es = esize(io_dtype);
+  const size_t nx = (size_t)batch * dim * seqlen * es;
+  const size_t nbc = (size_t)batch * bc_groups * dstate * seqlen * es;
+  const size_t nch = (size_t)batch * dim;
+  TRY(check_ptr(u, nx, es, "u"));
+  TRY(check_ptr(delta, nx, es, "delta"));
+  TRY(check_ptr(A, (size_t)dim * (scalar_a ? 1 : dstate) * 4, 4, "A"));
+  TRY(check_ptr(B, nbc, es, "B"));
+  TRY(check_ptr(C, nbc, es, "C"));
+  TRY(check_opt(dt_bias, (size_t)dim * 4, 4, "dt_bias"));
+  TRY(check_ptr(hend, nch * dstate * 4, 4, "hend"));
+  TRY(check_opt(dsum, nch * 4, 4, "dsum"));
+  const FwdPlan plan = plan_summary(batch, dim, seqlen);
+  if (!workspace || workspace_bytes < plan.ws_bytes)
+    return fail(SSM_EWORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes,
+                plan.ws_bytes);
+  if (reinterpret_cast<uintptr_t>(workspace) & 255)
+    return fail(SSM_EINVAL, "workspace is not 256-byte aligned");
+  TRY(check_ptr(workspace, plan.ws_bytes, 256, "workspace"));
+  const int S = plan.nchunk;
+  const size_t slots = (size_t)S + 1;
+  char* w = reinterpret_cast<char*>(workspace);
+  float* summ = reinterpret_cast<float*>(w);
+  float* hin = reinterpret_cast<float*>(w + align_up(slots * nch * ssm::kNS * 4));
+  float* ds = reinterpret_cast<float*>(w + 2 * align_up(slots * nch * ssm::kNS * 4));
+  const bool vec = (seqlen * es) % 16 == 0 && aligned16(u) && aligned16(delta) && aligned16(B) &&
+                   aligned16(C);
+  ssm::FwdArgs a;
+  memset(&a, 0, sizeof(a));
+  a.u = u; a.delta = delta; a.B = B; a.C = C; a.A = A; a.dt_bias = dt_bias;
+  a.summ = summ; a.dsum = ds;
+  a.batch = batch; a.dim = dim; a.L = seqlen; a.N = dstate;
+  a.chunk_len = plan.chunk_len;
+  a.nchunk = S + 1;  // the summary pass covers chunks 0 .. S-1, every one of the sequence
+  a.softplus = delta_softplus ? 1 : 0;
+  a.scalar_a = scalar_a ? 1 : 0;
+  a.zoh = (flags & SSM_ZOH) ? 1 : 0;
+  a.bc_groups = bc_groups;
+  a.lpc = 2;
+  a.warps_per_b = (dim + 15) / 16;
+  a.nwarps = (long long)batch * a.warps_per_b;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = ssm::launch_fwd(a, io_dtype, vec, ssm::kFwdSummary, fwd_wpb(),
+                                  fwd_kmufu(a.nwarps * (long long)S), s);
+  if (e != cudaSuccess) return cuda_fail(e, "sequence summary pass");
+  if ((e = ssm::launch_fwd_carry(a, summ, ds, hin, s)) != cudaSuccess)
+    return cuda_fail(e, "sequence summary carry");
+  const long long n = (long long)nch * dstate;
+  summary_finish_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
+      hin + (size_t)S * nch * ssm::kNS, ds, S, (long long)nch, dstate, hend, dsum);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "sequence summary finish");
+  return SSM_OK;
+}
+
+int ssm_scan_chain(const float* hend, const float* dsum, const float* A, const float* h0,
+                   float* hin, int nseg, int batch, int dim, int dstate, int flags, void* stream) {
+  g_err[0] = 0;
+  if (flags & ~SSM_SCALAR_A) return fail(SSM_EINVAL, "unsupported flags 0x%x for a chain", flags);
+  if (nseg <= 0) return fail(SSM_EINVAL, "nseg must be positive, got %d", nseg);
+  TRY(check_dims(batch, dim, 1, dstate, SSM_F32));
+  const bool scalar_a = (flags & SSM_SCALAR_A) != 0;
+  const size_t nch = (size_t)batch * dim;
+  TRY(check_ptr(hend, (size_t)nseg * nch * dstate * 4, 4, "hend"));
+  TRY(check_ptr(dsum, (size_t)nseg * nch * 4, 4, "dsum"));
+  TRY(check_ptr(A, (size_t)dim * (scalar_a ? 1 : dstate) * 4, 4, "A"));
+  TRY(check_opt(h0, nch * dstate * 4, 4, "h0"));
+  TRY(check_ptr(hin, (size_t)nseg * nch * dstate * 4, 4, "hin"));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long long n = (long long)nch * dstate;
+  chain_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(hend, dsum, A, scalar_a ? 1 : 0, h0,
+                                                           hin, nseg, (long long)nch, dim, dstate);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "segment chain");
+  return SSM_OK;
 }
 
 int ssm_state_update_ex(float* state, const void* x, const void* dt, const float* A,

@@ -1,5 +1,12 @@
 """Multi-process (one process per GPU) plumbing for the scan.
 
+Two ways to shard one scan over GPUs:
+
+* batch rows (below): independent, no exchange in the forward;
+* the sequence (:func:`seq_split_scan_fwd`): each GPU holds a segment of the time axis; one
+  all-gather of the segments' (end state, ΣΔ) summaries, a local chain over the earlier
+  segments, then each GPU's forward from its true entering state.
+
 The selective scan is independent across batch rows and channels (each channel's recurrence
 only reads its own inputs and the per-row B_t, C_t), so a batch is sharded across ranks with no
 data exchange: each rank scans its rows and nothing is communicated on the forward data path.
@@ -65,3 +72,60 @@ def allreduce_param_grads(grads: Dict[str, torch.Tensor],
         grads[k].copy_(flat[off:off + n].view_as(grads[k]))
         off += n
     return grads
+
+
+def _library_ops(scalar_a: bool, zoh: bool):
+    import selective_state_space_23_b200 as ssm
+
+    def summary(u, delta, A, B, C, dt_bias, delta_softplus):
+        return ssm.ssm_scan_fwd_summary(u, delta, A, B, C, dt_bias=dt_bias,
+                                        delta_softplus=delta_softplus, scalar_a=scalar_a, zoh=zoh)
+
+    def chain(hend_all, dsum_all, A, h0):
+        return ssm.ssm_scan_chain(hend_all, dsum_all, A, h0=h0, scalar_a=scalar_a)
+
+    def scan(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, return_final_state):
+        f = ssm.ssm_scan_fwd_scalar_a if scalar_a else ssm.ssm_scan_fwd
+        return f(u, delta, A, B, C, D=D, z=z, dt_bias=dt_bias, delta_softplus=delta_softplus,
+                 h0=h0, return_final_state=return_final_state, zoh=zoh)
+
+    return {"summary": summary, "chain": chain, "scan": scan}
+
+
+def seq_split_scan_fwd(u, delta, A, B, C, D=None, z=None, dt_bias=None, delta_softplus=True,
+                       h0=None, return_final_state=False, scalar_a=False, zoh=False, group=None,
+                       ops=None):
+    """Forward scan of a sequence split along time over the ranks of ``group``: rank r holds
+    steps [t_r, t_{r+1}) of every time-indexed input (u, delta, z [batch, dim, L_r]; B, C
+    [batch, N, L_r] or [batch, G, N, L_r]), in rank order; A, D, dt_bias and h0 (the state
+    before the first step, or None) are the same on every rank.
+
+    The scan composes affine maps of the state (the associative scan of "Temel Fikirler" on the
+    Mamba summary page), so:
+
+    1. each rank summarises its segment as h -> exp(A ΣΔ) h + hend (``summary``);
+    2. one all-gather gives every rank every segment's (hend, ΣΔ), the only exchange step;
+    3. each rank chains the maps of the segments before its own, starting from h0 (``chain``);
+    4. each rank runs its segment's forward from that entering state (``scan``).
+
+    Returns the rank's outputs (and its segment's final state; the last rank's is the
+    sequence's).  ``ops`` replaces the three library calls (the CPU tests pass stand-ins built
+    on the fp64 oracle); every rank takes the same collective.
+    """
+    import torch.distributed as dist
+    ops = ops or _library_ops(scalar_a, zoh)
+    hend, dsum = ops["summary"](u, delta, A, B, C, dt_bias, delta_softplus)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
+        world = dist.get_world_size(group)
+        rank = dist.get_rank(group)
+        packed = torch.cat([hend.reshape(-1), dsum.reshape(-1)])
+        parts = [torch.empty_like(packed) for _ in range(world)]
+        dist.all_gather(parts, packed, group=group)
+        nh = hend.numel()
+        hend_all = torch.stack([p[:nh].view_as(hend) for p in parts])
+        dsum_all = torch.stack([p[nh:].view_as(dsum) for p in parts])
+    else:
+        rank = 0
+        hend_all, dsum_all = hend.unsqueeze(0), dsum.unsqueeze(0)
+    hin = ops["chain"](hend_all, dsum_all, A, h0)[rank]
+    return ops["scan"](u, delta, A, B, C, D, z, dt_bias, delta_softplus, hin, return_final_state)
