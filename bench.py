@@ -325,6 +325,22 @@ def _ssd(dev, rnd, prm, timeit, g):
         res[f"N{N}"] = {"fwd_ms": ms, "tokens_per_s": b * L / (ms * 1e-3),
                         "hbm_gbs": (4 * b * d * L * 2 + 2 * b * N * L * 2) / (ms * 1e-3) / 1e9,
                         "mma_tflops": flops / (ms * 1e-3) / 1e12}
+    del u, de, z, o, B, C
+    # the long sequence (1 x 256 x 2^20) with 64 states: 16 warps of channels, so the time axis
+    # is split into segments (summary, chain, output launches)
+    b, d, L, N = 1, 256, 1 << 20, 64
+    u, de, z = rnd((b, d, L)), rnd((b, d, L), 0.5), rnd((b, d, L))
+    _, D, bias = prm(d, 16, 1e-4, 1e-2)
+    A1 = -(torch.rand(d, device=dev, generator=g) * 15.0 + 1.0)
+    B, C = rnd((b, N, L)), rnd((b, N, L))
+    ws = torch.empty(max(1, ssm._abi.lib().ssm_scan_fwd_ex_workspace_size(b, d, L, N, 1, 1, 1)),
+                     dtype=torch.uint8, device=dev)
+    ms = timeit(lambda: ssm.ssm_scan_fwd_scalar_a(u, de, A1, B, C, D=D, z=z, dt_bias=bias,
+                                                  workspace=ws), 5)
+    res["long_seq_N64"] = {"shape": "1x256x1048576 bf16, A [dim]", "fwd_ms": ms,
+                           "tokens_per_s": b * L / (ms * 1e-3)}
+    del u, de, z, B, C, ws
+    torch.cuda.empty_cache()
     out["scalar_decay_large_n"] = res
     return out
 

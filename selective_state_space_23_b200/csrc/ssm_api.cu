@@ -211,6 +211,33 @@ FwdPlan plan_fwd(int batch, int dim, int seqlen, int chw) {
   return p;
 }
 
+// Time segments of the chunked matrix form (scalar decay, N > 16): as for the per-state scan,
+// segments of whole 16-step chunks when the warps (16 channels each) fill fewer than half the
+// schedulers (SSM_SSD_SPLIT overrides); scratch for the segments' end states, entering states
+// and ΣΔ.
+FwdPlan plan_ssd(int batch, int dim, int seqlen, int dstate) {
+  const int smsp = 4 * sm_count();
+  const long long warps = (long long)batch * ((dim + 15) / 16);
+  const int nblk = (seqlen + ssm::kBlk - 1) / ssm::kBlk;
+  int S = env_int("SSM_SSD_SPLIT", 0);
+  if (S <= 0) S = warps * 2 < smsp ? (int)((2LL * smsp + warps - 1) / warps) : 1;
+  S = S < 1 ? 1 : (S > nblk ? nblk : S);
+  FwdPlan p;
+  const int blk_per = (nblk + S - 1) / S;
+  p.chunk_len = blk_per * ssm::kBlk;
+  p.nchunk = (seqlen + p.chunk_len - 1) / p.chunk_len;
+  const size_t nch = (size_t)batch * dim;
+  p.ws_bytes = p.nchunk > 1 ? 2 * align_up((size_t)p.nchunk * nch * dstate * 4) +
+                                  align_up((size_t)p.nchunk * nch * 4)
+                            : 0;
+  return p;
+}
+
+__global__ void chain_kernel(const float* __restrict__ hend, const float* __restrict__ dsum,
+                             const float* __restrict__ A, int scalar_a,
+                             const float* __restrict__ h0, float* __restrict__ hin, int nseg,
+                             long long nch, int dim, int N);
+
 // Workspace that covers the plan of either kernel family (the family is chosen per call, from
 // the pointers' alignment too).
 size_t fwd_ws_bytes(int batch, int dim, int seqlen) {
@@ -390,7 +417,34 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
     a.scalar_a = 1;
     a.bc_groups = bc_groups;
     a.rows16 = vec ? 1 : 0;
-    cudaError_t e = ssm::launch_ssd_fwd(a, reinterpret_cast<cudaStream_t>(stream));
+    FwdPlan plan = plan_ssd(batch, dim, seqlen, dstate);
+    if (plan.nchunk > 1 && (!workspace || workspace_bytes < plan.ws_bytes ||
+                            (reinterpret_cast<uintptr_t>(workspace) & 255))) {
+      plan.nchunk = 1;  // not enough scratch: same result without the time split
+      plan.chunk_len = (int)nblk * ssm::kBlk;
+    }
+    a.chunk_len = plan.chunk_len;
+    a.nchunk = plan.nchunk;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (plan.nchunk > 1) {
+      TRY(check_ptr(workspace, plan.ws_bytes, 256, "workspace"));
+      const size_t nch = (size_t)batch * dim;
+      const size_t seg = align_up((size_t)plan.nchunk * nch * dstate * 4);
+      char* w = reinterpret_cast<char*>(workspace);
+      a.summ = reinterpret_cast<float*>(w);
+      float* hin = reinterpret_cast<float*>(w + seg);
+      a.dsum = reinterpret_cast<float*>(w + 2 * seg);
+      if ((e = ssm::launch_ssd_fwd(a, true, s)) != cudaSuccess)
+        return cuda_fail(e, "summary pass (chunked matrix form)");
+      const long long n = (long long)nch * dstate;
+      chain_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(a.summ, a.dsum, A, 1, h0, hin,
+                                                               plan.nchunk, (long long)nch, dim,
+                                                               dstate);
+      if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "carry (chunked matrix form)");
+      a.hin = hin;
+    }
+    e = ssm::launch_ssd_fwd(a, false, s);
     if (e != cudaSuccess) return cuda_fail(e, "forward pass (chunked matrix form)");
     return SSM_OK;
   }
@@ -520,7 +574,8 @@ __global__ void chain_kernel(const float* __restrict__ hend, const float* __rest
   float h = h0 ? h0[i] : 0.f;
   for (int r = 0; r < nseg; ++r) {
     hin[(long long)r * stride + i] = h;
-    h = fmaf(expf(An * dsum[(long long)r * nch + ch]), h, hend[(long long)r * stride + i]);
+    if (r + 1 < nseg)  // the last segment's map is not needed (nor, for a split, written)
+      h = fmaf(expf(An * dsum[(long long)r * nch + ch]), h, hend[(long long)r * stride + i]);
   }
 }
 
@@ -556,8 +611,11 @@ int ssm_scan_fwd(const void* u, const void* delta, const float* A, const void* B
 
 size_t ssm_scan_fwd_ex_workspace_size(int batch, int dim, int seqlen, int dstate, int bc_groups,
                                       int io_dtype, int flags) {
-  (void)flags;  // the time-split scratch does not depend on the variant
   if (bc_groups < 1) return 0;
+  if ((flags & SSM_SCALAR_A) && dstate > SSM_MAX_DSTATE) {  // the chunked matrix form's segments
+    if (check_dims(batch, dim, seqlen, dstate, io_dtype, SSM_MAX_DSTATE_SCALAR) != SSM_OK) return 0;
+    return plan_ssd(batch, dim, seqlen, dstate).ws_bytes;
+  }
   return ssm_scan_fwd_workspace_size(batch, dim, seqlen, dstate, io_dtype);
 }
 

@@ -35,9 +35,9 @@ struct FwdArgs {
   void* out;
   float* hL;            // may be NULL
   float* ckpt;          // may be NULL; [batch][dim][ceil(L/16)][N]
-  float* summ;          // summary pass: per-chunk end state from zero [S][channels][16]
+  float* summ;          // summary pass: per-chunk end state from zero [S][channels][16] (N: chunked form)
   float* dsum;          // summary pass: per-chunk sum of Δ          [S][channels]
-  const float* hin;     // output pass with S > 1: state entering each chunk [S][channels][16]
+  const float* hin;     // output pass with S > 1: state entering each chunk [S][channels][16] (N: chunked form)
   int batch, dim, L, N;
   int chunk_len;        // multiple of kBlk
   int nchunk;           // S
@@ -119,8 +119,11 @@ cudaError_t launch_fwd(const FwdArgs& a, int io, bool vec, int mode, int wpb, in
 cudaError_t launch_fwd_lane(const FwdArgs& a, int io, int mode, int kmufu, cudaStream_t s);
 // Scalar decay with N = 32, 64 or 128 (bf16 io): the chunked matrix form on the tensor cores
 // (ssm_ssd.cu).  B, C shared by each CTA's 64 channels (bc_groups == 1 or dim / bc_groups a
-// multiple of 64); a.rows16 selects 16-byte row accesses.
-cudaError_t launch_ssd_fwd(const FwdArgs& a, cudaStream_t s);
+// multiple of 64); a.rows16 selects 16-byte row accesses.  Time segments of a.chunk_len steps
+// (a multiple of 16), a.nchunk of them: summary = true runs segments 0 .. nchunk-2 from zero and
+// writes a.summ [seg][batch][dim][N] and a.dsum [seg][batch][dim]; the output launch runs every
+// segment from a.hin [seg][batch][dim][N] when given (else segment 0 from a.h0).
+cudaError_t launch_ssd_fwd(const FwdArgs& a, bool summary, cudaStream_t s);
 cudaError_t launch_fwd_carry(const FwdArgs& a, const float* summ, const float* dsum, float* hin,
                              cudaStream_t s);
 cudaError_t launch_bwd(const BwdArgs& a, int io, bool vec, cudaStream_t s);

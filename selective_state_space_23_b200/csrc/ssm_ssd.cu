@@ -38,6 +38,12 @@
 //     an exact sequential pass over its states held by the quad instead.
 // The products are small (K = 16 or N per 16-step chunk) and carry the sequence's dependency from
 // chunk to chunk, so they run as warp-level mma.sync.m16n8k16 rather than tcgen05 tiles.
+//
+// Time split (few channels, long sequences): segments of whole chunks run side by side.  A
+// summary launch (SUMMARY = true) runs every segment but the last from a zero state, keeping
+// only the state update (no G, Y1, Y2, gate or outputs), and writes its end state and ΣΔ; the
+// host chains those segment maps (h -> e^{A ΣΔ} h + h_end) into each segment's entering state;
+// the output launch then runs every segment from its entering state.
 #include <stdint.h>
 #include <stdlib.h>
 
@@ -107,7 +113,7 @@ __device__ __forceinline__ uint32_t ld_pair(const uint16_t* p, long long t, int 
   return lo | (hi << 16);
 }
 
-template <int N, int W>
+template <int N, int W, bool SUMMARY>
 __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__ FwdArgs a) {
   constexpr int kNT = N / 8;  // n8 tiles of the state
   extern __shared__ float4 smem_ssd[];
@@ -118,7 +124,11 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
   const int b = blockIdx.x / tiles_d;
   const int d0 = (blockIdx.x % tiles_d) * 16 * W;
   const int L = a.L;
-  const int nchunk = (L + kT - 1) / kT;
+  // this CTA's time segment: chunks [kc0, kc0 + nchunk) (the whole sequence without a split)
+  const int seg = blockIdx.y;
+  const int kc0 = seg * (a.chunk_len / kT);
+  const int nchunk = (min(L, (seg + 1) * a.chunk_len) - kc0 * kT + kT - 1) / kT;
+  const long long nch = (long long)a.batch * a.dim;
   const int gbc = d0 / (a.dim / a.bc_groups);
   const uint16_t* Bg = reinterpret_cast<const uint16_t*>(a.B) + ((long long)b * a.bc_groups + gbc) * N * (long long)L;
   const uint16_t* Cg = reinterpret_cast<const uint16_t*>(a.C) + ((long long)b * a.bc_groups + gbc) * N * (long long)L;
@@ -145,22 +155,25 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
 
   // the transposed state H'[d][n] in accumulator layout: Ht[nt][0..1] = channel g, states
   // 8 nt + 2 tg + {0, 1}; Ht[nt][2..3] = channel g + 8, same states
+  // entering state: zero for a summary; the chained state of the segment with a split; else h0
+  const float* hsrc = SUMMARY ? nullptr : (a.hin ? a.hin + (long long)seg * nch * N : a.h0);
   float Ht[kNT][4];
 #pragma unroll
   for (int nt = 0; nt < kNT; ++nt) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int c = e >> 1, n = 8 * nt + 2 * tg + (e & 1);
-      Ht[nt][e] = a.h0 ? a.h0[((long long)b * a.dim + dch[c]) * N + n] : 0.f;
+      Ht[nt][e] = hsrc ? hsrc[((long long)b * a.dim + dch[c]) * N + n] : 0.f;
     }
   }
+  float dacc[2] = {0.f, 0.f}, dcmp[2] = {0.f, 0.f};  // ΣΔ of the segment (summary, Kahan)
 
   // B/C tiles of chunk k into ring slot k % kStages: 16-byte cp.async pieces when rows allow
   // them, else element loads (ragged tail, unaligned rows) with zeros past L
   const auto issue = [&](int k) {
     if (k < nchunk) {
       SsdStage<N>& st = ring[k % kStages];
-      const int t0 = k * kT;
+      const int t0 = (kc0 + k) * kT;
       if (a.rows16 && t0 + kT <= L) {
         for (int p = tid; p < 4 * N; p += 32 * W) {
           const int which = p / (2 * N), rem = p % (2 * N), n = rem >> 1, h = rem & 1;
@@ -180,7 +193,7 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
   };
   const bool vec_rows = a.rows16 != 0;
   const auto load_in = [&](int k, ChunkIn& in) {
-    const int t0 = k * kT;
+    const int t0 = (kc0 + k) * kT;
     const bool vec = vec_rows && t0 + kT <= L;
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
@@ -206,7 +219,7 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
     const ChunkIn cur = nxt;
     if (k + 1 < nchunk) load_in(k + 1, nxt);
     const SsdStage<N>& st = ring[k % kStages];
-    const int t0 = k * kT;
+    const int t0 = (kc0 + k) * kT;
 
     // ---- per (channel, step): Δ, Δx, gate; index j: steps 2tg, 2tg+1, 2tg+8, 2tg+9
     float dl[2][4], xv[2][4], gt[2][4], uv[2][4];
@@ -223,7 +236,7 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
         dl[c][j] = live ? D : 0.f;
         uv[c][j] = live ? u : 0.f;
         xv[c][j] = dl[c][j] * uv[c][j];
-        if (zp) {
+        if (zp && !SUMMARY) {
           const float z = (j & 1) ? bf16_hi(wz) : bf16_lo(wz);
           gt[c][j] = z * sigmoid_fast(z);
         } else {
@@ -256,6 +269,12 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
       S[c][3] = lo_total + iq;
       Sm[c] = lo_total;  // S at step 7, the chunk's middle
       Se[c] = lo_total + hi_total;
+      if (SUMMARY) {  // Kahan-compensated ΣΔ over the segment's chunks
+        const float yk = Se[c] - dcmp[c];
+        const float tk = dacc[c] + yk;
+        dcmp[c] = (tk - dacc[c]) - yk;
+        dacc[c] = tk;
+      }
       float mrel = 0.f, mabs = 0.f;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -296,7 +315,7 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
     float G[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // s tiles 0..7, 8..15
     float Y2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // t tiles 0..7, 8..15
 #pragma unroll
-    for (int kk = 0; kk < N / 16; ++kk) {
+    for (int kk = 0; kk < (SUMMARY ? 0 : N / 16); ++kk) {
       uint32_t cf[4], bf[4];
       ldsm_x4_t(cf, blk(st.Cs, 16 * kk, lane));  // {t0-7|n lo, t8-15|n lo, t0-7|n hi, t8-15|n hi}
       ldsm_x4_t(bf, blk(st.Bs, 16 * kk, lane));  // {s0-7|n lo, s8-15|n lo, s0-7|n hi, s8-15|n hi}
@@ -325,7 +344,7 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
     // ---- Y1' = X1' mask(G)^T: G's accumulators (rows t, cols s) are the B fragments
     // (k = s, n = t) once masked to s <= t
     float Y1[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    {
+    if (!SUMMARY) {
       const int s0 = 2 * tg, r0 = g;
       const auto m = [](float v, int s, int t) { return s <= t ? v : 0.f; };
       // t tile 0: rows t = g; t tile 1: rows t = g + 8
@@ -373,6 +392,7 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
               yp = fmaf(cv, h, yp);
             }
           }
+          if (SUMMARY) continue;
           yp += __shfl_xor_sync(0xffffffffu, yp, 1);
           yp += __shfl_xor_sync(0xffffffffu, yp, 2);
           if (fb[c] && tg == to) yo[c][jo] = fmaf(Dd[c], uv[c][jo], yp) * gt[c][jo];
@@ -382,7 +402,7 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
     // ---- store the chunk's outputs (bf16 pairs of steps)
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
-      if (!act[c]) continue;
+      if (SUMMARY || !act[c]) continue;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         const long long t = t0 + 2 * tg + 8 * hh;
@@ -397,7 +417,21 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
     }
   }
   cp_wait<0>();
-  if (a.hL) {
+  if (SUMMARY) {
+#pragma unroll
+    for (int nt = 0; nt < kNT; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int c = e >> 1, n = 8 * nt + 2 * tg + (e & 1);
+        if (act[c]) a.summ[((long long)seg * nch + (long long)b * a.dim + dch[c]) * N + n] = Ht[nt][e];
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+      if (act[c] && tg == 0) a.dsum[(long long)seg * nch + (long long)b * a.dim + dch[c]] = dacc[c];
+    return;
+  }
+  if (a.hL && (seg + 1) * a.chunk_len >= L) {
 #pragma unroll
     for (int nt = 0; nt < kNT; ++nt) {
 #pragma unroll
@@ -410,10 +444,12 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
 }
 
 template <int N, int W>
-cudaError_t launch_n(const FwdArgs& a, cudaStream_t s) {
-  const unsigned grid = (unsigned)((long long)a.batch * ((a.dim + 16 * W - 1) / (16 * W)));
+cudaError_t launch_n(const FwdArgs& a, bool summary, cudaStream_t s) {
+  const int segs = summary ? a.nchunk - 1 : a.nchunk;  // the last segment's summary is unused
+  if (segs <= 0) return cudaSuccess;
+  const dim3 grid((unsigned)((long long)a.batch * ((a.dim + 16 * W - 1) / (16 * W))), (unsigned)segs);
   const size_t smem = kStages * sizeof(SsdStage<N>);
-  auto k = ssd_fwd_kernel<N, W>;
+  auto k = summary ? ssd_fwd_kernel<N, W, true> : ssd_fwd_kernel<N, W, false>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   k<<<grid, 32 * W, smem, s>>>(a);
@@ -421,7 +457,7 @@ cudaError_t launch_n(const FwdArgs& a, cudaStream_t s) {
 }
 
 template <int N>
-cudaError_t launch_w(const FwdArgs& a, cudaStream_t s) {
+cudaError_t launch_w(const FwdArgs& a, bool summary, cudaStream_t s) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -431,16 +467,16 @@ cudaError_t launch_w(const FwdArgs& a, cudaStream_t s) {
   bool two = ctas4 < 2LL * sms;
   const char* env = getenv("SSM_SSD_WPB");
   if (env && (atoi(env) == 2 || atoi(env) == 4)) two = atoi(env) == 2;
-  return two ? launch_n<N, 2>(a, s) : launch_n<N, 4>(a, s);
+  return two ? launch_n<N, 2>(a, summary, s) : launch_n<N, 4>(a, summary, s);
 }
 
 }  // namespace
 
-cudaError_t launch_ssd_fwd(const FwdArgs& a, cudaStream_t s) {
+cudaError_t launch_ssd_fwd(const FwdArgs& a, bool summary, cudaStream_t s) {
   switch (a.N) {
-    case 32: return launch_w<32>(a, s);
-    case 64: return launch_w<64>(a, s);
-    case 128: return launch_w<128>(a, s);
+    case 32: return launch_w<32>(a, summary, s);
+    case 64: return launch_w<64>(a, summary, s);
+    case 128: return launch_w<128>(a, summary, s);
     default: return cudaErrorInvalidValue;
   }
 }

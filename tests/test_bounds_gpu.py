@@ -149,13 +149,14 @@ FWD_CASES = {
     "per_channel_bc": ({}, 2, 24, 120, 16, torch.bfloat16, 24, 0),
     "scalar_decay": ({}, 2, 96, 200, 16, torch.bfloat16, 1, 1),
     "chunked_n64": ({}, 2, 96, 200, 64, torch.bfloat16, 1, 1),
+    "chunked_n128_split": ({"SSM_SSD_SPLIT": "3"}, 1, 80, 333, 128, torch.bfloat16, 1, 1),
 }
 
 
 @pytest.mark.parametrize("case", sorted(FWD_CASES))
 def test_forward_stays_inside_its_tensors(monkeypatch, case):
     env, batch, dim, L, N, io, G, flags = FWD_CASES[case]
-    for k in ("SSM_FWD_KERNEL", "SSM_FWD_WPB", "SSM_FWD_SPLIT"):
+    for k in ("SSM_FWD_KERNEL", "SSM_FWD_WPB", "SSM_FWD_SPLIT", "SSM_SSD_SPLIT"):
         monkeypatch.delenv(k, raising=False)
     for k, v in env.items():
         monkeypatch.setenv(k, v)

@@ -114,3 +114,37 @@ def test_unsupported_requests_are_refused():
     x = {k: (v.float() if v.dtype == torch.bfloat16 else v) for k, v in x.items()}
     with pytest.raises(RuntimeError):
         gpu(x)  # f32 io
+
+
+@pytest.mark.parametrize("split", ["2", "3", "7"])
+@pytest.mark.parametrize("N", [64, 128])
+def test_time_split_matches_oracle(monkeypatch, split, N):
+    """Segments of whole chunks run side by side: summaries from zero, the chain of segment maps,
+    then every segment from its entering state (333 steps: a ragged last chunk)."""
+    monkeypatch.setenv("SSM_SSD_SPLIT", split)
+    x = inputs(2, 128, 333, N, seed=71)
+    out, hL = gpu(x)
+    r = ref(x)
+    assert_close(out, r["out"], torch.bfloat16, "out")
+    assert_close(hL, r["hL"], torch.bfloat16, "hL")
+
+
+def test_time_split_with_range_fallback(monkeypatch):
+    monkeypatch.setenv("SSM_SSD_SPLIT", "4")
+    x = inputs(1, 64, 256, 64, seed=72)
+    v = np.random.default_rng(5).uniform(-30, 30, size=x["delta"].shape).astype(np.float32)
+    x["delta"] = torch.from_numpy(v).to(torch.bfloat16)
+    x["dt_bias"] = torch.zeros_like(x["dt_bias"])
+    out, hL = gpu(x)
+    r = ref(x)
+    assert_close(out, r["out"], torch.bfloat16, "out")
+    assert_close(hL, r["hL"], torch.bfloat16, "hL")
+
+
+def test_natural_time_split_long_sequence():
+    """64 channels over 8192 steps: 4 warps of channels, so the time axis is split by itself."""
+    x = inputs(1, 64, 8192, 64, seed=73)
+    out, hL = gpu(x)
+    r = ref(x)
+    assert_close(out, r["out"], torch.bfloat16, "out")
+    assert_close(hL, r["hL"], torch.bfloat16, "hL")
