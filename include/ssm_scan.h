@@ -156,7 +156,8 @@ SSM_API int ssm_scan_bwd(const void* u, const void* delta, const float* A, const
  * The backward needs ssm_scan_bwd_scalar_a_workspace_size() bytes of workspace (256-byte
  * aligned): A broadcast to [dim][dstate] and the per-state dA, followed by the workspace of
  * ssm_scan_bwd for the same shape.  Checkpoints of ssm_scan_fwd_scalar_a feed the backward.
- * dstate may be up to SSM_MAX_DSTATE_SCALAR in the forward scan: above 16 it runs in the chunked
+ * dstate may be up to SSM_MAX_DSTATE_SCALAR in the forward scan: above 16 (and at 16 for bf16
+ * calls without checkpoints, the default layout and no other flag) it runs in the chunked
  * matrix form (per 16-step chunk and 64-channel tile, the products C B^T, masked with the decay
  * factors, times the step-scaled inputs, plus C times the entering state: the structured-matrix
  * view of the scan in the Mamba-2 notes of the same page) on the tensor cores.  That form takes

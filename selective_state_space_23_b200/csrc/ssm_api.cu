@@ -399,9 +399,16 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
                    aligned16(delta) && aligned16(z) && aligned16(out) && aligned16(B) &&
                    aligned16(C);
   // scalar decay with N > 16: the chunked matrix form on the tensor cores (bf16, N = 32, 64 or
-  // 128, forward direction, [batch][dim][L] rows, B/C shared by each 64-channel tile)
-  if (dstate > SSM_MAX_DSTATE) {
-    if (io_dtype != SSM_BF16 || (dstate != 32 && dstate != 64 && dstate != 128) || zoh ||
+  // 128, forward direction, [batch][dim][L] rows, B/C shared by each 64-channel tile).  With
+  // N = 16 the same form serves the requests it takes (no checkpoints); SSM_SCALAR_FORM=state
+  // keeps those on the per-state kernel.
+  const char* sform = getenv("SSM_SCALAR_FORM");
+  const bool chunked16 = scalar_a && dstate == ssm::kNS && io_dtype == SSM_BF16 && !ckpt &&
+                         !(flags & (SSM_ZOH | SSM_REVERSE | SSM_CHANNELS_LAST)) &&
+                         (bc_groups == 1 || (dim % bc_groups == 0 && (dim / bc_groups) % 64 == 0)) &&
+                         !(sform && strcmp(sform, "state") == 0);
+  if (dstate > SSM_MAX_DSTATE || chunked16) {
+    if (io_dtype != SSM_BF16 || (dstate != 16 && dstate != 32 && dstate != 64 && dstate != 128) || zoh ||
         reverse || channels_last || ckpt ||
         !(bc_groups == 1 || (dim % bc_groups == 0 && (dim / bc_groups) % 64 == 0)))
       return fail(SSM_EUNSUPPORTED,

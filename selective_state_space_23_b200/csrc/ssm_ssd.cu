@@ -1,4 +1,4 @@
-// Scalar-decay selective scan for large state sizes (N = 32, 64, 128) in its chunked matrix form,
+// Scalar-decay selective scan (N = 16, 32, 64, 128) in its chunked matrix form,
 // on the tensor cores, sm_100a, bf16 io.
 //
 // With one decay rate A_d per channel (the Mamba-2 restriction noted on the "2024 Reading List:
@@ -474,6 +474,7 @@ cudaError_t launch_w(const FwdArgs& a, bool summary, cudaStream_t s) {
 
 cudaError_t launch_ssd_fwd(const FwdArgs& a, bool summary, cudaStream_t s) {
   switch (a.N) {
+    case 16: return launch_w<16>(a, summary, s);
     case 32: return launch_w<32>(a, summary, s);
     case 64: return launch_w<64>(a, summary, s);
     case 128: return launch_w<128>(a, summary, s);
