@@ -325,7 +325,15 @@ def _ssd(dev, rnd, prm, timeit, g):
         res[f"N{N}"] = {"fwd_ms": ms, "tokens_per_s": b * L / (ms * 1e-3),
                         "hbm_gbs": (4 * b * d * L * 2 + 2 * b * N * L * 2) / (ms * 1e-3) / 1e9,
                         "mma_tflops": flops / (ms * 1e-3) / 1e12}
-    del u, de, z, o, B, C
+    # the backward with 64 states (the sum of four 16-state backwards)
+    B, C = rnd((b, 64, L)), rnd((b, 64, L))
+    dout = rnd((b, d, L))
+    wsb = torch.empty(ssm._abi.lib().ssm_scan_bwd_ex_workspace_size(b, d, L, 64, 1, 1, 0, 1),
+                      dtype=torch.uint8, device=dev)
+    ms = timeit(lambda: ssm.ssm_scan_bwd_scalar_a(u, de, A1, B, C, dout, D=D, z=z, dt_bias=bias,
+                                                  workspace=wsb), 3)
+    res["bwd_N64_ms"] = ms
+    del u, de, z, o, B, C, dout, wsb
     # the long sequence (1 x 256 x 2^20) with 64 states: 16 warps of channels, so the time axis
     # is split into segments (summary, chain, output launches)
     b, d, L, N = 1, 256, 1 << 20, 64

@@ -882,6 +882,9 @@ int ssm_scan_bwd(const void* u, const void* delta, const float* A, const void* B
 size_t ssm_scan_bwd_ex_workspace_size(int batch, int dim, int seqlen, int dstate, int bc_groups,
                                       int io_dtype, int have_ckpt, int flags) {
   if (flags & ~(SSM_SCALAR_A | SSM_REVERSE | SSM_ZOH | SSM_CHANNELS_LAST)) return 0;
+  if ((flags & SSM_SCALAR_A) && dstate > SSM_MAX_DSTATE)  // the sum over 16-state slices
+    return have_ckpt ? 0 : ssm::scan_bwd_slices_workspace(batch, dim, seqlen, dstate, bc_groups,
+                                                          io_dtype, flags);
   if (check_dims(batch, dim, seqlen, dstate, io_dtype) != SSM_OK) return 0;
   if (check_groups(dim, bc_groups) != SSM_OK) return 0;
   const size_t base = layout_bwd(batch, dim, seqlen, dstate, have_ckpt != 0, bc_groups, io_dtype,
@@ -902,6 +905,14 @@ int ssm_scan_bwd_ex(const void* u, const void* delta, const float* A, const void
     return fail(SSM_EINVAL, "unknown flags 0x%x", flags);
   const bool reverse = (flags & SSM_REVERSE) != 0, zoh = (flags & SSM_ZOH) != 0;
   const bool cl = (flags & SSM_CHANNELS_LAST) != 0;
+  if ((flags & SSM_SCALAR_A) && dstate > SSM_MAX_DSTATE) {  // the sum over 16-state slices
+    TRY(check_dims(batch, dim, seqlen, dstate, io_dtype, SSM_MAX_DSTATE_SCALAR));
+    TRY(check_groups(dim, bc_groups));
+    return ssm::scan_bwd_slices(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL,
+                                ckpt, du, ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, workspace,
+                                workspace_bytes, batch, dim, seqlen, dstate, bc_groups, io_dtype,
+                                flags, stream);
+  }
   TRY(check_dims(batch, dim, seqlen, dstate, io_dtype));
   if (!(flags & SSM_SCALAR_A))
     return scan_bwd_core(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL, ckpt,

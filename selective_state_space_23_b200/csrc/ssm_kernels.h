@@ -158,6 +158,21 @@ int decode_wait_timeouts(unsigned int* out);
 
 // Sets the message returned by ssm_last_error() on the calling thread.
 void set_last_error(const char* msg);
+// Copies the 4-index view (sizes n, element strides ss) at src into the view with strides ds at
+// dst, es = 2 or 4 bytes per element (ssm_strided.cu).
+cudaError_t copy_view(const void* src, const long long* n, const long long* ss, void* dst,
+                      const long long* ds, size_t es, cudaStream_t s);
+// Backward of the scalar-decay scan for dstate = 16 k (k = 2, 4, 8) as the sum of k 16-state
+// backwards (ssm_slices.cu); arguments as ssm_scan_bwd_ex.
+size_t scan_bwd_slices_workspace(int batch, int dim, int seqlen, int dstate, int bc_groups,
+                                 int io_dtype, int flags);
+int scan_bwd_slices(const void* u, const void* delta, const float* A, const void* B,
+                    const void* C, const float* D, const void* z, const float* dt_bias,
+                    int delta_softplus, const float* h0, const void* dout, const float* dhL,
+                    const float* ckpt, void* du, void* ddelta, float* dA, void* dB, void* dC,
+                    float* dD, void* dz, float* ddt_bias, float* dh0, void* workspace,
+                    size_t workspace_bytes, int batch, int dim, int seqlen, int dstate,
+                    int bc_groups, int io_dtype, int flags, void* stream);
 // The entry points' pointer check (device-accessible on the current device, allocation holds
 // `bytes` bytes, `align`-byte aligned); returns an ssm_status and sets the error message.
 int check_device_ptr(const void* p, size_t bytes, size_t align, const char* name);

@@ -416,3 +416,18 @@ int ssm_state_update_strided(float* state, const void* x, const void* dt, const 
 }
 
 }  // extern "C"
+
+namespace ssm {
+// The restride copy for other translation units: the 4-index view (sizes n, element strides ss)
+// at src into the view with strides ds at dst (es = 2 or 4 bytes per element), on stream s.
+cudaError_t copy_view(const void* src, const long long* n, const long long* ss, void* dst,
+                      const long long* ds, size_t es, cudaStream_t s) {
+  View4 sv, dv;
+  for (int k = 0; k < 4; ++k) {
+    sv.n[k] = dv.n[k] = n[k];
+    sv.s[k] = ss[k];
+    dv.s[k] = ds[k];
+  }
+  return restride(src, sv, dst, dv, es, s);
+}
+}  // namespace ssm

@@ -1,0 +1,89 @@
+"""Backward of the scalar-decay scan with N = 32, 64, 128 (the Mamba-2 state sizes of the "2024
+Reading List: Neural Network" page).  The states of a scalar-decay scan do not interact, so the
+library runs it as a sum over 16-state slices; every gradient is compared with the fp64
+oracle's chain-rule gradients (A broadcast over the states, dA summed over them), with dhL, h0,
+the ZOH input term, the reverse scan and grouped B/C."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import selective_state_space_23_b200 as ssm
+from selective_state_space_23_b200.inputs import make_inputs, workload
+
+from _parity import assert_close, f64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+GRADS = ("du", "ddelta", "dz", "dB", "dC", "dA", "dD", "ddt_bias", "dh0")
+
+
+def inputs(batch, dim, L, N, io, seed, groups=1, gate=True):
+    w = workload("mamba370m_fwd", batch=batch, dim=dim, seqlen=L, dstate=N, io_dtype=io)
+    x = make_inputs(w, seed=seed, with_dout=True, with_h0=True, scalar_a=True, gate=gate)
+    if groups > 1:
+        wg = workload("mamba370m_fwd", batch=batch * groups, dim=1, seqlen=L, dstate=N, io_dtype=io)
+        xg = make_inputs(wg, seed=seed + 1)
+        x["B"] = xg["B"].reshape(batch, groups, N, L).contiguous()
+        x["C"] = xg["C"].reshape(batch, groups, N, L).contiguous()
+    return x
+
+
+def run(x, dhL, **kw):
+    xd = {k: v.to(DEV) for k, v in x.items()}
+    return ssm.ssm_scan_bwd_scalar_a(xd["u"], xd["delta"], xd["A"], xd["B"], xd["C"], xd["dout"],
+                                     D=xd.get("D"), z=xd.get("z"), dt_bias=xd.get("dt_bias"),
+                                     h0=xd["h0"], dhL=None if dhL is None else dhL.to(DEV), **kw)
+
+
+def ref(x, dhL, **kw):
+    c = lambda k: None if x.get(k) is None else f64(x[k])
+    N = x["B"].shape[-2]
+    A = np.repeat(c("A")[:, None], N, axis=1)
+    g = oracle.scan_bwd(c("u"), c("delta"), A, c("B"), c("C"), c("dout"), D=c("D"), z=c("z"),
+                        dt_bias=c("dt_bias"), h0=c("h0"), dhL=None if dhL is None else f64(dhL),
+                        **kw)
+    g["dA"] = g["dA"].sum(1)  # chain rule through A[d, n] = A_d
+    return g
+
+
+@pytest.mark.parametrize("io", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("N", [32, 64, 128])
+def test_gradients_match_oracle(io, N):
+    x = inputs(2, 64, 160, N, io, seed=101)
+    dhL = torch.randn((2, 64, N), generator=torch.Generator().manual_seed(7))
+    g = run(x, dhL)
+    assert g["dA"].shape == (64,) and g["dB"].shape == (2, N, 160)
+    r = ref(x, dhL)
+    for k in GRADS:
+        assert_close(g[k], r[k], io, k)
+
+
+@pytest.mark.parametrize("variant", ["reverse_zoh", "groups", "no_gate"])
+def test_variants(variant):
+    kw = dict(reverse=variant == "reverse_zoh", zoh=variant == "reverse_zoh")
+    x = inputs(2, 128, 96, 64, torch.bfloat16, seed=102, groups=2 if variant == "groups" else 1,
+               gate=variant != "no_gate")
+    if variant == "no_gate":
+        del x["D"]
+    g = run(x, None, **kw)
+    r = ref(x, None, **kw)
+    for k in GRADS:
+        if r.get(k) is None or g.get(k) is None:
+            continue
+        assert_close(g[k], r[k], torch.bfloat16, k)
+
+
+def test_forward_then_backward_shapes_agree():
+    """The N = 64 forward (chunked matrix form) and backward (sum of slices) take the same
+    tensors; checkpoints are refused for N > 16 (the backward recomputes its states)."""
+    x = inputs(1, 64, 64, 64, torch.bfloat16, seed=103)
+    xd = {k: v.to(DEV) for k, v in x.items()}
+    out = ssm.ssm_scan_fwd_scalar_a(xd["u"], xd["delta"], xd["A"], xd["B"], xd["C"], D=xd["D"],
+                                    z=xd["z"], dt_bias=xd["dt_bias"], h0=xd["h0"])
+    assert out.shape == (1, 64, 64)
+    fake_ck = torch.zeros((1, 64, 4, 64), device=DEV)
+    with pytest.raises(RuntimeError):
+        ssm.ssm_scan_bwd_scalar_a(xd["u"], xd["delta"], xd["A"], xd["B"], xd["C"], xd["dout"],
+                                  D=xd["D"], z=xd["z"], dt_bias=xd["dt_bias"], h0=xd["h0"],
+                                  ckpt=fake_ck)
