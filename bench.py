@@ -78,10 +78,17 @@ KERNEL_SOURCES = ("ssm_fwd_impl.cuh", "ssm_fwd_bf16.cu", "ssm_device.cuh", "ssm_
 
 
 def kernel_source_hash() -> str:
+    """Hash of the forward kernel's code: its sources, and of the shared header only the argument
+    struct the kernel reads (comments dropped), so that unrelated declarations do not count."""
+    import re
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, "selective_state_space_23_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "selective_state_space_23_b200", "csrc", f), "r") as fh:
+            text = fh.read()
+        if f == "ssm_kernels.h":
+            m = re.search(r"struct FwdArgs \{.*?\n\};", text, re.S)
+            text = re.sub(r"//[^\n]*", "", m.group(0)) if m else text
+        h.update(text.encode())
     return h.hexdigest()[:16]
 
 
