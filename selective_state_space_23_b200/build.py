@@ -15,8 +15,8 @@ BUILD_DIR = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libssm_b200.so")
 SOURCES = ["ssm_api.cu", "ssm_fwd.cu", "ssm_fwd_bf16.cu", "ssm_fwd_f32.cu", "ssm_fwd_rev_bf16.cu",
            "ssm_fwd_rev_f32.cu", "ssm_fwd_lane_bf16.cu", "ssm_fwd_lane_f32.cu", "ssm_bwd.cu", "ssm_bwd_hist.cu", "ssm_pcbc.cu", "ssm_ssd.cu", "ssm_decode.cu", "ssm_noalloc.cu", "ssm_host.cu",
-           "ssm_strided.cu", "ssm_slices.cu"]
-HEADERS = ["ssm_device.cuh", "ssm_kernels.h", "ssm_rows.cuh", "ssm_fwd_impl.cuh", "ssm_fwd_lane.cuh"]
+           "ssm_strided.cu", "ssm_slices.cu", "ssm_ssd_bwd.cu"]
+HEADERS = ["ssm_device.cuh", "ssm_kernels.h", "ssm_rows.cuh", "ssm_fwd_impl.cuh", "ssm_fwd_lane.cuh", "ssm_mma.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",

@@ -442,7 +442,7 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
       a.summ = reinterpret_cast<float*>(w);
       float* hin = reinterpret_cast<float*>(w + seg);
       a.dsum = reinterpret_cast<float*>(w + 2 * seg);
-      if ((e = ssm::launch_ssd_fwd(a, true, s)) != cudaSuccess)
+      if ((e = ssm::launch_ssd_fwd(a, ssm::kSsdSummary, s)) != cudaSuccess)
         return cuda_fail(e, "summary pass (chunked matrix form)");
       const long long n = (long long)nch * dstate;
       chain_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(a.summ, a.dsum, A, 1, h0, hin,
@@ -451,7 +451,7 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
       if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "carry (chunked matrix form)");
       a.hin = hin;
     }
-    e = ssm::launch_ssd_fwd(a, false, s);
+    e = ssm::launch_ssd_fwd(a, ssm::kSsdOut, s);
     if (e != cudaSuccess) return cuda_fail(e, "forward pass (chunked matrix form)");
     return SSM_OK;
   }
@@ -865,6 +865,142 @@ int scan_bwd_core(const void* u, const void* delta, const float* A, const void* 
 
 }  // namespace
 
+namespace {
+
+// The chunked-form backward of scalar decay (bf16, N = 16..128, forward direction, default
+// layout, B/C shared by whole 64-channel tiles, no checkpoints given): the forward's checkpoint
+// pass (with its own time split), the backward kernel, and the finishing sums.
+bool chunked_bwd_ok(int dim, int dstate, int bc_groups, int io_dtype, int flags) {
+  const char* v = getenv("SSM_SCALAR_BWD");
+  if (v && strcmp(v, "slices") == 0) return false;
+  return io_dtype == SSM_BF16 && flags == SSM_SCALAR_A &&
+         (dstate == 32 || dstate == 64 || dstate == 128) &&
+         (bc_groups == 1 || (bc_groups < dim && dim % bc_groups == 0 && (dim / bc_groups) % 64 == 0));
+}
+
+struct ChunkedBwdLayout {
+  size_t ck, pbc, padt, fwd, total;
+};
+
+ChunkedBwdLayout chunked_bwd_layout(int batch, int dim, int seqlen, int dstate) {
+  ChunkedBwdLayout l;
+  const size_t nck = (seqlen + ssm::kBlk - 1) / ssm::kBlk;
+  l.ck = align_up((size_t)batch * dim * (nck + 1) * dstate * 4);
+  l.pbc = align_up((size_t)ssm::ssd_bwd_ctas_per_row(dim) * batch * 2 * dstate * seqlen * 4);
+  l.padt = align_up((size_t)batch * dim * 3 * 4);
+  l.fwd = plan_ssd(batch, dim, seqlen, dstate).ws_bytes;
+  l.total = l.ck + l.pbc + l.padt + l.fwd;
+  return l;
+}
+
+int scan_bwd_chunked(const void* u, const void* delta, const float* A, const void* B,
+                     const void* C, const float* D, const void* z, const float* dt_bias,
+                     int delta_softplus, const float* h0, const void* dout, const float* dhL,
+                     void* du, void* ddelta, float* dA, void* dB, void* dC, float* dD, void* dz,
+                     float* ddt_bias, float* dh0, void* workspace, size_t workspace_bytes,
+                     int batch, int dim, int seqlen, int dstate, int bc_groups, void* stream) {
+  const size_t es = 2;
+  const size_t nx = (size_t)batch * dim * seqlen * es;
+  const size_t nbc = (size_t)batch * bc_groups * dstate * seqlen * es;
+  const size_t nst = (size_t)batch * dim * dstate * 4;
+  TRY(check_ptr(u, nx, es, "u"));
+  TRY(check_ptr(delta, nx, es, "delta"));
+  TRY(check_ptr(A, (size_t)dim * 4, 4, "A"));
+  TRY(check_ptr(B, nbc, es, "B"));
+  TRY(check_ptr(C, nbc, es, "C"));
+  TRY(check_ptr(dout, nx, es, "dout"));
+  TRY(check_opt(D, (size_t)dim * 4, 4, "D"));
+  TRY(check_opt(z, nx, es, "z"));
+  TRY(check_opt(dt_bias, (size_t)dim * 4, 4, "dt_bias"));
+  TRY(check_opt(h0, nst, 4, "h0"));
+  TRY(check_opt(dhL, nst, 4, "dhL"));
+  TRY(check_opt(du, nx, es, "du"));
+  TRY(check_opt(ddelta, nx, es, "ddelta"));
+  TRY(check_opt(dz, nx, es, "dz"));
+  TRY(check_opt(dB, nbc, es, "dB"));
+  TRY(check_opt(dC, nbc, es, "dC"));
+  TRY(check_opt(dA, (size_t)dim * 4, 4, "dA"));
+  TRY(check_opt(dD, (size_t)dim * 4, 4, "dD"));
+  TRY(check_opt(ddt_bias, (size_t)dim * 4, 4, "ddt_bias"));
+  TRY(check_opt(dh0, nst, 4, "dh0"));
+  if (!du && !ddelta && !dA && !dB && !dC && !dD && !dz && !ddt_bias && !dh0)
+    return fail(SSM_EINVAL, "no gradient output requested");
+  if (dz && !z) return fail(SSM_EINVAL, "dz requested but z is NULL");
+  const ChunkedBwdLayout l = chunked_bwd_layout(batch, dim, seqlen, dstate);
+  if (!workspace || workspace_bytes < l.total)
+    return fail(SSM_EWORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes, l.total);
+  if (reinterpret_cast<uintptr_t>(workspace) & 255)
+    return fail(SSM_EINVAL, "workspace is not 256-byte aligned");
+  TRY(check_ptr(workspace, l.total, 256, "workspace"));
+  char* w = reinterpret_cast<char*>(workspace);
+  float* ck = reinterpret_cast<float*>(w);
+  float* pbc = reinterpret_cast<float*>(w + l.ck);
+  float* padt = reinterpret_cast<float*>(w + l.ck + l.pbc);
+  char* fws = w + l.ck + l.pbc + l.padt;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool vec = (seqlen * es) % 16 == 0 && aligned16(u) && aligned16(delta) && aligned16(z) &&
+                   aligned16(B) && aligned16(C);
+  // the state entering every chunk, from the forward in checkpoint mode
+  ssm::FwdArgs a;
+  memset(&a, 0, sizeof(a));
+  a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
+  a.A = A; a.dt_bias = dt_bias; a.h0 = h0;
+  a.ckpt = ck;  // [batch][dim][chunks + 1][N]: the state entering every chunk
+  a.batch = batch; a.dim = dim; a.L = seqlen; a.N = dstate;
+  a.softplus = delta_softplus ? 1 : 0;
+  a.scalar_a = 1;
+  a.bc_groups = bc_groups;
+  a.rows16 = vec ? 1 : 0;
+  const FwdPlan plan = plan_ssd(batch, dim, seqlen, dstate);
+  a.chunk_len = plan.chunk_len;
+  a.nchunk = plan.nchunk;
+  cudaError_t e;
+  if (plan.nchunk > 1) {
+    const size_t nch = (size_t)batch * dim;
+    const size_t seg = align_up((size_t)plan.nchunk * nch * dstate * 4);
+    a.summ = reinterpret_cast<float*>(fws);
+    float* hin = reinterpret_cast<float*>(fws + seg);
+    a.dsum = reinterpret_cast<float*>(fws + 2 * seg);
+    if ((e = ssm::launch_ssd_fwd(a, ssm::kSsdSummary, s)) != cudaSuccess)
+      return cuda_fail(e, "backward: summary pass (chunked matrix form)");
+    const long long n = (long long)nch * dstate;
+    chain_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(a.summ, a.dsum, A, 1, h0, hin,
+                                                             plan.nchunk, (long long)nch, dim,
+                                                             dstate);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward: carry");
+    a.hin = hin;
+  }
+  if ((e = ssm::launch_ssd_fwd(a, ssm::kSsdCkpt, s)) != cudaSuccess)
+    return cuda_fail(e, "backward: checkpoint pass (chunked matrix form)");
+  ssm::SsdBwdArgs b;
+  memset(&b, 0, sizeof(b));
+  b.u = reinterpret_cast<const uint16_t*>(u);
+  b.delta = reinterpret_cast<const uint16_t*>(delta);
+  b.z = reinterpret_cast<const uint16_t*>(z);
+  b.B = reinterpret_cast<const uint16_t*>(B);
+  b.C = reinterpret_cast<const uint16_t*>(C);
+  b.dout = reinterpret_cast<const uint16_t*>(dout);
+  b.A = A; b.D = D; b.dt_bias = dt_bias; b.dhL = dhL;
+  b.ck = ck;
+  b.du = reinterpret_cast<uint16_t*>(du);
+  b.ddelta = reinterpret_cast<uint16_t*>(ddelta);
+  b.dz = reinterpret_cast<uint16_t*>(dz);
+  b.dh0 = dh0;
+  b.part_bc = pbc;
+  b.part_adt = padt;
+  b.batch = batch; b.dim = dim; b.L = seqlen; b.N = dstate; b.bc_groups = bc_groups;
+  b.softplus = delta_softplus ? 1 : 0;
+  b.rows16 = vec ? 1 : 0;
+  b.need_bc = (dB || dC) ? 1 : 0;
+  if ((e = ssm::launch_ssd_bwd(b, s)) != cudaSuccess)
+    return cuda_fail(e, "backward pass (chunked matrix form)");
+  if ((e = ssm::launch_ssd_bwd_finish(b, dB, dC, dA, dD, ddt_bias, s)) != cudaSuccess)
+    return cuda_fail(e, "backward reduction (chunked matrix form)");
+  return SSM_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 int ssm_scan_bwd(const void* u, const void* delta, const float* A, const void* B, const void* C,
@@ -882,9 +1018,12 @@ int ssm_scan_bwd(const void* u, const void* delta, const float* A, const void* B
 size_t ssm_scan_bwd_ex_workspace_size(int batch, int dim, int seqlen, int dstate, int bc_groups,
                                       int io_dtype, int have_ckpt, int flags) {
   if (flags & ~(SSM_SCALAR_A | SSM_REVERSE | SSM_ZOH | SSM_CHANNELS_LAST)) return 0;
-  if ((flags & SSM_SCALAR_A) && dstate > SSM_MAX_DSTATE)  // the sum over 16-state slices
-    return have_ckpt ? 0 : ssm::scan_bwd_slices_workspace(batch, dim, seqlen, dstate, bc_groups,
-                                                          io_dtype, flags);
+  if ((flags & SSM_SCALAR_A) && dstate > SSM_MAX_DSTATE) {  // chunked form, or slices
+    if (have_ckpt) return 0;
+    if (chunked_bwd_ok(dim, dstate, bc_groups, io_dtype, flags))
+      return chunked_bwd_layout(batch, dim, seqlen, dstate).total;
+    return ssm::scan_bwd_slices_workspace(batch, dim, seqlen, dstate, bc_groups, io_dtype, flags);
+  }
   if (check_dims(batch, dim, seqlen, dstate, io_dtype) != SSM_OK) return 0;
   if (check_groups(dim, bc_groups) != SSM_OK) return 0;
   const size_t base = layout_bwd(batch, dim, seqlen, dstate, have_ckpt != 0, bc_groups, io_dtype,
@@ -905,9 +1044,13 @@ int ssm_scan_bwd_ex(const void* u, const void* delta, const float* A, const void
     return fail(SSM_EINVAL, "unknown flags 0x%x", flags);
   const bool reverse = (flags & SSM_REVERSE) != 0, zoh = (flags & SSM_ZOH) != 0;
   const bool cl = (flags & SSM_CHANNELS_LAST) != 0;
-  if ((flags & SSM_SCALAR_A) && dstate > SSM_MAX_DSTATE) {  // the sum over 16-state slices
+  if ((flags & SSM_SCALAR_A) && dstate > SSM_MAX_DSTATE) {  // chunked form, or slices
     TRY(check_dims(batch, dim, seqlen, dstate, io_dtype, SSM_MAX_DSTATE_SCALAR));
     TRY(check_groups(dim, bc_groups));
+    if (!ckpt && chunked_bwd_ok(dim, dstate, bc_groups, io_dtype, flags))
+      return scan_bwd_chunked(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL,
+                              du, ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, workspace,
+                              workspace_bytes, batch, dim, seqlen, dstate, bc_groups, stream);
     return ssm::scan_bwd_slices(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL,
                                 ckpt, du, ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, workspace,
                                 workspace_bytes, batch, dim, seqlen, dstate, bc_groups, io_dtype,

@@ -120,10 +120,41 @@ cudaError_t launch_fwd_lane(const FwdArgs& a, int io, int mode, int kmufu, cudaS
 // Scalar decay with N = 32, 64 or 128 (bf16 io): the chunked matrix form on the tensor cores
 // (ssm_ssd.cu).  B, C shared by each CTA's 64 channels (bc_groups == 1 or dim / bc_groups a
 // multiple of 64); a.rows16 selects 16-byte row accesses.  Time segments of a.chunk_len steps
-// (a multiple of 16), a.nchunk of them: summary = true runs segments 0 .. nchunk-2 from zero and
+// (a multiple of 16), a.nchunk of them: the summary mode runs segments 0 .. nchunk-2 from zero and
 // writes a.summ [seg][batch][dim][N] and a.dsum [seg][batch][dim]; the output launch runs every
 // segment from a.hin [seg][batch][dim][N] when given (else segment 0 from a.h0).
-cudaError_t launch_ssd_fwd(const FwdArgs& a, bool summary, cudaStream_t s);
+// Backward of the chunked matrix form (ssm_ssd_bwd.cu): scalar decay, bf16 io, N = 16..128.
+struct SsdBwdArgs {
+  const uint16_t* u;
+  const uint16_t* delta;
+  const uint16_t* z;        // NULL: no gate
+  const uint16_t* B;        // [batch][bc_groups][N][L]
+  const uint16_t* C;
+  const uint16_t* dout;
+  const float* A;           // [dim]
+  const float* D;
+  const float* dt_bias;
+  const float* dhL;
+  const float* ck;          // [batch][dim][ceil(L/16) + 1][N]: the state entering every chunk
+  uint16_t* du;
+  uint16_t* ddelta;
+  uint16_t* dz;
+  float* dh0;
+  float* part_bc;           // [CTAs per row][batch][2][N][L]: each CTA's dB, dC
+  float* part_adt;          // [batch][dim][3]: dA, dD, ddt_bias of each (row, channel)
+  int batch, dim, L, N, bc_groups, softplus, rows16, need_bc;
+};
+// 64 channels per CTA (dim / bc_groups a multiple of 64 with groups); a.ck from launch_ssd_fwd's
+// checkpoint mode.  The finishing launch sums part_bc over each group's CTAs into dB, dC (bf16)
+// and part_adt over the batch into dA, dD, ddt_bias.
+cudaError_t launch_ssd_bwd(const SsdBwdArgs& a, cudaStream_t s);
+cudaError_t launch_ssd_bwd_finish(const SsdBwdArgs& a, void* dB, void* dC, float* dA, float* dD,
+                                  float* ddt_bias, cudaStream_t s);
+int ssd_bwd_ctas_per_row(int dim);
+// mode: kSsdOut, kSsdSummary, or kSsdCkpt (no outputs; the state entering every chunk and the final
+// state into a.ckpt, f32 [batch][dim][ceil(L / 16) + 1][N]).
+enum SsdMode { kSsdOut = 0, kSsdSummary = 1, kSsdCkpt = 2 };
+cudaError_t launch_ssd_fwd(const FwdArgs& a, int mode, cudaStream_t s);
 cudaError_t launch_fwd_carry(const FwdArgs& a, const float* summ, const float* dsum, float* hin,
                              cudaStream_t s);
 cudaError_t launch_bwd(const BwdArgs& a, int io, bool vec, cudaStream_t s);

@@ -40,7 +40,7 @@
 // chunk to chunk, so they run as warp-level mma.sync.m16n8k16 rather than tcgen05 tiles.
 //
 // Time split (few channels, long sequences): segments of whole chunks run side by side.  A
-// summary launch (SUMMARY = true) runs every segment but the last from a zero state, keeping
+// summary launch (MODE kSsdSummary) runs every segment but the last from a zero state, keeping
 // only the state update (no G, Y1, Y2, gate or outputs), and writes its end state and ΣΔ; the
 // host chains those segment maps (h -> e^{A ΣΔ} h + h_end) into each segment's entering state;
 // the output launch then runs every segment from its entering state.
@@ -49,56 +49,12 @@
 
 #include "ssm_device.cuh"
 #include "ssm_kernels.h"
+#include "ssm_mma.cuh"
 
 namespace ssm {
 namespace {
 
-constexpr int kT = 16;       // steps per chunk (one MMA k-step)
-constexpr int kLdS = 24;     // bf16 per shared tile row: 16 steps + 8 pad (48-byte rows)
-constexpr int kStages = 4;   // B/C ring depth (chunks)
-
-template <int N>
-struct SsdStage {
-  uint16_t Bs[N * kLdS];  // B of the chunk as [n][t]
-  uint16_t Cs[N * kLdS];  // C of the chunk as [n][t]
-};
-
-__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                         uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};\n"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// Four 8x8 bf16 matrices from shared memory; lane i gives the address of row i % 8 of matrix
-// i / 8.  Plain: lane l receives (row l / 4, cols 2 (l % 4), +1) of each; .trans: the transpose.
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
-  const uint32_t a = (uint32_t)__cvta_generic_to_shared(p);
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(a));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* p) {
-  const uint32_t a = (uint32_t)__cvta_generic_to_shared(p);
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(a));
-}
-// The lane's row address for the four 8x8 blocks (rows n0 .. n0+7 | n0+8 .., cols 0..7 | 8..15)
-// of a [n][t] tile: matrix m = lane / 8 covers rows n0 + 8 (m / 2) .., cols 8 (m % 2) ..
-__device__ __forceinline__ const uint16_t* blk(const uint16_t* tile, int n0, int lane) {
-  return tile + (n0 + ((lane >> 4) << 3) + (lane & 7)) * kLdS + (((lane >> 3) & 1) << 3);
-}
-
-__device__ __forceinline__ void cp16(void* smem, const void* gmem) {
-  const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-template <int K>
-__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(K) : "memory"); }
+using namespace ssd;
 
 // u, delta, z of the lane's two channels and four steps of one chunk, as bf16 pairs:
 // w[c][0] = steps 2tg, 2tg+1 and w[c][1] = steps 2tg+8, 2tg+9 of channel c.
@@ -113,8 +69,29 @@ __device__ __forceinline__ uint32_t ld_pair(const uint16_t* p, long long t, int 
   return lo | (hi << 16);
 }
 
-template <int N, int W, bool SUMMARY>
+// The state (transposed accumulator layout, 2 channels x N/4 states per lane) into slot `slot`
+// of the f32 checkpoint array [batch][dim][chunks + 1][N].
+template <int N>
+__device__ __forceinline__ void store_state(const FwdArgs& a, const float (&Ht)[N / 8][4],
+                                            int slot, int b, const int (&dch)[2],
+                                            const bool (&act)[2], int tg) {
+  const long long nslots = (a.L + kT - 1) / kT + 1;
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    if (!act[c]) continue;
+    float* row = a.ckpt + (((long long)b * a.dim + dch[c]) * nslots + slot) * N + 2 * tg;
+#pragma unroll
+    for (int nt = 0; nt < N / 8; ++nt)
+      *reinterpret_cast<float2*>(row + 8 * nt) = make_float2(Ht[nt][2 * c], Ht[nt][2 * c + 1]);
+  }
+}
+
+// MODE: kSsdOut (gated outputs), kSsdSummary (segment end state and ΣΔ from zero), kSsdCkpt (the
+// state entering every chunk, and the final state, into a.ckpt (f32) for the backward).
+template <int N, int W, int MODE>
 __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__ FwdArgs a) {
+  constexpr bool SUMMARY = MODE == kSsdSummary;
+  constexpr bool NOOUT = MODE != kSsdOut;  // no gate, readout or outputs
   constexpr int kNT = N / 8;  // n8 tiles of the state
   extern __shared__ float4 smem_ssd[];
   SsdStage<N>* ring = reinterpret_cast<SsdStage<N>*>(smem_ssd);
@@ -220,6 +197,7 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
     if (k + 1 < nchunk) load_in(k + 1, nxt);
     const SsdStage<N>& st = ring[k % kStages];
     const int t0 = (kc0 + k) * kT;
+    if (MODE == kSsdCkpt) store_state<N>(a, Ht, kc0 + k, b, dch, act, tg);
 
     // ---- per (channel, step): Δ, Δx, gate; index j: steps 2tg, 2tg+1, 2tg+8, 2tg+9
     float dl[2][4], xv[2][4], gt[2][4], uv[2][4];
@@ -236,7 +214,7 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
         dl[c][j] = live ? D : 0.f;
         uv[c][j] = live ? u : 0.f;
         xv[c][j] = dl[c][j] * uv[c][j];
-        if (zp && !SUMMARY) {
+        if (zp && !NOOUT) {
           const float z = (j & 1) ? bf16_hi(wz) : bf16_lo(wz);
           gt[c][j] = z * sigmoid_fast(z);
         } else {
@@ -290,6 +268,7 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
     // ---- decay factors and the scaled inputs (A operands of Y1' and U')
     float P[2][4], E[2][4], scale[2];
     uint32_t x1[4], x2[4];  // A fragments: {row g k lo, row g+8 k lo, row g k hi, row g+8 k hi}
+    uint32_t x2l[4];        // the remainders of x2 (summary and checkpoint passes)
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       const float eAm = ex2_mufu(Sm[c] * al[c]);
@@ -307,15 +286,15 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
       }
       x1[c] = pack_bf16x2(q1[0], q1[1]);
       x1[2 + c] = pack_bf16x2(q1[2], q1[3]);
-      x2[c] = pack_bf16x2(q2[0], q2[1]);
-      x2[2 + c] = pack_bf16x2(q2[2], q2[3]);
+      split_bf16x2(q2[0], q2[1], x2[c], x2l[c]);
+      split_bf16x2(q2[2], q2[3], x2[2 + c], x2l[2 + c]);
     }
 
     // ---- G = C B^T and Y2' = H' C^T, sharing the C fragments of each 16-state k-step
     float G[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // s tiles 0..7, 8..15
     float Y2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // t tiles 0..7, 8..15
 #pragma unroll
-    for (int kk = 0; kk < (SUMMARY ? 0 : N / 16); ++kk) {
+    for (int kk = 0; kk < (NOOUT ? 0 : N / 16); ++kk) {
       uint32_t cf[4], bf[4];
       ldsm_x4_t(cf, blk(st.Cs, 16 * kk, lane));  // {t0-7|n lo, t8-15|n lo, t0-7|n hi, t8-15|n hi}
       ldsm_x4_t(bf, blk(st.Bs, 16 * kk, lane));  // {s0-7|n lo, s8-15|n lo, s0-7|n hi, s8-15|n hi}
@@ -340,11 +319,15 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
       }
       mma16816(Ht[nt], x2[0], x2[1], x2[2], x2[3], bn[0], bn[1]);
       mma16816(Ht[nt + 1], x2[0], x2[1], x2[2], x2[3], bn[2], bn[3]);
+      if (NOOUT) {  // states that a backward or a chain reads: the remainder term too
+        mma16816(Ht[nt], x2l[0], x2l[1], x2l[2], x2l[3], bn[0], bn[1]);
+        mma16816(Ht[nt + 1], x2l[0], x2l[1], x2l[2], x2l[3], bn[2], bn[3]);
+      }
     }
     // ---- Y1' = X1' mask(G)^T: G's accumulators (rows t, cols s) are the B fragments
     // (k = s, n = t) once masked to s <= t
     float Y1[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    if (!SUMMARY) {
+    if (!NOOUT) {
       const int s0 = 2 * tg, r0 = g;
       const auto m = [](float v, int s, int t) { return s <= t ? v : 0.f; };
       // t tile 0: rows t = g; t tile 1: rows t = g + 8
@@ -392,7 +375,7 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
               yp = fmaf(cv, h, yp);
             }
           }
-          if (SUMMARY) continue;
+          if (NOOUT) continue;
           yp += __shfl_xor_sync(0xffffffffu, yp, 1);
           yp += __shfl_xor_sync(0xffffffffu, yp, 2);
           if (fb[c] && tg == to) yo[c][jo] = fmaf(Dd[c], uv[c][jo], yp) * gt[c][jo];
@@ -402,7 +385,7 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
     // ---- store the chunk's outputs (bf16 pairs of steps)
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
-      if (SUMMARY || !act[c]) continue;
+      if (NOOUT || !act[c]) continue;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         const long long t = t0 + 2 * tg + 8 * hh;
@@ -417,6 +400,10 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
     }
   }
   cp_wait<0>();
+  if (MODE == kSsdCkpt) {
+    if ((seg + 1) * a.chunk_len >= L) store_state<N>(a, Ht, kc0 + nchunk, b, dch, act, tg);
+    return;
+  }
   if (SUMMARY) {
 #pragma unroll
     for (int nt = 0; nt < kNT; ++nt) {
@@ -444,12 +431,14 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
 }
 
 template <int N, int W>
-cudaError_t launch_n(const FwdArgs& a, bool summary, cudaStream_t s) {
-  const int segs = summary ? a.nchunk - 1 : a.nchunk;  // the last segment's summary is unused
+cudaError_t launch_n(const FwdArgs& a, int mode, cudaStream_t s) {
+  const int segs = mode == kSsdSummary ? a.nchunk - 1 : a.nchunk;  // the last summary is unused
   if (segs <= 0) return cudaSuccess;
   const dim3 grid((unsigned)((long long)a.batch * ((a.dim + 16 * W - 1) / (16 * W))), (unsigned)segs);
   const size_t smem = kStages * sizeof(SsdStage<N>);
-  auto k = summary ? ssd_fwd_kernel<N, W, true> : ssd_fwd_kernel<N, W, false>;
+  auto k = mode == kSsdSummary ? ssd_fwd_kernel<N, W, kSsdSummary>
+                               : (mode == kSsdCkpt ? ssd_fwd_kernel<N, W, kSsdCkpt>
+                                                   : ssd_fwd_kernel<N, W, kSsdOut>);
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   k<<<grid, 32 * W, smem, s>>>(a);
@@ -457,7 +446,7 @@ cudaError_t launch_n(const FwdArgs& a, bool summary, cudaStream_t s) {
 }
 
 template <int N>
-cudaError_t launch_w(const FwdArgs& a, bool summary, cudaStream_t s) {
+cudaError_t launch_w(const FwdArgs& a, int mode, cudaStream_t s) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -467,17 +456,17 @@ cudaError_t launch_w(const FwdArgs& a, bool summary, cudaStream_t s) {
   bool two = ctas4 < 2LL * sms;
   const char* env = getenv("SSM_SSD_WPB");
   if (env && (atoi(env) == 2 || atoi(env) == 4)) two = atoi(env) == 2;
-  return two ? launch_n<N, 2>(a, summary, s) : launch_n<N, 4>(a, summary, s);
+  return two ? launch_n<N, 2>(a, mode, s) : launch_n<N, 4>(a, mode, s);
 }
 
 }  // namespace
 
-cudaError_t launch_ssd_fwd(const FwdArgs& a, bool summary, cudaStream_t s) {
+cudaError_t launch_ssd_fwd(const FwdArgs& a, int mode, cudaStream_t s) {
   switch (a.N) {
-    case 16: return launch_w<16>(a, summary, s);
-    case 32: return launch_w<32>(a, summary, s);
-    case 64: return launch_w<64>(a, summary, s);
-    case 128: return launch_w<128>(a, summary, s);
+    case 16: return launch_w<16>(a, mode, s);
+    case 32: return launch_w<32>(a, mode, s);
+    case 64: return launch_w<64>(a, mode, s);
+    case 128: return launch_w<128>(a, mode, s);
     default: return cudaErrorInvalidValue;
   }
 }

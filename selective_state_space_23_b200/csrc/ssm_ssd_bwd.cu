@@ -1,0 +1,782 @@
+// Backward of the scalar-decay scan in its chunked matrix form, on the tensor cores, sm_100a,
+// bf16 io, N = 16, 32, 64, 128.
+//
+// Forward (ssm_ssd.cu), per channel d with rate A and a 16-step chunk with cumulative steps S_t,
+// a_t = A S_t, decay factors P_t = e^{a_t - a_m}, Q_s = 1 / P_s (m the middle step),
+// E_t = e^{a_t}, x'_s = Δ_s x_s, h_in the state entering the chunk:
+//   y_t   = Σ_{s<=t} G_ts P_t Q_s x'_s + E_t C_t.h_in + D x_t,   G = C B^T
+//   h_out = e^{a_15} h_in + Σ_s e^{a_15 - a_s} x'_s B_s.
+// Given g_t = dL/dy_t (dout times the gate) and μ = dL/dh_out (the adjoint carried in from the
+// next chunk), the chain rule gives, per chunk:
+//   dL/dx'_s  = Q_s [ Σ_{t>=s} (g P)_t G_ts ] + e^{a_15 - a_m} Q_s (μ . B_s)
+//   dL/dh_in  = Σ_t (g E)_t C_t + e^{a_15} μ                      (carried to the previous chunk)
+//   dL/da_t   = g_t y^ssm_t - x'_t dL/dx'_t + [t = 15] μ . h_out   (y^ssm = y - D x)
+//   dΔ_r = A Σ_{t>=r} dL/da_t + x_r dL/dx'_r,   dA = Σ_t S_t dL/da_t,   dx = Δ dL/dx' + D g
+//   dB_s = Σ_d [ Σ_{t>=s} M_st C_t + e^{a_15 - a_m} Q_s x'_s μ ],   M = (Q x')^T (g P) over d
+//   dC_t = Σ_d [ Σ_{s<=t} M_st B_s + (g E)_t h_in ]
+// (the Mamba-2 / Hydra structured-matrix view of the scan on the "2024 Reading List: Neural
+// Network" page; the chain rule through the recurrence is that of the backward of the other
+// variants, "Donanım Duyarlı Durum Genişletme": states are recomputed, not stored per step).
+//
+// B200 mapping: the same warp layout as the forward (16 channels per warp; lane (g, tg) holds
+// channels g, g+8 and steps 2tg, 2tg+1, 2tg+8, 2tg+9 of a chunk).  The chunks are walked in
+// reverse.  The adjoint μ (transposed, [d][n]) lives in MMA accumulator registers like the
+// forward's state; the entering state h_in of every chunk comes from the forward's f32
+// checkpoints.  Products whose operands must be transposed relative to their accumulator layout
+// go through small per-warp shared-memory tiles read with ldmatrix(.trans).  dL/da sums terms
+// that cancel (μ . h_out against the inputs' share of h_out, y g against x' dL/dx'), and dA,
+// ddt_bias sum dL/da over the whole sequence, so every product that feeds them takes its
+// non-input operands as bf16 pairs plus remainders (about 16 significant bits; B, C are exact
+// bf16 inputs): the forward's checkpoint states likewise.  dB, dC (bf16 outputs) use one bf16
+// operand per product.  dB, dC are summed
+// over the warp's 16 channels by the tensor cores (the contractions over d), over the CTA's
+// warps in shared memory in a fixed order, and over CTAs by a finishing kernel in a fixed order,
+// so the result is bitwise reproducible.  A channel whose chunk leaves the factorisation's range
+// (as in the forward) takes no part in that chunk's products and is computed by an exact
+// sequential pass over the states its quad holds.
+#include <stdint.h>
+#include <stdlib.h>
+
+#include "ssm_device.cuh"
+#include "ssm_kernels.h"
+#include "ssm_mma.cuh"
+
+namespace ssm {
+namespace {
+
+using namespace ssd;
+
+constexpr int kWb = 4;  // warps per CTA (64 channels of one batch row and B/C group)
+
+template <int N>
+struct BwdWarpSmem {
+  static constexpr int kLdN = N + 8;  // bf16 row stride of the [16][N] tiles
+  uint16_t x1[16 * kLdS];   // Q x'          [d][s]
+  uint16_t x2[16 * kLdS];   // e^{a15-am} Q x' [d][s]
+  uint16_t gp[16 * kLdS];   // g P           [d][t]
+  uint16_t ge[16 * kLdS];   // g E           [d][t]
+  uint16_t mu[16 * kLdN];   // μ (before this chunk's update) [d][n]
+  uint16_t hin[16 * kLdN];  // h_in          [d][n]
+  float red[2 * 16 * N];    // this warp's dB, dC of the chunk: [which][t][n]
+};
+
+template <int N>
+struct BwdSmem {
+  SsdStage<N> ring[kStages];
+  BwdWarpSmem<N> w[kWb];
+};
+
+struct ChunkInB {
+  uint32_t u[2][2], dl[2][2], z[2][2], go[2][2];
+};
+
+__device__ __forceinline__ uint32_t ldp(const uint16_t* p, long long t, int L, bool vec) {
+  if (vec) return __ldg(reinterpret_cast<const uint32_t*>(p + t));
+  const uint32_t lo = t < L ? (uint32_t)__ldg(p + t) : 0u;
+  const uint32_t hi = t + 1 < L ? (uint32_t)__ldg(p + t + 1) : 0u;
+  return lo | (hi << 16);
+}
+__device__ __forceinline__ float pick(uint32_t w, int odd) { return odd ? bf16_hi(w) : bf16_lo(w); }
+
+template <int N>
+__global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant__ SsdBwdArgs a) {
+  constexpr int kNT = N / 8;
+  constexpr int LDN = BwdWarpSmem<N>::kLdN;
+  extern __shared__ float4 smem_sb[];
+  BwdSmem<N>& sm = *reinterpret_cast<BwdSmem<N>*>(smem_sb);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, tg = lane & 3;
+  BwdWarpSmem<N>& ws = sm.w[warp];
+  const int tiles_d = (a.dim + 16 * kWb - 1) / (16 * kWb);
+  const int b = blockIdx.x / tiles_d, ctag = blockIdx.x % tiles_d;
+  const int d0 = ctag * 16 * kWb;
+  const int L = a.L;
+  const int nck = (L + kT - 1) / kT;
+  const long long nslots = nck + 1;
+  const int gbc = d0 / (a.dim / a.bc_groups);
+  const uint16_t* Bg = a.B + ((long long)b * a.bc_groups + gbc) * N * (long long)L;
+  const uint16_t* Cg = a.C + ((long long)b * a.bc_groups + gbc) * N * (long long)L;
+
+  int dch[2];
+  bool act[2];
+  long long row[2];
+  float al[2], bias[2], Dd[2];
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    const int d = d0 + 16 * warp + g + 8 * c;
+    act[c] = d < a.dim;
+    dch[c] = act[c] ? d : a.dim - 1;
+    row[c] = ((long long)b * a.dim + dch[c]) * L;
+    al[c] = a.A[dch[c]] * kLog2e;
+    bias[c] = a.dt_bias ? a.dt_bias[dch[c]] : 0.f;
+    Dd[c] = a.D ? a.D[dch[c]] : 0.f;
+  }
+  // the checkpointed states of the lane's channels; hck(c, k, nt): states 8 nt + 2 tg, +1 of the
+  // state entering chunk k (slot nck: the final state)
+  const float* ckr[2];
+#pragma unroll
+  for (int c = 0; c < 2; ++c) ckr[c] = a.ck + ((long long)b * a.dim + dch[c]) * nslots * N + 2 * tg;
+  const auto hck = [&](int c, int k, int nt) {
+    return __ldg(reinterpret_cast<const float2*>(ckr[c] + (long long)k * N + 8 * nt));
+  };
+
+  // the adjoint μ = dL/dh_out of the current chunk, transposed [d][n] in accumulator layout
+  float mu[kNT][4];
+#pragma unroll
+  for (int nt = 0; nt < kNT; ++nt) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int c = e >> 1, n = 8 * nt + 2 * tg + (e & 1);
+      mu[nt][e] = a.dhL && act[c] ? a.dhL[((long long)b * a.dim + dch[c]) * N + n] : 0.f;
+    }
+  }
+
+  float accA[2] = {0.f, 0.f}, accD[2] = {0.f, 0.f}, accT[2] = {0.f, 0.f};
+
+  // B/C tiles of chunk nck-1-i into ring slot i % kStages (chunks walked in reverse)
+  const auto issue = [&](int i) {
+    if (i < nck) {
+      SsdStage<N>& st = sm.ring[i % kStages];
+      const int t0 = (nck - 1 - i) * kT;
+      if (a.rows16 && t0 + kT <= L) {
+        for (int p = tid; p < 4 * N; p += 32 * kWb) {
+          const int which = p / (2 * N), rem = p % (2 * N), n = rem >> 1, h = rem & 1;
+          cp16((which ? st.Cs : st.Bs) + n * kLdS + 8 * h, (which ? Cg : Bg) + (long long)n * L + t0 + 8 * h);
+        }
+      } else {
+        for (int p = tid; p < 2 * N * kT; p += 32 * kWb) {
+          const int which = p / (N * kT), rem = p % (N * kT), n = rem / kT, t = rem % kT;
+          (which ? st.Cs : st.Bs)[n * kLdS + t] =
+              t0 + t < L ? (which ? Cg : Bg)[(long long)n * L + t0 + t] : (uint16_t)0;
+        }
+      }
+    }
+    cp_commit();
+  };
+  const bool vec_rows = a.rows16 != 0;
+  const auto load_in = [&](int k, ChunkInB& in) {
+    const int t0 = k * kT;
+    const bool vec = vec_rows && t0 + kT <= L;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const long long t = t0 + 2 * tg + 8 * hh;
+        in.u[c][hh] = ldp(a.u + row[c], t, L, vec);
+        in.dl[c][hh] = ldp(a.delta + row[c], t, L, vec);
+        in.z[c][hh] = a.z ? ldp(a.z + row[c], t, L, vec) : 0u;
+        in.go[c][hh] = ldp(a.dout + row[c], t, L, vec);
+      }
+    }
+  };
+
+#pragma unroll
+  for (int i = 0; i < kStages - 1; ++i) issue(i);
+  ChunkInB nxt;
+  load_in(nck - 1, nxt);
+
+  for (int i = 0; i < nck; ++i) {
+    const int k = nck - 1 - i;
+    cp_wait<kStages - 2>();
+    __syncthreads();  // chunk k's B/C landed; every warp is done with the previous chunk
+    issue(i + kStages - 1);
+    const ChunkInB cur = nxt;
+    if (k > 0) load_in(k - 1, nxt);
+    const SsdStage<N>& st = sm.ring[i % kStages];
+    const int t0 = k * kT;
+
+    // ---- per (channel, step) quantities; j: steps 2tg, 2tg+1, 2tg+8, 2tg+9.  Steps past L
+    // and idle channels (which shadow the last channel) take no part: zero step, input and g.
+    float dl[2][4], uv[2][4], xv[2][4], sg[2][4], gz[2][4], zz[2][4], gd[2][4], gg[2][4];
+    bool lv[2][4];
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int hh = j >> 1, od = j & 1;
+        const int t = t0 + 2 * tg + od + 8 * hh;
+        const bool live = act[c] && t < L;
+        lv[c][j] = live;
+        const float u = pick(cur.u[c][hh], od);
+        const float v = pick(cur.dl[c][hh], od) + bias[c];
+        const float D = a.softplus ? softplus_fast(v) : v;
+        sg[c][j] = a.softplus ? sigmoid_fast(v) : 1.f;  // dΔ/dv
+        dl[c][j] = live ? D : 0.f;
+        uv[c][j] = live ? u : 0.f;
+        xv[c][j] = dl[c][j] * uv[c][j];
+        gd[c][j] = live ? pick(cur.go[c][hh], od) : 0.f;
+        if (a.z) {
+          const float z = pick(cur.z[c][hh], od);
+          zz[c][j] = z;
+          gz[c][j] = sigmoid_fast(z);  // σ(z)
+          gg[c][j] = gd[c][j] * z * gz[c][j];
+        } else {
+          zz[c][j] = 0.f;
+          gz[c][j] = 1.f;
+          gg[c][j] = gd[c][j];
+        }
+      }
+    }
+    // cumulative steps (scan over the quad) and the factorisation's range
+    float S[2][4], Sm[2], Se[2];
+    bool fb[2];
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const float p = dl[c][0] + dl[c][1], q = dl[c][2] + dl[c][3];
+      float ip = p, iq = q;
+#pragma unroll
+      for (int off = 1; off < 4; off <<= 1) {
+        const float np = __shfl_up_sync(0xffffffffu, ip, off, 4);
+        const float nq = __shfl_up_sync(0xffffffffu, iq, off, 4);
+        if (tg >= off) {
+          ip += np;
+          iq += nq;
+        }
+      }
+      const float lo_total = __shfl_sync(0xffffffffu, ip, 3, 4);
+      const float hi_total = __shfl_sync(0xffffffffu, iq, 3, 4);
+      S[c][0] = ip - p + dl[c][0];
+      S[c][1] = ip;
+      S[c][2] = lo_total + iq - q + dl[c][2];
+      S[c][3] = lo_total + iq;
+      Sm[c] = lo_total;
+      Se[c] = lo_total + hi_total;
+      float mrel = 0.f, mabs = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        mrel = fmaxf(mrel, fabsf(S[c][j] - Sm[c]));
+        mabs = fmaxf(mabs, fabsf(S[c][j]));
+      }
+      int ok = (fabsf(al[c]) * kLn2 * mrel <= 60.f && fabsf(al[c]) * kLn2 * mabs <= 80.f) ? 1 : 0;
+      ok &= __shfl_xor_sync(0xffffffffu, ok, 1, 4);
+      ok &= __shfl_xor_sync(0xffffffffu, ok, 2, 4);
+      fb[c] = ok == 0;
+    }
+    float P[2][4], Qv[2][4], E[2][4], eEm[2], Eend[2];
+    // A fragments (bf16 pairs) and, for the products that feed dΔ, dA and the carried adjoint,
+    // the remainders (suffix l)
+    uint32_t x1[4], x2[4], gpA[4], geA[4], x1l[4], gpl[4], gel[4];
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const float eAm = ex2_mufu(Sm[c] * al[c]);
+      eEm[c] = ex2_mufu((Se[c] - Sm[c]) * al[c]);
+      Eend[c] = ex2_mufu(Se[c] * al[c]);
+      float q1[4], q2[4], gp[4], ge[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float r = (S[c][j] - Sm[c]) * al[c];
+        P[c][j] = ex2_mufu(r);
+        Qv[c][j] = ex2_mufu(-r);
+        E[c][j] = eAm * P[c][j];
+        q1[j] = fb[c] ? 0.f : Qv[c][j] * xv[c][j];
+        q2[j] = fb[c] ? 0.f : eEm[c] * q1[j];
+        gp[j] = fb[c] ? 0.f : gg[c][j] * P[c][j];
+        ge[j] = fb[c] ? 0.f : gg[c][j] * E[c][j];
+      }
+      split_bf16x2(q1[0], q1[1], x1[c], x1l[c]);
+      split_bf16x2(q1[2], q1[3], x1[2 + c], x1l[2 + c]);
+      x2[c] = pack_bf16x2(q2[0], q2[1]);
+      x2[2 + c] = pack_bf16x2(q2[2], q2[3]);
+      split_bf16x2(gp[0], gp[1], gpA[c], gpl[c]);
+      split_bf16x2(gp[2], gp[3], gpA[2 + c], gpl[2 + c]);
+      split_bf16x2(ge[0], ge[1], geA[c], gel[c]);
+      split_bf16x2(ge[2], ge[3], geA[2 + c], gel[2 + c]);
+    }
+    // per-warp tiles: rows d = g + 8 c, columns 2 tg + 8 hh
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int o = (g + 8 * c) * kLdS + 2 * tg + 8 * hh;
+        *reinterpret_cast<uint32_t*>(ws.x1 + o) = x1[2 * hh + c];
+        *reinterpret_cast<uint32_t*>(ws.x2 + o) = x2[2 * hh + c];
+        *reinterpret_cast<uint32_t*>(ws.gp + o) = gpA[2 * hh + c];
+        *reinterpret_cast<uint32_t*>(ws.ge + o) = geA[2 * hh + c];
+      }
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt) {
+        const int o = (g + 8 * c) * LDN + 8 * nt + 2 * tg;
+        const float2 hv = hck(c, k, nt);
+        *reinterpret_cast<uint32_t*>(ws.hin + o) = pack_bf16x2(hv.x, hv.y);
+        *reinterpret_cast<uint32_t*>(ws.mu + o) = pack_bf16x2(mu[nt][2 * c], mu[nt][2 * c + 1]);
+      }
+    }
+    __syncwarp();
+
+    // ---- recompute G (rows t) and G^T (rows s), Y2' = H_in C^T; and μ B^T, per 16 states
+    // (H_in and μ split into bf16 pairs and remainders; B, C are exact bf16 inputs)
+    float G[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    float GT[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    float Y2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    float Xm[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // Σ_n μ[d][n] B_s[n], [d][s]
+#pragma unroll
+    for (int kk = 0; kk < N / 16; ++kk) {
+      uint32_t cf[4], bf[4];
+      ldsm_x4_t(cf, blk(st.Cs, 16 * kk, lane));
+      ldsm_x4_t(bf, blk(st.Bs, 16 * kk, lane));
+      mma16816(G[0], cf[0], cf[1], cf[2], cf[3], bf[0], bf[2]);
+      mma16816(G[1], cf[0], cf[1], cf[2], cf[3], bf[1], bf[3]);
+      mma16816(GT[0], bf[0], bf[1], bf[2], bf[3], cf[0], cf[2]);
+      mma16816(GT[1], bf[0], bf[1], bf[2], bf[3], cf[1], cf[3]);
+      uint32_t hh[4], hl[4], mh[4], ml[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {  // {row g k lo, row g+8 k lo, row g k hi, row g+8 k hi}
+        const int nt = 2 * kk + (q >> 1), c = q & 1;
+        const float2 hv = hck(c, k, nt);
+        split_bf16x2(hv.x, hv.y, hh[q], hl[q]);
+        split_bf16x2(mu[nt][2 * c], mu[nt][2 * c + 1], mh[q], ml[q]);
+      }
+      mma16816(Y2[0], hh[0], hh[1], hh[2], hh[3], cf[0], cf[2]);
+      mma16816(Y2[1], hh[0], hh[1], hh[2], hh[3], cf[1], cf[3]);
+      mma16816(Y2[0], hl[0], hl[1], hl[2], hl[3], cf[0], cf[2]);
+      mma16816(Y2[1], hl[0], hl[1], hl[2], hl[3], cf[1], cf[3]);
+      mma16816(Xm[0], mh[0], mh[1], mh[2], mh[3], bf[0], bf[2]);
+      mma16816(Xm[1], mh[0], mh[1], mh[2], mh[3], bf[1], bf[3]);
+      mma16816(Xm[0], ml[0], ml[1], ml[2], ml[3], bf[0], bf[2]);
+      mma16816(Xm[1], ml[0], ml[1], ml[2], ml[3], bf[1], bf[3]);
+    }
+    const int s0 = 2 * tg;
+    const auto msk = [](float v, int s, int t) { return s <= t ? v : 0.f; };
+    // Y1' = X1' mask(G)^T  (B fragments from G's accumulators, rows t)
+    float Y1[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    {
+      uint32_t b00, b01, b10, b11, l00, l01, l10, l11;
+      split_bf16x2(msk(G[0][0], s0, g), msk(G[0][1], s0 + 1, g), b00, l00);
+      split_bf16x2(msk(G[1][0], s0 + 8, g), msk(G[1][1], s0 + 9, g), b01, l01);
+      split_bf16x2(msk(G[0][2], s0, g + 8), msk(G[0][3], s0 + 1, g + 8), b10, l10);
+      split_bf16x2(msk(G[1][2], s0 + 8, g + 8), msk(G[1][3], s0 + 9, g + 8), b11, l11);
+      mma16816(Y1[0], x1[0], x1[1], x1[2], x1[3], b00, b01);
+      mma16816(Y1[1], x1[0], x1[1], x1[2], x1[3], b10, b11);
+      mma16816(Y1[0], x1[0], x1[1], x1[2], x1[3], l00, l01);
+      mma16816(Y1[1], x1[0], x1[1], x1[2], x1[3], l10, l11);
+      mma16816(Y1[0], x1l[0], x1l[1], x1l[2], x1l[3], b00, b01);
+      mma16816(Y1[1], x1l[0], x1l[1], x1l[2], x1l[3], b10, b11);
+    }
+    // dX' (y part) = (g P) mask(G): B fragments (k = t, n = s) from G^T's accumulators (rows s)
+    float Xy[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    {
+      const int t0l = 2 * tg;
+      uint32_t b00, b01, b10, b11, l00, l01, l10, l11;
+      split_bf16x2(msk(GT[0][0], g, t0l), msk(GT[0][1], g, t0l + 1), b00, l00);
+      split_bf16x2(msk(GT[1][0], g, t0l + 8), msk(GT[1][1], g, t0l + 9), b01, l01);
+      split_bf16x2(msk(GT[0][2], g + 8, t0l), msk(GT[0][3], g + 8, t0l + 1), b10, l10);
+      split_bf16x2(msk(GT[1][2], g + 8, t0l + 8), msk(GT[1][3], g + 8, t0l + 9), b11, l11);
+      mma16816(Xy[0], gpA[0], gpA[1], gpA[2], gpA[3], b00, b01);
+      mma16816(Xy[1], gpA[0], gpA[1], gpA[2], gpA[3], b10, b11);
+      mma16816(Xy[0], gpA[0], gpA[1], gpA[2], gpA[3], l00, l01);
+      mma16816(Xy[1], gpA[0], gpA[1], gpA[2], gpA[3], l10, l11);
+      mma16816(Xy[0], gpl[0], gpl[1], gpl[2], gpl[3], b00, b01);
+      mma16816(Xy[1], gpl[0], gpl[1], gpl[2], gpl[3], b10, b11);
+    }
+    // μ . h_out of each channel (before μ is carried back), summed over the quad's states;
+    // h_out is the state entering chunk k + 1
+    float muh[2] = {0.f, 0.f};
+#pragma unroll
+    for (int nt = 0; nt < kNT; ++nt) {
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const float2 ho = hck(c, k + 1, nt);
+        muh[c] = fmaf(mu[nt][2 * c], ho.x, fmaf(mu[nt][2 * c + 1], ho.y, muh[c]));
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      muh[c] += __shfl_xor_sync(0xffffffffu, muh[c], 1);
+      muh[c] += __shfl_xor_sync(0xffffffffu, muh[c], 2);
+    }
+
+    // ---- per (channel, step): y, dx', da (accumulator (tile T, e): channel e/2, j = 2T + e%2)
+    float ys[2][4], dxp[2][4], da[2][4];
+#pragma unroll
+    for (int T = 0; T < 2; ++T) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int c = e >> 1, j = 2 * T + (e & 1);
+        ys[c][j] = fmaf(P[c][j], Y1[T][e], E[c][j] * Y2[T][e]);
+        dxp[c][j] = Qv[c][j] * fmaf(eEm[c], Xm[T][e], Xy[T][e]);
+      }
+    }
+
+    // ---- dB, dC of the chunk summed over the warp's channels on the tensor cores, then over
+    // the CTA's warps (fixed order) into this CTA's partial
+    if (a.need_bc) {
+      uint32_t x1T[4], x2T[4], gpT[4], geT[4];
+      ldsm_x4_t(x1T, blk(ws.x1, 0, lane));
+      ldsm_x4_t(x2T, blk(ws.x2, 0, lane));
+      ldsm_x4_t(gpT, blk(ws.gp, 0, lane));
+      ldsm_x4_t(geT, blk(ws.ge, 0, lane));
+      // M[s][t] = Σ_d X1'[d][s] (gP)[d][t] and its transpose Mt[t][s]
+      float M[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      float Mt[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      mma16816(M[0], x1T[0], x1T[1], x1T[2], x1T[3], gpT[0], gpT[2]);
+      mma16816(M[1], x1T[0], x1T[1], x1T[2], x1T[3], gpT[1], gpT[3]);
+      mma16816(Mt[0], gpT[0], gpT[1], gpT[2], gpT[3], x1T[0], x1T[2]);
+      mma16816(Mt[1], gpT[0], gpT[1], gpT[2], gpT[3], x1T[1], x1T[3]);
+      // M masked to t >= s as A fragments (rows s, k = t); Mt masked to s <= t (rows t, k = s)
+      const int t0l = 2 * tg;
+      const uint32_t ma0 = pack_bf16x2(msk(M[0][0], g, t0l), msk(M[0][1], g, t0l + 1));
+      const uint32_t ma1 = pack_bf16x2(msk(M[0][2], g + 8, t0l), msk(M[0][3], g + 8, t0l + 1));
+      const uint32_t ma2 = pack_bf16x2(msk(M[1][0], g, t0l + 8), msk(M[1][1], g, t0l + 9));
+      const uint32_t ma3 = pack_bf16x2(msk(M[1][2], g + 8, t0l + 8), msk(M[1][3], g + 8, t0l + 9));
+      const uint32_t mt0 = pack_bf16x2(msk(Mt[0][0], s0, g), msk(Mt[0][1], s0 + 1, g));
+      const uint32_t mt1 = pack_bf16x2(msk(Mt[0][2], s0, g + 8), msk(Mt[0][3], s0 + 1, g + 8));
+      const uint32_t mt2 = pack_bf16x2(msk(Mt[1][0], s0 + 8, g), msk(Mt[1][1], s0 + 9, g));
+      const uint32_t mt3 = pack_bf16x2(msk(Mt[1][2], s0 + 8, g + 8), msk(Mt[1][3], s0 + 9, g + 8));
+#pragma unroll
+      for (int nt = 0; nt < kNT; nt += 2) {
+        uint32_t cn[4], bn[4], mub[4], hib[4];
+        ldsm_x4(cn, blk(st.Cs, 8 * nt, lane));
+        ldsm_x4(bn, blk(st.Bs, 8 * nt, lane));
+        ldsm_x4_t(mub, blk(ws.mu + 8 * nt, 0, lane, LDN));
+        ldsm_x4_t(hib, blk(ws.hin + 8 * nt, 0, lane, LDN));
+        float dB0[4] = {0.f, 0.f, 0.f, 0.f}, dB1[4] = {0.f, 0.f, 0.f, 0.f};
+        float dC0[4] = {0.f, 0.f, 0.f, 0.f}, dC1[4] = {0.f, 0.f, 0.f, 0.f};
+        mma16816(dB0, ma0, ma1, ma2, ma3, cn[0], cn[1]);
+        mma16816(dB1, ma0, ma1, ma2, ma3, cn[2], cn[3]);
+        mma16816(dB0, x2T[0], x2T[1], x2T[2], x2T[3], mub[0], mub[2]);
+        mma16816(dB1, x2T[0], x2T[1], x2T[2], x2T[3], mub[1], mub[3]);
+        mma16816(dC0, mt0, mt1, mt2, mt3, bn[0], bn[1]);
+        mma16816(dC1, mt0, mt1, mt2, mt3, bn[2], bn[3]);
+        mma16816(dC0, geT[0], geT[1], geT[2], geT[3], hib[0], hib[2]);
+        mma16816(dC1, geT[0], geT[1], geT[2], geT[3], hib[1], hib[3]);
+        // rows (s or t) g, g+8; columns n = 8 nt' + 2 tg, +1
+        float* rb = ws.red;
+        float* rc = ws.red + 16 * N;
+        *reinterpret_cast<float2*>(rb + g * N + 8 * nt + 2 * tg) = make_float2(dB0[0], dB0[1]);
+        *reinterpret_cast<float2*>(rb + (g + 8) * N + 8 * nt + 2 * tg) = make_float2(dB0[2], dB0[3]);
+        *reinterpret_cast<float2*>(rb + g * N + 8 * nt + 8 + 2 * tg) = make_float2(dB1[0], dB1[1]);
+        *reinterpret_cast<float2*>(rb + (g + 8) * N + 8 * nt + 8 + 2 * tg) = make_float2(dB1[2], dB1[3]);
+        *reinterpret_cast<float2*>(rc + g * N + 8 * nt + 2 * tg) = make_float2(dC0[0], dC0[1]);
+        *reinterpret_cast<float2*>(rc + (g + 8) * N + 8 * nt + 2 * tg) = make_float2(dC0[2], dC0[3]);
+        *reinterpret_cast<float2*>(rc + g * N + 8 * nt + 8 + 2 * tg) = make_float2(dC1[0], dC1[1]);
+        *reinterpret_cast<float2*>(rc + (g + 8) * N + 8 * nt + 8 + 2 * tg) = make_float2(dC1[2], dC1[3]);
+      }
+    }
+    __syncwarp();  // this warp's dB, dC tile is written
+    const bool anyfb = __any_sync(0xffffffffu, fb[0] || fb[1]);
+    // ---- channels outside the factorisation's range this chunk: an exact sequential pass over
+    // the states each quad holds (rare).  Steps are walked backwards; the state before step t is
+    // recomputed from h_in.  Each step's dB, dC contributions are added to this warp's tile one
+    // quad at a time, in a fixed order.
+    if (anyfb) {
+      const int qb = lane & ~3;
+      const auto sel4 = [](const float (&v)[4], int j) {
+        return j == 0 ? v[0] : (j == 1 ? v[1] : (j == 2 ? v[2] : v[3]));
+      };
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        if (!__any_sync(0xffffffffu, fb[c])) continue;
+        float lam[kNT][2];
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt) {
+          lam[nt][0] = mu[nt][2 * c];
+          lam[nt][1] = mu[nt][2 * c + 1];
+        }
+        float yso[4] = {0.f, 0.f, 0.f, 0.f}, dxo[4] = {0.f, 0.f, 0.f, 0.f}, dao[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+        for (int t = kT - 1; t >= 0; --t) {
+          const int to = (t & 7) >> 1, jo = (t & 1) + 2 * (t >> 3);  // owner lane, its index
+          const float dts = __shfl_sync(0xffffffffu, sel4(dl[c], jo), qb | to);
+          const float xts = __shfl_sync(0xffffffffu, sel4(xv[c], jo), qb | to);
+          const float gts = __shfl_sync(0xffffffffu, sel4(gg[c], jo), qb | to);
+          float hp[kNT][2];  // h_{t-1}: steps 0 .. t-1 replayed from h_in
+#pragma unroll
+          for (int nt = 0; nt < kNT; ++nt) {
+            const float2 hv = hck(c, k, nt);
+            hp[nt][0] = hv.x;
+            hp[nt][1] = hv.y;
+          }
+#pragma unroll 1
+          for (int r = 0; r < t; ++r) {
+            const int ro = (r & 7) >> 1, rj = (r & 1) + 2 * (r >> 3);
+            const float dr = __shfl_sync(0xffffffffu, sel4(dl[c], rj), qb | ro);
+            const float xr = __shfl_sync(0xffffffffu, sel4(xv[c], rj), qb | ro);
+            const float abr = ex2_mufu(dr * al[c]);
+#pragma unroll
+            for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+              for (int e = 0; e < 2; ++e)
+                hp[nt][e] = fmaf(abr, hp[nt][e], xr * bf16_to_f32(st.Bs[(8 * nt + 2 * tg + e) * kLdS + r]));
+          }
+          const float ab = ex2_mufu(dts * al[c]);
+          float yp = 0.f, dx = 0.f, dab = 0.f;
+#pragma unroll
+          for (int nt = 0; nt < kNT; ++nt) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int n = 8 * nt + 2 * tg + e;
+              const float bv = bf16_to_f32(st.Bs[n * kLdS + t]);
+              const float cv = bf16_to_f32(st.Cs[n * kLdS + t]);
+              yp = fmaf(cv, fmaf(ab, hp[nt][e], xts * bv), yp);
+              lam[nt][e] = fmaf(gts, cv, lam[nt][e]);  // λ_t = g_t C_t + Ā_{t+1} λ_{t+1}
+              dx = fmaf(lam[nt][e], bv, dx);
+              dab = fmaf(lam[nt][e], hp[nt][e], dab);  // dL/dĀ_t = λ_t . h_{t-1}
+            }
+          }
+          yp += __shfl_xor_sync(0xffffffffu, yp, 1);
+          yp += __shfl_xor_sync(0xffffffffu, yp, 2);
+          dx += __shfl_xor_sync(0xffffffffu, dx, 1);
+          dx += __shfl_xor_sync(0xffffffffu, dx, 2);
+          dab += __shfl_xor_sync(0xffffffffu, dab, 1);
+          dab += __shfl_xor_sync(0xffffffffu, dab, 2);
+          if (a.need_bc) {  // dB_t += x'_t λ_t, dC_t += g_t h_t, quad after quad
+            for (int gq = 0; gq < 8; ++gq) {
+              if (g == gq && fb[c]) {
+#pragma unroll
+                for (int nt = 0; nt < kNT; ++nt) {
+#pragma unroll
+                  for (int e = 0; e < 2; ++e) {
+                    const int n = 8 * nt + 2 * tg + e;
+                    const float bv = bf16_to_f32(st.Bs[n * kLdS + t]);
+                    ws.red[t * N + n] += xts * lam[nt][e];
+                    ws.red[16 * N + t * N + n] += gts * fmaf(ab, hp[nt][e], xts * bv);
+                  }
+                }
+              }
+              __syncwarp();
+            }
+          }
+          if (tg == to) {
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj)
+              if (jj == jo) {
+                yso[jj] = yp;
+                dxo[jj] = dx;
+                dao[jj] = ab * dab;  // Ā_t dL/dĀ_t: dΔ_t = A times this, dA += Δ_t times this
+              }
+          }
+#pragma unroll
+          for (int nt = 0; nt < kNT; ++nt) {
+            lam[nt][0] *= ab;
+            lam[nt][1] *= ab;
+          }
+        }
+        if (fb[c]) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            ys[c][j] = yso[j];
+            dxp[c][j] = dxo[j];
+            da[c][j] = dao[j];
+          }
+#pragma unroll
+          for (int nt = 0; nt < kNT; ++nt) {  // dL/dh_in: the adjoint before step 0
+            mu[nt][2 * c] = lam[nt][0];
+            mu[nt][2 * c + 1] = lam[nt][1];
+          }
+        }
+      }
+    }
+
+    // ---- carry μ back to the previous chunk: μ <- e^{a_15} μ + (g E) C   (fallback channels
+    // already hold their carried adjoint and contribute zero (g E) rows)
+#pragma unroll
+    for (int nt = 0; nt < kNT; nt += 2) {
+      uint32_t cn[4];
+      ldsm_x4(cn, blk(st.Cs, 8 * nt, lane));
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float sc = fb[e >> 1] ? 1.f : Eend[e >> 1];
+        mu[nt][e] *= sc;
+        mu[nt + 1][e] *= sc;
+      }
+      mma16816(mu[nt], geA[0], geA[1], geA[2], geA[3], cn[0], cn[1]);
+      mma16816(mu[nt + 1], geA[0], geA[1], geA[2], geA[3], cn[2], cn[3]);
+      mma16816(mu[nt], gel[0], gel[1], gel[2], gel[3], cn[0], cn[1]);
+      mma16816(mu[nt + 1], gel[0], gel[1], gel[2], gel[3], cn[2], cn[3]);
+    }
+
+    // ---- dL/da and its reverse cumulative sum over the chunk (not for fallback channels,
+    // whose da already is A-free dΔ / A per step)
+    float dS[2][4];
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      if (!fb[c]) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) da[c][j] = fmaf(gg[c][j], ys[c][j], -xv[c][j] * dxp[c][j]);
+        if (tg == 3) da[c][3] += muh[c];  // step 15: h_out depends on a_15
+      }
+      const float p = da[c][0] + da[c][1], q = da[c][2] + da[c][3];
+      float ip = p, iq = q;  // suffix sums over the quad (lanes tg .. 3)
+#pragma unroll
+      for (int off = 1; off < 4; off <<= 1) {
+        const float np = __shfl_down_sync(0xffffffffu, ip, off, 4);
+        const float nq = __shfl_down_sync(0xffffffffu, iq, off, 4);
+        if (tg + off < 4) {
+          ip += np;
+          iq += nq;
+        }
+      }
+      const float hi_total = __shfl_sync(0xffffffffu, iq, 0, 4);
+      dS[c][2] = iq;
+      dS[c][3] = iq - da[c][2];
+      dS[c][0] = hi_total + ip;
+      dS[c][1] = hi_total + ip - da[c][0];
+      if (fb[c]) {  // fallback: dΔ_t = A Ā_t dL/dĀ_t per step, no sum over later steps
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dS[c][j] = da[c][j];
+      }
+    }
+
+    // ---- the channel gradients of the chunk's steps
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const float A = al[c] * kLn2;
+      uint32_t wdu[2], wdd[2], wdz[2];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        float vdu[2], vdd[2], vdz[2];
+#pragma unroll
+        for (int od = 0; od < 2; ++od) {
+          const int j = 2 * hh + od;
+          const float dD = fmaf(A, dS[c][j], dxp[c][j] * uv[c][j]);  // dL/dΔ_t
+          vdd[od] = dD * sg[c][j];                                     // through softplus
+          vdu[od] = fmaf(dxp[c][j], dl[c][j], Dd[c] * gg[c][j]);
+          const float y = fmaf(Dd[c], uv[c][j], ys[c][j]);
+          // dz = dout y silu'(z), silu'(z) = σ(z) (1 + z (1 - σ(z)))
+          vdz[od] = a.z ? gd[c][j] * y * gz[c][j] * fmaf(zz[c][j], 1.f - gz[c][j], 1.f) : 0.f;
+          // dA: Σ_t S_t dL/da_t; a fallback chunk's da holds Ā_t dL/dĀ_t, so Δ_t times it
+          accA[c] = fmaf(da[c][j], fb[c] ? dl[c][j] : S[c][j], accA[c]);
+          accD[c] = fmaf(gg[c][j], uv[c][j], accD[c]);
+          if (lv[c][j]) accT[c] += vdd[od];
+        }
+        wdu[hh] = pack_bf16x2(vdu[0], vdu[1]);
+        wdd[hh] = pack_bf16x2(vdd[0], vdd[1]);
+        wdz[hh] = pack_bf16x2(vdz[0], vdz[1]);
+      }
+      if (!act[c]) continue;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const long long t = t0 + 2 * tg + 8 * hh;
+        const auto put = [&](uint16_t* base, uint32_t w) {
+          if (!base) return;
+          if (vec_rows && t0 + kT <= L) {
+            *reinterpret_cast<uint32_t*>(base + row[c] + t) = w;
+          } else {
+            if (t < L) base[row[c] + t] = (uint16_t)(w & 0xffffu);
+            if (t + 1 < L) base[row[c] + t + 1] = (uint16_t)(w >> 16);
+          }
+        };
+        put(a.du, wdu[hh]);
+        put(a.ddelta, wdd[hh]);
+        if (a.z) put(a.dz, wdz[hh]);
+      }
+    }
+
+    // ---- the CTA's dB, dC of the chunk: its warps' tiles summed in warp order
+    if (a.need_bc) {
+      __syncthreads();  // every warp's tile is complete
+      // the CTA's sum over its warps, in warp order, into part_bc [ctag][b][which][n][t]
+      const int nvalid = min(kT, L - t0);
+      for (int p = tid; p < 2 * N * kT; p += 32 * kWb) {
+        const int which = p / (N * kT), rem = p % (N * kT), n = rem / kT, t = rem % kT;
+        float s = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWb; ++w) s += sm.w[w].red[which * 16 * N + t * N + n];
+        if (t < nvalid)
+          a.part_bc[((((long long)ctag * a.batch + b) * 2 + which) * N + n) * L + t0 + t] = s;
+      }
+    }
+  }
+  cp_wait<0>();
+
+  // dh0 and the per-channel parameter gradients
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    float vA = accA[c], vD = accD[c], vT = accT[c];
+    vA += __shfl_xor_sync(0xffffffffu, vA, 1);
+    vA += __shfl_xor_sync(0xffffffffu, vA, 2);
+    vD += __shfl_xor_sync(0xffffffffu, vD, 1);
+    vD += __shfl_xor_sync(0xffffffffu, vD, 2);
+    vT += __shfl_xor_sync(0xffffffffu, vT, 1);
+    vT += __shfl_xor_sync(0xffffffffu, vT, 2);
+    if (!act[c]) continue;
+    const long long ch = (long long)b * a.dim + dch[c];
+    if (a.dh0) {
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt) {
+        a.dh0[ch * N + 8 * nt + 2 * tg] = mu[nt][2 * c];
+        a.dh0[ch * N + 8 * nt + 2 * tg + 1] = mu[nt][2 * c + 1];
+      }
+    }
+    if (tg == 0) {
+      a.part_adt[ch * 3 + 0] = vA;
+      a.part_adt[ch * 3 + 1] = vD;
+      a.part_adt[ch * 3 + 2] = vT;
+    }
+  }
+}
+
+// dB, dC: each B/C group's CTAs summed in CTA order.
+__global__ void ssd_finish_bc(const SsdBwdArgs a, uint16_t* dB, uint16_t* dC, int ctas) {
+  const long long total = (long long)a.batch * a.bc_groups * 2 * a.N * a.L;
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= total) return;
+  const int t = (int)(i % a.L);
+  long long r = i / a.L;
+  const int n = (int)(r % a.N);
+  r /= a.N;
+  const int which = (int)(r % 2);
+  r /= 2;
+  const int gb = (int)(r % a.bc_groups);
+  const int b = (int)(r / a.bc_groups);
+  const int per = ctas / a.bc_groups;
+  float s = 0.f;
+  for (int cg = gb * per; cg < (gb + 1) * per; ++cg)
+    s += a.part_bc[((((long long)cg * a.batch + b) * 2 + which) * a.N + n) * a.L + t];
+  uint16_t* dst = which == 0 ? dB : dC;
+  if (dst) dst[(((long long)b * a.bc_groups + gb) * a.N + n) * a.L + t] = f32_to_bf16(s);
+}
+
+// dA, dD, ddt_bias: the rows' partials summed in row order.
+__global__ void ssd_finish_adt(const SsdBwdArgs a, float* dA, float* dD, float* ddt_bias) {
+  const int d = blockIdx.x * blockDim.x + threadIdx.x;
+  if (d >= a.dim) return;
+  float s[3] = {0.f, 0.f, 0.f};
+  for (int b = 0; b < a.batch; ++b)
+#pragma unroll
+    for (int k = 0; k < 3; ++k) s[k] += a.part_adt[((long long)b * a.dim + d) * 3 + k];
+  if (dA) dA[d] = s[0];
+  if (dD) dD[d] = s[1];
+  if (ddt_bias) ddt_bias[d] = s[2];
+}
+
+template <int N>
+cudaError_t launch_n(const SsdBwdArgs& a, cudaStream_t s) {
+  const unsigned grid = (unsigned)((long long)a.batch * ((a.dim + 16 * kWb - 1) / (16 * kWb)));
+  const size_t smem = sizeof(BwdSmem<N>);
+  auto k = ssd_bwd_kernel<N>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k<<<grid, 32 * kWb, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int ssd_bwd_ctas_per_row(int dim) { return (dim + 16 * kWb - 1) / (16 * kWb); }
+
+cudaError_t launch_ssd_bwd(const SsdBwdArgs& a, cudaStream_t s) {
+  switch (a.N) {
+    case 16: return launch_n<16>(a, s);
+    case 32: return launch_n<32>(a, s);
+    case 64: return launch_n<64>(a, s);
+    case 128: return launch_n<128>(a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_ssd_bwd_finish(const SsdBwdArgs& a, void* dB, void* dC, float* dA, float* dD,
+                                  float* ddt_bias, cudaStream_t s) {
+  if (dB || dC) {
+    const long long total = (long long)a.batch * a.bc_groups * 2 * a.N * a.L;
+    ssd_finish_bc<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
+        a, reinterpret_cast<uint16_t*>(dB), reinterpret_cast<uint16_t*>(dC),
+        ssd_bwd_ctas_per_row(a.dim));
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  ssd_finish_adt<<<(unsigned)((a.dim + 255) / 256), 256, 0, s>>>(a, dA, dD, ddt_bias);
+  return cudaGetLastError();
+}
+
+}  // namespace ssm

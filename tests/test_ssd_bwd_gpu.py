@@ -1,8 +1,9 @@
 """Backward of the scalar-decay scan with N = 32, 64, 128 (the Mamba-2 state sizes of the "2024
-Reading List: Neural Network" page).  The states of a scalar-decay scan do not interact, so the
-library runs it as a sum over 16-state slices; every gradient is compared with the fp64
-oracle's chain-rule gradients (A broadcast over the states, dA summed over them), with dhL, h0,
-the ZOH input term, the reverse scan and grouped B/C."""
+Reading List: Neural Network" page).  bf16 calls in the default direction run the chunked
+matrix form on the tensor cores; f32, reverse and ZOH calls (and SSM_SCALAR_BWD=slices) run the
+sum over 16-state slices (the states of a scalar-decay scan do not interact).  Every gradient is
+compared with the fp64 oracle's chain-rule gradients (A broadcast over the states, dA summed
+over them), with dhL, h0, the ZOH input term, the reverse scan and grouped B/C."""
 import numpy as np
 import pytest
 import torch
@@ -75,8 +76,8 @@ def test_variants(variant):
 
 
 def test_forward_then_backward_shapes_agree():
-    """The N = 64 forward (chunked matrix form) and backward (sum of slices) take the same
-    tensors; checkpoints are refused for N > 16 (the backward recomputes its states)."""
+    """The N = 64 forward and backward (both in the chunked matrix form) take the same tensors;
+    checkpoints are refused for N > 16 (the backward recomputes its states)."""
     x = inputs(1, 64, 64, 64, torch.bfloat16, seed=103)
     xd = {k: v.to(DEV) for k, v in x.items()}
     out = ssm.ssm_scan_fwd_scalar_a(xd["u"], xd["delta"], xd["A"], xd["B"], xd["C"], D=xd["D"],
@@ -87,3 +88,53 @@ def test_forward_then_backward_shapes_agree():
         ssm.ssm_scan_bwd_scalar_a(xd["u"], xd["delta"], xd["A"], xd["B"], xd["C"], xd["dout"],
                                   D=xd["D"], z=xd["z"], dt_bias=xd["dt_bias"], h0=xd["h0"],
                                   ckpt=fake_ck)
+
+
+# ------------------------------------------------------------------ the chunked-form backward
+@pytest.mark.parametrize("N", [32, 64, 128])
+@pytest.mark.parametrize("shape", [(2, 128, 160), (1, 80, 333), (2, 64, 17)])
+def test_chunked_backward_matches_oracle(monkeypatch, N, shape):
+    """bf16 scalar decay with N > 16 runs the chunked-form backward (tensor cores): partial
+    64-channel tiles, ragged time tails, dhL and h0."""
+    monkeypatch.delenv("SSM_SCALAR_BWD", raising=False)
+    batch, dim, L = shape
+    x = inputs(batch, dim, L, N, torch.bfloat16, seed=111)
+    dhL = torch.randn((batch, dim, N), generator=torch.Generator().manual_seed(9))
+    g = run(x, dhL)
+    r = ref(x, dhL)
+    for k in GRADS:
+        assert_close(g[k], r[k], torch.bfloat16, k)
+
+
+def test_chunked_and_slice_backwards_agree(monkeypatch):
+    x = inputs(2, 128, 200, 64, torch.bfloat16, seed=112)
+    monkeypatch.delenv("SSM_SCALAR_BWD", raising=False)
+    a = run(x, None)
+    monkeypatch.setenv("SSM_SCALAR_BWD", "slices")
+    b = run(x, None)
+    for k in GRADS:
+        assert_close(a[k], f64(b[k]), torch.bfloat16, k)
+
+
+def test_chunked_backward_range_fallback():
+    """Steps over v = delta + dt_bias in [-30, 30]: chunks leave the factorisation's range and
+    take the exact sequential pass inside the chunked backward."""
+    x = inputs(1, 64, 96, 64, torch.bfloat16, seed=113)
+    v = np.random.default_rng(4).uniform(-30, 30, size=x["delta"].shape).astype(np.float32)
+    x["delta"] = torch.from_numpy(v).to(torch.bfloat16)
+    x["dt_bias"] = torch.zeros_like(x["dt_bias"])
+    g = run(x, None)
+    r = ref(x, None)
+    for k in GRADS:
+        # dA, ddt_bias sum many terms of very different size here (steps up to 30)
+        scale = 5.0 if k in ("dA", "ddt_bias", "dD") else 1.0
+        assert_close(g[k], r[k], torch.bfloat16, k, scale=scale)
+
+
+def test_chunked_backward_with_time_split_checkpoints():
+    """64 channels over 2048 steps: the checkpoint pass splits time by itself."""
+    x = inputs(1, 64, 2048, 64, torch.bfloat16, seed=114)
+    g = run(x, None)
+    r = ref(x, None)
+    for k in GRADS:
+        assert_close(g[k], r[k], torch.bfloat16, k)
