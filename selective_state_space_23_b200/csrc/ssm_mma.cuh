@@ -37,6 +37,23 @@ __device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uin
   lo = pack_bf16x2(a - bf16_lo(hi), b - bf16_hi(hi));
 }
 
+// The transpose of an 8x8 b16 matrix held one pair per lane (lane l: row l / 4, cols 2 (l % 4),
+// +1), returned in the same layout.
+__device__ __forceinline__ uint32_t movt(uint32_t a) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(d) : "r"(a));
+  return d;
+}
+// A 16x16 tile held as an A fragment ({rows 0-7 | 8-15} x {cols 0-7 | 8-15}: a[0] rows lo cols
+// lo, a[1] rows hi cols lo, a[2] rows lo cols hi, a[3] rows hi cols hi) -> the A fragment of
+// its transpose (what ldmatrix .trans of the tile in shared memory would give).
+__device__ __forceinline__ void frag_t(uint32_t (&r)[4], const uint32_t (&a)[4]) {
+  r[0] = movt(a[0]);
+  r[1] = movt(a[2]);
+  r[2] = movt(a[1]);
+  r[3] = movt(a[3]);
+}
+
 // Four 8x8 bf16 matrices from shared memory; lane i gives the address of row i % 8 of matrix
 // i / 8.  Plain: lane l receives (row l / 4, cols 2 (l % 4), +1) of each; .trans: the transpose.
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {

@@ -32,8 +32,11 @@
 // over the warp's 16 channels by the tensor cores (the contractions over d), over the CTA's
 // warps in shared memory in a fixed order, and over CTAs by a finishing kernel in a fixed order,
 // so the result is bitwise reproducible.  A channel whose chunk leaves the factorisation's range
-// (as in the forward) takes no part in that chunk's products and is computed by an exact
-// sequential pass over the states its quad holds.
+// (as in the forward: P or Q would overflow) takes no part in the three products that use P and
+// Q (Y1, dX', M); its share of them is computed with the exact decay e^{a_t - a_s} of every
+// (t, s) pair in the same accumulator layouts (16 exponentials per lane and channel).  Every
+// other term uses E_t = e^{a_t} and e^{a_15 - a_s} directly, which stay <= 1, so the rest of the
+// chunk (dL/da, the carry, dB, dC) is the same for every channel.
 #include <stdint.h>
 #include <stdlib.h>
 
@@ -50,14 +53,10 @@ constexpr int kWb = 4;  // warps per CTA (64 channels of one batch row and B/C g
 
 template <int N>
 struct BwdWarpSmem {
-  static constexpr int kLdN = N + 8;  // bf16 row stride of the [16][N] tiles
-  uint16_t x1[16 * kLdS];   // Q x'          [d][s]
-  uint16_t x2[16 * kLdS];   // e^{a15-am} Q x' [d][s]
-  uint16_t gp[16 * kLdS];   // g P           [d][t]
-  uint16_t ge[16 * kLdS];   // g E           [d][t]
-  uint16_t mu[16 * kLdN];   // μ (before this chunk's update) [d][n]
-  uint16_t hin[16 * kLdN];  // h_in          [d][n]
   float red[2 * 16 * N];    // this warp's dB, dC of the chunk: [which][t][n]
+  // channels outside the factorisation's range: a_t (log2 units), x'_t, g_t per [d][t], and
+  // their exact y1, xy per [d][t]
+  float fa[16 * kT], fx[16 * kT], fg[16 * kT], fy[16 * kT], fxy[16 * kT];
 };
 
 template <int N>
@@ -81,7 +80,6 @@ __device__ __forceinline__ float pick(uint32_t w, int odd) { return odd ? bf16_h
 template <int N>
 __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant__ SsdBwdArgs a) {
   constexpr int kNT = N / 8;
-  constexpr int LDN = BwdWarpSmem<N>::kLdN;
   extern __shared__ float4 smem_sb[];
   BwdSmem<N>& sm = *reinterpret_cast<BwdSmem<N>*>(smem_sb);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -252,10 +250,13 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
       ok &= __shfl_xor_sync(0xffffffffu, ok, 2, 4);
       fb[c] = ok == 0;
     }
-    float P[2][4], Qv[2][4], E[2][4], eEm[2], Eend[2];
+    // decay factors: P, Q about the middle step for the factorised products; E_t = e^{a_t} and
+    // e^{a_15 - a_s} directly for channels outside the range (both <= 1)
+    float P[2][4], Qv[2][4], E[2][4], eEm[2], Eend[2], Ef[2][4];
+    float q2f[2][4];  // e^{a_15 - a_s} x'_s in f32
     // A fragments (bf16 pairs) and, for the products that feed dΔ, dA and the carried adjoint,
     // the remainders (suffix l)
-    uint32_t x1[4], x2[4], gpA[4], geA[4], x1l[4], gpl[4], gel[4];
+    uint32_t x1[4], x2[4], gpA[4], geA[4], x1l[4], x2l[4], gpl[4], gel[4];
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       const float eAm = ex2_mufu(Sm[c] * al[c]);
@@ -267,42 +268,32 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
         const float r = (S[c][j] - Sm[c]) * al[c];
         P[c][j] = ex2_mufu(r);
         Qv[c][j] = ex2_mufu(-r);
-        E[c][j] = eAm * P[c][j];
-        q1[j] = fb[c] ? 0.f : Qv[c][j] * xv[c][j];
-        q2[j] = fb[c] ? 0.f : eEm[c] * q1[j];
-        gp[j] = fb[c] ? 0.f : gg[c][j] * P[c][j];
-        ge[j] = fb[c] ? 0.f : gg[c][j] * E[c][j];
+        if (fb[c]) {
+          E[c][j] = ex2_mufu(S[c][j] * al[c]);
+          Ef[c][j] = ex2_mufu((Se[c] - S[c][j]) * al[c]);
+          q1[j] = 0.f;
+          q2[j] = Ef[c][j] * xv[c][j];
+          gp[j] = 0.f;
+        } else {
+          E[c][j] = eAm * P[c][j];
+          Ef[c][j] = 0.f;
+          q1[j] = Qv[c][j] * xv[c][j];
+          q2[j] = eEm[c] * q1[j];
+          gp[j] = gg[c][j] * P[c][j];
+        }
+        ge[j] = gg[c][j] * E[c][j];
       }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) q2f[c][j] = q2[j];
       split_bf16x2(q1[0], q1[1], x1[c], x1l[c]);
       split_bf16x2(q1[2], q1[3], x1[2 + c], x1l[2 + c]);
-      x2[c] = pack_bf16x2(q2[0], q2[1]);
-      x2[2 + c] = pack_bf16x2(q2[2], q2[3]);
+      split_bf16x2(q2[0], q2[1], x2[c], x2l[c]);
+      split_bf16x2(q2[2], q2[3], x2[2 + c], x2l[2 + c]);
       split_bf16x2(gp[0], gp[1], gpA[c], gpl[c]);
       split_bf16x2(gp[2], gp[3], gpA[2 + c], gpl[2 + c]);
       split_bf16x2(ge[0], ge[1], geA[c], gel[c]);
       split_bf16x2(ge[2], ge[3], geA[2 + c], gel[2 + c]);
     }
-    // per-warp tiles: rows d = g + 8 c, columns 2 tg + 8 hh
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int o = (g + 8 * c) * kLdS + 2 * tg + 8 * hh;
-        *reinterpret_cast<uint32_t*>(ws.x1 + o) = x1[2 * hh + c];
-        *reinterpret_cast<uint32_t*>(ws.x2 + o) = x2[2 * hh + c];
-        *reinterpret_cast<uint32_t*>(ws.gp + o) = gpA[2 * hh + c];
-        *reinterpret_cast<uint32_t*>(ws.ge + o) = geA[2 * hh + c];
-      }
-#pragma unroll
-      for (int nt = 0; nt < kNT; ++nt) {
-        const int o = (g + 8 * c) * LDN + 8 * nt + 2 * tg;
-        const float2 hv = hck(c, k, nt);
-        *reinterpret_cast<uint32_t*>(ws.hin + o) = pack_bf16x2(hv.x, hv.y);
-        *reinterpret_cast<uint32_t*>(ws.mu + o) = pack_bf16x2(mu[nt][2 * c], mu[nt][2 * c + 1]);
-      }
-    }
-    __syncwarp();
-
     // ---- recompute G (rows t) and G^T (rows s), Y2' = H_in C^T; and μ B^T, per 16 states
     // (H_in and μ split into bf16 pairs and remainders; B, C are exact bf16 inputs)
     float G[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -355,12 +346,11 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
     // dX' (y part) = (g P) mask(G): B fragments (k = t, n = s) from G^T's accumulators (rows s)
     float Xy[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
     {
-      const int t0l = 2 * tg;
       uint32_t b00, b01, b10, b11, l00, l01, l10, l11;
-      split_bf16x2(msk(GT[0][0], g, t0l), msk(GT[0][1], g, t0l + 1), b00, l00);
-      split_bf16x2(msk(GT[1][0], g, t0l + 8), msk(GT[1][1], g, t0l + 9), b01, l01);
-      split_bf16x2(msk(GT[0][2], g + 8, t0l), msk(GT[0][3], g + 8, t0l + 1), b10, l10);
-      split_bf16x2(msk(GT[1][2], g + 8, t0l + 8), msk(GT[1][3], g + 8, t0l + 9), b11, l11);
+      split_bf16x2(msk(GT[0][0], g, s0), msk(GT[0][1], g, s0 + 1), b00, l00);
+      split_bf16x2(msk(GT[1][0], g, s0 + 8), msk(GT[1][1], g, s0 + 9), b01, l01);
+      split_bf16x2(msk(GT[0][2], g + 8, s0), msk(GT[0][3], g + 8, s0 + 1), b10, l10);
+      split_bf16x2(msk(GT[1][2], g + 8, s0 + 8), msk(GT[1][3], g + 8, s0 + 9), b11, l11);
       mma16816(Xy[0], gpA[0], gpA[1], gpA[2], gpA[3], b00, b01);
       mma16816(Xy[1], gpA[0], gpA[1], gpA[2], gpA[3], b10, b11);
       mma16816(Xy[0], gpA[0], gpA[1], gpA[2], gpA[3], l00, l01);
@@ -368,17 +358,110 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
       mma16816(Xy[0], gpl[0], gpl[1], gpl[2], gpl[3], b00, b01);
       mma16816(Xy[1], gpl[0], gpl[1], gpl[2], gpl[3], b10, b11);
     }
-    // μ . h_out of each channel (before μ is carried back), summed over the quad's states;
-    // h_out is the state entering chunk k + 1
+    // M[s][t] = Σ_d X1'[d][s] (gP)[d][t] and its transpose Mt[t][s] (for dB, dC); the
+    // transposed operands are built in registers (movmatrix), bf16 pairs and remainders
+    float M[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    float Mt[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    if (a.need_bc) {
+      uint32_t x1T[4], gpT[4], x1Tl[4], gpTl[4];
+      frag_t(x1T, x1);
+      frag_t(gpT, gpA);
+      frag_t(x1Tl, x1l);
+      frag_t(gpTl, gpl);
+      const auto mm3 = [](float (&acc)[4], const uint32_t (&ah)[4], const uint32_t (&al_)[4],
+                          uint32_t bh0, uint32_t bh1, uint32_t bl0, uint32_t bl1) {
+        mma16816(acc, ah[0], ah[1], ah[2], ah[3], bh0, bh1);
+        mma16816(acc, ah[0], ah[1], ah[2], ah[3], bl0, bl1);
+        mma16816(acc, al_[0], al_[1], al_[2], al_[3], bh0, bh1);
+      };
+      mm3(M[0], x1T, x1Tl, gpT[0], gpT[2], gpTl[0], gpTl[2]);
+      mm3(M[1], x1T, x1Tl, gpT[1], gpT[3], gpTl[1], gpTl[3]);
+      mm3(Mt[0], gpT, gpTl, x1T[0], x1T[2], x1Tl[0], x1Tl[2]);
+      mm3(Mt[1], gpT, gpTl, x1T[1], x1T[3], x1Tl[1], x1Tl[3]);
+    }
+
+    // ---- channels outside the factorisation's range this chunk (x1, gP rows zero above): their
+    // intra-chunk products with the exact decay e^{a_t - a_s} per (t, s) pair, in the same
+    // accumulator layouts as G (rows t) and G^T (rows s): y1[t] = Σ_{s<=t} e^{a_t-a_s} G_ts x'_s,
+    // xy[s] = Σ_{t>=s} g_t e^{a_t-a_s} G_ts, and the channel's share of M, Mt.
+    bool fixed = false;
+    {
+      const unsigned q0 = __ballot_sync(0xffffffffu, fb[0] && tg == 0);
+      const unsigned q1 = __ballot_sync(0xffffffffu, fb[1] && tg == 0);
+      unsigned fbm = 0;  // bit d: channel d of the warp (d = g + 8 c)
+#pragma unroll
+      for (int gq = 0; gq < 8; ++gq) fbm |= (((q0 >> (4 * gq)) & 1u) << gq) | (((q1 >> (4 * gq)) & 1u) << (gq + 8));
+      if (fbm) {
+        fixed = true;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int t = 2 * tg + (j & 1) + 8 * (j >> 1), o = (g + 8 * c) * kT + t;
+            ws.fa[o] = S[c][j] * al[c];
+            ws.fx[o] = xv[c][j];
+            ws.fg[o] = gg[c][j];
+          }
+        }
+        __syncwarp();
+        for (unsigned m = fbm; m; m &= m - 1) {
+          const int d = __ffs(m) - 1;
+          const float* ad = ws.fa + d * kT;
+          const float* xd = ws.fx + d * kT;
+          const float* gd_ = ws.fg + d * kT;
+          float yr[2] = {0.f, 0.f}, xr[2] = {0.f, 0.f};
+#pragma unroll
+          for (int T = 0; T < 2; ++T) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int r = g + 8 * (e >> 1), cidx = 8 * T + 2 * tg + (e & 1);
+              // G layout: t = r, s = cidx
+              const float Lg = cidx <= r ? ex2_mufu(ad[r] - ad[cidx]) : 0.f;
+              yr[e >> 1] = fmaf(Lg * G[T][e], xd[cidx], yr[e >> 1]);
+              // G^T layout: s = r, t = cidx
+              const float Lt = r <= cidx ? ex2_mufu(ad[cidx] - ad[r]) : 0.f;
+              xr[e >> 1] = fmaf(gd_[cidx] * Lt, GT[T][e], xr[e >> 1]);
+              if (a.need_bc) {
+                Mt[T][e] = fmaf(Lg * gd_[r], xd[cidx], Mt[T][e]);
+                M[T][e] = fmaf(Lt * xd[r], gd_[cidx], M[T][e]);
+              }
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            yr[i] += __shfl_xor_sync(0xffffffffu, yr[i], 1);
+            yr[i] += __shfl_xor_sync(0xffffffffu, yr[i], 2);
+            xr[i] += __shfl_xor_sync(0xffffffffu, xr[i], 1);
+            xr[i] += __shfl_xor_sync(0xffffffffu, xr[i], 2);
+          }
+          if (tg == 0) ws.fy[d * kT + g] = yr[0];
+          if (tg == 1) ws.fy[d * kT + g + 8] = yr[1];
+          if (tg == 2) ws.fxy[d * kT + g] = xr[0];
+          if (tg == 3) ws.fxy[d * kT + g + 8] = xr[1];
+        }
+        __syncwarp();
+      }
+    }
+
+    // μ . h_out of each channel (μ before it is carried back), with h_out written out as the
+    // recurrence makes it: e^{a_15} μ.h_in + Σ_s e^{a_15 - a_s} x'_s (μ.B_s).  The x' dL/dx'
+    // terms of dL/da subtract the same products (q2f Xm), so as the decay grows the two cancel
+    // term by term instead of leaving the difference of two separately rounded sums.
     float muh[2] = {0.f, 0.f};
 #pragma unroll
     for (int nt = 0; nt < kNT; ++nt) {
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        const float2 ho = hck(c, k + 1, nt);
-        muh[c] = fmaf(mu[nt][2 * c], ho.x, fmaf(mu[nt][2 * c + 1], ho.y, muh[c]));
+        const float2 hv = hck(c, k, nt);
+        muh[c] = fmaf(mu[nt][2 * c], hv.x, fmaf(mu[nt][2 * c + 1], hv.y, muh[c]));
       }
     }
+#pragma unroll
+    for (int c = 0; c < 2; ++c) muh[c] *= Eend[c];
+#pragma unroll
+    for (int T = 0; T < 2; ++T)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) muh[e >> 1] = fmaf(q2f[e >> 1][2 * T + (e & 1)], Xm[T][e], muh[e >> 1]);
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       muh[c] += __shfl_xor_sync(0xffffffffu, muh[c], 1);
@@ -392,192 +475,89 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int c = e >> 1, j = 2 * T + (e & 1);
-        ys[c][j] = fmaf(P[c][j], Y1[T][e], E[c][j] * Y2[T][e]);
-        dxp[c][j] = Qv[c][j] * fmaf(eEm[c], Xm[T][e], Xy[T][e]);
+        if (fixed && fb[c]) {
+          const int o = (g + 8 * c) * kT + 2 * tg + (e & 1) + 8 * T;
+          ys[c][j] = fmaf(E[c][j], Y2[T][e], ws.fy[o]);
+          dxp[c][j] = fmaf(Ef[c][j], Xm[T][e], ws.fxy[o]);
+        } else {
+          ys[c][j] = fmaf(P[c][j], Y1[T][e], E[c][j] * Y2[T][e]);
+          dxp[c][j] = Qv[c][j] * fmaf(eEm[c], Xm[T][e], Xy[T][e]);
+        }
       }
     }
 
-    // ---- dB, dC of the chunk summed over the warp's channels on the tensor cores, then over
-    // the CTA's warps (fixed order) into this CTA's partial
+    // ---- dB, dC of the chunk summed over the warp's channels on the tensor cores (every
+    // operand that is not a B/C input as a bf16 pair plus remainder), then over the CTA's warps
+    // (fixed order) into this CTA's partial
     if (a.need_bc) {
-      uint32_t x1T[4], x2T[4], gpT[4], geT[4];
-      ldsm_x4_t(x1T, blk(ws.x1, 0, lane));
-      ldsm_x4_t(x2T, blk(ws.x2, 0, lane));
-      ldsm_x4_t(gpT, blk(ws.gp, 0, lane));
-      ldsm_x4_t(geT, blk(ws.ge, 0, lane));
-      // M[s][t] = Σ_d X1'[d][s] (gP)[d][t] and its transpose Mt[t][s]
-      float M[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-      float Mt[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-      mma16816(M[0], x1T[0], x1T[1], x1T[2], x1T[3], gpT[0], gpT[2]);
-      mma16816(M[1], x1T[0], x1T[1], x1T[2], x1T[3], gpT[1], gpT[3]);
-      mma16816(Mt[0], gpT[0], gpT[1], gpT[2], gpT[3], x1T[0], x1T[2]);
-      mma16816(Mt[1], gpT[0], gpT[1], gpT[2], gpT[3], x1T[1], x1T[3]);
+      uint32_t x2T[4], geT[4], x2Tl[4], geTl[4];
+      frag_t(x2T, x2);
+      frag_t(geT, geA);
+      frag_t(x2Tl, x2l);
+      frag_t(geTl, gel);
       // M masked to t >= s as A fragments (rows s, k = t); Mt masked to s <= t (rows t, k = s)
-      const int t0l = 2 * tg;
-      const uint32_t ma0 = pack_bf16x2(msk(M[0][0], g, t0l), msk(M[0][1], g, t0l + 1));
-      const uint32_t ma1 = pack_bf16x2(msk(M[0][2], g + 8, t0l), msk(M[0][3], g + 8, t0l + 1));
-      const uint32_t ma2 = pack_bf16x2(msk(M[1][0], g, t0l + 8), msk(M[1][1], g, t0l + 9));
-      const uint32_t ma3 = pack_bf16x2(msk(M[1][2], g + 8, t0l + 8), msk(M[1][3], g + 8, t0l + 9));
-      const uint32_t mt0 = pack_bf16x2(msk(Mt[0][0], s0, g), msk(Mt[0][1], s0 + 1, g));
-      const uint32_t mt1 = pack_bf16x2(msk(Mt[0][2], s0, g + 8), msk(Mt[0][3], s0 + 1, g + 8));
-      const uint32_t mt2 = pack_bf16x2(msk(Mt[1][0], s0 + 8, g), msk(Mt[1][1], s0 + 9, g));
-      const uint32_t mt3 = pack_bf16x2(msk(Mt[1][2], s0 + 8, g + 8), msk(Mt[1][3], s0 + 9, g + 8));
+      uint32_t ma[4], mal[4], mt[4], mtl[4];
+      split_bf16x2(msk(M[0][0], g, s0), msk(M[0][1], g, s0 + 1), ma[0], mal[0]);
+      split_bf16x2(msk(M[0][2], g + 8, s0), msk(M[0][3], g + 8, s0 + 1), ma[1], mal[1]);
+      split_bf16x2(msk(M[1][0], g, s0 + 8), msk(M[1][1], g, s0 + 9), ma[2], mal[2]);
+      split_bf16x2(msk(M[1][2], g + 8, s0 + 8), msk(M[1][3], g + 8, s0 + 9), ma[3], mal[3]);
+      split_bf16x2(msk(Mt[0][0], s0, g), msk(Mt[0][1], s0 + 1, g), mt[0], mtl[0]);
+      split_bf16x2(msk(Mt[0][2], s0, g + 8), msk(Mt[0][3], s0 + 1, g + 8), mt[1], mtl[1]);
+      split_bf16x2(msk(Mt[1][0], s0 + 8, g), msk(Mt[1][1], s0 + 9, g), mt[2], mtl[2]);
+      split_bf16x2(msk(Mt[1][2], s0 + 8, g + 8), msk(Mt[1][3], s0 + 9, g + 8), mt[3], mtl[3]);
 #pragma unroll
       for (int nt = 0; nt < kNT; nt += 2) {
-        uint32_t cn[4], bn[4], mub[4], hib[4];
+        uint32_t cn[4], bn[4];
         ldsm_x4(cn, blk(st.Cs, 8 * nt, lane));
         ldsm_x4(bn, blk(st.Bs, 8 * nt, lane));
-        ldsm_x4_t(mub, blk(ws.mu + 8 * nt, 0, lane, LDN));
-        ldsm_x4_t(hib, blk(ws.hin + 8 * nt, 0, lane, LDN));
-        float dB0[4] = {0.f, 0.f, 0.f, 0.f}, dB1[4] = {0.f, 0.f, 0.f, 0.f};
-        float dC0[4] = {0.f, 0.f, 0.f, 0.f}, dC1[4] = {0.f, 0.f, 0.f, 0.f};
-        mma16816(dB0, ma0, ma1, ma2, ma3, cn[0], cn[1]);
-        mma16816(dB1, ma0, ma1, ma2, ma3, cn[2], cn[3]);
-        mma16816(dB0, x2T[0], x2T[1], x2T[2], x2T[3], mub[0], mub[2]);
-        mma16816(dB1, x2T[0], x2T[1], x2T[2], x2T[3], mub[1], mub[3]);
-        mma16816(dC0, mt0, mt1, mt2, mt3, bn[0], bn[1]);
-        mma16816(dC1, mt0, mt1, mt2, mt3, bn[2], bn[3]);
-        mma16816(dC0, geT[0], geT[1], geT[2], geT[3], hib[0], hib[2]);
-        mma16816(dC1, geT[0], geT[1], geT[2], geT[3], hib[1], hib[3]);
-        // rows (s or t) g, g+8; columns n = 8 nt' + 2 tg, +1
-        float* rb = ws.red;
-        float* rc = ws.red + 16 * N;
-        *reinterpret_cast<float2*>(rb + g * N + 8 * nt + 2 * tg) = make_float2(dB0[0], dB0[1]);
-        *reinterpret_cast<float2*>(rb + (g + 8) * N + 8 * nt + 2 * tg) = make_float2(dB0[2], dB0[3]);
-        *reinterpret_cast<float2*>(rb + g * N + 8 * nt + 8 + 2 * tg) = make_float2(dB1[0], dB1[1]);
-        *reinterpret_cast<float2*>(rb + (g + 8) * N + 8 * nt + 8 + 2 * tg) = make_float2(dB1[2], dB1[3]);
-        *reinterpret_cast<float2*>(rc + g * N + 8 * nt + 2 * tg) = make_float2(dC0[0], dC0[1]);
-        *reinterpret_cast<float2*>(rc + (g + 8) * N + 8 * nt + 2 * tg) = make_float2(dC0[2], dC0[3]);
-        *reinterpret_cast<float2*>(rc + g * N + 8 * nt + 8 + 2 * tg) = make_float2(dC1[0], dC1[1]);
-        *reinterpret_cast<float2*>(rc + (g + 8) * N + 8 * nt + 8 + 2 * tg) = make_float2(dC1[2], dC1[3]);
-      }
-    }
-    __syncwarp();  // this warp's dB, dC tile is written
-    const bool anyfb = __any_sync(0xffffffffu, fb[0] || fb[1]);
-    // ---- channels outside the factorisation's range this chunk: an exact sequential pass over
-    // the states each quad holds (rare).  Steps are walked backwards; the state before step t is
-    // recomputed from h_in.  Each step's dB, dC contributions are added to this warp's tile one
-    // quad at a time, in a fixed order.
-    if (anyfb) {
-      const int qb = lane & ~3;
-      const auto sel4 = [](const float (&v)[4], int j) {
-        return j == 0 ? v[0] : (j == 1 ? v[1] : (j == 2 ? v[2] : v[3]));
-      };
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        if (!__any_sync(0xffffffffu, fb[c])) continue;
-        float lam[kNT][2];
+        for (int q = 0; q < 2; ++q) {
+          // μ and h_in of n tile nt + q as B fragments (k = d, n): transposes of their
+          // accumulator-layout pairs (channel g + 8 c, states 8 (nt + q) + 2 tg, +1)
+          uint32_t mbh[2], mbl[2], hbh[2], hbl[2];
 #pragma unroll
-        for (int nt = 0; nt < kNT; ++nt) {
-          lam[nt][0] = mu[nt][2 * c];
-          lam[nt][1] = mu[nt][2 * c + 1];
-        }
-        float yso[4] = {0.f, 0.f, 0.f, 0.f}, dxo[4] = {0.f, 0.f, 0.f, 0.f}, dao[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-        for (int t = kT - 1; t >= 0; --t) {
-          const int to = (t & 7) >> 1, jo = (t & 1) + 2 * (t >> 3);  // owner lane, its index
-          const float dts = __shfl_sync(0xffffffffu, sel4(dl[c], jo), qb | to);
-          const float xts = __shfl_sync(0xffffffffu, sel4(xv[c], jo), qb | to);
-          const float gts = __shfl_sync(0xffffffffu, sel4(gg[c], jo), qb | to);
-          float hp[kNT][2];  // h_{t-1}: steps 0 .. t-1 replayed from h_in
-#pragma unroll
-          for (int nt = 0; nt < kNT; ++nt) {
-            const float2 hv = hck(c, k, nt);
-            hp[nt][0] = hv.x;
-            hp[nt][1] = hv.y;
+          for (int c = 0; c < 2; ++c) {
+            uint32_t h_, l_;
+            split_bf16x2(mu[nt + q][2 * c], mu[nt + q][2 * c + 1], h_, l_);
+            mbh[c] = movt(h_);
+            mbl[c] = movt(l_);
+            const float2 hv = hck(c, k, nt + q);
+            split_bf16x2(hv.x, hv.y, h_, l_);
+            hbh[c] = movt(h_);
+            hbl[c] = movt(l_);
           }
-#pragma unroll 1
-          for (int r = 0; r < t; ++r) {
-            const int ro = (r & 7) >> 1, rj = (r & 1) + 2 * (r >> 3);
-            const float dr = __shfl_sync(0xffffffffu, sel4(dl[c], rj), qb | ro);
-            const float xr = __shfl_sync(0xffffffffu, sel4(xv[c], rj), qb | ro);
-            const float abr = ex2_mufu(dr * al[c]);
-#pragma unroll
-            for (int nt = 0; nt < kNT; ++nt)
-#pragma unroll
-              for (int e = 0; e < 2; ++e)
-                hp[nt][e] = fmaf(abr, hp[nt][e], xr * bf16_to_f32(st.Bs[(8 * nt + 2 * tg + e) * kLdS + r]));
-          }
-          const float ab = ex2_mufu(dts * al[c]);
-          float yp = 0.f, dx = 0.f, dab = 0.f;
-#pragma unroll
-          for (int nt = 0; nt < kNT; ++nt) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int n = 8 * nt + 2 * tg + e;
-              const float bv = bf16_to_f32(st.Bs[n * kLdS + t]);
-              const float cv = bf16_to_f32(st.Cs[n * kLdS + t]);
-              yp = fmaf(cv, fmaf(ab, hp[nt][e], xts * bv), yp);
-              lam[nt][e] = fmaf(gts, cv, lam[nt][e]);  // λ_t = g_t C_t + Ā_{t+1} λ_{t+1}
-              dx = fmaf(lam[nt][e], bv, dx);
-              dab = fmaf(lam[nt][e], hp[nt][e], dab);  // dL/dĀ_t = λ_t . h_{t-1}
-            }
-          }
-          yp += __shfl_xor_sync(0xffffffffu, yp, 1);
-          yp += __shfl_xor_sync(0xffffffffu, yp, 2);
-          dx += __shfl_xor_sync(0xffffffffu, dx, 1);
-          dx += __shfl_xor_sync(0xffffffffu, dx, 2);
-          dab += __shfl_xor_sync(0xffffffffu, dab, 1);
-          dab += __shfl_xor_sync(0xffffffffu, dab, 2);
-          if (a.need_bc) {  // dB_t += x'_t λ_t, dC_t += g_t h_t, quad after quad
-            for (int gq = 0; gq < 8; ++gq) {
-              if (g == gq && fb[c]) {
-#pragma unroll
-                for (int nt = 0; nt < kNT; ++nt) {
-#pragma unroll
-                  for (int e = 0; e < 2; ++e) {
-                    const int n = 8 * nt + 2 * tg + e;
-                    const float bv = bf16_to_f32(st.Bs[n * kLdS + t]);
-                    ws.red[t * N + n] += xts * lam[nt][e];
-                    ws.red[16 * N + t * N + n] += gts * fmaf(ab, hp[nt][e], xts * bv);
-                  }
-                }
-              }
-              __syncwarp();
-            }
-          }
-          if (tg == to) {
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj)
-              if (jj == jo) {
-                yso[jj] = yp;
-                dxo[jj] = dx;
-                dao[jj] = ab * dab;  // Ā_t dL/dĀ_t: dΔ_t = A times this, dA += Δ_t times this
-              }
-          }
-#pragma unroll
-          for (int nt = 0; nt < kNT; ++nt) {
-            lam[nt][0] *= ab;
-            lam[nt][1] *= ab;
-          }
-        }
-        if (fb[c]) {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            ys[c][j] = yso[j];
-            dxp[c][j] = dxo[j];
-            da[c][j] = dao[j];
-          }
-#pragma unroll
-          for (int nt = 0; nt < kNT; ++nt) {  // dL/dh_in: the adjoint before step 0
-            mu[nt][2 * c] = lam[nt][0];
-            mu[nt][2 * c + 1] = lam[nt][1];
-          }
+          float dB[4] = {0.f, 0.f, 0.f, 0.f}, dC[4] = {0.f, 0.f, 0.f, 0.f};
+          mma16816(dB, ma[0], ma[1], ma[2], ma[3], cn[2 * q], cn[2 * q + 1]);
+          mma16816(dB, mal[0], mal[1], mal[2], mal[3], cn[2 * q], cn[2 * q + 1]);
+          mma16816(dB, x2T[0], x2T[1], x2T[2], x2T[3], mbh[0], mbh[1]);
+          mma16816(dB, x2T[0], x2T[1], x2T[2], x2T[3], mbl[0], mbl[1]);
+          mma16816(dB, x2Tl[0], x2Tl[1], x2Tl[2], x2Tl[3], mbh[0], mbh[1]);
+          mma16816(dC, mt[0], mt[1], mt[2], mt[3], bn[2 * q], bn[2 * q + 1]);
+          mma16816(dC, mtl[0], mtl[1], mtl[2], mtl[3], bn[2 * q], bn[2 * q + 1]);
+          mma16816(dC, geT[0], geT[1], geT[2], geT[3], hbh[0], hbh[1]);
+          mma16816(dC, geT[0], geT[1], geT[2], geT[3], hbl[0], hbl[1]);
+          mma16816(dC, geTl[0], geTl[1], geTl[2], geTl[3], hbh[0], hbh[1]);
+          // rows (s or t) g, g+8; columns n = 8 (nt + q) + 2 tg, +1
+          const int n = 8 * (nt + q) + 2 * tg;
+          float* rb = ws.red;
+          float* rc = ws.red + 16 * N;
+          *reinterpret_cast<float2*>(rb + g * N + n) = make_float2(dB[0], dB[1]);
+          *reinterpret_cast<float2*>(rb + (g + 8) * N + n) = make_float2(dB[2], dB[3]);
+          *reinterpret_cast<float2*>(rc + g * N + n) = make_float2(dC[0], dC[1]);
+          *reinterpret_cast<float2*>(rc + (g + 8) * N + n) = make_float2(dC[2], dC[3]);
         }
       }
     }
 
-    // ---- carry μ back to the previous chunk: μ <- e^{a_15} μ + (g E) C   (fallback channels
-    // already hold their carried adjoint and contribute zero (g E) rows)
+    // ---- carry μ back to the previous chunk: μ <- e^{a_15} μ + (g E) C
 #pragma unroll
     for (int nt = 0; nt < kNT; nt += 2) {
       uint32_t cn[4];
       ldsm_x4(cn, blk(st.Cs, 8 * nt, lane));
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float sc = fb[e >> 1] ? 1.f : Eend[e >> 1];
-        mu[nt][e] *= sc;
-        mu[nt + 1][e] *= sc;
+        mu[nt][e] *= Eend[e >> 1];
+        mu[nt + 1][e] *= Eend[e >> 1];
       }
       mma16816(mu[nt], geA[0], geA[1], geA[2], geA[3], cn[0], cn[1]);
       mma16816(mu[nt + 1], geA[0], geA[1], geA[2], geA[3], cn[2], cn[3]);
@@ -585,16 +565,13 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
       mma16816(mu[nt + 1], gel[0], gel[1], gel[2], gel[3], cn[2], cn[3]);
     }
 
-    // ---- dL/da and its reverse cumulative sum over the chunk (not for fallback channels,
-    // whose da already is A-free dΔ / A per step)
+    // ---- dL/da and its reverse cumulative sum over the chunk
     float dS[2][4];
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
-      if (!fb[c]) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) da[c][j] = fmaf(gg[c][j], ys[c][j], -xv[c][j] * dxp[c][j]);
-        if (tg == 3) da[c][3] += muh[c];  // step 15: h_out depends on a_15
-      }
+      for (int j = 0; j < 4; ++j) da[c][j] = fmaf(gg[c][j], ys[c][j], -xv[c][j] * dxp[c][j]);
+      if (tg == 3) da[c][3] += muh[c];  // step 15: h_out depends on a_15
       const float p = da[c][0] + da[c][1], q = da[c][2] + da[c][3];
       float ip = p, iq = q;  // suffix sums over the quad (lanes tg .. 3)
 #pragma unroll
@@ -611,10 +588,6 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
       dS[c][3] = iq - da[c][2];
       dS[c][0] = hi_total + ip;
       dS[c][1] = hi_total + ip - da[c][0];
-      if (fb[c]) {  // fallback: dΔ_t = A Ā_t dL/dĀ_t per step, no sum over later steps
-#pragma unroll
-        for (int j = 0; j < 4; ++j) dS[c][j] = da[c][j];
-      }
     }
 
     // ---- the channel gradients of the chunk's steps
@@ -634,8 +607,7 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
           const float y = fmaf(Dd[c], uv[c][j], ys[c][j]);
           // dz = dout y silu'(z), silu'(z) = σ(z) (1 + z (1 - σ(z)))
           vdz[od] = a.z ? gd[c][j] * y * gz[c][j] * fmaf(zz[c][j], 1.f - gz[c][j], 1.f) : 0.f;
-          // dA: Σ_t S_t dL/da_t; a fallback chunk's da holds Ā_t dL/dĀ_t, so Δ_t times it
-          accA[c] = fmaf(da[c][j], fb[c] ? dl[c][j] : S[c][j], accA[c]);
+          accA[c] = fmaf(da[c][j], S[c][j], accA[c]);  // dA = Σ_t S_t dL/da_t
           accD[c] = fmaf(gg[c][j], uv[c][j], accD[c]);
           if (lv[c][j]) accT[c] += vdd[od];
         }
