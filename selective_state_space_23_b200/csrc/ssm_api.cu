@@ -884,8 +884,7 @@ struct ChunkedBwdLayout {
 
 ChunkedBwdLayout chunked_bwd_layout(int batch, int dim, int seqlen, int dstate) {
   ChunkedBwdLayout l;
-  const size_t nck = (seqlen + ssm::kBlk - 1) / ssm::kBlk;
-  l.ck = align_up((size_t)batch * dim * (nck + 1) * dstate * 4);
+  l.ck = align_up((size_t)ssm::ssd_ckpt_floats(batch, dim, seqlen, dstate) * 4);
   l.pbc = align_up((size_t)ssm::ssd_bwd_ctas_per_row(dim) * batch * 2 * dstate * seqlen * 4);
   l.padt = align_up((size_t)batch * dim * 3 * 4);
   l.fwd = plan_ssd(batch, dim, seqlen, dstate).ws_bytes;
@@ -945,7 +944,7 @@ int scan_bwd_chunked(const void* u, const void* delta, const float* A, const voi
   memset(&a, 0, sizeof(a));
   a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
   a.A = A; a.dt_bias = dt_bias; a.h0 = h0;
-  a.ckpt = ck;  // [batch][dim][chunks + 1][N]: the state entering every chunk
+  a.ckpt = ck;  // the state entering every chunk, in fragment order
   a.batch = batch; a.dim = dim; a.L = seqlen; a.N = dstate;
   a.softplus = delta_softplus ? 1 : 0;
   a.scalar_a = 1;

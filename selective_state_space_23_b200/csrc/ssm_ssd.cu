@@ -69,21 +69,22 @@ __device__ __forceinline__ uint32_t ld_pair(const uint16_t* p, long long t, int 
   return lo | (hi << 16);
 }
 
-// The state (transposed accumulator layout, 2 channels x N/4 states per lane) into slot `slot`
-// of the f32 checkpoint array [batch][dim][chunks + 1][N].
+// The state of the warp's 16 channels into slot `slot` of the checkpoint array in fragment
+// order, f32 [batch][chunks + 1][ceil(dim / 16)][N / 8][32 lanes][4]: lane l's accumulator
+// registers Ht[nt][0..3] (channels g, g + 8 of the group, states 8 nt + 2 tg, +1) as one float4,
+// so that a 64-channel tile's state of one chunk is one contiguous block and a warp's read of an
+// n8 tile is 512 consecutive bytes.
 template <int N>
 __device__ __forceinline__ void store_state(const FwdArgs& a, const float (&Ht)[N / 8][4],
-                                            int slot, int b, const int (&dch)[2],
-                                            const bool (&act)[2], int tg) {
+                                            int slot, int b, int grp, int lane) {
   const long long nslots = (a.L + kT - 1) / kT + 1;
+  const int ngrp = (a.dim + 15) / 16;
+  if (grp >= ngrp) return;  // a warp past the last channel
+  float4* dst = reinterpret_cast<float4*>(a.ckpt) +
+                (((long long)b * nslots + slot) * ngrp + grp) * (N / 8) * 32 + lane;
 #pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    if (!act[c]) continue;
-    float* row = a.ckpt + (((long long)b * a.dim + dch[c]) * nslots + slot) * N + 2 * tg;
-#pragma unroll
-    for (int nt = 0; nt < N / 8; ++nt)
-      *reinterpret_cast<float2*>(row + 8 * nt) = make_float2(Ht[nt][2 * c], Ht[nt][2 * c + 1]);
-  }
+  for (int nt = 0; nt < N / 8; ++nt)
+    dst[nt * 32] = make_float4(Ht[nt][0], Ht[nt][1], Ht[nt][2], Ht[nt][3]);
 }
 
 // MODE: kSsdOut (gated outputs), kSsdSummary (segment end state and ΣΔ from zero), kSsdCkpt (the
@@ -197,7 +198,7 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
     if (k + 1 < nchunk) load_in(k + 1, nxt);
     const SsdStage<N>& st = ring[k % kStages];
     const int t0 = (kc0 + k) * kT;
-    if (MODE == kSsdCkpt) store_state<N>(a, Ht, kc0 + k, b, dch, act, tg);
+    if (MODE == kSsdCkpt) store_state<N>(a, Ht, kc0 + k, b, d0 / 16 + warp, lane);
 
     // ---- per (channel, step): Δ, Δx, gate; index j: steps 2tg, 2tg+1, 2tg+8, 2tg+9
     float dl[2][4], xv[2][4], gt[2][4], uv[2][4];
@@ -384,8 +385,8 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
     }
     // ---- store the chunk's outputs (bf16 pairs of steps)
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      if (NOOUT || !act[c]) continue;
+    for (int c = 0; c < (NOOUT ? 0 : 2); ++c) {
+      if (!act[c]) continue;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         const long long t = t0 + 2 * tg + 8 * hh;
@@ -401,7 +402,7 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
   }
   cp_wait<0>();
   if (MODE == kSsdCkpt) {
-    if ((seg + 1) * a.chunk_len >= L) store_state<N>(a, Ht, kc0 + nchunk, b, dch, act, tg);
+    if ((seg + 1) * a.chunk_len >= L) store_state<N>(a, Ht, kc0 + nchunk, b, d0 / 16 + warp, lane);
     return;
   }
   if (SUMMARY) {

@@ -49,19 +49,23 @@ namespace {
 
 using namespace ssd;
 
-constexpr int kWb = 4;  // warps per CTA (64 channels of one batch row and B/C group)
+constexpr int kWb = 4;   // warps per CTA (64 channels of one batch row and B/C group)
+constexpr int kStB = 3;  // ring depth (chunks) of B, C and the entering state
+constexpr int kLdR = 20; // f32 row stride of the [n][t] reduction tile: conflict-free both ways
 
 template <int N>
-struct BwdWarpSmem {
-  float red[2 * 16 * N];    // this warp's dB, dC of the chunk: [which][t][n]
-  // channels outside the factorisation's range: a_t (log2 units), x'_t, g_t per [d][t], and
-  // their exact y1, xy per [d][t]
-  float fa[16 * kT], fx[16 * kT], fg[16 * kT], fy[16 * kT], fxy[16 * kT];
+union BwdWarpSmem {
+  float red[2 * N * kLdR];  // this warp's dB, dC of the chunk: [which][n][t]
+  struct {                  // channels outside the factorisation's range (dead before red is
+                            // written): a_t (log2 units), x'_t, g_t, and their y1, xy; [d][t]
+    float fa[16 * kT], fx[16 * kT], fg[16 * kT], fy[16 * kT], fxy[16 * kT];
+  } f;
 };
 
 template <int N>
 struct BwdSmem {
-  SsdStage<N> ring[kStages];
+  SsdStage<N> ring[kStB];
+  float4 hs[kStB][kWb * (N / 8) * 32];  // the entering state of the chunk, fragment order
   BwdWarpSmem<N> w[kWb];
 };
 
@@ -109,14 +113,12 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
     bias[c] = a.dt_bias ? a.dt_bias[dch[c]] : 0.f;
     Dd[c] = a.D ? a.D[dch[c]] : 0.f;
   }
-  // the checkpointed states of the lane's channels; hck(c, k, nt): states 8 nt + 2 tg, +1 of the
-  // state entering chunk k (slot nck: the final state)
-  const float* ckr[2];
-#pragma unroll
-  for (int c = 0; c < 2; ++c) ckr[c] = a.ck + ((long long)b * a.dim + dch[c]) * nslots * N + 2 * tg;
-  const auto hck = [&](int c, int k, int nt) {
-    return __ldg(reinterpret_cast<const float2*>(ckr[c] + (long long)k * N + 8 * nt));
-  };
+  // the checkpointed entering states of this CTA's four 16-channel groups (the last valid
+  // group stands in for groups past dim)
+  const int ngrp = (a.dim + 15) / 16;
+  const int gvalid = min(kWb, ngrp - kWb * ctag);
+  const float4* ckb = reinterpret_cast<const float4*>(a.ck) +
+                      ((long long)b * nslots * ngrp + kWb * ctag) * kNT * 32;
 
   // the adjoint μ = dL/dh_out of the current chunk, transposed [d][n] in accumulator layout
   float mu[kNT][4];
@@ -131,11 +133,17 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
 
   float accA[2] = {0.f, 0.f}, accD[2] = {0.f, 0.f}, accT[2] = {0.f, 0.f};
 
-  // B/C tiles of chunk nck-1-i into ring slot i % kStages (chunks walked in reverse)
+  // B/C tiles and the entering state of chunk nck-1-i into ring slot i % kStB (chunks walked
+  // in reverse)
   const auto issue = [&](int i) {
     if (i < nck) {
-      SsdStage<N>& st = sm.ring[i % kStages];
+      SsdStage<N>& st = sm.ring[i % kStB];
       const int t0 = (nck - 1 - i) * kT;
+      const float4* src = ckb + (long long)(nck - 1 - i) * ngrp * kNT * 32;
+      for (int p = tid; p < kWb * kNT * 32; p += 32 * kWb) {
+        const int j = p / (kNT * 32);
+        cp16(&sm.hs[i % kStB][p], src + (min(j, gvalid - 1) - j) * kNT * 32 + p);
+      }
       if (a.rows16 && t0 + kT <= L) {
         for (int p = tid; p < 4 * N; p += 32 * kWb) {
           const int which = p / (2 * N), rem = p % (2 * N), n = rem >> 1, h = rem & 1;
@@ -169,18 +177,24 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
   };
 
 #pragma unroll
-  for (int i = 0; i < kStages - 1; ++i) issue(i);
+  for (int i = 0; i < kStB - 1; ++i) issue(i);
   ChunkInB nxt;
   load_in(nck - 1, nxt);
 
   for (int i = 0; i < nck; ++i) {
     const int k = nck - 1 - i;
-    cp_wait<kStages - 2>();
-    __syncthreads();  // chunk k's B/C landed; every warp is done with the previous chunk
-    issue(i + kStages - 1);
+    cp_wait<kStB - 2>();
+    __syncthreads();  // chunk k's B/C and state landed; every warp is done with the previous chunk
+    issue(i + kStB - 1);
     const ChunkInB cur = nxt;
     if (k > 0) load_in(k - 1, nxt);
-    const SsdStage<N>& st = sm.ring[i % kStages];
+    const SsdStage<N>& st = sm.ring[i % kStB];
+    const float4* hsw = &sm.hs[i % kStB][warp * kNT * 32 + lane];
+    // the entering state: states 8 nt + 2 tg, +1 of channel g + 8 c
+    const auto hck = [&](int c, int nt) {
+      const float4 v = hsw[nt * 32];
+      return c ? make_float2(v.z, v.w) : make_float2(v.x, v.y);
+    };
     const int t0 = k * kT;
 
     // ---- per (channel, step) quantities; j: steps 2tg, 2tg+1, 2tg+8, 2tg+9.  Steps past L
@@ -313,7 +327,7 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
 #pragma unroll
       for (int q = 0; q < 4; ++q) {  // {row g k lo, row g+8 k lo, row g k hi, row g+8 k hi}
         const int nt = 2 * kk + (q >> 1), c = q & 1;
-        const float2 hv = hck(c, k, nt);
+        const float2 hv = hck(c, nt);
         split_bf16x2(hv.x, hv.y, hh[q], hl[q]);
         split_bf16x2(mu[nt][2 * c], mu[nt][2 * c + 1], mh[q], ml[q]);
       }
@@ -398,17 +412,17 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int t = 2 * tg + (j & 1) + 8 * (j >> 1), o = (g + 8 * c) * kT + t;
-            ws.fa[o] = S[c][j] * al[c];
-            ws.fx[o] = xv[c][j];
-            ws.fg[o] = gg[c][j];
+            ws.f.fa[o] = S[c][j] * al[c];
+            ws.f.fx[o] = xv[c][j];
+            ws.f.fg[o] = gg[c][j];
           }
         }
         __syncwarp();
         for (unsigned m = fbm; m; m &= m - 1) {
           const int d = __ffs(m) - 1;
-          const float* ad = ws.fa + d * kT;
-          const float* xd = ws.fx + d * kT;
-          const float* gd_ = ws.fg + d * kT;
+          const float* ad = ws.f.fa + d * kT;
+          const float* xd = ws.f.fx + d * kT;
+          const float* gd_ = ws.f.fg + d * kT;
           float yr[2] = {0.f, 0.f}, xr[2] = {0.f, 0.f};
 #pragma unroll
           for (int T = 0; T < 2; ++T) {
@@ -434,10 +448,10 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
             xr[i] += __shfl_xor_sync(0xffffffffu, xr[i], 1);
             xr[i] += __shfl_xor_sync(0xffffffffu, xr[i], 2);
           }
-          if (tg == 0) ws.fy[d * kT + g] = yr[0];
-          if (tg == 1) ws.fy[d * kT + g + 8] = yr[1];
-          if (tg == 2) ws.fxy[d * kT + g] = xr[0];
-          if (tg == 3) ws.fxy[d * kT + g + 8] = xr[1];
+          if (tg == 0) ws.f.fy[d * kT + g] = yr[0];
+          if (tg == 1) ws.f.fy[d * kT + g + 8] = yr[1];
+          if (tg == 2) ws.f.fxy[d * kT + g] = xr[0];
+          if (tg == 3) ws.f.fxy[d * kT + g + 8] = xr[1];
         }
         __syncwarp();
       }
@@ -452,7 +466,7 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
     for (int nt = 0; nt < kNT; ++nt) {
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        const float2 hv = hck(c, k, nt);
+        const float2 hv = hck(c, nt);
         muh[c] = fmaf(mu[nt][2 * c], hv.x, fmaf(mu[nt][2 * c + 1], hv.y, muh[c]));
       }
     }
@@ -477,8 +491,8 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
         const int c = e >> 1, j = 2 * T + (e & 1);
         if (fixed && fb[c]) {
           const int o = (g + 8 * c) * kT + 2 * tg + (e & 1) + 8 * T;
-          ys[c][j] = fmaf(E[c][j], Y2[T][e], ws.fy[o]);
-          dxp[c][j] = fmaf(Ef[c][j], Xm[T][e], ws.fxy[o]);
+          ys[c][j] = fmaf(E[c][j], Y2[T][e], ws.f.fy[o]);
+          dxp[c][j] = fmaf(Ef[c][j], Xm[T][e], ws.f.fxy[o]);
         } else {
           ys[c][j] = fmaf(P[c][j], Y1[T][e], E[c][j] * Y2[T][e]);
           dxp[c][j] = Qv[c][j] * fmaf(eEm[c], Xm[T][e], Xy[T][e]);
@@ -521,7 +535,7 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
             split_bf16x2(mu[nt + q][2 * c], mu[nt + q][2 * c + 1], h_, l_);
             mbh[c] = movt(h_);
             mbl[c] = movt(l_);
-            const float2 hv = hck(c, k, nt + q);
+            const float2 hv = hck(c, nt + q);
             split_bf16x2(hv.x, hv.y, h_, l_);
             hbh[c] = movt(h_);
             hbl[c] = movt(l_);
@@ -537,14 +551,17 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
           mma16816(dC, geT[0], geT[1], geT[2], geT[3], hbh[0], hbh[1]);
           mma16816(dC, geT[0], geT[1], geT[2], geT[3], hbl[0], hbl[1]);
           mma16816(dC, geTl[0], geTl[1], geTl[2], geTl[3], hbh[0], hbh[1]);
-          // rows (s or t) g, g+8; columns n = 8 (nt + q) + 2 tg, +1
-          const int n = 8 * (nt + q) + 2 * tg;
-          float* rb = ws.red;
-          float* rc = ws.red + 16 * N;
-          *reinterpret_cast<float2*>(rb + g * N + n) = make_float2(dB[0], dB[1]);
-          *reinterpret_cast<float2*>(rb + (g + 8) * N + n) = make_float2(dB[2], dB[3]);
-          *reinterpret_cast<float2*>(rc + g * N + n) = make_float2(dC[0], dC[1]);
-          *reinterpret_cast<float2*>(rc + (g + 8) * N + n) = make_float2(dC[2], dC[3]);
+          // rows (s or t) g, g+8; columns n = 8 (nt + q) + 2 tg, +1; stored [n][t]
+          float* rb = ws.red + (8 * (nt + q) + 2 * tg) * kLdR + g;
+          float* rc = rb + N * kLdR;
+          rb[0] = dB[0];
+          rb[kLdR] = dB[1];
+          rb[8] = dB[2];
+          rb[kLdR + 8] = dB[3];
+          rc[0] = dC[0];
+          rc[kLdR] = dC[1];
+          rc[8] = dC[2];
+          rc[kLdR + 8] = dC[3];
         }
       }
     }
@@ -643,7 +660,7 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
         const int which = p / (N * kT), rem = p % (N * kT), n = rem / kT, t = rem % kT;
         float s = 0.f;
 #pragma unroll
-        for (int w = 0; w < kWb; ++w) s += sm.w[w].red[which * 16 * N + t * N + n];
+        for (int w = 0; w < kWb; ++w) s += sm.w[w].red[(which * N + n) * kLdR + t];
         if (t < nvalid)
           a.part_bc[((((long long)ctag * a.batch + b) * 2 + which) * N + n) * L + t0 + t] = s;
       }
