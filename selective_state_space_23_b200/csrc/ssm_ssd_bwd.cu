@@ -199,33 +199,28 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
 
     // ---- per (channel, step) quantities; j: steps 2tg, 2tg+1, 2tg+8, 2tg+9.  Steps past L
     // and idle channels (which shadow the last channel) take no part: zero step, input and g.
-    float dl[2][4], uv[2][4], xv[2][4], sg[2][4], gz[2][4], zz[2][4], gd[2][4], gg[2][4];
-    bool lv[2][4];
+    // Only Δ, x' = Δ x and g = dout silu(z) stay live through the chunk's products; what only
+    // the gradients at the end need (x, σ(v), dout, z, σ(z)) is recomputed there from the
+    // packed inputs, which keeps the register file from spilling.
+    const auto live_at = [&](int c, int j) { return act[c] && t0 + 2 * tg + (j & 1) + 8 * (j >> 1) < L; };
+    float dl[2][4], xv[2][4], gg[2][4];
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int hh = j >> 1, od = j & 1;
-        const int t = t0 + 2 * tg + od + 8 * hh;
-        const bool live = act[c] && t < L;
-        lv[c][j] = live;
+        const bool live = live_at(c, j);
         const float u = pick(cur.u[c][hh], od);
         const float v = pick(cur.dl[c][hh], od) + bias[c];
         const float D = a.softplus ? softplus_fast(v) : v;
-        sg[c][j] = a.softplus ? sigmoid_fast(v) : 1.f;  // dΔ/dv
         dl[c][j] = live ? D : 0.f;
-        uv[c][j] = live ? u : 0.f;
-        xv[c][j] = dl[c][j] * uv[c][j];
-        gd[c][j] = live ? pick(cur.go[c][hh], od) : 0.f;
+        xv[c][j] = live ? D * u : 0.f;
+        const float go = live ? pick(cur.go[c][hh], od) : 0.f;
         if (a.z) {
           const float z = pick(cur.z[c][hh], od);
-          zz[c][j] = z;
-          gz[c][j] = sigmoid_fast(z);  // σ(z)
-          gg[c][j] = gd[c][j] * z * gz[c][j];
+          gg[c][j] = go * z * sigmoid_fast(z);
         } else {
-          zz[c][j] = 0.f;
-          gz[c][j] = 1.f;
-          gg[c][j] = gd[c][j];
+          gg[c][j] = go;
         }
       }
     }
@@ -266,39 +261,35 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
     }
     // decay factors: P, Q about the middle step for the factorised products; E_t = e^{a_t} and
     // e^{a_15 - a_s} directly for channels outside the range (both <= 1)
-    float P[2][4], Qv[2][4], E[2][4], eEm[2], Eend[2], Ef[2][4];
-    float q2f[2][4];  // e^{a_15 - a_s} x'_s in f32
+    // The per-step factors (P, Q, E, e^{a_15 - a_s}) are formed here for the operands and again
+    // after the products, rather than kept live through them.
+    float eAm[2], eEm[2], Eend[2];
     // A fragments (bf16 pairs) and, for the products that feed dΔ, dA and the carried adjoint,
     // the remainders (suffix l)
     uint32_t x1[4], x2[4], gpA[4], geA[4], x1l[4], x2l[4], gpl[4], gel[4];
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
-      const float eAm = ex2_mufu(Sm[c] * al[c]);
+      eAm[c] = ex2_mufu(Sm[c] * al[c]);
       eEm[c] = ex2_mufu((Se[c] - Sm[c]) * al[c]);
       Eend[c] = ex2_mufu(Se[c] * al[c]);
       float q1[4], q2[4], gp[4], ge[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const float r = (S[c][j] - Sm[c]) * al[c];
-        P[c][j] = ex2_mufu(r);
-        Qv[c][j] = ex2_mufu(-r);
+        float E;
         if (fb[c]) {
-          E[c][j] = ex2_mufu(S[c][j] * al[c]);
-          Ef[c][j] = ex2_mufu((Se[c] - S[c][j]) * al[c]);
+          E = ex2_mufu(S[c][j] * al[c]);
           q1[j] = 0.f;
-          q2[j] = Ef[c][j] * xv[c][j];
+          q2[j] = ex2_mufu((Se[c] - S[c][j]) * al[c]) * xv[c][j];
           gp[j] = 0.f;
         } else {
-          E[c][j] = eAm * P[c][j];
-          Ef[c][j] = 0.f;
-          q1[j] = Qv[c][j] * xv[c][j];
+          const float r = (S[c][j] - Sm[c]) * al[c], P = ex2_mufu(r);
+          E = eAm[c] * P;
+          q1[j] = ex2_mufu(-r) * xv[c][j];
           q2[j] = eEm[c] * q1[j];
-          gp[j] = gg[c][j] * P[c][j];
+          gp[j] = gg[c][j] * P;
         }
-        ge[j] = gg[c][j] * E[c][j];
+        ge[j] = gg[c][j] * E;
       }
-#pragma unroll
-      for (int j = 0; j < 4; ++j) q2f[c][j] = q2[j];
       split_bf16x2(q1[0], q1[1], x1[c], x1l[c]);
       split_bf16x2(q1[2], q1[3], x1[2 + c], x1l[2 + c]);
       split_bf16x2(q2[0], q2[1], x2[c], x2l[c]);
@@ -472,32 +463,36 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
     }
 #pragma unroll
     for (int c = 0; c < 2; ++c) muh[c] *= Eend[c];
-#pragma unroll
-    for (int T = 0; T < 2; ++T)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) muh[e >> 1] = fmaf(q2f[e >> 1][2 * T + (e & 1)], Xm[T][e], muh[e >> 1]);
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      muh[c] += __shfl_xor_sync(0xffffffffu, muh[c], 1);
-      muh[c] += __shfl_xor_sync(0xffffffffu, muh[c], 2);
-    }
 
-    // ---- per (channel, step): y, dx', da (accumulator (tile T, e): channel e/2, j = 2T + e%2)
+    // ---- per (channel, step): y, dx', da (accumulator (tile T, e): channel e/2, j = 2T + e%2);
+    // the factors again: P, Q, E in range; E and e^{a_15 - a_t} directly out of range (whose y1
+    // and xy come from the exact pair pass)
     float ys[2][4], dxp[2][4], da[2][4];
 #pragma unroll
     for (int T = 0; T < 2; ++T) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int c = e >> 1, j = 2 * T + (e & 1);
-        if (fixed && fb[c]) {
+        float q2;  // e^{a_15 - a_t} x'_t
+        if (fb[c]) {
           const int o = (g + 8 * c) * kT + 2 * tg + (e & 1) + 8 * T;
-          ys[c][j] = fmaf(E[c][j], Y2[T][e], ws.f.fy[o]);
-          dxp[c][j] = fmaf(Ef[c][j], Xm[T][e], ws.f.fxy[o]);
+          const float Ef = ex2_mufu((Se[c] - S[c][j]) * al[c]);
+          ys[c][j] = fmaf(ex2_mufu(S[c][j] * al[c]), Y2[T][e], ws.f.fy[o]);
+          dxp[c][j] = fmaf(Ef, Xm[T][e], ws.f.fxy[o]);
+          q2 = Ef * xv[c][j];
         } else {
-          ys[c][j] = fmaf(P[c][j], Y1[T][e], E[c][j] * Y2[T][e]);
-          dxp[c][j] = Qv[c][j] * fmaf(eEm[c], Xm[T][e], Xy[T][e]);
+          const float r = (S[c][j] - Sm[c]) * al[c], P = ex2_mufu(r), Q = ex2_mufu(-r);
+          ys[c][j] = fmaf(P, Y1[T][e], eAm[c] * P * Y2[T][e]);
+          dxp[c][j] = Q * fmaf(eEm[c], Xm[T][e], Xy[T][e]);
+          q2 = eEm[c] * (Q * xv[c][j]);
         }
+        muh[c] = fmaf(q2, Xm[T][e], muh[c]);
       }
+    }
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      muh[c] += __shfl_xor_sync(0xffffffffu, muh[c], 1);
+      muh[c] += __shfl_xor_sync(0xffffffffu, muh[c], 2);
     }
 
     // ---- dB, dC of the chunk summed over the warp's channels on the tensor cores (every
@@ -618,15 +613,24 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
 #pragma unroll
         for (int od = 0; od < 2; ++od) {
           const int j = 2 * hh + od;
-          const float dD = fmaf(A, dS[c][j], dxp[c][j] * uv[c][j]);  // dL/dΔ_t
-          vdd[od] = dD * sg[c][j];                                     // through softplus
+          const bool live = live_at(c, j);
+          const float u = live ? pick(cur.u[c][hh], od) : 0.f;
+          const float sg = a.softplus ? sigmoid_fast(pick(cur.dl[c][hh], od) + bias[c]) : 1.f;
+          const float dD = fmaf(A, dS[c][j], dxp[c][j] * u);  // dL/dΔ_t
+          vdd[od] = dD * sg;                                   // through softplus (dΔ/dv = σ(v))
           vdu[od] = fmaf(dxp[c][j], dl[c][j], Dd[c] * gg[c][j]);
-          const float y = fmaf(Dd[c], uv[c][j], ys[c][j]);
-          // dz = dout y silu'(z), silu'(z) = σ(z) (1 + z (1 - σ(z)))
-          vdz[od] = a.z ? gd[c][j] * y * gz[c][j] * fmaf(zz[c][j], 1.f - gz[c][j], 1.f) : 0.f;
+          if (a.z) {
+            // dz = dout y silu'(z), silu'(z) = σ(z) (1 + z (1 - σ(z)))
+            const float y = fmaf(Dd[c], u, ys[c][j]);
+            const float go = live ? pick(cur.go[c][hh], od) : 0.f;
+            const float z = pick(cur.z[c][hh], od), gz = sigmoid_fast(z);
+            vdz[od] = go * y * gz * fmaf(z, 1.f - gz, 1.f);
+          } else {
+            vdz[od] = 0.f;
+          }
           accA[c] = fmaf(da[c][j], S[c][j], accA[c]);  // dA = Σ_t S_t dL/da_t
-          accD[c] = fmaf(gg[c][j], uv[c][j], accD[c]);
-          if (lv[c][j]) accT[c] += vdd[od];
+          accD[c] = fmaf(gg[c][j], u, accD[c]);
+          if (live) accT[c] += vdd[od];
         }
         wdu[hh] = pack_bf16x2(vdu[0], vdu[1]);
         wdd[hh] = pack_bf16x2(vdd[0], vdd[1]);
