@@ -50,7 +50,7 @@ namespace {
 using namespace ssd;
 
 constexpr int kWb = 4;   // warps per CTA (64 channels of one batch row and B/C group)
-constexpr int kStB = 3;  // ring depth (chunks) of B, C and the entering state
+constexpr int kStB = 2;  // ring depth (chunks) of B, C and the entering state
 constexpr int kLdR = 20; // f32 row stride of the [n][t] reduction tile: conflict-free both ways
 
 template <int N>
@@ -66,6 +66,7 @@ template <int N>
 struct BwdSmem {
   SsdStage<N> ring[kStB];
   float4 hs[kStB][kWb * (N / 8) * 32];  // the entering state of the chunk, fragment order
+  float4 mu[kWb * (N / 8) * 32];        // the adjoint μ, fragment order (each lane its own)
   BwdWarpSmem<N> w[kWb];
 };
 
@@ -120,16 +121,25 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
   const float4* ckb = reinterpret_cast<const float4*>(a.ck) +
                       ((long long)b * nslots * ngrp + kWb * ctag) * kNT * 32;
 
-  // the adjoint μ = dL/dh_out of the current chunk, transposed [d][n] in accumulator layout
-  float mu[kNT][4];
+  // the adjoint μ = dL/dh_out of the current chunk, transposed [d][n] in accumulator layout:
+  // mus[32 nt] holds the lane's registers of n tile nt (channels g, g + 8; states 8 nt + 2 tg,
+  // +1).  It lives in shared memory, one float4 per lane and tile that no other lane touches,
+  // which frees N / 2 registers; the accesses are conflict-free and need no barrier.
+  float4* mus = &sm.mu[warp * kNT * 32 + lane];
 #pragma unroll
   for (int nt = 0; nt < kNT; ++nt) {
+    float v[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int c = e >> 1, n = 8 * nt + 2 * tg + (e & 1);
-      mu[nt][e] = a.dhL && act[c] ? a.dhL[((long long)b * a.dim + dch[c]) * N + n] : 0.f;
+      v[e] = a.dhL && act[c] ? a.dhL[((long long)b * a.dim + dch[c]) * N + n] : 0.f;
     }
+    mus[nt * 32] = make_float4(v[0], v[1], v[2], v[3]);
   }
+  const auto mupair = [&](int nt, int c) {
+    const float4 m = mus[nt * 32];
+    return c ? make_float2(m.z, m.w) : make_float2(m.x, m.y);
+  };
 
   float accA[2] = {0.f, 0.f}, accD[2] = {0.f, 0.f}, accT[2] = {0.f, 0.f};
 
@@ -320,7 +330,8 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
         const int nt = 2 * kk + (q >> 1), c = q & 1;
         const float2 hv = hck(c, nt);
         split_bf16x2(hv.x, hv.y, hh[q], hl[q]);
-        split_bf16x2(mu[nt][2 * c], mu[nt][2 * c + 1], mh[q], ml[q]);
+        const float2 mv = mupair(nt, c);
+        split_bf16x2(mv.x, mv.y, mh[q], ml[q]);
       }
       mma16816(Y2[0], hh[0], hh[1], hh[2], hh[3], cf[0], cf[2]);
       mma16816(Y2[1], hh[0], hh[1], hh[2], hh[3], cf[1], cf[3]);
@@ -458,7 +469,8 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         const float2 hv = hck(c, nt);
-        muh[c] = fmaf(mu[nt][2 * c], hv.x, fmaf(mu[nt][2 * c + 1], hv.y, muh[c]));
+        const float2 mv = mupair(nt, c);
+        muh[c] = fmaf(mv.x, hv.x, fmaf(mv.y, hv.y, muh[c]));
       }
     }
 #pragma unroll
@@ -527,7 +539,8 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             uint32_t h_, l_;
-            split_bf16x2(mu[nt + q][2 * c], mu[nt + q][2 * c + 1], h_, l_);
+            const float2 mv = mupair(nt + q, c);
+            split_bf16x2(mv.x, mv.y, h_, l_);
             mbh[c] = movt(h_);
             mbl[c] = movt(l_);
             const float2 hv = hck(c, nt + q);
@@ -566,15 +579,15 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
     for (int nt = 0; nt < kNT; nt += 2) {
       uint32_t cn[4];
       ldsm_x4(cn, blk(st.Cs, 8 * nt, lane));
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        mu[nt][e] *= Eend[e >> 1];
-        mu[nt + 1][e] *= Eend[e >> 1];
-      }
-      mma16816(mu[nt], geA[0], geA[1], geA[2], geA[3], cn[0], cn[1]);
-      mma16816(mu[nt + 1], geA[0], geA[1], geA[2], geA[3], cn[2], cn[3]);
-      mma16816(mu[nt], gel[0], gel[1], gel[2], gel[3], cn[0], cn[1]);
-      mma16816(mu[nt + 1], gel[0], gel[1], gel[2], gel[3], cn[2], cn[3]);
+      const float4 m0 = mus[nt * 32], m1 = mus[(nt + 1) * 32];
+      float u0[4] = {m0.x * Eend[0], m0.y * Eend[0], m0.z * Eend[1], m0.w * Eend[1]};
+      float u1[4] = {m1.x * Eend[0], m1.y * Eend[0], m1.z * Eend[1], m1.w * Eend[1]};
+      mma16816(u0, geA[0], geA[1], geA[2], geA[3], cn[0], cn[1]);
+      mma16816(u1, geA[0], geA[1], geA[2], geA[3], cn[2], cn[3]);
+      mma16816(u0, gel[0], gel[1], gel[2], gel[3], cn[0], cn[1]);
+      mma16816(u1, gel[0], gel[1], gel[2], gel[3], cn[2], cn[3]);
+      mus[nt * 32] = make_float4(u0[0], u0[1], u0[2], u0[3]);
+      mus[(nt + 1) * 32] = make_float4(u1[0], u1[1], u1[2], u1[3]);
     }
 
     // ---- dL/da and its reverse cumulative sum over the chunk
@@ -687,8 +700,9 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
     if (a.dh0) {
 #pragma unroll
       for (int nt = 0; nt < kNT; ++nt) {
-        a.dh0[ch * N + 8 * nt + 2 * tg] = mu[nt][2 * c];
-        a.dh0[ch * N + 8 * nt + 2 * tg + 1] = mu[nt][2 * c + 1];
+        const float2 mv = mupair(nt, c);
+        a.dh0[ch * N + 8 * nt + 2 * tg] = mv.x;
+        a.dh0[ch * N + 8 * nt + 2 * tg + 1] = mv.y;
       }
     }
     if (tg == 0) {
