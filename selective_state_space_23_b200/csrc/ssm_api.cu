@@ -871,10 +871,10 @@ namespace {
 // layout, B/C shared by whole 64-channel tiles, no checkpoints given): the forward's checkpoint
 // pass (with its own time split), the backward kernel, and the finishing sums.
 bool chunked_bwd_ok(int dim, int dstate, int bc_groups, int io_dtype, int flags) {
-  const char* v = getenv("SSM_SCALAR_BWD");
-  if (v && strcmp(v, "slices") == 0) return false;
+  const char* v = getenv("SSM_SCALAR_BWD");  // "slices" / "state": the per-state kernels
+  if (v && (strcmp(v, "slices") == 0 || strcmp(v, "state") == 0)) return false;
   return io_dtype == SSM_BF16 && flags == SSM_SCALAR_A &&
-         (dstate == 32 || dstate == 64 || dstate == 128) &&
+         (dstate == 16 || dstate == 32 || dstate == 64 || dstate == 128) &&
          (bc_groups == 1 || (bc_groups < dim && dim % bc_groups == 0 && (dim / bc_groups) % 64 == 0));
 }
 
@@ -1023,6 +1023,10 @@ size_t ssm_scan_bwd_ex_workspace_size(int batch, int dim, int seqlen, int dstate
       return chunked_bwd_layout(batch, dim, seqlen, dstate).total;
     return ssm::scan_bwd_slices_workspace(batch, dim, seqlen, dstate, bc_groups, io_dtype, flags);
   }
+  if (dstate == 16 && !have_ckpt && chunked_bwd_ok(dim, dstate, bc_groups, io_dtype, flags)) {
+    if (check_dims(batch, dim, seqlen, dstate, io_dtype) != SSM_OK) return 0;
+    return chunked_bwd_layout(batch, dim, seqlen, dstate).total;
+  }
   if (check_dims(batch, dim, seqlen, dstate, io_dtype) != SSM_OK) return 0;
   if (check_groups(dim, bc_groups) != SSM_OK) return 0;
   const size_t base = layout_bwd(batch, dim, seqlen, dstate, have_ckpt != 0, bc_groups, io_dtype,
@@ -1056,6 +1060,12 @@ int ssm_scan_bwd_ex(const void* u, const void* delta, const float* A, const void
                                 flags, stream);
   }
   TRY(check_dims(batch, dim, seqlen, dstate, io_dtype));
+  if (dstate == 16 && !ckpt && chunked_bwd_ok(dim, dstate, bc_groups, io_dtype, flags)) {
+    TRY(check_groups(dim, bc_groups));
+    return scan_bwd_chunked(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL, du,
+                            ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, workspace, workspace_bytes,
+                            batch, dim, seqlen, dstate, bc_groups, stream);
+  }
   if (!(flags & SSM_SCALAR_A))
     return scan_bwd_core(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL, ckpt,
                          du, ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, workspace,

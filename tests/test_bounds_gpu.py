@@ -187,6 +187,7 @@ BWD_CASES = {
     "reverse_zoh_grouped": ({}, 2, 64, 200, 16, torch.bfloat16, 2, 2 | 4),
     "per_channel_bc": ({}, 2, 24, 120, 16, torch.bfloat16, 24, 0),
     "scalar_decay": ({}, 2, 96, 200, 16, torch.bfloat16, 1, 1),
+    "scalar_decay_state": ({"SSM_SCALAR_BWD": "state"}, 2, 96, 200, 16, torch.bfloat16, 1, 1),
     "scalar_decay_n64_slices": ({"SSM_SCALAR_BWD": "slices"}, 2, 96, 120, 64, torch.bfloat16, 1, 1),
     "scalar_decay_n64_chunked": ({}, 2, 96, 120, 64, torch.bfloat16, 1, 1),
     "scalar_decay_n128_chunked": ({}, 1, 80, 333, 128, torch.bfloat16, 1, 1),

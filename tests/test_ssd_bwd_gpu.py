@@ -91,7 +91,7 @@ def test_forward_then_backward_shapes_agree():
 
 
 # ------------------------------------------------------------------ the chunked-form backward
-@pytest.mark.parametrize("N", [32, 64, 128])
+@pytest.mark.parametrize("N", [16, 32, 64, 128])
 @pytest.mark.parametrize("shape", [(2, 128, 160), (1, 80, 333), (2, 64, 17)])
 def test_chunked_backward_matches_oracle(monkeypatch, N, shape):
     """bf16 scalar decay with N > 16 runs the chunked-form backward (tensor cores): partial
@@ -106,17 +106,19 @@ def test_chunked_backward_matches_oracle(monkeypatch, N, shape):
         assert_close(g[k], r[k], torch.bfloat16, k)
 
 
-def test_chunked_and_slice_backwards_agree(monkeypatch):
-    x = inputs(2, 128, 200, 64, torch.bfloat16, seed=112)
+@pytest.mark.parametrize("N", [16, 64])
+def test_chunked_and_per_state_backwards_agree(monkeypatch, N):
+    """The chunked form against the per-state kernels (16-state slices above N = 16)."""
+    x = inputs(2, 128, 200, N, torch.bfloat16, seed=112)
     monkeypatch.delenv("SSM_SCALAR_BWD", raising=False)
     a = run(x, None)
-    monkeypatch.setenv("SSM_SCALAR_BWD", "slices")
+    monkeypatch.setenv("SSM_SCALAR_BWD", "state" if N == 16 else "slices")
     b = run(x, None)
     for k in GRADS:
         assert_close(a[k], f64(b[k]), torch.bfloat16, k)
 
 
-@pytest.mark.parametrize("N", [32, 64, 128])
+@pytest.mark.parametrize("N", [16, 32, 64, 128])
 def test_chunked_backward_range_fallback(N):
     """Steps over v = delta + dt_bias in [-30, 30]: most chunks leave the factorisation's range,
     and their intra-chunk products take the exact per-pair decay.  Gradients of size ~1 are
