@@ -314,8 +314,8 @@ def bench_extras(dev, which=EXTRAS):
 
 
 def _ssd(dev, rnd, prm, timeit, g):
-    """Scalar decay with 64 and 128 states on the Mamba-370m-shaped layer (the chunked matrix
-    form on the tensor cores)."""
+    """Scalar decay with 16, 64 and 128 states on the Mamba-370m-shaped layer (the chunked matrix
+    form on the tensor cores): forward at 64 and 128 states, backward at all three."""
     import selective_state_space_23_b200 as ssm
     out = {}
     b, d, L = 8, 2048, 2048
@@ -332,15 +332,21 @@ def _ssd(dev, rnd, prm, timeit, g):
         res[f"N{N}"] = {"fwd_ms": ms, "tokens_per_s": b * L / (ms * 1e-3),
                         "hbm_gbs": (4 * b * d * L * 2 + 2 * b * N * L * 2) / (ms * 1e-3) / 1e9,
                         "mma_tflops": flops / (ms * 1e-3) / 1e12}
-    # the backward with 64 states (the sum of four 16-state backwards)
-    B, C = rnd((b, 64, L)), rnd((b, 64, L))
+    # the backward (chunked form: checkpoint pass, reverse walk, dB/dC finish) with 16, 64 and
+    # 128 states; compulsory bytes: u, delta, z, dout in, du, ddelta, dz out, B, C in, dB, dC out
     dout = rnd((b, d, L))
-    wsb = torch.empty(ssm._abi.lib().ssm_scan_bwd_ex_workspace_size(b, d, L, 64, 1, 1, 0, 1),
-                      dtype=torch.uint8, device=dev)
-    ms = timeit(lambda: ssm.ssm_scan_bwd_scalar_a(u, de, A1, B, C, dout, D=D, z=z, dt_bias=bias,
-                                                  workspace=wsb), 3)
-    res["bwd_N64_ms"] = ms
-    del u, de, z, o, B, C, dout, wsb
+    res["bwd"] = {}
+    for N in (16, 64, 128):
+        B, C = rnd((b, N, L)), rnd((b, N, L))
+        wsb = torch.empty(ssm._abi.lib().ssm_scan_bwd_ex_workspace_size(b, d, L, N, 1, 1, 0, 1),
+                          dtype=torch.uint8, device=dev)
+        ms = timeit(lambda: ssm.ssm_scan_bwd_scalar_a(u, de, A1, B, C, dout, D=D, z=z,
+                                                      dt_bias=bias, workspace=wsb), 5)
+        byt = 7 * b * d * L * 2 + 4 * b * N * L * 2
+        res["bwd"][f"N{N}"] = {"bwd_ms": ms, "tokens_per_s": b * L / (ms * 1e-3),
+                               "compulsory_gbs": byt / (ms * 1e-3) / 1e9}
+        del B, C, wsb
+    del u, de, z, o, dout
     # the long sequence (1 x 256 x 2^20) with 64 states: 16 warps of channels, so the time axis
     # is split into segments (summary, chain, output launches)
     b, d, L, N = 1, 256, 1 << 20, 64

@@ -671,15 +671,31 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
     // ---- the CTA's dB, dC of the chunk: its warps' tiles summed in warp order
     if (a.need_bc) {
       __syncthreads();  // every warp's tile is complete
-      // the CTA's sum over its warps, in warp order, into part_bc [ctag][b][which][n][t]
+      // the CTA's sum over its warps, in warp order, into part_bc [ctag][b][which][n][t]; a
+      // thread takes 4 consecutive steps (128-bit shared loads, one 128-bit store when the
+      // chunk is whole and rows are 16-byte aligned)
       const int nvalid = min(kT, L - t0);
-      for (int p = tid; p < 2 * N * kT; p += 32 * kWb) {
-        const int which = p / (N * kT), rem = p % (N * kT), n = rem / kT, t = rem % kT;
-        float s = 0.f;
+      const bool vst = nvalid == kT && (L & 3) == 0;
+      for (int p = tid; p < 2 * N * (kT / 4); p += 32 * kWb) {
+        const int which = p / (N * (kT / 4)), n = (p / (kT / 4)) % N, t = 4 * (p % (kT / 4));
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int w = 0; w < kWb; ++w) s += sm.w[w].red[(which * N + n) * kLdR + t];
-        if (t < nvalid)
-          a.part_bc[((((long long)ctag * a.batch + b) * 2 + which) * N + n) * L + t0 + t] = s;
+        for (int w = 0; w < kWb; ++w) {
+          const float4 r = *reinterpret_cast<const float4*>(&sm.w[w].red[(which * N + n) * kLdR + t]);
+          v.x += r.x;
+          v.y += r.y;
+          v.z += r.z;
+          v.w += r.w;
+        }
+        float* dst = a.part_bc + ((((long long)ctag * a.batch + b) * 2 + which) * N + n) * L + t0 + t;
+        if (vst) {
+          __stcs(reinterpret_cast<float4*>(dst), v);
+        } else {
+          if (t < nvalid) dst[0] = v.x;
+          if (t + 1 < nvalid) dst[1] = v.y;
+          if (t + 2 < nvalid) dst[2] = v.z;
+          if (t + 3 < nvalid) dst[3] = v.w;
+        }
       }
     }
   }
@@ -713,7 +729,8 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
   }
 }
 
-// dB, dC: each B/C group's CTAs summed in CTA order.
+// dB, dC: each B/C group's CTAs summed in CTA order.  The partials are loaded eight at a time
+// before they are added (in the same order), so each thread keeps eight loads in flight.
 __global__ void ssd_finish_bc(const SsdBwdArgs a, uint16_t* dB, uint16_t* dC, int ctas) {
   const long long total = (long long)a.batch * a.bc_groups * 2 * a.N * a.L;
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -727,9 +744,18 @@ __global__ void ssd_finish_bc(const SsdBwdArgs a, uint16_t* dB, uint16_t* dC, in
   const int gb = (int)(r % a.bc_groups);
   const int b = (int)(r / a.bc_groups);
   const int per = ctas / a.bc_groups;
+  const long long step = (long long)a.batch * 2 * a.N * a.L;  // between consecutive CTAs
+  const float* p = a.part_bc + ((((long long)gb * per * a.batch + b) * 2 + which) * a.N + n) * a.L + t;
   float s = 0.f;
-  for (int cg = gb * per; cg < (gb + 1) * per; ++cg)
-    s += a.part_bc[((((long long)cg * a.batch + b) * 2 + which) * a.N + n) * a.L + t];
+  int cg = 0;
+  for (; cg + 8 <= per; cg += 8) {
+    float v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = __ldcs(p + (cg + k) * step);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) s += v[k];
+  }
+  for (; cg < per; ++cg) s += __ldcs(p + cg * step);
   uint16_t* dst = which == 0 ? dB : dC;
   if (dst) dst[(((long long)b * a.bc_groups + gb) * a.N + n) * a.L + t] = f32_to_bf16(s);
 }
