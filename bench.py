@@ -358,9 +358,16 @@ def _ssd(dev, rnd, prm, timeit, g):
                      dtype=torch.uint8, device=dev)
     ms = timeit(lambda: ssm.ssm_scan_fwd_scalar_a(u, de, A1, B, C, D=D, z=z, dt_bias=bias,
                                                   workspace=ws), 5)
+    del ws
+    # its backward: the reverse walk split into segments (summary, adjoint chain, segments)
+    dout = rnd((b, d, L))
+    wsb = torch.empty(ssm._abi.lib().ssm_scan_bwd_ex_workspace_size(b, d, L, N, 1, 1, 0, 1),
+                      dtype=torch.uint8, device=dev)
+    msb = timeit(lambda: ssm.ssm_scan_bwd_scalar_a(u, de, A1, B, C, dout, D=D, z=z, dt_bias=bias,
+                                                   workspace=wsb), 3)
     res["long_seq_N64"] = {"shape": "1x256x1048576 bf16, A [dim]", "fwd_ms": ms,
-                           "tokens_per_s": b * L / (ms * 1e-3)}
-    del u, de, z, B, C, ws
+                           "tokens_per_s": b * L / (ms * 1e-3), "bwd_ms": msb}
+    del u, de, z, B, C, dout, wsb
     torch.cuda.empty_cache()
     out["scalar_decay_large_n"] = res
     return out

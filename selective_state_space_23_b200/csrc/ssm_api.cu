@@ -878,17 +878,49 @@ bool chunked_bwd_ok(int dim, int dstate, int bc_groups, int io_dtype, int flags)
          (bc_groups == 1 || (bc_groups < dim && dim % bc_groups == 0 && (dim / bc_groups) % 64 == 0));
 }
 
+// Time split of the chunked backward: when its CTAs (batch rows x 64-channel tiles) fill at most
+// half of the resident slots (two per SM; one at N = 128, whose CTA takes most of an SM's shared
+// memory), the chunks are cut into as many segments as still fit in one wave, each of at least 16
+// chunks, and walked side by side from their chained adjoints (SSM_SSD_BWD_SPLIT overrides the
+// segment count).  A grid that already fills most of a wave is not split: a second wave and the
+// summary launch would cost more than the idle slots.
+struct BwdSegPlan {
+  int nseg, cps;  // segments, chunks per segment
+};
+BwdSegPlan plan_ssd_bwd(int batch, int dim, int seqlen, int dstate) {
+  const int nck = (seqlen + ssm::kBlk - 1) / ssm::kBlk;
+  const long long ctas = (long long)batch * ssm::ssd_bwd_ctas_per_row(dim);
+  const long long target = (long long)sm_count() * (dstate >= 128 ? 1 : 2);
+  const int forced = env_int("SSM_SSD_BWD_SPLIT", 0);
+  int S = forced;
+  if (S <= 0) {
+    S = (int)(target / ctas);  // whole segments per channel tile within one wave
+    S = S < nck / 16 ? S : (nck / 16 > 1 ? nck / 16 : 1);
+  }
+  S = S < 1 ? 1 : (S > nck ? nck : S);
+  BwdSegPlan p;
+  p.cps = (nck + S - 1) / S;
+  p.nseg = (nck + p.cps - 1) / p.cps;
+  return p;
+}
+
 struct ChunkedBwdLayout {
-  size_t ck, pbc, padt, fwd, total;
+  size_t ck, pbc, padt, musum, dsum, muin, fwd, total;
+  BwdSegPlan seg;
 };
 
 ChunkedBwdLayout chunked_bwd_layout(int batch, int dim, int seqlen, int dstate) {
   ChunkedBwdLayout l;
+  l.seg = plan_ssd_bwd(batch, dim, seqlen, dstate);
+  const size_t nch = (size_t)batch * dim, S = (size_t)l.seg.nseg;
   l.ck = align_up((size_t)ssm::ssd_ckpt_floats(batch, dim, seqlen, dstate) * 4);
   l.pbc = align_up((size_t)ssm::ssd_bwd_ctas_per_row(dim) * batch * 2 * dstate * seqlen * 4);
-  l.padt = align_up((size_t)batch * dim * 3 * 4);
+  l.padt = align_up(S * nch * 3 * 4);
+  l.musum = S > 1 ? align_up(S * nch * dstate * 4) : 0;
+  l.dsum = S > 1 ? align_up(S * nch * 4) : 0;
+  l.muin = l.musum;
   l.fwd = plan_ssd(batch, dim, seqlen, dstate).ws_bytes;
-  l.total = l.ck + l.pbc + l.padt + l.fwd;
+  l.total = l.ck + l.pbc + l.padt + l.musum + l.dsum + l.muin + l.fwd;
   return l;
 }
 
@@ -935,7 +967,10 @@ int scan_bwd_chunked(const void* u, const void* delta, const float* A, const voi
   float* ck = reinterpret_cast<float*>(w);
   float* pbc = reinterpret_cast<float*>(w + l.ck);
   float* padt = reinterpret_cast<float*>(w + l.ck + l.pbc);
-  char* fws = w + l.ck + l.pbc + l.padt;
+  float* musum = reinterpret_cast<float*>(w + l.ck + l.pbc + l.padt);
+  float* dsum = reinterpret_cast<float*>(w + l.ck + l.pbc + l.padt + l.musum);
+  float* muin = reinterpret_cast<float*>(w + l.ck + l.pbc + l.padt + l.musum + l.dsum);
+  char* fws = w + l.ck + l.pbc + l.padt + l.musum + l.dsum + l.muin;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool vec = (seqlen * es) % 16 == 0 && aligned16(u) && aligned16(delta) && aligned16(z) &&
                    aligned16(B) && aligned16(C);
@@ -991,7 +1026,21 @@ int scan_bwd_chunked(const void* u, const void* delta, const float* A, const voi
   b.softplus = delta_softplus ? 1 : 0;
   b.rows16 = vec ? 1 : 0;
   b.need_bc = (dB || dC) ? 1 : 0;
-  if ((e = ssm::launch_ssd_bwd(b, s)) != cudaSuccess)
+  b.nseg = l.seg.nseg;
+  b.cps = l.seg.cps;
+  if (l.seg.nseg > 1) {
+    // each segment's adjoint from zero at its end, then the chain of the segments in reverse
+    b.mu_sum = musum;
+    b.dsum = dsum;
+    b.mu_in = muin;
+    if ((e = ssm::launch_ssd_bwd(b, true, s)) != cudaSuccess)
+      return cuda_fail(e, "backward: segment summaries (chunked matrix form)");
+    const long long nch = (long long)batch * dim, n = nch * dstate;
+    chain_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(musum, dsum, A, 1, dhL, muin,
+                                                             l.seg.nseg, nch, dim, dstate);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward: adjoint chain");
+  }
+  if ((e = ssm::launch_ssd_bwd(b, false, s)) != cudaSuccess)
     return cuda_fail(e, "backward pass (chunked matrix form)");
   if ((e = ssm::launch_ssd_bwd_finish(b, dB, dC, dA, dD, ddt_bias, s)) != cudaSuccess)
     return cuda_fail(e, "backward reduction (chunked matrix form)");

@@ -141,13 +141,20 @@ struct SsdBwdArgs {
   uint16_t* dz;
   float* dh0;
   float* part_bc;           // [CTAs per row][batch][2][N][L]: each CTA's dB, dC
-  float* part_adt;          // [batch][dim][3]: dA, dD, ddt_bias of each (row, channel)
+  float* part_adt;          // [nseg][batch][dim][3]: dA, dD, ddt_bias of each (segment, row, channel)
+  // time split (nseg segments of cps chunks): the summary launch writes each segment's μ at its
+  // start from μ = 0 at its end and its ΣΔ, in reverse segment order ([nseg][batch][dim][N] and
+  // [nseg][batch][dim]); mu_in [nseg][batch][dim][N] is their chain (mu_in[0] = dhL)
+  float* mu_sum;
+  float* dsum;
+  const float* mu_in;
+  int nseg, cps;
   int batch, dim, L, N, bc_groups, softplus, rows16, need_bc;
 };
 // 64 channels per CTA (dim / bc_groups a multiple of 64 with groups); a.ck from launch_ssd_fwd's
 // checkpoint mode.  The finishing launch sums part_bc over each group's CTAs into dB, dC (bf16)
 // and part_adt over the batch into dA, dD, ddt_bias.
-cudaError_t launch_ssd_bwd(const SsdBwdArgs& a, cudaStream_t s);
+cudaError_t launch_ssd_bwd(const SsdBwdArgs& a, bool summary, cudaStream_t s);
 cudaError_t launch_ssd_bwd_finish(const SsdBwdArgs& a, void* dB, void* dC, float* dA, float* dD,
                                   float* ddt_bias, cudaStream_t s);
 int ssd_bwd_ctas_per_row(int dim);

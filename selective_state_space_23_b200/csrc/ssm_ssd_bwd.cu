@@ -82,7 +82,35 @@ __device__ __forceinline__ uint32_t ldp(const uint16_t* p, long long t, int L, b
 }
 __device__ __forceinline__ float pick(uint32_t w, int odd) { return odd ? bf16_hi(w) : bf16_lo(w); }
 
+// μ <- e^{a_15} μ + (g E) C for the warp's 16 channels: μ in the lane's float4 slots (one per
+// n tile), (g E) as bf16 pairs plus remainders, C exact bf16 from the ring.
 template <int N>
+__device__ __forceinline__ void carry_mu(float4* mus, const SsdStage<N>& st, int lane,
+                                         const uint32_t (&geA)[4], const uint32_t (&gel)[4],
+                                         const float (&Eend)[2]) {
+#pragma unroll
+  for (int nt = 0; nt < N / 8; nt += 2) {
+    uint32_t cn[4];
+    ldsm_x4(cn, blk(st.Cs, 8 * nt, lane));
+    const float4 m0 = mus[nt * 32], m1 = mus[(nt + 1) * 32];
+    float u0[4] = {m0.x * Eend[0], m0.y * Eend[0], m0.z * Eend[1], m0.w * Eend[1]};
+    float u1[4] = {m1.x * Eend[0], m1.y * Eend[0], m1.z * Eend[1], m1.w * Eend[1]};
+    mma16816(u0, geA[0], geA[1], geA[2], geA[3], cn[0], cn[1]);
+    mma16816(u1, geA[0], geA[1], geA[2], geA[3], cn[2], cn[3]);
+    mma16816(u0, gel[0], gel[1], gel[2], gel[3], cn[0], cn[1]);
+    mma16816(u1, gel[0], gel[1], gel[2], gel[3], cn[2], cn[3]);
+    mus[nt * 32] = make_float4(u0[0], u0[1], u0[2], u0[3]);
+    mus[(nt + 1) * 32] = make_float4(u1[0], u1[1], u1[2], u1[3]);
+  }
+}
+
+// SUMM: the summary launch of a time split.  Segment seg = blockIdx.y + 1 is walked in reverse
+// from μ = 0 at its end, keeping only the adjoint's carry; its μ at the segment start and its
+// Kahan-summed ΣΔ go to a.mu_sum / a.dsum at index nseg - 1 - seg (segments in reverse order,
+// the order the segment chain composes them).  Otherwise blockIdx.y is the segment, which starts
+// from μ = a.mu_in[nseg - 1 - seg] (the chained adjoint; dhL for the last segment, or dhL
+// itself without a split).
+template <int N, bool SUMM>
 __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant__ SsdBwdArgs a) {
   constexpr int kNT = N / 8;
   extern __shared__ float4 smem_sb[];
@@ -96,6 +124,10 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
   const int L = a.L;
   const int nck = (L + kT - 1) / kT;
   const long long nslots = nck + 1;
+  const int seg = SUMM ? blockIdx.y + 1 : blockIdx.y;
+  const int kc0 = seg * a.cps, kc1 = min(nck, kc0 + a.cps);  // this segment's chunks
+  const int nloc = kc1 - kc0;
+  const long long nch = (long long)a.batch * a.dim;
   const int gbc = d0 / (a.dim / a.bc_groups);
   const uint16_t* Bg = a.B + ((long long)b * a.bc_groups + gbc) * N * (long long)L;
   const uint16_t* Cg = a.C + ((long long)b * a.bc_groups + gbc) * N * (long long)L;
@@ -126,13 +158,15 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
   // +1).  It lives in shared memory, one float4 per lane and tile that no other lane touches,
   // which frees N / 2 registers; the accesses are conflict-free and need no barrier.
   float4* mus = &sm.mu[warp * kNT * 32 + lane];
+  const float* mu0 = SUMM ? nullptr
+                          : (a.nseg > 1 ? a.mu_in + (long long)(a.nseg - 1 - seg) * nch * N : a.dhL);
 #pragma unroll
   for (int nt = 0; nt < kNT; ++nt) {
     float v[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int c = e >> 1, n = 8 * nt + 2 * tg + (e & 1);
-      v[e] = a.dhL && act[c] ? a.dhL[((long long)b * a.dim + dch[c]) * N + n] : 0.f;
+      v[e] = mu0 && act[c] ? mu0[((long long)b * a.dim + dch[c]) * N + n] : 0.f;
     }
     mus[nt * 32] = make_float4(v[0], v[1], v[2], v[3]);
   }
@@ -142,17 +176,20 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
   };
 
   float accA[2] = {0.f, 0.f}, accD[2] = {0.f, 0.f}, accT[2] = {0.f, 0.f};
+  float dacc[2] = {0.f, 0.f}, dcmp[2] = {0.f, 0.f};  // ΣΔ of the segment (summary, Kahan)
 
-  // B/C tiles and the entering state of chunk nck-1-i into ring slot i % kStB (chunks walked
-  // in reverse)
+  // B/C tiles and the entering state of chunk kc1-1-i into ring slot i % kStB (chunks walked
+  // in reverse; the summary needs no entering states)
   const auto issue = [&](int i) {
-    if (i < nck) {
+    if (i < nloc) {
       SsdStage<N>& st = sm.ring[i % kStB];
-      const int t0 = (nck - 1 - i) * kT;
-      const float4* src = ckb + (long long)(nck - 1 - i) * ngrp * kNT * 32;
-      for (int p = tid; p < kWb * kNT * 32; p += 32 * kWb) {
-        const int j = p / (kNT * 32);
-        cp16(&sm.hs[i % kStB][p], src + (min(j, gvalid - 1) - j) * kNT * 32 + p);
+      const int t0 = (kc1 - 1 - i) * kT;
+      if (!SUMM) {
+        const float4* src = ckb + (long long)(kc1 - 1 - i) * ngrp * kNT * 32;
+        for (int p = tid; p < kWb * kNT * 32; p += 32 * kWb) {
+          const int j = p / (kNT * 32);
+          cp16(&sm.hs[i % kStB][p], src + (min(j, gvalid - 1) - j) * kNT * 32 + p);
+        }
       }
       if (a.rows16 && t0 + kT <= L) {
         for (int p = tid; p < 4 * N; p += 32 * kWb) {
@@ -189,15 +226,15 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
 #pragma unroll
   for (int i = 0; i < kStB - 1; ++i) issue(i);
   ChunkInB nxt;
-  load_in(nck - 1, nxt);
+  load_in(kc1 - 1, nxt);
 
-  for (int i = 0; i < nck; ++i) {
-    const int k = nck - 1 - i;
+  for (int i = 0; i < nloc; ++i) {
+    const int k = kc1 - 1 - i;
     cp_wait<kStB - 2>();
     __syncthreads();  // chunk k's B/C and state landed; every warp is done with the previous chunk
     issue(i + kStB - 1);
     const ChunkInB cur = nxt;
-    if (k > 0) load_in(k - 1, nxt);
+    if (k > kc0) load_in(k - 1, nxt);
     const SsdStage<N>& st = sm.ring[i % kStB];
     const float4* hsw = &sm.hs[i % kStB][warp * kNT * 32 + lane];
     // the entering state: states 8 nt + 2 tg, +1 of channel g + 8 c
@@ -269,9 +306,26 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
       ok &= __shfl_xor_sync(0xffffffffu, ok, 2, 4);
       fb[c] = ok == 0;
     }
+    if constexpr (SUMM) {  // the adjoint's carry only: μ <- e^{a_15} μ + (g E) C
+      float Eend[2];
+      uint32_t geA[4], gel[4];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const float yk = Se[c] - dcmp[c], tk = dacc[c] + yk;
+        dcmp[c] = (tk - dacc[c]) - yk;
+        dacc[c] = tk;
+        Eend[c] = ex2_mufu(Se[c] * al[c]);
+        float ge[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) ge[j] = gg[c][j] * ex2_mufu(S[c][j] * al[c]);
+        split_bf16x2(ge[0], ge[1], geA[c], gel[c]);
+        split_bf16x2(ge[2], ge[3], geA[2 + c], gel[2 + c]);
+      }
+      carry_mu<N>(mus, st, lane, geA, gel, Eend);
+      continue;
+    }
     // decay factors: P, Q about the middle step for the factorised products; E_t = e^{a_t} and
-    // e^{a_15 - a_s} directly for channels outside the range (both <= 1)
-    // The per-step factors (P, Q, E, e^{a_15 - a_s}) are formed here for the operands and again
+    // e^{a_15 - a_s} directly for channels outside the range (both <= 1).  The per-step factors (P, Q, E, e^{a_15 - a_s}) are formed here for the operands and again
     // after the products, rather than kept live through them.
     float eAm[2], eEm[2], Eend[2];
     // A fragments (bf16 pairs) and, for the products that feed dΔ, dA and the carried adjoint,
@@ -575,20 +629,7 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
     }
 
     // ---- carry μ back to the previous chunk: μ <- e^{a_15} μ + (g E) C
-#pragma unroll
-    for (int nt = 0; nt < kNT; nt += 2) {
-      uint32_t cn[4];
-      ldsm_x4(cn, blk(st.Cs, 8 * nt, lane));
-      const float4 m0 = mus[nt * 32], m1 = mus[(nt + 1) * 32];
-      float u0[4] = {m0.x * Eend[0], m0.y * Eend[0], m0.z * Eend[1], m0.w * Eend[1]};
-      float u1[4] = {m1.x * Eend[0], m1.y * Eend[0], m1.z * Eend[1], m1.w * Eend[1]};
-      mma16816(u0, geA[0], geA[1], geA[2], geA[3], cn[0], cn[1]);
-      mma16816(u1, geA[0], geA[1], geA[2], geA[3], cn[2], cn[3]);
-      mma16816(u0, gel[0], gel[1], gel[2], gel[3], cn[0], cn[1]);
-      mma16816(u1, gel[0], gel[1], gel[2], gel[3], cn[2], cn[3]);
-      mus[nt * 32] = make_float4(u0[0], u0[1], u0[2], u0[3]);
-      mus[(nt + 1) * 32] = make_float4(u1[0], u1[1], u1[2], u1[3]);
-    }
+    carry_mu<N>(mus, st, lane, geA, gel, Eend);
 
     // ---- dL/da and its reverse cumulative sum over the chunk
     float dS[2][4];
@@ -701,7 +742,24 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
   }
   cp_wait<0>();
 
-  // dh0 and the per-channel parameter gradients
+  if constexpr (SUMM) {  // the segment's μ at its start and its ΣΔ, in reverse segment order
+    const long long r = a.nseg - 1 - seg;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      if (!act[c]) continue;
+      const long long ch = (long long)b * a.dim + dch[c];
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt) {
+        const float2 mv = mupair(nt, c);
+        a.mu_sum[(r * nch + ch) * N + 8 * nt + 2 * tg] = mv.x;
+        a.mu_sum[(r * nch + ch) * N + 8 * nt + 2 * tg + 1] = mv.y;
+      }
+      if (tg == 0) a.dsum[r * nch + ch] = dacc[c];
+    }
+    return;
+  }
+
+  // dh0 (the first segment) and the per-channel parameter gradients of the segment
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
     float vA = accA[c], vD = accD[c], vT = accT[c];
@@ -713,7 +771,7 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
     vT += __shfl_xor_sync(0xffffffffu, vT, 2);
     if (!act[c]) continue;
     const long long ch = (long long)b * a.dim + dch[c];
-    if (a.dh0) {
+    if (a.dh0 && seg == 0) {
 #pragma unroll
       for (int nt = 0; nt < kNT; ++nt) {
         const float2 mv = mupair(nt, c);
@@ -722,9 +780,10 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
       }
     }
     if (tg == 0) {
-      a.part_adt[ch * 3 + 0] = vA;
-      a.part_adt[ch * 3 + 1] = vD;
-      a.part_adt[ch * 3 + 2] = vT;
+      float* pa = a.part_adt + ((long long)seg * nch + ch) * 3;
+      pa[0] = vA;
+      pa[1] = vD;
+      pa[2] = vT;
     }
   }
 }
@@ -760,24 +819,26 @@ __global__ void ssd_finish_bc(const SsdBwdArgs a, uint16_t* dB, uint16_t* dC, in
   if (dst) dst[(((long long)b * a.bc_groups + gb) * a.N + n) * a.L + t] = f32_to_bf16(s);
 }
 
-// dA, dD, ddt_bias: the rows' partials summed in row order.
+// dA, dD, ddt_bias: the (segment, row) partials summed in segment-major order.
 __global__ void ssd_finish_adt(const SsdBwdArgs a, float* dA, float* dD, float* ddt_bias) {
   const int d = blockIdx.x * blockDim.x + threadIdx.x;
   if (d >= a.dim) return;
   float s[3] = {0.f, 0.f, 0.f};
-  for (int b = 0; b < a.batch; ++b)
+  for (long long r = 0; r < (long long)a.nseg * a.batch; ++r)
 #pragma unroll
-    for (int k = 0; k < 3; ++k) s[k] += a.part_adt[((long long)b * a.dim + d) * 3 + k];
+    for (int k = 0; k < 3; ++k) s[k] += a.part_adt[(r * a.dim + d) * 3 + k];
   if (dA) dA[d] = s[0];
   if (dD) dD[d] = s[1];
   if (ddt_bias) ddt_bias[d] = s[2];
 }
 
-template <int N>
+template <int N, bool SUMM>
 cudaError_t launch_n(const SsdBwdArgs& a, cudaStream_t s) {
-  const unsigned grid = (unsigned)((long long)a.batch * ((a.dim + 16 * kWb - 1) / (16 * kWb)));
+  const dim3 grid((unsigned)((long long)a.batch * ((a.dim + 16 * kWb - 1) / (16 * kWb))),
+                  (unsigned)(SUMM ? a.nseg - 1 : a.nseg));
+  if (grid.y == 0) return cudaSuccess;
   const size_t smem = sizeof(BwdSmem<N>);
-  auto k = ssd_bwd_kernel<N>;
+  auto k = ssd_bwd_kernel<N, SUMM>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   k<<<grid, 32 * kWb, smem, s>>>(a);
@@ -788,12 +849,12 @@ cudaError_t launch_n(const SsdBwdArgs& a, cudaStream_t s) {
 
 int ssd_bwd_ctas_per_row(int dim) { return (dim + 16 * kWb - 1) / (16 * kWb); }
 
-cudaError_t launch_ssd_bwd(const SsdBwdArgs& a, cudaStream_t s) {
+cudaError_t launch_ssd_bwd(const SsdBwdArgs& a, bool summary, cudaStream_t s) {
   switch (a.N) {
-    case 16: return launch_n<16>(a, s);
-    case 32: return launch_n<32>(a, s);
-    case 64: return launch_n<64>(a, s);
-    case 128: return launch_n<128>(a, s);
+    case 16: return summary ? launch_n<16, true>(a, s) : launch_n<16, false>(a, s);
+    case 32: return summary ? launch_n<32, true>(a, s) : launch_n<32, false>(a, s);
+    case 64: return summary ? launch_n<64, true>(a, s) : launch_n<64, false>(a, s);
+    case 128: return summary ? launch_n<128, true>(a, s) : launch_n<128, false>(a, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -191,13 +191,15 @@ BWD_CASES = {
     "scalar_decay_n64_slices": ({"SSM_SCALAR_BWD": "slices"}, 2, 96, 120, 64, torch.bfloat16, 1, 1),
     "scalar_decay_n64_chunked": ({}, 2, 96, 120, 64, torch.bfloat16, 1, 1),
     "scalar_decay_n128_chunked": ({}, 1, 80, 333, 128, torch.bfloat16, 1, 1),
+    "scalar_decay_n64_chunked_split": ({"SSM_SSD_BWD_SPLIT": "3"}, 1, 80, 333, 64, torch.bfloat16, 1, 1),
 }
 
 
 @pytest.mark.parametrize("case", sorted(BWD_CASES))
 def test_backward_stays_inside_its_tensors(monkeypatch, case):
     env, batch, dim, L, N, io, G, flags = BWD_CASES[case]
-    for k in ("SSM_FWD_KERNEL", "SSM_BWD_KERNEL", "SSM_BWD_WPB", "SSM_BWD_SPLIT", "SSM_SCALAR_BWD"):
+    for k in ("SSM_FWD_KERNEL", "SSM_BWD_KERNEL", "SSM_BWD_WPB", "SSM_BWD_SPLIT", "SSM_SCALAR_BWD",
+              "SSM_SSD_BWD_SPLIT"):
         monkeypatch.delenv(k, raising=False)
     for k, v in env.items():
         monkeypatch.setenv(k, v)

@@ -156,3 +156,40 @@ def test_chunked_backward_with_time_split_checkpoints():
     r = ref(x, None)
     for k in GRADS:
         assert_close(g[k], r[k], torch.bfloat16, k)
+
+
+@pytest.mark.parametrize("N", [16, 64, 128])
+@pytest.mark.parametrize("split", ["3", "7"])
+def test_chunked_backward_forced_time_split(monkeypatch, N, split):
+    """Forced segments of the reverse walk (summary launch, adjoint chain, segment launch) over a
+    ragged tail, with dhL and h0: the same gradients as the oracle."""
+    monkeypatch.setenv("SSM_SSD_BWD_SPLIT", split)
+    x = inputs(2, 128, 333, N, torch.bfloat16, seed=116)
+    dhL = torch.randn((2, 128, N), generator=torch.Generator().manual_seed(10))
+    g = run(x, dhL)
+    r = ref(x, dhL)
+    for k in GRADS:
+        assert_close(g[k], r[k], torch.bfloat16, k)
+
+
+def test_chunked_backward_long_sequence_splits_by_itself(monkeypatch):
+    """64 channels over 16384 steps: one CTA of channels, so the planner cuts the reverse walk
+    into segments (and the checkpoint pass into its own)."""
+    monkeypatch.delenv("SSM_SSD_BWD_SPLIT", raising=False)
+    x = inputs(1, 64, 16384, 64, torch.bfloat16, seed=117)
+    dhL = torch.randn((1, 64, 64), generator=torch.Generator().manual_seed(11))
+    g = run(x, dhL)
+    r = ref(x, dhL)
+    for k in GRADS:
+        assert_close(g[k], r[k], torch.bfloat16, k)
+
+
+def test_chunked_backward_split_agrees_with_unsplit(monkeypatch):
+    """The split walk against the unsplit one on the same inputs (both in f32 accumulation)."""
+    x = inputs(1, 128, 1024, 64, torch.bfloat16, seed=118)
+    monkeypatch.setenv("SSM_SSD_BWD_SPLIT", "1")
+    a = run(x, None)
+    monkeypatch.setenv("SSM_SSD_BWD_SPLIT", "8")
+    b = run(x, None)
+    for k in GRADS:
+        assert_close(a[k], f64(b[k]), torch.bfloat16, k)
