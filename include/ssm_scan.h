@@ -157,24 +157,25 @@ SSM_API int ssm_scan_bwd(const void* u, const void* delta, const float* A, const
  * aligned): A broadcast to [dim][dstate] and the per-state dA, followed by the workspace of
  * ssm_scan_bwd for the same shape.  Checkpoints of ssm_scan_fwd_scalar_a feed the backward.
  * dstate may be up to SSM_MAX_DSTATE_SCALAR in the forward scan: above 16 (and at 16 for bf16
- * calls without checkpoints, the default layout and no other flag) it runs in the chunked
- * matrix form (per 16-step chunk and 64-channel tile, the products C B^T, masked with the decay
- * factors, times the step-scaled inputs, plus C times the entering state: the structured-matrix
- * view of the scan in the Mamba-2 notes of the same page) on the tensor cores.  That form takes
- * bf16 io, dstate 32, 64 or 128, the forward direction without SSM_ZOH, the default layout, no
- * checkpoints, and B/C groups of whole 64-channel tiles; other forward requests with dstate > 16
- * return SSM_EUNSUPPORTED.  The backward with dstate = 32, 64 or 128 takes ckpt = NULL (the
- * states are recomputed).  For bf16 io, no flag but SSM_SCALAR_A, B/C shared or in groups of
- * whole 64-channel tiles, and no checkpoints, the backward with dstate = 16, 32, 64 or 128 runs
- * in the chunked matrix form on the tensor cores: a forward pass writes the f32 state entering
- * every 16-step chunk into the workspace, then the chunks are walked in reverse with the adjoint
- * of the state (the chain rule through the products above).  Other requests with dstate > 16
- * (f32, reverse, ZOH, other groupings) run as the sum of the 16-state backwards of the state
- * slices (the states of a scalar-decay scan do not interact; D enters one slice); with
- * dstate <= 16 they run the per-state backward.  ssm_scan_bwd_scalar_a_workspace_size() covers
- * the scratch of the path the call takes (chunk states and per-CTA dB/dC partials; slice copies
- * of B, C, h0, dhL, per-slice gradients and f32 sums; or A broadcast plus the per-state
- * backward's workspace).
+ * calls in the default layout with no other flag) it runs in the chunked matrix form (per
+ * 16-step chunk and 64-channel tile, the products C B^T, masked with the decay factors, times
+ * the step-scaled inputs, plus C times the entering state: the structured-matrix view of the
+ * scan in the Mamba-2 notes of the same page) on the tensor cores.  That form takes bf16 io,
+ * dstate 16, 32, 64 or 128, the forward direction without SSM_ZOH, the default layout and B/C
+ * groups of whole 64-channel tiles; other forward requests with dstate > 16 return
+ * SSM_EUNSUPPORTED.  Its checkpoints (ckpt, 16-byte aligned) have the layout and meaning of the
+ * per-state scan's: the f32 state entering every 16-step block, [batch][dim][ceil(L/16)][dstate].
+ * For bf16 io, no flag but SSM_SCALAR_A and B/C shared or in groups of whole 64-channel tiles,
+ * the backward with dstate = 16, 32, 64 or 128 runs in the chunked matrix form too: the chunks
+ * are walked in reverse with the adjoint of the state (the chain rule through the products
+ * above), from the caller's checkpoints (either forward's; 16-byte aligned) or, with
+ * ckpt = NULL, from a checkpoint pass into the workspace.  Other requests with dstate > 16
+ * (f32, reverse, ZOH, other groupings) take ckpt = NULL and run as the sum of the 16-state
+ * backwards of the state slices (the states of a scalar-decay scan do not interact; D enters
+ * one slice); with dstate <= 16 they run the per-state backward.
+ * ssm_scan_bwd_scalar_a_workspace_size() covers the scratch of the path the call takes (chunk
+ * states unless given, and per-CTA dB/dC partials; slice copies of B, C, h0, dhL, per-slice
+ * gradients and f32 sums; or A broadcast plus the per-state backward's workspace).
  */
 SSM_API size_t ssm_scan_fwd_scalar_a_workspace_size(int batch, int dim, int seqlen, int dstate,
                                                     int io_dtype);

@@ -400,25 +400,27 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
                    aligned16(C);
   // scalar decay with N > 16: the chunked matrix form on the tensor cores (bf16, N = 32, 64 or
   // 128, forward direction, [batch][dim][L] rows, B/C shared by each 64-channel tile).  With
-  // N = 16 the same form serves the requests it takes (no checkpoints); SSM_SCALAR_FORM=state
-  // keeps those on the per-state kernel.
+  // N = 16 the same form serves the requests it takes; SSM_SCALAR_FORM=state keeps those on the
+  // per-state kernel.  Both write the same checkpoints (the state entering every 16-step block).
   const char* sform = getenv("SSM_SCALAR_FORM");
-  const bool chunked16 = scalar_a && dstate == ssm::kNS && io_dtype == SSM_BF16 && !ckpt &&
+  const bool chunked16 = scalar_a && dstate == ssm::kNS && io_dtype == SSM_BF16 &&
                          !(flags & (SSM_ZOH | SSM_REVERSE | SSM_CHANNELS_LAST)) &&
                          (bc_groups == 1 || (dim % bc_groups == 0 && (dim / bc_groups) % 64 == 0)) &&
                          !(sform && strcmp(sform, "state") == 0);
   if (dstate > SSM_MAX_DSTATE || chunked16) {
     if (io_dtype != SSM_BF16 || (dstate != 16 && dstate != 32 && dstate != 64 && dstate != 128) || zoh ||
-        reverse || channels_last || ckpt ||
+        reverse || channels_last ||
         !(bc_groups == 1 || (dim % bc_groups == 0 && (dim / bc_groups) % 64 == 0)))
       return fail(SSM_EUNSUPPORTED,
                   "scalar decay with dstate %d > %d needs bf16 io, dstate 32, 64 or 128, the "
-                  "forward direction without ZOH, the default layout, no checkpoints and B/C "
-                  "groups of whole 64-channel tiles", dstate, SSM_MAX_DSTATE);
+                  "forward direction without ZOH, the default layout and B/C groups of whole "
+                  "64-channel tiles", dstate, SSM_MAX_DSTATE);
+    if (!aligned16(ckpt))
+      return fail(SSM_EINVAL, "ckpt must be 16-byte aligned (chunked matrix form)");
     ssm::FwdArgs a;
     memset(&a, 0, sizeof(a));
     a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
-    a.A = A; a.D = D; a.dt_bias = dt_bias; a.h0 = h0; a.out = out; a.hL = hL;
+    a.A = A; a.D = D; a.dt_bias = dt_bias; a.h0 = h0; a.out = out; a.hL = hL; a.ckpt = ckpt;
     a.batch = batch; a.dim = dim; a.L = seqlen; a.N = dstate;
     a.softplus = delta_softplus ? 1 : 0;
     a.scalar_a = 1;
@@ -909,17 +911,19 @@ struct ChunkedBwdLayout {
   BwdSegPlan seg;
 };
 
-ChunkedBwdLayout chunked_bwd_layout(int batch, int dim, int seqlen, int dstate) {
+// have_ckpt: the caller passes the forward's checkpoints (no checkpoint pass, no room for them)
+ChunkedBwdLayout chunked_bwd_layout(int batch, int dim, int seqlen, int dstate, bool have_ckpt) {
   ChunkedBwdLayout l;
   l.seg = plan_ssd_bwd(batch, dim, seqlen, dstate);
   const size_t nch = (size_t)batch * dim, S = (size_t)l.seg.nseg;
-  l.ck = align_up((size_t)ssm::ssd_ckpt_floats(batch, dim, seqlen, dstate) * 4);
+  const size_t nck = (seqlen + ssm::kBlk - 1) / ssm::kBlk;
+  l.ck = have_ckpt ? 0 : align_up(nch * nck * dstate * 4);
   l.pbc = align_up((size_t)ssm::ssd_bwd_ctas_per_row(dim) * batch * 2 * dstate * seqlen * 4);
   l.padt = align_up(S * nch * 3 * 4);
   l.musum = S > 1 ? align_up(S * nch * dstate * 4) : 0;
   l.dsum = S > 1 ? align_up(S * nch * 4) : 0;
   l.muin = l.musum;
-  l.fwd = plan_ssd(batch, dim, seqlen, dstate).ws_bytes;
+  l.fwd = have_ckpt ? 0 : plan_ssd(batch, dim, seqlen, dstate).ws_bytes;
   l.total = l.ck + l.pbc + l.padt + l.musum + l.dsum + l.muin + l.fwd;
   return l;
 }
@@ -927,7 +931,7 @@ ChunkedBwdLayout chunked_bwd_layout(int batch, int dim, int seqlen, int dstate) 
 int scan_bwd_chunked(const void* u, const void* delta, const float* A, const void* B,
                      const void* C, const float* D, const void* z, const float* dt_bias,
                      int delta_softplus, const float* h0, const void* dout, const float* dhL,
-                     void* du, void* ddelta, float* dA, void* dB, void* dC, float* dD, void* dz,
+                     const float* ckpt, void* du, void* ddelta, float* dA, void* dB, void* dC, float* dD, void* dz,
                      float* ddt_bias, float* dh0, void* workspace, size_t workspace_bytes,
                      int batch, int dim, int seqlen, int dstate, int bc_groups, void* stream) {
   const size_t es = 2;
@@ -954,17 +958,21 @@ int scan_bwd_chunked(const void* u, const void* delta, const float* A, const voi
   TRY(check_opt(dD, (size_t)dim * 4, 4, "dD"));
   TRY(check_opt(ddt_bias, (size_t)dim * 4, 4, "ddt_bias"));
   TRY(check_opt(dh0, nst, 4, "dh0"));
+  const size_t nck = (seqlen + ssm::kBlk - 1) / ssm::kBlk;
+  TRY(check_opt(ckpt, (size_t)batch * dim * nck * dstate * 4, 4, "ckpt"));
+  if (!aligned16(ckpt))
+    return fail(SSM_EINVAL, "ckpt must be 16-byte aligned (chunked matrix form)");
   if (!du && !ddelta && !dA && !dB && !dC && !dD && !dz && !ddt_bias && !dh0)
     return fail(SSM_EINVAL, "no gradient output requested");
   if (dz && !z) return fail(SSM_EINVAL, "dz requested but z is NULL");
-  const ChunkedBwdLayout l = chunked_bwd_layout(batch, dim, seqlen, dstate);
+  const ChunkedBwdLayout l = chunked_bwd_layout(batch, dim, seqlen, dstate, ckpt != nullptr);
   if (!workspace || workspace_bytes < l.total)
     return fail(SSM_EWORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes, l.total);
   if (reinterpret_cast<uintptr_t>(workspace) & 255)
     return fail(SSM_EINVAL, "workspace is not 256-byte aligned");
   TRY(check_ptr(workspace, l.total, 256, "workspace"));
   char* w = reinterpret_cast<char*>(workspace);
-  float* ck = reinterpret_cast<float*>(w);
+  float* ck = ckpt ? nullptr : reinterpret_cast<float*>(w);
   float* pbc = reinterpret_cast<float*>(w + l.ck);
   float* padt = reinterpret_cast<float*>(w + l.ck + l.pbc);
   float* musum = reinterpret_cast<float*>(w + l.ck + l.pbc + l.padt);
@@ -974,38 +982,40 @@ int scan_bwd_chunked(const void* u, const void* delta, const float* A, const voi
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool vec = (seqlen * es) % 16 == 0 && aligned16(u) && aligned16(delta) && aligned16(z) &&
                    aligned16(B) && aligned16(C);
-  // the state entering every chunk, from the forward in checkpoint mode
-  ssm::FwdArgs a;
-  memset(&a, 0, sizeof(a));
-  a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
-  a.A = A; a.dt_bias = dt_bias; a.h0 = h0;
-  a.ckpt = ck;  // the state entering every chunk, in fragment order
-  a.batch = batch; a.dim = dim; a.L = seqlen; a.N = dstate;
-  a.softplus = delta_softplus ? 1 : 0;
-  a.scalar_a = 1;
-  a.bc_groups = bc_groups;
-  a.rows16 = vec ? 1 : 0;
-  const FwdPlan plan = plan_ssd(batch, dim, seqlen, dstate);
-  a.chunk_len = plan.chunk_len;
-  a.nchunk = plan.nchunk;
   cudaError_t e;
-  if (plan.nchunk > 1) {
-    const size_t nch = (size_t)batch * dim;
-    const size_t seg = align_up((size_t)plan.nchunk * nch * dstate * 4);
-    a.summ = reinterpret_cast<float*>(fws);
-    float* hin = reinterpret_cast<float*>(fws + seg);
-    a.dsum = reinterpret_cast<float*>(fws + 2 * seg);
-    if ((e = ssm::launch_ssd_fwd(a, ssm::kSsdSummary, s)) != cudaSuccess)
-      return cuda_fail(e, "backward: summary pass (chunked matrix form)");
-    const long long n = (long long)nch * dstate;
-    chain_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(a.summ, a.dsum, A, 1, h0, hin,
-                                                             plan.nchunk, (long long)nch, dim,
-                                                             dstate);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward: carry");
-    a.hin = hin;
+  if (!ckpt) {
+    // the state entering every chunk, from the forward in checkpoint mode
+    ssm::FwdArgs a;
+    memset(&a, 0, sizeof(a));
+    a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
+    a.A = A; a.dt_bias = dt_bias; a.h0 = h0;
+    a.ckpt = ck;  // the state entering every chunk
+    a.batch = batch; a.dim = dim; a.L = seqlen; a.N = dstate;
+    a.softplus = delta_softplus ? 1 : 0;
+    a.scalar_a = 1;
+    a.bc_groups = bc_groups;
+    a.rows16 = vec ? 1 : 0;
+    const FwdPlan plan = plan_ssd(batch, dim, seqlen, dstate);
+    a.chunk_len = plan.chunk_len;
+    a.nchunk = plan.nchunk;
+    if (plan.nchunk > 1) {
+      const size_t nch = (size_t)batch * dim;
+      const size_t seg = align_up((size_t)plan.nchunk * nch * dstate * 4);
+      a.summ = reinterpret_cast<float*>(fws);
+      float* hin = reinterpret_cast<float*>(fws + seg);
+      a.dsum = reinterpret_cast<float*>(fws + 2 * seg);
+      if ((e = ssm::launch_ssd_fwd(a, ssm::kSsdSummary, s)) != cudaSuccess)
+        return cuda_fail(e, "backward: summary pass (chunked matrix form)");
+      const long long n = (long long)nch * dstate;
+      chain_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(a.summ, a.dsum, A, 1, h0, hin,
+                                                               plan.nchunk, (long long)nch, dim,
+                                                               dstate);
+      if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward: carry");
+      a.hin = hin;
+    }
+    if ((e = ssm::launch_ssd_fwd(a, ssm::kSsdCkpt, s)) != cudaSuccess)
+      return cuda_fail(e, "backward: checkpoint pass (chunked matrix form)");
   }
-  if ((e = ssm::launch_ssd_fwd(a, ssm::kSsdCkpt, s)) != cudaSuccess)
-    return cuda_fail(e, "backward: checkpoint pass (chunked matrix form)");
   ssm::SsdBwdArgs b;
   memset(&b, 0, sizeof(b));
   b.u = reinterpret_cast<const uint16_t*>(u);
@@ -1015,7 +1025,7 @@ int scan_bwd_chunked(const void* u, const void* delta, const float* A, const voi
   b.C = reinterpret_cast<const uint16_t*>(C);
   b.dout = reinterpret_cast<const uint16_t*>(dout);
   b.A = A; b.D = D; b.dt_bias = dt_bias; b.dhL = dhL;
-  b.ck = ck;
+  b.ck = ckpt ? ckpt : ck;
   b.du = reinterpret_cast<uint16_t*>(du);
   b.ddelta = reinterpret_cast<uint16_t*>(ddelta);
   b.dz = reinterpret_cast<uint16_t*>(dz);
@@ -1067,14 +1077,14 @@ size_t ssm_scan_bwd_ex_workspace_size(int batch, int dim, int seqlen, int dstate
                                       int io_dtype, int have_ckpt, int flags) {
   if (flags & ~(SSM_SCALAR_A | SSM_REVERSE | SSM_ZOH | SSM_CHANNELS_LAST)) return 0;
   if ((flags & SSM_SCALAR_A) && dstate > SSM_MAX_DSTATE) {  // chunked form, or slices
-    if (have_ckpt) return 0;
     if (chunked_bwd_ok(dim, dstate, bc_groups, io_dtype, flags))
-      return chunked_bwd_layout(batch, dim, seqlen, dstate).total;
+      return chunked_bwd_layout(batch, dim, seqlen, dstate, have_ckpt != 0).total;
+    if (have_ckpt) return 0;
     return ssm::scan_bwd_slices_workspace(batch, dim, seqlen, dstate, bc_groups, io_dtype, flags);
   }
-  if (dstate == 16 && !have_ckpt && chunked_bwd_ok(dim, dstate, bc_groups, io_dtype, flags)) {
+  if (dstate == 16 && chunked_bwd_ok(dim, dstate, bc_groups, io_dtype, flags)) {
     if (check_dims(batch, dim, seqlen, dstate, io_dtype) != SSM_OK) return 0;
-    return chunked_bwd_layout(batch, dim, seqlen, dstate).total;
+    return chunked_bwd_layout(batch, dim, seqlen, dstate, have_ckpt != 0).total;
   }
   if (check_dims(batch, dim, seqlen, dstate, io_dtype) != SSM_OK) return 0;
   if (check_groups(dim, bc_groups) != SSM_OK) return 0;
@@ -1099,9 +1109,9 @@ int ssm_scan_bwd_ex(const void* u, const void* delta, const float* A, const void
   if ((flags & SSM_SCALAR_A) && dstate > SSM_MAX_DSTATE) {  // chunked form, or slices
     TRY(check_dims(batch, dim, seqlen, dstate, io_dtype, SSM_MAX_DSTATE_SCALAR));
     TRY(check_groups(dim, bc_groups));
-    if (!ckpt && chunked_bwd_ok(dim, dstate, bc_groups, io_dtype, flags))
+    if (chunked_bwd_ok(dim, dstate, bc_groups, io_dtype, flags))
       return scan_bwd_chunked(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL,
-                              du, ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, workspace,
+                              ckpt, du, ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, workspace,
                               workspace_bytes, batch, dim, seqlen, dstate, bc_groups, stream);
     return ssm::scan_bwd_slices(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL,
                                 ckpt, du, ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, workspace,
@@ -1109,11 +1119,11 @@ int ssm_scan_bwd_ex(const void* u, const void* delta, const float* A, const void
                                 flags, stream);
   }
   TRY(check_dims(batch, dim, seqlen, dstate, io_dtype));
-  if (dstate == 16 && !ckpt && chunked_bwd_ok(dim, dstate, bc_groups, io_dtype, flags)) {
+  if (dstate == 16 && chunked_bwd_ok(dim, dstate, bc_groups, io_dtype, flags)) {
     TRY(check_groups(dim, bc_groups));
-    return scan_bwd_chunked(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL, du,
-                            ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, workspace, workspace_bytes,
-                            batch, dim, seqlen, dstate, bc_groups, stream);
+    return scan_bwd_chunked(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL, ckpt,
+                            du, ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, workspace,
+                            workspace_bytes, batch, dim, seqlen, dstate, bc_groups, stream);
   }
   if (!(flags & SSM_SCALAR_A))
     return scan_bwd_core(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL, ckpt,

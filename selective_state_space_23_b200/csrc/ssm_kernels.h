@@ -135,7 +135,7 @@ struct SsdBwdArgs {
   const float* D;
   const float* dt_bias;
   const float* dhL;
-  const float* ck;          // the state entering every chunk, in the checkpoint mode's fragment order
+  const float* ck;          // [batch][dim][ceil(L/16)][N]: the state entering every chunk
   uint16_t* du;
   uint16_t* ddelta;
   uint16_t* dz;
@@ -158,12 +158,8 @@ cudaError_t launch_ssd_bwd(const SsdBwdArgs& a, bool summary, cudaStream_t s);
 cudaError_t launch_ssd_bwd_finish(const SsdBwdArgs& a, void* dB, void* dC, float* dA, float* dD,
                                   float* ddt_bias, cudaStream_t s);
 int ssd_bwd_ctas_per_row(int dim);
-inline long long ssd_ckpt_floats(int batch, int dim, int L, int N) {
-  return (long long)batch * ((L + 15) / 16 + 1) * ((dim + 15) / 16) * 16 * N;
-}
-// mode: kSsdOut, kSsdSummary, or kSsdCkpt (no outputs; the state entering every chunk and the final
-// state into a.ckpt in MMA fragment order, f32 [batch][ceil(L / 16) + 1][ceil(dim / 16)][N / 8]
-// [32][4]: ssd_ckpt_floats() floats).
+// mode: kSsdOut (with a.ckpt also the checkpoints), kSsdSummary, or kSsdCkpt (no outputs; only
+// the state entering every 16-step chunk into a.ckpt, f32 [batch][dim][ceil(L / 16)][N]).
 enum SsdMode { kSsdOut = 0, kSsdSummary = 1, kSsdCkpt = 2 };
 cudaError_t launch_ssd_fwd(const FwdArgs& a, int mode, cudaStream_t s);
 cudaError_t launch_fwd_carry(const FwdArgs& a, const float* summ, const float* dsum, float* hin,

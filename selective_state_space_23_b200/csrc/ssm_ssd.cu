@@ -69,30 +69,34 @@ __device__ __forceinline__ uint32_t ld_pair(const uint16_t* p, long long t, int 
   return lo | (hi << 16);
 }
 
-// The state of the warp's 16 channels into slot `slot` of the checkpoint array in fragment
-// order, f32 [batch][chunks + 1][ceil(dim / 16)][N / 8][32 lanes][4]: lane l's accumulator
-// registers Ht[nt][0..3] (channels g, g + 8 of the group, states 8 nt + 2 tg, +1) as one float4,
-// so that a 64-channel tile's state of one chunk is one contiguous block and a warp's read of an
-// n8 tile is 512 consecutive bytes.
+// The state entering chunk `slot` (transposed accumulator layout: 2 channels x N/4 states per
+// lane) into the checkpoint array, f32 [batch][dim][ceil(L / 16)][N]: the layout of the
+// per-state scan's checkpoints, which hold the same states (the state entering every 16-step
+// block), so either forward's checkpoints serve either backward.
 template <int N>
 __device__ __forceinline__ void store_state(const FwdArgs& a, const float (&Ht)[N / 8][4],
-                                            int slot, int b, int grp, int lane) {
-  const long long nslots = (a.L + kT - 1) / kT + 1;
-  const int ngrp = (a.dim + 15) / 16;
-  if (grp >= ngrp) return;  // a warp past the last channel
-  float4* dst = reinterpret_cast<float4*>(a.ckpt) +
-                (((long long)b * nslots + slot) * ngrp + grp) * (N / 8) * 32 + lane;
+                                            int slot, int b, const int (&dch)[2],
+                                            const bool (&act)[2], int tg) {
+  const long long nslots = (a.L + kT - 1) / kT;
 #pragma unroll
-  for (int nt = 0; nt < N / 8; ++nt)
-    dst[nt * 32] = make_float4(Ht[nt][0], Ht[nt][1], Ht[nt][2], Ht[nt][3]);
+  for (int c = 0; c < 2; ++c) {
+    if (!act[c]) continue;
+    float* row = a.ckpt + (((long long)b * a.dim + dch[c]) * nslots + slot) * N + 2 * tg;
+#pragma unroll
+    for (int nt = 0; nt < N / 8; ++nt)
+      *reinterpret_cast<float2*>(row + 8 * nt) = make_float2(Ht[nt][2 * c], Ht[nt][2 * c + 1]);
+  }
 }
 
-// MODE: kSsdOut (gated outputs), kSsdSummary (segment end state and ΣΔ from zero), kSsdCkpt (the
-// state entering every chunk, and the final state, into a.ckpt (f32) for the backward).
+// MODE: kSsdOut (gated outputs; with a.ckpt also the state entering every chunk),
+// kSsdSummary (segment end state and ΣΔ from zero), kSsdCkpt (only the state entering every
+// chunk into a.ckpt, for the backward).
 template <int N, int W, int MODE>
 __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__ FwdArgs a) {
   constexpr bool SUMMARY = MODE == kSsdSummary;
   constexpr bool NOOUT = MODE != kSsdOut;  // no gate, readout or outputs
+  // states that a backward or a chain reads take the state update's remainder term too
+  const bool exact = NOOUT || a.ckpt != nullptr;
   constexpr int kNT = N / 8;  // n8 tiles of the state
   extern __shared__ float4 smem_ssd[];
   SsdStage<N>* ring = reinterpret_cast<SsdStage<N>*>(smem_ssd);
@@ -198,7 +202,7 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
     if (k + 1 < nchunk) load_in(k + 1, nxt);
     const SsdStage<N>& st = ring[k % kStages];
     const int t0 = (kc0 + k) * kT;
-    if (MODE == kSsdCkpt) store_state<N>(a, Ht, kc0 + k, b, d0 / 16 + warp, lane);
+    if (MODE == kSsdCkpt || (MODE == kSsdOut && a.ckpt)) store_state<N>(a, Ht, kc0 + k, b, dch, act, tg);
 
     // ---- per (channel, step): Δ, Δx, gate; index j: steps 2tg, 2tg+1, 2tg+8, 2tg+9
     float dl[2][4], xv[2][4], gt[2][4], uv[2][4];
@@ -320,7 +324,7 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
       }
       mma16816(Ht[nt], x2[0], x2[1], x2[2], x2[3], bn[0], bn[1]);
       mma16816(Ht[nt + 1], x2[0], x2[1], x2[2], x2[3], bn[2], bn[3]);
-      if (NOOUT) {  // states that a backward or a chain reads: the remainder term too
+      if (exact) {  // states that a backward or a chain reads: the remainder term too
         mma16816(Ht[nt], x2l[0], x2l[1], x2l[2], x2l[3], bn[0], bn[1]);
         mma16816(Ht[nt + 1], x2l[0], x2l[1], x2l[2], x2l[3], bn[2], bn[3]);
       }
@@ -401,10 +405,7 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
     }
   }
   cp_wait<0>();
-  if (MODE == kSsdCkpt) {
-    if ((seg + 1) * a.chunk_len >= L) store_state<N>(a, Ht, kc0 + nchunk, b, d0 / 16 + warp, lane);
-    return;
-  }
+  if (MODE == kSsdCkpt) return;
   if (SUMMARY) {
 #pragma unroll
     for (int nt = 0; nt < kNT; ++nt) {

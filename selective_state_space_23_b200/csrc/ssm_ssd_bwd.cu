@@ -65,7 +65,9 @@ union BwdWarpSmem {
 template <int N>
 struct BwdSmem {
   SsdStage<N> ring[kStB];
-  float4 hs[kStB][kWb * (N / 8) * 32];  // the entering state of the chunk, fragment order
+  // the entering state of the chunk, [64 channels][N] with rows padded to N + 8 floats (the
+  // lanes' 64-bit reads of rows g, g + 8 at columns 8 nt + 2 tg fall in distinct banks)
+  float hs[kStB][16 * kWb * (N + 8)];
   float4 mu[kWb * (N / 8) * 32];        // the adjoint μ, fragment order (each lane its own)
   BwdWarpSmem<N> w[kWb];
 };
@@ -123,7 +125,6 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
   const int d0 = ctag * 16 * kWb;
   const int L = a.L;
   const int nck = (L + kT - 1) / kT;
-  const long long nslots = nck + 1;
   const int seg = SUMM ? blockIdx.y + 1 : blockIdx.y;
   const int kc0 = seg * a.cps, kc1 = min(nck, kc0 + a.cps);  // this segment's chunks
   const int nloc = kc1 - kc0;
@@ -146,12 +147,9 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
     bias[c] = a.dt_bias ? a.dt_bias[dch[c]] : 0.f;
     Dd[c] = a.D ? a.D[dch[c]] : 0.f;
   }
-  // the checkpointed entering states of this CTA's four 16-channel groups (the last valid
-  // group stands in for groups past dim)
-  const int ngrp = (a.dim + 15) / 16;
-  const int gvalid = min(kWb, ngrp - kWb * ctag);
-  const float4* ckb = reinterpret_cast<const float4*>(a.ck) +
-                      ((long long)b * nslots * ngrp + kWb * ctag) * kNT * 32;
+  // the checkpointed entering states of this CTA's channels, rows [batch][dim][chunk][N] (the
+  // last channel stands in for channels past dim)
+  const float* ckb = a.ck + (long long)b * a.dim * nck * N;
 
   // the adjoint μ = dL/dh_out of the current chunk, transposed [d][n] in accumulator layout:
   // mus[32 nt] holds the lane's registers of n tile nt (channels g, g + 8; states 8 nt + 2 tg,
@@ -185,10 +183,12 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
       SsdStage<N>& st = sm.ring[i % kStB];
       const int t0 = (kc1 - 1 - i) * kT;
       if (!SUMM) {
-        const float4* src = ckb + (long long)(kc1 - 1 - i) * ngrp * kNT * 32;
-        for (int p = tid; p < kWb * kNT * 32; p += 32 * kWb) {
-          const int j = p / (kNT * 32);
-          cp16(&sm.hs[i % kStB][p], src + (min(j, gvalid - 1) - j) * kNT * 32 + p);
+        const int kk = kc1 - 1 - i;
+        for (int p = tid; p < 16 * kWb * (N / 4); p += 32 * kWb) {
+          const int j = p / (N / 4), piece = p % (N / 4);
+          const int dsrc = min(d0 + j, a.dim - 1);
+          cp16(&sm.hs[i % kStB][j * (N + 8) + 4 * piece],
+               ckb + ((long long)dsrc * nck + kk) * N + 4 * piece);
         }
       }
       if (a.rows16 && t0 + kT <= L) {
@@ -236,11 +236,10 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
     const ChunkInB cur = nxt;
     if (k > kc0) load_in(k - 1, nxt);
     const SsdStage<N>& st = sm.ring[i % kStB];
-    const float4* hsw = &sm.hs[i % kStB][warp * kNT * 32 + lane];
+    const float* hsw = &sm.hs[i % kStB][(16 * warp + g) * (N + 8) + 2 * tg];
     // the entering state: states 8 nt + 2 tg, +1 of channel g + 8 c
     const auto hck = [&](int c, int nt) {
-      const float4 v = hsw[nt * 32];
-      return c ? make_float2(v.z, v.w) : make_float2(v.x, v.y);
+      return *reinterpret_cast<const float2*>(hsw + 8 * c * (N + 8) + 8 * nt);
     };
     const int t0 = k * kT;
 

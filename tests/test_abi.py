@@ -112,7 +112,7 @@ def _bwd_ex(lib, flags=0, groups=1, dim=64):
                                flags, None)
 
 
-def test_variant_flags_and_groups_are_checked_on_the_host(lib):
+def test_variant_flags_and_groups_are_checked_on_the_host(lib, monkeypatch):
     """The _ex entry points refuse unknown flag bits and unusable B/C groupings before touching
     any pointer (nothing here needs a GPU)."""
     known = _abi.SSM_SCALAR_A | _abi.SSM_REVERSE | _abi.SSM_ZOH | _abi.SSM_CHANNELS_LAST
@@ -130,10 +130,18 @@ def test_variant_flags_and_groups_are_checked_on_the_host(lib):
     assert lib.ssm_scan_fwd_ex_workspace_size(1, 256, 1 << 20, 16, 1, 1, known) > 0
     assert lib.ssm_scan_bwd_ex_workspace_size(4, 5120, 2048, 16, 8, 1, 1, 0) > 0
     assert lib.ssm_scan_bwd_ex_workspace_size(4, 64, 2048, 16, 8, 1, 1, 0) == 0   # bad groups
-    # the scalar decay adds the broadcast rate and per-state dA to the backward's workspace
+    # on the per-state kernel the scalar decay adds the broadcast rate and per-state dA to the
+    # backward's workspace
+    monkeypatch.setenv("SSM_SCALAR_BWD", "state")
     base = lib.ssm_scan_bwd_ex_workspace_size(4, 5120, 2048, 16, 1, 1, 1, 0)
     sa = lib.ssm_scan_bwd_ex_workspace_size(4, 5120, 2048, 16, 1, 1, 1, _abi.SSM_SCALAR_A)
     assert sa - base == 2 * 5120 * 16 * 4
+    # the chunked form (bf16): given checkpoints, it needs no room for them (4 x 5120 x 128
+    # chunks x 16 states of f32)
+    monkeypatch.delenv("SSM_SCALAR_BWD")
+    given = lib.ssm_scan_bwd_ex_workspace_size(4, 5120, 2048, 16, 1, 1, 1, _abi.SSM_SCALAR_A)
+    own = lib.ssm_scan_bwd_ex_workspace_size(4, 5120, 2048, 16, 1, 1, 0, _abi.SSM_SCALAR_A)
+    assert 0 < given and own - given >= 4 * 5120 * 128 * 16 * 4
 
 
 def test_decode_variants_refuse_the_reverse_flag(lib):

@@ -75,19 +75,75 @@ def test_variants(variant):
         assert_close(g[k], r[k], torch.bfloat16, k)
 
 
-def test_forward_then_backward_shapes_agree():
-    """The N = 64 forward and backward (both in the chunked matrix form) take the same tensors;
-    checkpoints are refused for N > 16 (the backward recomputes its states)."""
+def test_slice_backward_refuses_checkpoints(monkeypatch):
+    """The slice path (here forced) recomputes its states and refuses checkpoints."""
+    monkeypatch.setenv("SSM_SCALAR_BWD", "slices")
     x = inputs(1, 64, 64, 64, torch.bfloat16, seed=103)
     xd = {k: v.to(DEV) for k, v in x.items()}
-    out = ssm.ssm_scan_fwd_scalar_a(xd["u"], xd["delta"], xd["A"], xd["B"], xd["C"], D=xd["D"],
-                                    z=xd["z"], dt_bias=xd["dt_bias"], h0=xd["h0"])
-    assert out.shape == (1, 64, 64)
     fake_ck = torch.zeros((1, 64, 4, 64), device=DEV)
     with pytest.raises(RuntimeError):
         ssm.ssm_scan_bwd_scalar_a(xd["u"], xd["delta"], xd["A"], xd["B"], xd["C"], xd["dout"],
                                   D=xd["D"], z=xd["z"], dt_bias=xd["dt_bias"], h0=xd["h0"],
                                   ckpt=fake_ck)
+
+
+def fwd(x, **kw):
+    xd = {k: v.to(DEV) for k, v in x.items()}
+    return ssm.ssm_scan_fwd_scalar_a(xd["u"], xd["delta"], xd["A"], xd["B"], xd["C"], D=xd["D"],
+                                     z=xd["z"], dt_bias=xd["dt_bias"], h0=xd["h0"], **kw)
+
+
+@pytest.mark.parametrize("N", [16, 64, 128])
+@pytest.mark.parametrize("shape", [(2, 128, 333), (1, 80, 96)])
+def test_chunked_forward_checkpoints_are_block_entry_states(N, shape):
+    """The chunked forward's checkpoints: the state entering every 16-step block (slot 0 = h0),
+    against the oracle's final states of the prefixes; the outputs are unchanged by asking for
+    them."""
+    batch, dim, L = shape
+    x = inputs(batch, dim, L, N, torch.bfloat16, seed=119)
+    out, ck = fwd(x, return_ckpt=True)
+    assert ck.shape == (batch, dim, (L + 15) // 16, N)
+    assert torch.equal(out, fwd(x))
+    c = lambda k: f64(x[k])
+    A = np.repeat(c("A")[:, None], N, axis=1)
+    for k in range(ck.shape[2]):
+        t = 16 * k
+        if t == 0:
+            ref_h = c("h0")
+        else:
+            r = oracle.scan_fwd(c("u")[..., :t], c("delta")[..., :t], A, c("B")[..., :t],
+                                c("C")[..., :t], D=c("D"), z=c("z")[..., :t],
+                                dt_bias=c("dt_bias"), h0=c("h0"))
+            ref_h = r["hL"]
+        assert_close(ck[:, :, k, :], ref_h, torch.bfloat16, f"checkpoint {k}")
+
+
+@pytest.mark.parametrize("N", [16, 64, 128])
+def test_chunked_backward_from_forward_checkpoints(N):
+    """The backward given the chunked forward's checkpoints (no checkpoint pass) against the
+    oracle, and against the same backward recomputing them."""
+    x = inputs(2, 128, 333, N, torch.bfloat16, seed=120)
+    _, ck = fwd(x, return_ckpt=True)
+    dhL = torch.randn((2, 128, N), generator=torch.Generator().manual_seed(12))
+    g = run(x, dhL, ckpt=ck)
+    g0 = run(x, dhL)
+    r = ref(x, dhL)
+    for k in GRADS:
+        assert_close(g[k], r[k], torch.bfloat16, k)
+        assert_close(g[k], f64(g0[k]), torch.bfloat16, k)
+
+
+def test_chunked_backward_from_per_state_checkpoints(monkeypatch):
+    """N = 16: checkpoints written by the per-state forward kernel serve the chunked backward
+    (same layout, same states)."""
+    x = inputs(2, 64, 200, 16, torch.bfloat16, seed=121)
+    monkeypatch.setenv("SSM_SCALAR_FORM", "state")
+    _, ck = fwd(x, return_ckpt=True)
+    monkeypatch.delenv("SSM_SCALAR_FORM")
+    g = run(x, None, ckpt=ck)
+    r = ref(x, None)
+    for k in GRADS:
+        assert_close(g[k], r[k], torch.bfloat16, k)
 
 
 # ------------------------------------------------------------------ the chunked-form backward
