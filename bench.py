@@ -343,9 +343,20 @@ def _ssd(dev, rnd, prm, timeit, g):
         ms = timeit(lambda: ssm.ssm_scan_bwd_scalar_a(u, de, A1, B, C, dout, D=D, z=z,
                                                       dt_bias=bias, workspace=wsb), 5)
         byt = 7 * b * d * L * 2 + 4 * b * N * L * 2
+        # a training step: the forward writing checkpoints, the backward taking them
+        wsc = torch.empty(ssm._abi.lib().ssm_scan_bwd_ex_workspace_size(b, d, L, N, 1, 1, 1, 1),
+                          dtype=torch.uint8, device=dev)
+
+        def train():
+            _, ck = ssm.ssm_scan_fwd_scalar_a(u, de, A1, B, C, D=D, z=z, dt_bias=bias, out=o,
+                                              return_ckpt=True)
+            ssm.ssm_scan_bwd_scalar_a(u, de, A1, B, C, dout, D=D, z=z, dt_bias=bias, ckpt=ck,
+                                      workspace=wsc)
+        mt = timeit(train, 5)
         res["bwd"][f"N{N}"] = {"bwd_ms": ms, "tokens_per_s": b * L / (ms * 1e-3),
-                               "compulsory_gbs": byt / (ms * 1e-3) / 1e9}
-        del B, C, wsb
+                               "compulsory_gbs": byt / (ms * 1e-3) / 1e9,
+                               "train_step_ms": mt}
+        del B, C, wsb, wsc
     del u, de, z, o, dout
     # the long sequence (1 x 256 x 2^20) with 64 states: 16 warps of channels, so the time axis
     # is split into segments (summary, chain, output launches)
