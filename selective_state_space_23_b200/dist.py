@@ -1,8 +1,11 @@
 """Multi-process (one process per GPU) plumbing for the scan.
 
-Two ways to shard one scan over GPUs:
+Three ways to shard one scan over GPUs:
 
 * batch rows (below): independent, no exchange in the forward;
+* channels (:func:`shard_channels`): independent too; the backward's dB, dC are sums over the
+  channels and take one all-reduce (:func:`allreduce_bc_grads`), while dA, dD, ddt_bias belong
+  to the rank's own channels;
 * the sequence (:func:`seq_split_scan_fwd`): each GPU holds a segment of the time axis; one
   all-gather of the segments' (end state, ΣΔ) summaries, a local chain over the earlier
   segments, then each GPU's forward from its true entering state.
@@ -30,6 +33,20 @@ def shard_rows(total_rows: int, world: int, rank: int) -> Tuple[int, int]:
     base, extra = divmod(total_rows, world)
     begin = rank * base + min(rank, extra)
     return begin, begin + base + (1 if rank < extra else 0)
+
+
+def shard_channels(dim: int, world: int, rank: int, align: int = 16) -> Tuple[int, int]:
+    """Contiguous [begin, end) of channels d owned by ``rank``: whole blocks of ``align``
+    channels (16: the kernels' warps of channels; 64: the chunked form's tiles), the ranks'
+    block counts differing by at most one, the last block cut at ``dim``.  The rank scans the
+    channel slice of u, delta, z (a strided view, or a copy) with the matching rows of A, D and
+    dt_bias, and the whole B, C of its batch rows."""
+    if align <= 0:
+        raise ValueError("align must be positive")
+    if dim < 0:
+        raise ValueError("dim must be non-negative")
+    b0, b1 = shard_rows((dim + align - 1) // align, world, rank)
+    return min(dim, b0 * align), min(dim, b1 * align)
 
 
 def max_over_ranks(value: float, device=None) -> float:
@@ -65,6 +82,34 @@ def allreduce_param_grads(grads: Dict[str, torch.Tensor],
             or dist.get_world_size() == 1:
         return grads
     flat = torch.cat([grads[k].reshape(-1) for k in present])
+    dist.all_reduce(flat, op=dist.ReduceOp.SUM)
+    off = 0
+    for k in present:
+        n = grads[k].numel()
+        grads[k].copy_(flat[off:off + n].view_as(grads[k]))
+        off += n
+    return grads
+
+
+BC_GRADS = ("dB", "dC")
+
+
+def allreduce_bc_grads(grads: Dict[str, torch.Tensor],
+                       keys: Sequence[str] = BC_GRADS) -> Dict[str, torch.Tensor]:
+    """Channel-sharded backward: sum ``grads["dB"]``, ``grads["dC"]`` (each rank's sums over its
+    own channels) over the ranks of the default process group, in place, as one all-reduce of a
+    single flat bucket.  16-bit gradients are summed in f32 and rounded once at the end; f32 and
+    f64 ones in their own type.  The same rules as :func:`allreduce_param_grads` for absent keys,
+    shapes and a missing or single-rank group."""
+    import torch.distributed as dist
+    present = [k for k in keys if grads.get(k) is not None]
+    if not present or not (dist.is_available() and dist.is_initialized()) \
+            or dist.get_world_size() == 1:
+        return grads
+    acc = grads[present[0]].dtype
+    if acc in (torch.bfloat16, torch.float16):
+        acc = torch.float32
+    flat = torch.cat([grads[k].reshape(-1).to(acc) for k in present])
     dist.all_reduce(flat, op=dist.ReduceOp.SUM)
     off = 0
     for k in present:

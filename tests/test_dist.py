@@ -11,8 +11,9 @@ import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
-from selective_state_space_23_b200.dist import (allreduce_param_grads, barrier, max_over_ranks,
-                                                shard_rows)
+from selective_state_space_23_b200.dist import (allreduce_bc_grads, allreduce_param_grads, barrier,
+                                                 max_over_ranks, seq_split_scan_fwd, shard_channels,
+                                                 shard_rows)
 
 
 def test_shard_rows_partition():
@@ -148,6 +149,89 @@ def test_two_ranks_backward_param_grads_allreduced():
     for k in ("du", "ddelta", "dz", "dB", "dC", "dh0"):
         got = np.concatenate([r[4][k] for r in res], 0)
         np.testing.assert_array_equal(got, full[k])
+
+
+def test_shard_channels_partition():
+    for dim in (0, 5, 16, 40, 80, 2048):
+        for world in (1, 2, 3, 8):
+            for align in (1, 16, 64):
+                spans = [shard_channels(dim, world, r, align) for r in range(world)]
+                assert spans[0][0] == 0 and spans[-1][1] == dim
+                for (b0, e0), (b1, _) in zip(spans, spans[1:]):
+                    assert e0 == b1
+                for b, e in spans:   # every span starts on a block boundary
+                    assert b % align == 0 or b == dim
+                blocks = [-(-(e - b) // align) for b, e in spans]
+                assert max(blocks) - min(blocks) <= 1
+    with pytest.raises(ValueError):
+        shard_channels(16, 2, 2)
+
+
+CH_SHAPE = dict(batch=3, dim=10, seqlen=29, dstate=4)
+
+
+def _ch_inputs():
+    from selective_state_space_23_b200.inputs import make_inputs, to_f64, workload
+    w = workload("tiny_f32", **CH_SHAPE)
+    return {k: to_f64(v) for k, v in make_inputs(w, seed=6, with_h0=True, with_dout=True).items()}
+
+
+def _bwd_channels(oracle, x, d0, d1):
+    c = lambda k: x[k][:, d0:d1]
+    return oracle.scan_bwd(c("u"), c("delta"), x["A"][d0:d1], x["B"], x["C"], c("dout"),
+                           D=x["D"][d0:d1], z=c("z"), dt_bias=x["dt_bias"][d0:d1], h0=c("h0"),
+                           nthreads=1)
+
+
+def _bwd_channels_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import oracle
+        x = _ch_inputs()
+        d0, d1 = shard_channels(CH_SHAPE["dim"], world, rank, align=4)
+        g = _bwd_channels(oracle, x, d0, d1)
+        bc = {k: torch.from_numpy(np.ascontiguousarray(g[k])) for k in ("dB", "dC")}
+        before = {k: v.clone() for k, v in bc.items()}
+        allreduce_bc_grads(bc)
+        own = {k: g[k] for k in ("du", "ddelta", "dz", "dh0", "dA", "dD", "ddt_bias")}
+        q.put((rank, (d0, d1), {k: v.numpy() for k, v in bc.items()},
+               {k: v.numpy() for k, v in before.items()}, own))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_channel_sharded_backward_allreduces_dB_dC(world):
+    """Channels split over gloo ranks (the fp64 oracle as each rank's backward): dB, dC summed
+    over the ranks equal the whole layer's; every per-channel gradient needs no exchange."""
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_bwd_channels_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    res.sort(key=lambda r: r[0])
+    import oracle
+    x = _ch_inputs()
+    full = _bwd_channels(oracle, x, 0, CH_SHAPE["dim"])
+    for k in ("dB", "dC"):
+        for r in res:
+            np.testing.assert_allclose(r[2][k], full[k], rtol=1e-12, atol=1e-12)
+        assert not np.allclose(res[0][3][k], full[k])   # one rank's channels alone are not
+    for k in ("du", "ddelta", "dz", "dh0", "dA", "dD", "ddt_bias"):
+        got = np.concatenate([r[4][k] for r in res], 1 if k in ("du", "ddelta", "dz", "dh0") else 0)
+        np.testing.assert_array_equal(got, full[k])
+
+
+def test_allreduce_bc_grads_sums_16_bit_in_f32_without_group_is_identity():
+    g = {"dB": torch.ones(2, 3, dtype=torch.bfloat16), "dC": None}
+    out = allreduce_bc_grads(g)
+    assert out is g and torch.equal(g["dB"], torch.ones(2, 3, dtype=torch.bfloat16))
 
 
 def test_allreduce_param_grads_without_group_is_identity():
