@@ -238,6 +238,15 @@ __global__ void chain_kernel(const float* __restrict__ hend, const float* __rest
                              const float* __restrict__ h0, float* __restrict__ hin, int nseg,
                              long long nch, int dim, int N);
 
+// The reverse scan in the chunked matrix form runs the forward-direction kernels on inputs
+// mirrored along time into the workspace: `rows_x` bf16 rows of u-like tensors (u, delta, z;
+// and dout in the backward) and B, C.  Bytes of those copies.
+size_t mirror_bytes(int batch, int dim, int seqlen, int dstate, int bc_groups, int rows_x) {
+  const size_t nx = (size_t)batch * dim * seqlen * 2;
+  const size_t nbc = (size_t)batch * bc_groups * dstate * seqlen * 2;
+  return (size_t)rows_x * align_up(nx) + 2 * align_up(nbc);
+}
+
 // Workspace that covers the plan of either kernel family (the family is chosen per call, from
 // the pointers' alignment too).
 size_t fwd_ws_bytes(int batch, int dim, int seqlen) {
@@ -409,17 +418,47 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
                          !(sform && strcmp(sform, "state") == 0);
   if (dstate > SSM_MAX_DSTATE || chunked16) {
     if (io_dtype != SSM_BF16 || (dstate != 16 && dstate != 32 && dstate != 64 && dstate != 128) || zoh ||
-        reverse || channels_last ||
+        channels_last ||
         !(bc_groups == 1 || (dim % bc_groups == 0 && (dim / bc_groups) % 64 == 0)))
       return fail(SSM_EUNSUPPORTED,
-                  "scalar decay with dstate %d > %d needs bf16 io, dstate 32, 64 or 128, the "
-                  "forward direction without ZOH, the default layout and B/C groups of whole "
-                  "64-channel tiles", dstate, SSM_MAX_DSTATE);
+                  "scalar decay with dstate %d > %d needs bf16 io, dstate 32, 64 or 128, no "
+                  "ZOH, the default layout and B/C groups of whole 64-channel tiles", dstate,
+                  SSM_MAX_DSTATE);
     if (!aligned16(ckpt))
       return fail(SSM_EINVAL, "ckpt must be 16-byte aligned (chunked matrix form)");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    // reverse: the kernels scan inputs mirrored along time (copies at the workspace's start);
+    // the output is mirrored back in place at the end
+    const size_t mb = reverse ? mirror_bytes(batch, dim, seqlen, dstate, bc_groups, 3) : 0;
+    const void *ku = u, *kd = delta, *kz = z, *kB = B, *kC = C;
+    if (reverse) {
+      if (!workspace || workspace_bytes < mb)
+        return fail(SSM_EWORKSPACE, "workspace of %zu bytes given, %zu needed (reverse scan)",
+                    workspace_bytes, mb);
+      if (reinterpret_cast<uintptr_t>(workspace) & 255)
+        return fail(SSM_EINVAL, "workspace is not 256-byte aligned");
+      TRY(check_ptr(workspace, mb, 256, "workspace"));
+      char* m = reinterpret_cast<char*>(workspace);
+      const long long rx = (long long)batch * dim, rbc = (long long)batch * bc_groups * dstate;
+      void* mu = m;
+      void* md = m + align_up(nx);
+      void* mz = z ? m + 2 * align_up(nx) : nullptr;
+      void* mB = m + 3 * align_up(nx);
+      void* mC = m + 3 * align_up(nx) + align_up(nbc);
+      if ((e = ssm::mirror_rows(u, mu, rx, seqlen, s)) != cudaSuccess ||
+          (e = ssm::mirror_rows(delta, md, rx, seqlen, s)) != cudaSuccess ||
+          (z && (e = ssm::mirror_rows(z, mz, rx, seqlen, s)) != cudaSuccess) ||
+          (e = ssm::mirror_rows(B, mB, rbc, seqlen, s)) != cudaSuccess ||
+          (e = ssm::mirror_rows(C, mC, rbc, seqlen, s)) != cudaSuccess)
+        return cuda_fail(e, "reverse scan: mirrored inputs");
+      ku = mu; kd = md; kz = mz; kB = mB; kC = mC;
+      workspace = m + mb;
+      workspace_bytes -= mb;
+    }
     ssm::FwdArgs a;
     memset(&a, 0, sizeof(a));
-    a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
+    a.u = ku; a.delta = kd; a.z = kz; a.B = kB; a.C = kC;
     a.A = A; a.D = D; a.dt_bias = dt_bias; a.h0 = h0; a.out = out; a.hL = hL; a.ckpt = ckpt;
     a.batch = batch; a.dim = dim; a.L = seqlen; a.N = dstate;
     a.softplus = delta_softplus ? 1 : 0;
@@ -434,8 +473,6 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
     }
     a.chunk_len = plan.chunk_len;
     a.nchunk = plan.nchunk;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e;
     if (plan.nchunk > 1) {
       TRY(check_ptr(workspace, plan.ws_bytes, 256, "workspace"));
       const size_t nch = (size_t)batch * dim;
@@ -455,6 +492,8 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
     }
     e = ssm::launch_ssd_fwd(a, ssm::kSsdOut, s);
     if (e != cudaSuccess) return cuda_fail(e, "forward pass (chunked matrix form)");
+    if (reverse && (e = ssm::mirror_rows(out, out, (long long)batch * dim, seqlen, s)) != cudaSuccess)
+      return cuda_fail(e, "reverse scan: mirrored output");
     return SSM_OK;
   }
   // B/C per channel (bc_groups == dim > 1): the per-state kernel of ssm_pcbc.cu, no time split
@@ -623,7 +662,8 @@ size_t ssm_scan_fwd_ex_workspace_size(int batch, int dim, int seqlen, int dstate
   if (bc_groups < 1) return 0;
   if ((flags & SSM_SCALAR_A) && dstate > SSM_MAX_DSTATE) {  // the chunked matrix form's segments
     if (check_dims(batch, dim, seqlen, dstate, io_dtype, SSM_MAX_DSTATE_SCALAR) != SSM_OK) return 0;
-    return plan_ssd(batch, dim, seqlen, dstate).ws_bytes;
+    return plan_ssd(batch, dim, seqlen, dstate).ws_bytes +
+           ((flags & SSM_REVERSE) ? mirror_bytes(batch, dim, seqlen, dstate, bc_groups, 3) : 0);
   }
   return ssm_scan_fwd_workspace_size(batch, dim, seqlen, dstate, io_dtype);
 }
@@ -875,7 +915,7 @@ namespace {
 bool chunked_bwd_ok(int dim, int dstate, int bc_groups, int io_dtype, int flags) {
   const char* v = getenv("SSM_SCALAR_BWD");  // "slices" / "state": the per-state kernels
   if (v && (strcmp(v, "slices") == 0 || strcmp(v, "state") == 0)) return false;
-  return io_dtype == SSM_BF16 && flags == SSM_SCALAR_A &&
+  return io_dtype == SSM_BF16 && (flags & ~SSM_REVERSE) == SSM_SCALAR_A &&
          (dstate == 16 || dstate == 32 || dstate == 64 || dstate == 128) &&
          (bc_groups == 1 || (bc_groups < dim && dim % bc_groups == 0 && (dim / bc_groups) % 64 == 0));
 }
@@ -907,14 +947,17 @@ BwdSegPlan plan_ssd_bwd(int batch, int dim, int seqlen, int dstate) {
 }
 
 struct ChunkedBwdLayout {
-  size_t ck, pbc, padt, musum, dsum, muin, fwd, total;
+  size_t mir, ck, pbc, padt, musum, dsum, muin, fwd, total;
   BwdSegPlan seg;
 };
 
-// have_ckpt: the caller passes the forward's checkpoints (no checkpoint pass, no room for them)
-ChunkedBwdLayout chunked_bwd_layout(int batch, int dim, int seqlen, int dstate, bool have_ckpt) {
+// have_ckpt: the caller passes the forward's checkpoints (no checkpoint pass, no room for them);
+// reverse: room for the inputs mirrored along time at the start
+ChunkedBwdLayout chunked_bwd_layout(int batch, int dim, int seqlen, int dstate, int bc_groups,
+                                    bool have_ckpt, bool reverse) {
   ChunkedBwdLayout l;
   l.seg = plan_ssd_bwd(batch, dim, seqlen, dstate);
+  l.mir = reverse ? mirror_bytes(batch, dim, seqlen, dstate, bc_groups, 4) : 0;
   const size_t nch = (size_t)batch * dim, S = (size_t)l.seg.nseg;
   const size_t nck = (seqlen + ssm::kBlk - 1) / ssm::kBlk;
   l.ck = have_ckpt ? 0 : align_up(nch * nck * dstate * 4);
@@ -924,7 +967,7 @@ ChunkedBwdLayout chunked_bwd_layout(int batch, int dim, int seqlen, int dstate, 
   l.dsum = S > 1 ? align_up(S * nch * 4) : 0;
   l.muin = l.musum;
   l.fwd = have_ckpt ? 0 : plan_ssd(batch, dim, seqlen, dstate).ws_bytes;
-  l.total = l.ck + l.pbc + l.padt + l.musum + l.dsum + l.muin + l.fwd;
+  l.total = l.mir + l.ck + l.pbc + l.padt + l.musum + l.dsum + l.muin + l.fwd;
   return l;
 }
 
@@ -933,7 +976,8 @@ int scan_bwd_chunked(const void* u, const void* delta, const float* A, const voi
                      int delta_softplus, const float* h0, const void* dout, const float* dhL,
                      const float* ckpt, void* du, void* ddelta, float* dA, void* dB, void* dC, float* dD, void* dz,
                      float* ddt_bias, float* dh0, void* workspace, size_t workspace_bytes,
-                     int batch, int dim, int seqlen, int dstate, int bc_groups, void* stream) {
+                     int batch, int dim, int seqlen, int dstate, int bc_groups, bool reverse,
+                     void* stream) {
   const size_t es = 2;
   const size_t nx = (size_t)batch * dim * seqlen * es;
   const size_t nbc = (size_t)batch * bc_groups * dstate * seqlen * es;
@@ -965,13 +1009,36 @@ int scan_bwd_chunked(const void* u, const void* delta, const float* A, const voi
   if (!du && !ddelta && !dA && !dB && !dC && !dD && !dz && !ddt_bias && !dh0)
     return fail(SSM_EINVAL, "no gradient output requested");
   if (dz && !z) return fail(SSM_EINVAL, "dz requested but z is NULL");
-  const ChunkedBwdLayout l = chunked_bwd_layout(batch, dim, seqlen, dstate, ckpt != nullptr);
+  const ChunkedBwdLayout l =
+      chunked_bwd_layout(batch, dim, seqlen, dstate, bc_groups, ckpt != nullptr, reverse);
   if (!workspace || workspace_bytes < l.total)
     return fail(SSM_EWORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes, l.total);
   if (reinterpret_cast<uintptr_t>(workspace) & 255)
     return fail(SSM_EINVAL, "workspace is not 256-byte aligned");
   TRY(check_ptr(workspace, l.total, 256, "workspace"));
-  char* w = reinterpret_cast<char*>(workspace);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  // reverse: the kernels scan the inputs mirrored along time; the gradients along time are
+  // mirrored back in place at the end
+  if (reverse) {
+    char* m = reinterpret_cast<char*>(workspace);
+    const long long rx = (long long)batch * dim, rbc = (long long)batch * bc_groups * dstate;
+    void* mu = m;
+    void* md = m + align_up(nx);
+    void* mz = z ? m + 2 * align_up(nx) : nullptr;
+    void* mo = m + 3 * align_up(nx);
+    void* mB = m + 4 * align_up(nx);
+    void* mC = m + 4 * align_up(nx) + align_up(nbc);
+    if ((e = ssm::mirror_rows(u, mu, rx, seqlen, s)) != cudaSuccess ||
+        (e = ssm::mirror_rows(delta, md, rx, seqlen, s)) != cudaSuccess ||
+        (z && (e = ssm::mirror_rows(z, mz, rx, seqlen, s)) != cudaSuccess) ||
+        (e = ssm::mirror_rows(dout, mo, rx, seqlen, s)) != cudaSuccess ||
+        (e = ssm::mirror_rows(B, mB, rbc, seqlen, s)) != cudaSuccess ||
+        (e = ssm::mirror_rows(C, mC, rbc, seqlen, s)) != cudaSuccess)
+      return cuda_fail(e, "reverse scan backward: mirrored inputs");
+    u = mu; delta = md; z = mz; dout = mo; B = mB; C = mC;
+  }
+  char* w = reinterpret_cast<char*>(workspace) + l.mir;
   float* ck = ckpt ? nullptr : reinterpret_cast<float*>(w);
   float* pbc = reinterpret_cast<float*>(w + l.ck);
   float* padt = reinterpret_cast<float*>(w + l.ck + l.pbc);
@@ -979,10 +1046,8 @@ int scan_bwd_chunked(const void* u, const void* delta, const float* A, const voi
   float* dsum = reinterpret_cast<float*>(w + l.ck + l.pbc + l.padt + l.musum);
   float* muin = reinterpret_cast<float*>(w + l.ck + l.pbc + l.padt + l.musum + l.dsum);
   char* fws = w + l.ck + l.pbc + l.padt + l.musum + l.dsum + l.muin;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool vec = (seqlen * es) % 16 == 0 && aligned16(u) && aligned16(delta) && aligned16(z) &&
-                   aligned16(B) && aligned16(C);
-  cudaError_t e;
+                   aligned16(B) && aligned16(C) && aligned16(dout);
   if (!ckpt) {
     // the state entering every chunk, from the forward in checkpoint mode
     ssm::FwdArgs a;
@@ -1054,6 +1119,14 @@ int scan_bwd_chunked(const void* u, const void* delta, const float* A, const voi
     return cuda_fail(e, "backward pass (chunked matrix form)");
   if ((e = ssm::launch_ssd_bwd_finish(b, dB, dC, dA, dD, ddt_bias, s)) != cudaSuccess)
     return cuda_fail(e, "backward reduction (chunked matrix form)");
+  if (reverse) {
+    const long long rx = (long long)batch * dim, rbc = (long long)batch * bc_groups * dstate;
+    void* along[5] = {du, ddelta, dz, dB, dC};
+    const long long rows[5] = {rx, rx, rx, rbc, rbc};
+    for (int k = 0; k < 5; ++k)
+      if (along[k] && (e = ssm::mirror_rows(along[k], along[k], rows[k], seqlen, s)) != cudaSuccess)
+        return cuda_fail(e, "reverse scan backward: mirrored gradients");
+  }
   return SSM_OK;
 }
 
@@ -1078,13 +1151,15 @@ size_t ssm_scan_bwd_ex_workspace_size(int batch, int dim, int seqlen, int dstate
   if (flags & ~(SSM_SCALAR_A | SSM_REVERSE | SSM_ZOH | SSM_CHANNELS_LAST)) return 0;
   if ((flags & SSM_SCALAR_A) && dstate > SSM_MAX_DSTATE) {  // chunked form, or slices
     if (chunked_bwd_ok(dim, dstate, bc_groups, io_dtype, flags))
-      return chunked_bwd_layout(batch, dim, seqlen, dstate, have_ckpt != 0).total;
+      return chunked_bwd_layout(batch, dim, seqlen, dstate, bc_groups, have_ckpt != 0,
+                                (flags & SSM_REVERSE) != 0).total;
     if (have_ckpt) return 0;
     return ssm::scan_bwd_slices_workspace(batch, dim, seqlen, dstate, bc_groups, io_dtype, flags);
   }
   if (dstate == 16 && chunked_bwd_ok(dim, dstate, bc_groups, io_dtype, flags)) {
     if (check_dims(batch, dim, seqlen, dstate, io_dtype) != SSM_OK) return 0;
-    return chunked_bwd_layout(batch, dim, seqlen, dstate, have_ckpt != 0).total;
+    return chunked_bwd_layout(batch, dim, seqlen, dstate, bc_groups, have_ckpt != 0,
+                              (flags & SSM_REVERSE) != 0).total;
   }
   if (check_dims(batch, dim, seqlen, dstate, io_dtype) != SSM_OK) return 0;
   if (check_groups(dim, bc_groups) != SSM_OK) return 0;
@@ -1112,7 +1187,8 @@ int ssm_scan_bwd_ex(const void* u, const void* delta, const float* A, const void
     if (chunked_bwd_ok(dim, dstate, bc_groups, io_dtype, flags))
       return scan_bwd_chunked(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL,
                               ckpt, du, ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, workspace,
-                              workspace_bytes, batch, dim, seqlen, dstate, bc_groups, stream);
+                              workspace_bytes, batch, dim, seqlen, dstate, bc_groups, reverse,
+                              stream);
     return ssm::scan_bwd_slices(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL,
                                 ckpt, du, ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, workspace,
                                 workspace_bytes, batch, dim, seqlen, dstate, bc_groups, io_dtype,
@@ -1123,7 +1199,8 @@ int ssm_scan_bwd_ex(const void* u, const void* delta, const float* A, const void
     TRY(check_groups(dim, bc_groups));
     return scan_bwd_chunked(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL, ckpt,
                             du, ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, workspace,
-                            workspace_bytes, batch, dim, seqlen, dstate, bc_groups, stream);
+                            workspace_bytes, batch, dim, seqlen, dstate, bc_groups, reverse,
+                            stream);
   }
   if (!(flags & SSM_SCALAR_A))
     return scan_bwd_core(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL, ckpt,

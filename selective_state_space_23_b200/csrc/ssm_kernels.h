@@ -200,6 +200,9 @@ void set_last_error(const char* msg);
 // dst, es = 2 or 4 bytes per element (ssm_strided.cu).
 cudaError_t copy_view(const void* src, const long long* n, const long long* ss, void* dst,
                       const long long* ds, size_t es, cudaStream_t s);
+// Rows [rows][L] of 16-bit elements mirrored along L from src into dst, or in place when
+// src == dst (ssm_strided.cu).
+cudaError_t mirror_rows(const void* src, void* dst, long long rows, int L, cudaStream_t s);
 // Backward of the scalar-decay scan for dstate = 16 k (k = 2, 4, 8) as the sum of k 16-state
 // backwards (ssm_slices.cu); arguments as ssm_scan_bwd_ex.
 size_t scan_bwd_slices_workspace(int batch, int dim, int seqlen, int dstate, int bc_groups,

@@ -417,7 +417,39 @@ int ssm_state_update_strided(float* state, const void* x, const void* dt, const 
 
 }  // extern "C"
 
+namespace {
+// Rows of L 16-bit elements mirrored along L: dst[r][t] = src[r][L - 1 - t].  In place
+// (src == dst) each thread swaps one pair; otherwise each thread copies one element.
+__global__ void mirror_rows_kernel(const uint16_t* __restrict__ src, uint16_t* dst,
+                                   long long rows, int L, int in_place) {
+  const long long per = in_place ? L / 2 : L;
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= rows * per) return;
+  const long long r = i / per;
+  const int t = (int)(i % per);
+  const long long a = r * L + t, m = r * L + (L - 1 - t);
+  if (in_place) {
+    const uint16_t x = dst[a];
+    dst[a] = dst[m];
+    dst[m] = x;
+  } else {
+    dst[a] = src[m];
+  }
+}
+}  // namespace
+
 namespace ssm {
+// The reverse scan of the chunked matrix form runs its kernels on rows mirrored along time: rows
+// [rows][L] of 16-bit elements from src into dst mirrored, or in place when src == dst.
+cudaError_t mirror_rows(const void* src, void* dst, long long rows, int L, cudaStream_t s) {
+  const int in_place = src == dst ? 1 : 0;
+  const long long n = rows * (in_place ? L / 2 : L);
+  if (n <= 0) return cudaSuccess;
+  mirror_rows_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
+      reinterpret_cast<const uint16_t*>(src), reinterpret_cast<uint16_t*>(dst), rows, L, in_place);
+  return cudaGetLastError();
+}
+
 // The restride copy for other translation units: the 4-index view (sizes n, element strides ss)
 // at src into the view with strides ds at dst (es = 2 or 4 bytes per element), on stream s.
 cudaError_t copy_view(const void* src, const long long* n, const long long* ss, void* dst,

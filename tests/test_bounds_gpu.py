@@ -150,6 +150,7 @@ FWD_CASES = {
     "scalar_decay": ({}, 2, 96, 200, 16, torch.bfloat16, 1, 1),
     "chunked_n64": ({}, 2, 96, 200, 64, torch.bfloat16, 1, 1),
     "chunked_n128_split": ({"SSM_SSD_SPLIT": "3"}, 1, 80, 333, 128, torch.bfloat16, 1, 1),
+    "chunked_n64_reverse": ({}, 1, 80, 333, 64, torch.bfloat16, 1, 1 | 2),
 }
 
 
@@ -167,7 +168,7 @@ def test_forward_stays_inside_its_tensors(monkeypatch, case):
         xg = make_inputs(w, seed=77)
         x["B"] = xg["B"].reshape(batch, dim, N, L).contiguous()
         x["C"] = xg["C"].reshape(batch, dim, N, L).contiguous()
-    ckpt = N <= 16
+    ckpt = N <= 16 or (flags & 1)  # the chunked form (scalar decay) writes checkpoints too
     plain = run_fwd(x, False, batch, dim, L, N, G, flags, ckpt)
     guarded = run_fwd(x, True, batch, dim, L, N, G, flags, ckpt)
     same(guarded, plain)
@@ -192,6 +193,7 @@ BWD_CASES = {
     "scalar_decay_n64_chunked": ({}, 2, 96, 120, 64, torch.bfloat16, 1, 1),
     "scalar_decay_n128_chunked": ({}, 1, 80, 333, 128, torch.bfloat16, 1, 1),
     "scalar_decay_n64_chunked_split": ({"SSM_SSD_BWD_SPLIT": "3"}, 1, 80, 333, 64, torch.bfloat16, 1, 1),
+    "scalar_decay_n64_chunked_reverse": ({}, 1, 80, 333, 64, torch.bfloat16, 1, 1 | 2),
 }
 
 

@@ -60,9 +60,9 @@ def test_gradients_match_oracle(io, N):
         assert_close(g[k], r[k], io, k)
 
 
-@pytest.mark.parametrize("variant", ["reverse_zoh", "groups", "no_gate"])
+@pytest.mark.parametrize("variant", ["reverse_zoh", "reverse", "groups", "no_gate"])
 def test_variants(variant):
-    kw = dict(reverse=variant == "reverse_zoh", zoh=variant == "reverse_zoh")
+    kw = dict(reverse=variant.startswith("reverse"), zoh=variant == "reverse_zoh")
     x = inputs(2, 128, 96, 64, torch.bfloat16, seed=102, groups=2 if variant == "groups" else 1,
                gate=variant != "no_gate")
     if variant == "no_gate":
@@ -249,3 +249,42 @@ def test_chunked_backward_split_agrees_with_unsplit(monkeypatch):
     b = run(x, None)
     for k in GRADS:
         assert_close(a[k], f64(b[k]), torch.bfloat16, k)
+
+
+# ------------------------------------------------------------------ the reverse scan
+@pytest.mark.parametrize("N", [32, 64, 128])
+def test_chunked_reverse_forward_matches_oracle(N):
+    """The reverse scan (the anti-causal half of a bidirectional layer) in the chunked form:
+    outputs, final state and checkpoints (the state entering every block in scan order)."""
+    x = inputs(2, 128, 333, N, torch.bfloat16, seed=122)
+    out, hL, ck = fwd(x, reverse=True, return_final_state=True, return_ckpt=True)
+    c = lambda k: f64(x[k])
+    A = np.repeat(c("A")[:, None], N, axis=1)
+    r = oracle.scan_fwd(c("u"), c("delta"), A, c("B"), c("C"), D=c("D"), z=c("z"),
+                        dt_bias=c("dt_bias"), h0=c("h0"), reverse=True)
+    assert_close(out, r["out"], torch.bfloat16, "out")
+    assert_close(hL, r["hL"], torch.bfloat16, "hL")
+    # checkpoint k: the state after the scan's first 16 k steps, i.e. rows L - 16 k .. L - 1
+    L = x["u"].shape[-1]
+    for k in (1, 7, ck.shape[2] - 1):
+        t = L - 16 * k
+        rk = oracle.scan_fwd(c("u")[..., t:], c("delta")[..., t:], A, c("B")[..., t:],
+                             c("C")[..., t:], D=c("D"), z=c("z")[..., t:], dt_bias=c("dt_bias"),
+                             h0=c("h0"), reverse=True)
+        assert_close(ck[:, :, k, :], rk["hL"], torch.bfloat16, f"checkpoint {k}")
+
+
+@pytest.mark.parametrize("N", [16, 64, 128])
+def test_chunked_reverse_backward_matches_oracle(N):
+    """The reverse scan's backward in the chunked form, recomputing its states and from the
+    reverse forward's checkpoints, with dhL and h0, over a ragged length."""
+    x = inputs(2, 128, 333, N, torch.bfloat16, seed=123)
+    dhL = torch.randn((2, 128, N), generator=torch.Generator().manual_seed(13))
+    r = ref(x, dhL, reverse=True)
+    g = run(x, dhL, reverse=True)
+    for k in GRADS:
+        assert_close(g[k], r[k], torch.bfloat16, k)
+    _, ck = fwd(x, reverse=True, return_ckpt=True)
+    g2 = run(x, dhL, reverse=True, ckpt=ck)
+    for k in GRADS:
+        assert_close(g2[k], r[k], torch.bfloat16, k)
