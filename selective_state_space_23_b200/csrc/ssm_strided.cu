@@ -77,7 +77,6 @@ bool is_dense(const View4& v) {
   return true;
 }
 
-long long count_of(const View4& v) { return v.n[0] * v.n[1] * v.n[2] * v.n[3]; }
 
 // Elements from the first to the last one the view reaches (strides >= 0).
 long long extent_of(const View4& v) {
@@ -436,6 +435,32 @@ __global__ void mirror_rows_kernel(const uint16_t* __restrict__ src, uint16_t* d
     dst[a] = src[m];
   }
 }
+
+// Eight 16-bit elements of a 16-byte word in reverse order.
+__device__ __forceinline__ uint4 rev8(uint4 v) {
+  const auto sw = [](uint32_t w) { return __byte_perm(w, 0, 0x1032); };  // swap the halves
+  return make_uint4(sw(v.w), sw(v.z), sw(v.y), sw(v.x));
+}
+
+// The same with rows of L = 8 k elements and 16-byte aligned rows: one 16-byte piece per thread
+// (copy), or, in place, a piece and its mirror image swapped (the middle piece of an odd count
+// reversed by itself).
+__global__ void mirror_rows8_kernel(const uint4* __restrict__ src, uint4* dst, long long rows,
+                                    int L8, int in_place) {
+  const long long per = in_place ? (L8 + 1) / 2 : L8;
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= rows * per) return;
+  const long long r = i / per;
+  const int p = (int)(i % per);
+  const long long a = r * L8 + p, m = r * L8 + (L8 - 1 - p);
+  if (in_place) {
+    const uint4 x = dst[a], y = dst[m];
+    dst[a] = rev8(y);
+    if (m != a) dst[m] = rev8(x);
+  } else {
+    dst[a] = rev8(__ldcs(src + m));
+  }
+}
 }  // namespace
 
 namespace ssm {
@@ -443,6 +468,16 @@ namespace ssm {
 // [rows][L] of 16-bit elements from src into dst mirrored, or in place when src == dst.
 cudaError_t mirror_rows(const void* src, void* dst, long long rows, int L, cudaStream_t s) {
   const int in_place = src == dst ? 1 : 0;
+  const bool v8 = L % 8 == 0 && (reinterpret_cast<uintptr_t>(src) & 15) == 0 &&
+                  (reinterpret_cast<uintptr_t>(dst) & 15) == 0;
+  if (v8) {
+    const int L8 = L / 8;
+    const long long n = rows * (in_place ? (L8 + 1) / 2 : L8);
+    if (n <= 0) return cudaSuccess;
+    mirror_rows8_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
+        reinterpret_cast<const uint4*>(src), reinterpret_cast<uint4*>(dst), rows, L8, in_place);
+    return cudaGetLastError();
+  }
   const long long n = rows * (in_place ? L / 2 : L);
   if (n <= 0) return cudaSuccess;
   mirror_rows_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(

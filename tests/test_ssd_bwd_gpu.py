@@ -275,11 +275,14 @@ def test_chunked_reverse_forward_matches_oracle(N):
 
 
 @pytest.mark.parametrize("N", [16, 64, 128])
-def test_chunked_reverse_backward_matches_oracle(N):
+@pytest.mark.parametrize("shape", [(2, 128, 333), (1, 64, 512), (1, 64, 520)])
+def test_chunked_reverse_backward_matches_oracle(N, shape):
     """The reverse scan's backward in the chunked form, recomputing its states and from the
-    reverse forward's checkpoints, with dhL and h0, over a ragged length."""
-    x = inputs(2, 128, 333, N, torch.bfloat16, seed=123)
-    dhL = torch.randn((2, 128, N), generator=torch.Generator().manual_seed(13))
+    reverse forward's checkpoints, with dhL and h0.  Lengths: ragged (element-wise mirror
+    copies), a multiple of 16, and 65 pieces of 8 (the in-place mirror's middle piece)."""
+    batch, dim, L = shape
+    x = inputs(batch, dim, L, N, torch.bfloat16, seed=123)
+    dhL = torch.randn((batch, dim, N), generator=torch.Generator().manual_seed(13))
     r = ref(x, dhL, reverse=True)
     g = run(x, dhL, reverse=True)
     for k in GRADS:
