@@ -161,20 +161,21 @@ SSM_API int ssm_scan_bwd(const void* u, const void* delta, const float* A, const
  * 16-step chunk and 64-channel tile, the products C B^T, masked with the decay factors, times
  * the step-scaled inputs, plus C times the entering state: the structured-matrix view of the
  * scan in the Mamba-2 notes of the same page) on the tensor cores.  That form takes bf16 io,
- * dstate 16, 32, 64 or 128, no SSM_ZOH, the default layout and B/C groups of whole 64-channel
- * tiles; other forward requests with dstate > 16 return SSM_EUNSUPPORTED.  With SSM_REVERSE
+ * dstate 16, 32, 64 or 128, the default layout and B/C groups of whole 64-channel tiles (with
+ * SSM_ZOH: the coefficient (e^{ΔA} - 1)/A by the library expm1f); other forward requests with
+ * dstate > 16 return SSM_EUNSUPPORTED.  With SSM_REVERSE
  * (dstate > 16; ssm_scan_fwd_ex) it scans the inputs mirrored along time into the workspace
  * and mirrors the output back in place, so ssm_scan_fwd_ex_workspace_size() then covers those
  * copies (u, delta, z, B, C) too.  Its checkpoints (ckpt, 16-byte aligned) have the layout and meaning of the
  * per-state scan's: the f32 state entering every 16-step block, [batch][dim][ceil(L/16)][dstate].
- * For bf16 io, no flag but SSM_SCALAR_A (and SSM_REVERSE: mirrored copies of u, delta, z, dout,
- * B, C in the workspace, the gradients along time mirrored back in place) and B/C shared or in
+ * For bf16 io, no flag but SSM_SCALAR_A, SSM_ZOH and SSM_REVERSE (mirrored copies of u, delta,
+ * z, dout, B, C in the workspace, the gradients along time mirrored back in place) and B/C shared or in
  * groups of whole 64-channel tiles, the backward with dstate = 16, 32, 64 or 128 runs in the
  * chunked matrix form too: the chunks
  * are walked in reverse with the adjoint of the state (the chain rule through the products
  * above), from the caller's checkpoints (either forward's; 16-byte aligned) or, with
  * ckpt = NULL, from a checkpoint pass into the workspace.  Other requests with dstate > 16
- * (f32, ZOH, other groupings) take ckpt = NULL and run as the sum of the 16-state
+ * (f32, other groupings) take ckpt = NULL and run as the sum of the 16-state
  * backwards of the state slices (the states of a scalar-decay scan do not interact; D enters
  * one slice); with dstate <= 16 they run the per-state backward.
  * ssm_scan_bwd_scalar_a_workspace_size() covers the scratch of the path the call takes (chunk

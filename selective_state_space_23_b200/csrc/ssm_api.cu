@@ -417,12 +417,12 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
                          (bc_groups == 1 || (dim % bc_groups == 0 && (dim / bc_groups) % 64 == 0)) &&
                          !(sform && strcmp(sform, "state") == 0);
   if (dstate > SSM_MAX_DSTATE || chunked16) {
-    if (io_dtype != SSM_BF16 || (dstate != 16 && dstate != 32 && dstate != 64 && dstate != 128) || zoh ||
+    if (io_dtype != SSM_BF16 || (dstate != 16 && dstate != 32 && dstate != 64 && dstate != 128) ||
         channels_last ||
         !(bc_groups == 1 || (dim % bc_groups == 0 && (dim / bc_groups) % 64 == 0)))
       return fail(SSM_EUNSUPPORTED,
-                  "scalar decay with dstate %d > %d needs bf16 io, dstate 32, 64 or 128, no "
-                  "ZOH, the default layout and B/C groups of whole 64-channel tiles", dstate,
+                  "scalar decay with dstate %d > %d needs bf16 io, dstate 32, 64 or 128, the "
+                  "default layout and B/C groups of whole 64-channel tiles", dstate,
                   SSM_MAX_DSTATE);
     if (!aligned16(ckpt))
       return fail(SSM_EINVAL, "ckpt must be 16-byte aligned (chunked matrix form)");
@@ -463,6 +463,7 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
     a.batch = batch; a.dim = dim; a.L = seqlen; a.N = dstate;
     a.softplus = delta_softplus ? 1 : 0;
     a.scalar_a = 1;
+    a.zoh = zoh ? 1 : 0;
     a.bc_groups = bc_groups;
     a.rows16 = vec ? 1 : 0;
     FwdPlan plan = plan_ssd(batch, dim, seqlen, dstate);
@@ -915,7 +916,7 @@ namespace {
 bool chunked_bwd_ok(int dim, int dstate, int bc_groups, int io_dtype, int flags) {
   const char* v = getenv("SSM_SCALAR_BWD");  // "slices" / "state": the per-state kernels
   if (v && (strcmp(v, "slices") == 0 || strcmp(v, "state") == 0)) return false;
-  return io_dtype == SSM_BF16 && (flags & ~SSM_REVERSE) == SSM_SCALAR_A &&
+  return io_dtype == SSM_BF16 && (flags & ~(SSM_REVERSE | SSM_ZOH)) == SSM_SCALAR_A &&
          (dstate == 16 || dstate == 32 || dstate == 64 || dstate == 128) &&
          (bc_groups == 1 || (bc_groups < dim && dim % bc_groups == 0 && (dim / bc_groups) % 64 == 0));
 }
@@ -977,7 +978,7 @@ int scan_bwd_chunked(const void* u, const void* delta, const float* A, const voi
                      const float* ckpt, void* du, void* ddelta, float* dA, void* dB, void* dC, float* dD, void* dz,
                      float* ddt_bias, float* dh0, void* workspace, size_t workspace_bytes,
                      int batch, int dim, int seqlen, int dstate, int bc_groups, bool reverse,
-                     void* stream) {
+                     bool zoh, void* stream) {
   const size_t es = 2;
   const size_t nx = (size_t)batch * dim * seqlen * es;
   const size_t nbc = (size_t)batch * bc_groups * dstate * seqlen * es;
@@ -1058,6 +1059,7 @@ int scan_bwd_chunked(const void* u, const void* delta, const float* A, const voi
     a.batch = batch; a.dim = dim; a.L = seqlen; a.N = dstate;
     a.softplus = delta_softplus ? 1 : 0;
     a.scalar_a = 1;
+    a.zoh = zoh ? 1 : 0;
     a.bc_groups = bc_groups;
     a.rows16 = vec ? 1 : 0;
     const FwdPlan plan = plan_ssd(batch, dim, seqlen, dstate);
@@ -1101,6 +1103,7 @@ int scan_bwd_chunked(const void* u, const void* delta, const float* A, const voi
   b.softplus = delta_softplus ? 1 : 0;
   b.rows16 = vec ? 1 : 0;
   b.need_bc = (dB || dC) ? 1 : 0;
+  b.zoh = zoh ? 1 : 0;
   b.nseg = l.seg.nseg;
   b.cps = l.seg.cps;
   if (l.seg.nseg > 1) {
@@ -1188,7 +1191,7 @@ int ssm_scan_bwd_ex(const void* u, const void* delta, const float* A, const void
       return scan_bwd_chunked(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL,
                               ckpt, du, ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, workspace,
                               workspace_bytes, batch, dim, seqlen, dstate, bc_groups, reverse,
-                              stream);
+                              zoh, stream);
     return ssm::scan_bwd_slices(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL,
                                 ckpt, du, ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, workspace,
                                 workspace_bytes, batch, dim, seqlen, dstate, bc_groups, io_dtype,
@@ -1200,7 +1203,7 @@ int ssm_scan_bwd_ex(const void* u, const void* delta, const float* A, const void
     return scan_bwd_chunked(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL, ckpt,
                             du, ddelta, dA, dB, dC, dD, dz, ddt_bias, dh0, workspace,
                             workspace_bytes, batch, dim, seqlen, dstate, bc_groups, reverse,
-                            stream);
+                            zoh, stream);
   }
   if (!(flags & SSM_SCALAR_A))
     return scan_bwd_core(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, dout, dhL, ckpt,

@@ -150,6 +150,7 @@ struct SsdBwdArgs {
   const float* mu_in;
   int nseg, cps;
   int batch, dim, L, N, bc_groups, softplus, rows16, need_bc;
+  int zoh;  // zero-order-hold input coefficient (e^{ΔA} - 1)/A instead of Δ
 };
 // 64 channels per CTA (dim / bc_groups a multiple of 64 with groups); a.ck from launch_ssd_fwd's
 // checkpoint mode.  The finishing launch sums part_bc over each group's CTAs into dB, dC (bf16)

@@ -37,6 +37,20 @@ __device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uin
   lo = pack_bf16x2(a - bf16_lo(hi), b - bf16_hi(hi));
 }
 
+// Zero-order-hold input coefficient of a step Δ with one rate A per channel (the chunked form):
+// c = (e^{ΔA} - 1)/A (library expm1f; Δ as A -> 0), its derivatives dc/dΔ = e^{ΔA} and
+// dc/dA = Δ² φ'(ΔA) with φ(z) = (e^z - 1)/z: the series 1/2 + z/3 + z²/8 + z³/30 + z⁴/144 for
+// |z| < 1/8 (truncation below 4e-8 relative), else (Δ e^{ΔA} - c)/A, which no longer cancels.
+__device__ __forceinline__ float zoh_c(float d, float A) {
+  return fabsf(A) < 1e-20f ? d : expm1f(d * A) / A;
+}
+__device__ __forceinline__ float zoh_dc_da(float d, float A, float c) {
+  const float z = d * A;
+  if (fabsf(z) < 0.125f)
+    return d * d * fmaf(z, fmaf(z, fmaf(z, fmaf(z, 1.f / 144.f, 1.f / 30.f), 0.125f), 1.f / 3.f), 0.5f);
+  return (d * expf(z) - c) / A;
+}
+
 // The transpose of an 8x8 b16 matrix held one pair per lane (lane l: row l / 4, cols 2 (l % 4),
 // +1), returned in the same layout.
 __device__ __forceinline__ uint32_t movt(uint32_t a) {

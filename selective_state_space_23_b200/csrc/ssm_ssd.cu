@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
         const float D = a.softplus ? softplus_fast(v) : v;
         dl[c][j] = live ? D : 0.f;
         uv[c][j] = live ? u : 0.f;
-        xv[c][j] = dl[c][j] * uv[c][j];
+        xv[c][j] = (a.zoh ? zoh_c(dl[c][j], al[c] * kLn2) : dl[c][j]) * uv[c][j];
         if (zp && !NOOUT) {
           const float z = (j & 1) ? bf16_hi(wz) : bf16_lo(wz);
           gt[c][j] = z * sigmoid_fast(z);

@@ -151,6 +151,7 @@ FWD_CASES = {
     "chunked_n64": ({}, 2, 96, 200, 64, torch.bfloat16, 1, 1),
     "chunked_n128_split": ({"SSM_SSD_SPLIT": "3"}, 1, 80, 333, 128, torch.bfloat16, 1, 1),
     "chunked_n64_reverse": ({}, 1, 80, 333, 64, torch.bfloat16, 1, 1 | 2),
+    "chunked_n64_zoh": ({}, 1, 80, 333, 64, torch.bfloat16, 1, 1 | 4),
 }
 
 
@@ -194,6 +195,7 @@ BWD_CASES = {
     "scalar_decay_n128_chunked": ({}, 1, 80, 333, 128, torch.bfloat16, 1, 1),
     "scalar_decay_n64_chunked_split": ({"SSM_SSD_BWD_SPLIT": "3"}, 1, 80, 333, 64, torch.bfloat16, 1, 1),
     "scalar_decay_n64_chunked_reverse": ({}, 1, 80, 333, 64, torch.bfloat16, 1, 1 | 2),
+    "scalar_decay_n64_chunked_zoh": ({}, 1, 80, 333, 64, torch.bfloat16, 1, 1 | 4),
 }
 
 

@@ -291,3 +291,53 @@ def test_chunked_reverse_backward_matches_oracle(N, shape):
     g2 = run(x, dhL, reverse=True, ckpt=ck)
     for k in GRADS:
         assert_close(g2[k], r[k], torch.bfloat16, k)
+
+
+# ------------------------------------------------------------------ the zero-order hold
+@pytest.mark.parametrize("N", [32, 64, 128])
+@pytest.mark.parametrize("reverse", [False, True])
+def test_chunked_zoh_forward_matches_oracle(N, reverse):
+    """The zero-order-hold input coefficient (e^{ΔA} - 1)/A in the chunked forward, either
+    direction: outputs and final state against the oracle."""
+    x = inputs(2, 128, 333, N, torch.bfloat16, seed=124)
+    out, hL = fwd(x, zoh=True, reverse=reverse, return_final_state=True)
+    c = lambda k: f64(x[k])
+    A = np.repeat(c("A")[:, None], N, axis=1)
+    r = oracle.scan_fwd(c("u"), c("delta"), A, c("B"), c("C"), D=c("D"), z=c("z"),
+                        dt_bias=c("dt_bias"), h0=c("h0"), zoh=True, reverse=reverse)
+    assert_close(out, r["out"], torch.bfloat16, "out")
+    assert_close(hL, r["hL"], torch.bfloat16, "hL")
+
+
+@pytest.mark.parametrize("N", [16, 64, 128])
+@pytest.mark.parametrize("reverse", [False, True])
+def test_chunked_zoh_backward_matches_oracle(N, reverse):
+    """The zero-order hold's gradients in the chunked backward (through c's step and rate),
+    either direction, with dhL and h0, recomputed and from the forward's checkpoints."""
+    x = inputs(2, 128, 333, N, torch.bfloat16, seed=125)
+    dhL = torch.randn((2, 128, N), generator=torch.Generator().manual_seed(14))
+    r = ref(x, dhL, zoh=True, reverse=reverse)
+    g = run(x, dhL, zoh=True, reverse=reverse)
+    for k in GRADS:
+        assert_close(g[k], r[k], torch.bfloat16, k)
+    if N > 16:
+        _, ck = fwd(x, zoh=True, reverse=reverse, return_ckpt=True)
+        g2 = run(x, dhL, zoh=True, reverse=reverse, ckpt=ck)
+        for k in GRADS:
+            assert_close(g2[k], r[k], torch.bfloat16, k)
+
+
+def test_chunked_zoh_large_and_small_rates():
+    """Rates from 1e-6 to 30 (the dc/dA series near ΔA = 0 and the direct form far from it),
+    with steps up to 30 (chunks out of the factorisation's range): gradients against the
+    oracle."""
+    x = inputs(1, 64, 160, 64, torch.bfloat16, seed=126)
+    a = np.geomspace(1e-6, 30, 64).astype(np.float32)
+    x["A"] = -torch.from_numpy(a)
+    v = np.random.default_rng(7).uniform(-12, 6, size=x["delta"].shape).astype(np.float32)
+    x["delta"] = torch.from_numpy(v).to(torch.bfloat16)
+    x["dt_bias"] = torch.zeros_like(x["dt_bias"])
+    r = ref(x, None, zoh=True)
+    g = run(x, None, zoh=True)
+    for k in GRADS:
+        assert_close(g[k], r[k], torch.bfloat16, k)
