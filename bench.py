@@ -511,6 +511,19 @@ def _decode(dev, rnd, prm, timeit):
                           "hbm_gbs": byt / (us * 1e-6) / 1e9,
                           "l2": "flushed before each step by reading 256 MB",
                           "us_per_step_state_in_l2": t_hot}
+    del state, flush
+    # one rate per channel with 64 and 128 states (a Mamba-2 layer's decode): the state (335 and
+    # 671 MB) is larger than L2, so no flush is needed
+    A1 = -(torch.rand(d, device=dev) * 15.0 + 1.0)
+    for N2 in (64, 128):
+        st2 = torch.zeros((b, d, N2), device=dev)
+        B2, C2 = rnd((b, N2)), rnd((b, N2))
+        t2 = timeit(lambda: ssm.ssm_state_update(st2, x, dtr, A1, B2, C2, D=D, z=zz, dt_bias=bias,
+                                                 scalar_a=True), 50) * 1e3
+        byt2 = 2 * b * d * N2 * 4 + 4 * b * d * 2 + 2 * b * N2 * 2
+        out[f"decode_b256_scalar_n{N2}"] = {"shape": f"256x5120x{N2} f32 state, bf16 io, A [dim]",
+                                            "us_per_step": t2, "hbm_gbs": byt2 / (t2 * 1e-6) / 1e9}
+        del st2
     return out
 
 

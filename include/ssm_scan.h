@@ -326,7 +326,9 @@ SSM_API int ssm_state_update(float* state, const void* x, const void* dt, const 
  * group d / (dim / bc_groups); dim / bc_groups a multiple of 16 when 1 < bc_groups < dim;
  * bc_groups == dim gives B, C per channel, [batch][dim][dstate]).  A decode
  * step runs forward in time: SSM_REVERSE is rejected with SSM_EINVAL, as is any unknown bit.
- * Calling it L times reproduces ssm_scan_fwd_ex with the same flags and groups.
+ * Calling it L times reproduces ssm_scan_fwd_ex with the same flags and groups.  With
+ * SSM_SCALAR_A, dstate may also be 32, 64 or 128 (the state sizes of the chunked scan; the
+ * state 16-byte aligned, else SSM_EINVAL); other dstate > 16 return SSM_EUNSUPPORTED.
  */
 SSM_API int ssm_state_update_ex(float* state, const void* x, const void* dt, const float* A,
                                 const void* B, const void* C, const float* D, const void* z,

@@ -1368,9 +1368,16 @@ int ssm_state_update_ex(float* state, const void* x, const void* dt, const float
   g_err[0] = 0;
   if (flags & ~(SSM_SCALAR_A | SSM_ZOH))
     return fail(SSM_EINVAL, "unsupported flags 0x%x for a decode step", flags);
-  TRY(check_dims(batch, dim, 1, dstate, io_dtype));
-  TRY(check_groups(dim, bc_groups));
   const bool scalar_a = (flags & SSM_SCALAR_A) != 0;
+  // one rate per channel also takes N = 32, 64 or 128 (the chunked scan's state sizes)
+  TRY(check_dims(batch, dim, 1, dstate, io_dtype, scalar_a ? SSM_MAX_DSTATE_SCALAR : SSM_MAX_DSTATE));
+  TRY(check_groups(dim, bc_groups));
+  if (dstate > SSM_MAX_DSTATE) {
+    if (dstate != 32 && dstate != 64 && dstate != 128)
+      return fail(SSM_EUNSUPPORTED, "a decode step with dstate %d > %d takes 32, 64 or 128",
+                  dstate, SSM_MAX_DSTATE);
+    if (!aligned16(state)) return fail(SSM_EINVAL, "state must be 16-byte aligned for dstate > 16");
+  }
   const size_t es = esize(io_dtype);
   const size_t nx = (size_t)batch * dim * es;
   const size_t nbc = (size_t)batch * bc_groups * dstate * es;

@@ -42,6 +42,14 @@ template <> __device__ __forceinline__ void st_io<uint16_t>(void* p, long long i
 
 // SSM_DECODE_STREAM=0 selects the per-thread form of the N = 16 decode step instead of the
 // streamed one (for measurements; both compute the same arithmetic).
+// float4 state vectors per lane of the one-rate decode with more than 16 states (1, 2 or 4;
+// SSM_DECODE_VECTORS overrides the default)
+int decode_scalar_vectors() {
+  const char* v = getenv("SSM_DECODE_VECTORS");
+  const int n = v ? atoi(v) : 2;
+  return (n == 1 || n == 2 || n == 4) ? n : 2;
+}
+
 bool getenv_stream_enabled() {
   const char* v = getenv("SSM_DECODE_STREAM");
   return !(v && v[0] == '0');
@@ -106,6 +114,59 @@ __global__ void __launch_bounds__(256) decode_kernel(const DecodeArgs a) {
     for (int i = 0; i < 4; ++i)
       if (4 * q + i < N) sp[i] = h[i];
   }
+  if (q == 0) {
+    y += (a.D ? a.D[d] : 0.f) * xv;
+    if (a.z) {
+      const float zv = ld_io<IO>(a.z, ch);
+      y *= zv * (kPrecise ? sigmoid_precise(zv) : sigmoid_fast(zv));
+    }
+    st_io<IO>(a.out, ch, y);
+  }
+}
+
+// One decay rate per channel with N = 32, 64 or 128 states (the state sizes of the scan's
+// chunked matrix form): LPC lanes per channel, V x 4 states each (N = 4 V LPC), the state V
+// 128-bit loads and stores per lane, all issued before the first is used.  With one rate per
+// channel the decay and the input coefficient are formed once per lane (rounded as in the other
+// decode forms); the readout is a shuffle reduction over the channel's lanes.
+template <typename IO, int LPC, int V>
+__global__ void __launch_bounds__(256) decode_scalar_kernel(const DecodeArgs a) {
+  constexpr bool kPrecise = std::is_same<IO, float>::value;
+  constexpr int N = 4 * V * LPC;
+  const long long nch = (long long)a.batch * a.dim;
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const bool act = gid / LPC < nch;
+  const long long ch = act ? gid / LPC : nch - 1;  // idle lanes shadow a valid channel
+  const int q = (int)(gid % LPC);                    // states [4Vq, 4Vq + 4V)
+  const int b = (int)(ch / a.dim), d = (int)(ch % a.dim);
+
+  const float xv = ld_io<IO>(a.x, ch);
+  const float v = ld_io<IO>(a.dt, ch) + (a.dt_bias ? a.dt_bias[d] : 0.f);
+  const float dt = !a.softplus ? v : (kPrecise ? softplus_precise(v) : softplus_fast(v));
+  const float An = a.A[d] * ((kPrecise || a.zoh) ? 1.f : kLog2e);
+  const float abar = (kPrecise || a.zoh) ? expf(dt * An) : ex2_mufu(dt * An);
+  const float bx = (a.zoh ? decode_coef(dt, An, true) : dt) * xv;
+
+  float4* sp = reinterpret_cast<float4*>(a.state + ch * N) + V * q;
+  float4 h[V];
+#pragma unroll
+  for (int k = 0; k < V; ++k) h[k] = sp[k];
+  const long long bc = ((long long)b * a.bc_groups + d / (a.dim / a.bc_groups)) * N + 4 * V * q;
+  float y = 0.f;
+#pragma unroll
+  for (int k = 0; k < V; ++k) {
+    float* hk = reinterpret_cast<float*>(&h[k]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      hk[i] = fmaf(abar, hk[i], bx * ld_io<IO>(a.B, bc + 4 * k + i));
+      y = fmaf(ld_io<IO>(a.C, bc + 4 * k + i), hk[i], y);
+    }
+  }
+#pragma unroll
+  for (int m = 1; m < LPC; m <<= 1) y += __shfl_xor_sync(0xffffffffu, y, m);
+  if (!act) return;
+#pragma unroll
+  for (int k = 0; k < V; ++k) sp[k] = h[k];
   if (q == 0) {
     y += (a.D ? a.D[d] : 0.f) * xv;
     if (a.z) {
@@ -416,6 +477,34 @@ cudaError_t launch_io(const DecodeArgs& a, cudaStream_t s) {
                          al16(a.x) && al16(a.dt) && (a.z == nullptr || al16(a.z)) &&
                          kNS * sizeof(IO) % 16 == 0 && getenv_stream_enabled();
   if (stream_ok) return launch_stream<IO>(a, s);
+  if (a.N > kNS) {  // one rate per channel, N = 32, 64 or 128, 16-byte aligned state (host-checked)
+    const int V = decode_scalar_vectors();
+    const long long threads = (long long)a.batch * a.dim * (a.N / (4 * V));
+    const unsigned grid = (unsigned)((threads + tpb - 1) / tpb);
+    if (V == 1) {
+      switch (a.N) {
+        case 32: decode_scalar_kernel<IO, 8, 1><<<grid, tpb, 0, s>>>(a); break;
+        case 64: decode_scalar_kernel<IO, 16, 1><<<grid, tpb, 0, s>>>(a); break;
+        case 128: decode_scalar_kernel<IO, 32, 1><<<grid, tpb, 0, s>>>(a); break;
+        default: return cudaErrorInvalidValue;
+      }
+    } else if (V == 2) {
+      switch (a.N) {
+        case 32: decode_scalar_kernel<IO, 4, 2><<<grid, tpb, 0, s>>>(a); break;
+        case 64: decode_scalar_kernel<IO, 8, 2><<<grid, tpb, 0, s>>>(a); break;
+        case 128: decode_scalar_kernel<IO, 16, 2><<<grid, tpb, 0, s>>>(a); break;
+        default: return cudaErrorInvalidValue;
+      }
+    } else {
+      switch (a.N) {
+        case 32: decode_scalar_kernel<IO, 2, 4><<<grid, tpb, 0, s>>>(a); break;
+        case 64: decode_scalar_kernel<IO, 4, 4><<<grid, tpb, 0, s>>>(a); break;
+        case 128: decode_scalar_kernel<IO, 8, 4><<<grid, tpb, 0, s>>>(a); break;
+        default: return cudaErrorInvalidValue;
+      }
+    }
+    return cudaGetLastError();
+  }
   if (a.N == kNS && al16(a.state) && (a.scalar_a || al16(a.A)) && al16(a.B) && al16(a.C)) {
     const long long threads = (long long)a.batch * a.dim * 2;
     decode16_kernel<IO><<<(unsigned)((threads + tpb - 1) / tpb), tpb, 0, s>>>(a);

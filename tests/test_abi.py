@@ -213,3 +213,13 @@ def test_strided_entry_points_check_on_the_host(lib):
     assert lib.ssm_state_update_strided(*dargs, _abi.SSM_REVERSE, ctypes.byref(dst),
                                         None) == _abi.SSM_EINVAL
     assert lib.ssm_state_update_strided(*dargs, 0, ctypes.byref(dst), None) == _abi.SSM_EWORKSPACE
+
+
+def test_large_n_decode_is_checked_on_the_host(lib):
+    """Decode steps: per-state rates stop at 16 states; one rate per channel takes 32, 64 or 128
+    (refused before any launch)."""
+    assert lib.ssm_state_update_ex(*([None] * 9), 1, None, 2, 64, 64, 1, 1, 0, None) == \
+        _abi.SSM_EUNSUPPORTED
+    assert lib.ssm_state_update_ex(*([None] * 9), 1, None, 2, 64, 48, 1, 1, _abi.SSM_SCALAR_A,
+                                   None) == _abi.SSM_EUNSUPPORTED
+    assert b"32, 64 or 128" in lib.ssm_last_error()

@@ -220,18 +220,20 @@ def test_backward_stays_inside_its_tensors(monkeypatch, case):
 
 
 DECODE_CASES = {
-    # name: (env, batch, dim, N, io, G)
-    "streamed": ({}, 7, 384, 16, torch.bfloat16, 1),
-    "streamed_grouped": ({}, 5, 384, 16, torch.float32, 3),
-    "per_thread": ({"SSM_DECODE_STREAM": "0"}, 7, 96, 16, torch.bfloat16, 1),
-    "per_thread_ragged": ({}, 3, 40, 5, torch.float32, 1),
-    "per_channel_bc": ({}, 3, 40, 16, torch.bfloat16, 40),
+    # name: (env, batch, dim, N, io, G, flags)
+    "streamed": ({}, 7, 384, 16, torch.bfloat16, 1, 0),
+    "streamed_grouped": ({}, 5, 384, 16, torch.float32, 3, 0),
+    "per_thread": ({"SSM_DECODE_STREAM": "0"}, 7, 96, 16, torch.bfloat16, 1, 0),
+    "per_thread_ragged": ({}, 3, 40, 5, torch.float32, 1, 0),
+    "per_channel_bc": ({}, 3, 40, 16, torch.bfloat16, 40, 0),
+    "scalar_n64": ({}, 3, 40, 64, torch.bfloat16, 1, 1),
+    "scalar_n128_grouped_zoh": ({}, 3, 64, 128, torch.float32, 2, 1 | 4),
 }
 
 
 @pytest.mark.parametrize("case", sorted(DECODE_CASES))
 def test_decode_stays_inside_its_tensors(monkeypatch, case):
-    env, batch, dim, N, io, G = DECODE_CASES[case]
+    env, batch, dim, N, io, G, flags = DECODE_CASES[case]
     monkeypatch.delenv("SSM_DECODE_STREAM", raising=False)
     for k, v in env.items():
         monkeypatch.setenv(k, v)
@@ -239,7 +241,8 @@ def test_decode_stays_inside_its_tensors(monkeypatch, case):
     rnd = lambda *s: torch.randn(*s, generator=gen)
     state0 = 0.5 * rnd(batch, dim, N)
     vals = {"x": rnd(batch, dim).to(io), "dt": (0.3 * rnd(batch, dim)).to(io),
-            "z": rnd(batch, dim).to(io), "A": -torch.rand(dim, N, generator=gen) * 4 - 0.1,
+            "z": rnd(batch, dim).to(io),
+            "A": -torch.rand(*((dim,) if flags & 1 else (dim, N)), generator=gen) * 4 - 0.1,
             "B": rnd(batch, G, N).to(io), "C": rnd(batch, G, N).to(io), "D": rnd(dim),
             "dt_bias": 0.1 * rnd(dim)}
     res = []
@@ -251,7 +254,7 @@ def test_decode_stays_inside_its_tensors(monkeypatch, case):
         out = ar.out((batch, dim), io)
         rc = _abi.lib().ssm_state_update_ex(p(st), p(t["x"]), p(t["dt"]), p(t["A"]), p(t["B"]),
                                             p(t["C"]), p(t["D"]), p(t["z"]), p(t["dt_bias"]), 1,
-                                            p(out), batch, dim, N, G, IO_CODE[io], 0, 0)
+                                            p(out), batch, dim, N, G, IO_CODE[io], flags, 0)
         _abi.check(rc, "ssm_state_update_ex")
         ar.check_margins()
         res.append([out.clone(), st.clone()])
