@@ -489,9 +489,10 @@ def _decode(dev, rnd, prm, timeit):
     import selective_state_space_23_b200 as ssm
     out = {}
     N = 16
-    # decode: 256 x 5120 x 16 state.  The 84 MB state fits in L2 (126 MB), so L2 is flushed
-    # before every step by READING 256 MB (clean lines: no write-back lands inside the step) and
-    # the state comes from HBM; the flush is timed separately and subtracted
+    # decode: 256 x 5120 x 16 state.  The 84 MB state fits in L2 (126 MB).  Side figures: L2
+    # flushed before every step by READING 256 MB (the flush is timed separately and
+    # subtracted; the previous step's dirty state is written back during the flush and so
+    # counted), and the state left in L2.  Main figure: below, one state per layer
     b, d = 256, 5120
     state = torch.zeros((b, d, N), device=dev)
     x, dtr, zz = rnd((b, d)), rnd((b, d), 0.5), rnd((b, d))
@@ -507,11 +508,24 @@ def _decode(dev, rnd, prm, timeit):
     t_hot = timeit(lambda: ssm.ssm_state_update(state, x, dtr, A, Bd, Cd, D=D, z=zz,
                                                 dt_bias=bias), 50) * 1e3
     byt = 2 * b * d * N * 4 + 4 * b * d * 2 + 2 * b * N * 2
-    out["decode_b256"] = {"shape": "256x5120x16 f32 state, bf16 io", "us_per_step": us,
-                          "hbm_gbs": byt / (us * 1e-6) / 1e9,
-                          "l2": "flushed before each step by reading 256 MB",
+    del flush
+    # the steps of a model with several layers: each step updates another layer's state (4 of
+    # them, 336 MB, more than twice L2), so no step finds its state in L2 and every step's
+    # written state leaves L2 during later steps, as in a decode over many layers
+    states = [state] + [torch.zeros((b, d, N), device=dev) for _ in range(3)]
+    cyc = [0]
+
+    def layer_step():
+        st = states[cyc[0] % len(states)]
+        cyc[0] += 1
+        ssm.ssm_state_update(st, x, dtr, A, Bd, Cd, D=D, z=zz, dt_bias=bias)
+    t_rot = timeit(layer_step, 48) * 1e3
+    out["decode_b256"] = {"shape": "256x5120x16 f32 state, bf16 io",
+                          "us_per_step": t_rot, "hbm_gbs": byt / (t_rot * 1e-6) / 1e9,
+                          "l2": "each step updates another of 4 layer states (336 MB)",
+                          "us_per_step_after_read_flush": us,
                           "us_per_step_state_in_l2": t_hot}
-    del state, flush
+    del state, states
     # one rate per channel with 64 and 128 states (a Mamba-2 layer's decode): the state (335 and
     # 671 MB) is larger than L2, so no flush is needed
     A1 = -(torch.rand(d, device=dev) * 15.0 + 1.0)
