@@ -161,7 +161,8 @@ cudaError_t launch_ssd_bwd_finish(const SsdBwdArgs& a, void* dB, void* dC, float
 int ssd_bwd_ctas_per_row(int dim);
 // mode: kSsdOut (with a.ckpt also the checkpoints), kSsdSummary, or kSsdCkpt (no outputs; only
 // the state entering every 16-step chunk into a.ckpt, f32 [batch][dim][ceil(L / 16)][N]).
-enum SsdMode { kSsdOut = 0, kSsdSummary = 1, kSsdCkpt = 2 };
+// kSsdOutCkpt is kSsdOut with checkpoints (chosen by the launcher when a.ckpt is set).
+enum SsdMode { kSsdOut = 0, kSsdSummary = 1, kSsdCkpt = 2, kSsdOutCkpt = 3 };
 cudaError_t launch_ssd_fwd(const FwdArgs& a, int mode, cudaStream_t s);
 cudaError_t launch_fwd_carry(const FwdArgs& a, const float* summ, const float* dsum, float* hin,
                              cudaStream_t s);

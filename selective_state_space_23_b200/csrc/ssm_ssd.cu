@@ -47,6 +47,8 @@
 #include <stdint.h>
 #include <stdlib.h>
 
+#include <type_traits>
+
 #include "ssm_device.cuh"
 #include "ssm_kernels.h"
 #include "ssm_mma.cuh"
@@ -88,15 +90,17 @@ __device__ __forceinline__ void store_state(const FwdArgs& a, const float (&Ht)[
   }
 }
 
-// MODE: kSsdOut (gated outputs; with a.ckpt also the state entering every chunk),
+// MODE: kSsdOut (gated outputs), kSsdOutCkpt (and the state entering every chunk into a.ckpt),
 // kSsdSummary (segment end state and ΣΔ from zero), kSsdCkpt (only the state entering every
-// chunk into a.ckpt, for the backward).
-template <int N, int W, int MODE>
+// chunk into a.ckpt, for the backward).  ZOH: the zero-order-hold input coefficient.  Both are
+// template parameters so that the plain output kernel carries no code of the others.
+template <int N, int W, int MODE, bool ZOH>
 __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__ FwdArgs a) {
   constexpr bool SUMMARY = MODE == kSsdSummary;
-  constexpr bool NOOUT = MODE != kSsdOut;  // no gate, readout or outputs
+  constexpr bool NOOUT = MODE == kSsdSummary || MODE == kSsdCkpt;  // no gate, readout or outputs
+  constexpr bool CKPT = MODE == kSsdCkpt || MODE == kSsdOutCkpt;    // checkpoints written
   // states that a backward or a chain reads take the state update's remainder term too
-  const bool exact = NOOUT || a.ckpt != nullptr;
+  constexpr bool EXACT = MODE != kSsdOut;
   constexpr int kNT = N / 8;  // n8 tiles of the state
   extern __shared__ float4 smem_ssd[];
   SsdStage<N>* ring = reinterpret_cast<SsdStage<N>*>(smem_ssd);
@@ -202,7 +206,7 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
     if (k + 1 < nchunk) load_in(k + 1, nxt);
     const SsdStage<N>& st = ring[k % kStages];
     const int t0 = (kc0 + k) * kT;
-    if (MODE == kSsdCkpt || (MODE == kSsdOut && a.ckpt)) store_state<N>(a, Ht, kc0 + k, b, dch, act, tg);
+    if (CKPT) store_state<N>(a, Ht, kc0 + k, b, dch, act, tg);
 
     // ---- per (channel, step): Δ, Δx, gate; index j: steps 2tg, 2tg+1, 2tg+8, 2tg+9
     float dl[2][4], xv[2][4], gt[2][4], uv[2][4];
@@ -218,7 +222,8 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
         const float D = a.softplus ? softplus_fast(v) : v;
         dl[c][j] = live ? D : 0.f;
         uv[c][j] = live ? u : 0.f;
-        xv[c][j] = (a.zoh ? zoh_c(dl[c][j], al[c] * kLn2) : dl[c][j]) * uv[c][j];
+        if constexpr (ZOH) xv[c][j] = zoh_c(dl[c][j], al[c] * kLn2) * uv[c][j];
+        else xv[c][j] = dl[c][j] * uv[c][j];
         if (zp && !NOOUT) {
           const float z = (j & 1) ? bf16_hi(wz) : bf16_lo(wz);
           gt[c][j] = z * sigmoid_fast(z);
@@ -324,7 +329,7 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
       }
       mma16816(Ht[nt], x2[0], x2[1], x2[2], x2[3], bn[0], bn[1]);
       mma16816(Ht[nt + 1], x2[0], x2[1], x2[2], x2[3], bn[2], bn[3]);
-      if (exact) {  // states that a backward or a chain reads: the remainder term too
+      if constexpr (EXACT) {  // states that a backward or a chain reads: the remainder term too
         mma16816(Ht[nt], x2l[0], x2l[1], x2l[2], x2l[3], bn[0], bn[1]);
         mma16816(Ht[nt + 1], x2l[0], x2l[1], x2l[2], x2l[3], bn[2], bn[3]);
       }
@@ -438,9 +443,15 @@ cudaError_t launch_n(const FwdArgs& a, int mode, cudaStream_t s) {
   if (segs <= 0) return cudaSuccess;
   const dim3 grid((unsigned)((long long)a.batch * ((a.dim + 16 * W - 1) / (16 * W))), (unsigned)segs);
   const size_t smem = kStages * sizeof(SsdStage<N>);
-  auto k = mode == kSsdSummary ? ssd_fwd_kernel<N, W, kSsdSummary>
-                               : (mode == kSsdCkpt ? ssd_fwd_kernel<N, W, kSsdCkpt>
-                                                   : ssd_fwd_kernel<N, W, kSsdOut>);
+  if (mode == kSsdOut && a.ckpt) mode = kSsdOutCkpt;
+  const auto pick = [&](auto zoh) {
+    constexpr bool Z = decltype(zoh)::value;
+    return mode == kSsdSummary ? ssd_fwd_kernel<N, W, kSsdSummary, Z>
+         : mode == kSsdCkpt    ? ssd_fwd_kernel<N, W, kSsdCkpt, Z>
+         : mode == kSsdOutCkpt ? ssd_fwd_kernel<N, W, kSsdOutCkpt, Z>
+                               : ssd_fwd_kernel<N, W, kSsdOut, Z>;
+  };
+  auto k = a.zoh ? pick(std::true_type()) : pick(std::false_type());
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   k<<<grid, 32 * W, smem, s>>>(a);

@@ -116,7 +116,7 @@ __device__ __forceinline__ void carry_mu(float4* mus, const SsdStage<N>& st, int
 // the order the segment chain composes them).  Otherwise blockIdx.y is the segment, which starts
 // from μ = a.mu_in[nseg - 1 - seg] (the chained adjoint; dhL for the last segment, or dhL
 // itself without a split).
-template <int N, bool SUMM>
+template <int N, bool SUMM, bool ZOH>
 __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant__ SsdBwdArgs a) {
   constexpr int kNT = N / 8;
   extern __shared__ float4 smem_sb[];
@@ -265,7 +265,8 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
         const float D = a.softplus ? softplus_fast(v) : v;
         dl[c][j] = live ? D : 0.f;
         // x' = c u with c = Δ, or the zero-order-hold coefficient (e^{ΔA} - 1)/A
-        xv[c][j] = live ? (a.zoh ? zoh_c(D, al[c] * kLn2) : D) * u : 0.f;
+        if constexpr (ZOH) xv[c][j] = live ? zoh_c(D, al[c] * kLn2) * u : 0.f;
+        else xv[c][j] = live ? D * u : 0.f;
         const float go = live ? pick(cur.go[c][hh], od) : 0.f;
         if (a.z) {
           const float z = pick(cur.z[c][hh], od);
@@ -675,12 +676,13 @@ __global__ void __launch_bounds__(32 * kWb) ssd_bwd_kernel(const __grid_constant
           const float u = live ? pick(cur.u[c][hh], od) : 0.f;
           const float sg = a.softplus ? sigmoid_fast(pick(cur.dl[c][hh], od) + bias[c]) : 1.f;
           // the input coefficient c_t (Δ_t, or the zero-order hold's) and its derivatives
-          float cz = dl[c][j], dcdd = 1.f, dcda = 0.f;
-          if (a.zoh && live) {
-            cz = zoh_c(dl[c][j], A);
-            dcdd = expf(dl[c][j] * A);
-            dcda = zoh_dc_da(dl[c][j], A, cz);
-            accA[c] = fmaf(dxp[c][j] * u, dcda, accA[c]);  // through c's rate
+          float cz = dl[c][j], dcdd = 1.f;
+          if constexpr (ZOH) {
+            if (live) {
+              cz = zoh_c(dl[c][j], A);
+              dcdd = expf(dl[c][j] * A);
+              accA[c] = fmaf(dxp[c][j] * u, zoh_dc_da(dl[c][j], A, cz), accA[c]);  // c's rate
+            }
           }
           const float dD = fmaf(A, dS[c][j], dxp[c][j] * u * dcdd);  // dL/dΔ_t
           vdd[od] = dD * sg;                                           // through softplus (dΔ/dv = σ(v))
@@ -844,13 +846,13 @@ __global__ void ssd_finish_adt(const SsdBwdArgs a, float* dA, float* dD, float* 
   if (ddt_bias) ddt_bias[d] = s[2];
 }
 
-template <int N, bool SUMM>
+template <int N, bool SUMM, bool ZOH>
 cudaError_t launch_n(const SsdBwdArgs& a, cudaStream_t s) {
   const dim3 grid((unsigned)((long long)a.batch * ((a.dim + 16 * kWb - 1) / (16 * kWb))),
                   (unsigned)(SUMM ? a.nseg - 1 : a.nseg));
   if (grid.y == 0) return cudaSuccess;
   const size_t smem = sizeof(BwdSmem<N>);
-  auto k = ssd_bwd_kernel<N, SUMM>;
+  auto k = ssd_bwd_kernel<N, SUMM, ZOH>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   k<<<grid, 32 * kWb, smem, s>>>(a);
@@ -861,12 +863,19 @@ cudaError_t launch_n(const SsdBwdArgs& a, cudaStream_t s) {
 
 int ssd_bwd_ctas_per_row(int dim) { return (dim + 16 * kWb - 1) / (16 * kWb); }
 
+// The summary needs no input coefficient (it carries only the adjoint), so it has no ZOH form.
+template <int N>
+cudaError_t launch_nz(const SsdBwdArgs& a, bool summary, cudaStream_t s) {
+  if (summary) return launch_n<N, true, false>(a, s);
+  return a.zoh ? launch_n<N, false, true>(a, s) : launch_n<N, false, false>(a, s);
+}
+
 cudaError_t launch_ssd_bwd(const SsdBwdArgs& a, bool summary, cudaStream_t s) {
   switch (a.N) {
-    case 16: return summary ? launch_n<16, true>(a, s) : launch_n<16, false>(a, s);
-    case 32: return summary ? launch_n<32, true>(a, s) : launch_n<32, false>(a, s);
-    case 64: return summary ? launch_n<64, true>(a, s) : launch_n<64, false>(a, s);
-    case 128: return summary ? launch_n<128, true>(a, s) : launch_n<128, false>(a, s);
+    case 16: return launch_nz<16>(a, summary, s);
+    case 32: return launch_nz<32>(a, summary, s);
+    case 64: return launch_nz<64>(a, summary, s);
+    case 128: return launch_nz<128>(a, summary, s);
     default: return cudaErrorInvalidValue;
   }
 }
