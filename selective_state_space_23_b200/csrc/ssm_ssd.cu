@@ -71,22 +71,49 @@ __device__ __forceinline__ uint32_t ld_pair(const uint16_t* p, long long t, int 
   return lo | (hi << 16);
 }
 
-// The state entering chunk `slot` (transposed accumulator layout: 2 channels x N/4 states per
-// lane) into the checkpoint array, f32 [batch][dim][ceil(L / 16)][N]: the layout of the
-// per-state scan's checkpoints, which hold the same states (the state entering every 16-step
-// block), so either forward's checkpoints serve either backward.
+// The state entering chunk `slot` of the warp's 16 channels (transposed accumulator layout: 2
+// channels x N/4 states per lane) into the checkpoint array, f32 [batch][dim][ceil(L / 16)][N]:
+// the layout of the per-state scan's checkpoints, which hold the same states (the state
+// entering every 16-step block), so either forward's checkpoints serve either backward.
+// kStageCkpt<N>: the lanes' pairs go through the warp's staging tile (rows of N + 8 floats:
+// conflict-free 64-bit writes and 128-bit reads), so that each channel's row leaves as whole
+// 16-byte pieces of consecutive lanes rather than 8-byte pieces of 16 rows per store (1 x 256 x
+// 2^20, N = 64: the backward's checkpoint pass 2 ms faster).  At N = 128 the tile would cost the
+// kernel a resident CTA per SM, and the pairs are stored directly.
+template <int N>
+constexpr bool kStageCkpt = N <= 64;
+
 template <int N>
 __device__ __forceinline__ void store_state(const FwdArgs& a, const float (&Ht)[N / 8][4],
-                                            int slot, int b, const int (&dch)[2],
-                                            const bool (&act)[2], int tg) {
+                                            float* stage, int slot, int b, int dw, int lane) {
+  constexpr int LD = N + 8;
+  const int g = lane >> 2, tg = lane & 3;
   const long long nslots = (a.L + kT - 1) / kT;
+  if constexpr (!kStageCkpt<N>) {
 #pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    if (!act[c]) continue;
-    float* row = a.ckpt + (((long long)b * a.dim + dch[c]) * nslots + slot) * N + 2 * tg;
+    for (int c = 0; c < 2; ++c) {
+      if (dw + g + 8 * c >= a.dim) continue;
+      float* row = a.ckpt + (((long long)b * a.dim + dw + g + 8 * c) * nslots + slot) * N + 2 * tg;
+#pragma unroll
+      for (int nt = 0; nt < N / 8; ++nt)
+        *reinterpret_cast<float2*>(row + 8 * nt) = make_float2(Ht[nt][2 * c], Ht[nt][2 * c + 1]);
+    }
+    return;
+  }
+  __syncwarp();  // the previous chunk's rows have left the tile
+#pragma unroll
+  for (int c = 0; c < 2; ++c)
 #pragma unroll
     for (int nt = 0; nt < N / 8; ++nt)
-      *reinterpret_cast<float2*>(row + 8 * nt) = make_float2(Ht[nt][2 * c], Ht[nt][2 * c + 1]);
+      *reinterpret_cast<float2*>(stage + (g + 8 * c) * LD + 8 * nt + 2 * tg) =
+          make_float2(Ht[nt][2 * c], Ht[nt][2 * c + 1]);
+  __syncwarp();
+#pragma unroll
+  for (int i = lane; i < 16 * (N / 4); i += 32) {
+    const int r = i / (N / 4), q = i % (N / 4);
+    if (dw + r < a.dim)
+      *reinterpret_cast<float4*>(a.ckpt + (((long long)b * a.dim + dw + r) * nslots + slot) * N + 4 * q) =
+          *reinterpret_cast<const float4*>(stage + r * LD + 4 * q);
   }
 }
 
@@ -105,6 +132,9 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
   extern __shared__ float4 smem_ssd[];
   SsdStage<N>* ring = reinterpret_cast<SsdStage<N>*>(smem_ssd);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // checkpoint modes: the warp's staging tile of 16 rows after the ring
+  float* stage = reinterpret_cast<float*>(ring + kStages) +
+                 ((CKPT && kStageCkpt<N>) ? warp * 16 * (N + 8) : 0);
   const int g = lane >> 2, tg = lane & 3;
   const int tiles_d = (a.dim + 16 * W - 1) / (16 * W);
   const int b = blockIdx.x / tiles_d;
@@ -206,7 +236,7 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
     if (k + 1 < nchunk) load_in(k + 1, nxt);
     const SsdStage<N>& st = ring[k % kStages];
     const int t0 = (kc0 + k) * kT;
-    if (CKPT) store_state<N>(a, Ht, kc0 + k, b, dch, act, tg);
+    if (CKPT) store_state<N>(a, Ht, stage, kc0 + k, b, d0 + 16 * warp, lane);
 
     // ---- per (channel, step): Δ, Δx, gate; index j: steps 2tg, 2tg+1, 2tg+8, 2tg+9
     float dl[2][4], xv[2][4], gt[2][4], uv[2][4];
@@ -442,8 +472,10 @@ cudaError_t launch_n(const FwdArgs& a, int mode, cudaStream_t s) {
   const int segs = mode == kSsdSummary ? a.nchunk - 1 : a.nchunk;  // the last summary is unused
   if (segs <= 0) return cudaSuccess;
   const dim3 grid((unsigned)((long long)a.batch * ((a.dim + 16 * W - 1) / (16 * W))), (unsigned)segs);
-  const size_t smem = kStages * sizeof(SsdStage<N>);
   if (mode == kSsdOut && a.ckpt) mode = kSsdOutCkpt;
+  const size_t smem =
+      kStages * sizeof(SsdStage<N>) +
+      ((kStageCkpt<N> && (mode == kSsdCkpt || mode == kSsdOutCkpt)) ? (size_t)W * 16 * (N + 8) * 4 : 0);
   const auto pick = [&](auto zoh) {
     constexpr bool Z = decltype(zoh)::value;
     return mode == kSsdSummary ? ssd_fwd_kernel<N, W, kSsdSummary, Z>
