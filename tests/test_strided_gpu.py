@@ -137,3 +137,31 @@ def test_overlapping_output_is_refused():
     with pytest.raises(RuntimeError, match="one address"):
         ssm.ssm_scan_fwd_strided(xd["u"], xd["delta"], xd["A"], xd["B"], xd["C"],
                                  out=one.expand(2, -1, -1))
+
+
+
+@pytest.mark.parametrize("N", [64, 128])
+@pytest.mark.parametrize("reverse", [False, True])
+def test_large_n_chunked_form_takes_strided_views(N, reverse):
+    """Scalar decay with 64 or 128 states (the chunked matrix form) from the views a Mamba-2
+    block holds: the projection halves, a (B, L, D) gate, strided B, C.  Forward and backward
+    equal the dense calls bitwise."""
+    w = workload("mamba2p8b_train", batch=2, dim=128, seqlen=160, dstate=N)
+    x = make_inputs(w, seed=84, with_dout=True, with_h0=True, scalar_a=True)
+    s = strided_copies(x, seed=3)
+    xd = {k: v.to(DEV) for k, v in x.items()}
+    kw = dict(scalar_a=True, reverse=reverse)
+    out, hL = ssm.ssm_scan_fwd_strided(s["u"], s["delta"], s["A"], s["B"], s["C"], D=s["D"],
+                                       z=s["z"], dt_bias=s["dt_bias"], h0=s["h0"],
+                                       return_final_state=True, **kw)
+    ref, hL_ref = ssm.ssm_scan_fwd_scalar_a(xd["u"], xd["delta"], xd["A"], xd["B"], xd["C"],
+                                            D=xd["D"], z=xd["z"], dt_bias=xd["dt_bias"],
+                                            h0=xd["h0"], return_final_state=True, reverse=reverse)
+    assert torch.equal(out, ref) and torch.equal(hL, hL_ref)
+    g = ssm.ssm_scan_bwd_strided(s["u"], s["delta"], s["A"], s["B"], s["C"], s["dout"], D=s["D"],
+                                 z=s["z"], dt_bias=s["dt_bias"], h0=s["h0"], **kw)
+    r = ssm.ssm_scan_bwd_scalar_a(xd["u"], xd["delta"], xd["A"], xd["B"], xd["C"], xd["dout"],
+                                  D=xd["D"], z=xd["z"], dt_bias=xd["dt_bias"], h0=xd["h0"],
+                                  reverse=reverse)
+    for k in ("du", "ddelta", "dz", "dB", "dC", "dA", "dD", "ddt_bias", "dh0"):
+        assert torch.equal(g[k], r[k]), k
