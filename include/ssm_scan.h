@@ -162,8 +162,13 @@ SSM_API int ssm_scan_bwd(const void* u, const void* delta, const float* A, const
  * the step-scaled inputs, plus C times the entering state: the structured-matrix view of the
  * scan in the Mamba-2 notes of the same page) on the tensor cores.  That form takes bf16 io,
  * dstate 16, 32, 64 or 128, the default layout and B/C groups of whole 64-channel tiles (with
- * SSM_ZOH: the coefficient (e^{ΔA} - 1)/A by the library expm1f); other forward requests with
- * dstate > 16 return SSM_EUNSUPPORTED.  With SSM_REVERSE
+ * SSM_ZOH: the coefficient (e^{ΔA} - 1)/A by the library expm1f).  f32 io with dstate a
+ * multiple of 16 up to 128 (default layout, B/C shared or grouped) runs as the sum of the f32
+ * 16-state forwards of the state slices: the first slice (with D) writes out, each further
+ * slice's gated output is added to it in f32, and hL and ckpt are written slice by slice; its
+ * workspace (ssm_scan_fwd_ex_workspace_size) holds the slice copies of B, C, h0, one slice's
+ * hL, checkpoints and output, and the 16-state forward's own workspace.  Other forward requests
+ * with dstate > 16 return SSM_EUNSUPPORTED.  With SSM_REVERSE
  * (dstate > 16; ssm_scan_fwd_ex) it scans the inputs mirrored along time into the workspace
  * and mirrors the output back in place, so ssm_scan_fwd_ex_workspace_size() then covers those
  * copies (u, delta, z, B, C) too.  Its checkpoints (ckpt, 16-byte aligned) have the layout and meaning of the

@@ -416,12 +416,17 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
                          !(flags & (SSM_ZOH | SSM_REVERSE | SSM_CHANNELS_LAST)) &&
                          (bc_groups == 1 || (dim % bc_groups == 0 && (dim / bc_groups) % 64 == 0)) &&
                          !(sform && strcmp(sform, "state") == 0);
+  // f32 io with N > 16: the sum of 16-state f32 forwards over the state slices (ssm_slices.cu)
+  if (dstate > SSM_MAX_DSTATE && io_dtype == SSM_F32)
+    return ssm::scan_fwd_slices(u, delta, A, B, C, D, z, dt_bias, delta_softplus, h0, hL, out,
+                                ckpt, workspace, workspace_bytes, batch, dim, seqlen, dstate,
+                                bc_groups, io_dtype, flags, stream);
   if (dstate > SSM_MAX_DSTATE || chunked16) {
     if (io_dtype != SSM_BF16 || (dstate != 16 && dstate != 32 && dstate != 64 && dstate != 128) ||
         channels_last ||
         !(bc_groups == 1 || (dim % bc_groups == 0 && (dim / bc_groups) % 64 == 0)))
       return fail(SSM_EUNSUPPORTED,
-                  "scalar decay with dstate %d > %d needs bf16 io, dstate 32, 64 or 128, the "
+                  "scalar decay with dstate %d > %d needs bf16 or f32 io, dstate 32, 64 or 128, the "
                   "default layout and B/C groups of whole 64-channel tiles", dstate,
                   SSM_MAX_DSTATE);
     if (!aligned16(ckpt))
@@ -661,6 +666,8 @@ int ssm_scan_fwd(const void* u, const void* delta, const float* A, const void* B
 size_t ssm_scan_fwd_ex_workspace_size(int batch, int dim, int seqlen, int dstate, int bc_groups,
                                       int io_dtype, int flags) {
   if (bc_groups < 1) return 0;
+  if ((flags & SSM_SCALAR_A) && dstate > SSM_MAX_DSTATE && io_dtype == SSM_F32)  // 16-state slices
+    return ssm::scan_fwd_slices_workspace(batch, dim, seqlen, dstate, bc_groups, io_dtype, flags);
   if ((flags & SSM_SCALAR_A) && dstate > SSM_MAX_DSTATE) {  // the chunked matrix form's segments
     if (check_dims(batch, dim, seqlen, dstate, io_dtype, SSM_MAX_DSTATE_SCALAR) != SSM_OK) return 0;
     return plan_ssd(batch, dim, seqlen, dstate).ws_bytes +
@@ -681,7 +688,7 @@ int ssm_scan_fwd_ex(const void* u, const void* delta, const float* A, const void
 
 size_t ssm_scan_fwd_scalar_a_workspace_size(int batch, int dim, int seqlen, int dstate,
                                             int io_dtype) {
-  return ssm_scan_fwd_workspace_size(batch, dim, seqlen, dstate, io_dtype);
+  return ssm_scan_fwd_ex_workspace_size(batch, dim, seqlen, dstate, 1, io_dtype, SSM_SCALAR_A);
 }
 
 int ssm_scan_fwd_scalar_a(const void* u, const void* delta, const float* A, const void* B,

@@ -207,6 +207,15 @@ cudaError_t copy_view(const void* src, const long long* n, const long long* ss, 
 cudaError_t mirror_rows(const void* src, void* dst, long long rows, int L, cudaStream_t s);
 // Backward of the scalar-decay scan for dstate = 16 k (k = 2, 4, 8) as the sum of k 16-state
 // backwards (ssm_slices.cu); arguments as ssm_scan_bwd_ex.
+// The f32 forward of the scalar-decay scan for dstate = 16 k as the sum of k 16-state forwards
+// (ssm_slices.cu); arguments as ssm_scan_fwd_ex.
+size_t scan_fwd_slices_workspace(int batch, int dim, int seqlen, int dstate, int bc_groups,
+                                 int io_dtype, int flags);
+int scan_fwd_slices(const void* u, const void* delta, const float* A, const void* B,
+                    const void* C, const float* D, const void* z, const float* dt_bias,
+                    int delta_softplus, const float* h0, float* hL, void* out, float* ckpt,
+                    void* workspace, size_t workspace_bytes, int batch, int dim, int seqlen,
+                    int dstate, int bc_groups, int io_dtype, int flags, void* stream);
 size_t scan_bwd_slices_workspace(int batch, int dim, int seqlen, int dstate, int bc_groups,
                                  int io_dtype, int flags);
 int scan_bwd_slices(const void* u, const void* delta, const float* A, const void* B,

@@ -13,7 +13,12 @@
 // So the backward runs the library's 16-state backward once per slice (B, C, h0, dhL gathered
 // into dense slices by the view copy kernel), accumulates du, ddelta, dz, dA, ddt_bias in f32,
 // and scatters dB, dC, dh0 back.  It costs k times the 16-state backward: the compatibility path
-// for training with N > 16 (the forward runs the chunked matrix form, ssm_ssd.cu).
+// for training with N > 16 (bf16 runs the chunked matrix form, ssm_ssd.cu, ssm_ssd_bwd.cu).
+//
+// The forward in f32 io (which the chunked form, a bf16 tensor-core form, does not take) is the
+// same sum: the gate multiplies the whole readout, so out = Σ_slices (y_slice + [first] D x)
+// silu(z) is each slice's gated output summed in f32; hL and the checkpoints are disjoint per
+// slice.  The first slice writes the output and each further one adds its own (f32).
 #include <cuda_runtime.h>
 #include <stdio.h>
 #include <string.h>
@@ -118,7 +123,123 @@ int fail(int code, const char* msg) {
   return code;
 }
 
+// Workspace layout of the slice forward (byte offsets).
+struct FwdSliceLayout {
+  size_t bj, cj, h0j, hlj, ckj, oj, inner, inner_bytes, total;
+};
+
+FwdSliceLayout fwd_slice_layout(int batch, int dim, int seqlen, int bc_groups, int io_dtype,
+                                int flags) {
+  const size_t es = io_dtype == SSM_BF16 ? 2 : 4;
+  const size_t nblk = (seqlen + kBlk - 1) / kBlk;
+  FwdSliceLayout l;
+  size_t o = 0;
+  l.bj = o; o += align256((size_t)batch * bc_groups * kNS * seqlen * es);
+  l.cj = o; o += align256((size_t)batch * bc_groups * kNS * seqlen * es);
+  l.h0j = o; o += align256((size_t)batch * dim * kNS * 4);
+  l.hlj = o; o += align256((size_t)batch * dim * kNS * 4);
+  l.ckj = o; o += align256((size_t)batch * dim * nblk * kNS * 4);
+  l.oj = o; o += align256((size_t)batch * dim * seqlen * es);
+  l.inner = o;
+  l.inner_bytes = align256(ssm_scan_fwd_ex_workspace_size(batch, dim, seqlen, kNS, bc_groups,
+                                                          io_dtype, flags));
+  l.total = o + l.inner_bytes;
+  return l;
+}
+
 }  // namespace
+
+size_t scan_fwd_slices_workspace(int batch, int dim, int seqlen, int dstate, int bc_groups,
+                                 int io_dtype, int flags) {
+  if (dstate % kNS != 0 || dstate > SSM_MAX_DSTATE_SCALAR || !(flags & SSM_SCALAR_A) ||
+      (flags & SSM_CHANNELS_LAST) || batch <= 0 || dim <= 0 || seqlen <= 0 || bc_groups < 1 ||
+      io_dtype != SSM_F32)
+    return 0;
+  return fwd_slice_layout(batch, dim, seqlen, bc_groups, io_dtype, flags).total;
+}
+
+int scan_fwd_slices(const void* u, const void* delta, const float* A, const void* B,
+                    const void* C, const float* D, const void* z, const float* dt_bias,
+                    int delta_softplus, const float* h0, float* hL, void* out, float* ckpt,
+                    void* workspace, size_t workspace_bytes, int batch, int dim, int seqlen,
+                    int dstate, int bc_groups, int io_dtype, int flags, void* stream) {
+  if (dstate % kNS != 0 || dstate > SSM_MAX_DSTATE_SCALAR)
+    return fail(SSM_EUNSUPPORTED, "scalar-decay f32 forward with dstate > 16 needs a multiple of 16 "
+                                  "up to 128");
+  if (flags & SSM_CHANNELS_LAST)
+    return fail(SSM_EUNSUPPORTED, "scalar-decay forward with dstate > 16 takes the default layout");
+  if (bc_groups == dim && bc_groups > 1)
+    return fail(SSM_EUNSUPPORTED, "scalar-decay forward with dstate > 16 takes shared or grouped B/C");
+  const size_t need = scan_fwd_slices_workspace(batch, dim, seqlen, dstate, bc_groups, io_dtype, flags);
+  if (need == 0) return fail(SSM_EINVAL, "invalid sizes, groups or io_dtype");
+  if (!workspace || workspace_bytes < need) {
+    char msg[128];
+    snprintf(msg, sizeof(msg), "workspace of %zu bytes given, %zu needed", workspace_bytes, need);
+    return fail(SSM_EWORKSPACE, msg);
+  }
+  if (reinterpret_cast<uintptr_t>(workspace) & 255)
+    return fail(SSM_EINVAL, "workspace is not 256-byte aligned");
+  int rc = check_device_ptr(workspace, need, 256, "workspace");
+  if (rc != SSM_OK) return rc;
+  const size_t es = 4;
+  const size_t N = (size_t)dstate;
+  const long long nbc = (long long)bc_groups * dstate * seqlen;
+  const long long nblk = (seqlen + kBlk - 1) / kBlk;
+  if ((rc = check_device_ptr(B, (size_t)batch * nbc * es, es, "B")) != SSM_OK) return rc;
+  if ((rc = check_device_ptr(C, (size_t)batch * nbc * es, es, "C")) != SSM_OK) return rc;
+  if ((rc = check_device_ptr(out, (size_t)batch * dim * seqlen * es, es, "out")) != SSM_OK) return rc;
+  const size_t nst = (size_t)batch * dim * N * 4;
+  if (h0 && (rc = check_device_ptr(h0, nst, 4, "h0")) != SSM_OK) return rc;
+  if (hL && (rc = check_device_ptr(hL, nst, 4, "hL")) != SSM_OK) return rc;
+  if (ckpt && (rc = check_device_ptr(ckpt, (size_t)batch * dim * nblk * N * 4, 4, "ckpt")) != SSM_OK)
+    return rc;
+
+  const FwdSliceLayout l = fwd_slice_layout(batch, dim, seqlen, bc_groups, io_dtype, flags);
+  char* w = reinterpret_cast<char*>(workspace);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long long nx = (long long)batch * dim * seqlen;
+  const int k = dstate / kNS;
+  const long long n_bc[4] = {batch, bc_groups, kNS, seqlen};
+  const long long s_bc[4] = {(long long)bc_groups * dstate * seqlen, (long long)dstate * seqlen, seqlen, 1};
+  const long long d_bc[4] = {(long long)bc_groups * kNS * seqlen, (long long)kNS * seqlen, seqlen, 1};
+  const long long n_st[4] = {1, batch, dim, kNS};
+  const long long s_st[4] = {0, (long long)dim * dstate, dstate, 1};
+  const long long d_st[4] = {0, (long long)dim * kNS, kNS, 1};
+  // a slice of the checkpoints [batch][dim][blocks][N]
+  const long long n_ck[4] = {batch, dim, nblk, kNS};
+  const long long s_ck[4] = {(long long)dim * nblk * dstate, (long long)nblk * dstate, dstate, 1};
+  const long long d_ck[4] = {(long long)dim * nblk * kNS, (long long)nblk * kNS, kNS, 1};
+  cudaError_t e = cudaSuccess;
+#define CK(x)                                         \
+  do {                                                \
+    if ((e = (x)) != cudaSuccess) {                   \
+      set_last_error(cudaGetErrorString(e));          \
+      return SSM_ECUDA;                               \
+    }                                                 \
+  } while (0)
+  for (int j = 0; j < k; ++j) {
+    const size_t off = (size_t)j * kNS;
+    void* Bj = w + l.bj;
+    void* Cj = w + l.cj;
+    CK(copy_view(reinterpret_cast<const char*>(B) + off * seqlen * es, n_bc, s_bc, Bj, d_bc, es, s));
+    CK(copy_view(reinterpret_cast<const char*>(C) + off * seqlen * es, n_bc, s_bc, Cj, d_bc, es, s));
+    float* h0j = h0 ? reinterpret_cast<float*>(w + l.h0j) : nullptr;
+    if (h0j) CK(copy_view(h0 + off, n_st, s_st, h0j, d_st, 4, s));
+    float* hLj = hL ? reinterpret_cast<float*>(w + l.hlj) : nullptr;
+    float* ckj = ckpt ? reinterpret_cast<float*>(w + l.ckj) : nullptr;
+    // the first slice (with D) writes out; the others add theirs to it
+    void* oj = j == 0 ? out : w + l.oj;
+    rc = ssm_scan_fwd_ex(u, delta, A, Bj, Cj, j == 0 ? D : nullptr, z, dt_bias, delta_softplus,
+                         h0j, hLj, oj, ckj, w + l.inner, l.inner_bytes, batch, dim, seqlen, kNS,
+                         bc_groups, io_dtype, flags, stream);
+    if (rc != SSM_OK) return rc;
+    if (j > 0) CK(accumulate(oj, reinterpret_cast<float*>(out), nx, false, es, s));
+    if (hLj) CK(copy_view(hLj, n_st, d_st, hL + off, s_st, 4, s));
+    if (ckj) CK(copy_view(ckj, n_ck, d_ck, ckpt + off, s_ck, 4, s));
+  }
+#undef CK
+  return SSM_OK;
+}
 
 size_t scan_bwd_slices_workspace(int batch, int dim, int seqlen, int dstate, int bc_groups,
                                  int io_dtype, int flags) {

@@ -152,6 +152,8 @@ FWD_CASES = {
     "chunked_n128_split": ({"SSM_SSD_SPLIT": "3"}, 1, 80, 333, 128, torch.bfloat16, 1, 1),
     "chunked_n64_reverse": ({}, 1, 80, 333, 64, torch.bfloat16, 1, 1 | 2),
     "chunked_n64_zoh": ({}, 1, 80, 333, 64, torch.bfloat16, 1, 1 | 4),
+    "slices_f32_n64": ({}, 2, 40, 37, 64, torch.float32, 1, 1),
+    "slices_f32_n32_reverse_zoh_grouped": ({}, 2, 64, 120, 32, torch.float32, 2, 1 | 2 | 4),
 }
 
 

@@ -140,13 +140,14 @@ def test_overlapping_output_is_refused():
 
 
 
+@pytest.mark.parametrize("io", [torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("N", [64, 128])
 @pytest.mark.parametrize("reverse", [False, True])
-def test_large_n_chunked_form_takes_strided_views(N, reverse):
-    """Scalar decay with 64 or 128 states (the chunked matrix form) from the views a Mamba-2
-    block holds: the projection halves, a (B, L, D) gate, strided B, C.  Forward and backward
-    equal the dense calls bitwise."""
-    w = workload("mamba2p8b_train", batch=2, dim=128, seqlen=160, dstate=N)
+def test_large_n_chunked_form_takes_strided_views(io, N, reverse):
+    """Scalar decay with 64 or 128 states (the chunked matrix form in bf16, the 16-state slices
+    in f32) from the views a Mamba-2 block holds: the projection halves, a (B, L, D) gate,
+    strided B, C.  Forward and backward equal the dense calls bitwise."""
+    w = workload("mamba2p8b_train", batch=2, dim=128, seqlen=160, dstate=N, io_dtype=io)
     x = make_inputs(w, seed=84, with_dout=True, with_h0=True, scalar_a=True)
     s = strided_copies(x, seed=3)
     xd = {k: v.to(DEV) for k, v in x.items()}
