@@ -364,11 +364,15 @@ SSM_API int ssm_wait_timeouts(unsigned int* count);
  *     hend  [batch][dim][dstate] f32   OUT: the state after the segment from a zero state
  *     dsum  [batch][dim] f32 or NULL   OUT: ΣΔ over the segment (Kahan-summed in f32)
  *   and ssm_scan_fwd_summary_workspace_size() bytes of workspace (256-byte aligned).
+ *   With SSM_SCALAR_A, dstate may exceed 16 as in the scalar-decay scan: bf16 with dstate 32,
+ *   64 or 128 and B/C shared or in groups of whole 64-channel tiles runs the chunked matrix
+ *   form's summary pass over the planner's segments and chains them; f32 with dstate a multiple
+ *   of 16 up to 128 sums 16-state slices (C is not read then).
  * ssm_scan_chain: the state entering each of nseg consecutive segments,
  *     hin[0] = h0 (zero if NULL),  hin[r+1] = exp(A dsum[r]) hin[r] + hend[r],
  *   hend, hin [nseg][batch][dim][dstate] f32, dsum [nseg][batch][dim] f32, A as for the scan
- *   (flags: SSM_SCALAR_A).  Running each segment's forward scan from its hin[r] gives the
- *   full-sequence results, up to rounding.
+ *   (flags: SSM_SCALAR_A, which allows dstate up to SSM_MAX_DSTATE_SCALAR).  Running each
+ *   segment's forward scan from its hin[r] gives the full-sequence results, up to rounding.
  * Errors as for the scans.
  */
 SSM_API size_t ssm_scan_fwd_summary_workspace_size(int batch, int dim, int seqlen, int dstate,

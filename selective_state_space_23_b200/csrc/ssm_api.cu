@@ -582,6 +582,89 @@ int scan_fwd_impl(const void* u, const void* delta, const float* A, const void* 
 
 // Time chunks of a whole-sequence summary and its scratch: the forward's plan with one more
 // chunk slot (summaries, entering states, ΣΔ).
+// Sequence summary of a scalar-decay scan with N = 32, 64 or 128 in bf16: the chunked matrix
+// form's summary pass over every one of the planner's S segments (each from a zero state), the
+// chain of the S segment maps from zero (its (S+1)-th entering state is the sequence's end
+// state), and the finishing kernel.  Workspace: per-segment end states [S][batch*dim][N],
+// entering states [S+1][batch*dim][N], per-segment ΣΔ [S][batch*dim].
+struct SummaryChunkedLayout {
+  FwdPlan plan;
+  size_t summ, hin, ds, total;
+};
+
+SummaryChunkedLayout summary_chunked_layout(int batch, int dim, int seqlen, int dstate) {
+  SummaryChunkedLayout l;
+  l.plan = plan_ssd(batch, dim, seqlen, dstate);
+  const size_t nch = (size_t)batch * dim, S = (size_t)l.plan.nchunk;
+  l.summ = 0;
+  l.hin = align_up(S * nch * dstate * 4);
+  l.ds = l.hin + align_up((S + 1) * nch * dstate * 4);
+  l.total = l.ds + align_up(S * nch * 4);
+  return l;
+}
+
+__global__ void summary_finish_kernel(const float* __restrict__ hin_end, int hs,
+                                      const float* __restrict__ dsum, int S, long long nch, int N,
+                                      float* __restrict__ hend, float* __restrict__ dsum_out);
+
+int summary_chunked(const void* u, const void* delta, const float* A, const void* B,
+                    const void* C, const float* dt_bias, int delta_softplus, float* hend,
+                    float* dsum, void* workspace, size_t workspace_bytes, int batch, int dim,
+                    int seqlen, int dstate, int bc_groups, int flags, void* stream) {
+  if (dstate != 32 && dstate != 64 && dstate != 128)
+    return fail(SSM_EUNSUPPORTED, "a bf16 sequence summary with dstate %d > %d takes 32, 64 or 128",
+                dstate, SSM_MAX_DSTATE);
+  if (!(bc_groups == 1 || (dim % bc_groups == 0 && (dim / bc_groups) % 64 == 0)))
+    return fail(SSM_EUNSUPPORTED, "a bf16 sequence summary with dstate > %d takes B/C shared or in "
+                "groups of whole 64-channel tiles", SSM_MAX_DSTATE);
+  const size_t es = 2;
+  const size_t nx = (size_t)batch * dim * seqlen * es;
+  const size_t nbc = (size_t)batch * bc_groups * dstate * seqlen * es;
+  const size_t nch = (size_t)batch * dim;
+  TRY(check_ptr(u, nx, es, "u"));
+  TRY(check_ptr(delta, nx, es, "delta"));
+  TRY(check_ptr(A, (size_t)dim * 4, 4, "A"));
+  TRY(check_ptr(B, nbc, es, "B"));
+  TRY(check_ptr(C, nbc, es, "C"));
+  TRY(check_opt(dt_bias, (size_t)dim * 4, 4, "dt_bias"));
+  TRY(check_ptr(hend, nch * dstate * 4, 4, "hend"));
+  TRY(check_opt(dsum, nch * 4, 4, "dsum"));
+  const SummaryChunkedLayout l = summary_chunked_layout(batch, dim, seqlen, dstate);
+  if (!workspace || workspace_bytes < l.total)
+    return fail(SSM_EWORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes, l.total);
+  if (reinterpret_cast<uintptr_t>(workspace) & 255)
+    return fail(SSM_EINVAL, "workspace is not 256-byte aligned");
+  TRY(check_ptr(workspace, l.total, 256, "workspace"));
+  char* w = reinterpret_cast<char*>(workspace);
+  const int S = l.plan.nchunk;
+  ssm::FwdArgs a;
+  memset(&a, 0, sizeof(a));
+  a.u = u; a.delta = delta; a.B = B; a.C = C; a.A = A; a.dt_bias = dt_bias;
+  a.summ = reinterpret_cast<float*>(w + l.summ);
+  a.dsum = reinterpret_cast<float*>(w + l.ds);
+  a.batch = batch; a.dim = dim; a.L = seqlen; a.N = dstate;
+  a.softplus = delta_softplus ? 1 : 0;
+  a.scalar_a = 1;
+  a.zoh = (flags & SSM_ZOH) ? 1 : 0;
+  a.bc_groups = bc_groups;
+  a.rows16 = ((size_t)seqlen * es) % 16 == 0 && aligned16(u) && aligned16(delta) &&
+             aligned16(B) && aligned16(C);
+  a.chunk_len = l.plan.chunk_len;
+  a.nchunk = S + 1;  // the summary pass covers segments 0 .. S-1, every one of the sequence
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = ssm::launch_ssd_fwd(a, ssm::kSsdSummary, s);
+  if (e != cudaSuccess) return cuda_fail(e, "sequence summary (chunked matrix form)");
+  float* hin = reinterpret_cast<float*>(w + l.hin);
+  const long long n = (long long)nch * dstate;
+  chain_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(a.summ, a.dsum, A, 1, nullptr, hin,
+                                                           S + 1, (long long)nch, dim, dstate);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "sequence summary chain");
+  summary_finish_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
+      hin + (size_t)S * nch * dstate, dstate, a.dsum, S, (long long)nch, dstate, hend, dsum);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "sequence summary finish");
+  return SSM_OK;
+}
+
 FwdPlan plan_summary(int batch, int dim, int seqlen) {
   FwdPlan p = plan_fwd(batch, dim, seqlen, fwd_chw(false));
   const size_t nch = (size_t)batch * dim;
@@ -590,16 +673,17 @@ FwdPlan plan_summary(int batch, int dim, int seqlen) {
   return p;
 }
 
-// The end state from zero of a whole sequence, out of the carry's entering states (16-state
-// rows) into [batch][dim][N], and each channel's ΣΔ summed (Kahan) over the S chunk summaries.
-__global__ void summary_finish_kernel(const float* __restrict__ hin_end,
+// The end state from zero of a whole sequence, out of the carry's entering states (rows of hs
+// floats per channel) into [batch][dim][N], and each channel's ΣΔ summed (Kahan) over the S
+// chunk summaries.
+__global__ void summary_finish_kernel(const float* __restrict__ hin_end, int hs,
                                       const float* __restrict__ dsum, int S, long long nch, int N,
                                       float* __restrict__ hend, float* __restrict__ dsum_out) {
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= nch * N) return;
   const long long ch = i / N;
   const int n = (int)(i % N);
-  hend[i] = hin_end[ch * ssm::kNS + n];
+  hend[i] = hin_end[ch * hs + n];
   if (n == 0 && dsum_out) {
     float acc = 0.f, comp = 0.f;
     for (int j = 0; j < S; ++j) {
@@ -1274,6 +1358,15 @@ int ssm_scan_bwd_scalar_a(const void* u, const void* delta, const float* A, cons
 size_t ssm_scan_fwd_summary_workspace_size(int batch, int dim, int seqlen, int dstate,
                                            int bc_groups, int io_dtype, int flags) {
   if (flags & ~(SSM_SCALAR_A | SSM_ZOH)) return 0;
+  if ((flags & SSM_SCALAR_A) && dstate > SSM_MAX_DSTATE) {
+    if (check_dims(batch, dim, seqlen, dstate, io_dtype, SSM_MAX_DSTATE_SCALAR) != SSM_OK ||
+        check_groups(dim, bc_groups) != SSM_OK)
+      return 0;
+    if (io_dtype == SSM_F32)
+      return ssm::scan_summary_slices_workspace(batch, dim, seqlen, dstate, bc_groups, flags);
+    if (dstate != 32 && dstate != 64 && dstate != 128) return 0;
+    return summary_chunked_layout(batch, dim, seqlen, dstate).total;
+  }
   if (check_dims(batch, dim, seqlen, dstate, io_dtype) != SSM_OK) return 0;
   if (check_groups(dim, bc_groups) != SSM_OK) return 0;
   return plan_summary(batch, dim, seqlen).ws_bytes;
@@ -1287,6 +1380,16 @@ int ssm_scan_fwd_summary(const void* u, const void* delta, const float* A, const
   g_err[0] = 0;
   if (flags & ~(SSM_SCALAR_A | SSM_ZOH))
     return fail(SSM_EINVAL, "unsupported flags 0x%x for a sequence summary", flags);
+  if ((flags & SSM_SCALAR_A) && dstate > SSM_MAX_DSTATE) {
+    TRY(check_dims(batch, dim, seqlen, dstate, io_dtype, SSM_MAX_DSTATE_SCALAR));
+    TRY(check_groups(dim, bc_groups));
+    if (io_dtype == SSM_F32)
+      return ssm::scan_summary_slices(u, delta, A, B, C, dt_bias, delta_softplus, hend, dsum,
+                                      workspace, workspace_bytes, batch, dim, seqlen, dstate,
+                                      bc_groups, flags, stream);
+    return summary_chunked(u, delta, A, B, C, dt_bias, delta_softplus, hend, dsum, workspace,
+                           workspace_bytes, batch, dim, seqlen, dstate, bc_groups, flags, stream);
+  }
   TRY(check_dims(batch, dim, seqlen, dstate, io_dtype));
   TRY(check_groups(dim, bc_groups));
   if (bc_groups == dim && bc_groups > 1)
@@ -1341,7 +1444,7 @@ int ssm_scan_fwd_summary(const void* u, const void* delta, const float* A, const
     return cuda_fail(e, "sequence summary carry");
   const long long n = (long long)nch * dstate;
   summary_finish_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
-      hin + (size_t)S * nch * ssm::kNS, ds, S, (long long)nch, dstate, hend, dsum);
+      hin + (size_t)S * nch * ssm::kNS, ssm::kNS, ds, S, (long long)nch, dstate, hend, dsum);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "sequence summary finish");
   return SSM_OK;
 }
@@ -1351,8 +1454,8 @@ int ssm_scan_chain(const float* hend, const float* dsum, const float* A, const f
   g_err[0] = 0;
   if (flags & ~SSM_SCALAR_A) return fail(SSM_EINVAL, "unsupported flags 0x%x for a chain", flags);
   if (nseg <= 0) return fail(SSM_EINVAL, "nseg must be positive, got %d", nseg);
-  TRY(check_dims(batch, dim, 1, dstate, SSM_F32));
   const bool scalar_a = (flags & SSM_SCALAR_A) != 0;
+  TRY(check_dims(batch, dim, 1, dstate, SSM_F32, scalar_a ? SSM_MAX_DSTATE_SCALAR : SSM_MAX_DSTATE));
   const size_t nch = (size_t)batch * dim;
   TRY(check_ptr(hend, (size_t)nseg * nch * dstate * 4, 4, "hend"));
   TRY(check_ptr(dsum, (size_t)nseg * nch * 4, 4, "dsum"));

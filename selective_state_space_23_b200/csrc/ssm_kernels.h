@@ -216,6 +216,14 @@ int scan_fwd_slices(const void* u, const void* delta, const float* A, const void
                     int delta_softplus, const float* h0, float* hL, void* out, float* ckpt,
                     void* workspace, size_t workspace_bytes, int batch, int dim, int seqlen,
                     int dstate, int bc_groups, int io_dtype, int flags, void* stream);
+// The f32 sequence summary of the scalar-decay scan for dstate = 16 k as k 16-state summaries
+// (ssm_slices.cu); arguments as ssm_scan_fwd_summary.
+size_t scan_summary_slices_workspace(int batch, int dim, int seqlen, int dstate, int bc_groups,
+                                     int flags);
+int scan_summary_slices(const void* u, const void* delta, const float* A, const void* B,
+                        const void* C, const float* dt_bias, int delta_softplus, float* hend,
+                        float* dsum, void* workspace, size_t workspace_bytes, int batch, int dim,
+                        int seqlen, int dstate, int bc_groups, int flags, void* stream);
 size_t scan_bwd_slices_workspace(int batch, int dim, int seqlen, int dstate, int bc_groups,
                                  int io_dtype, int flags);
 int scan_bwd_slices(const void* u, const void* delta, const float* A, const void* B,

@@ -241,6 +241,91 @@ int scan_fwd_slices(const void* u, const void* delta, const float* A, const void
   return SSM_OK;
 }
 
+// Sequence summary (end state from zero, ΣΔ) of the f32 scalar-decay scan with dstate = 16 k: the
+// 16-state summary of each slice of B gives that slice of the end state; ΣΔ does not depend on
+// the states and is taken from the first slice.  The summary reads no C: each slice's call is
+// given its B slice in C's place.
+namespace {
+struct SummarySliceLayout {
+  size_t bj, hj, inner, inner_bytes, total;
+};
+
+SummarySliceLayout summary_slice_layout(int batch, int dim, int seqlen, int bc_groups, int flags) {
+  SummarySliceLayout l;
+  size_t o = 0;
+  l.bj = o; o += align256((size_t)batch * bc_groups * kNS * seqlen * 4);
+  l.hj = o; o += align256((size_t)batch * dim * kNS * 4);
+  l.inner = o;
+  l.inner_bytes = align256(ssm_scan_fwd_summary_workspace_size(batch, dim, seqlen, kNS, bc_groups,
+                                                               SSM_F32, flags));
+  l.total = l.inner_bytes == 0 ? 0 : o + l.inner_bytes;
+  return l;
+}
+}  // namespace
+
+size_t scan_summary_slices_workspace(int batch, int dim, int seqlen, int dstate, int bc_groups,
+                                     int flags) {
+  if (dstate % kNS != 0 || dstate > SSM_MAX_DSTATE_SCALAR || !(flags & SSM_SCALAR_A) ||
+      batch <= 0 || dim <= 0 || seqlen <= 0 || bc_groups < 1)
+    return 0;
+  return summary_slice_layout(batch, dim, seqlen, bc_groups, flags).total;
+}
+
+int scan_summary_slices(const void* u, const void* delta, const float* A, const void* B,
+                        const void* C, const float* dt_bias, int delta_softplus, float* hend,
+                        float* dsum, void* workspace, size_t workspace_bytes, int batch, int dim,
+                        int seqlen, int dstate, int bc_groups, int flags, void* stream) {
+  if (dstate % kNS != 0 || dstate > SSM_MAX_DSTATE_SCALAR)
+    return fail(SSM_EUNSUPPORTED, "an f32 sequence summary with dstate > 16 needs a multiple of 16 "
+                                  "up to 128");
+  if (bc_groups == dim && bc_groups > 1)
+    return fail(SSM_EUNSUPPORTED, "sequence summaries take shared or grouped B/C");
+  const size_t need = scan_summary_slices_workspace(batch, dim, seqlen, dstate, bc_groups, flags);
+  if (need == 0) return fail(SSM_EINVAL, "invalid sizes or groups");
+  if (!workspace || workspace_bytes < need) {
+    char msg[128];
+    snprintf(msg, sizeof(msg), "workspace of %zu bytes given, %zu needed", workspace_bytes, need);
+    return fail(SSM_EWORKSPACE, msg);
+  }
+  if (reinterpret_cast<uintptr_t>(workspace) & 255)
+    return fail(SSM_EINVAL, "workspace is not 256-byte aligned");
+  int rc = check_device_ptr(workspace, need, 256, "workspace");
+  if (rc != SSM_OK) return rc;
+  const long long nbc = (long long)bc_groups * dstate * seqlen;
+  if ((rc = check_device_ptr(B, (size_t)batch * nbc * 4, 4, "B")) != SSM_OK) return rc;
+  if ((rc = check_device_ptr(C, (size_t)batch * nbc * 4, 4, "C")) != SSM_OK) return rc;
+  if ((rc = check_device_ptr(hend, (size_t)batch * dim * dstate * 4, 4, "hend")) != SSM_OK) return rc;
+  const SummarySliceLayout l = summary_slice_layout(batch, dim, seqlen, bc_groups, flags);
+  char* w = reinterpret_cast<char*>(workspace);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long long n_bc[4] = {batch, bc_groups, kNS, seqlen};
+  const long long s_bc[4] = {(long long)bc_groups * dstate * seqlen, (long long)dstate * seqlen, seqlen, 1};
+  const long long d_bc[4] = {(long long)bc_groups * kNS * seqlen, (long long)kNS * seqlen, seqlen, 1};
+  const long long n_st[4] = {1, batch, dim, kNS};
+  const long long s_st[4] = {0, (long long)dim * dstate, dstate, 1};
+  const long long d_st[4] = {0, (long long)dim * kNS, kNS, 1};
+  cudaError_t e = cudaSuccess;
+  for (int j = 0; j < dstate / kNS; ++j) {
+    const size_t off = (size_t)j * kNS;
+    void* Bj = w + l.bj;
+    float* hj = reinterpret_cast<float*>(w + l.hj);
+    if ((e = copy_view(reinterpret_cast<const float*>(B) + off * seqlen, n_bc, s_bc, Bj, d_bc, 4,
+                       s)) != cudaSuccess) {
+      set_last_error(cudaGetErrorString(e));
+      return SSM_ECUDA;
+    }
+    rc = ssm_scan_fwd_summary(u, delta, A, Bj, Bj, dt_bias, delta_softplus, hj,
+                              j == 0 ? dsum : nullptr, w + l.inner, l.inner_bytes, batch, dim,
+                              seqlen, kNS, bc_groups, SSM_F32, flags, stream);
+    if (rc != SSM_OK) return rc;
+    if ((e = copy_view(hj, n_st, d_st, hend + off, s_st, 4, s)) != cudaSuccess) {
+      set_last_error(cudaGetErrorString(e));
+      return SSM_ECUDA;
+    }
+  }
+  return SSM_OK;
+}
+
 size_t scan_bwd_slices_workspace(int batch, int dim, int seqlen, int dstate, int bc_groups,
                                  int io_dtype, int flags) {
   if (dstate % kNS != 0 || dstate > SSM_MAX_DSTATE_SCALAR || !(flags & SSM_SCALAR_A) ||

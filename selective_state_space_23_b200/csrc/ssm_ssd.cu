@@ -16,6 +16,7 @@
 //   G   = C B^T                     [16 t x 16 s]   K = N    (masked to s <= t)
 //   Y1' = X1' mask(G)^T              [16 d x 16 t]   K = 16,  X1'[d][s] = Q_s Δ_s x_s
 //   Y2' = H' C^T                     [16 d x 16 t]   K = N,   H' = h_in transposed [d][n]
+//                                    (H' as a bf16 pair plus its remainder: two products)
 //   U'  = X2' B                      [16 d x N]      K = 16,  X2'[d][s] = e^{A (S_end - S_s)} Δ_s x_s
 // and y = P Y1 + e^{A S_t} Y2 + D x,  H' <- e^{A S_end} H' + U'.
 //
@@ -340,12 +341,17 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
       ldsm_x4_t(bf, blk(st.Bs, 16 * kk, lane));  // {s0-7|n lo, s8-15|n lo, s0-7|n hi, s8-15|n hi}
       mma16816(G[0], cf[0], cf[1], cf[2], cf[3], bf[0], bf[2]);
       mma16816(G[1], cf[0], cf[1], cf[2], cf[3], bf[1], bf[3]);
-      const uint32_t h0 = pack_bf16x2(Ht[2 * kk][0], Ht[2 * kk][1]);
-      const uint32_t h1 = pack_bf16x2(Ht[2 * kk][2], Ht[2 * kk][3]);
-      const uint32_t h2 = pack_bf16x2(Ht[2 * kk + 1][0], Ht[2 * kk + 1][1]);
-      const uint32_t h3 = pack_bf16x2(Ht[2 * kk + 1][2], Ht[2 * kk + 1][3]);
+      // the f32 state as a bf16 pair plus its bf16 remainder: one bf16 operand would round h to
+      // 8 bits, an error of 2^-9 |h| per state summed over N states in C . h_in
+      uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
+      split_bf16x2(Ht[2 * kk][0], Ht[2 * kk][1], h0, l0);
+      split_bf16x2(Ht[2 * kk][2], Ht[2 * kk][3], h1, l1);
+      split_bf16x2(Ht[2 * kk + 1][0], Ht[2 * kk + 1][1], h2, l2);
+      split_bf16x2(Ht[2 * kk + 1][2], Ht[2 * kk + 1][3], h3, l3);
       mma16816(Y2[0], h0, h1, h2, h3, cf[0], cf[2]);
       mma16816(Y2[1], h0, h1, h2, h3, cf[1], cf[3]);
+      mma16816(Y2[0], l0, l1, l2, l3, cf[0], cf[2]);
+      mma16816(Y2[1], l0, l1, l2, l3, cf[1], cf[3]);
     }
     // ---- H' <- e^{A S_end} H' + X2' B   (fb channels: scale 1, zero inputs: unchanged)
 #pragma unroll

@@ -223,3 +223,21 @@ def test_large_n_decode_is_checked_on_the_host(lib):
     assert lib.ssm_state_update_ex(*([None] * 9), 1, None, 2, 64, 48, 1, 1, _abi.SSM_SCALAR_A,
                                    None) == _abi.SSM_EUNSUPPORTED
     assert b"32, 64 or 128" in lib.ssm_last_error()
+
+
+def test_large_n_workspace_queries(lib):
+    """Scalar decay with N > 16: the forward and summary queries cover the path each call takes
+    (bf16: the chunked matrix form, N = 32, 64, 128; f32: 16-state slices, any multiple of 16 up
+    to 128); other sizes ask for nothing because the call refuses them."""
+    sa = _abi.SSM_SCALAR_A
+    for io in (_abi.SSM_BF16, _abi.SSM_F32):
+        for N in (32, 64, 128):
+            assert lib.ssm_scan_fwd_summary_workspace_size(1, 64, 400, N, 1, io, sa) > 0
+            assert lib.ssm_scan_fwd_scalar_a_workspace_size(1, 64, 4096, N, io) > 0
+    assert lib.ssm_scan_fwd_summary_workspace_size(1, 64, 400, 48, 1, _abi.SSM_F32, sa) > 0
+    assert lib.ssm_scan_fwd_summary_workspace_size(1, 64, 400, 48, 1, _abi.SSM_BF16, sa) == 0
+    assert lib.ssm_scan_fwd_summary_workspace_size(1, 64, 400, 40, 1, _abi.SSM_F32, sa) == 0
+    assert lib.ssm_scan_fwd_summary_workspace_size(1, 64, 400, 64, 1, _abi.SSM_BF16, 0) == 0
+    # the f32 slice forward holds slice copies of B, C and one slice's output at least
+    f32 = lib.ssm_scan_fwd_ex_workspace_size(2, 64, 256, 64, 1, _abi.SSM_F32, sa)
+    assert f32 >= 2 * 2 * 16 * 256 * 4 + 2 * 64 * 256 * 4

@@ -131,3 +131,49 @@ def test_helper_without_process_group():
     r = ref(x)
     assert_close(out, r["out"], torch.bfloat16, "out")
     assert_close(hL, h2.cpu().numpy().astype(np.float64), torch.bfloat16, "hL")
+
+
+@pytest.mark.parametrize("io,N", [(torch.bfloat16, 64), (torch.bfloat16, 128), (torch.float32, 32),
+                                  (torch.float32, 64)])
+@pytest.mark.parametrize("nseg", [1, 3])
+def test_large_state_scalar_decay_segments(io, N, nseg):
+    """Scalar decay with N = 32 to 128 (the Mamba-2 state sizes): bf16 summaries run the chunked
+    matrix form's summary pass, f32 ones sum 16-state slices; the split reproduces the whole
+    sequence, and each summary is the segment's end state from zero with its summed steps."""
+    w = workload("long_seq_1m", batch=2, dim=64, seqlen=400, dstate=N, io_dtype=io)
+    x = make_inputs(w, seed=93, with_h0=True, scalar_a=True)
+    spans, hs, ds, out, hL = split_run(x, nseg, scalar_a=True)
+    r = ref(x, scalar_a=True)
+    assert_close(out, r["out"], io, "out")
+    assert_close(hL, r["hL"], io, "hL")
+    c = lambda k: f64(x[k])
+    A = np.repeat(c("A")[:, None], N, axis=1)
+    for (t0, t1), h, d in zip(spans, hs, ds):
+        rs = oracle.scan_fwd(c("u")[..., t0:t1], c("delta")[..., t0:t1], A, c("B")[..., t0:t1],
+                             c("C")[..., t0:t1], dt_bias=c("dt_bias"))
+        assert_close(h, rs["hL"], io, f"hend {t0}")
+        v = c("delta")[..., t0:t1] + c("dt_bias")[None, :, None]
+        dref = np.logaddexp(0.0, v).sum(-1)
+        assert_close(d, dref, torch.float32, f"dsum {t0}")
+
+
+@pytest.mark.parametrize("N", [64, 128])
+def test_large_state_summary_splits_itself(monkeypatch, N):
+    """Few channels: the chunked form's planner cuts the segment into several pieces, chained
+    from zero inside the call; forced counts agree with the unsplit summary."""
+    w = workload("long_seq_1m", batch=1, dim=64, seqlen=1000, dstate=N)
+    x = make_inputs(w, seed=94, scalar_a=True)
+    xd = {k: v.to(DEV) for k, v in x.items()}
+    run = lambda: ssm.ssm_scan_fwd_summary(xd["u"], xd["delta"], xd["A"], xd["B"], xd["C"],
+                                           dt_bias=xd["dt_bias"], scalar_a=True)
+    monkeypatch.setenv("SSM_SSD_SPLIT", "1")
+    h1, d1 = run()
+    c = lambda k: f64(x[k])
+    A = np.repeat(c("A")[:, None], N, axis=1)
+    rs = oracle.scan_fwd(c("u"), c("delta"), A, c("B"), c("C"), dt_bias=c("dt_bias"))
+    assert_close(h1, rs["hL"], torch.bfloat16, "hend unsplit")
+    for split in ("4", "9"):
+        monkeypatch.setenv("SSM_SSD_SPLIT", split)
+        h, d = run()
+        assert_close(h, rs["hL"], torch.bfloat16, f"hend split {split}")
+        torch.testing.assert_close(d, d1, rtol=1e-5, atol=1e-5)
