@@ -151,16 +151,17 @@ def test_natural_time_split_long_sequence():
 def test_large_entering_state_is_read_out_at_f32_precision(N):
     """The readout of the state entering a chunk, C_t . h_in, sums N products: with h rounded to
     one bf16 each product carries 2^-9 |h|, and at N = 128 with |h| ~ 3 the sum misses by ~0.1.
-    The state is a bf16 pair plus remainder there, so the outputs keep the bf16 tolerance with
-    an entering state of any size (here h0 ~ N(0, 3^2), on top of the inputs' own state)."""
+    The state is a bf16 pair plus remainder there, so the error does not grow with the entering
+    state: h0 ~ N(0, 3^2) gives the same worst error as a zero h0 on the same inputs (whose
+    floor is the bf16 operands of the intra-chunk products), and both keep the bf16 bound."""
     x = inputs(2, 64, 96, N, seed=68)
-    x["h0"] = torch.from_numpy(
-        np.random.default_rng(9).normal(0.0, 3.0, size=(2, 64, N)).astype(np.float32))
-    out, hL = gpu(x)
-    r = ref(x)
-    assert_close(out, r["out"], torch.bfloat16, "out")
-    assert_close(hL, r["hL"], torch.bfloat16, "hL")
-    # normalised errors well inside the bound (the rounding of the bf16 output itself dominates)
-    g = f64(out)
-    err = np.abs(g - r["out"]) / np.maximum(1.0, np.abs(r["out"]))
-    assert err.max() < 1e-2, err.max()
+    errs = []
+    for h0 in (torch.zeros_like(x["h0"]), torch.from_numpy(
+            np.random.default_rng(9).normal(0.0, 3.0, size=(2, 64, N)).astype(np.float32))):
+        x["h0"] = h0
+        out, hL = gpu(x)
+        r = ref(x)
+        assert_close(out, r["out"], torch.bfloat16, "out")
+        assert_close(hL, r["hL"], torch.bfloat16, "hL")
+        errs.append(np.max(np.abs(f64(out) - r["out"]) / np.maximum(1.0, np.abs(r["out"]))))
+    assert errs[1] <= 1.25 * errs[0] + 2e-3, errs
