@@ -522,7 +522,8 @@ def ssm_scan_fwd_summary(u, delta, A, B, C, dt_bias=None, delta_softplus=True, s
                          zoh=False, workspace=None):
     """The affine map of one sequence segment: returns (hend [batch, dim, N], dsum [batch, dim]),
     the state after the segment from a zero state and ΣΔ over it, so that the segment maps an
-    entering state h to exp(A dsum) h + hend."""
+    entering state h to exp(A dsum) h + hend.  With scalar_a, N may be 32 to 128 as in the
+    scalar-decay scan (bf16: 32, 64 or 128; f32: any multiple of 16)."""
     dev = _on_gpu(u, "u")
     batch, dim, L = u.shape
     io = u.dtype
