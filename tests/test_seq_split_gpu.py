@@ -177,3 +177,15 @@ def test_large_state_summary_splits_itself(monkeypatch, N):
         h, d = run()
         assert_close(h, rs["hL"], torch.bfloat16, f"hend split {split}")
         torch.testing.assert_close(d, d1, rtol=1e-5, atol=1e-5)
+
+
+@pytest.mark.parametrize("io", [torch.bfloat16, torch.float32])
+def test_large_state_zoh_segments(io):
+    """The zero-order-hold input term with 64 states: summaries (chunked summary pass in bf16,
+    16-state slices in f32), chain and segment forwards reproduce the whole sequence."""
+    w = workload("long_seq_1m", batch=1, dim=64, seqlen=300, dstate=64, io_dtype=io)
+    x = make_inputs(w, seed=95, with_h0=True, scalar_a=True)
+    _, _, _, out, hL = split_run(x, 3, scalar_a=True, zoh=True)
+    r = ref(x, scalar_a=True, zoh=True)
+    assert_close(out, r["out"], io, "out")
+    assert_close(hL, r["hL"], io, "hL")

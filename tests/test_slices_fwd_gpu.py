@@ -148,3 +148,15 @@ def test_refusals():
     y = inputs(1, 32, 32, 40, seed=217)
     with pytest.raises(RuntimeError):
         gpu(y)
+
+
+@pytest.mark.parametrize("shape", [(1, 1, 1), (1, 3, 2), (1, 16, 4000)])
+def test_edge_shapes(shape):
+    """One step, one channel, and few channels over a long sequence (the 16-state forward then
+    splits time inside each slice's call)."""
+    batch, dim, L = shape
+    x = inputs(batch, dim, L, 64, seed=218)
+    out, hL = gpu(x, return_final_state=True)
+    r = ref(x)
+    assert_close(out, r["out"], F32, "out")
+    assert_close(hL, r["hL"], F32, "hL")
