@@ -357,3 +357,18 @@ def test_chunked_backward_gradient_subsets(need):
             assert torch.equal(part[k], full[k]), k
         else:
             assert part.get(k) is None, k
+
+
+@pytest.mark.parametrize("N", [64, 128])
+def test_chunked_backward_large_entering_state(N):
+    """An entering state h0 ~ N(0, 3^2), larger than the inputs' own state: every product that
+    reads the state (or its adjoint) takes it as a bf16 pair plus remainder, so the gradients,
+    dh0 and dC included, keep the bf16 bound."""
+    x = inputs(2, 64, 96, N, torch.bfloat16, seed=131)
+    x["h0"] = torch.from_numpy(
+        np.random.default_rng(10).normal(0.0, 3.0, size=(2, 64, N)).astype(np.float32))
+    dhL = torch.randn((2, 64, N), generator=torch.Generator().manual_seed(11))
+    g = run(x, dhL)
+    r = ref(x, dhL)
+    for k in GRADS:
+        assert_close(g[k], r[k], torch.bfloat16, k)
