@@ -34,7 +34,10 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 // both operands are split (hi.hi + hi.lo + lo.hi; the lo.lo term is below f32 rounding).
 __device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
   hi = pack_bf16x2(a, b);
-  lo = pack_bf16x2(a - bf16_lo(hi), b - bf16_hi(hi));
+  // (a, b) - hi as one packed f32x2 operation; the differences are exact either way
+  const float2 r = fma2(make_float2(bf16_lo(hi), bf16_hi(hi)), make_float2(-1.f, -1.f),
+                        make_float2(a, b));
+  lo = pack_bf16x2(r.x, r.y);
 }
 
 // Zero-order-hold input coefficient of a step Δ with one rate A per channel (the chunked form):
