@@ -317,13 +317,20 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
       scale[c] = fb[c] ? 1.f : ex2_mufu(Se[c] * al[c]);
       float q1[4], q2[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float r = (S[c][j] - Sm[c]) * al[c];
-        P[c][j] = ex2_mufu(r);
-        E[c][j] = eAm * P[c][j];
-        const float Q = ex2_mufu(-r);
-        q1[j] = fb[c] ? 0.f : Q * xv[c][j];
-        q2[j] = fb[c] ? 0.f : eEm * q1[j];
+      for (int j = 0; j < 4; j += 2) {  // packed f32x2 over step pairs
+        const float2 r = mul2(add2(make_float2(S[c][j], S[c][j + 1]), f2(-Sm[c])), f2(al[c]));
+        P[c][j] = ex2_mufu(r.x);
+        P[c][j + 1] = ex2_mufu(r.y);
+        const float2 e = mul2(f2(eAm), make_float2(P[c][j], P[c][j + 1]));
+        E[c][j] = e.x;
+        E[c][j + 1] = e.y;
+        const float2 q = mul2(make_float2(ex2_mufu(-r.x), ex2_mufu(-r.y)),
+                              make_float2(xv[c][j], xv[c][j + 1]));
+        const float2 qq = mul2(f2(eEm), q);
+        q1[j] = fb[c] ? 0.f : q.x;
+        q1[j + 1] = fb[c] ? 0.f : q.y;
+        q2[j] = fb[c] ? 0.f : qq.x;
+        q2[j + 1] = fb[c] ? 0.f : qq.y;
       }
       x1[c] = pack_bf16x2(q1[0], q1[1]);
       x1[2 + c] = pack_bf16x2(q1[2], q1[3]);
@@ -359,9 +366,14 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
       uint32_t bn[4];
       ldsm_x4(bn, blk(st.Bs, 8 * nt, lane));  // {n tile nt: s lo, s hi; n tile nt+1: s lo, s hi}
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        Ht[nt][e] *= scale[e >> 1];
-        Ht[nt + 1][e] *= scale[e >> 1];
+      for (int c = 0; c < 2; ++c) {  // packed f32x2: the two states of a channel share its scale
+        const float2 sc = make_float2(scale[c], scale[c]);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const float2 h = mul2(make_float2(Ht[nt + u][2 * c], Ht[nt + u][2 * c + 1]), sc);
+          Ht[nt + u][2 * c] = h.x;
+          Ht[nt + u][2 * c + 1] = h.y;
+        }
       }
       mma16816(Ht[nt], x2[0], x2[1], x2[2], x2[3], bn[0], bn[1]);
       mma16816(Ht[nt + 1], x2[0], x2[1], x2[2], x2[3], bn[2], bn[3]);
@@ -390,10 +402,16 @@ __global__ void __launch_bounds__(32 * W) ssd_fwd_kernel(const __grid_constant__
 #pragma unroll
     for (int T = 0; T < 2; ++T) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int c = e >> 1, j = 2 * T + (e & 1);
-        const float y = fmaf(P[c][j], Y1[T][e], fmaf(E[c][j], Y2[T][e], Dd[c] * uv[c][j]));
-        yo[c][j] = y * gt[c][j];
+      for (int c = 0; c < 2; ++c) {  // packed f32x2 over the steps j = 2T, 2T + 1
+        const int j = 2 * T;
+        const float2 du = mul2(make_float2(Dd[c], Dd[c]), make_float2(uv[c][j], uv[c][j + 1]));
+        const float2 y2 = fma2(make_float2(E[c][j], E[c][j + 1]),
+                               make_float2(Y2[T][2 * c], Y2[T][2 * c + 1]), du);
+        const float2 y = fma2(make_float2(P[c][j], P[c][j + 1]),
+                              make_float2(Y1[T][2 * c], Y1[T][2 * c + 1]), y2);
+        const float2 o = mul2(y, make_float2(gt[c][j], gt[c][j + 1]));
+        yo[c][j] = o.x;
+        yo[c][j + 1] = o.y;
       }
     }
     // ---- channels outside the factorisation's range this chunk: exact sequential pass over
