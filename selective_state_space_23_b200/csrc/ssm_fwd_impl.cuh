@@ -61,14 +61,26 @@ struct Layout {
   // floats per step in the partial-readout table: a multiple of LPC (aligned vector reads of a
   // channel's LPC partials) chosen so that the owners' reads of different steps spread over banks
   static constexpr int kYpStride = LPC == 1 ? 33 : (LPC == 2 ? 34 : 36);
+  // Steps 8..15 of the B/C tiles and of the step table sit one bank group further on.  Rows 8
+  // apart otherwise share banks for any 16-byte-aligned stride, and the lanes that write a step
+  // table row or a B/C row come in pairs 8 steps apart (the two halves of a block), which made
+  // every such store a 2-way bank conflict.  The shift in float4 entries of the step table
+  // spreads the LPC owners of a row group over distinct bank groups.
+  static constexpr int kSdShift = LPC == 2 ? 4 : (LPC == 4 ? 2 : 0);
+  // float4 offset of step k's row in the B/C tiles ([step][16 states] f32) and step table
+  static __device__ __host__ constexpr int bc4(int k) { return 4 * k + (k >= 8 ? 4 : 0); }
+  static __device__ __host__ constexpr int sd4(int k) {
+    return k * kSdStride + (k >= 8 ? kSdShift : 0);
+  }
 };
 
 // Shared memory of one 16-step block of a warp.
 template <int LPC>
 struct BlockBuf {
-  float4 sB[kBlk * kNS / 4];                          // B_t,n as f32 [step][state]
-  float4 sC[kBlk * kNS / 4];                          // C_t,n
-  float4 sd[kBlk * Layout<LPC>::kSdStride];           // (Δ_t, Δ_t, Δ_t x_t, Δ_t x_t) per [step][slot]
+  float4 sB[kBlk * kNS / 4 + 4];                      // B_t,n as f32 [step][state] (Layout::bc4)
+  float4 sC[kBlk * kNS / 4 + 4];                      // C_t,n
+  // (Δ_t, Δ_t, Δ_t x_t, Δ_t x_t) per [step][slot] (Layout::sd4)
+  float4 sd[kBlk * Layout<LPC>::kSdStride + Layout<LPC>::kSdShift];
   float yp[kBlk * Layout<LPC>::kYpStride];            // partial readouts per [step][slot][lane]
 };
 
@@ -179,18 +191,18 @@ __device__ __forceinline__ void state_loop(BlockBuf<LPC>& tile, float2 (&hh)[Lay
   int k = 0;
 #pragma unroll 1
   for (; k + 2 <= nvalid; k += 2) {
-    prepare_step<kPrecise, PPL, KO>(p1, al, ra, sdp[(k + 1) * Lay::kSdStride], bq + (k + 1) * 4);
-    const float y0 = consume_step<kReadout, PPL>(hh, p0, cq + k * 4);
+    prepare_step<kPrecise, PPL, KO>(p1, al, ra, sdp[Lay::sd4(k + 1)], bq + Lay::bc4(k + 1));
+    const float y0 = consume_step<kReadout, PPL>(hh, p0, cq + Lay::bc4(k));
     const int k2 = min(k + 2, kBlk - 1);
-    prepare_step<kPrecise, PPL, KE>(p0, al, ra, sdp[k2 * Lay::kSdStride], bq + k2 * 4);
-    const float y1 = consume_step<kReadout, PPL>(hh, p1, cq + (k + 1) * 4);
+    prepare_step<kPrecise, PPL, KE>(p0, al, ra, sdp[Lay::sd4(k2)], bq + Lay::bc4(k2));
+    const float y1 = consume_step<kReadout, PPL>(hh, p1, cq + Lay::bc4(k + 1));
     if (kReadout) {
       yp[k * Lay::kYpStride] = y0;
       yp[(k + 1) * Lay::kYpStride] = y1;
     }
   }
   if (k < nvalid) {  // odd number of valid steps: the last one was prepared into p0
-    const float y0 = consume_step<kReadout, PPL>(hh, p0, cq + k * 4);
+    const float y0 = consume_step<kReadout, PPL>(hh, p0, cq + Lay::bc4(k));
     if (kReadout) yp[k * Lay::kYpStride] = y0;
   }
 }
@@ -353,8 +365,9 @@ struct ChunkLane {
   // Stage B_t,bn and C_t,bn of step 8 bh + j of the block as f32 [step][state].
   __device__ __forceinline__ void stage_row(float* __restrict__ sB, float* __restrict__ sC,
                                             const Rows& r, int j) const {
-    sB[(8 * bh + j) * kNS + bn] = r.b.get(j);
-    if (kReadout) sC[(8 * bh + j) * kNS + bn] = r.c.get(j);
+    const int o = 4 * Lay::bc4(8 * bh + j) + bn;
+    sB[o] = r.b.get(j);
+    if (kReadout) sC[o] = r.c.get(j);
   }
 
   // Δ and Δx of owned steps j, j+1 into the block's table.  ok stays true while every |Δ| is
@@ -385,8 +398,8 @@ struct ChunkLane {
       }
       dx = mul2(g, xv);
     }
-    sd[(SPL * q + j) * Lay::kSdStride + slot] = make_float4(tv.x, tv.x, dx.x, dx.x);
-    sd[(SPL * q + j + 1) * Lay::kSdStride + slot] = make_float4(tv.y, tv.y, dx.y, dx.y);
+    sd[Lay::sd4(SPL * q + j) + slot] = make_float4(tv.x, tv.x, dx.x, dx.x);
+    sd[Lay::sd4(SPL * q + j + 1) + slot] = make_float4(tv.y, tv.y, dx.y, dx.y);
     if (MODE == kFwdSummary) dblk += (j < nown ? dl.x : 0.f) + (j + 1 < nown ? dl.y : 0.f);
     ok = ok && fabsf(dl.x) < dlim && fabsf(dl.y) < dlim;
   }
@@ -487,17 +500,17 @@ __device__ __forceinline__ void interleaved_block(
   // two steps prepared ahead: steps k+2, k+3 are prepared while k, k+1 update the state
   StepPrep<PPL> p0, p1;
   prepare_step<kPrecise, PPL, KE>(p0, al, ra, sdp[0], bq);
-  prepare_step<kPrecise, PPL, KO>(p1, al, ra, sdp[Lay::kSdStride], bq + 4);
+  prepare_step<kPrecise, PPL, KO>(p1, al, ra, sdp[Lay::sd4(1)], bq + Lay::bc4(1));
 #pragma unroll
   for (int m = 0; m < 8; ++m) {
     const int k = 2 * m;
     StepPrep<PPL> q0, q1;
     if (m < 7)
-      prepare_step<kPrecise, PPL, KE>(q0, al, ra, sdp[(k + 2) * Lay::kSdStride], bq + (k + 2) * 4);
-    const float y0 = consume_step<kReadout, PPL>(hh, p0, cq + k * 4);
+      prepare_step<kPrecise, PPL, KE>(q0, al, ra, sdp[Lay::sd4(k + 2)], bq + Lay::bc4(k + 2));
+    const float y0 = consume_step<kReadout, PPL>(hh, p0, cq + Lay::bc4(k));
     if (m < 7)
-      prepare_step<kPrecise, PPL, KO>(q1, al, ra, sdp[(k + 3) * Lay::kSdStride], bq + (k + 3) * 4);
-    const float y1 = consume_step<kReadout, PPL>(hh, p1, cq + (k + 1) * 4);
+      prepare_step<kPrecise, PPL, KO>(q1, al, ra, sdp[Lay::sd4(k + 3)], bq + Lay::bc4(k + 3));
+    const float y1 = consume_step<kReadout, PPL>(hh, p1, cq + Lay::bc4(k + 1));
     p0 = q0;
     p1 = q1;
     if (kReadout) {
