@@ -40,6 +40,11 @@ namespace {
 constexpr int kCW = 16;                   // channels per warp
 constexpr int kBCS = kBlk * kNS + 16;     // f32 B/C tile [step][state], steps 8..15 shifted
 __device__ __forceinline__ int bco(int k) { return k * kNS + (k >= 8 ? 16 : 0); }
+// Per-step table [step][channel slot] (float4), steps 8..15 one bank group further on: the two
+// lanes of a channel write and read the rows of steps j and 8 + j together, and rows 8 apart
+// would otherwise share their banks.
+constexpr int kTbl = kBlk * kCW + 4;
+__device__ __forceinline__ int tbo(int k) { return k * kCW + (k >= 8 ? 4 : 0); }
 
 template <typename IO>
 struct HGeo {
@@ -51,7 +56,7 @@ struct HGeo {
   static constexpr int kSlotBytes = kRowsBytes + kRawBytes + kCkBytes;
   static constexpr int kWarpBytes = 2 * kSlotBytes          // ring: this block and the next
                                     + 2 * kBCS * 4          // B/C tile as f32
-                                    + kBlk * kCW * 16       // per-step scalars, then outputs
+                                    + kTbl * 16             // per-step scalars, then outputs
                                     + kBlk * 32 * 4;        // dB/dC warp sums of the block
 };
 
@@ -131,7 +136,7 @@ struct HistBwd {
   // the outputs of step k replace its scalars once both lanes of the channel have read them
   __device__ __forceinline__ float4* outs() const { return table(); }
   __device__ __forceinline__ float* red() const {
-    return reinterpret_cast<float*>(table() + kBlk * kCW);
+    return reinterpret_cast<float*>(table() + kTbl);
   }
 
   // Copies of block blk: the lane's 8 steps (8 q ..) of its channel's u, delta, z, dout; its
@@ -174,9 +179,11 @@ struct HistBwd {
              reinterpret_cast<const unsigned char*>(reinterpret_cast<const IO*>(a.C) + bcrow) + off, nbc);
       }
       const float* ck = a.ckpt + (ch * nblk + blk) * kNS + 8 * q;
+      // halves swapped for lanes with bit 2 set: lanes 4 apart then use different bank groups
       unsigned char* cks = sl + G::kRowsBytes + G::kRawBytes + lane * 32;
-      cp16(cks, ck);
-      cp16(cks + 16, ck + 4);
+      const int sw = (lane >> 2) & 1;
+      cp16(cks + 16 * sw, ck);
+      cp16(cks + 16 * (1 - sw), ck + 4);
     }
     cp_commit();
   }
@@ -198,8 +205,9 @@ struct HistBwd {
   // The checkpointed state entering block blk, in the lane's rotated order.
   __device__ __forceinline__ void entry_state(int blk, float2 (&h)[4]) const {
     const float* ck = reinterpret_cast<const float*>(slot(blk) + G::kRowsBytes + G::kRawBytes + lane * 32);
-    const float4 lo = *reinterpret_cast<const float4*>(ck + 4 * rot);
-    const float4 hi = *reinterpret_cast<const float4*>(ck + 4 * (1 - rot));
+    const int sw = (lane >> 2) & 1;  // the halves as issue() placed them
+    const float4 lo = *reinterpret_cast<const float4*>(ck + 4 * (rot ^ sw));
+    const float4 hi = *reinterpret_cast<const float4*>(ck + 4 * ((1 - rot) ^ sw));
     h[0] = make_float2(lo.x, lo.y);
     h[1] = make_float2(lo.z, lo.w);
     h[2] = make_float2(hi.x, hi.y);
@@ -209,7 +217,7 @@ struct HistBwd {
   // One replayed step k: h <- Ā h + Δx B.
   template <int KP>
   __device__ __forceinline__ void replay(int k, float2 (&h)[4], const float2 (&al)[4]) const {
-    const float4 sc = table()[k * kCW + s];
+    const float4 sc = table()[tbo(k) + s];
     float2 bq[4];
     quads(bcf() + bco(k), qlo, qhi, bq);
     const float2 d2 = f2(sc.x), du2 = f2(sc.y);
@@ -224,7 +232,7 @@ struct HistBwd {
                                           float2 (&dA)[4], const float2 (&al)[4], float uk,
                                           float svk, float Dd, float live, float& dD_acc,
                                           float& db_acc) const {
-    const float4 sc = table()[k * kCW + s];  // (Δ, Δx, g, dout silu'(z))
+    const float4 sc = table()[tbo(k) + s];  // (Δ, Δx, g, dout silu'(z))
     float2 bq[4], cq[4];
     quads(bcf() + bco(k), qlo, qhi, bq);
     quads(bcf() + kBCS + bco(k), qlo, qhi, cq);
@@ -259,7 +267,7 @@ struct HistBwd {
       const float dz = sc.w * fmaf(Dd, uk, y);
       dD_acc = fmaf(sc.z * live, uk, dD_acc);
       db_acc = fmaf(live, ddl, db_acc);
-      outs()[k * kCW + s] = make_float4(du, ddl, dz, 0.f);
+      outs()[tbo(k) + s] = make_float4(du, ddl, dz, 0.f);
     }
     // dB, dC over the warp's 16 channels (lane bits 1..4 = channel slot bits 0..3)
 #pragma unroll
@@ -416,8 +424,8 @@ __global__ void __launch_bounds__(32 * W) bwd_hist_kernel(const __grid_constant_
           // silu'(z) = σ(z) (1 + z (1 - σ(z)))
           zf = mul2(mul2(go, sg), fma2(z2, add2(f2(1.f), mul2(sg, f2(-1.f))), f2(1.f)));
         }
-        hb.table()[(8 * q + j) * kCW + hb.s] = make_float4(dl.x, dx.x, g.x, zf.x);
-        hb.table()[(8 * q + j + 1) * kCW + hb.s] = make_float4(dl.y, dx.y, g.y, zf.y);
+        hb.table()[tbo(8 * q + j) + hb.s] = make_float4(dl.x, dx.x, g.x, zf.x);
+        hb.table()[tbo(8 * q + j + 1) + hb.s] = make_float4(dl.y, dx.y, g.y, zf.y);
         uo[j] = xv.x; uo[j + 1] = xv.y;
         svo[j] = sp.x; svo[j + 1] = sp.y;
         dabs = fmaxf(dabs, fmaxf(fabsf(dl.x), fabsf(dl.y)));
@@ -438,7 +446,7 @@ __global__ void __launch_bounds__(32 * W) bwd_hist_kernel(const __grid_constant_
       float odu[8], odd[8], odz[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const float4 o = hb.outs()[(8 * q + j) * kCW + hb.s];
+        const float4 o = hb.outs()[tbo(8 * q + j) + hb.s];
         odu[j] = o.x; odd[j] = o.y; odz[j] = o.z;
       }
       const long long row = hb.ch * (long long)a.L + t0 + 8 * q;
@@ -467,7 +475,7 @@ __global__ void __launch_bounds__(32 * W) bwd_hist_kernel(const __grid_constant_
       for (int w = 0; w < W; ++w) {
         const float* rw = reinterpret_cast<const float*>(
             reinterpret_cast<const unsigned char*>(redw0) + (size_t)w * G::kWarpBytes +
-            2 * G::kSlotBytes + 2 * kBCS * 4 + kBlk * kCW * 16);
+            2 * G::kSlotBytes + 2 * kBCS * 4 + kTbl * 16);
 #pragma unroll
         for (int i = 0; i < 4; ++i) sum[i] += rw[(4 * tq + i) * 32 + e];
       }
