@@ -278,15 +278,36 @@ struct BwdLayout {
 };
 
 // Time split of the register-history backward: when its CTAs (batch rows x channel groups) fill
-// less than one wave, time is cut into chunks of whole 16-step blocks so that about one wave of
-// CTAs runs (SSM_BWD_SPLIT overrides).  Returns the number of chunks (1: none); *bpc = blocks
-// per chunk.
+// less than one wave, time is cut into chunks of whole 16-step blocks (SSM_BWD_SPLIT
+// overrides).  Returns the number of chunks (1: none); *bpc = blocks per chunk.
+//
+// Measured on B200 (backward of 4 x 5120, 8 x 2048, 2 x 2048, 1 x 2048 and 1 x 256 channels):
+// a grid just over one wave (e.g. 640 CTAs on 444 slots) is the worst case, since its second
+// wave runs nearly a whole chunk for a few CTAs; a grid that fills one wave exactly does well
+// when its chunks stay long (>= 32 blocks); otherwise about four waves of chunks of >= 16 blocks
+// balance the SMs best (4 x 5120 x 2048: 1.52 -> 1.35 ms, 2 x 2048 x 8192: 1.43 -> 1.13 ms),
+// and where chunks of 16 blocks cannot make two waves, one wave.
 int plan_bwd_split(int batch, int dim, int seqlen, int wpb, int ctas_per_sm, int* bpc) {
   const int nblk = (seqlen + ssm::kBlk - 1) / ssm::kBlk;
   const long long ctas = (long long)batch * (((dim + 15) / 16 + wpb - 1) / wpb);
   const long long slots = (long long)sm_count() * ctas_per_sm;
   long long S = env_int("SSM_BWD_SPLIT", 0);
-  if (S <= 0) S = ctas >= slots ? 1 : (slots + ctas - 1) / ctas;
+  if (S <= 0) {
+    if (ctas >= slots) {
+      S = 1;
+    } else {
+      const long long s1 = slots / ctas;  // the most chunks that still fit one wave
+      if (s1 >= 2 && 20 * s1 * ctas >= 19 * slots && nblk >= 32 * s1) {
+        S = s1;
+      } else {
+        const long long by_len = nblk / 16 > 1 ? nblk / 16 : 1;
+        S = (4 * slots + ctas - 1) / ctas;
+        S = S < by_len ? S : by_len;
+        // too short a sequence for several waves: rather one wave than just over one
+        if (S * ctas < 2 * slots) S = s1 < by_len ? s1 : by_len;
+      }
+    }
+  }
   S = S < 1 ? 1 : (S > nblk ? nblk : S);
   *bpc = (int)((nblk + S - 1) / S);
   return (nblk + *bpc - 1) / *bpc;
