@@ -332,6 +332,17 @@ def _ssd(dev, rnd, prm, timeit, g):
         res[f"N{N}"] = {"fwd_ms": ms, "tokens_per_s": b * L / (ms * 1e-3),
                         "hbm_gbs": (4 * b * d * L * 2 + 2 * b * N * L * 2) / (ms * 1e-3) / 1e9,
                         "mma_tflops": flops / (ms * 1e-3) / 1e12}
+    # f32 io with 64 states: the sum of four 16-state f32 forwards over the state slices
+    N = 64
+    uf, df, zf = u.float(), de.float(), z.float()
+    Bf, Cf = rnd((b, N, L)).float(), rnd((b, N, L)).float()
+    of = torch.empty_like(uf)
+    wsf = torch.empty(max(1, ssm._abi.lib().ssm_scan_fwd_ex_workspace_size(b, d, L, N, 1, 0, 1)),
+                      dtype=torch.uint8, device=dev)
+    ms = timeit(lambda: ssm.ssm_scan_fwd_scalar_a(uf, df, A1, Bf, Cf, D=D, z=zf, dt_bias=bias,
+                                                  out=of, workspace=wsf), 5)
+    res["N64_f32_slices"] = {"fwd_ms": ms, "tokens_per_s": b * L / (ms * 1e-3)}
+    del uf, df, zf, Bf, Cf, of, wsf
     # the backward (chunked form: checkpoint pass, reverse walk, dB/dC finish) with 16, 64 and
     # 128 states; compulsory bytes: u, delta, z, dout in, du, ddelta, dz out, B, C in, dB, dC out
     dout = rnd((b, d, L))
