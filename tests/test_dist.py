@@ -242,21 +242,30 @@ def test_allreduce_param_grads_without_group_is_identity():
 
 # ------------------------------------------------------------------ sequence split
 SEQ_SHAPE = dict(batch=2, dim=5, seqlen=53, dstate=4)
+# one decay rate per channel with the larger state of the Mamba-2 setting
+SEQ_SHAPE_SCALAR = dict(batch=1, dim=3, seqlen=41, dstate=32)
 
 
-def _seq_inputs():
+def _seq_inputs(scalar=False):
     from selective_state_space_23_b200.inputs import make_inputs, to_f64, workload
-    w = workload("tiny_f32", **SEQ_SHAPE)
-    return {k: to_f64(v) for k, v in make_inputs(w, seed=8, with_h0=True).items()}
+    w = workload("tiny_f32", **(SEQ_SHAPE_SCALAR if scalar else SEQ_SHAPE))
+    return {k: to_f64(v) for k, v in make_inputs(w, seed=8, with_h0=True, scalar_a=scalar).items()}
+
+
+def _full_a(A, N):
+    """A as [dim][N] for the oracle: a per-channel rate [dim] repeated over the states."""
+    return np.repeat(A[:, None], N, axis=1) if A.ndim == 1 else A
 
 
 def _oracle_ops():
     """Stand-ins for the library's summary, chain and scan calls, built on the fp64 oracle, so
-    that the exchange and composition logic runs on CPU ranks."""
+    that the exchange and composition logic runs on CPU ranks (A [dim][N], or [dim] for one
+    decay rate per channel)."""
     import oracle
 
     def summary(u, delta, A, B, C, dt_bias, softplus):
-        hend = oracle.scan_fwd(u.numpy(), delta.numpy(), A.numpy(), B.numpy(), C.numpy(),
+        Af = _full_a(A.numpy(), B.shape[-2])
+        hend = oracle.scan_fwd(u.numpy(), delta.numpy(), Af, B.numpy(), C.numpy(),
                                dt_bias=dt_bias.numpy(), delta_softplus=softplus, nthreads=1)["hL"]
         v = delta.numpy() + dt_bias.numpy()[None, :, None]
         dsum = (np.logaddexp(0.0, v) if softplus else v).sum(axis=2)
@@ -267,43 +276,48 @@ def _oracle_ops():
         hin = np.empty(hend_all.shape)
         for r in range(hend_all.shape[0]):
             hin[r] = h
-            h = np.exp(A.numpy()[None] * dsum_all[r].numpy()[..., None]) * h + hend_all[r].numpy()
+            Af = _full_a(A.numpy(), hend_all.shape[-1])
+            h = np.exp(Af[None] * dsum_all[r].numpy()[..., None]) * h + hend_all[r].numpy()
         return torch.from_numpy(hin)
 
     def scan(u, delta, A, B, C, D, z, dt_bias, softplus, h0, return_final_state):
-        r = oracle.scan_fwd(u.numpy(), delta.numpy(), A.numpy(), B.numpy(), C.numpy(),
-                            D=D.numpy(), z=z.numpy(), dt_bias=dt_bias.numpy(),
+        r = oracle.scan_fwd(u.numpy(), delta.numpy(), _full_a(A.numpy(), B.shape[-2]), B.numpy(),
+                            C.numpy(), D=D.numpy(), z=z.numpy(), dt_bias=dt_bias.numpy(),
                             delta_softplus=softplus, h0=h0.numpy(), nthreads=1)
         return r["out"], r["hL"]
 
     return {"summary": summary, "chain": chain, "scan": scan}
 
 
-def _seq_worker(rank, world, port, q):
+def _seq_worker(rank, world, port, q, scalar=False):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         from selective_state_space_23_b200.dist import seq_split_scan_fwd
-        x = _seq_inputs()
-        t0, t1 = shard_rows(SEQ_SHAPE["seqlen"], world, rank)   # this rank's time segment
+        x = _seq_inputs(scalar)
+        L = (SEQ_SHAPE_SCALAR if scalar else SEQ_SHAPE)["seqlen"]
+        t0, t1 = shard_rows(L, world, rank)   # this rank's time segment
         seg = lambda k: torch.from_numpy(np.ascontiguousarray(x[k][..., t0:t1]))
         full = lambda k: torch.from_numpy(x[k])
         out, hL = seq_split_scan_fwd(seg("u"), seg("delta"), full("A"), seg("B"), seg("C"),
                                      D=full("D"), z=seg("z"), dt_bias=full("dt_bias"),
-                                     h0=full("h0"), return_final_state=True, ops=_oracle_ops())
+                                     h0=full("h0"), return_final_state=True, scalar_a=scalar,
+                                     ops=_oracle_ops())
         q.put((rank, (t0, t1), out, hL))
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
-def test_sequence_split_over_ranks_matches_full_sequence(world):
+@pytest.mark.parametrize("world,scalar", [(2, False), (3, False), (3, True)])
+def test_sequence_split_over_ranks_matches_full_sequence(world, scalar):
     """Each rank scans its time segment from the state that the all-gathered segment summaries
-    chain to; the concatenated outputs and the last rank's final state are the full sequence's."""
+    chain to; the concatenated outputs and the last rank's final state are the full sequence's
+    (also with one decay rate per channel and 32 states)."""
     port = _free_port()
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    procs = [ctx.Process(target=_seq_worker, args=(r, world, port, q)) for r in range(world)]
+    procs = [ctx.Process(target=_seq_worker, args=(r, world, port, q, scalar))
+             for r in range(world)]
     for p in procs:
         p.start()
     res = [q.get(timeout=120) for _ in range(world)]
@@ -312,10 +326,11 @@ def test_sequence_split_over_ranks_matches_full_sequence(world):
         assert p.exitcode == 0
     res.sort(key=lambda r: r[0])
     import oracle
-    x = _seq_inputs()
+    x = _seq_inputs(scalar)
+    x["A"] = _full_a(x["A"], x["B"].shape[-2])
     full = oracle.scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], D=x["D"], z=x["z"],
                            dt_bias=x["dt_bias"], h0=x["h0"], nthreads=1)
-    assert res[0][1][0] == 0 and res[-1][1][1] == SEQ_SHAPE["seqlen"]
+    assert res[0][1][0] == 0 and res[-1][1][1] == (SEQ_SHAPE_SCALAR if scalar else SEQ_SHAPE)["seqlen"]
     out = np.concatenate([r[2] for r in res], axis=2)
     np.testing.assert_allclose(out, full["out"], rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(res[-1][3], full["hL"], rtol=1e-10, atol=1e-12)
