@@ -382,8 +382,12 @@ __global__ void __launch_bounds__(kStreamThreads) decode_stream_kernel(const __g
     const float v = ld_io<IO>(sg.dt, cl) + bias;
     const float dt = !a.softplus ? v : (kPrecise ? softplus_precise(v) : softplus_fast(v));
     const float dx = dt * xv;
-    const float4 h0 = reinterpret_cast<const float4*>(sg.state + cl * kNS + 8 * q)[0];
-    const float4 h1 = reinterpret_cast<const float4*>(sg.state + cl * kNS + 8 * q)[1];
+    // each thread's 8 states are 32 bytes, so threads 4 apart would read the same banks: those
+    // with bit 2 set read their two halves in the other order
+    const int sw = (tid >> 2) & 1;
+    const float4* hp = reinterpret_cast<const float4*>(sg.state + cl * kNS + 8 * q);
+    const float4 ha = hp[sw], hb = hp[sw ^ 1];
+    const float4 h0 = sw ? hb : ha, h1 = sw ? ha : hb;
     float h[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
     float Bn[8], Cn[8];
     if constexpr (sizeof(IO) == 2) {
